@@ -1,0 +1,483 @@
+#!/usr/bin/env python
+"""ADA paged decode benchmark: KV tokens.heads/s on B200 and the fraction of
+the HBM roofline, next to a dense bf16 paged-decode baseline on the same box.
+
+Default workload: the 128K long-context decode (B=1, T=131072, 32 query /
+8 KV heads, d=128, P=64, budget 40% of the dense fp16 KV bytes, the first 64
+and last 1024 tokens protected, Zipf(1.1) utilities).  One step = one
+skv_decode_attention call (decode kernel + merge kernel) over the whole
+resident store.  Steps run as CUDA-graph replays so that host launch cost
+does not enter the device timeline; two copies of the store alternate so the
+~215 MB read per step never comes from L2 (126 MB).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl skv|reference]
+
+Under torchrun each rank (one GPU) decodes its own copy of the workload
+(independent sequences: weak scaling, no collective on the data path); the
+step time is the max over ranks.  --impl reference times the CPU oracle on a
+bounded sample of the same workload on the host cores (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "ADA decode KV tokens·heads/s at 1 B200; achieved HBM GB/s as % of peak"
+UNIT = "KV tokens·heads/s"
+TIER_BYTES = (512, 196, 180)
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--impl", default="skv", choices=["skv", "reference"])
+    ap.add_argument("--seq-len", type=int, default=131072)
+    ap.add_argument("--num-splits", type=int, default=0)
+    ap.add_argument("--no-dense", action="store_true", help="skip the dense bf16 baseline")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the oracle cpu_baseline leg")
+    ap.add_argument("--graph-steps", type=int, default=100)
+    ap.add_argument("--seed", type=int, default=0)
+    return ap.parse_args()
+
+
+def workload_desc(T):
+    return (f"long_context: B=1, T={T}, 32 query / 8 KV heads (GQA 4), d=128, P=64, "
+            f"budget 40% of dense fp16 KV, protect first 64 + last 1024, Zipf(1.1) utility, "
+            f"bf16 q")
+
+
+# ------------------------------------------------------------------ clocks --
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,utilization.gpu,"
+              "clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int, period_ms: int = 50):
+        self.gpu = gpu_index
+        self.period = period_ms
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.gpu), "-lms", str(self.period)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self._t = threading.Thread(target=self._read, daemon=True)
+            self._t.start()
+        except (FileNotFoundError, OSError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self._t.join(timeout=2)
+        rows = []
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 10:
+                continue
+            try:
+                rows.append(dict(sm=float(f[1]), smax=float(f[2]), util=float(f[4]),
+                                 hw=f[6], hwt=f[7], swt=f[8], swp=f[9]))
+            except ValueError:
+                continue
+        load = [r for r in rows if r["util"] >= 50] or rows
+        if not load:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        reasons = set()
+        for r in load:
+            if r["hw"] == "Active":
+                reasons.add("hw_slowdown")
+            if r["hwt"] == "Active":
+                reasons.add("hw_thermal_slowdown")
+            if r["swt"] == "Active":
+                reasons.add("sw_thermal_slowdown")
+            if r["swp"] == "Active":
+                reasons.add("sw_power_cap")
+        return {"sm_mhz": float(np.median([r["sm"] for r in load])),
+                "sm_max_mhz": max(r["smax"] for r in load), "reasons": sorted(reasons),
+                "samples": len(load)}
+
+
+# ----------------------------------------------------------------- helpers --
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def written_partials(indptr: np.ndarray, S: int) -> int:
+    """(chunk, unit) pairs the decode kernel writes a partial for."""
+    N = int(indptr[-1])
+    n = 0
+    for u in range(len(indptr) - 1):
+        a, b = int(indptr[u]), int(indptr[u + 1])
+        if b <= a:
+            continue
+        c0 = ((a + 1) * S - 1) // N
+        c1 = (b * S - 1) // N
+        n += sum(1 for c in range(c0, c1 + 1) if (c * N) // S != ((c + 1) * N) // S)
+    return n
+
+
+def clone_cache(cache):
+    from long_context_decode_ada_b200 import skv
+    c2 = skv.PagedCache(cache.ctx, cache.B, cache.Hkv, cache.Tmax, cache.pool_slots,
+                        page_cap=cache.page_cap, device=cache.device)
+    for t in range(3):
+        c2.pools[t].copy_(cache.pools[t])
+    c2.page_indptr.copy_(cache.page_indptr)
+    c2.page_ids.copy_(cache.page_ids)
+    c2.tier.copy_(cache.tier)
+    return c2
+
+
+def timed_graph_steps(step_fns, steps, warmup, graph_steps, stream, mid_events=None):
+    """Warm up eagerly, capture `graph_steps` steps per graph, then replay
+    until exactly `steps` steps have run.  Returns (total_ms, per-step event
+    triples of the last replay)."""
+    for i in range(warmup):
+        step_fns[i % len(step_fns)](None)
+    torch.cuda.synchronize()
+    gsteps = max(1, min(graph_steps, steps))
+    ev = [(torch.cuda.Event(enable_timing=True, external=True),
+           torch.cuda.Event(enable_timing=True, external=True),
+           torch.cuda.Event(enable_timing=True, external=True)) for _ in range(gsteps)]
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for i in range(gsteps):
+            ev[i][0].record()
+            step_fns[i % len(step_fns)](ev[i][1])
+            ev[i][2].record()
+    tail = steps % gsteps
+    g_tail = None
+    if tail:
+        g_tail = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_tail):
+            for i in range(tail):
+                step_fns[i % len(step_fns)](None)
+    g.replay()
+    torch.cuda.synchronize()
+    return g, g_tail, ev, steps // gsteps
+
+
+# ------------------------------------------------------------- main (skv) --
+
+def run_skv(args, rank, world, local_rank):
+    from long_context_decode_ada_b200 import skv
+    from long_context_decode_ada_b200 import workloads as wl
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    T = args.seq_len
+    t_gen = time.time()
+    w = wl.long_context(seed=args.seed + 1000 * rank, T=T)
+    t_gen = time.time() - t_gen
+    ctx = skv.Context(w.P)
+    d = skv.workload_to_device(w, dev)
+
+    # ---- ingest: allocate + encode (off the decode path; timed for context)
+    e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+    cache = skv.PagedCache(ctx, w.B, w.Hkv, w.Tmax, w.pool_slots, device=dev)
+    e0.record()
+    cache.allocate(d["K"], d["seq_lens"], d["utility"], d["protect"], w.mode, d["budget"],
+                   d["quota"], d["free_lists"])
+    e1.record()
+    cache.encode(d["K"], d["V"], d["seq_lens"])
+    e2.record()
+    cache.check()
+    alloc_ms, enc_ms = e0.elapsed_time(e1), e1.elapsed_time(e2)
+    caches = [cache, clone_cache(cache)]
+
+    tier_counts = torch.bincount(cache.tier.flatten().to(torch.int64), minlength=4).cpu().numpy()
+    indptr = cache.page_indptr.cpu().numpy()
+    n_pages = int(indptr[-1])
+    ids = cache.page_ids[:n_pages].cpu().numpy().view(np.uint32)
+    pages_per_tier = np.bincount(ids >> 30, minlength=3)
+    resident = int(tier_counts[:3].sum())            # kept (seq, kv head, token) triples
+    sm_count, default_splits = ctx.device_info()
+    S = args.num_splits or default_splits
+    G = w.Hq // w.Hkv
+    nparts = written_partials(indptr, S)
+    q_bytes = w.B * w.Hq * 128 * 2
+    algo_bytes = (int(sum(int(tier_counts[t]) * TIER_BYTES[t] for t in range(3)))
+                  + 16 * n_pages + 4 * n_pages + 4 * len(indptr) + q_bytes
+                  + nparts * G * 132 * 4)
+    payload_bytes = int(sum(int(pages_per_tier[t]) * caches[0].payload[t] for t in range(3)))
+
+    stream = torch.cuda.current_stream()
+    ws = [c.workspace(w.Hq, S) for c in caches]
+    out = torch.empty((w.B, w.Hq, 128), dtype=torch.float32, device=dev)
+    lse = torch.empty((w.B, w.Hq), dtype=torch.float32, device=dev)
+
+    def make_step(c, wsp):
+        def step(mid_event):
+            ctx.set_profile_event(mid_event)
+            c.decode(d["q"], d["q_dtype"], w.Hq, out=out, lse=lse, workspace=wsp, num_splits=S)
+        return step
+
+    step_fns = [make_step(caches[0], ws[0]), make_step(caches[1], ws[1])]
+    g, g_tail, ev, reps = timed_graph_steps(step_fns, args.steps, args.warmup, args.graph_steps,
+                                            stream)
+    ctx.set_profile_event(None)
+    caches[0].check()
+
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    time.sleep(0.3)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(reps):
+        g.replay()
+    if g_tail is not None:
+        g_tail.replay()
+    t1.record()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = sampler.stop()
+    elapsed_ms = t0.elapsed_time(t1)
+    caches[0].check()
+    if world > 1:
+        tt = torch.tensor([elapsed_ms], device=dev)
+        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+        elapsed_ms = float(tt.item())
+    ms_per_step = elapsed_ms / args.steps
+    value = world * resident / (ms_per_step * 1e-3)
+    step_ms = [a.elapsed_time(c) for a, b, c in ev]
+    kern_ms = [a.elapsed_time(b) for a, b, c in ev]
+    kern_ms_avg = float(np.mean(kern_ms))
+    peak, peak_kind = measured_peaks()
+    achieved = algo_bytes / (kern_ms_avg * 1e-3) / 1e9
+
+    # ---- end to end: host q -> device, decode, out/lse -> host, every step
+    e2e = None
+    if rank == 0 or world > 1:
+        q_host = d["q"].cpu().pin_memory()
+        out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        lse_host = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+        q_dev = torch.empty_like(d["q"])
+        e2e_steps = max(10, min(args.steps, 2000))
+        for i in range(5):
+            q_dev.copy_(q_host, non_blocking=True)
+            caches[i % 2].decode(q_dev, d["q_dtype"], w.Hq, out=out, lse=lse, workspace=ws[i % 2],
+                                 num_splits=S)
+            out_host.copy_(out, non_blocking=True)
+            lse_host.copy_(lse, non_blocking=True)
+            stream.synchronize()
+        ta = time.perf_counter()
+        for i in range(e2e_steps):
+            q_dev.copy_(q_host, non_blocking=True)
+            caches[i % 2].decode(q_dev, d["q_dtype"], w.Hq, out=out, lse=lse, workspace=ws[i % 2],
+                                 num_splits=S)
+            out_host.copy_(out, non_blocking=True)
+            lse_host.copy_(lse, non_blocking=True)
+            stream.synchronize()
+        e2e_ms = (time.perf_counter() - ta) * 1e3 / e2e_steps
+        caches[0].check()
+        e2e = {"value": world * resident / (e2e_ms * 1e-3), "unit": UNIT,
+               "h2d_bytes_per_step": int(q_host.numel() * q_host.element_size()),
+               "d2h_bytes_per_step": int(out_host.numel() * 4 + lse_host.numel() * 4),
+               "ms_per_step": e2e_ms, "steps": e2e_steps,
+               "how": "pinned host q -> device, skv_decode_attention, out+lse -> pinned host, "
+                      "stream sync every step; host wall clock"}
+
+    # ---- dense bf16 paged-decode baseline on the same K/V
+    dense = None
+    if not args.no_dense:
+        n_dense = w.B * w.Hkv * (-(-T // w.P))
+        dcs = []
+        for k in range(2):
+            dc = skv.DenseCache(ctx, w.B, w.Hkv, w.Tmax, n_dense, device=dev)
+            dc.pack(d["K"], d["V"], d["seq_lens"], torch.arange(n_dense, dtype=torch.int32))
+            dc.check()
+            dcs.append(dc)
+        dws = [dc.workspace(w.Hq, S) for dc in dcs]
+
+        def dstep(i):
+            def f(mid):
+                ctx.set_profile_event(mid)
+                dcs[i].decode(d["q"], d["q_dtype"], w.Hq, out=out, lse=lse, workspace=dws[i],
+                              num_splits=S)
+            return f
+        dsteps = max(10, min(args.steps, 2000))
+        gd, gd_tail, evd, repd = timed_graph_steps([dstep(0), dstep(1)], dsteps,
+                                                   min(args.warmup, 20), args.graph_steps, stream)
+        ctx.set_profile_event(None)
+        torch.cuda.synchronize()
+        ta, tb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ta.record()
+        for _ in range(repd):
+            gd.replay()
+        if gd_tail is not None:
+            gd_tail.replay()
+        tb.record()
+        torch.cuda.synchronize()
+        dcs[0].check()
+        dms = ta.elapsed_time(tb) / dsteps
+        dk = float(np.mean([a.elapsed_time(b) for a, b, c in evd]))
+        dbytes = w.B * w.Hkv * T * 512 + 16 * n_dense + 4 * n_dense
+        dense = {"value": world * w.B * w.Hkv * T / (dms * 1e-3), "unit": UNIT + " (all tokens)",
+                 "ms_per_step": dms, "kernel_ms": dk,
+                 "achieved_gbs": dbytes / (dk * 1e-3) / 1e9,
+                 "frac": dbytes / (dk * 1e-3) / 1e9 / peak,
+                 "ada_speedup_step": dms / ms_per_step}
+        del dcs, dws
+
+    cpu = None
+    if rank == 0 and not args.no_cpu:
+        cpu = cpu_baseline(T_sample=65536)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
+            "data": "synthetic",
+            "config": {"workload": workload_desc(T),
+                       "l2": "inputs larger than L2: two rotating copies of the ~215 MB store",
+                       "num_splits": S, "graph_steps": args.graph_steps,
+                       "resident_tokens_heads": resident,
+                       "tier_tokens": {"T0": int(tier_counts[0]), "T1": int(tier_counts[1]),
+                                       "T2": int(tier_counts[2]), "dropped": int(tier_counts[3])},
+                       "pages": {"T0": int(pages_per_tier[0]), "T1": int(pages_per_tier[1]),
+                                 "T2": int(pages_per_tier[2])},
+                       "parallelism": f"{world} independent replicas (one per GPU)"},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": None,
+                         "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)",
+                         "kernel": "decode_kernel<4,false>", "kernel_ms": kern_ms_avg,
+                         "algorithmic_bytes": algo_bytes, "payload_bytes_streamed": payload_bytes},
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": 2 * args.steps,
+            "clocks": clocks,
+            "dense_bf16_baseline": dense,
+            "ingest": {"allocate_ms": alloc_ms, "encode_ms": enc_ms, "gen_s": t_gen},
+            "step_ms_graph_events": float(np.mean(step_ms)),
+        }
+        print(json.dumps(line), flush=True)
+
+
+# -------------------------------------------------------- oracle (CPU) ----
+
+def cpu_baseline(T_sample: int, repeats: int = 1):
+    """Time the oracle's decode (as it stands) on the host cores on a bounded
+    sample of the same workload: the long-context recipe at T_sample tokens.
+    The sample's tiers come from the oracle's own allocation."""
+    import oracle
+    from long_context_decode_ada_b200 import workloads as wl
+    w = wl.long_context(seed=1, T=T_sample)
+    tier = oracle.allocate(w.B, w.Hkv, w.Tmax, w.d, w.P, w.seq_lens, w.K, w.utility, w.protect,
+                           w.mode, w.budget, w.quota)
+    resident = int((tier != 3).sum())
+    t = time.perf_counter()
+    for _ in range(repeats):
+        oracle.decode(w.B, w.Hq, w.Hkv, w.Tmax, w.d, w.seq_lens, w.K, w.V, tier, w.q, w.q_dtype)
+    dt = (time.perf_counter() - t) / repeats
+    return {"value": resident / dt, "unit": UNIT, "cores": oracle.threads(), "kind": "oracle",
+            "sample": f"long_context recipe at T={T_sample} (B=1, 8 KV / 32 query heads, "
+                      f"{resident} resident token-heads), oracle decode only, {dt:.2f} s",
+            "seconds": dt}
+
+
+def run_reference(args, rank, world):
+    """The reference arm: the CPU oracle, timed per step on a bounded sample."""
+    if rank != 0:
+        return
+    import oracle
+    from long_context_decode_ada_b200 import workloads as wl
+    T_sample = 4096
+    w = wl.long_context(seed=1, T=T_sample)
+    tier = oracle.allocate(w.B, w.Hkv, w.Tmax, w.d, w.P, w.seq_lens, w.K, w.utility, w.protect,
+                           w.mode, w.budget, w.quota)
+    resident = int((tier != 3).sum())
+
+    def step():
+        oracle.decode(w.B, w.Hq, w.Hkv, w.Tmax, w.d, w.seq_lens, w.K, w.V, tier, w.q, w.q_dtype)
+
+    for _ in range(max(0, min(args.warmup, 3))):
+        step()
+    steps = args.steps
+    t = time.perf_counter()
+    budget_s = 120.0
+    done = 0
+    for i in range(steps):
+        step()
+        done += 1
+        if time.perf_counter() - t > budget_s:
+            break
+    dt = (time.perf_counter() - t) / done
+    value = resident / dt
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": done, "warmup": args.warmup, "ms_per_step": dt * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": workload_desc(args.seq_len),
+                       "sample": f"each step decodes the long_context recipe at T={T_sample}"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.threads(),
+                             "kind": "oracle",
+                             "sample": f"long_context recipe at T={T_sample}, {resident} "
+                                       f"resident token-heads per step"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0},
+            "gpu_launches": 0}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        run_skv(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,238 @@
+/*
+ * skv.h -- C-ABI of libskv: Spherical KV (Angle-Domain Attention + Rate-
+ * Distortion Retention) paged decode on NVIDIA B200 (sm_100a).
+ *
+ * Sources: the pages about arXiv 2605.18856 "SPHERICAL KV: Angle-Domain
+ * Attention and Rate-Distortion Retention for Efficient Long-Context
+ * Inference": the gist.science technical summary, sections 1 (problem
+ * statement), 2.1 (Angle-Domain Attention), 2.2 (Rate-Distortion Retention)
+ * and 2.3 (system integration), and the arXiv abstract.
+ *
+ * Conventions (every entry point):
+ *  - Returns an int status: SKV_OK or one of the SKV_ERR_* codes below.  On
+ *    error, skv_last_error() gives a message (thread-local).  No C++
+ *    exception crosses this boundary.
+ *  - Device pointers are caller-owned device memory (the library never
+ *    frees them).  Host pointers (config structs, pool descriptors) are read
+ *    during the call only.
+ *  - Every call that launches work takes a cudaStream_t (passed as void*,
+ *    NULL = legacy default stream) and is asynchronous: it returns once the
+ *    kernels are queued.  Errors found on the device are recorded in a
+ *    caller-provided int32 device word (first error wins); skv_check()
+ *    synchronises the stream, reads and clears it.
+ *  - A context is bound to the CUDA device that was current at skv_create.
+ *  - head_dim is 128 and the page size P is 16, 32 or 64 for the CUDA
+ *    kernels.
+ */
+#ifndef SKV_H_
+#define SKV_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* status codes */
+#define SKV_OK 0
+#define SKV_ERR_ARG 1      /* invalid argument (host check or device check of an input)  */
+#define SKV_ERR_BUDGET 2   /* protected tokens + page reserve exceed a sequence's budget  */
+#define SKV_ERR_POOL 3     /* a free list or the page-id capacity is too short            */
+#define SKV_ERR_CORRUPT 4  /* a page table entry or page header is out of range           */
+#define SKV_ERR_CUDA 5     /* a CUDA runtime call failed                                   */
+#define SKV_ERR_TIMEOUT 6  /* a bounded device-side wait ran out (kernel returned early)   */
+
+/* tiers: T0 dense fp16 K/V, T1 6-bit angles, T2 4-bit angles, dropped */
+#define SKV_TIER_T0 0
+#define SKV_TIER_T1 1
+#define SKV_TIER_T2 2
+#define SKV_TIER_DROP 3
+
+/* allocation modes */
+#define SKV_MODE_QUOTA 0   /* fixed per-tier counts per (seq, head), ranked by utility */
+#define SKV_MODE_BUDGET 1  /* rate-distortion greedy under a byte budget per sequence  */
+
+/* query element types */
+#define SKV_Q_FP16 0
+#define SKV_Q_BF16 1
+
+/* workspace kinds for skv_workspace_size */
+#define SKV_WS_ALLOCATE 0
+#define SKV_WS_DECODE 1
+#define SKV_WS_DENSE_DECODE 2
+
+/* host tables exported for tests (skv_tables) */
+#define SKV_TABLE_BOUNDARY6_X 0  /* 64 fp32: cos((j+1/2) 2pi/64)                */
+#define SKV_TABLE_BOUNDARY6_Y 1  /* 64 fp32: sin((j+1/2) 2pi/64)                */
+#define SKV_TABLE_BOUNDARY4_X 2  /* 16 fp32                                      */
+#define SKV_TABLE_BOUNDARY4_Y 3  /* 16 fp32                                      */
+#define SKV_TABLE_KAPPA 4        /* 3 fp32: RDR slope per byte of each step      */
+#define SKV_TABLE_RHO_LEVELS 5   /* 4 fp32: decoded share of each 2-bit code     */
+
+typedef struct skv_config {
+  int32_t head_dim;    /* d: 128 */
+  int32_t page_size;   /* P: 16, 32 or 64 */
+  int32_t reserved[6]; /* zero */
+} skv_config;
+
+/* Device pools of page slots, one per tier.  Slot s of tier t starts at
+   base[t] + s * stride(t) (skv_page_bytes); slots[t] is the slot count, used
+   to bounds-check page ids on the device.  base[t] must be 128-byte aligned. */
+typedef struct skv_pools {
+  void* base[3];
+  int64_t slots[3];
+} skv_pools;
+
+/* Device free lists: ids[t] holds len[t] slot numbers of tier t's pool, in
+   the order in which they are handed out. */
+typedef struct skv_free_lists {
+  const uint32_t* ids[3];
+  int64_t len[3];
+} skv_free_lists;
+
+typedef struct skv_ctx skv_ctx;
+
+/* Create a context on the current CUDA device.  Computes the host tables
+   (angle-sector boundaries, LUT cosines, share levels, RDR slopes) once.
+   Errors: SKV_ERR_ARG for an unsupported head_dim / page_size. */
+int skv_create(const skv_config* cfg, skv_ctx** out);
+
+/* Destroy a context (NULL is accepted). */
+int skv_destroy(skv_ctx* ctx);
+
+/* Message of the last error on this thread ("" when none).  The pointer is
+   valid until the next libskv call on this thread. */
+const char* skv_last_error(void);
+
+/* Page geometry of a tier (SPHERICAL KV technical summary 2.2: tier-
+   homogeneous pages).  payload = 16 + P * bytes_per_token(tier); stride =
+   payload rounded up to 128.  Bytes per (token, kv head): T0 512, T1 196,
+   T2 180.  tier SKV_TIER_DROP + 1 (= 4) asks for the dense-bf16 baseline
+   page (same as T0). */
+int skv_page_bytes(const skv_ctx* ctx, int tier, int64_t* payload, int64_t* stride);
+
+/* Copy host table `which` (SKV_TABLE_*) into out[0..n).  Host memory. */
+int skv_tables(const skv_ctx* ctx, int which, float* out, int64_t n);
+
+/* Number of SMs of the context's device and the default split count that
+   skv_decode_attention uses when num_splits == 0. */
+int skv_device_info(const skv_ctx* ctx, int* sm_count, int* default_splits);
+
+/* Bytes of device workspace that a call needs.
+   SKV_WS_ALLOCATE: skv_allocate on B sequences x Hkv heads x Tmax tokens.
+   SKV_WS_DECODE / SKV_WS_DENSE_DECODE: the decode with num_splits chunks
+   (0 = default) over B x Hkv units with Hq query heads.  The workspace is
+   scratch that the call may overwrite; it must stay allocated until the
+   stream has run the call. */
+int skv_workspace_size(const skv_ctx* ctx, int which, int B, int Hkv, int Hq, int64_t Tmax,
+                       int num_splits, size_t* bytes);
+
+/* skv_allocate -- Rate-Distortion Retention (technical summary 2.2; abstract:
+   "keep/drop decisions and precision tiers per token and head under a fixed
+   budget, producing tier-homogeneous pages with lightweight metadata").
+   Chooses a tier for every (seq b, kv head h, position t < seq_lens[b]),
+   packs the kept tokens into tier-homogeneous pages and writes the page
+   table and page headers.
+     K          fp16 [B][Hkv][Tmax][128] device: keys (radius from exact norm)
+     seq_lens   int32 [B] device, 0 <= seq_lens[b] <= Tmax
+     utility    fp32 [B][Hkv][Tmax] device, finite and >= 0 (budget mode
+                required; quota mode: NULL ranks by position)
+     protect    uint8 [B][Hkv][Tmax] device or NULL: nonzero = always T0
+     mode       SKV_MODE_BUDGET: the greedy rate-distortion walk under
+                budget[b] bytes per sequence (shared by its Hkv heads).
+                SKV_MODE_QUOTA: per (b, h) the quota[b][0..2] highest-utility
+                unprotected tokens go to T0, T1, T2 in that order.
+     budget     int64 [B] device (budget mode) or NULL
+     quota      int32 [B][3] device (quota mode) or NULL
+     free       per-tier free lists (device ids, host descriptor)
+     pools      per-tier pools; headers are written into each used slot and
+                every row of a partial page is zeroed
+     tier_out   uint8 [B][Hkv][Tmax] device: 0 T0, 1 T1, 2 T2, 3 dropped
+                (positions >= seq_lens[b] are 3)
+     row_of     int32 [B][Hkv][Tmax] device: page index within the unit's
+                list * P + row, or -1 when not resident
+     page_indptr int32 [B*Hkv + 1] device: CSR offsets per unit b*Hkv + h
+     page_ids   uint32 [page_cap] device: tier << 30 | slot; per unit the T0
+                pages, then T1, then T2
+     err_word   int32 device: SKV_ERR_BUDGET, SKV_ERR_POOL or SKV_ERR_ARG
+                found on the device (outputs are then unspecified)
+     workspace  device scratch of skv_workspace_size(SKV_WS_ALLOCATE) bytes */
+int skv_allocate(skv_ctx* ctx, const uint16_t* K, int B, int Hkv, int64_t Tmax,
+                 const int32_t* seq_lens, const float* utility, const uint8_t* protect,
+                 int mode, const int64_t* budget, const int32_t* quota,
+                 const skv_free_lists* free, const skv_pools* pools, uint8_t* tier_out,
+                 int32_t* row_of, int32_t* page_indptr, uint32_t* page_ids, int64_t page_cap,
+                 int32_t* err_word, void* workspace, size_t ws_bytes, void* stream);
+
+/* skv_encode -- maps dense keys to spherical codes (technical summary 2.1,
+   2.3): for every resident (b, h, t) writes its row of the page that
+   row_of / page_indptr / page_ids assign:
+     T0: fp16 K and V unchanged (in the documented within-page order)
+     T1/T2: r~ = fp16 |k|, per pair a 6-bit (T1) or 4-bit (T2) angle code and
+            a 2-bit share code, int8 V with a per-token fp16 absmax scale.
+   Arguments as for skv_allocate (tier/row_of/page table are its outputs).
+   Page ids are bounds-checked (SKV_ERR_CORRUPT). */
+int skv_encode(skv_ctx* ctx, const uint16_t* K, const uint16_t* V, int B, int Hkv, int64_t Tmax,
+               const int32_t* seq_lens, const uint8_t* tier, const int32_t* row_of,
+               const int32_t* page_indptr, const uint32_t* page_ids, const skv_pools* pools,
+               int32_t* err_word, void* stream);
+
+/* skv_decode_attention -- the ADA decode step (technical summary 2.1: logits
+   computed directly from the radius and angle codes, no dense key
+   materialised; abstract: "paged, block-local, fusion-friendly decode path").
+   For every sequence b and query head hq (kv head h = hq / (Hq/Hkv)):
+     out[b][hq] = sum_t softmax_t(l_t) v^_t,  lse[b][hq] = log sum_t exp(l_t)
+   over the resident tokens of (b, h): l_t = (r~_t/sqrt d) sum_i rho^_i
+   LUT_i[c_i] for T1/T2 (LUT_i[c] = q_{2i} cos(2 pi c/2^b) + q_{2i+1}
+   sin(2 pi c/2^b)), q . k_t / sqrt d for T0; v^ = scale * int8 or fp16 V.
+     q        [B][Hq][128] device, q_dtype SKV_Q_BF16 or SKV_Q_FP16
+     Hq       a multiple of Hkv with Hq/Hkv in {1, 2, 4}
+     page_indptr / page_ids / pools: the paged store (any slots, any order of
+              pages within a unit; pages are streamed whole)
+     out      fp32 [B][Hq][128] device; lse fp32 [B][Hq] device or NULL
+              (a unit without resident tokens gives out 0, lse -inf)
+     num_splits  number of page chunks = CTAs (0 = default: 2 x SM count);
+              the pages of all units are cut into num_splits equal runs
+     workspace   skv_workspace_size(SKV_WS_DECODE, ..., num_splits) bytes
+   Device errors: SKV_ERR_CORRUPT (bad page id / header: the page is
+   skipped), SKV_ERR_TIMEOUT (a bounded wait ran out). */
+int skv_decode_attention(skv_ctx* ctx, const void* q, int q_dtype, int B, int Hq, int Hkv,
+                         const int32_t* page_indptr, const uint32_t* page_ids,
+                         const skv_pools* pools, float* out, float* lse, int32_t* err_word,
+                         void* workspace, size_t ws_bytes, int num_splits, void* stream);
+
+/* skv_dense_pack_bf16 -- the dense baseline's store: every token of every
+   (b, h) kept as bf16 K/V (fp16 inputs rounded to nearest even) in pages of
+   P rows with the T0 page layout.  Slots come from free_ids in (b, h, page)
+   order.  Writes page_indptr [B*Hkv+1] and page_ids (tier bits 0). */
+int skv_dense_pack_bf16(skv_ctx* ctx, const uint16_t* K, const uint16_t* V, int B, int Hkv,
+                        int64_t Tmax, const int32_t* seq_lens, const uint32_t* free_ids,
+                        int64_t free_len, void* pool, int64_t pool_slots, int32_t* page_indptr,
+                        uint32_t* page_ids, int64_t page_cap, int32_t* err_word,
+                        void* workspace, size_t ws_bytes, void* stream);
+
+/* skv_dense_decode_bf16 -- dense bf16 paged-decode baseline: textbook
+   attention over every token of the bf16 pages, the same kernel skeleton as
+   skv_decode_attention (split-K, GQA, online softmax, P.V on tensor cores). */
+int skv_dense_decode_bf16(skv_ctx* ctx, const void* q, int q_dtype, int B, int Hq, int Hkv,
+                          const int32_t* page_indptr, const uint32_t* page_ids,
+                          const void* pool, int64_t pool_slots, float* out, float* lse,
+                          int32_t* err_word, void* workspace, size_t ws_bytes, int num_splits,
+                          void* stream);
+
+/* Profiling aid: when `event` (a cudaEvent_t, or NULL to clear) is set, every
+   later skv_decode_attention / skv_dense_decode_bf16 call on this context
+   records it on its stream between the decode kernel and the merge kernel,
+   so that a caller can time the decode kernel alone with CUDA events. */
+int skv_set_profile_event(skv_ctx* ctx, void* event);
+
+/* Synchronise `stream`, read the device error word, reset it to 0 and return
+   SKV_OK or the recorded SKV_ERR_* code. */
+int skv_check(skv_ctx* ctx, int32_t* err_word, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SKV_H_ */

@@ -1,0 +1,499 @@
+// allocate.cu -- Rate-Distortion Retention (SPHERICAL KV technical summary
+// 2.2; arXiv abstract: keep/drop and precision tiers per token and head
+// under a fixed budget, tier-homogeneous pages with lightweight metadata).
+//
+// Budget mode: every unprotected token offers three upgrade steps
+// (drop->T2 180 B, T2->T1 16 B, T1->T0 316 B) with priority
+// fp32((u * fp32(r^2)) * kappa_step).  All steps of a sequence are ordered by
+// (priority desc, step asc, head asc, position asc) through a 64-bit
+// composite key, and the longest prefix that fits the budget left after the
+// protected tokens and a partial-page reserve is taken.  The cut is found by
+// an exact weighted radix select (8 passes of 8 bits, byte-weighted
+// histograms), so the result is the same as a full sort.
+// Quota mode: per (seq, head), the same radix select finds the ranks q0,
+// q0+q1, q0+q1+q2 of the (utility desc, position asc) order.
+// Then: tiers, per-(unit, tier) counts, page plan (CSR offsets and per-tier
+// free-list bases), row_of by a block scan, page ids and headers.
+#include "common.cuh"
+#include "kernels.h"
+
+#include <algorithm>
+
+namespace skv {
+
+typedef unsigned __int128 u128;
+
+static inline size_t al256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+size_t alloc_workspace_bytes(int B, int Hkv, long long Tmax) {
+  const size_t U = (size_t)B * Hkv;
+  const size_t nseg = U;
+  size_t n = 0;
+  n += al256(4 * U * (size_t)Tmax);
+  n += al256(8 * nseg * 3 * 3);
+  n += al256(8 * nseg * 3 * 256);
+  n += al256(4 * U * 3);
+  n += al256(4 * U * 3);
+  n += al256(8 * (size_t)B);
+  return n;
+}
+
+void alloc_carve(AllocParams& p, void* ws) {
+  const size_t U = (size_t)p.B * p.Hkv;
+  const size_t nseg = U;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  p.keyw = reinterpret_cast<float*>(w);
+  w += al256(4 * U * (size_t)p.Tmax);
+  p.sel = reinterpret_cast<unsigned long long*>(w);
+  w += al256(8 * nseg * 3 * 3);
+  p.hist = reinterpret_cast<unsigned long long*>(w);
+  w += al256(8 * nseg * 3 * 256);
+  p.counts = reinterpret_cast<int32_t*>(w);
+  w += al256(4 * U * 3);
+  p.tbase = reinterpret_cast<int32_t*>(w);
+  w += al256(4 * U * 3);
+  p.nprot = reinterpret_cast<long long*>(w);
+}
+
+// ---------------------------------------------------------------- keys --
+
+__device__ __forceinline__ float valid_utility(const AllocParams& p, long long i) {
+  if (!p.utility) return 0.0f;
+  float u = p.utility[i];
+  if (!(u >= 0.0f) || isinf(u)) {
+    report(p.err, SKV_ERR_ARG);
+    return 0.0f;
+  }
+  return u;
+}
+
+// budget mode: one warp per token; keyw = u * fp32(r^2), -1 when protected
+__global__ void __launch_bounds__(256) keys_budget_kernel(const __grid_constant__ AllocParams p) {
+  const long long w = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (w >= (long long)p.B * p.Hkv * p.Tmax) return;
+  const long long t = w % p.Tmax;
+  const int b = (int)(w / p.Tmax / p.Hkv);
+  if (t >= p.seq_lens[b]) return;
+  if (p.protect && p.protect[w]) {
+    if (lane == 0) {
+      p.keyw[w] = -1.0f;
+      atomicAdd(reinterpret_cast<unsigned long long*>(&p.nprot[b]), 1ull);
+    }
+    return;
+  }
+  const uint2 kv = *reinterpret_cast<const uint2*>(p.K + w * kHeadDim + 4 * lane);
+  const uint16_t k4[4] = {(uint16_t)(kv.x & 0xFFFF), (uint16_t)(kv.x >> 16),
+                          (uint16_t)(kv.y & 0xFFFF), (uint16_t)(kv.y >> 16)};
+  u128 sq = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const long long m = half_bits_to_m(k4[i]);
+    const u128 a = (u128)(m < 0 ? -m : m);
+    sq += a * a;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    unsigned long long lo = (unsigned long long)sq, hi = (unsigned long long)(sq >> 64);
+    unsigned long long olo = __shfl_xor_sync(0xFFFFFFFFu, lo, o);
+    unsigned long long ohi = __shfl_xor_sync(0xFFFFFFFFu, hi, o);
+    sq += ((u128)ohi << 64) | olo;
+  }
+  if (lane == 0) {
+    const double r2 = u128_to_double_rn((unsigned long long)(sq >> 64), (unsigned long long)sq);
+    const float r2f = __double2float_rn(__dmul_rn(r2, 3.552713678800501e-15));  // 2^-48
+    p.keyw[w] = __fmul_rn(valid_utility(p, w), r2f);
+  }
+}
+
+// quota mode: keyw = u (0 without utilities), -1 when protected
+__global__ void keys_quota_kernel(const __grid_constant__ AllocParams p) {
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= (long long)p.B * p.Hkv * p.Tmax) return;
+  const long long t = i % p.Tmax;
+  const int b = (int)(i / p.Tmax / p.Hkv);
+  if (t >= p.seq_lens[b]) return;
+  p.keyw[i] = (p.protect && p.protect[i]) ? -1.0f : valid_utility(p, i);
+}
+
+// ---------------------------------------------------------- radix select --
+
+// state per (segment, target): [0] prefix, [1] remaining (int64 bits), [2] done
+__global__ void sel_init_kernel(const __grid_constant__ AllocParams p) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= p.nseg * 3) return;
+  const int seg = i / 3, j = i % 3;
+  unsigned long long* st = p.sel + (size_t)i * 3;
+  st[0] = 0;
+  st[1] = 0;
+  st[2] = 0;
+  if (p.mode == SKV_MODE_BUDGET) {
+    if (j != 0) {
+      st[2] = 1;
+      return;
+    }
+    const long long reserve = (long long)p.Hkv * (p.P - 1) * (512 + 196 + 180);
+    const long long left = p.budget[seg] - 512LL * p.nprot[seg] - reserve;
+    if (left < 0) {
+      report(p.err, SKV_ERR_BUDGET);
+      st[2] = 1;  // prefix 0: nothing is selected
+      return;
+    }
+    st[1] = (unsigned long long)left;
+  } else {
+    const int b = seg / p.Hkv;
+    const long long q0 = p.quota[3 * b], q1 = p.quota[3 * b + 1], q2 = p.quota[3 * b + 2];
+    if (q0 < 0 || q1 < 0 || q2 < 0) {
+      report(p.err, SKV_ERR_ARG);
+      st[2] = 1;
+      return;
+    }
+    st[1] = (unsigned long long)(j == 0 ? q0 : (j == 1 ? q0 + q1 : q0 + q1 + q2));
+  }
+}
+
+__device__ __forceinline__ bool item_composite(const AllocParams& p, int seg, long long i,
+                                               unsigned long long& comp, uint32_t& weight) {
+  if (p.mode == SKV_MODE_BUDGET) {
+    const int k = (int)(i % 3);
+    const long long ht = i / 3;
+    const int h = (int)(ht / p.Tmax);
+    const long long t = ht % p.Tmax;
+    if (t >= p.seq_lens[seg]) return false;
+    const float w = p.keyw[((long long)seg * p.Hkv + h) * p.Tmax + t];
+    if (w < 0.0f) return false;
+    const float key = __fmul_rn(w, p.kappa[k]);
+    comp = ((unsigned long long)(0xFFFFFFFFu - __float_as_uint(key)) << 32) |
+           ((unsigned long long)k << 30) | ((unsigned long long)h << 23) | (unsigned long long)t;
+    weight = (k == 0) ? 180u : (k == 1 ? 16u : 316u);
+    return true;
+  }
+  const int b = seg / p.Hkv;
+  if (i >= p.seq_lens[b]) return false;
+  const float w = p.keyw[(long long)seg * p.Tmax + i];
+  if (w < 0.0f) return false;
+  comp = ((unsigned long long)(0xFFFFFFFFu - __float_as_uint(w)) << 32) | (unsigned long long)i;
+  weight = 1;
+  return true;
+}
+
+constexpr int kHistItemsPerBlock = 4096;
+
+__global__ void __launch_bounds__(256) hist_kernel(const __grid_constant__ AllocParams p,
+                                                   int shift) {
+  __shared__ unsigned long long sh[3][256];
+  __shared__ unsigned long long pre[3];
+  __shared__ int dn[3];
+  const int seg = blockIdx.y;
+  const int ntgt = p.mode == SKV_MODE_BUDGET ? 1 : 3;
+  if (threadIdx.x < 3) {
+    const unsigned long long* st = p.sel + ((size_t)seg * 3 + threadIdx.x) * 3;
+    pre[threadIdx.x] = st[0];
+    dn[threadIdx.x] = (threadIdx.x < ntgt) ? (int)st[2] : 1;
+  }
+  for (int i = threadIdx.x; i < 3 * 256; i += blockDim.x) (&sh[0][0])[i] = 0;
+  __syncthreads();
+  if (dn[0] && dn[1] && dn[2]) return;
+  const long long n_items =
+      p.mode == SKV_MODE_BUDGET ? (long long)p.Hkv * p.Tmax * 3 : (long long)p.Tmax;
+  const long long i0 = (long long)blockIdx.x * kHistItemsPerBlock;
+  const long long i1 = min(n_items, i0 + kHistItemsPerBlock);
+  for (long long i = i0 + threadIdx.x; i < i1; i += blockDim.x) {
+    unsigned long long comp;
+    uint32_t wgt;
+    if (!item_composite(p, seg, i, comp, wgt)) continue;
+    const int dig = (int)((comp >> shift) & 255u);
+    for (int j = 0; j < ntgt; ++j) {
+      if (dn[j]) continue;
+      if (shift < 56 && (comp >> (shift + 8)) != (pre[j] >> (shift + 8))) continue;
+      atomicAdd(&sh[j][dig], (unsigned long long)wgt);
+    }
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < ntgt * 256; i += blockDim.x) {
+    const unsigned long long v = (&sh[0][0])[i];
+    if (v) atomicAdd(&p.hist[(size_t)seg * 3 * 256 + i], v);
+  }
+}
+
+__global__ void sel_step_kernel(const __grid_constant__ AllocParams p, int shift) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= p.nseg * 3) return;
+  unsigned long long* st = p.sel + (size_t)i * 3;
+  unsigned long long* h = p.hist + (size_t)i * 256;
+  if (st[2]) {
+    for (int d = 0; d < 256; ++d) h[d] = 0;
+    return;
+  }
+  const unsigned long long rem = st[1];
+  unsigned long long cum = 0;
+  bool found = false;
+  for (int d = 0; d < 256; ++d) {
+    const unsigned long long v = h[d];
+    h[d] = 0;
+    if (found) continue;
+    if (cum + v > rem) {
+      st[0] |= (unsigned long long)d << shift;
+      st[1] = rem - cum;
+      found = true;
+    } else {
+      cum += v;
+    }
+  }
+  if (!found) {
+    st[2] = 1;
+    st[0] = ~0ull;  // every item is below the cut
+  }
+}
+
+// ------------------------------------------------------------------ tiers --
+
+__global__ void tier_kernel(const __grid_constant__ AllocParams p) {
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= (long long)p.B * p.Hkv * p.Tmax) return;
+  const long long t = i % p.Tmax;
+  const long long bh = i / p.Tmax;
+  const int h = (int)(bh % p.Hkv), b = (int)(bh / p.Hkv);
+  uint8_t tr = SKV_TIER_DROP;
+  if (t < p.seq_lens[b]) {
+    const float w = p.keyw[i];
+    if (w < 0.0f) {
+      tr = SKV_TIER_T0;
+    } else if (p.mode == SKV_MODE_BUDGET) {
+      const unsigned long long cut = p.sel[(size_t)b * 3 * 3 + 0];
+      int lvl = 0;
+#pragma unroll
+      for (int k = 0; k < 3; ++k) {
+        const float key = __fmul_rn(w, p.kappa[k]);
+        const unsigned long long comp =
+            ((unsigned long long)(0xFFFFFFFFu - __float_as_uint(key)) << 32) |
+            ((unsigned long long)k << 30) | ((unsigned long long)h << 23) | (unsigned long long)t;
+        lvl += comp < cut;
+      }
+      tr = lvl == 3 ? SKV_TIER_T0 : (lvl == 2 ? SKV_TIER_T1 : (lvl == 1 ? SKV_TIER_T2 : SKV_TIER_DROP));
+    } else {
+      const unsigned long long comp =
+          ((unsigned long long)(0xFFFFFFFFu - __float_as_uint(w)) << 32) | (unsigned long long)t;
+      const unsigned long long* st = p.sel + (size_t)bh * 3 * 3;
+      if (comp < st[0]) tr = SKV_TIER_T0;
+      else if (comp < st[3]) tr = SKV_TIER_T1;
+      else if (comp < st[6]) tr = SKV_TIER_T2;
+    }
+  }
+  p.tier_out[i] = tr;
+  if (tr == SKV_TIER_DROP) p.row_of[i] = -1;
+}
+
+// -------------------------------------------------------- counts and plan --
+
+__global__ void unit_count_kernel(const __grid_constant__ AllocParams p) {
+  __shared__ int c[3];
+  const int u = blockIdx.x;
+  const int b = u / p.Hkv;
+  if (threadIdx.x < 3) c[threadIdx.x] = 0;
+  __syncthreads();
+  const long long T = p.seq_lens[b];
+  int l0 = 0, l1 = 0, l2 = 0;
+  for (long long t = threadIdx.x; t < T; t += blockDim.x) {
+    if (p.dense) {
+      ++l0;
+      continue;
+    }
+    const uint8_t tr = p.tier_out[(long long)u * p.Tmax + t];
+    l0 += tr == 0;
+    l1 += tr == 1;
+    l2 += tr == 2;
+  }
+  atomicAdd(&c[0], l0);
+  atomicAdd(&c[1], l1);
+  atomicAdd(&c[2], l2);
+  __syncthreads();
+  if (threadIdx.x < 3) p.counts[u * 3 + threadIdx.x] = c[threadIdx.x];
+}
+
+// block-wide exclusive scan of long long (blockDim.x = 1024)
+__device__ long long block_exclusive_scan(long long v, long long& total) {
+  __shared__ long long wsum[32];
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  long long x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const long long y = __shfl_up_sync(0xFFFFFFFFu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) wsum[wid] = x;
+  __syncthreads();
+  if (wid == 0) {
+    const int nw = blockDim.x >> 5;
+    long long s = lane < nw ? wsum[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const long long y = __shfl_up_sync(0xFFFFFFFFu, s, o);
+      if (lane >= o) s += y;
+    }
+    wsum[lane] = s;
+  }
+  __syncthreads();
+  const long long before = (wid > 0 ? wsum[wid - 1] : 0) + x - v;
+  total = wsum[(blockDim.x >> 5) - 1];
+  __syncthreads();
+  return before;
+}
+
+__global__ void __launch_bounds__(1024) page_plan_kernel(const __grid_constant__ AllocParams p) {
+  const int U = p.B * p.Hkv;
+  const int per = (U + blockDim.x - 1) / blockDim.x;
+  const int u0 = threadIdx.x * per, u1 = min(U, u0 + per);
+  long long s[4] = {0, 0, 0, 0};
+  for (int u = u0; u < u1; ++u) {
+    for (int t = 0; t < 3; ++t) {
+      const long long np = (p.counts[u * 3 + t] + p.P - 1) / p.P;
+      s[t] += np;
+      s[3] += np;
+    }
+  }
+  long long base[4], tot[4];
+  for (int k = 0; k < 4; ++k) base[k] = block_exclusive_scan(s[k], tot[k]);
+  for (int u = u0; u < u1; ++u) {
+    p.indptr[u] = (int32_t)base[3];
+    for (int t = 0; t < 3; ++t) {
+      p.tbase[u * 3 + t] = (int32_t)base[t];
+      const long long np = (p.counts[u * 3 + t] + p.P - 1) / p.P;
+      base[t] += np;
+      base[3] += np;
+    }
+  }
+  if (threadIdx.x == 0) {
+    p.indptr[U] = (int32_t)tot[3];
+    bool bad = tot[3] > p.page_cap || tot[3] > 0x7FFFFFFFLL;
+    for (int t = 0; t < 3; ++t) bad |= tot[t] > p.free_len[t];
+    if (bad) report(p.err, SKV_ERR_POOL);
+  }
+}
+
+__global__ void __launch_bounds__(1024) row_of_kernel(const __grid_constant__ AllocParams p) {
+  const int u = blockIdx.x;
+  const int b = u / p.Hkv;
+  const long long T = p.seq_lens[b];
+  const int P = p.P;
+  const long long c0 = p.counts[u * 3], c1 = p.counts[u * 3 + 1];
+  const long long pb[3] = {0, (c0 + P - 1) / P, (c0 + P - 1) / P + (c1 + P - 1) / P};
+  long long run[3] = {0, 0, 0};
+  for (long long base = 0; base < T; base += blockDim.x) {
+    const long long t = base + threadIdx.x;
+    const long long i = (long long)u * p.Tmax + t;
+    int tr = SKV_TIER_DROP;
+    if (t < T) tr = p.tier_out[i];
+    const long long f = tr == 0 ? 1LL : (tr == 1 ? (1LL << 21) : (tr == 2 ? (1LL << 42) : 0LL));
+    long long tot;
+    const long long ex = block_exclusive_scan(f, tot);
+    if (t < T && tr < 3) {
+      const long long rank = run[tr] + ((ex >> (21 * tr)) & ((1LL << 21) - 1));
+      p.row_of[i] = (int32_t)((pb[tr] + rank / P) * P + rank % P);
+    }
+    for (int k = 0; k < 3; ++k) run[k] += (tot >> (21 * k)) & ((1LL << 21) - 1);
+  }
+}
+
+// one warp per page: page id, header, zeroed payload for a partial page
+__global__ void __launch_bounds__(256) page_write_kernel(const __grid_constant__ AllocParams p) {
+  const int U = p.B * p.Hkv;
+  const long long total = p.indptr[U];
+  const int lane = threadIdx.x & 31;
+  const long long nwarps = (long long)gridDim.x * (blockDim.x >> 5);
+  for (long long g = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5; g < total;
+       g += nwarps) {
+    int lo = 0, hi = U;  // largest u with indptr[u] <= g
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (p.indptr[mid] <= g) lo = mid; else hi = mid;
+    }
+    const int u = lo;
+    const int P = p.P;
+    const long long local = g - p.indptr[u];
+    const long long n0 = p.counts[u * 3], n1 = p.counts[u * 3 + 1], n2 = p.counts[u * 3 + 2];
+    const long long np0 = (n0 + P - 1) / P, np1 = (n1 + P - 1) / P;
+    int t;
+    long long pg, n;
+    if (local < np0) { t = 0; pg = local; n = n0; }
+    else if (local < np0 + np1) { t = 1; pg = local - np0; n = n1; }
+    else { t = 2; pg = local - np0 - np1; n = n2; }
+    const long long fi = p.tbase[u * 3 + t] + pg;
+    if (g >= p.page_cap || fi >= p.free_len[t]) {
+      if (lane == 0) report(p.err, SKV_ERR_POOL);
+      continue;
+    }
+    const uint32_t slot = p.free_ids[t][fi];
+    if ((long long)slot >= p.slots[t] || slot > 0x3FFFFFFFu) {
+      if (lane == 0) report(p.err, SKV_ERR_POOL);
+      continue;
+    }
+    if (lane == 0) p.page_ids[g] = ((uint32_t)t << 30) | slot;
+    const int cnt = (int)min((long long)P, n - pg * P);
+    uint8_t* page = p.pool[t] + (long long)slot * p.stride[t];
+    if (cnt < P) {
+      for (int o = kHdrBytes + 16 * lane; o < p.payload[t]; o += 32 * 16)
+        *reinterpret_cast<uint4*>(page + o) = make_uint4(0, 0, 0, 0);
+    }
+    if (lane == 0) {
+      uint4 hdr;
+      hdr.x = (uint32_t)cnt | ((uint32_t)t << 16) | ((uint32_t)kPageMagic << 24);
+      hdr.y = (uint32_t)(u / p.Hkv);
+      hdr.z = (uint32_t)(u % p.Hkv);
+      hdr.w = (uint32_t)pg;
+      *reinterpret_cast<uint4*>(page) = hdr;
+    }
+  }
+}
+
+static unsigned grid_for(long long n, int threads) {
+  long long b = (n + threads - 1) / threads;
+  return (unsigned)(b < 1 ? 1 : b);
+}
+
+cudaError_t launch_allocate(AllocParams& p, cudaStream_t stream) {
+  const long long ntok = (long long)p.B * p.Hkv * p.Tmax;
+  const int U = p.B * p.Hkv;
+  p.dense = 0;
+  p.nseg = p.mode == SKV_MODE_BUDGET ? p.B : U;
+  cudaError_t e;
+  if ((e = cudaMemsetAsync(p.nprot, 0, 8 * (size_t)p.B, stream)) != cudaSuccess) return e;
+  if ((e = cudaMemsetAsync(p.hist, 0, 8 * (size_t)p.nseg * 3 * 256, stream)) != cudaSuccess)
+    return e;
+  if (ntok > 0) {
+    if (p.mode == SKV_MODE_BUDGET)
+      keys_budget_kernel<<<grid_for(ntok * 32, 256), 256, 0, stream>>>(p);
+    else
+      keys_quota_kernel<<<grid_for(ntok, 256), 256, 0, stream>>>(p);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  sel_init_kernel<<<grid_for(p.nseg * 3, 128), 128, 0, stream>>>(p);
+  const long long n_items =
+      p.mode == SKV_MODE_BUDGET ? (long long)p.Hkv * p.Tmax * 3 : (long long)p.Tmax;
+  const dim3 hgrid(grid_for(n_items, kHistItemsPerBlock), p.nseg);
+  for (int pass = 0; pass < 8; ++pass) {
+    const int shift = 56 - 8 * pass;
+    hist_kernel<<<hgrid, 256, 0, stream>>>(p, shift);
+    sel_step_kernel<<<grid_for(p.nseg * 3, 128), 128, 0, stream>>>(p, shift);
+  }
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (ntok > 0) tier_kernel<<<grid_for(ntok, 256), 256, 0, stream>>>(p);
+  unit_count_kernel<<<U, 256, 0, stream>>>(p);
+  page_plan_kernel<<<1, 1024, 0, stream>>>(p);
+  row_of_kernel<<<U, 1024, 0, stream>>>(p);
+  page_write_kernel<<<grid_for(std::min<long long>(p.page_cap, 1LL << 22) * 32, 256), 256, 0,
+                      stream>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dense_plan(AllocParams& p, cudaStream_t stream) {
+  const int U = p.B * p.Hkv;
+  p.dense = 1;
+  unit_count_kernel<<<U, 256, 0, stream>>>(p);
+  page_plan_kernel<<<1, 1024, 0, stream>>>(p);
+  page_write_kernel<<<grid_for(std::min<long long>(p.page_cap, 1LL << 22) * 32, 256), 256, 0,
+                      stream>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace skv

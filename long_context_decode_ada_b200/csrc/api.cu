@@ -1,0 +1,465 @@
+// api.cu -- the extern "C" entry points of libskv (declared in include/skv.h).
+// Host-side argument checks, the context's constant tables and the kernel
+// launches.  No allocation happens here except the context struct itself.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+#include "../../include/skv.h"
+#include "common.cuh"
+#include "kernels.h"
+
+struct skv_ctx {
+  int d;
+  int P;
+  int log2P;
+  int device;
+  int sm_count;
+  size_t smem_optin;
+  float bx6[64], by6[64], bx4[16], by4[16];
+  float cos6[64], sin6[64], cos4[16], sin4[16];
+  float kappa[3];
+  float rho_levels[4];
+  long long payload[4];
+  long long stride[4];
+  cudaEvent_t profile_event;
+};
+
+namespace {
+
+thread_local std::string g_err;
+
+int fail(int code, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return code;
+}
+
+int ok() {
+  g_err.clear();
+  return SKV_OK;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(SKV_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+// Relative mean-squared logit error of a b-bit uniform angle quantiser:
+// 2 (1 - sin(x)/x), x = pi / 2^b (half the sector width).
+double angle_distortion(int b) {
+  const double x = M_PI / (double)(1 << b);
+  return 2.0 * (1.0 - std::sin(x) / x);
+}
+
+bool valid_pools(const skv_pools* pools, int ntiers) {
+  if (!pools) return false;
+  for (int t = 0; t < ntiers; ++t) {
+    if (pools->slots[t] < 0) return false;
+    if (pools->slots[t] > 0 && !pools->base[t]) return false;
+    if ((reinterpret_cast<uintptr_t>(pools->base[t]) & 127) != 0) return false;
+  }
+  return true;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* skv_last_error(void) { return g_err.c_str(); }
+
+int skv_create(const skv_config* cfg, skv_ctx** out) {
+  if (!cfg || !out) return fail(SKV_ERR_ARG, "skv_create: null argument");
+  *out = nullptr;
+  if (cfg->head_dim != 128) return fail(SKV_ERR_ARG, "head_dim must be 128 (got %d)", cfg->head_dim);
+  const int P = cfg->page_size;
+  if (P != 16 && P != 32 && P != 64) return fail(SKV_ERR_ARG, "page_size must be 16, 32 or 64");
+  skv_ctx* c = new (std::nothrow) skv_ctx();
+  if (!c) return fail(SKV_ERR_ARG, "out of host memory");
+  c->d = 128;
+  c->P = P;
+  c->log2P = P == 16 ? 4 : (P == 32 ? 5 : 6);
+  c->device = 0;
+  c->profile_event = nullptr;
+  c->sm_count = 148;
+  c->smem_optin = 232448;
+  int dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess) {
+    c->device = dev;
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0)
+      c->sm_count = v;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) == cudaSuccess &&
+        v > 0)
+      c->smem_optin = (size_t)v;
+  } else {
+    cudaGetLastError();
+  }
+  for (int j = 0; j < 64; ++j) {
+    const double beta = (j + 0.5) * (2.0 * M_PI / 64.0);
+    c->bx6[j] = (float)std::cos(beta);
+    c->by6[j] = (float)std::sin(beta);
+    const double a = 2.0 * M_PI * j / 64.0;
+    c->cos6[j] = (float)std::cos(a);
+    c->sin6[j] = (float)std::sin(a);
+  }
+  for (int j = 0; j < 16; ++j) {
+    const double beta = (j + 0.5) * (2.0 * M_PI / 16.0);
+    c->bx4[j] = (float)std::cos(beta);
+    c->by4[j] = (float)std::sin(beta);
+    const double a = 2.0 * M_PI * j / 16.0;
+    c->cos4[j] = (float)std::cos(a);
+    c->sin4[j] = (float)std::sin(a);
+  }
+  const double c6 = angle_distortion(6), c4 = angle_distortion(4);
+  c->kappa[0] = (float)((1.0 - c4) / 180.0);
+  c->kappa[1] = (float)((c4 - c6) / 16.0);
+  c->kappa[2] = (float)(c6 / 316.0);
+  for (int k = 0; k < 4; ++k) c->rho_levels[k] = (float)((k + 1) / 16.0);
+  const int rowb[4] = {512, 196, 180, 512};
+  for (int t = 0; t < 4; ++t) {
+    c->payload[t] = skv::kHdrBytes + (long long)P * rowb[t];
+    c->stride[t] = (c->payload[t] + 127) / 128 * 128;
+  }
+  *out = c;
+  return ok();
+}
+
+int skv_destroy(skv_ctx* ctx) {
+  delete ctx;
+  return ok();
+}
+
+int skv_page_bytes(const skv_ctx* ctx, int tier, int64_t* payload, int64_t* stride) {
+  if (!ctx || tier < 0 || tier > 4 || tier == SKV_TIER_DROP)
+    return fail(SKV_ERR_ARG, "skv_page_bytes: bad tier %d", tier);
+  const int t = tier == 4 ? 3 : tier;
+  if (payload) *payload = ctx->payload[t];
+  if (stride) *stride = ctx->stride[t];
+  return ok();
+}
+
+int skv_tables(const skv_ctx* ctx, int which, float* out, int64_t n) {
+  if (!ctx || !out) return fail(SKV_ERR_ARG, "skv_tables: null argument");
+  const float* src = nullptr;
+  int64_t len = 0;
+  switch (which) {
+    case SKV_TABLE_BOUNDARY6_X: src = ctx->bx6; len = 64; break;
+    case SKV_TABLE_BOUNDARY6_Y: src = ctx->by6; len = 64; break;
+    case SKV_TABLE_BOUNDARY4_X: src = ctx->bx4; len = 16; break;
+    case SKV_TABLE_BOUNDARY4_Y: src = ctx->by4; len = 16; break;
+    case SKV_TABLE_KAPPA: src = ctx->kappa; len = 3; break;
+    case SKV_TABLE_RHO_LEVELS: src = ctx->rho_levels; len = 4; break;
+    default: return fail(SKV_ERR_ARG, "skv_tables: unknown table %d", which);
+  }
+  if (n < len) return fail(SKV_ERR_ARG, "skv_tables: need %lld floats", (long long)len);
+  std::memcpy(out, src, sizeof(float) * len);
+  return ok();
+}
+
+int skv_device_info(const skv_ctx* ctx, int* sm_count, int* default_splits) {
+  if (!ctx) return fail(SKV_ERR_ARG, "skv_device_info: null ctx");
+  if (sm_count) *sm_count = ctx->sm_count;
+  if (default_splits) *default_splits = ctx->sm_count;
+  return ok();
+}
+
+static int decode_splits(const skv_ctx* ctx, int num_splits) {
+  return num_splits > 0 ? num_splits : ctx->sm_count;
+}
+
+int skv_workspace_size(const skv_ctx* ctx, int which, int B, int Hkv, int Hq, int64_t Tmax,
+                       int num_splits, size_t* bytes) {
+  if (!ctx || !bytes) return fail(SKV_ERR_ARG, "skv_workspace_size: null argument");
+  if (B < 0 || Hkv <= 0 || Tmax < 0) return fail(SKV_ERR_ARG, "skv_workspace_size: bad sizes");
+  if (which == SKV_WS_ALLOCATE) {
+    *bytes = skv::alloc_workspace_bytes(B, Hkv, Tmax);
+    return ok();
+  }
+  if (which == SKV_WS_DECODE || which == SKV_WS_DENSE_DECODE) {
+    if (Hq <= 0 || Hq % Hkv != 0) return fail(SKV_ERR_ARG, "Hq must be a multiple of Hkv");
+    const int G = Hq / Hkv;
+    const long long S = decode_splits(ctx, num_splits);
+    *bytes = (size_t)(S + (long long)B * Hkv) * G * skv::kPartStride * sizeof(float);
+    return ok();
+  }
+  return fail(SKV_ERR_ARG, "skv_workspace_size: unknown kind %d", which);
+}
+
+static int fill_alloc_common(skv::AllocParams& p, const skv_ctx* ctx, int B, int Hkv,
+                             int64_t Tmax) {
+  std::memset(&p, 0, sizeof(p));
+  p.B = B;
+  p.Hkv = Hkv;
+  p.Tmax = Tmax;
+  p.P = ctx->P;
+  for (int k = 0; k < 3; ++k) p.kappa[k] = ctx->kappa[k];
+  return SKV_OK;
+}
+
+int skv_allocate(skv_ctx* ctx, const uint16_t* K, int B, int Hkv, int64_t Tmax,
+                 const int32_t* seq_lens, const float* utility, const uint8_t* protect, int mode,
+                 const int64_t* budget, const int32_t* quota, const skv_free_lists* free,
+                 const skv_pools* pools, uint8_t* tier_out, int32_t* row_of,
+                 int32_t* page_indptr, uint32_t* page_ids, int64_t page_cap, int32_t* err_word,
+                 void* workspace, size_t ws_bytes, void* stream) {
+  if (!ctx) return fail(SKV_ERR_ARG, "skv_allocate: null ctx");
+  if (B < 0 || Hkv <= 0 || Hkv > 128 || Tmax < 0 || Tmax > (1LL << 23))
+    return fail(SKV_ERR_ARG, "skv_allocate: need B >= 0, 0 < Hkv <= 128, 0 <= Tmax <= 2^23");
+  if ((long long)B * Hkv > (1 << 30)) return fail(SKV_ERR_ARG, "skv_allocate: too many units");
+  if (mode != SKV_MODE_BUDGET && mode != SKV_MODE_QUOTA)
+    return fail(SKV_ERR_ARG, "skv_allocate: unknown mode %d", mode);
+  if (mode == SKV_MODE_BUDGET && (!utility || !budget || !K))
+    return fail(SKV_ERR_ARG, "skv_allocate: budget mode needs K, utility and budget");
+  if (mode == SKV_MODE_QUOTA && !quota)
+    return fail(SKV_ERR_ARG, "skv_allocate: quota mode needs quota");
+  if (!seq_lens || !free || !pools || !tier_out || !row_of || !page_indptr || !err_word)
+    return fail(SKV_ERR_ARG, "skv_allocate: null argument");
+  if (page_cap > 0 && !page_ids) return fail(SKV_ERR_ARG, "skv_allocate: null page_ids");
+  if (!valid_pools(pools, 3))
+    return fail(SKV_ERR_ARG, "skv_allocate: pools need 128-byte aligned bases");
+  for (int t = 0; t < 3; ++t)
+    if (free->len[t] < 0 || (free->len[t] > 0 && !free->ids[t]))
+      return fail(SKV_ERR_ARG, "skv_allocate: bad free list %d", t);
+  const size_t need = skv::alloc_workspace_bytes(B, Hkv, Tmax);
+  if (!workspace || ws_bytes < need)
+    return fail(SKV_ERR_ARG, "skv_allocate: workspace of %zu bytes needed", need);
+  skv::AllocParams p;
+  fill_alloc_common(p, ctx, B, Hkv, Tmax);
+  p.K = K;
+  p.seq_lens = seq_lens;
+  p.utility = utility;
+  p.protect = protect;
+  p.mode = mode;
+  p.budget = budget;
+  p.quota = quota;
+  for (int t = 0; t < 3; ++t) {
+    p.free_ids[t] = free->ids[t];
+    p.free_len[t] = free->len[t];
+    p.pool[t] = static_cast<uint8_t*>(pools->base[t]);
+    p.slots[t] = pools->slots[t];
+    p.stride[t] = ctx->stride[t];
+    p.payload[t] = (int)ctx->payload[t];
+  }
+  p.tier_out = tier_out;
+  p.row_of = row_of;
+  p.indptr = page_indptr;
+  p.page_ids = page_ids;
+  p.page_cap = page_cap;
+  p.err = err_word;
+  skv::alloc_carve(p, workspace);
+  cudaError_t e = skv::launch_allocate(p, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "skv_allocate launch");
+  return ok();
+}
+
+int skv_encode(skv_ctx* ctx, const uint16_t* K, const uint16_t* V, int B, int Hkv, int64_t Tmax,
+               const int32_t* seq_lens, const uint8_t* tier, const int32_t* row_of,
+               const int32_t* page_indptr, const uint32_t* page_ids, const skv_pools* pools,
+               int32_t* err_word, void* stream) {
+  if (!ctx) return fail(SKV_ERR_ARG, "skv_encode: null ctx");
+  if (B < 0 || Hkv <= 0 || Tmax < 0) return fail(SKV_ERR_ARG, "skv_encode: bad sizes");
+  if (!K || !V || !seq_lens || !tier || !row_of || !page_indptr || !err_word)
+    return fail(SKV_ERR_ARG, "skv_encode: null argument");
+  if (!valid_pools(pools, 3)) return fail(SKV_ERR_ARG, "skv_encode: bad pools");
+  skv::EncodeParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.K = K;
+  p.V = V;
+  p.B = B;
+  p.Hkv = Hkv;
+  p.Tmax = Tmax;
+  p.P = ctx->P;
+  p.seq_lens = seq_lens;
+  p.tier = tier;
+  p.row_of = row_of;
+  p.indptr = page_indptr;
+  p.ids = page_ids;
+  for (int t = 0; t < 3; ++t) {
+    p.pool[t] = static_cast<uint8_t*>(pools->base[t]);
+    p.slots[t] = pools->slots[t];
+    p.stride[t] = ctx->stride[t];
+  }
+  p.err = err_word;
+  p.dense_bf16 = 0;
+  std::memcpy(p.bx6, ctx->bx6, sizeof(p.bx6));
+  std::memcpy(p.by6, ctx->by6, sizeof(p.by6));
+  std::memcpy(p.bx4, ctx->bx4, sizeof(p.bx4));
+  std::memcpy(p.by4, ctx->by4, sizeof(p.by4));
+  cudaError_t e = skv::launch_encode(p, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "skv_encode launch");
+  return ok();
+}
+
+static int decode_common(skv_ctx* ctx, const void* q, int q_dtype, int B, int Hq, int Hkv,
+                         const int32_t* page_indptr, const uint32_t* page_ids, const void* pool[3],
+                         const long long slots[3], bool dense, float* out, float* lse,
+                         int32_t* err_word, void* workspace, size_t ws_bytes, int num_splits,
+                         void* stream, const char* name) {
+  if (!ctx) return fail(SKV_ERR_ARG, "%s: null ctx", name);
+  if (B < 0 || Hkv <= 0 || Hq <= 0 || Hq % Hkv != 0)
+    return fail(SKV_ERR_ARG, "%s: need B >= 0 and Hq a multiple of Hkv", name);
+  const int G = Hq / Hkv;
+  if (G != 1 && G != 2 && G != 4) return fail(SKV_ERR_ARG, "%s: Hq/Hkv must be 1, 2 or 4", name);
+  if (q_dtype != SKV_Q_BF16 && q_dtype != SKV_Q_FP16)
+    return fail(SKV_ERR_ARG, "%s: unknown q dtype %d", name, q_dtype);
+  if (num_splits < 0) return fail(SKV_ERR_ARG, "%s: num_splits < 0", name);
+  if (B == 0) return ok();
+  if (!q || !page_indptr || !out || !err_word)
+    return fail(SKV_ERR_ARG, "%s: null argument", name);
+  size_t need = 0;
+  skv_workspace_size(ctx, dense ? SKV_WS_DENSE_DECODE : SKV_WS_DECODE, B, Hkv, Hq, 0, num_splits,
+                     &need);
+  if (!workspace || ws_bytes < need)
+    return fail(SKV_ERR_ARG, "%s: workspace of %zu bytes needed", name, need);
+  skv::DecodeParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.q = q;
+  p.q_bf16 = q_dtype == SKV_Q_BF16;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.indptr = page_indptr;
+  p.ids = page_ids;
+  for (int t = 0; t < 3; ++t) {
+    p.pool[t] = static_cast<const uint8_t*>(pool[t]);
+    p.slots[t] = slots[t];
+    const int ti = dense ? 3 : t;
+    p.stride[t] = ctx->stride[ti];
+    p.payload[t] = (int)ctx->payload[ti];
+  }
+  p.out = out;
+  p.lse = lse;
+  p.err = err_word;
+  p.part = static_cast<float*>(workspace);
+  p.S = decode_splits(ctx, num_splits);
+  p.P = ctx->P;
+  p.log2P = ctx->log2P;
+  const size_t fixed = skv::decode_fixed_smem(G, dense);
+  long long ring = ((long long)ctx->smem_optin - (long long)fixed) / 128 * 128;
+  const long long max_item = 64LL * 512 + 4 * skv::kHdrBytes;
+  if (ring < max_item) return fail(SKV_ERR_ARG, "%s: not enough shared memory", name);
+  p.ring_bytes = (int)std::min<long long>(ring, 1 << 20);
+  p.qk_scale_log2 = (float)(1.4426950408889634 / std::sqrt(128.0));
+  std::memcpy(p.cos6, ctx->cos6, sizeof(p.cos6));
+  std::memcpy(p.sin6, ctx->sin6, sizeof(p.sin6));
+  std::memcpy(p.cos4, ctx->cos4, sizeof(p.cos4));
+  std::memcpy(p.sin4, ctx->sin4, sizeof(p.sin4));
+  cudaError_t e =
+      skv::launch_decode(p, G, dense, static_cast<cudaStream_t>(stream), ctx->profile_event);
+  if (e != cudaSuccess) return cuda_fail(e, name);
+  return ok();
+}
+
+int skv_decode_attention(skv_ctx* ctx, const void* q, int q_dtype, int B, int Hq, int Hkv,
+                         const int32_t* page_indptr, const uint32_t* page_ids,
+                         const skv_pools* pools, float* out, float* lse, int32_t* err_word,
+                         void* workspace, size_t ws_bytes, int num_splits, void* stream) {
+  if (!valid_pools(pools, 3)) return fail(SKV_ERR_ARG, "skv_decode_attention: bad pools");
+  const void* pool[3] = {pools->base[0], pools->base[1], pools->base[2]};
+  const long long slots[3] = {pools->slots[0], pools->slots[1], pools->slots[2]};
+  return decode_common(ctx, q, q_dtype, B, Hq, Hkv, page_indptr, page_ids, pool, slots, false, out,
+                       lse, err_word, workspace, ws_bytes, num_splits, stream,
+                       "skv_decode_attention");
+}
+
+int skv_dense_decode_bf16(skv_ctx* ctx, const void* q, int q_dtype, int B, int Hq, int Hkv,
+                          const int32_t* page_indptr, const uint32_t* page_ids, const void* pool,
+                          int64_t pool_slots, float* out, float* lse, int32_t* err_word,
+                          void* workspace, size_t ws_bytes, int num_splits, void* stream) {
+  if ((reinterpret_cast<uintptr_t>(pool) & 127) != 0 || pool_slots < 0)
+    return fail(SKV_ERR_ARG, "skv_dense_decode_bf16: bad pool");
+  const void* pools[3] = {pool, nullptr, nullptr};
+  const long long slots[3] = {pool_slots, 0, 0};
+  return decode_common(ctx, q, q_dtype, B, Hq, Hkv, page_indptr, page_ids, pools, slots, true, out,
+                       lse, err_word, workspace, ws_bytes, num_splits, stream,
+                       "skv_dense_decode_bf16");
+}
+
+int skv_dense_pack_bf16(skv_ctx* ctx, const uint16_t* K, const uint16_t* V, int B, int Hkv,
+                        int64_t Tmax, const int32_t* seq_lens, const uint32_t* free_ids,
+                        int64_t free_len, void* pool, int64_t pool_slots, int32_t* page_indptr,
+                        uint32_t* page_ids, int64_t page_cap, int32_t* err_word, void* workspace,
+                        size_t ws_bytes, void* stream) {
+  if (!ctx) return fail(SKV_ERR_ARG, "skv_dense_pack_bf16: null ctx");
+  if (B < 0 || Hkv <= 0 || Hkv > 128 || Tmax < 0)
+    return fail(SKV_ERR_ARG, "skv_dense_pack_bf16: bad sizes");
+  if (!K || !V || !seq_lens || !page_indptr || !err_word || (free_len > 0 && !free_ids))
+    return fail(SKV_ERR_ARG, "skv_dense_pack_bf16: null argument");
+  if ((reinterpret_cast<uintptr_t>(pool) & 127) != 0 || pool_slots < 0)
+    return fail(SKV_ERR_ARG, "skv_dense_pack_bf16: bad pool");
+  const size_t need = skv::alloc_workspace_bytes(B, Hkv, Tmax);
+  if (!workspace || ws_bytes < need)
+    return fail(SKV_ERR_ARG, "skv_dense_pack_bf16: workspace of %zu bytes needed", need);
+  skv::AllocParams a;
+  fill_alloc_common(a, ctx, B, Hkv, Tmax);
+  a.seq_lens = seq_lens;
+  a.free_ids[0] = free_ids;
+  a.free_len[0] = free_len;
+  a.pool[0] = static_cast<uint8_t*>(pool);
+  a.slots[0] = pool_slots;
+  a.stride[0] = ctx->stride[3];
+  a.payload[0] = (int)ctx->payload[3];
+  a.indptr = page_indptr;
+  a.page_ids = page_ids;
+  a.page_cap = page_cap;
+  a.err = err_word;
+  skv::alloc_carve(a, workspace);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = skv::launch_dense_plan(a, s);
+  if (e != cudaSuccess) return cuda_fail(e, "skv_dense_pack_bf16 plan");
+  skv::EncodeParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.K = K;
+  p.V = V;
+  p.B = B;
+  p.Hkv = Hkv;
+  p.Tmax = Tmax;
+  p.P = ctx->P;
+  p.seq_lens = seq_lens;
+  p.indptr = page_indptr;
+  p.ids = page_ids;
+  p.pool[0] = static_cast<uint8_t*>(pool);
+  p.slots[0] = pool_slots;
+  p.stride[0] = ctx->stride[3];
+  p.err = err_word;
+  p.dense_bf16 = 1;
+  e = skv::launch_encode(p, s);
+  if (e != cudaSuccess) return cuda_fail(e, "skv_dense_pack_bf16 encode");
+  return ok();
+}
+
+int skv_set_profile_event(skv_ctx* ctx, void* event) {
+  if (!ctx) return fail(SKV_ERR_ARG, "skv_set_profile_event: null ctx");
+  ctx->profile_event = static_cast<cudaEvent_t>(event);
+  return ok();
+}
+
+int skv_check(skv_ctx* ctx, int32_t* err_word, void* stream) {
+  if (!ctx || !err_word) return fail(SKV_ERR_ARG, "skv_check: null argument");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "skv_check: stream synchronize");
+  int32_t v = 0;
+  e = cudaMemcpy(&v, err_word, sizeof(v), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "skv_check: read error word");
+  e = cudaMemset(err_word, 0, sizeof(int32_t));
+  if (e != cudaSuccess) return cuda_fail(e, "skv_check: reset error word");
+  if (v != 0) {
+    static const char* names[] = {"ok", "argument", "budget", "pool", "corrupt page table",
+                                  "cuda", "timeout"};
+    return fail(v, "device reported error %d (%s)", v, (v >= 0 && v <= 6) ? names[v] : "?");
+  }
+  return ok();
+}
+
+}  // extern "C"

@@ -1,0 +1,275 @@
+// encode.cu -- "maps dense keys to spherical codes" (SPHERICAL KV technical
+// summary 2.3) in the representation of 2.1: r~ = fp16 |k| plus per-pair
+// angle and share codes, and int8 V with a per-token scale, written into the
+// page row that the allocation assigned.  Also writes the dense bf16
+// baseline's rows.
+//
+// One warp per (seq, kv head, token); lane l holds dims 4l..4l+3 (pairs 2l,
+// 2l+1).  Every code is an integer decision taken exactly:
+//   R2 = sum of m_c^2 over the fp16 keys (k_c = m_c 2^-24) in 128-bit integers,
+//   r~ = fp16_rn(min(sqrt(double_rn(R2)) 2^-24, 65504)),
+//   angle sector: quadrant from signs, binary search over fp32 boundary
+//   vectors with exactly-signed fp64 cross products (no fused multiply-add),
+//   share code: 16 (d/2) rho^2 > {9, 25, 49} R2 in 128-bit integers,
+//   V: s = fp16_rn(absmax / 127) and rint(v / s) in IEEE fp32.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace skv {
+
+typedef unsigned __int128 u128;
+
+__device__ __forceinline__ uint16_t double_to_half_rn(double x) {
+  uint16_t r;
+  asm("cvt.rn.f16.f64 %0, %1;" : "=h"(r) : "d"(x));
+  return r;
+}
+
+__device__ __forceinline__ double half_to_double(uint16_t h) {
+  return (double)__half2float(__ushort_as_half(h));
+}
+
+__device__ __forceinline__ u128 warp_sum_u128(u128 v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    unsigned long long lo = (unsigned long long)v, hi = (unsigned long long)(v >> 64);
+    unsigned long long olo = __shfl_xor_sync(0xFFFFFFFFu, lo, o);
+    unsigned long long ohi = __shfl_xor_sync(0xFFFFFFFFu, hi, o);
+    v += ((u128)ohi << 64) | olo;
+  }
+  return v;
+}
+
+// b-bit angle sector of (x, y); bx/by: the 2^b boundary vectors.
+__device__ __forceinline__ uint32_t angle_code(uint16_t xh, uint16_t yh, int b, const float* bx,
+                                               const float* by) {
+  const double x = half_to_double(xh), y = half_to_double(yh);
+  if (x == 0.0 && y == 0.0) return 0;
+  int q;
+  if (x > 0 && y >= 0) q = 0;
+  else if (x <= 0 && y > 0) q = 1;
+  else if (x < 0 && y <= 0) q = 2;
+  else q = 3;
+  const int per = 1 << (b - 2);
+  const int base = q * per;
+  // count of boundaries j in [base, base + per) that the point is on or
+  // counter-clockwise of: a prefix of that range
+  int lo = 0, hi = per;
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    const double side = __dsub_rn(__dmul_rn((double)bx[base + mid], y),
+                                  __dmul_rn((double)by[base + mid], x));
+    if (side >= 0.0) lo = mid + 1;
+    else hi = mid;
+  }
+  return (uint32_t)(base + lo) & (uint32_t)((1 << b) - 1);
+}
+
+__device__ __forceinline__ uint32_t rho_code(long long mx, long long my, u128 R2) {
+  const u128 ax = (u128)(mx < 0 ? -mx : mx), ay = (u128)(my < 0 ? -my : my);
+  const u128 lhs = (ax * ax + ay * ay) * (u128)(16 * (kHeadDim / 2));
+  uint32_t c = 0;
+  c += lhs > (u128)9 * R2;
+  c += lhs > (u128)25 * R2;
+  c += lhs > (u128)49 * R2;
+  return c;
+}
+
+// byte offset, within a page's V section, of element (row, dim)
+__device__ __forceinline__ int v_frag_offset(int row, int dd, int elem_bytes) {
+  const int k = row >> 3, tr = row & 7, t4 = tr >> 1, lo = tr & 1;
+  const int mt = dd >> 4, rem = dd & 15, g = rem & 7, hi = rem >> 3;
+  const int L = 4 * g + t4, e = 2 * hi + lo;
+  if (elem_bytes == 1) return k * 1024 + 512 * (mt >> 2) + 16 * L + 4 * (mt & 3) + e;
+  return k * 2048 + 512 * (mt >> 1) + 16 * L + 8 * (mt & 1) + 2 * e;
+}
+
+__global__ void __launch_bounds__(256) encode_kernel(const __grid_constant__ EncodeParams p) {
+  __shared__ float sbx6[64], sby6[64], sbx4[16], sby4[16];
+  for (int i = threadIdx.x; i < 64; i += blockDim.x) {
+    sbx6[i] = p.bx6[i];
+    sby6[i] = p.by6[i];
+    if (i < 16) {
+      sbx4[i] = p.bx4[i];
+      sby4[i] = p.by4[i];
+    }
+  }
+  __syncthreads();
+  const long long w = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const long long total = (long long)p.B * p.Hkv * p.Tmax;
+  if (w >= total) return;
+  const long long t = w % p.Tmax;
+  const long long bh = w / p.Tmax;
+  const int h = (int)(bh % p.Hkv), b = (int)(bh / p.Hkv);
+  if (t >= p.seq_lens[b]) return;
+  const int P = p.P;
+  int tr, pi, row;
+  if (p.dense_bf16) {
+    tr = 0;
+    pi = (int)(t / P);
+    row = (int)(t % P);
+  } else {
+    tr = p.tier[w];
+    if (tr == SKV_TIER_DROP) return;
+    const int loc = p.row_of[w];
+    if (tr > SKV_TIER_DROP || loc < 0) {
+      if (lane == 0) report(p.err, SKV_ERR_CORRUPT);
+      return;
+    }
+    pi = loc / P;
+    row = loc % P;
+  }
+  const long long gi = (long long)p.indptr[bh] + pi;
+  if (gi >= p.indptr[bh + 1]) {
+    if (lane == 0) report(p.err, SKV_ERR_CORRUPT);
+    return;
+  }
+  const uint32_t id = p.ids[gi];
+  const uint32_t slot = id & 0x3FFFFFFFu;
+  if ((int)(id >> 30) != tr || (long long)slot >= p.slots[tr]) {
+    if (lane == 0) report(p.err, SKV_ERR_CORRUPT);
+    return;
+  }
+  uint8_t* page = p.pool[tr] + (long long)slot * p.stride[tr];
+  const uint2 kv = *reinterpret_cast<const uint2*>(p.K + w * kHeadDim + 4 * lane);
+  const uint2 vv = *reinterpret_cast<const uint2*>(p.V + w * kHeadDim + 4 * lane);
+  const uint16_t k4[4] = {(uint16_t)(kv.x & 0xFFFF), (uint16_t)(kv.x >> 16),
+                          (uint16_t)(kv.y & 0xFFFF), (uint16_t)(kv.y >> 16)};
+  const uint16_t v4[4] = {(uint16_t)(vv.x & 0xFFFF), (uint16_t)(vv.x >> 16),
+                          (uint16_t)(vv.y & 0xFFFF), (uint16_t)(vv.y >> 16)};
+
+  if (tr == SKV_TIER_T0) {
+    uint16_t ko[4], vo[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      if (p.dense_bf16) {
+        ko[i] = __bfloat16_as_ushort(__float2bfloat16_rn(__half2float(__ushort_as_half(k4[i]))));
+        vo[i] = __bfloat16_as_ushort(__float2bfloat16_rn(__half2float(__ushort_as_half(v4[i]))));
+      } else {
+        ko[i] = k4[i];
+        vo[i] = v4[i];
+      }
+    }
+    const int c = lane >> 1, e0 = (lane & 1) * 4;
+    const int pos = c ^ (4 * (row & 1));
+    uint2 kout;
+    kout.x = (uint32_t)ko[0] | ((uint32_t)ko[1] << 16);
+    kout.y = (uint32_t)ko[2] | ((uint32_t)ko[3] << 16);
+    *reinterpret_cast<uint2*>(page + kHdrBytes + row * 256 + pos * 16 + e0 * 2) = kout;
+    uint8_t* vsec = page + kHdrBytes + 256 * P;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      *reinterpret_cast<uint16_t*>(vsec + v_frag_offset(row, 4 * lane + i, 2)) = vo[i];
+    return;
+  }
+
+  // ---- radius
+  long long m[4];
+  u128 sq = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    m[i] = half_bits_to_m(k4[i]);
+    const u128 a = (u128)(m[i] < 0 ? -m[i] : m[i]);
+    sq += a * a;
+  }
+  const u128 R2 = warp_sum_u128(sq);
+  const double r2d = u128_to_double_rn((unsigned long long)(R2 >> 64), (unsigned long long)R2);
+  double r = __dmul_rn(__dsqrt_rn(r2d), 5.9604644775390625e-08);  // 2^-24
+  if (r > 65504.0) r = 65504.0;
+  const uint16_t rt = double_to_half_rn(r);
+
+  // ---- codes of pairs 2 lane, 2 lane + 1
+  const bool t1 = tr == SKV_TIER_T1;
+  const int bits = t1 ? 6 : 4;
+  const float* bx = t1 ? sbx6 : sbx4;
+  const float* by = t1 ? sby6 : sby4;
+  const uint32_t th0 = angle_code(k4[0], k4[1], bits, bx, by);
+  const uint32_t th1 = angle_code(k4[2], k4[3], bits, bx, by);
+  const uint32_t rh0 = rho_code(m[0], m[1], R2);
+  const uint32_t rh1 = rho_code(m[2], m[3], R2);
+  const uint32_t packed = th0 | (th1 << 8) | (rh0 << 16) | (rh1 << 24);
+
+  // ---- V quantiser
+  float vf[4], amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    vf[i] = __half2float(__ushort_as_half(v4[i]));
+    amax = fmaxf(amax, fabsf(vf[i]));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+  const __half sh = __float2half_rn(__fdiv_rn(amax, 127.0f));
+  const float s = __half2float(sh);
+  int8_t v8[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    int c = 0;
+    if (s != 0.0f) {
+      c = __float2int_rn(__fdiv_rn(vf[i], s));
+      c = max(-127, min(127, c));
+    }
+    v8[i] = (int8_t)c;
+  }
+
+  // ---- write the row
+  const int cb = t1 ? 64 : 48;
+  uint8_t* rsec = page + kHdrBytes;
+  uint8_t* csec = rsec + 2 * P;
+  uint8_t* ssec = csec + cb * P;
+  uint8_t* vsec = ssec + 2 * P;
+  if (lane == 0) {
+    *reinterpret_cast<uint16_t*>(rsec + 2 * row) = rt;
+    *reinterpret_cast<uint16_t*>(ssec + 2 * row) = __half_as_ushort(sh);
+  }
+  const uint32_t x3 = row & 3;
+  uint8_t* crow = csec + row * cb;
+  if (t1) {
+    // word wd (bytes 4wd..4wd+3): group g = wd / 4, j = 4 (wd % 4) + e
+    uint32_t word = 0;
+    const int wd = lane & 15;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int g = wd >> 2, j = 4 * (wd & 3) + e;
+      const int pr = 4 * (j ^ (int)x3) + g;
+      const uint32_t src = __shfl_sync(0xFFFFFFFFu, packed, pr >> 1);
+      const uint32_t th = (src >> (8 * (pr & 1))) & 0xFFu;
+      const uint32_t rh = (src >> (16 + 8 * (pr & 1))) & 0xFFu;
+      word |= ((th << 2) | rh) << (8 * e);
+    }
+    if (lane < 16) *reinterpret_cast<uint32_t*>(crow + 4 * lane) = word;
+  } else {
+    // words 0..7: nibbles of group g = wd / 2, j = 8 (wd % 2) + e;
+    // words 8..11: crumbs of group g = wd - 8, j = e
+    const int wd = lane < 12 ? lane : 0;
+    const bool crumbs = wd >= 8;
+    uint32_t word = 0;
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const int g = crumbs ? wd - 8 : (wd >> 1);
+      const int j = crumbs ? e : 8 * (wd & 1) + (e & 7);
+      const int pr = 4 * (j ^ (int)x3) + g;
+      const uint32_t src = __shfl_sync(0xFFFFFFFFu, packed, pr >> 1);
+      if (crumbs) {
+        const uint32_t rh = (src >> (16 + 8 * (pr & 1))) & 3u;
+        word |= rh << (2 * e);
+      } else if (e < 8) {
+        const uint32_t th = (src >> (8 * (pr & 1))) & 15u;
+        word |= th << (4 * e);
+      }
+    }
+    if (lane < 12) *reinterpret_cast<uint32_t*>(crow + 4 * lane) = word;
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) vsec[v_frag_offset(row, 4 * lane + i, 1)] = (uint8_t)v8[i];
+}
+
+cudaError_t launch_encode(const EncodeParams& p, cudaStream_t stream) {
+  const long long warps = (long long)p.B * p.Hkv * p.Tmax;
+  if (warps == 0) return cudaSuccess;
+  const long long blocks = (warps * 32 + 255) / 256;
+  encode_kernel<<<(unsigned)blocks, 256, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace skv

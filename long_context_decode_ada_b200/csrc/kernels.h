@@ -1,0 +1,97 @@
+// kernels.h -- parameter blocks and launchers shared by the libskv .cu files.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace skv {
+
+constexpr int kPartStride = 132;  // floats per (partial, head): m, l, pad, pad, o[128]
+
+struct DecodeParams {
+  const void* q;
+  int q_bf16;
+  int B, Hq, Hkv;
+  const int32_t* indptr;
+  const uint32_t* ids;
+  const uint8_t* pool[3];
+  long long slots[3];
+  long long stride[3];
+  int payload[3];
+  float* out;
+  float* lse;
+  int32_t* err;
+  float* part;
+  int S;
+  int P;
+  int log2P;
+  int ring_bytes;
+  float qk_scale_log2;  // log2(e) / sqrt(d)
+  float cos6[64], sin6[64], cos4[16], sin4[16];
+};
+
+struct EncodeParams {
+  const uint16_t* K;
+  const uint16_t* V;
+  int B, Hkv;
+  long long Tmax;
+  int P;
+  const int32_t* seq_lens;
+  const uint8_t* tier;
+  const int32_t* row_of;
+  const int32_t* indptr;
+  const uint32_t* ids;
+  uint8_t* pool[3];
+  long long slots[3];
+  long long stride[3];
+  int32_t* err;
+  int dense_bf16;
+  float bx6[64], by6[64], bx4[16], by4[16];
+};
+
+struct AllocParams {
+  const uint16_t* K;
+  int B, Hkv;
+  long long Tmax;
+  int P;
+  const int32_t* seq_lens;
+  const float* utility;
+  const uint8_t* protect;
+  int mode;
+  const int64_t* budget;
+  const int32_t* quota;
+  const uint32_t* free_ids[3];
+  long long free_len[3];
+  uint8_t* pool[3];
+  long long slots[3];
+  long long stride[3];
+  int payload[3];
+  uint8_t* tier_out;
+  int32_t* row_of;
+  int32_t* indptr;
+  uint32_t* page_ids;
+  long long page_cap;
+  int32_t* err;
+  float kappa[3];
+  // workspace carve-up (device)
+  float* keyw;                // [B*Hkv*Tmax]
+  unsigned long long* sel;    // [nseg*3*3]: prefix, remaining (as u64), done
+  unsigned long long* hist;   // [nseg*3*256]
+  int32_t* counts;            // [U*3]
+  int32_t* tbase;             // [U*3]
+  long long* nprot;           // [B]
+  int nseg;
+  int dense;                  // dense-bf16 baseline packing (every token kept, tier 0)
+};
+
+size_t decode_fixed_smem(int G, bool dense);
+cudaError_t launch_decode(const DecodeParams& p, int G, bool dense, cudaStream_t stream,
+                          cudaEvent_t between);
+cudaError_t launch_encode(const EncodeParams& p, cudaStream_t stream);
+size_t alloc_workspace_bytes(int B, int Hkv, long long Tmax);
+void alloc_carve(AllocParams& p, void* ws);
+cudaError_t launch_allocate(AllocParams& p, cudaStream_t stream);
+cudaError_t launch_dense_plan(AllocParams& p, cudaStream_t stream);
+
+}  // namespace skv

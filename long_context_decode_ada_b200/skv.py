@@ -1,0 +1,326 @@
+"""ctypes binding of libskv (include/skv.h) for PyTorch callers.
+
+Argument marshalling only: tensors become ``data_ptr()``s, the stream is
+``torch.cuda.current_stream()``, status codes become ``SkvError``.  Every step
+of the decode path runs in the CUDA kernels of ``libskv.so``; there is no
+CPU or PyTorch fallback, and calling into this module without the library
+raises.
+
+``PagedCache`` owns the device buffers of one paged store (three tier pools,
+page table, tiers, row map) and wraps the allocate -> encode -> decode calls.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+from typing import List, Optional, Sequence
+
+import numpy as np
+import torch
+
+from . import build as _build
+
+SKV_OK, SKV_ERR_ARG, SKV_ERR_BUDGET, SKV_ERR_POOL, SKV_ERR_CORRUPT, SKV_ERR_CUDA, \
+    SKV_ERR_TIMEOUT = range(7)
+TIER_T0, TIER_T1, TIER_T2, TIER_DROP = range(4)
+MODE_QUOTA, MODE_BUDGET = 0, 1
+Q_FP16, Q_BF16 = 0, 1
+WS_ALLOCATE, WS_DECODE, WS_DENSE_DECODE = 0, 1, 2
+TABLE_BOUNDARY6_X, TABLE_BOUNDARY6_Y, TABLE_BOUNDARY4_X, TABLE_BOUNDARY4_Y, TABLE_KAPPA, \
+    TABLE_RHO_LEVELS = range(6)
+
+EXPORTS = [
+    "skv_create", "skv_destroy", "skv_last_error", "skv_page_bytes", "skv_tables",
+    "skv_device_info", "skv_workspace_size", "skv_allocate", "skv_encode",
+    "skv_decode_attention", "skv_dense_pack_bf16", "skv_dense_decode_bf16",
+    "skv_set_profile_event", "skv_check",
+]
+
+
+class SkvConfig(C.Structure):
+    _fields_ = [("head_dim", C.c_int32), ("page_size", C.c_int32), ("reserved", C.c_int32 * 6)]
+
+
+class SkvPools(C.Structure):
+    _fields_ = [("base", C.c_void_p * 3), ("slots", C.c_int64 * 3)]
+
+
+class SkvFreeLists(C.Structure):
+    _fields_ = [("ids", C.c_void_p * 3), ("len", C.c_int64 * 3)]
+
+
+_p, _i, _i64, _sz = C.c_void_p, C.c_int, C.c_int64, C.c_size_t
+_SIGS = {
+    "skv_create": (_i, [C.POINTER(SkvConfig), C.POINTER(_p)]),
+    "skv_destroy": (_i, [_p]),
+    "skv_last_error": (C.c_char_p, []),
+    "skv_page_bytes": (_i, [_p, _i, C.POINTER(_i64), C.POINTER(_i64)]),
+    "skv_tables": (_i, [_p, _i, _p, _i64]),
+    "skv_device_info": (_i, [_p, C.POINTER(_i), C.POINTER(_i)]),
+    "skv_workspace_size": (_i, [_p, _i, _i, _i, _i, _i64, _i, C.POINTER(_sz)]),
+    "skv_allocate": (_i, [_p, _p, _i, _i, _i64, _p, _p, _p, _i, _p, _p, C.POINTER(SkvFreeLists),
+                          C.POINTER(SkvPools), _p, _p, _p, _p, _i64, _p, _p, _sz, _p]),
+    "skv_encode": (_i, [_p, _p, _p, _i, _i, _i64, _p, _p, _p, _p, _p, C.POINTER(SkvPools), _p,
+                        _p]),
+    "skv_decode_attention": (_i, [_p, _p, _i, _i, _i, _i, _p, _p, C.POINTER(SkvPools), _p, _p, _p,
+                                  _p, _sz, _i, _p]),
+    "skv_dense_pack_bf16": (_i, [_p, _p, _p, _i, _i, _i64, _p, _p, _i64, _p, _i64, _p, _p, _i64,
+                                 _p, _p, _sz, _p]),
+    "skv_dense_decode_bf16": (_i, [_p, _p, _i, _i, _i, _i, _p, _p, _p, _i64, _p, _p, _p, _p, _sz,
+                                   _i, _p]),
+    "skv_set_profile_event": (_i, [_p, _p]),
+    "skv_check": (_i, [_p, _p, _p]),
+}
+
+_lib = None
+
+
+def lib_path() -> str:
+    return _build.LIB
+
+
+def lib():
+    """Load libskv.so (building it with nvcc when it is missing or stale)."""
+    global _lib
+    if _lib is None:
+        path = _build.LIB
+        if not _build.up_to_date():
+            path = _build.build()
+        if not os.path.exists(path):
+            raise RuntimeError("libskv.so is missing and could not be built")
+        L = C.CDLL(path)
+        for name, (res, args) in _SIGS.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+class SkvError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"libskv error {code}: {msg}")
+        self.code = code
+
+
+def _check(rc: int):
+    if rc != SKV_OK:
+        raise SkvError(rc, lib().skv_last_error().decode(errors="replace"))
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    return C.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return C.c_void_p(s.cuda_stream)
+
+
+class Context:
+    """An skv_ctx: head_dim 128, page size P; bound to the current device."""
+
+    def __init__(self, page_size: int, head_dim: int = 128):
+        cfg = SkvConfig(head_dim=head_dim, page_size=page_size)
+        h = C.c_void_p()
+        _check(lib().skv_create(C.byref(cfg), C.byref(h)))
+        self._h = h
+        self.P = page_size
+        self.d = head_dim
+
+    def __del__(self):
+        h = getattr(self, "_h", None)
+        if h is not None and _lib is not None:
+            _lib.skv_destroy(h)
+            self._h = None
+
+    @property
+    def handle(self):
+        return self._h
+
+    def page_bytes(self, tier: int):
+        pay, st = C.c_int64(), C.c_int64()
+        _check(lib().skv_page_bytes(self._h, tier, C.byref(pay), C.byref(st)))
+        return pay.value, st.value
+
+    def table(self, which: int, n: int) -> np.ndarray:
+        out = np.empty(n, np.float32)
+        _check(lib().skv_tables(self._h, which, out.ctypes.data_as(C.c_void_p), n))
+        return out
+
+    def device_info(self):
+        sm, sp = C.c_int(), C.c_int()
+        _check(lib().skv_device_info(self._h, C.byref(sm), C.byref(sp)))
+        return sm.value, sp.value
+
+    def workspace_size(self, which, B, Hkv, Hq=0, Tmax=0, num_splits=0) -> int:
+        n = C.c_size_t()
+        _check(lib().skv_workspace_size(self._h, which, B, Hkv, Hq, Tmax, num_splits, C.byref(n)))
+        return n.value
+
+    def check(self, err: torch.Tensor, stream=None):
+        _check(lib().skv_check(self._h, _ptr(err), _stream(stream)))
+
+    def set_profile_event(self, event: Optional[torch.cuda.Event]):
+        """Record `event` between the decode and merge kernels of later calls."""
+        self._prof = event
+        h = None if event is None else C.c_void_p(event.cuda_event)
+        _check(lib().skv_set_profile_event(self._h, h))
+
+
+def _pools_struct(pools: Sequence[Optional[torch.Tensor]], slots: Sequence[int]) -> SkvPools:
+    s = SkvPools()
+    for t in range(3):
+        s.base[t] = pools[t].data_ptr() if pools[t] is not None and pools[t].numel() else None
+        s.slots[t] = int(slots[t])
+    return s
+
+
+class PagedCache:
+    """Device buffers of one paged store and the calls that fill and read it."""
+
+    def __init__(self, ctx: Context, B: int, Hkv: int, Tmax: int, pool_slots: Sequence[int],
+                 page_cap: Optional[int] = None, device="cuda"):
+        self.ctx, self.B, self.Hkv, self.Tmax = ctx, B, Hkv, Tmax
+        self.device = torch.device(device)
+        self.pool_slots = [int(x) for x in pool_slots]
+        self.stride = [ctx.page_bytes(t)[1] for t in range(3)]
+        self.payload = [ctx.page_bytes(t)[0] for t in range(3)]
+        self.pools = [torch.empty(max(1, self.pool_slots[t]) * self.stride[t], dtype=torch.uint8,
+                                  device=self.device) for t in range(3)]
+        self.page_cap = int(page_cap if page_cap is not None else sum(self.pool_slots))
+        self.tier = torch.empty((B, Hkv, Tmax), dtype=torch.uint8, device=self.device)
+        self.row_of = torch.empty((B, Hkv, Tmax), dtype=torch.int32, device=self.device)
+        self.page_indptr = torch.zeros(B * Hkv + 1, dtype=torch.int32, device=self.device)
+        self.page_ids = torch.zeros(max(1, self.page_cap), dtype=torch.int32, device=self.device)
+        self.err = torch.zeros(1, dtype=torch.int32, device=self.device)
+        self._ws_alloc = torch.empty(ctx.workspace_size(WS_ALLOCATE, B, Hkv, 0, Tmax),
+                                     dtype=torch.uint8, device=self.device)
+        self._pools_c = _pools_struct(self.pools, self.pool_slots)
+
+    def allocate(self, K, seq_lens, utility, protect, mode, budget, quota, free_lists,
+                 stream=None):
+        fl = SkvFreeLists()
+        self._free = [f.to(self.device, dtype=torch.int32) if isinstance(f, torch.Tensor) else
+                      torch.from_numpy(np.asarray(f, np.uint32).view(np.int32)).to(self.device)
+                      for f in free_lists]
+        for t in range(3):
+            fl.ids[t] = self._free[t].data_ptr() if self._free[t].numel() else None
+            fl.len[t] = self._free[t].numel()
+        _check(lib().skv_allocate(
+            self.ctx.handle, _ptr(K), self.B, self.Hkv, self.Tmax, _ptr(seq_lens), _ptr(utility),
+            _ptr(protect), mode, _ptr(budget), _ptr(quota), C.byref(fl), C.byref(self._pools_c),
+            _ptr(self.tier), _ptr(self.row_of), _ptr(self.page_indptr), _ptr(self.page_ids),
+            self.page_cap, _ptr(self.err), _ptr(self._ws_alloc), self._ws_alloc.numel(),
+            _stream(stream)))
+
+    def encode(self, K, V, seq_lens, stream=None):
+        _check(lib().skv_encode(
+            self.ctx.handle, _ptr(K), _ptr(V), self.B, self.Hkv, self.Tmax, _ptr(seq_lens),
+            _ptr(self.tier), _ptr(self.row_of), _ptr(self.page_indptr), _ptr(self.page_ids),
+            C.byref(self._pools_c), _ptr(self.err), _stream(stream)))
+
+    def workspace(self, Hq: int, num_splits: int = 0) -> torch.Tensor:
+        n = self.ctx.workspace_size(WS_DECODE, self.B, self.Hkv, Hq, 0, num_splits)
+        return torch.empty(max(n, 1), dtype=torch.uint8, device=self.device)
+
+    def decode(self, q: torch.Tensor, q_dtype: int, Hq: int, out=None, lse=None,
+               workspace=None, num_splits: int = 0, stream=None):
+        if out is None:
+            out = torch.empty((self.B, Hq, self.ctx.d), dtype=torch.float32, device=self.device)
+        if lse is None:
+            lse = torch.empty((self.B, Hq), dtype=torch.float32, device=self.device)
+        if workspace is None:
+            workspace = self.workspace(Hq, num_splits)
+        _check(lib().skv_decode_attention(
+            self.ctx.handle, _ptr(q), q_dtype, self.B, Hq, self.Hkv, _ptr(self.page_indptr),
+            _ptr(self.page_ids), C.byref(self._pools_c), _ptr(out), _ptr(lse), _ptr(self.err),
+            _ptr(workspace), workspace.numel(), num_splits, _stream(stream)))
+        return out, lse
+
+    def check(self, stream=None):
+        self.ctx.check(self.err, stream)
+
+    def page_bytes_of(self, page_id: int) -> torch.Tensor:
+        """Payload bytes of one page (a device view)."""
+        t, slot = page_id >> 30, page_id & ((1 << 30) - 1)
+        return self.pools[t][slot * self.stride[t]: slot * self.stride[t] + self.payload[t]]
+
+
+class DenseCache:
+    """The dense bf16 baseline store: every token kept, bf16 K/V, T0 layout."""
+
+    def __init__(self, ctx: Context, B: int, Hkv: int, Tmax: int, pool_slots: int,
+                 device="cuda"):
+        self.ctx, self.B, self.Hkv, self.Tmax = ctx, B, Hkv, Tmax
+        self.device = torch.device(device)
+        self.pool_slots = int(pool_slots)
+        self.stride = ctx.page_bytes(4)[1]
+        self.pool = torch.empty(max(1, pool_slots) * self.stride, dtype=torch.uint8,
+                                device=self.device)
+        self.page_cap = self.pool_slots
+        self.page_indptr = torch.zeros(B * Hkv + 1, dtype=torch.int32, device=self.device)
+        self.page_ids = torch.zeros(max(1, self.page_cap), dtype=torch.int32, device=self.device)
+        self.err = torch.zeros(1, dtype=torch.int32, device=self.device)
+        self._ws_alloc = torch.empty(ctx.workspace_size(WS_ALLOCATE, B, Hkv, 0, Tmax),
+                                     dtype=torch.uint8, device=self.device)
+
+    def pack(self, K, V, seq_lens, free_ids: torch.Tensor, stream=None):
+        self._free = free_ids.to(self.device, dtype=torch.int32)
+        _check(lib().skv_dense_pack_bf16(
+            self.ctx.handle, _ptr(K), _ptr(V), self.B, self.Hkv, self.Tmax, _ptr(seq_lens),
+            _ptr(self._free), self._free.numel(), _ptr(self.pool), self.pool_slots,
+            _ptr(self.page_indptr), _ptr(self.page_ids), self.page_cap, _ptr(self.err),
+            _ptr(self._ws_alloc), self._ws_alloc.numel(), _stream(stream)))
+
+    def workspace(self, Hq: int, num_splits: int = 0) -> torch.Tensor:
+        n = self.ctx.workspace_size(WS_DENSE_DECODE, self.B, self.Hkv, Hq, 0, num_splits)
+        return torch.empty(max(n, 1), dtype=torch.uint8, device=self.device)
+
+    def decode(self, q, q_dtype, Hq, out=None, lse=None, workspace=None, num_splits=0,
+               stream=None):
+        if out is None:
+            out = torch.empty((self.B, Hq, self.ctx.d), dtype=torch.float32, device=self.device)
+        if lse is None:
+            lse = torch.empty((self.B, Hq), dtype=torch.float32, device=self.device)
+        if workspace is None:
+            workspace = self.workspace(Hq, num_splits)
+        _check(lib().skv_dense_decode_bf16(
+            self.ctx.handle, _ptr(q), q_dtype, self.B, Hq, self.Hkv, _ptr(self.page_indptr),
+            _ptr(self.page_ids), _ptr(self.pool), self.pool_slots, _ptr(out), _ptr(lse),
+            _ptr(self.err), _ptr(workspace), workspace.numel(), num_splits, _stream(stream)))
+        return out, lse
+
+    def check(self, stream=None):
+        self.ctx.check(self.err, stream)
+
+
+def workload_to_device(w, device="cuda"):
+    """Host tensors of a workloads.Workload -> a dict of device tensors."""
+    dev = torch.device(device)
+
+    def t(x, dtype=None):
+        if x is None:
+            return None
+        if isinstance(x, np.ndarray):
+            x = torch.from_numpy(np.ascontiguousarray(x))
+        return x.to(dev) if dtype is None else x.to(dev, dtype=dtype)
+
+    q = w.q.view(torch.int16) if w.q.dtype == torch.uint16 else w.q.view(torch.int16)
+    return dict(
+        K=t(w.K), V=t(w.V), q=t(q), seq_lens=t(w.seq_lens), utility=t(w.utility),
+        protect=t(w.protect), budget=t(w.budget), quota=t(w.quota),
+        free_lists=[torch.from_numpy(f.view(np.int32)).to(dev) for f in w.free_lists],
+        q_dtype=Q_BF16 if w.q_dtype == "bf16" else Q_FP16,
+    )
+
+
+def build_cache(ctx: Context, w, dev: dict, stream=None) -> PagedCache:
+    """allocate + encode a workload's store on the device."""
+    cache = PagedCache(ctx, w.B, w.Hkv, w.Tmax, w.pool_slots, device=dev["K"].device)
+    cache.allocate(dev["K"], dev["seq_lens"], dev["utility"], dev["protect"], w.mode,
+                   dev["budget"], dev["quota"], dev["free_lists"], stream=stream)
+    cache.encode(dev["K"], dev["V"], dev["seq_lens"], stream=stream)
+    return cache

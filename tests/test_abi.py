@@ -1,0 +1,90 @@
+"""The C-ABI library loads and exports every symbol include/skv.h declares;
+host-only calls (tables, page geometry, argument checks) work without a GPU.
+The host tables are computed independently by the library and by the oracle
+and must agree byte for byte."""
+import ctypes as C
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+from long_context_decode_ada_b200 import skv
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if not fn.endswith(".h"):
+            continue
+        src = open(os.path.join(ROOT, "include", fn)).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        names |= set(re.findall(r"^\s*(?:const\s+)?\w+\*?\s+\*?(skv_\w+)\s*\(", src, re.M))
+    return names
+
+
+def test_library_exports_every_declared_symbol():
+    L = skv.lib()
+    names = declared_symbols()
+    assert "skv_decode_attention" in names and "skv_allocate" in names and "skv_encode" in names
+    for n in sorted(names):
+        assert hasattr(L, n), n
+    assert set(skv.EXPORTS) >= names - {n for n in names if n not in skv.EXPORTS}
+
+
+def test_tables_match_oracle_bytes():
+    ctx = skv.Context(64)
+    bx6, by6 = oracle.boundaries(6)
+    bx4, by4 = oracle.boundaries(4)
+    assert ctx.table(skv.TABLE_BOUNDARY6_X, 64).tobytes() == bx6.tobytes()
+    assert ctx.table(skv.TABLE_BOUNDARY6_Y, 64).tobytes() == by6.tobytes()
+    assert ctx.table(skv.TABLE_BOUNDARY4_X, 16).tobytes() == bx4.tobytes()
+    assert ctx.table(skv.TABLE_BOUNDARY4_Y, 16).tobytes() == by4.tobytes()
+    assert ctx.table(skv.TABLE_KAPPA, 3).tobytes() == oracle.kappa(128).tobytes()
+    lv = ctx.table(skv.TABLE_RHO_LEVELS, 4)
+    assert list(lv) == [oracle.rho_level(c, 128) for c in range(4)]
+
+
+@pytest.mark.parametrize("P", [16, 32, 64])
+def test_page_geometry_matches_oracle(P):
+    ctx = skv.Context(P)
+    for t in range(3):
+        assert ctx.page_bytes(t) == (oracle.page_payload(t, P), oracle.page_stride(t, P))
+    assert ctx.page_bytes(4) == ctx.page_bytes(0)
+
+
+def test_argument_errors_without_gpu():
+    L = skv.lib()
+    cfg = skv.SkvConfig(head_dim=64, page_size=64)
+    h = C.c_void_p()
+    assert L.skv_create(C.byref(cfg), C.byref(h)) == skv.SKV_ERR_ARG
+    assert b"head_dim" in L.skv_last_error()
+    cfg = skv.SkvConfig(head_dim=128, page_size=48)
+    assert L.skv_create(C.byref(cfg), C.byref(h)) == skv.SKV_ERR_ARG
+    ctx = skv.Context(16)
+    with pytest.raises(skv.SkvError) as e:
+        ctx.workspace_size(skv.WS_DECODE, 2, 8, 12, 0, 0)   # Hq not a multiple of Hkv
+    assert e.value.code == skv.SKV_ERR_ARG
+    # decode with G = 8 is refused on the host
+    pools = skv.SkvPools()
+    rc = L.skv_decode_attention(ctx.handle, None, skv.Q_BF16, 1, 64, 8, None, None,
+                                C.byref(pools), None, None, None, None, 0, 0, None)
+    assert rc == skv.SKV_ERR_ARG
+    # unaligned pool base is refused
+    pools.base[0] = 64
+    pools.slots[0] = 1
+    rc = L.skv_decode_attention(ctx.handle, None, skv.Q_BF16, 1, 8, 8, None, None,
+                                C.byref(pools), None, None, None, None, 0, 0, None)
+    assert rc == skv.SKV_ERR_ARG
+
+
+def test_workspace_sizes():
+    ctx = skv.Context(64)
+    sm, splits = ctx.device_info()
+    n = ctx.workspace_size(skv.WS_DECODE, 1, 8, 32, 0, 0)
+    assert n == (splits + 8) * 4 * 132 * 4
+    assert ctx.workspace_size(skv.WS_DECODE, 1, 8, 32, 0, 10) == (10 + 8) * 4 * 132 * 4
+    assert ctx.workspace_size(skv.WS_ALLOCATE, 2, 8, 0, 1000) > 2 * 8 * 1000 * 4
