@@ -175,6 +175,10 @@ def timed_graph_steps(step_fns, steps, warmup, graph_steps, stream, mid_events=N
     ev = [(torch.cuda.Event(enable_timing=True, external=True),
            torch.cuda.Event(enable_timing=True, external=True),
            torch.cuda.Event(enable_timing=True, external=True)) for _ in range(gsteps)]
+    for e3 in ev:                 # torch creates the CUDA events on first record
+        for e in e3:
+            e.record()
+    torch.cuda.synchronize()
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g):
         for i in range(gsteps):

@@ -189,7 +189,9 @@ int skv_workspace_size(const skv_ctx* ctx, int which, int B, int Hkv, int Hq, in
     if (Hq <= 0 || Hq % Hkv != 0) return fail(SKV_ERR_ARG, "Hq must be a multiple of Hkv");
     const int G = Hq / Hkv;
     const long long S = decode_splits(ctx, num_splits);
-    *bytes = (size_t)(S + (long long)B * Hkv) * G * skv::kPartStride * sizeof(float);
+    // split partials, then one ticket counter per unit
+    *bytes = (size_t)(S + (long long)B * Hkv) * G * skv::kPartStride * sizeof(float) +
+             sizeof(int) * (size_t)B * Hkv;
     return ok();
   }
   return fail(SKV_ERR_ARG, "skv_workspace_size: unknown kind %d", which);
@@ -345,10 +347,11 @@ static int decode_common(skv_ctx* ctx, const void* q, int q_dtype, int B, int Hq
   p.P = ctx->P;
   p.log2P = ctx->log2P;
   const size_t fixed = skv::decode_fixed_smem(G, dense);
-  long long ring = ((long long)ctx->smem_optin - (long long)fixed) / 128 * 128;
-  const long long max_item = 64LL * 512 + 4 * skv::kHdrBytes;
-  if (ring < max_item) return fail(SKV_ERR_ARG, "%s: not enough shared memory", name);
-  p.ring_bytes = (int)std::min<long long>(ring, 1 << 20);
+  const long long luts = dense ? 0 : 80LL * 256 * G;   // 6-bit + 4-bit fp32 LUTs
+  const long long max_item = 128LL * 512 + 8 * skv::kHdrBytes;
+  if ((long long)ctx->smem_optin < (long long)fixed + luts + max_item + 65536)
+    return fail(SKV_ERR_ARG, "%s: not enough shared memory per block", name);
+  p.smem_bytes = (int)ctx->smem_optin;
   p.qk_scale_log2 = (float)(1.4426950408889634 / std::sqrt(128.0));
   std::memcpy(p.cos6, ctx->cos6, sizeof(p.cos6));
   std::memcpy(p.sin6, ctx->sin6, sizeof(p.sin6));

@@ -2,8 +2,8 @@
 //
 // Everything here is hand-written for Blackwell: mbarrier-tracked bulk
 // asynchronous copies (cp.async.bulk, no multicast), legacy-form mma.sync
-// for the small P.V contraction, mixed-precision fma (f16 x f16 + f32),
-// exact integer / IEEE-rounded conversions for the bit-exact encode.
+// for the small P.V contraction, exact integer / IEEE-rounded conversions
+// for the bit-exact encode.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -104,19 +104,6 @@ __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
 // arithmetic helpers
 // ---------------------------------------------------------------------------
 
-// f32 = f16 * f16 + f32 in one rounding (the product of two halves is exact).
-__device__ __forceinline__ float fma_f16f16f32(uint16_t a, uint16_t b, float c) {
-  float d;
-  asm("fma.rn.f32.f16 %0, %1, %2, %3;" : "=f"(d) : "h"(a), "h"(b), "f"(c));
-  return d;
-}
-
-__device__ __forceinline__ float fma_bf16bf16f32(uint16_t a, uint16_t b, float c) {
-  float d;
-  asm("fma.rn.f32.bf16 %0, %1, %2, %3;" : "=f"(d) : "h"(a), "h"(b), "f"(c));
-  return d;
-}
-
 // Four signed int8 (one 32-bit word, byte i = element i) -> two f16x2:
 // lo = (e0, e1), hi = (e2, e3).  Exact: 0x64XX is 1024 + XX in fp16, with
 // XX = e + 128, and 1152 = 1024 + 128 is subtracted.
@@ -156,6 +143,25 @@ __device__ __forceinline__ void mma_16816_bf16(float* d, uint32_t a0, uint32_t a
       "{%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a0), "r"(a1), "r"(b));
+}
+
+// D += A * B, m16n8k16 (A: 4 x f16x2, B: 2 x f16x2), f32 accumulation.
+__device__ __forceinline__ void mma_16816k16_f16(float* d, uint32_t a0, uint32_t a1, uint32_t a2,
+                                                 uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void mma_16816k16_bf16(float* d, uint32_t a0, uint32_t a1, uint32_t a2,
+                                                  uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
 // Unsigned 128-bit integer to double, correctly rounded (nearest-even): keep

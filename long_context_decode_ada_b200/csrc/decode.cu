@@ -5,30 +5,56 @@
 //
 // Work split ("split-K over pages"): the CSR page list of all units
 // (unit = (seq, kv head)) is one array of N pages; CTA c streams the run
-// [floor(c N / S), floor((c+1) N / S)) and emits one partial (m, l, o) per
-// unit it touches, at partial slot c + u.  A merge kernel combines them.
+// [floor(c N / S), floor((c+1) N / S)) and produces one partial (m, l, o)
+// per unit it touches.  A unit covered by a single run is finished in
+// place; otherwise the partial goes to slot c + u of the workspace and the
+// CTA that brings the unit's ticket counter to its run count merges them
+// (log-sum-exp) -- no CTA ever waits for another.
 //
 // CTA = 8 consumer warps + 1 producer warp.  The producer copies whole
-// pages (header included) with 1-D bulk async copies into a byte ring in
-// shared memory, 64 tokens per "item" (64/P pages), tracked by full/empty
-// mbarriers; consumer warp w takes rows [8w, 8w+8) of each item.
+// pages (header included) with 1-D bulk asynchronous copies (no multicast)
+// into a byte ring in shared memory, 128 tokens per "item" (128/P pages),
+// tracked by full/empty mbarriers; consumer warp w takes rows
+// [16w, 16w+16) of each item, i.e. 16 rows of one page.
 //
-// Consumer lane map: lane = 4 t + g, t = token of the 8-row group, g = pair
-// group.  Logits: lane (t, g) sums 16 pairs (T1/T2, LUT gathers from shared
-// memory) or 32 dims (T0) for all G query heads of the group, then a 4-lane
-// reduce-scatter leaves head g's logit in lane (t, g).  P.V: mma.sync
-// m16n8k8, A = V^T fragment read straight from the page (the page stores V
-// in fragment order), B = P (8 tokens x 8 heads, zero-padded), f32 accum.
+// Consumer lane map: lane = 4 t + g, t = token of an 8-row group, g = pair
+// group; each lane carries rows t and t + 8.  Logits: lane (t, g) sums 16
+// pairs (T1/T2: gathers from an fp32 shared-memory LUT holding all G query
+// heads of the group) or 32 dims (T0), a 4-lane reduce-scatter leaves head
+// g's logit in lane (t, g).  P.V: mma.sync m16n8k16, A = V^T fragments read
+// straight from the page (pages store V in fragment order), B = P of the 16
+// rows x 8 heads (zero-padded beyond G), fp32 accumulation.
+#include <algorithm>
+
 #include "common.cuh"
 #include "kernels.h"
 
 namespace skv {
 
-constexpr int kNCW = 8;
+#ifndef SKV_DECODE_GROUPS
+#define SKV_DECODE_GROUPS 1
+#endif
+constexpr int kGW = 8;                            // consumer warps per group (one item)
+constexpr int kGroups = SKV_DECODE_GROUPS;        // groups take items in turn
+constexpr int kNCW = kGroups * kGW;
 constexpr int kDecodeThreads = (kNCW + 1) * 32;
 constexpr int kNSlot = 16;
-constexpr int kMaxIPP = 4;
+constexpr int kMaxIPP = 8;
+constexpr int kIdBatch = 256;    // page ids staged per producer batch
+constexpr int kMergeRuns = 128;  // runs per unit merged through shared memory
 constexpr uint32_t kInvalidOff = 0xFFFFFFFFu;
+
+// Shared-memory plan: [fixed block][ring][LUT1][LUT2].  LUT1 / LUT2 start at
+// shared addresses aligned to their own size, so that a gather address is
+// (code bits) | (pair offset) | (table base) -- one shift and one LOP3.
+template <int G>
+struct LutGeom {
+  static constexpr uint32_t kEnt = 4 * G;                // bytes per entry (G fp32)
+  static constexpr uint32_t kCode = kPairs * kEnt;       // bytes per code row
+  static constexpr uint32_t kLut1 = 64 * kCode;          // 6-bit codes
+  static constexpr uint32_t kLut2 = 16 * kCode;          // 4-bit codes
+  static constexpr int kCodeShift = (G == 4) ? 10 : (G == 2 ? 9 : 8);  // log2(kCode)
+};
 
 template <int G, bool DENSE>
 struct __align__(16) DecodeSmem {
@@ -36,112 +62,175 @@ struct __align__(16) DecodeSmem {
   unsigned long long empty[kNSlot];
   uint32_t item_off[kNSlot][kMaxIPP];
   uint32_t item_np[kNSlot];
-  uint32_t item_tier[kNSlot];          // byte k = tier of page k
-  long long item_start[kNSlot];         // producer bookkeeping (ring position)
+  uint32_t item_tier[kNSlot];   // 2 bits per page
+  uint32_t item_start[kNSlot];  // producer bookkeeping (ring offset)
   int abort_flag;
-  int pad_[3];
+  int last_flag;
+  int pad_[2];
   float ml[kNCW][4][2];
   float O[4][kHeadDim];
   float q32[4][kHeadDim];
-  uint16_t q16[4][kHeadDim];            // fp16 (ADA T0) or bf16 (dense) bits
-  uint16_t lut1[DENSE ? 8 : 64 * kPairs * G];   // [code 64][pair 64][G] fp16
-  uint16_t lut2[DENSE ? 8 : 16 * kPairs * G];   // [code 16][pair 64][G] fp16
+  float mw[4][kMergeRuns];        // merge: per-run weights
+  uint32_t ids[kIdBatch + kMaxIPP];  // producer: staged page ids
 };
 
 __device__ __forceinline__ long long chunk_begin(int c, long long N, int S) {
   return (long long)c * N / S;
 }
 
-// share level (code + 1) / 16 as fp16 bits: 0x2C00, 0x3000, 0x3200, 0x3400
-__device__ __forceinline__ uint16_t rho_half(uint32_t rh) {
-  return (uint16_t)__byte_perm(0x30002C00u, 0x34003200u, rh * 0x22u + 0x10u);
+// ------------------------------------------------------ shared loads (PTX) --
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(a));
+  return v;
+}
+__device__ __forceinline__ uint2 lds64(uint32_t a) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ uint32_t lds32(uint32_t a) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ uint32_t lds16(uint32_t a) {
+  unsigned short v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(a));
+  return v;
 }
 
+// (code & 3) + 1 as a float, without a conversion instruction
+__device__ __forceinline__ float share_plus_one(uint32_t byte_or_bits) {
+  return __int_as_float(0x4B000000u | (byte_or_bits & 3u)) - 8388607.0f;
+}
+
+// G fp32 LUT entries at a shared address
 template <int G>
-__device__ __forceinline__ void lut_gather(const uint16_t* e, uint16_t rho, float (&s)[G]) {
+__device__ __forceinline__ void lut_fma(uint32_t a, float w, float (&s)[G]) {
   if constexpr (G == 4) {
-    uint2 v = *reinterpret_cast<const uint2*>(e);
-    s[0] = fma_f16f16f32(rho, (uint16_t)(v.x & 0xFFFF), s[0]);
-    s[1] = fma_f16f16f32(rho, (uint16_t)(v.x >> 16), s[1]);
-    s[2] = fma_f16f16f32(rho, (uint16_t)(v.y & 0xFFFF), s[2]);
-    s[3] = fma_f16f16f32(rho, (uint16_t)(v.y >> 16), s[3]);
+    const uint4 v = lds128(a);
+    s[0] = fmaf(w, __uint_as_float(v.x), s[0]);
+    s[1] = fmaf(w, __uint_as_float(v.y), s[1]);
+    s[2] = fmaf(w, __uint_as_float(v.z), s[2]);
+    s[3] = fmaf(w, __uint_as_float(v.w), s[3]);
   } else if constexpr (G == 2) {
-    uint32_t v = *reinterpret_cast<const uint32_t*>(e);
-    s[0] = fma_f16f16f32(rho, (uint16_t)(v & 0xFFFF), s[0]);
-    s[1] = fma_f16f16f32(rho, (uint16_t)(v >> 16), s[1]);
+    const uint2 v = lds64(a);
+    s[0] = fmaf(w, __uint_as_float(v.x), s[0]);
+    s[1] = fmaf(w, __uint_as_float(v.y), s[1]);
   } else {
-    s[0] = fma_f16f16f32(rho, *e, s[0]);
+    s[0] = fmaf(w, __uint_as_float(lds32(a)), s[0]);
   }
 }
 
-// Per-lane partial logits of token `row` for the T1 page at pg.
+// Partial logits (times 16: shares enter as code + 1) of rows rA, rA + 8 of
+// the T1 page at shared address pg.  Code byte 16g + j of a row holds pair
+// 4 (j ^ (row & 3)) + g as (angle6 << 2) | share2.
 template <int G>
-__device__ __forceinline__ void logits_t1(const uint8_t* pg, int P, int row, int g,
-                                          const uint16_t* lut1, float (&s)[G]) {
-  const uint8_t* cd = pg + kHdrBytes + 2 * P;
-  uint4 cw = *reinterpret_cast<const uint4*>(cd + row * 64 + 16 * g);
-  const uint32_t w[4] = {cw.x, cw.y, cw.z, cw.w};
-  const uint32_t x3 = row & 3;
-  // element (code th, pair 4*(j ^ x3) + g) sits at lut1 + (th*64 + pair)*G
-  const uint16_t* base = lut1 + g * G;
+__device__ __forceinline__ void logits_t1(uint32_t pg, int P, int rA, int g, uint32_t lut,
+                                          float (&sA)[G], float (&sB)[G]) {
+  const uint32_t cd = pg + kHdrBytes + 2 * P;
+  const uint4 ca = lds128(cd + rA * 64 + 16 * g);
+  const uint4 cb = lds128(cd + (rA + 8) * 64 + 16 * g);
+  const uint32_t wa[4] = {ca.x, ca.y, ca.z, ca.w};
+  const uint32_t wb[4] = {cb.x, cb.y, cb.z, cb.w};
+  const uint32_t x3 = rA & 3;  // rows rA and rA + 8 share it
+  using L = LutGeom<G>;
+  // the table base is aligned to the table size: base | pair offset | code bits
   uint32_t xo[4];
 #pragma unroll
-  for (int jj = 0; jj < 4; ++jj) xo[jj] = ((uint32_t)jj ^ x3) * 4 * G;
+  for (int jj = 0; jj < 4; ++jj) xo[jj] = lut | ((((uint32_t)jj ^ x3) * 4 + g) * L::kEnt);
+  constexpr uint32_t kMask = 0xFCu << (L::kCodeShift - 2);  // angle bits of a byte, scaled
 #pragma unroll
   for (int j = 0; j < 16; ++j) {
-    uint32_t byte = (w[j >> 2] >> (8 * (j & 3))) & 0xFFu;
-    uint32_t th = byte >> 2;
-    const uint16_t* e = base + (j & ~3) * 4 * G + xo[j & 3] + th * (kPairs * G);
-    lut_gather<G>(e, rho_half(byte & 3u), s);
+    const int sh = 8 * (j & 3) - (L::kCodeShift - 2);   // byte j sits at bit 8 (j & 3)
+    const uint32_t xa = sh >= 0 ? (wa[j >> 2] >> sh) : (wa[j >> 2] << -sh);
+    const uint32_t xb = sh >= 0 ? (wb[j >> 2] >> sh) : (wb[j >> 2] << -sh);
+    const uint32_t col = xo[j & 3] | ((j & ~3) * 4 * L::kEnt);
+    lut_fma<G>((xa & kMask) | col, share_plus_one(wa[j >> 2] >> (8 * (j & 3))), sA);
+    lut_fma<G>((xb & kMask) | col, share_plus_one(wb[j >> 2] >> (8 * (j & 3))), sB);
   }
 }
 
+// T2: nibble j of bytes [8g, 8g+8) holds the 4-bit angle of pair
+// 4 (j ^ (row & 3)) + g, crumb j of bytes [32+4g, 36+4g) its share.
 template <int G>
-__device__ __forceinline__ void logits_t2(const uint8_t* pg, int P, int row, int g,
-                                          const uint16_t* lut2, float (&s)[G]) {
-  const uint8_t* cd = pg + kHdrBytes + 2 * P + row * 48;
-  uint2 nw = *reinterpret_cast<const uint2*>(cd + 8 * g);
-  uint32_t cr = *reinterpret_cast<const uint32_t*>(cd + 32 + 4 * g);
-  const uint32_t x3 = row & 3;
-  const uint16_t* base = lut2 + g * G;
+__device__ __forceinline__ void logits_t2(uint32_t pg, int P, int rA, int g, uint32_t lut,
+                                          float (&sA)[G], float (&sB)[G]) {
+  const uint32_t cd = pg + kHdrBytes + 2 * P;
+  const uint2 na = lds64(cd + rA * 48 + 8 * g);
+  const uint2 nb = lds64(cd + (rA + 8) * 48 + 8 * g);
+  const uint32_t ra = lds32(cd + rA * 48 + 32 + 4 * g);
+  const uint32_t rb = lds32(cd + (rA + 8) * 48 + 32 + 4 * g);
+  const uint32_t x3 = rA & 3;
+  using L = LutGeom<G>;
   uint32_t xo[4];
 #pragma unroll
-  for (int jj = 0; jj < 4; ++jj) xo[jj] = ((uint32_t)jj ^ x3) * 4 * G;
+  for (int jj = 0; jj < 4; ++jj) xo[jj] = lut | ((((uint32_t)jj ^ x3) * 4 + g) * L::kEnt);
+  constexpr uint32_t kMask = 0xFu << L::kCodeShift;
 #pragma unroll
   for (int j = 0; j < 16; ++j) {
-    uint32_t word = (j < 8) ? nw.x : nw.y;
-    uint32_t th = (word >> (4 * (j & 7))) & 15u;
-    uint32_t rh = (cr >> (2 * j)) & 3u;
-    const uint16_t* e = base + (j & ~3) * 4 * G + xo[j & 3] + th * (kPairs * G);
-    lut_gather<G>(e, rho_half(rh), s);
+    const int sh = 4 * (j & 7) - L::kCodeShift;   // nibble j sits at bit 4 (j & 7)
+    const uint32_t wa = (j < 8) ? na.x : na.y, wb = (j < 8) ? nb.x : nb.y;
+    const uint32_t xa = sh >= 0 ? (wa >> sh) : (wa << -sh);
+    const uint32_t xb = sh >= 0 ? (wb >> sh) : (wb << -sh);
+    const uint32_t col = xo[j & 3] | ((j & ~3) * 4 * L::kEnt);
+    lut_fma<G>((xa & kMask) | col, share_plus_one(ra >> (2 * j)), sA);
+    lut_fma<G>((xb & kMask) | col, share_plus_one(rb >> (2 * j)), sB);
   }
+}
+
+// fp16 pair (one 32-bit word) -> two fp32 values scaled by 2^-112, exactly
+// (normal and subnormal halves): the half's exponent and mantissa bits are
+// moved into an fp32 at bit 13; the 2^112 goes into the logit scale.
+__device__ __forceinline__ void half2_bits_to_f32_scaled(uint32_t w, float& lo, float& hi) {
+  lo = __int_as_float(((int32_t)(w << 16) >> 3) & (int32_t)0x8FFFE000);
+  hi = __int_as_float(((int32_t)w >> 3) & (int32_t)0x8FFFE000);
+}
+__device__ __forceinline__ void bf162_bits_to_f32(uint32_t w, float& lo, float& hi) {
+  lo = __int_as_float(w << 16);
+  hi = __int_as_float(w & 0xFFFF0000u);
 }
 
 // T0 (fp16 K) or dense (bf16 K): lane (t, g) covers dims 8c..8c+7 for the
-// chunks c = 4i + g, stored at chunk position c ^ 4(row & 1).
+// chunks c = 4i + g, stored at chunk position c ^ 4 (row & 1).
 template <int G, bool BF16>
-__device__ __forceinline__ void logits_dense(const uint8_t* pg, int row, int g,
-                                             const uint16_t (*q16)[kHeadDim], float (&s)[G]) {
-  const uint8_t* krow = pg + kHdrBytes + row * 256;
-  const uint32_t sw = 4u * (row & 1);
+__device__ __forceinline__ void logits_dense(uint32_t pg, int rA, int g, uint32_t q32,
+                                             float (&sA)[G], float (&sB)[G]) {
+  const uint32_t ka = pg + kHdrBytes + rA * 256;
+  const uint32_t kb = ka + 8 * 256;
+  const uint32_t sw = 4u * (rA & 1);
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const uint32_t c = 4 * i + g;
-    uint4 kc = *reinterpret_cast<const uint4*>(krow + ((c ^ sw) * 16));
-    const uint32_t kw[4] = {kc.x, kc.y, kc.z, kc.w};
+    const uint4 xa = lds128(ka + (c ^ sw) * 16);
+    const uint4 xb = lds128(kb + (c ^ sw) * 16);
+    const uint32_t wa[4] = {xa.x, xa.y, xa.z, xa.w};
+    const uint32_t wb[4] = {xb.x, xb.y, xb.z, xb.w};
+    float fa[8], fb[8];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      if constexpr (BF16) {
+        bf162_bits_to_f32(wa[e], fa[2 * e], fa[2 * e + 1]);
+        bf162_bits_to_f32(wb[e], fb[2 * e], fb[2 * e + 1]);
+      } else {
+        half2_bits_to_f32_scaled(wa[e], fa[2 * e], fa[2 * e + 1]);
+        half2_bits_to_f32_scaled(wb[e], fb[2 * e], fb[2 * e + 1]);
+      }
+    }
 #pragma unroll
     for (int h = 0; h < G; ++h) {
-      uint4 qc = *reinterpret_cast<const uint4*>(&q16[h][8 * c]);
-      const uint32_t qw[4] = {qc.x, qc.y, qc.z, qc.w};
+      const uint4 q0 = lds128(q32 + (h * kHeadDim + 8 * c) * 4);
+      const uint4 q1 = lds128(q32 + (h * kHeadDim + 8 * c + 4) * 4);
+      const float qv[8] = {__uint_as_float(q0.x), __uint_as_float(q0.y), __uint_as_float(q0.z),
+                           __uint_as_float(q0.w), __uint_as_float(q1.x), __uint_as_float(q1.y),
+                           __uint_as_float(q1.z), __uint_as_float(q1.w)};
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        if constexpr (BF16) {
-          s[h] = fma_bf16bf16f32((uint16_t)(kw[e] & 0xFFFF), (uint16_t)(qw[e] & 0xFFFF), s[h]);
-          s[h] = fma_bf16bf16f32((uint16_t)(kw[e] >> 16), (uint16_t)(qw[e] >> 16), s[h]);
-        } else {
-          s[h] = fma_f16f16f32((uint16_t)(kw[e] & 0xFFFF), (uint16_t)(qw[e] & 0xFFFF), s[h]);
-          s[h] = fma_f16f16f32((uint16_t)(kw[e] >> 16), (uint16_t)(qw[e] >> 16), s[h]);
-        }
+      for (int e = 0; e < 8; ++e) {
+        sA[h] = fmaf(fa[e], qv[e], sA[h]);
+        sB[h] = fmaf(fb[e], qv[e], sB[h]);
       }
     }
   }
@@ -152,19 +241,19 @@ template <int G>
 __device__ __forceinline__ float reduce_scatter(float (&s)[G], int g) {
   if constexpr (G == 4) {
     const bool up = (g & 2) != 0;
-    float x0 = __shfl_xor_sync(0xFFFFFFFFu, up ? s[0] : s[2], 2);
-    float x1 = __shfl_xor_sync(0xFFFFFFFFu, up ? s[1] : s[3], 2);
-    float a0 = (up ? s[2] : s[0]) + x0;
-    float a1 = (up ? s[3] : s[1]) + x1;
+    const float x0 = __shfl_xor_sync(0xFFFFFFFFu, up ? s[0] : s[2], 2);
+    const float x1 = __shfl_xor_sync(0xFFFFFFFFu, up ? s[1] : s[3], 2);
+    const float a0 = (up ? s[2] : s[0]) + x0;
+    const float a1 = (up ? s[3] : s[1]) + x1;
     const bool odd = (g & 1) != 0;
-    float y = __shfl_xor_sync(0xFFFFFFFFu, odd ? a0 : a1, 1);
+    const float y = __shfl_xor_sync(0xFFFFFFFFu, odd ? a0 : a1, 1);
     return (odd ? a1 : a0) + y;
   } else if constexpr (G == 2) {
-    s[0] += __shfl_xor_sync(0xFFFFFFFFu, s[0], 2);
-    s[1] += __shfl_xor_sync(0xFFFFFFFFu, s[1], 2);
+    const float a0 = s[0] + __shfl_xor_sync(0xFFFFFFFFu, s[0], 2);
+    const float a1 = s[1] + __shfl_xor_sync(0xFFFFFFFFu, s[1], 2);
     const bool odd = (g & 1) != 0;
-    float y = __shfl_xor_sync(0xFFFFFFFFu, odd ? s[0] : s[1], 1);
-    return (odd ? s[1] : s[0]) + y;
+    const float y = __shfl_xor_sync(0xFFFFFFFFu, odd ? a0 : a1, 1);
+    return (odd ? a1 : a0) + y;
   } else {
     float a = s[0];
     a += __shfl_xor_sync(0xFFFFFFFFu, a, 2);
@@ -174,32 +263,33 @@ __device__ __forceinline__ float reduce_scatter(float (&s)[G], int g) {
 }
 
 struct WarpState {
-  float m;         // running max (log2 domain) of head g % G
-  float l;         // partial denominator of (token slot t, head g % G)
+  float m;          // running max (log2 domain) of head g % G
+  float l;          // partial denominator of (token slot t, head g % G)
   float acc[8][4];  // O^T fragments: [m-tile][c0..c3]
 };
 
-// Online softmax of one 8-token chunk and P.V into the accumulators.
-// logit: log2-domain logit of (token t, head g % G) or -inf.
-// VK: 0 int8 V (1 KB group block), 1 fp16 V (2 KB), 2 bf16 V (2 KB).
+// Online softmax of 16 rows and P.V into the accumulators.
+// lA / lB: log2-domain logits of rows t and t + 8 (head g % G) or -inf.
+// VK: 0 int8 V (1 KB per 8-row group), 1 fp16 V, 2 bf16 V (2 KB per group).
 template <int G, int VK>
-__device__ __forceinline__ void softmax_pv(float logit, float vscale, const uint8_t* vblock,
-                                           WarpState& st, int lane) {
-  float cm = logit;
+__device__ __forceinline__ void softmax_pv(float lA, float lB, float vsA, float vsB, uint32_t va,
+                                           uint32_t vb, WarpState& st, int lane) {
+  float cm = fmaxf(lA, lB);
   cm = fmaxf(cm, __shfl_xor_sync(0xFFFFFFFFu, cm, 4));
   cm = fmaxf(cm, __shfl_xor_sync(0xFFFFFFFFu, cm, 8));
   cm = fmaxf(cm, __shfl_xor_sync(0xFFFFFFFFu, cm, 16));
   const float m_new = fmaxf(st.m, cm);
   const bool fin = m_new != -INFINITY;
   const float alpha = (fin && st.m != m_new) ? exp2f(st.m - m_new) : 1.0f;
-  const float p = (logit != -INFINITY) ? exp2f(logit - m_new) : 0.0f;
-  st.l = st.l * alpha + p;
+  const float pA = (lA != -INFINITY) ? exp2f(lA - m_new) : 0.0f;
+  const float pB = (lB != -INFINITY) ? exp2f(lB - m_new) : 0.0f;
+  st.l = st.l * alpha + (pA + pB);
   st.m = m_new;
   const int gq = lane >> 2, t4 = lane & 3;
   if (__any_sync(0xFFFFFFFFu, alpha != 1.0f)) {
     const int n0 = 2 * t4, n1 = 2 * t4 + 1;
-    float a0 = __shfl_sync(0xFFFFFFFFu, alpha, n0 < G ? n0 : 0);
-    float a1 = __shfl_sync(0xFFFFFFFFu, alpha, n1 < G ? n1 : 0);
+    const float a0 = __shfl_sync(0xFFFFFFFFu, alpha, n0 < G ? n0 : 0);
+    const float a1 = __shfl_sync(0xFFFFFFFFu, alpha, n1 < G ? n1 : 0);
 #pragma unroll
     for (int mt = 0; mt < 8; ++mt) {
       st.acc[mt][0] *= a0;
@@ -208,87 +298,103 @@ __device__ __forceinline__ void softmax_pv(float logit, float vscale, const uint
       st.acc[mt][3] *= a1;
     }
   }
-  const float pp = p * vscale;
-  // B fragment: (k = tokens 2 t4, 2 t4 + 1; n = head gq), zero for gq >= G
+  const float ppA = pA * vsA, ppB = pB * vsB;
+  // B fragment (k16 x n8): k = rows 2t4, 2t4+1 | 8+2t4, 9+2t4, n = head gq
   const int src = 8 * t4 + (gq < G ? gq : 0);
-  float b0 = __shfl_sync(0xFFFFFFFFu, pp, src);
-  float b1 = __shfl_sync(0xFFFFFFFFu, pp, src + 4);
+  float b0 = __shfl_sync(0xFFFFFFFFu, ppA, src);
+  float b1 = __shfl_sync(0xFFFFFFFFu, ppA, src + 4);
+  float b2 = __shfl_sync(0xFFFFFFFFu, ppB, src);
+  float b3 = __shfl_sync(0xFFFFFFFFu, ppB, src + 4);
   if (gq >= G) {
     b0 = 0.0f;
     b1 = 0.0f;
+    b2 = 0.0f;
+    b3 = 0.0f;
   }
   if constexpr (VK == 0) {
-    const uint32_t bf = pack_f16x2(b0, b1);
-    uint4 x = *reinterpret_cast<const uint4*>(vblock + lane * 16);
-    uint4 y = *reinterpret_cast<const uint4*>(vblock + 512 + lane * 16);
-    const uint32_t vw[8] = {x.x, x.y, x.z, x.w, y.x, y.y, y.z, y.w};
+    const uint32_t bf0 = pack_f16x2(b0, b1), bf1 = pack_f16x2(b2, b3);
+    const uint4 xa = lds128(va + lane * 16), ya = lds128(va + 512 + lane * 16);
+    const uint4 xb = lds128(vb + lane * 16), yb = lds128(vb + 512 + lane * 16);
+    const uint32_t wa[8] = {xa.x, xa.y, xa.z, xa.w, ya.x, ya.y, ya.z, ya.w};
+    const uint32_t wb[8] = {xb.x, xb.y, xb.z, xb.w, yb.x, yb.y, yb.z, yb.w};
 #pragma unroll
     for (int mt = 0; mt < 8; ++mt) {
-      uint32_t a0, a1;
-      s8x4_to_f16x2x2(vw[mt], a0, a1);
-      mma_16816_f16(st.acc[mt], a0, a1, bf);
+      uint32_t a0, a1, a2, a3;
+      s8x4_to_f16x2x2(wa[mt], a0, a1);
+      s8x4_to_f16x2x2(wb[mt], a2, a3);
+      mma_16816k16_f16(st.acc[mt], a0, a1, a2, a3, bf0, bf1);
     }
   } else {
-    const uint32_t bf = (VK == 1) ? pack_f16x2(b0, b1) : pack_bf16x2(b0, b1);
+    const uint32_t bf0 = (VK == 1) ? pack_f16x2(b0, b1) : pack_bf16x2(b0, b1);
+    const uint32_t bf1 = (VK == 1) ? pack_f16x2(b2, b3) : pack_bf16x2(b2, b3);
 #pragma unroll
     for (int qq = 0; qq < 4; ++qq) {
-      uint4 z = *reinterpret_cast<const uint4*>(vblock + qq * 512 + lane * 16);
+      const uint4 za = lds128(va + qq * 512 + lane * 16);
+      const uint4 zb = lds128(vb + qq * 512 + lane * 16);
       if constexpr (VK == 1) {
-        mma_16816_f16(st.acc[2 * qq], z.x, z.y, bf);
-        mma_16816_f16(st.acc[2 * qq + 1], z.z, z.w, bf);
+        mma_16816k16_f16(st.acc[2 * qq], za.x, za.y, zb.x, zb.y, bf0, bf1);
+        mma_16816k16_f16(st.acc[2 * qq + 1], za.z, za.w, zb.z, zb.w, bf0, bf1);
       } else {
-        mma_16816_bf16(st.acc[2 * qq], z.x, z.y, bf);
-        mma_16816_bf16(st.acc[2 * qq + 1], z.z, z.w, bf);
+        mma_16816k16_bf16(st.acc[2 * qq], za.x, za.y, zb.x, zb.y, bf0, bf1);
+        mma_16816k16_bf16(st.acc[2 * qq + 1], za.z, za.w, zb.z, zb.w, bf0, bf1);
       }
     }
   }
 }
 
+// 16 rows [row0, row0 + 16) of one page at shared address pg.
 template <int G, bool DENSE>
-__device__ __forceinline__ void process_rows(const DecodeParams& p, DecodeSmem<G, DENSE>& sm,
-                                             const uint8_t* pg, uint32_t tier, int row0,
-                                             WarpState& st, int lane) {
+__device__ __forceinline__ void process_rows(const DecodeParams& p, uint32_t pg, uint32_t tier,
+                                             int row0, uint32_t lut1, uint32_t lut2,
+                                             uint32_t q32, WarpState& st, int lane) {
   const int t = lane >> 2, g = lane & 3;
   const int P = p.P;
-  const uint32_t cnt = *reinterpret_cast<const uint16_t*>(pg);
-  const uint32_t htier = pg[2];
-  const uint32_t magic = pg[3];
+  const uint32_t h0 = lds32(pg);
+  const uint32_t cnt = h0 & 0xFFFFu, htier = (h0 >> 16) & 0xFFu, magic = h0 >> 24;
   if (htier != tier || magic != kPageMagic || cnt > (uint32_t)P) {
     if (lane == 0) report(p.err, SKV_ERR_CORRUPT);
     return;
   }
   if ((uint32_t)row0 >= cnt) return;
-  const int row = row0 + t;
-  const bool valid = (uint32_t)row < cnt;
-  float s[G];
+  const int rA = row0 + t, rB = rA + 8;
+  const bool vA = (uint32_t)rA < cnt, vB = (uint32_t)rB < cnt;
+  float sA[G], sB[G];
 #pragma unroll
-  for (int h = 0; h < G; ++h) s[h] = 0.0f;
+  for (int h = 0; h < G; ++h) {
+    sA[h] = 0.0f;
+    sB[h] = 0.0f;
+  }
+  const uint32_t vsec_dense = pg + kHdrBytes + 256 * P + (row0 >> 3) * 2048;
   if constexpr (DENSE) {
-    logits_dense<G, true>(pg, row, g, sm.q16, s);
-    float r = reduce_scatter<G>(s, g);
-    float logit = valid ? r * p.qk_scale_log2 : -INFINITY;
-    softmax_pv<G, 2>(logit, 1.0f, pg + kHdrBytes + 256 * P + (row0 >> 3) * 2048, st, lane);
+    logits_dense<G, true>(pg, rA, g, q32, sA, sB);
+    const float a = reduce_scatter<G>(sA, g), b = reduce_scatter<G>(sB, g);
+    const float c = p.qk_scale_log2;
+    softmax_pv<G, 2>(vA ? a * c : -INFINITY, vB ? b * c : -INFINITY, 1.0f, 1.0f, vsec_dense,
+                     vsec_dense + 2048, st, lane);
   } else {
     if (tier == SKV_TIER_T0) {
-      logits_dense<G, false>(pg, row, g, sm.q16, s);
-      float r = reduce_scatter<G>(s, g);
-      float logit = valid ? r * p.qk_scale_log2 : -INFINITY;
-      softmax_pv<G, 1>(logit, 1.0f, pg + kHdrBytes + 256 * P + (row0 >> 3) * 2048, st, lane);
+      logits_dense<G, false>(pg, rA, g, q32, sA, sB);
+      const float a = reduce_scatter<G>(sA, g), b = reduce_scatter<G>(sB, g);
+      const float c = p.qk_scale_log2 * 5.192296858534828e+33f;  // 2^112
+      softmax_pv<G, 1>(vA ? a * c : -INFINITY, vB ? b * c : -INFINITY, 1.0f, 1.0f, vsec_dense,
+                       vsec_dense + 2048, st, lane);
     } else {
       const bool t1 = tier == SKV_TIER_T1;
       if (t1)
-        logits_t1<G>(pg, P, row, g, sm.lut1, s);
+        logits_t1<G>(pg, P, rA, g, lut1, sA, sB);
       else
-        logits_t2<G>(pg, P, row, g, sm.lut2, s);
-      float r = reduce_scatter<G>(s, g);
-      const uint16_t* rt = reinterpret_cast<const uint16_t*>(pg + kHdrBytes);
+        logits_t2<G>(pg, P, rA, g, lut2, sA, sB);
+      const float a = reduce_scatter<G>(sA, g), b = reduce_scatter<G>(sB, g);
       const int cb = t1 ? 64 : 48;
-      const uint16_t* sc = reinterpret_cast<const uint16_t*>(pg + kHdrBytes + 2 * P + cb * P);
-      const float rtil = __half2float(__ushort_as_half(rt[row]));
-      const float vs = __half2float(__ushort_as_half(sc[row]));
-      float logit = valid ? r * (rtil * p.qk_scale_log2) : -INFINITY;
-      const uint8_t* vsec = pg + kHdrBytes + (2 + cb + 2) * P;
-      softmax_pv<G, 0>(logit, valid ? vs : 0.0f, vsec + (row0 >> 3) * 1024, st, lane);
+      const uint32_t rs = pg + kHdrBytes, ss = pg + kHdrBytes + (2 + cb) * P;
+      const float rtA = __half2float(__ushort_as_half((unsigned short)lds16(rs + 2 * rA)));
+      const float rtB = __half2float(__ushort_as_half((unsigned short)lds16(rs + 2 * rB)));
+      const float vsA = __half2float(__ushort_as_half((unsigned short)lds16(ss + 2 * rA)));
+      const float vsB = __half2float(__ushort_as_half((unsigned short)lds16(ss + 2 * rB)));
+      const float c = p.qk_scale_log2 * 0.0625f;  // shares entered as code + 1 = 16 rho^
+      const uint32_t vsec = pg + kHdrBytes + (2 + cb + 2) * P + (row0 >> 3) * 1024;
+      softmax_pv<G, 0>(vA ? a * (rtA * c) : -INFINITY, vB ? b * (rtB * c) : -INFINITY,
+                       vA ? vsA : 0.0f, vB ? vsB : 0.0f, vsec, vsec + 1024, st, lane);
     }
   }
 }
@@ -298,23 +404,43 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     decode_kernel(const __grid_constant__ DecodeParams p) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
   using Smem = DecodeSmem<G, DENSE>;
+  using LG = LutGeom<G>;
   Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
-  uint8_t* ring = smem_raw + ((sizeof(Smem) + 127) / 128) * 128;
+  const uint32_t base = smem_u32(smem_raw);
+  const uint32_t ring_u32 = base + (uint32_t)(((sizeof(Smem) + 127) / 128) * 128);
+  const uint32_t limit = base + (uint32_t)p.smem_bytes;
+  uint32_t lut1 = 0, lut2 = 0, ring_end = limit;
+  if constexpr (!DENSE) {
+    lut1 = (limit - LG::kLut1 - LG::kLut2) / LG::kLut1 * LG::kLut1;
+    lut2 = lut1 + LG::kLut1;
+    ring_end = lut1;
+  }
+  const uint32_t ring_bytes = (ring_end - ring_u32) / 128 * 128;
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   const int c = blockIdx.x;
   const int U = p.B * p.Hkv;
   const long long N = p.indptr[U];
   const long long g0 = chunk_begin(c, N, p.S), g1 = chunk_begin(c + 1, N, p.S);
-  const int ipp = 64 >> p.log2P;
+  const int ipp = 128 >> p.log2P;
 
   if (tid == 0) {
     for (int i = 0; i < kNSlot; ++i) {
       mbar_init(smem_u32(&sm.full[i]), 1);
-      mbar_init(smem_u32(&sm.empty[i]), kNCW);
+      mbar_init(smem_u32(&sm.empty[i]), kGW);
     }
     sm.abort_flag = 0;
+    if (ring_bytes < 128u * 512u + kMaxIPP * kHdrBytes) report(p.err, SKV_ERR_ARG);
     fence_mbar_init();
+  }
+  // units without any resident page: out = 0, lse = -inf (written by CTA 0)
+  if (c == 0) {
+    for (int u = warp; u < U; u += kDecodeThreads / 32) {
+      if (p.indptr[u + 1] > p.indptr[u]) continue;
+      const long long o = (long long)(u / p.Hkv) * p.Hq + (long long)(u % p.Hkv) * G;
+      for (int i = lane; i < G * kHeadDim; i += 32) p.out[o * kHeadDim + i] = 0.0f;
+      if (p.lse && lane < G) p.lse[o + lane] = -INFINITY;
+    }
   }
   __syncthreads();
   if (g0 >= g1) return;
@@ -322,99 +448,141 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   // first unit whose pages reach past g0: largest u with indptr[u] <= g0
   int lo = 0, hi = U;
   while (hi - lo > 1) {
-    int mid = (lo + hi) >> 1;
+    const int mid = (lo + hi) >> 1;
     if (p.indptr[mid] <= g0) lo = mid; else hi = mid;
   }
   const int u0 = lo;
 
   if (warp == kNCW) {
     // ------------------------------------------------------------ producer
-    const uint32_t R = (uint32_t)p.ring_bytes;
-    long long head = 0;
+    // One thread places items in the ring and issues the copies; the warp
+    // stages the chunk's page ids into shared memory in coalesced batches.
+    // The per-item path is kept short: it bounds the streaming rate.
+    const uint32_t R = ring_bytes;
+    const uint32_t pay0 = (uint32_t)p.payload[0], pay1 = (uint32_t)p.payload[1],
+                   pay2 = (uint32_t)p.payload[2];
+    const uint8_t *pool0 = p.pool[0], *pool1 = p.pool[1], *pool2 = p.pool[2];
+    const long long st0 = p.stride[0], st1 = p.stride[1], st2 = p.stride[2];
+    const unsigned long long sl0 = (unsigned long long)p.slots[0],
+                             sl1 = (unsigned long long)p.slots[1],
+                             sl2 = (unsigned long long)p.slots[2];
+    int u = u0;
+    long long ub = min(g1, (long long)p.indptr[u0 + 1]);  // end of the current unit's run
+    long long pg = g0;                                     // first page of the next item
     int it = 0, tail = 0;
-    long long wbase = -1;  // first page of the id window held in lanes
-    uint32_t idwin = 0;
+    uint32_t wr = 0, rd = 0;
     bool ok = true;
-    for (int u = u0; u < U && ok; ++u) {
-      const long long iu0 = p.indptr[u], iu1 = p.indptr[u + 1];
-      if (iu0 >= g1) break;
-      const long long a = max(g0, iu0), b = min(g1, iu1);
-      for (long long pg = a; pg < b && ok; pg += ipp) {
-        const int n = (int)min((long long)ipp, b - pg);
-        uint32_t sizes[kMaxIPP], ids[kMaxIPP];
-        uint32_t total = 0;
+    for (long long bbase = g0; bbase < g1 && ok && pg < g1; bbase += kIdBatch) {
+      const long long bend = min(g1, bbase + kIdBatch + kMaxIPP);
+      __syncwarp();
+      for (long long gp = bbase + lane; gp < bend; gp += 32) sm.ids[gp - bbase] = p.ids[gp];
+      __syncwarp();
+      if (lane == 0) {
+        while (pg < g1 && pg < bbase + kIdBatch) {
+          while (pg >= ub) {  // next unit with pages in this chunk
+            ++u;
+            ub = min(g1, (long long)p.indptr[u + 1]);
+          }
+          const int n = (int)min((long long)ipp, ub - pg);
+          uint32_t sz[kMaxIPP];
+          const uint8_t* src[kMaxIPP];
+          uint32_t total = 0, tiers = 0;
 #pragma unroll
-        for (int k = 0; k < kMaxIPP; ++k) {
-          sizes[k] = 0;
-          ids[k] = 0;
-          if (k < n) {
-            const long long gp = pg + k;
-            if (wbase < 0 || gp >= wbase + 32) {
-              wbase = gp;
-              idwin = (gp + lane < g1) ? p.ids[gp + lane] : 0u;
+          for (int k = 0; k < kMaxIPP; ++k) {
+            sz[k] = 0;
+            src[k] = nullptr;
+            if (k < n) {
+              const uint32_t id = sm.ids[pg + k - bbase];
+              const uint32_t tr = id >> 30, slot = id & 0x3FFFFFFFu;
+              bool valid;
+              if (DENSE) {
+                valid = tr == 0 && slot < sl0;
+              } else {
+                valid = (tr == 0 && slot < sl0) || (tr == 1 && slot < sl1) ||
+                        (tr == 2 && slot < sl2);
+              }
+              if (valid) {
+                sz[k] = tr == 0 ? pay0 : (tr == 1 ? pay1 : pay2);
+                src[k] = tr == 0 ? pool0 + (long long)slot * st0
+                                 : (tr == 1 ? pool1 + (long long)slot * st1
+                                            : pool2 + (long long)slot * st2);
+              } else {
+                report(p.err, SKV_ERR_CORRUPT);
+              }
+              tiers |= (tr & 3u) << (2 * k);
+              total += sz[k];
             }
-            const uint32_t id = __shfl_sync(0xFFFFFFFFu, idwin, (int)(gp - wbase));
-            const uint32_t tr = id >> 30, slot = id & 0x3FFFFFFFu;
-            ids[k] = id;
-            const bool valid = DENSE ? (tr == 0 && slot < (uint64_t)p.slots[0])
-                                     : (tr < 3 && slot < (uint64_t)p.slots[tr]);
-            if (valid) sizes[k] = (uint32_t)p.payload[tr];
-            else if (lane == 0) report(p.err, SKV_ERR_CORRUPT);
-            total += sizes[k];
           }
-        }
-        if (lane == 0) {
+          // ring placement: live items occupy [rd, wr) (or wrap around)
           const int s = it % kNSlot;
-          long long pos = head;
-          uint32_t off = (uint32_t)(pos % R);
-          if (off + total > R) {
-            pos += R - off;
-            off = 0;
-          }
-          while (tail < it && (it - tail >= kNSlot ||
-                               sm.item_start[tail % kNSlot] < pos + (long long)total - R)) {
+          uint32_t off = 0;
+          while (true) {
+            bool fits = false;
+            if (it == tail) {
+              wr = 0;
+              rd = 0;
+              off = 0;
+              fits = total <= R;
+              if (!fits) {  // cannot happen for the supported page sizes
+                report(p.err, SKV_ERR_ARG);
+                ok = false;
+                break;
+              }
+            } else if (it - tail < kNSlot) {
+              if (wr > rd) {
+                if (wr + total <= R) {
+                  off = wr;
+                  fits = true;
+                } else if (total <= rd) {
+                  off = 0;
+                  fits = true;
+                }
+              } else if (wr < rd && wr + total <= rd) {
+                off = wr;
+                fits = true;
+              }
+            }
+            if (fits) break;
             if (!mbar_wait_bounded(smem_u32(&sm.empty[tail % kNSlot]),
                                    (uint32_t)((tail / kNSlot) & 1), &sm.abort_flag)) {
               ok = false;
               break;
             }
             ++tail;
+            rd = (tail < it) ? sm.item_start[tail % kNSlot] : wr;
           }
-          if (ok) {
-            sm.item_start[s] = pos;
-            sm.item_np[s] = (uint32_t)n;
-            uint32_t o = off, tiers = 0;
-            for (int k = 0; k < n; ++k) {
-              sm.item_off[s][k] = sizes[k] ? o : kInvalidOff;
-              tiers |= (ids[k] >> 30) << (8 * k);
-              o += sizes[k];
-            }
-            sm.item_tier[s] = tiers;
-            const uint32_t full = smem_u32(&sm.full[s]);
-            mbar_arrive_expect_tx(full, total);
-            o = off;
-            for (int k = 0; k < n; ++k) {
-              if (sizes[k]) {
-                const uint32_t tr = ids[k] >> 30, slot = ids[k] & 0x3FFFFFFFu;
-                bulk_g2s(smem_u32(ring + o), p.pool[tr] + (long long)slot * p.stride[tr], sizes[k],
-                         full);
-                o += sizes[k];
-              }
-            }
-            head = pos + total;
-            ++it;
+          if (!ok) break;
+          sm.item_start[s] = off;
+          sm.item_np[s] = (uint32_t)n;
+          sm.item_tier[s] = tiers;
+          uint32_t o = off;
+#pragma unroll
+          for (int k = 0; k < kMaxIPP; ++k) {
+            if (k < n) sm.item_off[s][k] = sz[k] ? o : kInvalidOff;
+            o += sz[k];
           }
+          wr = off + total;
+          const uint32_t fullb = smem_u32(&sm.full[s]);
+          mbar_arrive_expect_tx(fullb, total);
+          o = off;
+#pragma unroll
+          for (int k = 0; k < kMaxIPP; ++k) {
+            if (sz[k]) bulk_g2s(ring_u32 + o, src[k], sz[k], fullb);
+            o += sz[k];
+          }
+          ++it;
+          pg += n;
         }
-        ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
-        it = __shfl_sync(0xFFFFFFFFu, it, 0);
       }
+      ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
+      pg = __shfl_sync(0xFFFFFFFFu, pg, 0);
     }
     if (lane == 0 && !ok) {
       report(p.err, SKV_ERR_TIMEOUT);
       sm.abort_flag = 1;
       // let every copy already issued land before the CTA can exit
       for (int j = max(0, it - kNSlot); j < it; ++j) {
-        long long t0 = clock64();
+        const long long t0 = clock64();
         while (!mbar_try_wait(smem_u32(&sm.full[j % kNSlot]), (uint32_t)((j / kNSlot) & 1)) &&
                clock64() - t0 < kWaitLimitCycles) {
         }
@@ -424,11 +592,16 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   }
 
   // -------------------------------------------------------------- consumers
-  const int nct = kNCW * 32;
-  const int t4 = lane & 3, gq = lane >> 2;
   // A failed (timed-out) wait never breaks the loops: every consumer warp
   // must run the same sequence of named barriers.  After a failure the CTA's
   // abort flag makes every later wait return at once and work is skipped.
+  const int nct = kNCW * 32;
+  const int t4 = lane & 3, gq = lane >> 2;
+  const int group = warp / kGW, wig = warp % kGW;
+  const uint32_t q32 = smem_u32(sm.q32);
+  float* lut1p = reinterpret_cast<float*>(smem_raw + (lut1 - base));
+  float* lut2p = reinterpret_cast<float*>(smem_raw + (lut2 - base));
+  int* counters = reinterpret_cast<int*>(p.part + (long long)(p.S + U) * G * kPartStride);
   int it = 0;
   bool ok = true;
   for (int u = u0; u < U; ++u) {
@@ -438,18 +611,12 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     if (a >= b) continue;
     const int bb = u / p.Hkv, hkv = u % p.Hkv;
     named_bar_sync(1, nct);
-    // q of the G query heads of this kv head, as fp32 and as 16-bit
     for (int i = tid; i < G * kHeadDim; i += nct) {
       const int h = i / kHeadDim, d = i % kHeadDim;
       const long long qi = ((long long)bb * p.Hq + (long long)hkv * G + h) * kHeadDim + d;
       const uint16_t raw = reinterpret_cast<const uint16_t*>(p.q)[qi];
-      const float qf = p.q_bf16 ? __bfloat162float(__ushort_as_bfloat16(raw))
-                                : __half2float(__ushort_as_half(raw));
-      sm.q32[h][d] = qf;
-      if constexpr (DENSE)
-        sm.q16[h][d] = p.q_bf16 ? raw : __bfloat16_as_ushort(__float2bfloat16_rn(qf));
-      else
-        sm.q16[h][d] = p.q_bf16 ? __half_as_ushort(__float2half_rn(qf)) : raw;
+      sm.q32[h][d] = p.q_bf16 ? __bfloat162float(__ushort_as_bfloat16(raw))
+                              : __half2float(__ushort_as_half(raw));
       sm.O[h][d] = 0.0f;
     }
     named_bar_sync(1, nct);
@@ -457,23 +624,28 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       for (int i = tid; i < 64 * kPairs; i += nct) {
         const int cc = i >> 6, pr = i & 63;
         const float cs = p.cos6[cc], sn = p.sin6[cc];
-        uint16_t v[G];
+        float v[G];
 #pragma unroll
-        for (int h = 0; h < G; ++h)
-          v[h] = __half_as_ushort(
-              __float2half_rn(fmaf(sm.q32[h][2 * pr], cs, sm.q32[h][2 * pr + 1] * sn)));
-        uint16_t* dst = sm.lut1 + i * G;
+        for (int h = 0; h < G; ++h) v[h] = fmaf(sm.q32[h][2 * pr], cs, sm.q32[h][2 * pr + 1] * sn);
+        if constexpr (G == 4) {
+          *reinterpret_cast<float4*>(&lut1p[i * 4]) = make_float4(v[0], v[1], v[2], v[3]);
+        } else {
 #pragma unroll
-        for (int h = 0; h < G; ++h) dst[h] = v[h];
+          for (int h = 0; h < G; ++h) lut1p[i * G + h] = v[h];
+        }
       }
       for (int i = tid; i < 16 * kPairs; i += nct) {
         const int cc = i >> 6, pr = i & 63;
         const float cs = p.cos4[cc], sn = p.sin4[cc];
-        uint16_t* dst = sm.lut2 + i * G;
+        float v[G];
 #pragma unroll
-        for (int h = 0; h < G; ++h)
-          dst[h] = __half_as_ushort(
-              __float2half_rn(fmaf(sm.q32[h][2 * pr], cs, sm.q32[h][2 * pr + 1] * sn)));
+        for (int h = 0; h < G; ++h) v[h] = fmaf(sm.q32[h][2 * pr], cs, sm.q32[h][2 * pr + 1] * sn);
+        if constexpr (G == 4) {
+          *reinterpret_cast<float4*>(&lut2p[i * 4]) = make_float4(v[0], v[1], v[2], v[3]);
+        } else {
+#pragma unroll
+          for (int h = 0; h < G; ++h) lut2p[i * G + h] = v[h];
+        }
       }
       named_bar_sync(1, nct);
     }
@@ -486,9 +658,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       for (int e = 0; e < 4; ++e) st.acc[mt][e] = 0.0f;
 
     const long long nitems = (b - a + ipp - 1) / ipp;
-    const int kpage = (8 * warp) >> p.log2P;
-    const int row0 = (8 * warp) & (p.P - 1);
+    const int kpage = (16 * wig) >> p.log2P;
+    const int row0 = (16 * wig) & (p.P - 1);
     for (long long i = 0; i < nitems; ++i, ++it) {
+      if (kGroups > 1 && (it % kGroups) != group) continue;  // another group's item
       const int s = it % kNSlot;
       if (ok && !mbar_wait_bounded(smem_u32(&sm.full[s]), (uint32_t)((it / kNSlot) & 1),
                                    &sm.abort_flag)) {
@@ -501,14 +674,14 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       if (ok && kpage < (int)sm.item_np[s]) {
         const uint32_t off = sm.item_off[s][kpage];
         if (off != kInvalidOff)
-          process_rows<G, DENSE>(p, sm, ring + off, (sm.item_tier[s] >> (8 * kpage)) & 0xFFu,
-                                 row0, st, lane);
+          process_rows<G, DENSE>(p, ring_u32 + off, (sm.item_tier[s] >> (2 * kpage)) & 3u, row0,
+                                 lut1, lut2, q32, st, lane);
       }
       __syncwarp();
       if (lane == 0 && ok) mbar_arrive(smem_u32(&sm.empty[s]));
     }
 
-    // ---- combine the warps' states into this chunk's partial for unit u
+    // ---- combine the warps' states into this CTA's partial for unit u
     float l = st.l;
     l += __shfl_xor_sync(0xFFFFFFFFu, l, 4);
     l += __shfl_xor_sync(0xFFFFFFFFu, l, 8);
@@ -535,74 +708,144 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       }
     }
     named_bar_sync(1, nct);
-    float* part = p.part + (long long)(c + u) * G * kPartStride;
-    for (int i = tid; i < G * kHeadDim; i += nct) {
-      const int n = i / kHeadDim, d = i % kHeadDim;
-      part[n * kPartStride + 4 + d] = sm.O[n][d];
-      if (d == 0) {
-        float M = -INFINITY;
-        for (int w = 0; w < kNCW; ++w) M = fmaxf(M, sm.ml[w][n][0]);
-        float L = 0.0f;
-        if (M != -INFINITY)
+    // this CTA's (M, L) per head
+    float Mh[4], Lh[4];
+#pragma unroll
+    for (int n = 0; n < 4; ++n) {
+      Mh[n] = -INFINITY;
+      Lh[n] = 0.0f;
+      if (n < G) {
+        for (int w = 0; w < kNCW; ++w) Mh[n] = fmaxf(Mh[n], sm.ml[w][n][0]);
+        if (Mh[n] != -INFINITY)
           for (int w = 0; w < kNCW; ++w) {
             const float mw = sm.ml[w][n][0];
-            if (mw != -INFINITY) L += sm.ml[w][n][1] * exp2f(mw - M);
+            if (mw != -INFINITY) Lh[n] += sm.ml[w][n][1] * exp2f(mw - Mh[n]);
           }
-        part[n * kPartStride + 0] = M;
-        part[n * kPartStride + 1] = L;
       }
     }
-  }
-}
-
-// Merge the partials of every (unit, query head): one warp each.
-template <int G>
-__global__ void merge_kernel(const __grid_constant__ DecodeParams p) {
-  const int wid = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  const int U = p.B * p.Hkv;
-  if (wid >= U * G) return;
-  const int u = wid / G, n = wid % G;
-  const int bb = u / p.Hkv, hkv = u % p.Hkv;
-  const long long N = p.indptr[U];
-  const long long a = p.indptr[u], b = p.indptr[u + 1];
-  const long long oi = ((long long)bb * p.Hq + (long long)hkv * G + n);
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  float M = -INFINITY, L = 0.0f;
-  if (b > a && N > 0) {
+    // runs of the page list that touch unit u
     const long long S = p.S;
-    const int c0 = (int)(((a + 1) * S - 1) / N);
-    const int c1 = (int)((b * S - 1) / N);
-    for (int c = c0; c <= c1; ++c) {
-      if (chunk_begin(c, N, p.S) == chunk_begin(c + 1, N, p.S)) continue;
-      const float m = p.part[(long long)(c + u) * G * kPartStride + n * kPartStride];
-      M = fmaxf(M, m);
+    const int c0 = (int)(((iu0 + 1) * S - 1) / N);
+    const int c1 = (int)((iu1 * S - 1) / N);
+    int nruns = 0;
+    if (S <= N) {
+      nruns = c1 - c0 + 1;
+    } else {
+      for (int cc = c0; cc <= c1; ++cc)
+        nruns += chunk_begin(cc, N, p.S) != chunk_begin(cc + 1, N, p.S);
     }
-    if (M != -INFINITY) {
-      for (int c = c0; c <= c1; ++c) {
-        if (chunk_begin(c, N, p.S) == chunk_begin(c + 1, N, p.S)) continue;
-        const float* pp = p.part + (long long)(c + u) * G * kPartStride + n * kPartStride;
-        const float m = pp[0];
-        if (m == -INFINITY) continue;
-        const float sc = exp2f(m - M);
-        L += pp[1] * sc;
-        const float4 o = *reinterpret_cast<const float4*>(pp + 4 + 4 * lane);
-        acc.x += o.x * sc;
-        acc.y += o.y * sc;
-        acc.z += o.z * sc;
-        acc.w += o.w * sc;
+    const long long obase = (long long)bb * p.Hq + (long long)hkv * G;
+    if (nruns == 1) {
+      for (int i = tid; i < G * kHeadDim; i += nct) {
+        const int n = i / kHeadDim, d = i % kHeadDim;
+        const float L = Lh[n];
+        p.out[(obase + n) * kHeadDim + d] = L > 0.0f ? sm.O[n][d] / L : 0.0f;
+        if (d == 0 && p.lse)
+          p.lse[obase + n] = L > 0.0f ? (Mh[n] + log2f(L)) * 0.69314718055994530942f : -INFINITY;
+      }
+    } else {
+      float* part = p.part + (long long)(c + u) * G * kPartStride;
+      for (int i = tid; i < G * kHeadDim; i += nct) {
+        const int n = i / kHeadDim, d = i % kHeadDim;
+        __stcg(part + n * kPartStride + 4 + d, sm.O[n][d]);
+        if (d == 0) {
+          __stcg(part + n * kPartStride + 0, Mh[n]);
+          __stcg(part + n * kPartStride + 1, Lh[n]);
+        }
+      }
+      __threadfence();
+      named_bar_sync(1, nct);
+      if (tid == 0) {
+        const int ticket = atomicAdd(&counters[u], 1);
+        const int last = ticket == nruns - 1;
+        if (last) {
+          __threadfence();
+          counters[u] = 0;
+        }
+        sm.last_flag = last;
+      }
+      named_bar_sync(1, nct);
+      if (sm.last_flag) {
+        // merge the runs' partials of unit u (this CTA's included): run
+        // weights 2^(m_run - M) / L per head first, then one weighted sum per
+        // output element with the run loads issued back to back
+        const int nr = c1 - c0 + 1;
+        if (nr <= kMergeRuns) {
+          for (int i = tid; i < G * nr; i += nct) {
+            const int n = i / nr, r = i % nr;
+            const int cc = c0 + r;
+            float m = -INFINITY;  // an empty run contributes nothing
+            if (!(S > N && chunk_begin(cc, N, p.S) == chunk_begin(cc + 1, N, p.S)))
+              m = __ldcg(p.part + (long long)(cc + u) * G * kPartStride + n * kPartStride);
+            sm.mw[n][r] = m;
+          }
+          named_bar_sync(1, nct);
+          for (int i = tid; i < G * kHeadDim; i += nct) {
+            const int n = i / kHeadDim, d = i % kHeadDim;
+            float M = -INFINITY;
+            for (int r = 0; r < nr; ++r) M = fmaxf(M, sm.mw[n][r]);
+            float L = 0.0f, O = 0.0f;
+            if (M != -INFINITY) {
+              int r = 0;
+              for (; r + 4 <= nr; r += 4) {
+                float lv[4], ov[4], wv[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                  const float* pp =
+                      p.part + (long long)(c0 + r + k + u) * G * kPartStride + n * kPartStride;
+                  const float m = sm.mw[n][r + k];
+                  wv[k] = (m == -INFINITY) ? 0.0f : exp2f(m - M);
+                  lv[k] = (m == -INFINITY) ? 0.0f : __ldcg(pp + 1);
+                  ov[k] = (m == -INFINITY) ? 0.0f : __ldcg(pp + 4 + d);
+                }
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                  L += lv[k] * wv[k];
+                  O += ov[k] * wv[k];
+                }
+              }
+              for (; r < nr; ++r) {
+                const float m = sm.mw[n][r];
+                if (m == -INFINITY) continue;
+                const float* pp =
+                    p.part + (long long)(c0 + r + u) * G * kPartStride + n * kPartStride;
+                const float wgt = exp2f(m - M);
+                L += __ldcg(pp + 1) * wgt;
+                O += __ldcg(pp + 4 + d) * wgt;
+              }
+            }
+            p.out[(obase + n) * kHeadDim + d] = L > 0.0f ? O / L : 0.0f;
+            if (d == 0 && p.lse)
+              p.lse[obase + n] = L > 0.0f ? (M + log2f(L)) * 0.69314718055994530942f : -INFINITY;
+          }
+        } else {
+          for (int i = tid; i < G * kHeadDim; i += nct) {
+            const int n = i / kHeadDim, d = i % kHeadDim;
+            float M = -INFINITY, L = 0.0f, O = 0.0f;
+            for (int cc = c0; cc <= c1; ++cc) {
+              if (S > N && chunk_begin(cc, N, p.S) == chunk_begin(cc + 1, N, p.S)) continue;
+              const float* pp = p.part + (long long)(cc + u) * G * kPartStride + n * kPartStride;
+              const float m = __ldcg(pp), lc = __ldcg(pp + 1), oc = __ldcg(pp + 4 + d);
+              if (m == -INFINITY) continue;
+              if (m > M) {
+                const float r = (M == -INFINITY) ? 0.0f : exp2f(M - m);
+                L = L * r + lc;
+                O = O * r + oc;
+                M = m;
+              } else {
+                const float r = exp2f(m - M);
+                L += lc * r;
+                O += oc * r;
+              }
+            }
+            p.out[(obase + n) * kHeadDim + d] = L > 0.0f ? O / L : 0.0f;
+            if (d == 0 && p.lse)
+              p.lse[obase + n] = L > 0.0f ? (M + log2f(L)) * 0.69314718055994530942f : -INFINITY;
+          }
+        }
       }
     }
   }
-  float4 res = make_float4(0.f, 0.f, 0.f, 0.f);
-  float lse = -INFINITY;
-  if (L > 0.0f) {
-    const float inv = 1.0f / L;
-    res = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
-    lse = (M + log2f(L)) * 0.69314718055994530942f;
-  }
-  *reinterpret_cast<float4*>(p.out + oi * kHeadDim + 4 * lane) = res;
-  if (p.lse && lane == 0) p.lse[oi] = lse;
 }
 
 template <int G, bool DENSE>
@@ -611,9 +854,8 @@ size_t decode_smem_fixed() {
 }
 
 template <int G, bool DENSE>
-cudaError_t launch_decode_g(const DecodeParams& p, int ring_bytes, cudaStream_t stream,
-                            cudaEvent_t between) {
-  const size_t smem = decode_smem_fixed<G, DENSE>() + ring_bytes;
+cudaError_t launch_decode_g(const DecodeParams& p, cudaStream_t stream, cudaEvent_t between) {
+  const size_t smem = (size_t)p.smem_bytes;
   // The shared-memory opt-in is set once per device and size (outside any
   // stream capture: the first call on a device is expected to be eager).
   static size_t configured[64] = {};
@@ -626,7 +868,11 @@ cudaError_t launch_decode_g(const DecodeParams& p, int ring_bytes, cudaStream_t 
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64) configured[dev] = smem;
   }
-  decode_kernel<G, DENSE><<<p.S, kDecodeThreads, smem, stream>>>(p);
+  const int U = p.B * p.Hkv;
+  int* counters = reinterpret_cast<int*>(p.part + (long long)(p.S + U) * G * kPartStride);
+  e = cudaMemsetAsync(counters, 0, sizeof(int) * (size_t)U, stream);
+  if (e != cudaSuccess) return e;
+  decode_kernel<G, DENSE><<<p.S, kDecodeThreads, p.smem_bytes, stream>>>(p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (between) {
@@ -634,10 +880,7 @@ cudaError_t launch_decode_g(const DecodeParams& p, int ring_bytes, cudaStream_t 
     e = cudaEventRecordWithFlags(between, stream, cudaEventRecordExternal);
     if (e != cudaSuccess) return e;
   }
-  const int warps = p.B * p.Hkv * G;
-  const int threads = 256;
-  merge_kernel<G><<<(warps * 32 + threads - 1) / threads, threads, 0, stream>>>(p);
-  return cudaGetLastError();
+  return cudaSuccess;
 }
 
 size_t decode_fixed_smem(int G, bool dense) {
@@ -659,15 +902,15 @@ cudaError_t launch_decode(const DecodeParams& p, int G, bool dense, cudaStream_t
                           cudaEvent_t between) {
   if (dense) {
     switch (G) {
-      case 1: return launch_decode_g<1, true>(p, p.ring_bytes, stream, between);
-      case 2: return launch_decode_g<2, true>(p, p.ring_bytes, stream, between);
-      case 4: return launch_decode_g<4, true>(p, p.ring_bytes, stream, between);
+      case 1: return launch_decode_g<1, true>(p, stream, between);
+      case 2: return launch_decode_g<2, true>(p, stream, between);
+      case 4: return launch_decode_g<4, true>(p, stream, between);
     }
   } else {
     switch (G) {
-      case 1: return launch_decode_g<1, false>(p, p.ring_bytes, stream, between);
-      case 2: return launch_decode_g<2, false>(p, p.ring_bytes, stream, between);
-      case 4: return launch_decode_g<4, false>(p, p.ring_bytes, stream, between);
+      case 1: return launch_decode_g<1, false>(p, stream, between);
+      case 2: return launch_decode_g<2, false>(p, stream, between);
+      case 4: return launch_decode_g<4, false>(p, stream, between);
     }
   }
   return cudaErrorInvalidValue;

@@ -26,7 +26,7 @@ struct DecodeParams {
   int S;
   int P;
   int log2P;
-  int ring_bytes;
+  int smem_bytes;       // dynamic shared memory of the decode kernel
   float qk_scale_log2;  // log2(e) / sqrt(d)
   float cos6[64], sin6[64], cos4[16], sin4[16];
 };

@@ -85,6 +85,6 @@ def test_workspace_sizes():
     ctx = skv.Context(64)
     sm, splits = ctx.device_info()
     n = ctx.workspace_size(skv.WS_DECODE, 1, 8, 32, 0, 0)
-    assert n == (splits + 8) * 4 * 132 * 4
-    assert ctx.workspace_size(skv.WS_DECODE, 1, 8, 32, 0, 10) == (10 + 8) * 4 * 132 * 4
+    assert n == (splits + 8) * 4 * 132 * 4 + 8 * 4
+    assert ctx.workspace_size(skv.WS_DECODE, 1, 8, 32, 0, 10) == (10 + 8) * 4 * 132 * 4 + 8 * 4
     assert ctx.workspace_size(skv.WS_ALLOCATE, 2, 8, 0, 1000) > 2 * 8 * 1000 * 4
