@@ -346,10 +346,10 @@ static int decode_common(skv_ctx* ctx, const void* q, int q_dtype, int B, int Hq
   p.S = decode_splits(ctx, num_splits);
   p.P = ctx->P;
   p.log2P = ctx->log2P;
-  const size_t fixed = skv::decode_fixed_smem(G, dense);
-  const long long luts = dense ? 0 : 80LL * 256 * G;   // 6-bit + 4-bit fp32 LUTs
-  const long long max_item = 128LL * 512 + 8 * skv::kHdrBytes;
-  if ((long long)ctx->smem_optin < (long long)fixed + luts + max_item + 65536)
+  long long max_pay = p.payload[0];
+  if (!dense) max_pay = std::max(max_pay, (long long)std::max(p.payload[1], p.payload[2]));
+  const long long max_item = (skv::kDecodeItemRows / p.P) * max_pay;
+  if (!skv::decode_smem_ok(G, dense, (int)ctx->smem_optin, (int)max_item))
     return fail(SKV_ERR_ARG, "%s: not enough shared memory per block", name);
   p.smem_bytes = (int)ctx->smem_optin;
   p.qk_scale_log2 = (float)(1.4426950408889634 / std::sqrt(128.0));

@@ -11,11 +11,20 @@
 // CTA that brings the unit's ticket counter to its run count merges them
 // (log-sum-exp) -- no CTA ever waits for another.
 //
-// CTA = 8 consumer warps + 1 producer warp.  The producer copies whole
-// pages (header included) with 1-D bulk asynchronous copies (no multicast)
-// into a byte ring in shared memory, 128 tokens per "item" (128/P pages),
-// tracked by full/empty mbarriers; consumer warp w takes rows
-// [16w, 16w+16) of each item, i.e. 16 rows of one page.
+// CTA = 8 consumer warps in kCG groups + 1 planner warp + kIss issuer
+// warps around one byte ring in shared memory.  The CTA's run is cut into
+// "items" of 64 tokens (64/P pages, never crossing a unit).  The planner
+// decodes page ids lane-parallel (a window of 64 pages at a time), places
+// each item in the ring, writes its descriptors and signals it ready;
+// issuer k copies the items i = k (mod kIss) with 1-D bulk asynchronous
+// copies (no multicast), whole pages with their headers; consumer group g
+// takes the items i = g (mod kCG), warp w of the group rows
+// [64 w / kGW, 64 (w + 1) / kGW) of each, 16 rows per pass.  Slots carry
+// ready (planner -> issuer), full (copies -> consumers) and empty
+// (consumers -> planner) mbarriers.  The bulk-copy issue holds its thread
+// for hundreds of cycles under load, so placement is kept off the issuing
+// threads and several issuers run at once; one shared ring keeps several
+// of even the largest (dense 64-token) items in flight.
 //
 // Consumer lane map: lane = 4 t + g, t = token of an 8-row group, g = pair
 // group; each lane carries rows t and t + 8.  Logits: lane (t, g) sums 16
@@ -31,22 +40,38 @@
 
 namespace skv {
 
-#ifndef SKV_DECODE_GROUPS
-#define SKV_DECODE_GROUPS 1
+#ifndef SKV_DECODE_ISSUERS
+#define SKV_DECODE_ISSUERS 2
 #endif
-constexpr int kGW = 8;                            // consumer warps per group (one item)
-constexpr int kGroups = SKV_DECODE_GROUPS;        // groups take items in turn
-constexpr int kNCW = kGroups * kGW;
-constexpr int kDecodeThreads = (kNCW + 1) * 32;
-constexpr int kNSlot = 16;
-constexpr int kMaxIPP = 8;
-constexpr int kIdBatch = 256;    // page ids staged per producer batch
-constexpr int kMergeRuns = 128;  // runs per unit merged through shared memory
-constexpr uint32_t kInvalidOff = 0xFFFFFFFFu;
+constexpr int kNCW = 8;                       // consumer warps per CTA
+constexpr int kCG = 2;                        // consumer groups
+constexpr int kGW = kNCW / kCG;               // consumer warps per group
+constexpr int kIss = SKV_DECODE_ISSUERS;      // issuer warps
+constexpr int kPlannerWarp = kNCW;
+constexpr int kDecodeThreads = (kNCW + 1 + kIss) * 32;
+constexpr int kItemRows = 64;                 // tokens per item
+constexpr int kRowsPerWarp = kItemRows / kGW;  // rows of an item per consumer warp
+constexpr int kPasses = kRowsPerWarp / 16;
+constexpr int kNSlot = 16;                    // items in flight, at most
+constexpr int kMaxIPP = kItemRows / 16;       // pages per item (P >= 16)
+constexpr int kMergeRuns = 128;               // runs per unit merged through shared memory
+static_assert(kCG == 1 || kCG == 2 || kCG == 4, "consumer groups: 1, 2 or 4");
+static_assert(kIss >= 1 && kIss <= 4, "issuers: 1..4");
+static_assert(kPasses >= 1 && kGW * kRowsPerWarp == kItemRows, "warp row split");
 
-// Shared-memory plan: [fixed block][ring][LUT1][LUT2].  LUT1 / LUT2 start at
-// shared addresses aligned to their own size, so that a gather address is
-// (code bits) | (pair offset) | (table base) -- one shift and one LOP3.
+// Item descriptor (16 B, written by the producer before it arms the slot's
+// full barrier): x = shared address of the item, y = meta, z/w = byte
+// offsets of pages 1..3 from the item start (16 bits each).
+// meta: bits 0-2 page count, bits 4 + 2k tier of page k, bit 12 + k page k
+// unusable (bad id: nothing copied for it).
+constexpr int kMetaTierShift = 4;
+constexpr int kMetaBadShift = 12;
+
+// Shared-memory plan: [ring][LUT1][LUT2][fixed block] (ADA) or
+// [ring][fixed block] (dense).  LUT1 / LUT2 start at shared addresses
+// aligned to their own size, so that a gather address is (code bits) |
+// (pair offset) | (table base) -- one shift and one LOP3; LUT1 is put as
+// high as the fixed block allows, which leaves the ring one contiguous run.
 template <int G>
 struct LutGeom {
   static constexpr uint32_t kEnt = 4 * G;                // bytes per entry (G fp32)
@@ -56,14 +81,18 @@ struct LutGeom {
   static constexpr int kCodeShift = (G == 4) ? 10 : (G == 2 ? 9 : 8);  // log2(kCode)
 };
 
+struct PageCopy {  // one page of a ready item, for its issuer
+  uint32_t src_lo, src_hi, bytes, dst;
+};
+
 template <int G, bool DENSE>
 struct __align__(16) DecodeSmem {
   unsigned long long full[kNSlot];
   unsigned long long empty[kNSlot];
-  uint32_t item_off[kNSlot][kMaxIPP];
-  uint32_t item_np[kNSlot];
-  uint32_t item_tier[kNSlot];   // 2 bits per page
-  uint32_t item_start[kNSlot];  // producer bookkeeping (ring offset)
+  unsigned long long ready[kNSlot];
+  uint4 desc[kNSlot];                  // consumers' view of an item
+  PageCopy copy[kNSlot][kMaxIPP];      // issuers' view of an item
+  uint32_t copy_bytes[kNSlot];         // bytes of the item (0xFFFFFFFF: no more items)
   int abort_flag;
   int last_flag;
   int pad_[2];
@@ -71,8 +100,36 @@ struct __align__(16) DecodeSmem {
   float O[4][kHeadDim];
   float q32[4][kHeadDim];
   float mw[4][kMergeRuns];        // merge: per-run weights
-  uint32_t ids[kIdBatch + kMaxIPP];  // producer: staged page ids
 };
+constexpr uint32_t kEndOfRun = 0xFFFFFFFFu;
+
+// Shared addresses of the ring, LUT1 (LUT2 follows it) and the fixed block
+// for a dynamic shared window [base, limit).  False when the ring would be
+// smaller than min_ring bytes.
+template <int G, bool DENSE>
+__host__ __device__ __forceinline__ bool smem_layout(uint32_t base, uint32_t limit,
+                                                     uint32_t fixed_bytes, uint32_t min_ring,
+                                                     uint32_t& ring_lo, uint32_t& ring_sz,
+                                                     uint32_t& lut1, uint32_t& fixed_at) {
+  using L = LutGeom<G>;
+  ring_lo = (base + 127) / 128 * 128;
+  lut1 = 0;
+  uint32_t ring_hi;
+  if constexpr (DENSE) {
+    if (limit < ring_lo + fixed_bytes + 128) return false;
+    fixed_at = (limit - fixed_bytes) / 128 * 128;
+    ring_hi = fixed_at;
+  } else {
+    const uint32_t tot = L::kLut1 + L::kLut2;
+    if (limit < ring_lo + fixed_bytes + tot) return false;
+    lut1 = (limit - fixed_bytes - tot) / L::kLut1 * L::kLut1;
+    if (lut1 <= ring_lo) return false;
+    fixed_at = lut1 + tot;  // 128-aligned: tot is a multiple of 128
+    ring_hi = lut1;
+  }
+  ring_sz = (ring_hi - ring_lo) / 128 * 128;
+  return ring_sz >= min_ring;
+}
 
 __device__ __forceinline__ long long chunk_begin(int c, long long N, int S) {
   return (long long)c * N / S;
@@ -405,33 +462,36 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   extern __shared__ __align__(128) uint8_t smem_raw[];
   using Smem = DecodeSmem<G, DENSE>;
   using LG = LutGeom<G>;
-  Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
   const uint32_t base = smem_u32(smem_raw);
-  const uint32_t ring_u32 = base + (uint32_t)(((sizeof(Smem) + 127) / 128) * 128);
   const uint32_t limit = base + (uint32_t)p.smem_bytes;
-  uint32_t lut1 = 0, lut2 = 0, ring_end = limit;
-  if constexpr (!DENSE) {
-    lut1 = (limit - LG::kLut1 - LG::kLut2) / LG::kLut1 * LG::kLut1;
-    lut2 = lut1 + LG::kLut1;
-    ring_end = lut1;
-  }
-  const uint32_t ring_bytes = (ring_end - ring_u32) / 128 * 128;
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   const int c = blockIdx.x;
   const int U = p.B * p.Hkv;
   const long long N = p.indptr[U];
   const long long g0 = chunk_begin(c, N, p.S), g1 = chunk_begin(c + 1, N, p.S);
-  const int ipp = 128 >> p.log2P;
+  const int ipp = kItemRows >> p.log2P;
+  // the largest item: ipp pages of the largest payload
+  int maxpay = p.payload[0];
+  if (!DENSE) maxpay = max(maxpay, max(p.payload[1], p.payload[2]));
+  uint32_t ring_lo, R, lut1, fixed_at;
+  const bool plan_ok = smem_layout<G, DENSE>(base, limit, (uint32_t)sizeof(Smem),
+                                             (uint32_t)(ipp * maxpay), ring_lo, R, lut1, fixed_at);
+  const uint32_t lut2 = lut1 + LG::kLut1;
+  Smem& sm = *reinterpret_cast<Smem*>(smem_raw + (plan_ok ? fixed_at - base : 0u));
 
   if (tid == 0) {
-    for (int i = 0; i < kNSlot; ++i) {
-      mbar_init(smem_u32(&sm.full[i]), 1);
-      mbar_init(smem_u32(&sm.empty[i]), kGW);
+    if (plan_ok) {
+      for (int i = 0; i < kNSlot; ++i) {
+        mbar_init(smem_u32(&sm.full[i]), 1);
+        mbar_init(smem_u32(&sm.empty[i]), kGW);
+        mbar_init(smem_u32(&sm.ready[i]), 1);
+      }
+      sm.abort_flag = 0;
+      fence_mbar_init();
+    } else {
+      report(p.err, SKV_ERR_ARG);
     }
-    sm.abort_flag = 0;
-    if (ring_bytes < 128u * 512u + kMaxIPP * kHdrBytes) report(p.err, SKV_ERR_ARG);
-    fence_mbar_init();
   }
   // units without any resident page: out = 0, lse = -inf (written by CTA 0)
   if (c == 0) {
@@ -443,7 +503,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     }
   }
   __syncthreads();
-  if (g0 >= g1) return;
+  if (g0 >= g1 || !plan_ok) return;
 
   // first unit whose pages reach past g0: largest u with indptr[u] <= g0
   int lo = 0, hi = U;
@@ -453,137 +513,173 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   }
   const int u0 = lo;
 
-  if (warp == kNCW) {
-    // ------------------------------------------------------------ producer
-    // One thread places items in the ring and issues the copies; the warp
-    // stages the chunk's page ids into shared memory in coalesced batches.
-    // The per-item path is kept short: it bounds the streaming rate.
-    const uint32_t R = ring_bytes;
-    const uint32_t pay0 = (uint32_t)p.payload[0], pay1 = (uint32_t)p.payload[1],
-                   pay2 = (uint32_t)p.payload[2];
-    const uint8_t *pool0 = p.pool[0], *pool1 = p.pool[1], *pool2 = p.pool[2];
-    const long long st0 = p.stride[0], st1 = p.stride[1], st2 = p.stride[2];
-    const unsigned long long sl0 = (unsigned long long)p.slots[0],
-                             sl1 = (unsigned long long)p.slots[1],
-                             sl2 = (unsigned long long)p.slots[2];
+  if (warp == kPlannerWarp) {
+    // ------------------------------------------------------------- planner
+    // Batches of up to 32 items of one unit: lane i decodes item it + i (its
+    // page ids -> sources, sizes, tiers) in parallel; a short uniform loop
+    // then places the items one by one.  Placement is deterministic: an item
+    // goes at the write offset, or at 0 when it would cross the ring's end;
+    // before it is published every older item whose bytes it may overwrite
+    // (virtual start < its virtual end - R) and the previous user of its
+    // slot must be released.  The lane that decoded the item writes its
+    // descriptors and signals the slot ready.  kIss end-of-run markers
+    // follow the last item, one per issuer.
     int u = u0;
     long long ub = min(g1, (long long)p.indptr[u0 + 1]);  // end of the current unit's run
-    long long pg = g0;                                     // first page of the next item
-    int it = 0, tail = 0;
-    uint32_t wr = 0, rd = 0;
+    long long pg = g0;                                     // first page of the next batch
+    int it = 0;                 // next item
+    int tail = 0;               // oldest item not known to be released
+    uint32_t wr = 0;            // ring write offset
+    unsigned long long V = 0;   // virtual position of the write offset (grows by laps of R)
+    unsigned long long vmine = 0;  // lane (j % 32): virtual start of in-flight item j
     bool ok = true;
-    for (long long bbase = g0; bbase < g1 && ok && pg < g1; bbase += kIdBatch) {
-      const long long bend = min(g1, bbase + kIdBatch + kMaxIPP);
-      __syncwarp();
-      for (long long gp = bbase + lane; gp < bend; gp += 32) sm.ids[gp - bbase] = p.ids[gp];
-      __syncwarp();
-      if (lane == 0) {
-        while (pg < g1 && pg < bbase + kIdBatch) {
-          while (pg >= ub) {  // next unit with pages in this chunk
-            ++u;
-            ub = min(g1, (long long)p.indptr[u + 1]);
-          }
-          const int n = (int)min((long long)ipp, ub - pg);
-          uint32_t sz[kMaxIPP];
-          const uint8_t* src[kMaxIPP];
-          uint32_t total = 0, tiers = 0;
+    // wait until item `tail` is released, then advance tail
+    auto release_tail = [&]() -> bool {
+      if (!mbar_wait_bounded(smem_u32(&sm.empty[tail % kNSlot]), (uint32_t)((tail / kNSlot) & 1),
+                             &sm.abort_flag))
+        return false;
+      ++tail;
+      return true;
+    };
+    while (ok && pg < g1) {
+      while (pg >= ub) {  // next unit with pages in this run
+        ++u;
+        ub = min(g1, (long long)p.indptr[u + 1]);
+      }
+      const int nb = (int)min(32LL, (ub - pg + ipp - 1) / ipp);  // items in this batch
+      // ---- lane-parallel decode of item it + lane
+      uint32_t plo[kMaxIPP], phi[kMaxIPP], psz[kMaxIPP];
+      uint32_t total = 0, imeta = 0, relz = 0, relw = 0;
+      if (lane < nb) {
+        const long long ps = pg + (long long)lane * ipp;
+        const int n = (int)min((long long)ipp, ub - ps);
+        imeta = (uint32_t)n;
+        uint32_t id[kMaxIPP];
 #pragma unroll
-          for (int k = 0; k < kMaxIPP; ++k) {
-            sz[k] = 0;
-            src[k] = nullptr;
-            if (k < n) {
-              const uint32_t id = sm.ids[pg + k - bbase];
-              const uint32_t tr = id >> 30, slot = id & 0x3FFFFFFFu;
-              bool valid;
-              if (DENSE) {
-                valid = tr == 0 && slot < sl0;
-              } else {
-                valid = (tr == 0 && slot < sl0) || (tr == 1 && slot < sl1) ||
-                        (tr == 2 && slot < sl2);
-              }
-              if (valid) {
-                sz[k] = tr == 0 ? pay0 : (tr == 1 ? pay1 : pay2);
-                src[k] = tr == 0 ? pool0 + (long long)slot * st0
-                                 : (tr == 1 ? pool1 + (long long)slot * st1
-                                            : pool2 + (long long)slot * st2);
-              } else {
-                report(p.err, SKV_ERR_CORRUPT);
-              }
-              tiers |= (tr & 3u) << (2 * k);
-              total += sz[k];
-            }
-          }
-          // ring placement: live items occupy [rd, wr) (or wrap around)
-          const int s = it % kNSlot;
-          uint32_t off = 0;
-          while (true) {
-            bool fits = false;
-            if (it == tail) {
-              wr = 0;
-              rd = 0;
-              off = 0;
-              fits = total <= R;
-              if (!fits) {  // cannot happen for the supported page sizes
-                report(p.err, SKV_ERR_ARG);
-                ok = false;
-                break;
-              }
-            } else if (it - tail < kNSlot) {
-              if (wr > rd) {
-                if (wr + total <= R) {
-                  off = wr;
-                  fits = true;
-                } else if (total <= rd) {
-                  off = 0;
-                  fits = true;
-                }
-              } else if (wr < rd && wr + total <= rd) {
-                off = wr;
-                fits = true;
-              }
-            }
-            if (fits) break;
-            if (!mbar_wait_bounded(smem_u32(&sm.empty[tail % kNSlot]),
-                                   (uint32_t)((tail / kNSlot) & 1), &sm.abort_flag)) {
-              ok = false;
-              break;
-            }
-            ++tail;
-            rd = (tail < it) ? sm.item_start[tail % kNSlot] : wr;
-          }
-          if (!ok) break;
-          sm.item_start[s] = off;
-          sm.item_np[s] = (uint32_t)n;
-          sm.item_tier[s] = tiers;
-          uint32_t o = off;
+        for (int q = 0; q < kMaxIPP; ++q) id[q] = q < n ? __ldg(p.ids + ps + q) : 0u;
 #pragma unroll
-          for (int k = 0; k < kMaxIPP; ++k) {
-            if (k < n) sm.item_off[s][k] = sz[k] ? o : kInvalidOff;
-            o += sz[k];
+        for (int q = 0; q < kMaxIPP; ++q) {
+          plo[q] = 0;
+          phi[q] = 0;
+          psz[q] = 0;
+          if (q == 1) relz = total;
+          if (q == 2) relz |= total << 16;
+          if (q == 3) relw = total;
+          if (q < n) {
+            const uint32_t tr = id[q] >> 30, slot = id[q] & 0x3FFFFFFFu;
+            bool valid;
+            if (DENSE) {
+              valid = tr == 0 && slot < (unsigned long long)p.slots[0];
+            } else {
+              valid = (tr == 0 && slot < (unsigned long long)p.slots[0]) ||
+                      (tr == 1 && slot < (unsigned long long)p.slots[1]) ||
+                      (tr == 2 && slot < (unsigned long long)p.slots[2]);
+            }
+            if (valid) {
+              const uint8_t* src = tr == 0 ? p.pool[0] + (long long)slot * p.stride[0]
+                                           : (tr == 1 ? p.pool[1] + (long long)slot * p.stride[1]
+                                                      : p.pool[2] + (long long)slot * p.stride[2]);
+              plo[q] = (uint32_t)reinterpret_cast<uintptr_t>(src);
+              phi[q] = (uint32_t)(reinterpret_cast<uintptr_t>(src) >> 32);
+              psz[q] = (uint32_t)(tr == 0 ? p.payload[0] : (tr == 1 ? p.payload[1] : p.payload[2]));
+            } else {
+              report(p.err, SKV_ERR_CORRUPT);
+              imeta |= 1u << (kMetaBadShift + q);
+            }
+            imeta |= (tr & 3u) << (kMetaTierShift + 2 * q);
+            total += psz[q];
           }
-          wr = off + total;
-          const uint32_t fullb = smem_u32(&sm.full[s]);
-          mbar_arrive_expect_tx(fullb, total);
-          o = off;
-#pragma unroll
-          for (int k = 0; k < kMaxIPP; ++k) {
-            if (sz[k]) bulk_g2s(ring_u32 + o, src[k], sz[k], fullb);
-            o += sz[k];
-          }
-          ++it;
-          pg += n;
         }
       }
-      ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
-      pg = __shfl_sync(0xFFFFFFFFu, pg, 0);
+      // ---- uniform placement, one item at a time
+      for (int i = 0; i < nb && ok; ++i) {
+        const uint32_t t = __shfl_sync(0xFFFFFFFFu, total, i);
+        const uint32_t off = (wr + t <= R) ? wr : 0u;
+        const unsigned long long vi = (off == wr) ? V : V + (R - wr);
+        // release what this item may overwrite, and its slot's previous item
+        while (tail < it) {
+          const unsigned long long vt = __shfl_sync(0xFFFFFFFFu, vmine, tail & 31);
+          if (it - tail < kNSlot && vt + R >= vi + t) break;
+          if (!release_tail()) {
+            ok = false;
+            break;
+          }
+        }
+        if (!ok) break;
+        const int s = it % kNSlot;
+        if (lane == (it & 31)) vmine = vi;
+        if (lane == i) {
+          sm.desc[s] = make_uint4(ring_lo + off, imeta, relz, relw);
+          const uint32_t rel[kMaxIPP] = {0u, relz & 0xFFFFu, relz >> 16, relw};
+#pragma unroll
+          for (int q = 0; q < kMaxIPP; ++q)
+            if (q < (int)(imeta & 7u))
+              sm.copy[s][q] = PageCopy{plo[q], phi[q], psz[q], ring_lo + off + rel[q]};
+          sm.copy_bytes[s] = total;
+          mbar_arrive(smem_u32(&sm.ready[s]));
+        }
+        wr = off + t;
+        V = vi + t;
+        ++it;
+      }
+      pg = min(ub, pg + (long long)nb * ipp);
+    }
+    // end-of-run markers: a slot each (its previous item released)
+    for (int e = 0; e < kIss && ok; ++e) {
+      while (it - tail >= kNSlot) {
+        if (!release_tail()) {
+          ok = false;
+          break;
+        }
+      }
+      if (!ok) break;
+      const int s = it % kNSlot;
+      if (lane == 0) {
+        sm.copy_bytes[s] = kEndOfRun;
+        mbar_arrive(smem_u32(&sm.ready[s]));
+      }
+      ++it;
     }
     if (lane == 0 && !ok) {
       report(p.err, SKV_ERR_TIMEOUT);
       sm.abort_flag = 1;
-      // let every copy already issued land before the CTA can exit
-      for (int j = max(0, it - kNSlot); j < it; ++j) {
-        const long long t0 = clock64();
-        while (!mbar_try_wait(smem_u32(&sm.full[j % kNSlot]), (uint32_t)((j / kNSlot) & 1)) &&
+    }
+    return;
+  }
+  if (warp > kPlannerWarp) {
+    // ------------------------------------------------------------- issuers
+    if (lane != 0) return;
+    const int k = warp - kPlannerWarp - 1;
+    int it = k;
+    bool ok = true;
+    while (true) {
+      const int s = it % kNSlot;
+      if (!mbar_wait_bounded(smem_u32(&sm.ready[s]), (uint32_t)((it / kNSlot) & 1),
+                             &sm.abort_flag)) {
+        ok = false;
+        break;
+      }
+      const uint32_t total = sm.copy_bytes[s];
+      if (total == kEndOfRun) break;
+      const uint32_t np = sm.desc[s].y & 7u;
+      const uint32_t fullb = smem_u32(&sm.full[s]);
+      mbar_arrive_expect_tx(fullb, total);
+      for (uint32_t q = 0; q < np; ++q) {
+        const PageCopy cp = sm.copy[s][q];
+        if (cp.bytes)
+          bulk_g2s(cp.dst, reinterpret_cast<const void*>((uintptr_t)cp.src_lo |
+                                                         ((uintptr_t)cp.src_hi << 32)),
+                   cp.bytes, fullb);
+      }
+      it += kIss;
+    }
+    if (!ok) {
+      report(p.err, SKV_ERR_TIMEOUT);
+      sm.abort_flag = 1;
+      // let every copy this issuer started land before the CTA can exit
+      const long long t0 = clock64();
+      for (int jj = it - kIss; jj >= 0 && jj >= it - kNSlot; jj -= kIss) {
+        while (!mbar_try_wait(smem_u32(&sm.full[jj % kNSlot]), (uint32_t)((jj / kNSlot) & 1)) &&
                clock64() - t0 < kWaitLimitCycles) {
         }
       }
@@ -597,12 +693,12 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   // abort flag makes every later wait return at once and work is skipped.
   const int nct = kNCW * 32;
   const int t4 = lane & 3, gq = lane >> 2;
-  const int group = warp / kGW, wig = warp % kGW;
+  const int grp = warp / kGW, wi = warp % kGW;  // consumer group, warp within it
   const uint32_t q32 = smem_u32(sm.q32);
   float* lut1p = reinterpret_cast<float*>(smem_raw + (lut1 - base));
   float* lut2p = reinterpret_cast<float*>(smem_raw + (lut2 - base));
   int* counters = reinterpret_cast<int*>(p.part + (long long)(p.S + U) * G * kPartStride);
-  int it = 0;
+  int it = 0;  // item index within the run
   bool ok = true;
   for (int u = u0; u < U; ++u) {
     const long long iu0 = p.indptr[u], iu1 = p.indptr[u + 1];
@@ -657,13 +753,11 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
 #pragma unroll
       for (int e = 0; e < 4; ++e) st.acc[mt][e] = 0.0f;
 
-    const long long nitems = (b - a + ipp - 1) / ipp;
-    const int kpage = (16 * wig) >> p.log2P;
-    const int row0 = (16 * wig) & (p.P - 1);
-    for (long long i = 0; i < nitems; ++i, ++it) {
-      if (kGroups > 1 && (it % kGroups) != group) continue;  // another group's item
-      const int s = it % kNSlot;
-      if (ok && !mbar_wait_bounded(smem_u32(&sm.full[s]), (uint32_t)((it / kNSlot) & 1),
+    const int nitems = (int)((b - a + ipp - 1) / ipp);
+    // this group's items of the unit: it + i with (it + i) % kCG == grp
+    for (int i = (grp - it) & (kCG - 1); i < nitems; i += kCG) {
+      const int itm = it + i, s = itm % kNSlot;
+      if (ok && !mbar_wait_bounded(smem_u32(&sm.full[s]), (uint32_t)((itm / kNSlot) & 1),
                                    &sm.abort_flag)) {
         ok = false;
         if (lane == 0) {
@@ -671,15 +765,27 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
           sm.abort_flag = 1;
         }
       }
-      if (ok && kpage < (int)sm.item_np[s]) {
-        const uint32_t off = sm.item_off[s][kpage];
-        if (off != kInvalidOff)
-          process_rows<G, DENSE>(p, ring_u32 + off, (sm.item_tier[s] >> (2 * kpage)) & 3u, row0,
-                                 lut1, lut2, q32, st, lane);
+      if (ok) {
+        const uint4 d = lds128(smem_u32(&sm.desc[s]));
+        const uint32_t np = d.y & 7u;
+#pragma unroll
+        for (int ps = 0; ps < kPasses; ++ps) {
+          const int r = kRowsPerWarp * wi + 16 * ps;  // row within the item
+          const uint32_t kp = (uint32_t)(r >> p.log2P);
+          const int row0 = r & (p.P - 1);
+          if (kp < np && !((d.y >> (kMetaBadShift + kp)) & 1u)) {
+            const uint32_t rel = kp == 0 ? 0u
+                                         : (kp == 1 ? (d.z & 0xFFFFu)
+                                                    : (kp == 2 ? (d.z >> 16) : d.w));
+            process_rows<G, DENSE>(p, d.x + rel, (d.y >> (kMetaTierShift + 2 * kp)) & 3u, row0,
+                                   lut1, lut2, q32, st, lane);
+          }
+        }
       }
       __syncwarp();
       if (lane == 0 && ok) mbar_arrive(smem_u32(&sm.empty[s]));
     }
+    it += nitems;
 
     // ---- combine the warps' states into this CTA's partial for unit u
     float l = st.l;
@@ -881,6 +987,33 @@ cudaError_t launch_decode_g(const DecodeParams& p, cudaStream_t stream, cudaEven
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;
+}
+
+template <int G, bool DENSE>
+bool decode_plan_ok(int smem_bytes, int max_item) {
+  // the dynamic shared window starts at offset 0 or after a 1 KB reserve
+  for (uint32_t b = 0; b <= 1024; b += 1024) {
+    uint32_t rlo, rsz, lut1, fixed_at;
+    if (!smem_layout<G, DENSE>(b, b + (uint32_t)smem_bytes, (uint32_t)sizeof(DecodeSmem<G, DENSE>),
+                               (uint32_t)max_item, rlo, rsz, lut1, fixed_at))
+      return false;
+  }
+  return true;
+}
+
+bool decode_smem_ok(int G, bool dense, int smem_bytes, int max_item) {
+  if (dense) {
+    switch (G) {
+      case 1: return decode_plan_ok<1, true>(smem_bytes, max_item);
+      case 2: return decode_plan_ok<2, true>(smem_bytes, max_item);
+      default: return decode_plan_ok<4, true>(smem_bytes, max_item);
+    }
+  }
+  switch (G) {
+    case 1: return decode_plan_ok<1, false>(smem_bytes, max_item);
+    case 2: return decode_plan_ok<2, false>(smem_bytes, max_item);
+    default: return decode_plan_ok<4, false>(smem_bytes, max_item);
+  }
 }
 
 size_t decode_fixed_smem(int G, bool dense) {

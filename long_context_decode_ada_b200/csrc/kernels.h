@@ -86,6 +86,10 @@ struct AllocParams {
 };
 
 size_t decode_fixed_smem(int G, bool dense);
+// True when smem_bytes of dynamic shared memory hold the decode kernel's
+// fixed block, LUTs and rings for items of up to max_item bytes.
+bool decode_smem_ok(int G, bool dense, int smem_bytes, int max_item);
+constexpr int kDecodeItemRows = 64;  // tokens per decode item
 cudaError_t launch_decode(const DecodeParams& p, int G, bool dense, cudaStream_t stream,
                           cudaEvent_t between);
 cudaError_t launch_encode(const EncodeParams& p, cudaStream_t stream);
