@@ -138,17 +138,23 @@ def measured_peaks():
     return 6650.0, "fallback"
 
 
-def written_partials(indptr: np.ndarray, S: int) -> int:
-    """(chunk, unit) pairs the decode kernel writes a partial for."""
+def written_partials(indptr: np.ndarray, ids: np.ndarray, payload, S: int) -> int:
+    """(run, unit) partials the decode kernel writes: the page list is cut
+    into S runs of equal payload bytes (page g is in run floor(C(g) S / C),
+    C(g) the bytes before it); a unit spread over several runs gets one
+    partial per run, a unit inside one run none."""
     N = int(indptr[-1])
+    if N == 0:
+        return 0
+    cost = np.asarray(payload, np.int64)[np.asarray(ids[:N], np.uint32) >> 30]
+    before = np.concatenate([[0], np.cumsum(cost)[:-1]])
+    total = int(cost.sum())
+    run = np.array([(int(x) * S) // total for x in before], np.int64)
     n = 0
     for u in range(len(indptr) - 1):
         a, b = int(indptr[u]), int(indptr[u + 1])
-        if b <= a:
-            continue
-        c0 = ((a + 1) * S - 1) // N
-        c1 = (b * S - 1) // N
-        n += sum(1 for c in range(c0, c1 + 1) if (c * N) // S != ((c + 1) * N) // S)
+        k = len(np.unique(run[a:b])) if b > a else 0
+        n += k if k > 1 else 0
     return n
 
 
@@ -159,6 +165,7 @@ def clone_cache(cache):
     for t in range(3):
         c2.pools[t].copy_(cache.pools[t])
     c2.page_indptr.copy_(cache.page_indptr)
+    c2.page_tier_indptr.copy_(cache.page_tier_indptr)
     c2.page_ids.copy_(cache.page_ids)
     c2.tier.copy_(cache.tier)
     return c2
@@ -234,7 +241,7 @@ def run_skv(args, rank, world, local_rank):
     sm_count, default_splits = ctx.device_info()
     S = args.num_splits or default_splits
     G = w.Hq // w.Hkv
-    nparts = written_partials(indptr, S)
+    nparts = written_partials(indptr, ids, caches[0].payload, S)
     q_bytes = w.B * w.Hq * 128 * 2
     algo_bytes = (int(sum(int(tier_counts[t]) * TIER_BYTES[t] for t in range(3)))
                   + 16 * n_pages + 4 * n_pages + 4 * len(indptr) + q_bytes

@@ -153,6 +153,9 @@ int skv_workspace_size(const skv_ctx* ctx, int which, int B, int Hkv, int Hq, in
      row_of     int32 [B][Hkv][Tmax] device: page index within the unit's
                 list * P + row, or -1 when not resident
      page_indptr int32 [B*Hkv + 1] device: CSR offsets per unit b*Hkv + h
+     page_tier_indptr int32 [3*B*Hkv + 1] device or NULL: CSR offsets per
+                (unit, tier) segment 3*u + t (entry 3u = page_indptr[u]);
+                lets the decode split its work by streamed bytes
      page_ids   uint32 [page_cap] device: tier << 30 | slot; per unit the T0
                 pages, then T1, then T2
      err_word   int32 device: SKV_ERR_BUDGET, SKV_ERR_POOL or SKV_ERR_ARG
@@ -162,8 +165,9 @@ int skv_allocate(skv_ctx* ctx, const uint16_t* K, int B, int Hkv, int64_t Tmax,
                  const int32_t* seq_lens, const float* utility, const uint8_t* protect,
                  int mode, const int64_t* budget, const int32_t* quota,
                  const skv_free_lists* free, const skv_pools* pools, uint8_t* tier_out,
-                 int32_t* row_of, int32_t* page_indptr, uint32_t* page_ids, int64_t page_cap,
-                 int32_t* err_word, void* workspace, size_t ws_bytes, void* stream);
+                 int32_t* row_of, int32_t* page_indptr, int32_t* page_tier_indptr,
+                 uint32_t* page_ids, int64_t page_cap, int32_t* err_word, void* workspace,
+                 size_t ws_bytes, void* stream);
 
 /* skv_encode -- maps dense keys to spherical codes (technical summary 2.1,
    2.3): for every resident (b, h, t) writes its row of the page that
@@ -190,16 +194,18 @@ int skv_encode(skv_ctx* ctx, const uint16_t* K, const uint16_t* V, int B, int Hk
      Hq       a multiple of Hkv with Hq/Hkv in {1, 2, 4}
      page_indptr / page_ids / pools: the paged store (any slots, any order of
               pages within a unit; pages are streamed whole)
+     page_tier_indptr  NULL, or skv_allocate's per-(unit, tier) offsets: the
+              pages of all units are then cut into runs of equal payload
+              bytes instead of equal page counts (same results either way)
      out      fp32 [B][Hq][128] device; lse fp32 [B][Hq] device or NULL
               (a unit without resident tokens gives out 0, lse -inf)
-     num_splits  number of page chunks = CTAs (0 = default: 2 x SM count);
-              the pages of all units are cut into num_splits equal runs
+     num_splits  number of page runs = CTAs (0 = default: the SM count)
      workspace   skv_workspace_size(SKV_WS_DECODE, ..., num_splits) bytes
    Device errors: SKV_ERR_CORRUPT (bad page id / header: the page is
    skipped), SKV_ERR_TIMEOUT (a bounded wait ran out). */
 int skv_decode_attention(skv_ctx* ctx, const void* q, int q_dtype, int B, int Hq, int Hkv,
-                         const int32_t* page_indptr, const uint32_t* page_ids,
-                         const skv_pools* pools, float* out, float* lse, int32_t* err_word,
+                         const int32_t* page_indptr, const int32_t* page_tier_indptr,
+                         const uint32_t* page_ids, const skv_pools* pools, float* out, float* lse, int32_t* err_word,
                          void* workspace, size_t ws_bytes, int num_splits, void* stream);
 
 /* skv_dense_pack_bf16 -- the dense baseline's store: every token of every

@@ -357,6 +357,7 @@ __global__ void __launch_bounds__(1024) page_plan_kernel(const __grid_constant__
   for (int u = u0; u < u1; ++u) {
     p.indptr[u] = (int32_t)base[3];
     for (int t = 0; t < 3; ++t) {
+      if (p.tier_indptr) p.tier_indptr[u * 3 + t] = (int32_t)base[3];
       p.tbase[u * 3 + t] = (int32_t)base[t];
       const long long np = (p.counts[u * 3 + t] + p.P - 1) / p.P;
       base[t] += np;
@@ -365,6 +366,7 @@ __global__ void __launch_bounds__(1024) page_plan_kernel(const __grid_constant__
   }
   if (threadIdx.x == 0) {
     p.indptr[U] = (int32_t)tot[3];
+    if (p.tier_indptr) p.tier_indptr[3 * U] = (int32_t)tot[3];
     bool bad = tot[3] > p.page_cap || tot[3] > 0x7FFFFFFFLL;
     for (int t = 0; t < 3; ++t) bad |= tot[t] > p.free_len[t];
     if (bad) report(p.err, SKV_ERR_POOL);

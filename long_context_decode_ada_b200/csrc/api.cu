@@ -189,9 +189,8 @@ int skv_workspace_size(const skv_ctx* ctx, int which, int B, int Hkv, int Hq, in
     if (Hq <= 0 || Hq % Hkv != 0) return fail(SKV_ERR_ARG, "Hq must be a multiple of Hkv");
     const int G = Hq / Hkv;
     const long long S = decode_splits(ctx, num_splits);
-    // split partials, then one ticket counter per unit
-    *bytes = (size_t)(S + (long long)B * Hkv) * G * skv::kPartStride * sizeof(float) +
-             sizeof(int) * (size_t)B * Hkv;
+    // split partials, ticket counters, the split's published cost prefix
+    *bytes = skv::decode_ws(S, (long long)B * Hkv, G).bytes;
     return ok();
   }
   return fail(SKV_ERR_ARG, "skv_workspace_size: unknown kind %d", which);
@@ -212,8 +211,9 @@ int skv_allocate(skv_ctx* ctx, const uint16_t* K, int B, int Hkv, int64_t Tmax,
                  const int32_t* seq_lens, const float* utility, const uint8_t* protect, int mode,
                  const int64_t* budget, const int32_t* quota, const skv_free_lists* free,
                  const skv_pools* pools, uint8_t* tier_out, int32_t* row_of,
-                 int32_t* page_indptr, uint32_t* page_ids, int64_t page_cap, int32_t* err_word,
-                 void* workspace, size_t ws_bytes, void* stream) {
+                 int32_t* page_indptr, int32_t* page_tier_indptr, uint32_t* page_ids,
+                 int64_t page_cap, int32_t* err_word, void* workspace, size_t ws_bytes,
+                 void* stream) {
   if (!ctx) return fail(SKV_ERR_ARG, "skv_allocate: null ctx");
   if (B < 0 || Hkv <= 0 || Hkv > 128 || Tmax < 0 || Tmax > (1LL << 23))
     return fail(SKV_ERR_ARG, "skv_allocate: need B >= 0, 0 < Hkv <= 128, 0 <= Tmax <= 2^23");
@@ -255,6 +255,7 @@ int skv_allocate(skv_ctx* ctx, const uint16_t* K, int B, int Hkv, int64_t Tmax,
   p.tier_out = tier_out;
   p.row_of = row_of;
   p.indptr = page_indptr;
+  p.tier_indptr = page_tier_indptr;
   p.page_ids = page_ids;
   p.page_cap = page_cap;
   p.err = err_word;
@@ -303,7 +304,8 @@ int skv_encode(skv_ctx* ctx, const uint16_t* K, const uint16_t* V, int B, int Hk
 }
 
 static int decode_common(skv_ctx* ctx, const void* q, int q_dtype, int B, int Hq, int Hkv,
-                         const int32_t* page_indptr, const uint32_t* page_ids, const void* pool[3],
+                         const int32_t* page_indptr, const int32_t* page_tier_indptr,
+                         const uint32_t* page_ids, const void* pool[3],
                          const long long slots[3], bool dense, float* out, float* lse,
                          int32_t* err_word, void* workspace, size_t ws_bytes, int num_splits,
                          void* stream, const char* name) {
@@ -331,6 +333,7 @@ static int decode_common(skv_ctx* ctx, const void* q, int q_dtype, int B, int Hq
   p.Hq = Hq;
   p.Hkv = Hkv;
   p.indptr = page_indptr;
+  p.tier_indptr = page_tier_indptr;
   p.ids = page_ids;
   for (int t = 0; t < 3; ++t) {
     p.pool[t] = static_cast<const uint8_t*>(pool[t]);
@@ -364,13 +367,15 @@ static int decode_common(skv_ctx* ctx, const void* q, int q_dtype, int B, int Hq
 }
 
 int skv_decode_attention(skv_ctx* ctx, const void* q, int q_dtype, int B, int Hq, int Hkv,
-                         const int32_t* page_indptr, const uint32_t* page_ids,
-                         const skv_pools* pools, float* out, float* lse, int32_t* err_word,
-                         void* workspace, size_t ws_bytes, int num_splits, void* stream) {
+                         const int32_t* page_indptr, const int32_t* page_tier_indptr,
+                         const uint32_t* page_ids, const skv_pools* pools, float* out,
+                         float* lse, int32_t* err_word, void* workspace, size_t ws_bytes,
+                         int num_splits, void* stream) {
   if (!valid_pools(pools, 3)) return fail(SKV_ERR_ARG, "skv_decode_attention: bad pools");
   const void* pool[3] = {pools->base[0], pools->base[1], pools->base[2]};
   const long long slots[3] = {pools->slots[0], pools->slots[1], pools->slots[2]};
-  return decode_common(ctx, q, q_dtype, B, Hq, Hkv, page_indptr, page_ids, pool, slots, false, out,
+  return decode_common(ctx, q, q_dtype, B, Hq, Hkv, page_indptr, page_tier_indptr, page_ids, pool,
+                       slots, false, out,
                        lse, err_word, workspace, ws_bytes, num_splits, stream,
                        "skv_decode_attention");
 }
@@ -383,7 +388,8 @@ int skv_dense_decode_bf16(skv_ctx* ctx, const void* q, int q_dtype, int B, int H
     return fail(SKV_ERR_ARG, "skv_dense_decode_bf16: bad pool");
   const void* pools[3] = {pool, nullptr, nullptr};
   const long long slots[3] = {pool_slots, 0, 0};
-  return decode_common(ctx, q, q_dtype, B, Hq, Hkv, page_indptr, page_ids, pools, slots, true, out,
+  return decode_common(ctx, q, q_dtype, B, Hq, Hkv, page_indptr, nullptr, page_ids, pools, slots,
+                       true, out,
                        lse, err_word, workspace, ws_bytes, num_splits, stream,
                        "skv_dense_decode_bf16");
 }

@@ -4,14 +4,15 @@
 // and the dense bf16 paged-decode baseline built on the same skeleton.
 //
 // Work split ("split-K over pages"): the CSR page list of all units
-// (unit = (seq, kv head)) is one array of N pages; CTA c streams the run
-// [floor(c N / S), floor((c+1) N / S)) and produces one partial (m, l, o)
-// per unit it touches.  A unit covered by a single run is finished in
-// place; otherwise the partial goes to slot c + u of the workspace and the
-// CTA that brings the unit's ticket counter to its run count merges them
-// (log-sum-exp) -- no CTA ever waits for another.
+// (unit = (seq, kv head)) is one array of N pages, cut into S runs of about
+// equal streamed bytes (T0 pages cost 2.6x a T1 page); CTA c streams run c
+// and produces one partial (m, l, o) per unit it touches.  A unit covered
+// by a single run is finished in place; otherwise the partial goes to slot
+// c + u of the workspace and the CTA that brings the unit's ticket counter
+// to its run count merges them (log-sum-exp).  The only cross-CTA wait is
+// for the published split prefix, which the first CTA writes at its start.
 //
-// CTA = 8 consumer warps in kCG groups + 1 planner warp + kIss issuer
+// CTA = kCG groups of 4 consumer warps + 1 planner warp + kIss issuer
 // warps around one byte ring in shared memory.  The CTA's run is cut into
 // "items" of 64 tokens (64/P pages, never crossing a unit).  The planner
 // decodes page ids lane-parallel (a window of 64 pages at a time), places
@@ -34,6 +35,7 @@
 // straight from the page (pages store V in fragment order), B = P of the 16
 // rows x 8 heads (zero-padded beyond G), fp32 accumulation.
 #include <algorithm>
+#include <cstddef>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -43,9 +45,12 @@ namespace skv {
 #ifndef SKV_DECODE_ISSUERS
 #define SKV_DECODE_ISSUERS 2
 #endif
-constexpr int kNCW = 8;                       // consumer warps per CTA
-constexpr int kCG = 2;                        // consumer groups
-constexpr int kGW = kNCW / kCG;               // consumer warps per group
+#ifndef SKV_DECODE_GROUPS
+#define SKV_DECODE_GROUPS 3
+#endif
+constexpr int kGW = 4;                        // consumer warps per group
+constexpr int kCG = SKV_DECODE_GROUPS;        // consumer groups
+constexpr int kNCW = kCG * kGW;               // consumer warps per CTA
 constexpr int kIss = SKV_DECODE_ISSUERS;      // issuer warps
 constexpr int kPlannerWarp = kNCW;
 constexpr int kDecodeThreads = (kNCW + 1 + kIss) * 32;
@@ -55,7 +60,7 @@ constexpr int kPasses = kRowsPerWarp / 16;
 constexpr int kNSlot = 16;                    // items in flight, at most
 constexpr int kMaxIPP = kItemRows / 16;       // pages per item (P >= 16)
 constexpr int kMergeRuns = 128;               // runs per unit merged through shared memory
-static_assert(kCG == 1 || kCG == 2 || kCG == 4, "consumer groups: 1, 2 or 4");
+static_assert(kCG >= 1 && kCG <= 4, "consumer groups: 1..4");
 static_assert(kIss >= 1 && kIss <= 4, "issuers: 1..4");
 static_assert(kPasses >= 1 && kGW * kRowsPerWarp == kItemRows, "warp row split");
 
@@ -93,15 +98,22 @@ struct __align__(16) DecodeSmem {
   uint4 desc[kNSlot];                  // consumers' view of an item
   PageCopy copy[kNSlot][kMaxIPP];      // issuers' view of an item
   uint32_t copy_bytes[kNSlot];         // bytes of the item (0xFFFFFFFF: no more items)
+  unsigned long long scan[kDecodeThreads / 32];
+  unsigned long long cunit[5];         // merge: cost before each segment of a unit, end, total
+  long long useg[4];                   // merge: the unit's tier segment starts
+  long long run[2];                    // this CTA's pages [run[0], run[1])
   int abort_flag;
   int last_flag;
   int pad_[2];
-  float ml[kNCW][4][2];
-  float O[4][kHeadDim];
-  float q32[4][kHeadDim];
-  float mw[4][kMergeRuns];        // merge: per-run weights
+  __align__(16) float ml[kNCW][4][2];
+  __align__(16) float O[4][kHeadDim];
+  __align__(16) float q32[4][kHeadDim];   // read with 16-byte shared loads
+  __align__(16) float mw[4][kMergeRuns];  // merge: per-run weights
 };
 constexpr uint32_t kEndOfRun = 0xFFFFFFFFu;
+using DecodeSmemG4 = DecodeSmem<4, false>;
+static_assert(offsetof(DecodeSmemG4, q32) % 16 == 0, "q32 must be 16-byte aligned");
+static_assert(offsetof(DecodeSmemG4, desc) % 16 == 0, "desc must be 16-byte aligned");
 
 // Shared addresses of the ring, LUT1 (LUT2 follows it) and the fixed block
 // for a dynamic shared window [base, limit).  False when the ring would be
@@ -131,8 +143,113 @@ __host__ __device__ __forceinline__ bool smem_layout(uint32_t base, uint32_t lim
   return ring_sz >= min_ring;
 }
 
-__device__ __forceinline__ long long chunk_begin(int c, long long N, int S) {
-  return (long long)c * N / S;
+// ---------------------------------------------------------------- the split
+// The page list is cut into S runs of about equal streamed bytes (one per
+// CTA).  Segment k = 3 u + t holds the tier-t pages of unit u (all pages
+// count as tier 0 when no per-tier offsets are given); a page costs its
+// tier's payload bytes.  With C(g) the cost of the pages before page g and
+// C the total, page g belongs to run floor(C(g) S / C); run c starts at the
+// first page g with C(g) S >= c C.  Every CTA scans the segment costs
+// itself; the first to finish publishes the prefix to the workspace for the
+// merges (published flag: 0 none, 1 writing, 2 done).
+struct SplitInfo {
+  const int32_t* indptr;
+  const int32_t* tier_indptr;
+  int U;
+  int w[3];
+  __device__ __forceinline__ long long seg_start(int k) const {
+    if (tier_indptr) return tier_indptr[k];
+    const int u = k / 3;
+    return (k - 3 * u) == 0 ? indptr[u] : indptr[u + 1];
+  }
+  __device__ __forceinline__ unsigned long long weight(int k) const {
+    return (unsigned long long)w[k % 3];
+  }
+};
+
+// First page of the run that starts at cost target T (= run index x total)
+// among one unit's pages: seg[0..3] are the unit's tier segment starts,
+// cseg[0..3] the costs before them; clamped to [seg[0], seg[3]].
+__device__ __forceinline__ long long run_begin_in_unit(const SplitInfo& si,
+                                                       const long long* seg,
+                                                       const unsigned long long* cseg,
+                                                       unsigned long long T,
+                                                       unsigned long long S) {
+  for (int t = 0; t < 3; ++t) {
+    const unsigned long long lo = cseg[t] * S, hi = cseg[t + 1] * S;
+    if (T <= lo) return seg[t];
+    if (T <= hi) {
+      const unsigned long long ws = si.weight(t) * S;
+      return seg[t] + (long long)((T - lo + ws - 1) / ws);
+    }
+  }
+  return seg[3];
+}
+
+// This CTA's run [sm.run[0], sm.run[1]) (block-wide; contains barriers).
+// The first CTA to get here also publishes the cost before every segment
+// (and the total) to pub[0 .. 3U] and then sets *pub_flag to 2.
+template <class Smem>
+__device__ __noinline__ void find_run(const SplitInfo& si, int c, int S, Smem& sm,
+                                      unsigned long long* pub, int* pub_flag, int tid) {
+  constexpr int nt = kDecodeThreads;
+  const int nseg = 3 * si.U;
+  const int per = (nseg + nt - 1) / nt;
+  const int k0 = min(nseg, tid * per), k1 = min(nseg, k0 + per);
+  unsigned long long loc = 0;
+  for (int k = k0; k < k1; ++k)
+    loc += (unsigned long long)(si.seg_start(k + 1) - si.seg_start(k)) * si.weight(k);
+  const int lane = tid & 31, w = tid >> 5;
+  unsigned long long x = loc;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned long long y = __shfl_up_sync(0xFFFFFFFFu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) sm.scan[w] = x;
+  if (tid == 0) {
+    sm.run[0] = 0;  // the run boundaries that no segment claims (T = 0)
+    sm.run[1] = 0;
+    sm.last_flag = atomicCAS(pub_flag, 0, 1) == 0;  // this CTA publishes
+  }
+  __syncthreads();
+  unsigned long long before = x - loc, tot = 0;
+#pragma unroll
+  for (int i = 0; i < nt / 32; ++i) {
+    if (i < w) before += sm.scan[i];
+    tot += sm.scan[i];
+  }
+  const unsigned long long Su = (unsigned long long)S;
+  const unsigned long long T0 = (unsigned long long)c * tot, T1 = (unsigned long long)(c + 1) * tot;
+  const bool publish = sm.last_flag != 0;
+  unsigned long long cc = before;
+  for (int k = k0; k < k1; ++k) {
+    const long long a = si.seg_start(k), b = si.seg_start(k + 1);
+    const unsigned long long ws = si.weight(k) * Su;
+    const unsigned long long lo = cc * Su, hi = lo + (unsigned long long)(b - a) * ws;
+    if (lo < T0 && T0 <= hi) sm.run[0] = a + (long long)((T0 - lo + ws - 1) / ws);
+    if (lo < T1 && T1 <= hi) sm.run[1] = a + (long long)((T1 - lo + ws - 1) / ws);
+    if (publish) pub[k] = cc;
+    cc += (unsigned long long)(b - a) * si.weight(k);
+  }
+  if (publish) {
+    if (tid == 0) pub[nseg] = tot;
+    __threadfence();
+  }
+  __syncthreads();
+  if (publish && tid == 0) atomicExch(pub_flag, 2);
+}
+
+// Wait (bounded) until the segment-cost prefix is published; false on timeout.
+__device__ __forceinline__ bool wait_published(const int* pub_flag) {
+  const long long t0 = clock64();
+  while (true) {
+    int f;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(f) : "l"(pub_flag) : "memory");
+    if (f == 2) return true;
+    if (clock64() - t0 > kWaitLimitCycles) return false;
+    __nanosleep(256);
+  }
 }
 
 // ------------------------------------------------------ shared loads (PTX) --
@@ -159,27 +276,52 @@ __device__ __forceinline__ uint32_t lds16(uint32_t a) {
   return v;
 }
 
-// (code & 3) + 1 as a float, without a conversion instruction
-__device__ __forceinline__ float share_plus_one(uint32_t byte_or_bits) {
-  return __int_as_float(0x4B000000u | (byte_or_bits & 3u)) - 8388607.0f;
+// Logit accumulators of one row: G fp32 sums, as packed pairs for G >= 2
+// (fma.rn.f32x2: one issue slot for two heads).
+template <int G>
+struct RowAcc {
+  static constexpr int kN = G >= 2 ? G / 2 : 1;
+  float2 v[kN];
+  __device__ __forceinline__ void zero() {
+#pragma unroll
+    for (int i = 0; i < kN; ++i) v[i] = make_float2(0.0f, 0.0f);
+  }
+  __device__ __forceinline__ void to(float (&s)[G]) const {
+    if constexpr (G >= 2) {
+#pragma unroll
+      for (int i = 0; i < kN; ++i) {
+        s[2 * i] = v[i].x;
+        s[2 * i + 1] = v[i].y;
+      }
+    } else {
+      s[0] = v[0].x;
+    }
+  }
+};
+
+// s += w * (G fp32 LUT entries at shared address a), where x holds the
+// 2-bit share b as the float 2^23 + b and w = b + 1 (no conversion
+// instruction: the share bits are placed into the mantissa of 2^23).
+template <int G>
+__device__ __forceinline__ void lut_fma(uint32_t a, float x, RowAcc<G>& s) {
+  if constexpr (G == 4) {
+    const uint4 e = lds128(a);
+    const float2 w = __fadd2_rn(make_float2(x, x), make_float2(-8388607.0f, -8388607.0f));
+    s.v[0] = __ffma2_rn(w, make_float2(__uint_as_float(e.x), __uint_as_float(e.y)), s.v[0]);
+    s.v[1] = __ffma2_rn(w, make_float2(__uint_as_float(e.z), __uint_as_float(e.w)), s.v[1]);
+  } else if constexpr (G == 2) {
+    const uint2 e = lds64(a);
+    const float2 w = __fadd2_rn(make_float2(x, x), make_float2(-8388607.0f, -8388607.0f));
+    s.v[0] = __ffma2_rn(w, make_float2(__uint_as_float(e.x), __uint_as_float(e.y)), s.v[0]);
+  } else {
+    s.v[0].x = fmaf(x - 8388607.0f, __uint_as_float(lds32(a)), s.v[0].x);
+  }
 }
 
-// G fp32 LUT entries at a shared address
-template <int G>
-__device__ __forceinline__ void lut_fma(uint32_t a, float w, float (&s)[G]) {
-  if constexpr (G == 4) {
-    const uint4 v = lds128(a);
-    s[0] = fmaf(w, __uint_as_float(v.x), s[0]);
-    s[1] = fmaf(w, __uint_as_float(v.y), s[1]);
-    s[2] = fmaf(w, __uint_as_float(v.z), s[2]);
-    s[3] = fmaf(w, __uint_as_float(v.w), s[3]);
-  } else if constexpr (G == 2) {
-    const uint2 v = lds64(a);
-    s[0] = fmaf(w, __uint_as_float(v.x), s[0]);
-    s[1] = fmaf(w, __uint_as_float(v.y), s[1]);
-  } else {
-    s[0] = fmaf(w, __uint_as_float(lds32(a)), s[0]);
-  }
+// byte k of a word whose bytes each hold a 2-bit share, as the float 2^23 + share
+template <int K>
+__device__ __forceinline__ float share_byte(uint32_t spread) {
+  return __uint_as_float(__byte_perm(spread, 0x4B000000u, 0x7440u | K));
 }
 
 // Partial logits (times 16: shares enter as code + 1) of rows rA, rA + 8 of
@@ -187,15 +329,23 @@ __device__ __forceinline__ void lut_fma(uint32_t a, float w, float (&s)[G]) {
 // 4 (j ^ (row & 3)) + g as (angle6 << 2) | share2.
 template <int G>
 __device__ __forceinline__ void logits_t1(uint32_t pg, int P, int rA, int g, uint32_t lut,
-                                          float (&sA)[G], float (&sB)[G]) {
+                                          RowAcc<G>& sA, RowAcc<G>& sB) {
   const uint32_t cd = pg + kHdrBytes + 2 * P;
   const uint4 ca = lds128(cd + rA * 64 + 16 * g);
   const uint4 cb = lds128(cd + (rA + 8) * 64 + 16 * g);
   const uint32_t wa[4] = {ca.x, ca.y, ca.z, ca.w};
   const uint32_t wb[4] = {cb.x, cb.y, cb.z, cb.w};
+  uint32_t qa[4], qb[4];  // shares, one per byte
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    qa[k] = wa[k] & 0x03030303u;
+    qb[k] = wb[k] & 0x03030303u;
+  }
   const uint32_t x3 = rA & 3;  // rows rA and rA + 8 share it
   using L = LutGeom<G>;
-  // the table base is aligned to the table size: base | pair offset | code bits
+  // the table base is aligned to the table size: base | pair offset | code
+  // bits; the part of the pair offset that depends on j alone is added (an
+  // immediate of the shared load)
   uint32_t xo[4];
 #pragma unroll
   for (int jj = 0; jj < 4; ++jj) xo[jj] = lut | ((((uint32_t)jj ^ x3) * 4 + g) * L::kEnt);
@@ -205,9 +355,16 @@ __device__ __forceinline__ void logits_t1(uint32_t pg, int P, int rA, int g, uin
     const int sh = 8 * (j & 3) - (L::kCodeShift - 2);   // byte j sits at bit 8 (j & 3)
     const uint32_t xa = sh >= 0 ? (wa[j >> 2] >> sh) : (wa[j >> 2] << -sh);
     const uint32_t xb = sh >= 0 ? (wb[j >> 2] >> sh) : (wb[j >> 2] << -sh);
-    const uint32_t col = xo[j & 3] | ((j & ~3) * 4 * L::kEnt);
-    lut_fma<G>((xa & kMask) | col, share_plus_one(wa[j >> 2] >> (8 * (j & 3))), sA);
-    lut_fma<G>((xb & kMask) | col, share_plus_one(wb[j >> 2] >> (8 * (j & 3))), sB);
+    const uint32_t hi = (j & ~3) * 4 * L::kEnt;
+    float fa, fb;
+    switch (j & 3) {
+      case 0: fa = share_byte<0>(qa[j >> 2]); fb = share_byte<0>(qb[j >> 2]); break;
+      case 1: fa = share_byte<1>(qa[j >> 2]); fb = share_byte<1>(qb[j >> 2]); break;
+      case 2: fa = share_byte<2>(qa[j >> 2]); fb = share_byte<2>(qb[j >> 2]); break;
+      default: fa = share_byte<3>(qa[j >> 2]); fb = share_byte<3>(qb[j >> 2]); break;
+    }
+    lut_fma<G>(((xa & kMask) | xo[j & 3]) + hi, fa, sA);
+    lut_fma<G>(((xb & kMask) | xo[j & 3]) + hi, fb, sB);
   }
 }
 
@@ -215,12 +372,19 @@ __device__ __forceinline__ void logits_t1(uint32_t pg, int P, int rA, int g, uin
 // 4 (j ^ (row & 3)) + g, crumb j of bytes [32+4g, 36+4g) its share.
 template <int G>
 __device__ __forceinline__ void logits_t2(uint32_t pg, int P, int rA, int g, uint32_t lut,
-                                          float (&sA)[G], float (&sB)[G]) {
+                                          RowAcc<G>& sA, RowAcc<G>& sB) {
   const uint32_t cd = pg + kHdrBytes + 2 * P;
   const uint2 na = lds64(cd + rA * 48 + 8 * g);
   const uint2 nb = lds64(cd + (rA + 8) * 48 + 8 * g);
   const uint32_t ra = lds32(cd + rA * 48 + 32 + 4 * g);
   const uint32_t rb = lds32(cd + (rA + 8) * 48 + 32 + 4 * g);
+  // crumb j -> byte j >> 2 of word j & 3
+  uint32_t qa[4], qb[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    qa[k] = (ra >> (2 * k)) & 0x03030303u;
+    qb[k] = (rb >> (2 * k)) & 0x03030303u;
+  }
   const uint32_t x3 = rA & 3;
   using L = LutGeom<G>;
   uint32_t xo[4];
@@ -233,9 +397,16 @@ __device__ __forceinline__ void logits_t2(uint32_t pg, int P, int rA, int g, uin
     const uint32_t wa = (j < 8) ? na.x : na.y, wb = (j < 8) ? nb.x : nb.y;
     const uint32_t xa = sh >= 0 ? (wa >> sh) : (wa << -sh);
     const uint32_t xb = sh >= 0 ? (wb >> sh) : (wb << -sh);
-    const uint32_t col = xo[j & 3] | ((j & ~3) * 4 * L::kEnt);
-    lut_fma<G>((xa & kMask) | col, share_plus_one(ra >> (2 * j)), sA);
-    lut_fma<G>((xb & kMask) | col, share_plus_one(rb >> (2 * j)), sB);
+    const uint32_t hi = (j & ~3) * 4 * L::kEnt;
+    float fa, fb;
+    switch (j >> 2) {
+      case 0: fa = share_byte<0>(qa[j & 3]); fb = share_byte<0>(qb[j & 3]); break;
+      case 1: fa = share_byte<1>(qa[j & 3]); fb = share_byte<1>(qb[j & 3]); break;
+      case 2: fa = share_byte<2>(qa[j & 3]); fb = share_byte<2>(qb[j & 3]); break;
+      default: fa = share_byte<3>(qa[j & 3]); fb = share_byte<3>(qb[j & 3]); break;
+    }
+    lut_fma<G>(((xa & kMask) | xo[j & 3]) + hi, fa, sA);
+    lut_fma<G>(((xb & kMask) | xo[j & 3]) + hi, fb, sB);
   }
 }
 
@@ -320,10 +491,24 @@ __device__ __forceinline__ float reduce_scatter(float (&s)[G], int g) {
 }
 
 struct WarpState {
-  float m;          // running max (log2 domain) of head g % G
+  float m;          // running max (log2 domain) of head g % G, or kNoMax
   float l;          // partial denominator of (token slot t, head g % G)
   float acc[8][4];  // O^T fragments: [m-tile][c0..c3]
 };
+
+// Start value of the running max: finite, so that exp2 of (-inf - m) is 0
+// and never NaN; any real logit is far above it.
+constexpr float kNoMax = -1.0e30f;
+// The running max is raised (and the accumulators rescaled) only when a
+// logit exceeds it by more than this (log2 units): weights then stay below
+// 2^4 and most 16-row steps skip the rescale.
+constexpr float kLazyMax = 4.0f;
+
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 
 // Online softmax of 16 rows and P.V into the accumulators.
 // lA / lB: log2-domain logits of rows t and t + 8 (head g % G) or -inf.
@@ -335,15 +520,12 @@ __device__ __forceinline__ void softmax_pv(float lA, float lB, float vsA, float 
   cm = fmaxf(cm, __shfl_xor_sync(0xFFFFFFFFu, cm, 4));
   cm = fmaxf(cm, __shfl_xor_sync(0xFFFFFFFFu, cm, 8));
   cm = fmaxf(cm, __shfl_xor_sync(0xFFFFFFFFu, cm, 16));
-  const float m_new = fmaxf(st.m, cm);
-  const bool fin = m_new != -INFINITY;
-  const float alpha = (fin && st.m != m_new) ? exp2f(st.m - m_new) : 1.0f;
-  const float pA = (lA != -INFINITY) ? exp2f(lA - m_new) : 0.0f;
-  const float pB = (lB != -INFINITY) ? exp2f(lB - m_new) : 0.0f;
-  st.l = st.l * alpha + (pA + pB);
-  st.m = m_new;
   const int gq = lane >> 2, t4 = lane & 3;
-  if (__any_sync(0xFFFFFFFFu, alpha != 1.0f)) {
+  if (__any_sync(0xFFFFFFFFu, cm > st.m + kLazyMax)) {
+    const float m_new = fmaxf(st.m, cm);
+    const float alpha = ex2_approx(st.m - m_new);  // 0 when st.m is kNoMax
+    st.l *= alpha;
+    st.m = m_new;
     const int n0 = 2 * t4, n1 = 2 * t4 + 1;
     const float a0 = __shfl_sync(0xFFFFFFFFu, alpha, n0 < G ? n0 : 0);
     const float a1 = __shfl_sync(0xFFFFFFFFu, alpha, n1 < G ? n1 : 0);
@@ -355,6 +537,8 @@ __device__ __forceinline__ void softmax_pv(float lA, float lB, float vsA, float 
       st.acc[mt][3] *= a1;
     }
   }
+  const float pA = ex2_approx(lA - st.m), pB = ex2_approx(lB - st.m);  // -inf -> 0
+  st.l += pA + pB;
   const float ppA = pA * vsA, ppB = pB * vsB;
   // B fragment (k16 x n8): k = rows 2t4, 2t4+1 | 8+2t4, 9+2t4, n = head gq
   const int src = 8 * t4 + (gq < G ? gq : 0);
@@ -421,6 +605,9 @@ __device__ __forceinline__ void process_rows(const DecodeParams& p, uint32_t pg,
     sA[h] = 0.0f;
     sB[h] = 0.0f;
   }
+  RowAcc<G> rA2, rB2;
+  rA2.zero();
+  rB2.zero();
   const uint32_t vsec_dense = pg + kHdrBytes + 256 * P + (row0 >> 3) * 2048;
   if constexpr (DENSE) {
     logits_dense<G, true>(pg, rA, g, q32, sA, sB);
@@ -438,9 +625,11 @@ __device__ __forceinline__ void process_rows(const DecodeParams& p, uint32_t pg,
     } else {
       const bool t1 = tier == SKV_TIER_T1;
       if (t1)
-        logits_t1<G>(pg, P, rA, g, lut1, sA, sB);
+        logits_t1<G>(pg, P, rA, g, lut1, rA2, rB2);
       else
-        logits_t2<G>(pg, P, rA, g, lut2, sA, sB);
+        logits_t2<G>(pg, P, rA, g, lut2, rA2, rB2);
+      rA2.to(sA);
+      rB2.to(sB);
       const float a = reduce_scatter<G>(sA, g), b = reduce_scatter<G>(sB, g);
       const int cb = t1 ? 64 : 48;
       const uint32_t rs = pg + kHdrBytes, ss = pg + kHdrBytes + (2 + cb) * P;
@@ -468,8 +657,18 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   const int warp = tid >> 5, lane = tid & 31;
   const int c = blockIdx.x;
   const int U = p.B * p.Hkv;
-  const long long N = p.indptr[U];
-  const long long g0 = chunk_begin(c, N, p.S), g1 = chunk_begin(c + 1, N, p.S);
+  SplitInfo si;
+  si.indptr = p.indptr;
+  si.tier_indptr = p.tier_indptr;
+  si.U = U;
+  si.w[0] = p.payload[0];
+  si.w[1] = DENSE ? p.payload[0] : p.payload[1];
+  si.w[2] = DENSE ? p.payload[0] : p.payload[2];
+  const DecodeWs wsl = decode_ws(p.S, U, G);
+  uint8_t* const wsb = reinterpret_cast<uint8_t*>(p.part);
+  int* const counters = reinterpret_cast<int*>(wsb + wsl.ctr);
+  int* const pub_flag = reinterpret_cast<int*>(wsb + wsl.flag);
+  unsigned long long* const pub = reinterpret_cast<unsigned long long*>(wsb + wsl.pub);
   const int ipp = kItemRows >> p.log2P;
   // the largest item: ipp pages of the largest payload
   int maxpay = p.payload[0];
@@ -502,8 +701,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       if (p.lse && lane < G) p.lse[o + lane] = -INFINITY;
     }
   }
-  __syncthreads();
-  if (g0 >= g1 || !plan_ok) return;
+  if (!plan_ok) return;  // uniform: every thread computed the same layout
+  find_run(si, c, p.S, sm, pub, pub_flag, tid);
+  const long long g0 = sm.run[0], g1 = sm.run[1];
+  if (g0 >= g1) return;
 
   // first unit whose pages reach past g0: largest u with indptr[u] <= g0
   int lo = 0, hi = U;
@@ -697,7 +898,6 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   const uint32_t q32 = smem_u32(sm.q32);
   float* lut1p = reinterpret_cast<float*>(smem_raw + (lut1 - base));
   float* lut2p = reinterpret_cast<float*>(smem_raw + (lut2 - base));
-  int* counters = reinterpret_cast<int*>(p.part + (long long)(p.S + U) * G * kPartStride);
   int it = 0;  // item index within the run
   bool ok = true;
   for (int u = u0; u < U; ++u) {
@@ -746,7 +946,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       named_bar_sync(1, nct);
     }
     WarpState st;
-    st.m = -INFINITY;
+    st.m = kNoMax;
     st.l = 0.0f;
 #pragma unroll
     for (int mt = 0; mt < 8; ++mt)
@@ -755,7 +955,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
 
     const int nitems = (int)((b - a + ipp - 1) / ipp);
     // this group's items of the unit: it + i with (it + i) % kCG == grp
-    for (int i = (grp - it) & (kCG - 1); i < nitems; i += kCG) {
+    for (int i = ((grp - it % kCG) + kCG) % kCG; i < nitems; i += kCG) {
       const int itm = it + i, s = itm % kNSlot;
       if (ok && !mbar_wait_bounded(smem_u32(&sm.full[s]), (uint32_t)((itm / kNSlot) & 1),
                                    &sm.abort_flag)) {
@@ -793,7 +993,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     l += __shfl_xor_sync(0xFFFFFFFFu, l, 8);
     l += __shfl_xor_sync(0xFFFFFFFFu, l, 16);
     if (lane < G) {
-      sm.ml[warp][lane][0] = st.m;
+      sm.ml[warp][lane][0] = st.m <= kNoMax ? -INFINITY : st.m;  // no row seen: -inf
       sm.ml[warp][lane][1] = l;
     }
     named_bar_sync(1, nct);
@@ -829,17 +1029,45 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
           }
       }
     }
-    // runs of the page list that touch unit u
-    const long long S = p.S;
-    const int c0 = (int)(((iu0 + 1) * S - 1) / N);
-    const int c1 = (int)((iu1 * S - 1) / N);
-    int nruns = 0;
-    if (S <= N) {
-      nruns = c1 - c0 + 1;
-    } else {
-      for (int cc = c0; cc <= c1; ++cc)
-        nruns += chunk_begin(cc, N, p.S) != chunk_begin(cc + 1, N, p.S);
+    // runs of the page list that touch unit u: run c holds page g when
+    // floor(C(g) S / total) == c; the first and the last page of u give the
+    // range, a run strictly inside it may be empty (a page costlier than a run)
+    if (tid == 0) {
+#pragma unroll
+      for (int t = 0; t < 4; ++t) sm.useg[t] = si.seg_start(3 * u + t);
+      if (wait_published(pub_flag)) {
+#pragma unroll
+        for (int t = 0; t < 4; ++t) sm.cunit[t] = __ldcg(pub + 3 * u + t);
+        sm.cunit[4] = __ldcg(pub + 3 * U);
+      } else {
+        report(p.err, SKV_ERR_TIMEOUT);
+#pragma unroll
+        for (int t = 0; t < 5; ++t) sm.cunit[t] = 0;
+      }
     }
+    named_bar_sync(1, nct);
+    const unsigned long long Su = (unsigned long long)p.S, ctot = sm.cunit[4];
+    int c0 = c, c1 = c;
+    if (ctot > 0) {
+      int tl = 2;  // tier of the unit's last page
+      while (tl > 0 && sm.useg[tl] == iu1) --tl;
+      c0 = (int)(sm.cunit[0] * Su / ctot);
+      c1 = (int)((sm.cunit[3] - si.weight(tl)) * Su / ctot);
+    }
+    // when no page costs more than a run (the usual case) every run from c0
+    // to c1 holds pages of u; otherwise a run inside may be empty
+    const unsigned long long wmax = (unsigned long long)max(si.w[0], max(si.w[1], si.w[2]));
+    const bool dense_runs = wmax * Su <= ctot;
+    auto run_has_u = [&](int cc) -> bool {
+      if (dense_runs || cc == c0 || cc == c1) return true;
+      const long long ra = run_begin_in_unit(si, sm.useg, sm.cunit, (unsigned long long)cc * ctot, Su);
+      const long long rb =
+          run_begin_in_unit(si, sm.useg, sm.cunit, (unsigned long long)(cc + 1) * ctot, Su);
+      return rb > ra;
+    };
+    int nruns = c1 - c0 + 1;
+    if (!dense_runs)
+      for (int cc = c0 + 1; cc < c1; ++cc) nruns -= run_has_u(cc) ? 0 : 1;
     const long long obase = (long long)bb * p.Hq + (long long)hkv * G;
     if (nruns == 1) {
       for (int i = tid; i < G * kHeadDim; i += nct) {
@@ -881,7 +1109,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
             const int n = i / nr, r = i % nr;
             const int cc = c0 + r;
             float m = -INFINITY;  // an empty run contributes nothing
-            if (!(S > N && chunk_begin(cc, N, p.S) == chunk_begin(cc + 1, N, p.S)))
+            if (run_has_u(cc))
               m = __ldcg(p.part + (long long)(cc + u) * G * kPartStride + n * kPartStride);
             sm.mw[n][r] = m;
           }
@@ -929,7 +1157,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
             const int n = i / kHeadDim, d = i % kHeadDim;
             float M = -INFINITY, L = 0.0f, O = 0.0f;
             for (int cc = c0; cc <= c1; ++cc) {
-              if (S > N && chunk_begin(cc, N, p.S) == chunk_begin(cc + 1, N, p.S)) continue;
+              if (!run_has_u(cc)) continue;
               const float* pp = p.part + (long long)(cc + u) * G * kPartStride + n * kPartStride;
               const float m = __ldcg(pp), lc = __ldcg(pp + 1), oc = __ldcg(pp + 4 + d);
               if (m == -INFINITY) continue;
@@ -975,8 +1203,10 @@ cudaError_t launch_decode_g(const DecodeParams& p, cudaStream_t stream, cudaEven
     if (dev >= 0 && dev < 64) configured[dev] = smem;
   }
   const int U = p.B * p.Hkv;
-  int* counters = reinterpret_cast<int*>(p.part + (long long)(p.S + U) * G * kPartStride);
-  e = cudaMemsetAsync(counters, 0, sizeof(int) * (size_t)U, stream);
+  // ticket counters and the split's publication flag start at zero
+  const DecodeWs wsl = decode_ws(p.S, U, G);
+  e = cudaMemsetAsync(reinterpret_cast<uint8_t*>(p.part) + wsl.ctr, 0, sizeof(int) * ((size_t)U + 1),
+                      stream);
   if (e != cudaSuccess) return e;
   decode_kernel<G, DENSE><<<p.S, kDecodeThreads, p.smem_bytes, stream>>>(p);
   e = cudaGetLastError();

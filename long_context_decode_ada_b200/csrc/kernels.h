@@ -14,6 +14,7 @@ struct DecodeParams {
   int q_bf16;
   int B, Hq, Hkv;
   const int32_t* indptr;
+  const int32_t* tier_indptr;  // [3U + 1] page offsets per (unit, tier) segment, or NULL
   const uint32_t* ids;
   const uint8_t* pool[3];
   long long slots[3];
@@ -41,6 +42,7 @@ struct EncodeParams {
   const uint8_t* tier;
   const int32_t* row_of;
   const int32_t* indptr;
+  const int32_t* tier_indptr;  // [3U + 1] page offsets per (unit, tier) segment, or NULL
   const uint32_t* ids;
   uint8_t* pool[3];
   long long slots[3];
@@ -70,6 +72,7 @@ struct AllocParams {
   uint8_t* tier_out;
   int32_t* row_of;
   int32_t* indptr;
+  int32_t* tier_indptr;       // [3U + 1] per (unit, tier) or NULL
   uint32_t* page_ids;
   long long page_cap;
   int32_t* err;
@@ -84,6 +87,21 @@ struct AllocParams {
   int nseg;
   int dense;                  // dense-bf16 baseline packing (every token kept, tier 0)
 };
+
+// Decode workspace: partials [(S + U) G][kPartStride] fp32, then U ticket
+// counters and the split's publication flag (int32, zeroed by every call),
+// then the published segment-cost prefix (uint64 [3U + 1]).
+struct DecodeWs {
+  size_t ctr, flag, pub, bytes;
+};
+__host__ __device__ inline DecodeWs decode_ws(long long S, long long U, int G) {
+  DecodeWs w;
+  w.ctr = (size_t)(S + U) * G * kPartStride * 4;
+  w.flag = w.ctr + 4 * (size_t)U;
+  w.pub = (w.flag + 4 + 7) / 8 * 8;
+  w.bytes = w.pub + 8 * (size_t)(3 * U + 1);
+  return w;
+}
 
 size_t decode_fixed_smem(int G, bool dense);
 // True when smem_bytes of dynamic shared memory hold the decode kernel's

@@ -59,11 +59,11 @@ _SIGS = {
     "skv_device_info": (_i, [_p, C.POINTER(_i), C.POINTER(_i)]),
     "skv_workspace_size": (_i, [_p, _i, _i, _i, _i, _i64, _i, C.POINTER(_sz)]),
     "skv_allocate": (_i, [_p, _p, _i, _i, _i64, _p, _p, _p, _i, _p, _p, C.POINTER(SkvFreeLists),
-                          C.POINTER(SkvPools), _p, _p, _p, _p, _i64, _p, _p, _sz, _p]),
+                          C.POINTER(SkvPools), _p, _p, _p, _p, _p, _i64, _p, _p, _sz, _p]),
     "skv_encode": (_i, [_p, _p, _p, _i, _i, _i64, _p, _p, _p, _p, _p, C.POINTER(SkvPools), _p,
                         _p]),
-    "skv_decode_attention": (_i, [_p, _p, _i, _i, _i, _i, _p, _p, C.POINTER(SkvPools), _p, _p, _p,
-                                  _p, _sz, _i, _p]),
+    "skv_decode_attention": (_i, [_p, _p, _i, _i, _i, _i, _p, _p, _p, C.POINTER(SkvPools), _p, _p,
+                                  _p, _p, _sz, _i, _p]),
     "skv_dense_pack_bf16": (_i, [_p, _p, _p, _i, _i, _i64, _p, _p, _i64, _p, _i64, _p, _p, _i64,
                                  _p, _p, _sz, _p]),
     "skv_dense_decode_bf16": (_i, [_p, _p, _i, _i, _i, _i, _p, _p, _p, _i64, _p, _p, _p, _p, _sz,
@@ -194,6 +194,9 @@ class PagedCache:
         self.tier = torch.empty((B, Hkv, Tmax), dtype=torch.uint8, device=self.device)
         self.row_of = torch.empty((B, Hkv, Tmax), dtype=torch.int32, device=self.device)
         self.page_indptr = torch.zeros(B * Hkv + 1, dtype=torch.int32, device=self.device)
+        self.page_tier_indptr = torch.zeros(3 * B * Hkv + 1, dtype=torch.int32, device=self.device)
+        # the decode cuts its work by streamed bytes (False: by page count)
+        self.split_by_bytes = True
         self.page_ids = torch.zeros(max(1, self.page_cap), dtype=torch.int32, device=self.device)
         self.err = torch.zeros(1, dtype=torch.int32, device=self.device)
         self._ws_alloc = torch.empty(ctx.workspace_size(WS_ALLOCATE, B, Hkv, 0, Tmax),
@@ -212,7 +215,8 @@ class PagedCache:
         _check(lib().skv_allocate(
             self.ctx.handle, _ptr(K), self.B, self.Hkv, self.Tmax, _ptr(seq_lens), _ptr(utility),
             _ptr(protect), mode, _ptr(budget), _ptr(quota), C.byref(fl), C.byref(self._pools_c),
-            _ptr(self.tier), _ptr(self.row_of), _ptr(self.page_indptr), _ptr(self.page_ids),
+            _ptr(self.tier), _ptr(self.row_of), _ptr(self.page_indptr),
+            _ptr(self.page_tier_indptr), _ptr(self.page_ids),
             self.page_cap, _ptr(self.err), _ptr(self._ws_alloc), self._ws_alloc.numel(),
             _stream(stream)))
 
@@ -236,6 +240,7 @@ class PagedCache:
             workspace = self.workspace(Hq, num_splits)
         _check(lib().skv_decode_attention(
             self.ctx.handle, _ptr(q), q_dtype, self.B, Hq, self.Hkv, _ptr(self.page_indptr),
+            _ptr(self.page_tier_indptr) if self.split_by_bytes else None,
             _ptr(self.page_ids), C.byref(self._pools_c), _ptr(out), _ptr(lse), _ptr(self.err),
             _ptr(workspace), workspace.numel(), num_splits, _stream(stream)))
         return out, lse
@@ -262,6 +267,9 @@ class DenseCache:
                                 device=self.device)
         self.page_cap = self.pool_slots
         self.page_indptr = torch.zeros(B * Hkv + 1, dtype=torch.int32, device=self.device)
+        self.page_tier_indptr = torch.zeros(3 * B * Hkv + 1, dtype=torch.int32, device=self.device)
+        # the decode cuts its work by streamed bytes (False: by page count)
+        self.split_by_bytes = True
         self.page_ids = torch.zeros(max(1, self.page_cap), dtype=torch.int32, device=self.device)
         self.err = torch.zeros(1, dtype=torch.int32, device=self.device)
         self._ws_alloc = torch.empty(ctx.workspace_size(WS_ALLOCATE, B, Hkv, 0, Tmax),

@@ -24,6 +24,21 @@ def run_gpu(w, num_splits=0, ctx=None, decode=True):
     return res
 
 
+def tier_indptr_of(indptr, ids):
+    """CSR offsets per (unit, tier) segment 3u + t of a page table whose
+    units list their T0 pages, then T1, then T2 (checked here)."""
+    U = len(indptr) - 1
+    out = np.zeros(3 * U + 1, np.int32)
+    for u in range(U):
+        a, b = int(indptr[u]), int(indptr[u + 1])
+        tiers = np.asarray(ids[a:b], np.uint32) >> 30
+        assert np.all(np.diff(tiers.astype(np.int64)) >= 0), "unit pages not ordered by tier"
+        for t in range(3):
+            out[3 * u + t] = a + int((tiers < t).sum())
+    out[3 * U] = int(indptr[-1])
+    return out
+
+
 def compare_store(w, g, ref):
     """Tiers, row map, page table and every used page's payload bytes."""
     cache = g["cache"]
@@ -36,6 +51,9 @@ def compare_store(w, g, ref):
     n = int(ip[-1])
     ids = cache.page_ids[:n].cpu().numpy().view(np.uint32)
     assert np.array_equal(ids, ref["page_ids"][:n]), "page_ids mismatch"
+    tip = cache.page_tier_indptr.cpu().numpy()
+    assert np.array_equal(tip, tier_indptr_of(ref["page_indptr"], ref["page_ids"])), \
+        "page_tier_indptr mismatch"
     pools_gpu = [p.cpu().numpy() for p in cache.pools]
     bad = 0
     for pid in ids:
@@ -75,6 +93,8 @@ def upload_oracle_store(ctx, w, ref):
         src = torch.from_numpy(ref["pools"][t])
         cache.pools[t][: src.numel()].copy_(src.to(cache.device))
     cache.page_indptr.copy_(torch.from_numpy(ref["page_indptr"]).to(cache.device))
+    cache.page_tier_indptr.copy_(torch.from_numpy(
+        tier_indptr_of(ref["page_indptr"], ref["page_ids"])).to(cache.device))
     n = int(ref["page_indptr"][-1])
     if n:
         cache.page_ids[:n].copy_(torch.from_numpy(ref["page_ids"][:n].view(np.int32)).to(

@@ -70,13 +70,13 @@ def test_argument_errors_without_gpu():
     assert e.value.code == skv.SKV_ERR_ARG
     # decode with G = 8 is refused on the host
     pools = skv.SkvPools()
-    rc = L.skv_decode_attention(ctx.handle, None, skv.Q_BF16, 1, 64, 8, None, None,
+    rc = L.skv_decode_attention(ctx.handle, None, skv.Q_BF16, 1, 64, 8, None, None, None,
                                 C.byref(pools), None, None, None, None, 0, 0, None)
     assert rc == skv.SKV_ERR_ARG
     # unaligned pool base is refused
     pools.base[0] = 64
     pools.slots[0] = 1
-    rc = L.skv_decode_attention(ctx.handle, None, skv.Q_BF16, 1, 8, 8, None, None,
+    rc = L.skv_decode_attention(ctx.handle, None, skv.Q_BF16, 1, 8, 8, None, None, None,
                                 C.byref(pools), None, None, None, None, 0, 0, None)
     assert rc == skv.SKV_ERR_ARG
 
@@ -84,7 +84,13 @@ def test_argument_errors_without_gpu():
 def test_workspace_sizes():
     ctx = skv.Context(64)
     sm, splits = ctx.device_info()
+    def expect(S, U, G):
+        # partials, U ticket counters + the split flag (8-byte aligned), cost prefix
+        ctr = (S + U) * G * 132 * 4
+        pub = (ctr + 4 * U + 4 + 7) // 8 * 8
+        return pub + 8 * (3 * U + 1)
     n = ctx.workspace_size(skv.WS_DECODE, 1, 8, 32, 0, 0)
-    assert n == (splits + 8) * 4 * 132 * 4 + 8 * 4
-    assert ctx.workspace_size(skv.WS_DECODE, 1, 8, 32, 0, 10) == (10 + 8) * 4 * 132 * 4 + 8 * 4
+    assert n == expect(splits, 8, 4)
+    assert ctx.workspace_size(skv.WS_DECODE, 1, 8, 32, 0, 10) == expect(10, 8, 4)
+    assert ctx.workspace_size(skv.WS_DECODE, 3, 3, 6, 0, 10) == expect(10, 9, 2)
     assert ctx.workspace_size(skv.WS_ALLOCATE, 2, 8, 0, 1000) > 2 * 8 * 1000 * 4

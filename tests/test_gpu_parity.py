@@ -80,6 +80,26 @@ def test_split_counts_do_not_change_results(splits):
     full_check(w, num_splits=splits, decode_oracle_pages=False)
 
 
+@pytest.mark.parametrize("splits", [1, 3, 148, 5000])
+def test_split_by_bytes_and_by_pages_agree_with_oracle(splits):
+    """The decode cuts the page list into runs of equal bytes (per-tier
+    offsets given) or of equal page counts (offsets withheld); both, at run
+    counts from one up to far more runs than pages (empty runs, pages
+    costlier than a run), match the oracle."""
+    lens = [900, 64, 2500, 17]
+    w = wl.custom(63, 4, 2, 4, 64, lens, wl.MODE_QUOTA,
+                  quota=[[T // 3, T // 3, T // 6] for T in lens], scatter=True)
+    ref = oracle.run_workload(w)
+    g = run_gpu(w, num_splits=splits)
+    cache = g["cache"]
+    for by_bytes in (True, False):
+        cache.split_by_bytes = by_bytes
+        out, lse = cache.decode(g["dev"]["q"], g["dev"]["q_dtype"], w.Hq, num_splits=splits)
+        cache.check()
+        assert_close(out.cpu().numpy(), ref["out"], f"out (by_bytes={by_bytes})")
+        assert_close(lse.cpu().numpy(), ref["lse"], f"lse (by_bytes={by_bytes})")
+
+
 def test_edge_cases_empty_dropped_single():
     # seq 0 empty, seq 1 has every token dropped, seq 2 a single token, seq 3 ragged tail
     lens = [0, 40, 1, 77]
