@@ -24,6 +24,7 @@ import datetime
 import json
 import math
 import os
+import re
 import subprocess
 import sys
 import threading
@@ -158,6 +159,23 @@ def written_partials(indptr: np.ndarray, ids: np.ndarray, payload, S: int) -> in
     return n
 
 
+def max_over_ranks(elapsed_ms: float, device) -> float:
+    """The max over ranks of a device-timed region (every rank gets it); the
+    value itself on a single process."""
+    dist = torch.distributed
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return elapsed_ms
+    t = torch.tensor([elapsed_ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_value(units_per_rank: int, world: int, ms_per_step: float) -> float:
+    """Whole-job throughput: every rank decodes its own store of
+    units_per_rank token-heads per step (weak scaling, no exchange)."""
+    return world * units_per_rank / (ms_per_step * 1e-3)
+
+
 def clone_cache(cache):
     from long_context_decode_ada_b200 import skv
     c2 = skv.PagedCache(cache.ctx, cache.B, cache.Hkv, cache.Tmax, cache.pool_slots,
@@ -284,12 +302,9 @@ def run_skv(args, rank, world, local_rank):
     clocks = sampler.stop()
     elapsed_ms = t0.elapsed_time(t1)
     caches[0].check()
-    if world > 1:
-        tt = torch.tensor([elapsed_ms], device=dev)
-        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-        elapsed_ms = float(tt.item())
+    elapsed_ms = max_over_ranks(elapsed_ms, dev)
     ms_per_step = elapsed_ms / args.steps
-    value = world * resident / (ms_per_step * 1e-3)
+    value = whole_job_value(resident, world, ms_per_step)
     step_ms = [a.elapsed_time(c) for a, b, c in ev]
     kern_ms = [a.elapsed_time(b) for a, b, c in ev]
     kern_ms_avg = float(np.mean(kern_ms))
@@ -372,7 +387,7 @@ def run_skv(args, rank, world, local_rank):
 
     cpu = None
     if rank == 0 and not args.no_cpu:
-        cpu = cpu_baseline(T_sample=65536)
+        cpu = cpu_baseline(T_sample=args.seq_len)
 
     if rank == 0:
         line = {
@@ -390,13 +405,13 @@ def run_skv(args, rank, world, local_rank):
                                  "T2": int(pages_per_tier[2])},
                        "parallelism": f"{world} independent replicas (one per GPU)"},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak, "traffic": None,
+                         "frac": achieved / peak, "traffic": profiled_traffic(),
                          "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)",
                          "kernel": "decode_kernel<4,false>", "kernel_ms": kern_ms_avg,
                          "algorithmic_bytes": algo_bytes, "payload_bytes_streamed": payload_bytes},
             "cpu_baseline": cpu,
             "e2e": e2e,
-            "gpu_launches": 2 * args.steps,
+            "gpu_launches": args.steps,  # one decode_kernel per step (plus a driver memset)
             "clocks": clocks,
             "dense_bf16_baseline": dense,
             "ingest": {"allocate_ms": alloc_ms, "encode_ms": enc_ms, "gen_s": t_gen},
@@ -405,26 +420,62 @@ def run_skv(args, rank, world, local_rank):
         print(json.dumps(line), flush=True)
 
 
+def decode_source_digest() -> str:
+    """sha256 of the decode kernel's sources (decides whether a profiled
+    DRAM traffic figure still describes the kernel that runs)."""
+    import hashlib
+    h = hashlib.sha256()
+    for f in ("decode.cu", "common.cuh", "kernels.h"):
+        with open(os.path.join(ROOT, "long_context_decode_ada_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def profiled_traffic():
+    """dram__bytes_read.sum + dram__bytes_write.sum per decode launch from the
+    committed ncu summary, or None when the kernel changed since it was taken."""
+    path = os.path.join(ROOT, "profiles", "decode_kernel_long_context.md")
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    vals = dict(re.findall(r"^- (traffic_bytes_per_launch|decode_source_sha256): (\S+)$", text,
+                           re.M))
+    if vals.get("decode_source_sha256") != decode_source_digest():
+        return None
+    try:
+        return int(vals["traffic_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
 # -------------------------------------------------------- oracle (CPU) ----
 
-def cpu_baseline(T_sample: int, repeats: int = 1):
+def cpu_baseline(T_sample: int, min_seconds: float = 10.0):
     """Time the oracle's decode (as it stands) on the host cores on a bounded
-    sample of the same workload: the long-context recipe at T_sample tokens.
-    The sample's tiers come from the oracle's own allocation."""
+    sample of the same workload: the long-context recipe at T_sample tokens,
+    decoded repeatedly until at least min_seconds of CPU work have run.  The
+    sample's tiers come from the oracle's own allocation."""
     import oracle
     from long_context_decode_ada_b200 import workloads as wl
     w = wl.long_context(seed=1, T=T_sample)
     tier = oracle.allocate(w.B, w.Hkv, w.Tmax, w.d, w.P, w.seq_lens, w.K, w.utility, w.protect,
                            w.mode, w.budget, w.quota)
     resident = int((tier != 3).sum())
+    reps = 0
     t = time.perf_counter()
-    for _ in range(repeats):
+    while True:
         oracle.decode(w.B, w.Hq, w.Hkv, w.Tmax, w.d, w.seq_lens, w.K, w.V, tier, w.q, w.q_dtype)
-    dt = (time.perf_counter() - t) / repeats
+        reps += 1
+        if time.perf_counter() - t >= min_seconds:
+            break
+    total = time.perf_counter() - t
+    dt = total / reps
     return {"value": resident / dt, "unit": UNIT, "cores": oracle.threads(), "kind": "oracle",
             "sample": f"long_context recipe at T={T_sample} (B=1, 8 KV / 32 query heads, "
-                      f"{resident} resident token-heads), oracle decode only, {dt:.2f} s",
-            "seconds": dt}
+                      f"{resident} resident token-heads), oracle decode only, {reps} decodes "
+                      f"in {total:.1f} s",
+            "seconds": total}
 
 
 def run_reference(args, rank, world):

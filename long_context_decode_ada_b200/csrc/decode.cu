@@ -102,6 +102,8 @@ struct __align__(16) DecodeSmem {
   unsigned long long cunit[5];         // merge: cost before each segment of a unit, end, total
   long long useg[4];                   // merge: the unit's tier segment starts
   long long run[2];                    // this CTA's pages [run[0], run[1])
+  int unit0;                           // the unit of page run[0]
+  int pad_unit;
   int abort_flag;
   int last_flag;
   int pad_[2];
@@ -238,6 +240,11 @@ __device__ __noinline__ void find_run(const SplitInfo& si, int c, int S, Smem& s
   }
   __syncthreads();
   if (publish && tid == 0) atomicExch(pub_flag, 2);
+  // the unit of the run's first page (its segment holds it)
+  const long long g0 = sm.run[0];
+  for (int k = k0; k < k1; ++k)
+    if (si.seg_start(k) <= g0 && g0 < si.seg_start(k + 1)) sm.unit0 = k / 3;
+  __syncthreads();
 }
 
 // Wait (bounded) until the segment-cost prefix is published; false on timeout.
@@ -706,13 +713,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   const long long g0 = sm.run[0], g1 = sm.run[1];
   if (g0 >= g1) return;
 
-  // first unit whose pages reach past g0: largest u with indptr[u] <= g0
-  int lo = 0, hi = U;
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if (p.indptr[mid] <= g0) lo = mid; else hi = mid;
-  }
-  const int u0 = lo;
+  const int u0 = sm.unit0;  // the unit holding page g0
 
   if (warp == kPlannerWarp) {
     // ------------------------------------------------------------- planner
