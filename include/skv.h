@@ -208,6 +208,27 @@ int skv_decode_attention(skv_ctx* ctx, const void* q, int q_dtype, int B, int Hq
                          const uint32_t* page_ids, const skv_pools* pools, float* out, float* lse, int32_t* err_word,
                          void* workspace, size_t ws_bytes, int num_splits, void* stream);
 
+/* skv_decode_attention_static -- skv_decode_attention without a caller
+   workspace (the paper has no counterpart: this is an interface convenience
+   of this library).  Same arguments, results and device errors as
+   skv_decode_attention (ADA decode only; page_tier_indptr may be NULL), but
+   the split partials, ticket counters and split prefix live in a fixed
+   4 MiB device array inside libskv, so the call allocates nothing.
+     - A call that would need more than 4 MiB of scratch (the size
+       skv_workspace_size(SKV_WS_DECODE) reports) is refused with
+       SKV_ERR_ARG before anything is launched.
+     - The array is shared by every call on a device: calls that overlap in
+       time (on different streams or host threads) race on it.  Serialise
+       them, e.g. by issuing them on one stream.
+     - The first call on each device looks up the array's device address and
+       configures the kernel; make it before any stream capture begins on
+       that device. */
+int skv_decode_attention_static(skv_ctx* ctx, const void* q, int q_dtype, int B, int Hq,
+                                int Hkv, const int32_t* page_indptr,
+                                const int32_t* page_tier_indptr, const uint32_t* page_ids,
+                                const skv_pools* pools, float* out, float* lse,
+                                int32_t* err_word, int num_splits, void* stream);
+
 /* skv_dense_pack_bf16 -- the dense baseline's store: every token of every
    (b, h) kept as bf16 K/V (fp16 inputs rounded to nearest even) in pages of
    P rows with the T0 page layout.  Slots come from free_ids in (b, h, page)

@@ -8,6 +8,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <string>
 
 #include "../../include/skv.h"
@@ -72,6 +73,35 @@ bool valid_pools(const skv_pools* pools, int ntiers) {
 }
 
 }  // namespace
+
+// ---------------------------------------------------------------------------
+// Fixed decode scratch for skv_decode_attention_static: the partials, ticket
+// counters, split flag and cost prefix live in this array instead of a
+// caller workspace.  Its device address is looked up once per device.
+// ---------------------------------------------------------------------------
+constexpr size_t kStaticScratchBytes = size_t(4) << 20;  // 4 MiB
+static __device__ __align__(256) unsigned char g_decode_scratch[kStaticScratchBytes];
+
+static std::mutex g_scratch_mu;
+static void* g_scratch_ptr[64] = {};
+
+// The scratch's device address on the current device (looked up once per
+// device, with that device current).  Returns the CUDA status.
+static cudaError_t static_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_ptr[dev]) {
+    void* ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_decode_scratch);
+    if (e != cudaSuccess) return e;
+    g_scratch_ptr[dev] = ptr;
+  }
+  *out = g_scratch_ptr[dev];
+  return cudaSuccess;
+}
 
 extern "C" {
 
@@ -445,6 +475,35 @@ int skv_dense_pack_bf16(skv_ctx* ctx, const uint16_t* K, const uint16_t* V, int 
   e = skv::launch_encode(p, s);
   if (e != cudaSuccess) return cuda_fail(e, "skv_dense_pack_bf16 encode");
   return ok();
+}
+
+int skv_decode_attention_static(skv_ctx* ctx, const void* q, int q_dtype, int B, int Hq,
+                                int Hkv, const int32_t* page_indptr,
+                                const int32_t* page_tier_indptr, const uint32_t* page_ids,
+                                const skv_pools* pools, float* out, float* lse,
+                                int32_t* err_word, int num_splits, void* stream) {
+  static const char* name = "skv_decode_attention_static";
+  if (!ctx) return fail(SKV_ERR_ARG, "%s: null ctx", name);
+  if (B < 0 || Hkv <= 0 || Hq <= 0 || Hq % Hkv != 0 || num_splits < 0)
+    return fail(SKV_ERR_ARG, "%s: need B >= 0, Hq a multiple of Hkv, num_splits >= 0", name);
+  if (B == 0) return ok();
+  size_t need = 0;
+  const int rc = skv_workspace_size(ctx, SKV_WS_DECODE, B, Hkv, Hq, 0, num_splits, &need);
+  if (rc != SKV_OK) return rc;
+  if (need > kStaticScratchBytes)
+    return fail(SKV_ERR_ARG,
+                "%s: this call needs %zu bytes of scratch; the static scratch holds %zu "
+                "(use skv_decode_attention with a workspace)",
+                name, need, kStaticScratchBytes);
+  if (!valid_pools(pools, 3)) return fail(SKV_ERR_ARG, "%s: bad pools", name);
+  void* scratch = nullptr;
+  cudaError_t e = static_scratch(&scratch);
+  if (e != cudaSuccess) return cuda_fail(e, "skv_decode_attention_static: scratch address");
+  const void* pool[3] = {pools->base[0], pools->base[1], pools->base[2]};
+  const long long slots[3] = {pools->slots[0], pools->slots[1], pools->slots[2]};
+  return decode_common(ctx, q, q_dtype, B, Hq, Hkv, page_indptr, page_tier_indptr, page_ids, pool,
+                       slots, false, out, lse, err_word, scratch, kStaticScratchBytes, num_splits,
+                       stream, name);
 }
 
 int skv_set_profile_event(skv_ctx* ctx, void* event) {

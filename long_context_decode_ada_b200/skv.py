@@ -32,7 +32,8 @@ TABLE_BOUNDARY6_X, TABLE_BOUNDARY6_Y, TABLE_BOUNDARY4_X, TABLE_BOUNDARY4_Y, TABL
 EXPORTS = [
     "skv_create", "skv_destroy", "skv_last_error", "skv_page_bytes", "skv_tables",
     "skv_device_info", "skv_workspace_size", "skv_allocate", "skv_encode",
-    "skv_decode_attention", "skv_dense_pack_bf16", "skv_dense_decode_bf16",
+    "skv_decode_attention", "skv_decode_attention_static", "skv_dense_pack_bf16",
+    "skv_dense_decode_bf16",
     "skv_set_profile_event", "skv_check",
 ]
 
@@ -64,6 +65,8 @@ _SIGS = {
                         _p]),
     "skv_decode_attention": (_i, [_p, _p, _i, _i, _i, _i, _p, _p, _p, C.POINTER(SkvPools), _p, _p,
                                   _p, _p, _sz, _i, _p]),
+    "skv_decode_attention_static": (_i, [_p, _p, _i, _i, _i, _i, _p, _p, _p,
+                                         C.POINTER(SkvPools), _p, _p, _p, _i, _p]),
     "skv_dense_pack_bf16": (_i, [_p, _p, _p, _i, _i, _i64, _p, _p, _i64, _p, _i64, _p, _p, _i64,
                                  _p, _p, _sz, _p]),
     "skv_dense_decode_bf16": (_i, [_p, _p, _i, _i, _i, _i, _p, _p, _p, _i64, _p, _p, _p, _p, _sz,
@@ -243,6 +246,21 @@ class PagedCache:
             _ptr(self.page_tier_indptr) if self.split_by_bytes else None,
             _ptr(self.page_ids), C.byref(self._pools_c), _ptr(out), _ptr(lse), _ptr(self.err),
             _ptr(workspace), workspace.numel(), num_splits, _stream(stream)))
+        return out, lse
+
+    def decode_static(self, q: torch.Tensor, q_dtype: int, Hq: int, out=None, lse=None,
+                      num_splits: int = 0, stream=None):
+        """decode() with the library's fixed scratch instead of a workspace
+        (skv_decode_attention_static: calls must not overlap in time)."""
+        if out is None:
+            out = torch.empty((self.B, Hq, self.ctx.d), dtype=torch.float32, device=self.device)
+        if lse is None:
+            lse = torch.empty((self.B, Hq), dtype=torch.float32, device=self.device)
+        _check(lib().skv_decode_attention_static(
+            self.ctx.handle, _ptr(q), q_dtype, self.B, Hq, self.Hkv, _ptr(self.page_indptr),
+            _ptr(self.page_tier_indptr) if self.split_by_bytes else None,
+            _ptr(self.page_ids), C.byref(self._pools_c), _ptr(out), _ptr(lse), _ptr(self.err),
+            num_splits, _stream(stream)))
         return out, lse
 
     def check(self, stream=None):
