@@ -69,6 +69,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test of a phase (never suspends the thread).
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // try_wait that lets the thread sleep (until the phase completes, or at
 // most `hint_ns`) instead of returning at once: waiting warps then take no
 // issue slots and no shared-memory pipe bandwidth from the working warps.
@@ -131,6 +143,14 @@ __device__ __forceinline__ void s8x4_to_f16x2x2(uint32_t w, uint32_t& lo, uint32
   __half2 hb = __hsub2(*reinterpret_cast<__half2*>(&b), bias);
   lo = *reinterpret_cast<uint32_t*>(&ha);
   hi = *reinterpret_cast<uint32_t*>(&hb);
+}
+
+// The same four int8 as fp16 values offset by +1152 (0x64XX = 1024 + XX,
+// XX = e + 128): exact, one subtraction fewer; the caller removes 1152.
+__device__ __forceinline__ void s8x4_to_f16x2x2_biased(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  const uint32_t u = w ^ 0x80808080u;
+  lo = __byte_perm(u, 0x64646464u, 0x4140);
+  hi = __byte_perm(u, 0x64646464u, 0x4342);
 }
 
 __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {

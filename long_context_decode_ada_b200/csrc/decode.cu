@@ -9,8 +9,7 @@
 // and produces one partial (m, l, o) per unit it touches.  A unit covered
 // by a single run is finished in place; otherwise the partial goes to slot
 // c + u of the workspace and the CTA that brings the unit's ticket counter
-// to its run count merges them (log-sum-exp).  The only cross-CTA wait is
-// for the published split prefix, which the first CTA writes at its start.
+// to its run count merges them (log-sum-exp); no CTA waits for another.
 //
 // CTA = kCG groups of 4 consumer warps + 1 planner warp + kIss issuer
 // warps around one byte ring in shared memory.  The CTA's run is cut into
@@ -60,6 +59,7 @@ constexpr int kPasses = kRowsPerWarp / 16;
 constexpr int kNSlot = 16;                    // items in flight, at most
 constexpr int kMaxIPP = kItemRows / 16;       // pages per item (P >= 16)
 constexpr int kMergeRuns = 128;               // runs per unit merged through shared memory
+constexpr int kTouchedUnits = 16;             // units whose segment costs a CTA keeps
 static_assert(kCG >= 1 && kCG <= 4, "consumer groups: 1..4");
 static_assert(kIss >= 1 && kIss <= 4, "issuers: 1..4");
 static_assert(kPasses >= 1 && kGW * kRowsPerWarp == kItemRows, "warp row split");
@@ -98,12 +98,14 @@ struct __align__(16) DecodeSmem {
   uint4 desc[kNSlot];                  // consumers' view of an item
   PageCopy copy[kNSlot][kMaxIPP];      // issuers' view of an item
   uint32_t copy_bytes[kNSlot];         // bytes of the item (0xFFFFFFFF: no more items)
+  unsigned long long vstart[64];       // planner: virtual ring start of item j at j % 64
   unsigned long long scan[kDecodeThreads / 32];
-  unsigned long long cunit[5];         // merge: cost before each segment of a unit, end, total
+  unsigned long long ucost[3 * kTouchedUnits + 1];  // cost before segments 3 unit0 ..
+  unsigned long long ctot;             // total cost of the page list
+  unsigned long long cunit[4];         // merge: cost before each segment of a unit, and its end
   long long useg[4];                   // merge: the unit's tier segment starts
   long long run[2];                    // this CTA's pages [run[0], run[1])
-  int unit0;                           // the unit of page run[0]
-  int pad_unit;
+  int unit0, unit1;                    // the units of pages run[0] and run[1] - 1
   int abort_flag;
   int last_flag;
   int pad_[2];
@@ -152,8 +154,8 @@ __host__ __device__ __forceinline__ bool smem_layout(uint32_t base, uint32_t lim
 // tier's payload bytes.  With C(g) the cost of the pages before page g and
 // C the total, page g belongs to run floor(C(g) S / C); run c starts at the
 // first page g with C(g) S >= c C.  Every CTA scans the segment costs
-// itself; the first to finish publishes the prefix to the workspace for the
-// merges (published flag: 0 none, 1 writing, 2 done).
+// itself and keeps the prefix at the segments of the units it touches,
+// which its merges need.
 struct SplitInfo {
   const int32_t* indptr;
   const int32_t* tier_indptr;
@@ -188,12 +190,11 @@ __device__ __forceinline__ long long run_begin_in_unit(const SplitInfo& si,
   return seg[3];
 }
 
-// This CTA's run [sm.run[0], sm.run[1]) (block-wide; contains barriers).
-// The first CTA to get here also publishes the cost before every segment
-// (and the total) to pub[0 .. 3U] and then sets *pub_flag to 2.
+// This CTA's run [sm.run[0], sm.run[1]) (block-wide; contains barriers),
+// its first and last unit, the total cost, and the cost before every
+// segment of the units it touches (when they are at most kTouchedUnits).
 template <class Smem>
-__device__ __noinline__ void find_run(const SplitInfo& si, int c, int S, Smem& sm,
-                                      unsigned long long* pub, int* pub_flag, int tid) {
+__device__ __noinline__ void find_run(const SplitInfo& si, int c, int S, Smem& sm, int tid) {
   constexpr int nt = kDecodeThreads;
   const int nseg = 3 * si.U;
   const int per = (nseg + nt - 1) / nt;
@@ -212,7 +213,8 @@ __device__ __noinline__ void find_run(const SplitInfo& si, int c, int S, Smem& s
   if (tid == 0) {
     sm.run[0] = 0;  // the run boundaries that no segment claims (T = 0)
     sm.run[1] = 0;
-    sm.last_flag = atomicCAS(pub_flag, 0, 1) == 0;  // this CTA publishes
+    sm.unit0 = 0;
+    sm.unit1 = -1;
   }
   __syncthreads();
   unsigned long long before = x - loc, tot = 0;
@@ -223,7 +225,6 @@ __device__ __noinline__ void find_run(const SplitInfo& si, int c, int S, Smem& s
   }
   const unsigned long long Su = (unsigned long long)S;
   const unsigned long long T0 = (unsigned long long)c * tot, T1 = (unsigned long long)(c + 1) * tot;
-  const bool publish = sm.last_flag != 0;
   unsigned long long cc = before;
   for (int k = k0; k < k1; ++k) {
     const long long a = si.seg_start(k), b = si.seg_start(k + 1);
@@ -231,32 +232,29 @@ __device__ __noinline__ void find_run(const SplitInfo& si, int c, int S, Smem& s
     const unsigned long long lo = cc * Su, hi = lo + (unsigned long long)(b - a) * ws;
     if (lo < T0 && T0 <= hi) sm.run[0] = a + (long long)((T0 - lo + ws - 1) / ws);
     if (lo < T1 && T1 <= hi) sm.run[1] = a + (long long)((T1 - lo + ws - 1) / ws);
-    if (publish) pub[k] = cc;
     cc += (unsigned long long)(b - a) * si.weight(k);
   }
-  if (publish) {
-    if (tid == 0) pub[nseg] = tot;
-    __threadfence();
+  if (tid == 0) sm.ctot = tot;
+  __syncthreads();
+  // the units of the run's first and last page (their segments hold them)
+  const long long g0 = sm.run[0], g1 = sm.run[1];
+  for (int k = k0; k < k1; ++k) {
+    const long long a = si.seg_start(k), b = si.seg_start(k + 1);
+    if (a <= g0 && g0 < b) sm.unit0 = k / 3;
+    if (a < g1 && g1 <= b) sm.unit1 = k / 3;
   }
   __syncthreads();
-  if (publish && tid == 0) atomicExch(pub_flag, 2);
-  // the unit of the run's first page (its segment holds it)
-  const long long g0 = sm.run[0];
-  for (int k = k0; k < k1; ++k)
-    if (si.seg_start(k) <= g0 && g0 < si.seg_start(k + 1)) sm.unit0 = k / 3;
-  __syncthreads();
-}
-
-// Wait (bounded) until the segment-cost prefix is published; false on timeout.
-__device__ __forceinline__ bool wait_published(const int* pub_flag) {
-  const long long t0 = clock64();
-  while (true) {
-    int f;
-    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(f) : "l"(pub_flag) : "memory");
-    if (f == 2) return true;
-    if (clock64() - t0 > kWaitLimitCycles) return false;
-    __nanosleep(256);
+  const int ua = sm.unit0, ub = sm.unit1;
+  if (ub >= ua && ub - ua < kTouchedUnits) {
+    cc = before;
+    for (int k = k0; k < k1; ++k) {
+      if (k >= 3 * ua && k <= 3 * ub + 3) sm.ucost[k - 3 * ua] = cc;
+      cc += (unsigned long long)(si.seg_start(k + 1) - si.seg_start(k)) * si.weight(k);
+    }
+    // the cost after the last segment (the end of the page list)
+    if (k1 == nseg && k0 < k1 && nseg <= 3 * ub + 3) sm.ucost[nseg - 3 * ua] = cc;
   }
+  __syncthreads();
 }
 
 // ------------------------------------------------------ shared loads (PTX) --
@@ -331,12 +329,22 @@ __device__ __forceinline__ float share_byte(uint32_t spread) {
   return __uint_as_float(__byte_perm(spread, 0x4B000000u, 0x7440u | K));
 }
 
+// A lane's LUT columns: table base | ((jj ^ (row & 3)) * 4 + g) * entry
+// bytes for jj = 0..3 (rows rA and rA + 8 of a 16-row step share row & 3,
+// which is t & 3 for every step).
+template <int G>
+__device__ __forceinline__ void lut_columns(uint32_t lut, int t, int g, uint32_t (&xo)[4]) {
+  const uint32_t x3 = (uint32_t)t & 3u;
+#pragma unroll
+  for (int jj = 0; jj < 4; ++jj) xo[jj] = lut | ((((uint32_t)jj ^ x3) * 4 + g) * LutGeom<G>::kEnt);
+}
+
 // Partial logits (times 16: shares enter as code + 1) of rows rA, rA + 8 of
 // the T1 page at shared address pg.  Code byte 16g + j of a row holds pair
 // 4 (j ^ (row & 3)) + g as (angle6 << 2) | share2.
 template <int G>
-__device__ __forceinline__ void logits_t1(uint32_t pg, int P, int rA, int g, uint32_t lut,
-                                          RowAcc<G>& sA, RowAcc<G>& sB) {
+__device__ __forceinline__ void logits_t1(uint32_t pg, int P, int rA, int g,
+                                          const uint32_t (&xo)[4], RowAcc<G>& sA, RowAcc<G>& sB) {
   const uint32_t cd = pg + kHdrBytes + 2 * P;
   const uint4 ca = lds128(cd + rA * 64 + 16 * g);
   const uint4 cb = lds128(cd + (rA + 8) * 64 + 16 * g);
@@ -348,14 +356,11 @@ __device__ __forceinline__ void logits_t1(uint32_t pg, int P, int rA, int g, uin
     qa[k] = wa[k] & 0x03030303u;
     qb[k] = wb[k] & 0x03030303u;
   }
-  const uint32_t x3 = rA & 3;  // rows rA and rA + 8 share it
   using L = LutGeom<G>;
   // the table base is aligned to the table size: base | pair offset | code
-  // bits; the part of the pair offset that depends on j alone is added (an
-  // immediate of the shared load)
-  uint32_t xo[4];
-#pragma unroll
-  for (int jj = 0; jj < 4; ++jj) xo[jj] = lut | ((((uint32_t)jj ^ x3) * 4 + g) * L::kEnt);
+  // bits (xo: base | the lane's pair offset, see lut_columns); the part of
+  // the pair offset that depends on j alone is added (an immediate of the
+  // shared load)
   constexpr uint32_t kMask = 0xFCu << (L::kCodeShift - 2);  // angle bits of a byte, scaled
 #pragma unroll
   for (int j = 0; j < 16; ++j) {
@@ -378,8 +383,8 @@ __device__ __forceinline__ void logits_t1(uint32_t pg, int P, int rA, int g, uin
 // T2: nibble j of bytes [8g, 8g+8) holds the 4-bit angle of pair
 // 4 (j ^ (row & 3)) + g, crumb j of bytes [32+4g, 36+4g) its share.
 template <int G>
-__device__ __forceinline__ void logits_t2(uint32_t pg, int P, int rA, int g, uint32_t lut,
-                                          RowAcc<G>& sA, RowAcc<G>& sB) {
+__device__ __forceinline__ void logits_t2(uint32_t pg, int P, int rA, int g,
+                                          const uint32_t (&xo)[4], RowAcc<G>& sA, RowAcc<G>& sB) {
   const uint32_t cd = pg + kHdrBytes + 2 * P;
   const uint2 na = lds64(cd + rA * 48 + 8 * g);
   const uint2 nb = lds64(cd + (rA + 8) * 48 + 8 * g);
@@ -392,11 +397,7 @@ __device__ __forceinline__ void logits_t2(uint32_t pg, int P, int rA, int g, uin
     qa[k] = (ra >> (2 * k)) & 0x03030303u;
     qb[k] = (rb >> (2 * k)) & 0x03030303u;
   }
-  const uint32_t x3 = rA & 3;
   using L = LutGeom<G>;
-  uint32_t xo[4];
-#pragma unroll
-  for (int jj = 0; jj < 4; ++jj) xo[jj] = lut | ((((uint32_t)jj ^ x3) * 4 + g) * L::kEnt);
   constexpr uint32_t kMask = 0xFu << L::kCodeShift;
 #pragma unroll
   for (int j = 0; j < 16; ++j) {
@@ -501,6 +502,7 @@ struct WarpState {
   float m;          // running max (log2 domain) of head g % G, or kNoMax
   float l;          // partial denominator of (token slot t, head g % G)
   float acc[8][4];  // O^T fragments: [m-tile][c0..c3]
+  float ones[4];    // sum of the P.V B operand per head (int8 V bias, see softmax_pv)
 };
 
 // Start value of the running max: finite, so that exp2 of (-inf - m) is 0
@@ -543,23 +545,27 @@ __device__ __forceinline__ void softmax_pv(float lA, float lB, float vsA, float 
       st.acc[mt][2] *= a0;
       st.acc[mt][3] *= a1;
     }
+    st.ones[0] *= a0;
+    st.ones[1] *= a1;
+    st.ones[2] *= a0;
+    st.ones[3] *= a1;
   }
   const float pA = ex2_approx(lA - st.m), pB = ex2_approx(lB - st.m);  // -inf -> 0
   st.l += pA + pB;
   const float ppA = pA * vsA, ppB = pB * vsB;
   // B fragment (k16 x n8): k = rows 2t4, 2t4+1 | 8+2t4, 9+2t4, n = head gq
   const int src = 8 * t4 + (gq < G ? gq : 0);
-  float b0 = __shfl_sync(0xFFFFFFFFu, ppA, src);
-  float b1 = __shfl_sync(0xFFFFFFFFu, ppA, src + 4);
-  float b2 = __shfl_sync(0xFFFFFFFFu, ppB, src);
-  float b3 = __shfl_sync(0xFFFFFFFFu, ppB, src + 4);
-  if (gq >= G) {
-    b0 = 0.0f;
-    b1 = 0.0f;
-    b2 = 0.0f;
-    b3 = 0.0f;
-  }
+  // columns n >= G (lanes gq >= G) carry copies of head 0: their outputs
+  // are never read
+  const float b0 = __shfl_sync(0xFFFFFFFFu, ppA, src);
+  const float b1 = __shfl_sync(0xFFFFFFFFu, ppA, src + 4);
+  const float b2 = __shfl_sync(0xFFFFFFFFu, ppB, src);
+  const float b3 = __shfl_sync(0xFFFFFFFFu, ppB, src + 4);
   if constexpr (VK == 0) {
+    // int8 V enters the MMA as the fp16 value v + 1152 (exact: 0x64XX with
+    // XX = v + 128); one more MMA against an all-ones A tile accumulates the
+    // B column sums, and 1152 times them is taken off when the warps'
+    // states are combined
     const uint32_t bf0 = pack_f16x2(b0, b1), bf1 = pack_f16x2(b2, b3);
     const uint4 xa = lds128(va + lane * 16), ya = lds128(va + 512 + lane * 16);
     const uint4 xb = lds128(vb + lane * 16), yb = lds128(vb + 512 + lane * 16);
@@ -568,10 +574,12 @@ __device__ __forceinline__ void softmax_pv(float lA, float lB, float vsA, float 
 #pragma unroll
     for (int mt = 0; mt < 8; ++mt) {
       uint32_t a0, a1, a2, a3;
-      s8x4_to_f16x2x2(wa[mt], a0, a1);
-      s8x4_to_f16x2x2(wb[mt], a2, a3);
+      s8x4_to_f16x2x2_biased(wa[mt], a0, a1);
+      s8x4_to_f16x2x2_biased(wb[mt], a2, a3);
       mma_16816k16_f16(st.acc[mt], a0, a1, a2, a3, bf0, bf1);
     }
+    constexpr uint32_t kOnes = 0x3C003C00u;  // fp16 (1, 1)
+    mma_16816k16_f16(st.ones, kOnes, kOnes, kOnes, kOnes, bf0, bf1);
   } else {
     const uint32_t bf0 = (VK == 1) ? pack_f16x2(b0, b1) : pack_bf16x2(b0, b1);
     const uint32_t bf1 = (VK == 1) ? pack_f16x2(b2, b3) : pack_bf16x2(b2, b3);
@@ -593,13 +601,15 @@ __device__ __forceinline__ void softmax_pv(float lA, float lB, float vsA, float 
 // 16 rows [row0, row0 + 16) of one page at shared address pg.
 template <int G, bool DENSE>
 __device__ __forceinline__ void process_rows(const DecodeParams& p, uint32_t pg, uint32_t tier,
-                                             int row0, uint32_t lut1, uint32_t lut2,
-                                             uint32_t q32, WarpState& st, int lane) {
+                                             int row0, const uint32_t (&xo1)[4],
+                                             const uint32_t (&xo2)[4], uint32_t q32,
+                                             WarpState& st, int lane) {
   const int t = lane >> 2, g = lane & 3;
   const int P = p.P;
+  // header {u16 count, u8 tier, u8 magic}
   const uint32_t h0 = lds32(pg);
-  const uint32_t cnt = h0 & 0xFFFFu, htier = (h0 >> 16) & 0xFFu, magic = h0 >> 24;
-  if (htier != tier || magic != kPageMagic || cnt > (uint32_t)P) {
+  const uint32_t cnt = h0 & 0xFFFFu;
+  if ((h0 >> 16) != (tier | ((uint32_t)kPageMagic << 8)) || cnt > (uint32_t)P) {
     if (lane == 0) report(p.err, SKV_ERR_CORRUPT);
     return;
   }
@@ -607,16 +617,13 @@ __device__ __forceinline__ void process_rows(const DecodeParams& p, uint32_t pg,
   const int rA = row0 + t, rB = rA + 8;
   const bool vA = (uint32_t)rA < cnt, vB = (uint32_t)rB < cnt;
   float sA[G], sB[G];
-#pragma unroll
-  for (int h = 0; h < G; ++h) {
-    sA[h] = 0.0f;
-    sB[h] = 0.0f;
-  }
-  RowAcc<G> rA2, rB2;
-  rA2.zero();
-  rB2.zero();
   const uint32_t vsec_dense = pg + kHdrBytes + 256 * P + (row0 >> 3) * 2048;
   if constexpr (DENSE) {
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      sA[h] = 0.0f;
+      sB[h] = 0.0f;
+    }
     logits_dense<G, true>(pg, rA, g, q32, sA, sB);
     const float a = reduce_scatter<G>(sA, g), b = reduce_scatter<G>(sB, g);
     const float c = p.qk_scale_log2;
@@ -624,6 +631,11 @@ __device__ __forceinline__ void process_rows(const DecodeParams& p, uint32_t pg,
                      vsec_dense + 2048, st, lane);
   } else {
     if (tier == SKV_TIER_T0) {
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        sA[h] = 0.0f;
+        sB[h] = 0.0f;
+      }
       logits_dense<G, false>(pg, rA, g, q32, sA, sB);
       const float a = reduce_scatter<G>(sA, g), b = reduce_scatter<G>(sB, g);
       const float c = p.qk_scale_log2 * 5.192296858534828e+33f;  // 2^112
@@ -631,10 +643,13 @@ __device__ __forceinline__ void process_rows(const DecodeParams& p, uint32_t pg,
                        vsec_dense + 2048, st, lane);
     } else {
       const bool t1 = tier == SKV_TIER_T1;
+      RowAcc<G> rA2, rB2;
+      rA2.zero();
+      rB2.zero();
       if (t1)
-        logits_t1<G>(pg, P, rA, g, lut1, rA2, rB2);
+        logits_t1<G>(pg, P, rA, g, xo1, rA2, rB2);
       else
-        logits_t2<G>(pg, P, rA, g, lut2, rA2, rB2);
+        logits_t2<G>(pg, P, rA, g, xo2, rA2, rB2);
       rA2.to(sA);
       rB2.to(sB);
       const float a = reduce_scatter<G>(sA, g), b = reduce_scatter<G>(sB, g);
@@ -674,8 +689,6 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   const DecodeWs wsl = decode_ws(p.S, U, G);
   uint8_t* const wsb = reinterpret_cast<uint8_t*>(p.part);
   int* const counters = reinterpret_cast<int*>(wsb + wsl.ctr);
-  int* const pub_flag = reinterpret_cast<int*>(wsb + wsl.flag);
-  unsigned long long* const pub = reinterpret_cast<unsigned long long*>(wsb + wsl.pub);
   const int ipp = kItemRows >> p.log2P;
   // the largest item: ipp pages of the largest payload
   int maxpay = p.payload[0];
@@ -709,7 +722,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     }
   }
   if (!plan_ok) return;  // uniform: every thread computed the same layout
-  find_run(si, c, p.S, sm, pub, pub_flag, tid);
+  find_run(si, c, p.S, sm, tid);
   const long long g0 = sm.run[0], g1 = sm.run[1];
   if (g0 >= g1) return;
 
@@ -718,14 +731,14 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   if (warp == kPlannerWarp) {
     // ------------------------------------------------------------- planner
     // Batches of up to 32 items of one unit: lane i decodes item it + i (its
-    // page ids -> sources, sizes, tiers) in parallel; a short uniform loop
-    // then places the items one by one.  Placement is deterministic: an item
-    // goes at the write offset, or at 0 when it would cross the ring's end;
-    // before it is published every older item whose bytes it may overwrite
-    // (virtual start < its virtual end - R) and the previous user of its
-    // slot must be released.  The lane that decoded the item writes its
-    // descriptors and signals the slot ready.  kIss end-of-run markers
-    // follow the last item, one per issuer.
+    // page ids -> sources, sizes, tiers) in parallel.  Placement is
+    // deterministic: an item goes at the write offset, or at 0 when it would
+    // cross the ring's end.  Before an item is published every older item
+    // whose bytes it may overwrite (virtual start < its virtual end - R) and
+    // the previous user of its slot must be released; each lane works out
+    // that count, and the lanes publish (descriptors + ready signal) in
+    // parallel as releases arrive.  kIss end-of-run markers follow the last
+    // item, one per issuer.
     int u = u0;
     long long ub = min(g1, (long long)p.indptr[u0 + 1]);  // end of the current unit's run
     long long pg = g0;                                     // first page of the next batch
@@ -733,7 +746,6 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     int tail = 0;               // oldest item not known to be released
     uint32_t wr = 0;            // ring write offset
     unsigned long long V = 0;   // virtual position of the write offset (grows by laps of R)
-    unsigned long long vmine = 0;  // lane (j % 32): virtual start of in-flight item j
     bool ok = true;
     // wait until item `tail` is released, then advance tail
     auto release_tail = [&]() -> bool {
@@ -793,37 +805,70 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
           }
         }
       }
-      // ---- uniform placement, one item at a time
-      for (int i = 0; i < nb && ok; ++i) {
+      // ---- placement: a cheap serial scan of the sizes, then each lane
+      // finds how many items must be released before its item may be
+      // written (need: all items before it), and the lanes publish in
+      // parallel, a prefix of the batch at a time, as releases come in
+      uint32_t my_off = 0;
+      unsigned long long my_v = 0;
+      for (int i = 0; i < nb; ++i) {
         const uint32_t t = __shfl_sync(0xFFFFFFFFu, total, i);
         const uint32_t off = (wr + t <= R) ? wr : 0u;
         const unsigned long long vi = (off == wr) ? V : V + (R - wr);
-        // release what this item may overwrite, and its slot's previous item
-        while (tail < it) {
-          const unsigned long long vt = __shfl_sync(0xFFFFFFFFu, vmine, tail & 31);
-          if (it - tail < kNSlot && vt + R >= vi + t) break;
-          if (!release_tail()) {
-            ok = false;
+        if (lane == i) {
+          my_off = off;
+          my_v = vi;
+        }
+        wr = off + t;
+        V = vi + t;
+      }
+      if (lane < nb) sm.vstart[(it + lane) & 63] = my_v;
+      __syncwarp();
+      int need = 0;
+      if (lane < nb) {
+        const int me = it + lane;
+        // slot reuse: item me - kNSlot must be released
+        need = max(0, me - kNSlot + 1);
+        // space: every item whose bytes start more than R before this
+        // item's end (V grows with the item index: a prefix of them)
+        const unsigned long long lim = my_v + total;
+        int J = me;
+        for (int j = need; j < me; ++j)
+          if (sm.vstart[j & 63] + R >= lim) {
+            J = j;
             break;
           }
-        }
-        if (!ok) break;
-        const int s = it % kNSlot;
-        if (lane == (it & 31)) vmine = vi;
-        if (lane == i) {
-          sm.desc[s] = make_uint4(ring_lo + off, imeta, relz, relw);
+        need = J;
+      }
+      bool done = lane >= nb;
+      while (true) {
+        // released items, in order, without blocking
+        while (tail < it + nb &&
+               mbar_test_wait(smem_u32(&sm.empty[tail % kNSlot]), (uint32_t)((tail / kNSlot) & 1)))
+          ++tail;
+        const bool now = !done && need <= tail;
+        if (now) {
+          const int s = (it + lane) % kNSlot;
+          sm.desc[s] = make_uint4(ring_lo + my_off, imeta, relz, relw);
           const uint32_t rel[kMaxIPP] = {0u, relz & 0xFFFFu, relz >> 16, relw};
 #pragma unroll
           for (int q = 0; q < kMaxIPP; ++q)
             if (q < (int)(imeta & 7u))
-              sm.copy[s][q] = PageCopy{plo[q], phi[q], psz[q], ring_lo + off + rel[q]};
+              sm.copy[s][q] = PageCopy{plo[q], phi[q], psz[q], ring_lo + my_off + rel[q]};
           sm.copy_bytes[s] = total;
           mbar_arrive(smem_u32(&sm.ready[s]));
         }
-        wr = off + t;
-        V = vi + t;
-        ++it;
+        done = done || now;
+        if (__all_sync(0xFFFFFFFFu, done)) break;
+        // the oldest unreleased item is published (its own need is met):
+        // sleep until it is released
+        if (!release_tail()) {
+          ok = false;
+          break;
+        }
       }
+      if (!ok) break;
+      it += nb;
       pg = min(ub, pg + (long long)nb * ipp);
     }
     // end-of-run markers: a slot each (its previous item released)
@@ -896,6 +941,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   const int nct = kNCW * 32;
   const int t4 = lane & 3, gq = lane >> 2;
   const int grp = warp / kGW, wi = warp % kGW;  // consumer group, warp within it
+  uint32_t xo1[4], xo2[4];  // this lane's LUT columns (see lut_columns)
+  lut_columns<G>(lut1, lane >> 2, lane & 3, xo1);
+  lut_columns<G>(lut2, lane >> 2, lane & 3, xo2);
   const uint32_t q32 = smem_u32(sm.q32);
   float* lut1p = reinterpret_cast<float*>(smem_raw + (lut1 - base));
   float* lut2p = reinterpret_cast<float*>(smem_raw + (lut2 - base));
@@ -953,6 +1001,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     for (int mt = 0; mt < 8; ++mt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) st.acc[mt][e] = 0.0f;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) st.ones[e] = 0.0f;
 
     const int nitems = (int)((b - a + ipp - 1) / ipp);
     // this group's items of the unit: it + i with (it + i) % kCG == grp
@@ -979,7 +1029,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
                                          : (kp == 1 ? (d.z & 0xFFFFu)
                                                     : (kp == 2 ? (d.z >> 16) : d.w));
             process_rows<G, DENSE>(p, d.x + rel, (d.y >> (kMetaTierShift + 2 * kp)) & 3u, row0,
-                                   lut1, lut2, q32, st, lane);
+                                   xo1, xo2, q32, st, lane);
           }
         }
       }
@@ -1007,10 +1057,11 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         for (int w = 0; w < kNCW; ++w) M = fmaxf(M, sm.ml[w][n][0]);
         const float mw = sm.ml[warp][n][0];
         const float sc = (mw == -INFINITY) ? 0.0f : exp2f(mw - M);
+        const float bias = 1152.0f * st.ones[j];  // int8 V offset (see softmax_pv)
 #pragma unroll
         for (int mt = 0; mt < 8; ++mt) {
-          atomicAdd(&sm.O[n][16 * mt + gq], st.acc[mt][j] * sc);
-          atomicAdd(&sm.O[n][16 * mt + gq + 8], st.acc[mt][2 + j] * sc);
+          atomicAdd(&sm.O[n][16 * mt + gq], (st.acc[mt][j] - bias) * sc);
+          atomicAdd(&sm.O[n][16 * mt + gq + 8], (st.acc[mt][2 + j] - bias) * sc);
         }
       }
     }
@@ -1036,18 +1087,30 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     if (tid == 0) {
 #pragma unroll
       for (int t = 0; t < 4; ++t) sm.useg[t] = si.seg_start(3 * u + t);
-      if (wait_published(pub_flag)) {
+    }
+    if (sm.unit1 - sm.unit0 < kTouchedUnits) {
+      if (tid < 4) sm.cunit[tid] = sm.ucost[3 * (u - sm.unit0) + tid];
+    } else {
+      // many units in this run: the cost before unit u, summed afresh
+      unsigned long long part = 0;
+      for (int k = tid; k < 3 * u; k += nct)
+        part += (unsigned long long)(si.seg_start(k + 1) - si.seg_start(k)) * si.weight(k);
 #pragma unroll
-        for (int t = 0; t < 4; ++t) sm.cunit[t] = __ldcg(pub + 3 * u + t);
-        sm.cunit[4] = __ldcg(pub + 3 * U);
-      } else {
-        report(p.err, SKV_ERR_TIMEOUT);
-#pragma unroll
-        for (int t = 0; t < 5; ++t) sm.cunit[t] = 0;
+      for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xFFFFFFFFu, part, o);
+      if (lane == 0) sm.scan[warp] = part;
+      named_bar_sync(1, nct);
+      if (tid == 0) {
+        unsigned long long cb = 0;
+        for (int w2 = 0; w2 < kNCW; ++w2) cb += sm.scan[w2];
+        sm.cunit[0] = cb;
+        for (int t = 0; t < 3; ++t)
+          sm.cunit[t + 1] = sm.cunit[t] + (unsigned long long)(si.seg_start(3 * u + t + 1) -
+                                                               si.seg_start(3 * u + t)) *
+                                              si.weight(t);
       }
     }
     named_bar_sync(1, nct);
-    const unsigned long long Su = (unsigned long long)p.S, ctot = sm.cunit[4];
+    const unsigned long long Su = (unsigned long long)p.S, ctot = sm.ctot;
     int c0 = c, c1 = c;
     if (ctot > 0) {
       int tl = 2;  // tier of the unit's last page
@@ -1204,9 +1267,9 @@ cudaError_t launch_decode_g(const DecodeParams& p, cudaStream_t stream, cudaEven
     if (dev >= 0 && dev < 64) configured[dev] = smem;
   }
   const int U = p.B * p.Hkv;
-  // ticket counters and the split's publication flag start at zero
+  // the ticket counters start at zero
   const DecodeWs wsl = decode_ws(p.S, U, G);
-  e = cudaMemsetAsync(reinterpret_cast<uint8_t*>(p.part) + wsl.ctr, 0, sizeof(int) * ((size_t)U + 1),
+  e = cudaMemsetAsync(reinterpret_cast<uint8_t*>(p.part) + wsl.ctr, 0, sizeof(int) * (size_t)U,
                       stream);
   if (e != cudaSuccess) return e;
   decode_kernel<G, DENSE><<<p.S, kDecodeThreads, p.smem_bytes, stream>>>(p);

@@ -89,17 +89,14 @@ struct AllocParams {
 };
 
 // Decode workspace: partials [(S + U) G][kPartStride] fp32, then U ticket
-// counters and the split's publication flag (int32, zeroed by every call),
-// then the published segment-cost prefix (uint64 [3U + 1]).
+// counters (int32, zeroed by every call).
 struct DecodeWs {
-  size_t ctr, flag, pub, bytes;
+  size_t ctr, bytes;
 };
 __host__ __device__ inline DecodeWs decode_ws(long long S, long long U, int G) {
   DecodeWs w;
   w.ctr = (size_t)(S + U) * G * kPartStride * 4;
-  w.flag = w.ctr + 4 * (size_t)U;
-  w.pub = (w.flag + 4 + 7) / 8 * 8;
-  w.bytes = w.pub + 8 * (size_t)(3 * U + 1);
+  w.bytes = w.ctr + 4 * (size_t)U;
   return w;
 }
 

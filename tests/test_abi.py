@@ -85,10 +85,8 @@ def test_workspace_sizes():
     ctx = skv.Context(64)
     sm, splits = ctx.device_info()
     def expect(S, U, G):
-        # partials, U ticket counters + the split flag (8-byte aligned), cost prefix
-        ctr = (S + U) * G * 132 * 4
-        pub = (ctr + 4 * U + 4 + 7) // 8 * 8
-        return pub + 8 * (3 * U + 1)
+        # split partials, then one ticket counter per unit
+        return (S + U) * G * 132 * 4 + 4 * U
     n = ctx.workspace_size(skv.WS_DECODE, 1, 8, 32, 0, 0)
     assert n == expect(splits, 8, 4)
     assert ctx.workspace_size(skv.WS_DECODE, 1, 8, 32, 0, 10) == expect(10, 8, 4)
