@@ -525,12 +525,14 @@ __device__ __forceinline__ float ex2_approx(float x) {
 template <int G, int VK>
 __device__ __forceinline__ void softmax_pv(float lA, float lB, float vsA, float vsB, uint32_t va,
                                            uint32_t vb, WarpState& st, int lane) {
-  float cm = fmaxf(lA, lB);
-  cm = fmaxf(cm, __shfl_xor_sync(0xFFFFFFFFu, cm, 4));
-  cm = fmaxf(cm, __shfl_xor_sync(0xFFFFFFFFu, cm, 8));
-  cm = fmaxf(cm, __shfl_xor_sync(0xFFFFFFFFu, cm, 16));
   const int gq = lane >> 2, t4 = lane & 3;
-  if (__any_sync(0xFFFFFFFFu, cm > st.m + kLazyMax)) {
+  // a lane's own rows decide whether the running max must rise; only then
+  // is the max over the 16 rows (lanes of the same head) formed
+  if (__any_sync(0xFFFFFFFFu, fmaxf(lA, lB) > st.m + kLazyMax)) {
+    float cm = fmaxf(lA, lB);
+    cm = fmaxf(cm, __shfl_xor_sync(0xFFFFFFFFu, cm, 4));
+    cm = fmaxf(cm, __shfl_xor_sync(0xFFFFFFFFu, cm, 8));
+    cm = fmaxf(cm, __shfl_xor_sync(0xFFFFFFFFu, cm, 16));
     const float m_new = fmaxf(st.m, cm);
     const float alpha = ex2_approx(st.m - m_new);  // 0 when st.m is kNoMax
     st.l *= alpha;
@@ -766,11 +768,13 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       uint32_t total = 0, imeta = 0, relz = 0, relw = 0;
       if (lane < nb) {
         const long long ps = pg + (long long)lane * ipp;
-        const int n = (int)min((long long)ipp, ub - ps);
-        imeta = (uint32_t)n;
+        // the ids are read up to the end of the run, not of the unit: the
+        // loads do not wait for the unit bound
         uint32_t id[kMaxIPP];
 #pragma unroll
-        for (int q = 0; q < kMaxIPP; ++q) id[q] = q < n ? __ldg(p.ids + ps + q) : 0u;
+        for (int q = 0; q < kMaxIPP; ++q) id[q] = (q < ipp && ps + q < g1) ? __ldg(p.ids + ps + q) : 0u;
+        const int n = (int)min((long long)ipp, ub - ps);
+        imeta = (uint32_t)n;
 #pragma unroll
         for (int q = 0; q < kMaxIPP; ++q) {
           plo[q] = 0;
@@ -805,22 +809,45 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
           }
         }
       }
-      // ---- placement: a cheap serial scan of the sizes, then each lane
+      // ---- placement: a warp-parallel scan of the sizes, then each lane
       // finds how many items must be released before its item may be
       // written (need: all items before it), and the lanes publish in
       // parallel, a prefix of the batch at a time, as releases come in
       uint32_t my_off = 0;
       unsigned long long my_v = 0;
-      for (int i = 0; i < nb; ++i) {
-        const uint32_t t = __shfl_sync(0xFFFFFFFFu, total, i);
-        const uint32_t off = (wr + t <= R) ? wr : 0u;
-        const unsigned long long vi = (off == wr) ? V : V + (R - wr);
-        if (lane == i) {
-          my_off = off;
-          my_v = vi;
+      {
+        // offsets = write offset + exclusive prefix of the sizes, restarted
+        // at 0 (after a pad to the next lap of the virtual position) at the
+        // first item of each stretch that would cross the ring's end
+        uint32_t incl = total;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+          if (lane >= o) incl += y;
         }
-        wr = off + t;
-        V = vi + t;
+        const uint32_t excl = incl - total;
+        uint32_t base = wr;
+        unsigned long long vbase = V;
+        int from = 0;
+        while (true) {
+          const uint32_t ex0 = __shfl_sync(0xFFFFFFFFu, excl, from);
+          const uint32_t off = base + (excl - ex0);
+          const unsigned cross =
+              __ballot_sync(0xFFFFFFFFu, lane >= from && lane < nb && off + total > R);
+          const int j = cross ? __ffs(cross) - 1 : 32;
+          if (lane >= from && lane < j) {
+            my_off = off;
+            my_v = vbase + (excl - ex0);
+          }
+          if (!cross) break;
+          const uint32_t exj = __shfl_sync(0xFFFFFFFFu, excl, j);
+          vbase = vbase + (exj - ex0) + (R - (base + (exj - ex0)));
+          base = 0;
+          from = j;
+        }
+        const uint32_t lt = __shfl_sync(0xFFFFFFFFu, total, nb - 1);
+        wr = __shfl_sync(0xFFFFFFFFu, my_off, nb - 1) + lt;
+        V = __shfl_sync(0xFFFFFFFFu, my_v, nb - 1) + lt;
       }
       if (lane < nb) sm.vstart[(it + lane) & 63] = my_v;
       __syncwarp();
@@ -832,13 +859,13 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         // space: every item whose bytes start more than R before this
         // item's end (V grows with the item index: a prefix of them)
         const unsigned long long lim = my_v + total;
-        int J = me;
-        for (int j = need; j < me; ++j)
-          if (sm.vstart[j & 63] + R >= lim) {
-            J = j;
-            break;
-          }
-        need = J;
+        // binary search: the first j in [need, me) with vstart[j] + R >= lim
+        int lo = need, hi = me;
+        while (lo < hi) {
+          const int mid = (lo + hi) >> 1;
+          if (sm.vstart[mid & 63] + R >= lim) hi = mid; else lo = mid + 1;
+        }
+        need = lo;
       }
       bool done = lane >= nb;
       while (true) {
@@ -966,7 +993,16 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     }
     named_bar_sync(1, nct);
     if constexpr (!DENSE) {
-      for (int i = tid; i < 64 * kPairs; i += nct) {
+      // the tables this CTA's pages of the unit read (both when the page
+      // table gives no per-tier offsets)
+      bool need1 = true, need2 = true;
+      if (p.tier_indptr) {
+        const long long s1 = si.seg_start(3 * u + 1), s2 = si.seg_start(3 * u + 2),
+                        s3 = si.seg_start(3 * u + 3);
+        need1 = max(a, s1) < min(b, s2);
+        need2 = max(a, s2) < min(b, s3);
+      }
+      for (int i = tid; need1 && i < 64 * kPairs; i += nct) {
         const int cc = i >> 6, pr = i & 63;
         const float cs = p.cos6[cc], sn = p.sin6[cc];
         float v[G];
@@ -979,7 +1015,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
           for (int h = 0; h < G; ++h) lut1p[i * G + h] = v[h];
         }
       }
-      for (int i = tid; i < 16 * kPairs; i += nct) {
+      for (int i = tid; need2 && i < 16 * kPairs; i += nct) {
         const int cc = i >> 6, pr = i & 63;
         const float cs = p.cos4[cc], sn = p.sin4[cc];
         float v[G];
