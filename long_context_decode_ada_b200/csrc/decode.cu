@@ -110,6 +110,8 @@ struct __align__(16) DecodeSmem {
   int last_flag;
   int pad_[2];
   __align__(16) float ml[kNCW][4][2];
+  float wsc[kNCW][4];                   // combine: each warp's scale per head
+  float MH[4], LH[4];                   // combine: this CTA's (M, L) per head
   __align__(16) float O[4][kHeadDim];
   __align__(16) float q32[4][kHeadDim];   // read with 16-byte shared loads
   __align__(16) float mw[4][kMergeRuns];  // merge: per-run weights
@@ -1002,12 +1004,16 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         need1 = max(a, s1) < min(b, s2);
         need2 = max(a, s2) < min(b, s3);
       }
+#pragma unroll 2
       for (int i = tid; need1 && i < 64 * kPairs; i += nct) {
         const int cc = i >> 6, pr = i & 63;
         const float cs = p.cos6[cc], sn = p.sin6[cc];
         float v[G];
 #pragma unroll
-        for (int h = 0; h < G; ++h) v[h] = fmaf(sm.q32[h][2 * pr], cs, sm.q32[h][2 * pr + 1] * sn);
+        for (int h = 0; h < G; ++h) {
+          const float2 qp = *reinterpret_cast<const float2*>(&sm.q32[h][2 * pr]);
+          v[h] = fmaf(qp.x, cs, qp.y * sn);
+        }
         if constexpr (G == 4) {
           *reinterpret_cast<float4*>(&lut1p[i * 4]) = make_float4(v[0], v[1], v[2], v[3]);
         } else {
@@ -1015,12 +1021,16 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
           for (int h = 0; h < G; ++h) lut1p[i * G + h] = v[h];
         }
       }
+#pragma unroll 2
       for (int i = tid; need2 && i < 16 * kPairs; i += nct) {
         const int cc = i >> 6, pr = i & 63;
         const float cs = p.cos4[cc], sn = p.sin4[cc];
         float v[G];
 #pragma unroll
-        for (int h = 0; h < G; ++h) v[h] = fmaf(sm.q32[h][2 * pr], cs, sm.q32[h][2 * pr + 1] * sn);
+        for (int h = 0; h < G; ++h) {
+          const float2 qp = *reinterpret_cast<const float2*>(&sm.q32[h][2 * pr]);
+          v[h] = fmaf(qp.x, cs, qp.y * sn);
+        }
         if constexpr (G == 4) {
           *reinterpret_cast<float4*>(&lut2p[i * 4]) = make_float4(v[0], v[1], v[2], v[3]);
         } else {
@@ -1044,8 +1054,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     // this group's items of the unit: it + i with (it + i) % kCG == grp
     for (int i = ((grp - it % kCG) + kCG) % kCG; i < nitems; i += kCG) {
       const int itm = it + i, s = itm % kNSlot;
-      if (ok && !mbar_wait_bounded(smem_u32(&sm.full[s]), (uint32_t)((itm / kNSlot) & 1),
-                                   &sm.abort_flag)) {
+      const uint32_t fullb = smem_u32(&sm.full[s]), par = (uint32_t)((itm / kNSlot) & 1);
+      if (ok && !mbar_test_wait(fullb, par) && !mbar_wait_bounded(fullb, par, &sm.abort_flag)) {
         ok = false;
         if (lane == 0) {
           report(p.err, SKV_ERR_TIMEOUT);
@@ -1074,7 +1084,11 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     }
     it += nitems;
 
-    // ---- combine the warps' states into this CTA's partial for unit u
+    // ---- combine the warps' states into this CTA's partial for unit u:
+    // one thread per head forms M, L and every warp's scale; each warp then
+    // writes its scaled accumulators to a stash (the idle LUT1 space; the
+    // dense kernel, which has none, adds them into O with shared atomics)
+    // and every output element is summed over the warps
     float l = st.l;
     l += __shfl_xor_sync(0xFFFFFFFFu, l, 4);
     l += __shfl_xor_sync(0xFFFFFFFFu, l, 8);
@@ -1084,38 +1098,53 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       sm.ml[warp][lane][1] = l;
     }
     named_bar_sync(1, nct);
+    if (tid < G) {
+      const int n = tid;
+      float M = -INFINITY;
+      for (int w = 0; w < kNCW; ++w) M = fmaxf(M, sm.ml[w][n][0]);
+      float L = 0.0f;
+      for (int w = 0; w < kNCW; ++w) {
+        const float mw = sm.ml[w][n][0];
+        const float sc = (mw == -INFINITY) ? 0.0f : exp2f(mw - M);
+        sm.wsc[w][n] = sc;
+        L += sm.ml[w][n][1] * sc;
+      }
+      sm.MH[n] = M;
+      sm.LH[n] = M == -INFINITY ? 0.0f : L;
+    }
+    named_bar_sync(1, nct);
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
       const int n = 2 * t4 + j;
       if (n < G) {
-        float M = -INFINITY;
-#pragma unroll
-        for (int w = 0; w < kNCW; ++w) M = fmaxf(M, sm.ml[w][n][0]);
-        const float mw = sm.ml[warp][n][0];
-        const float sc = (mw == -INFINITY) ? 0.0f : exp2f(mw - M);
+        const float sc = sm.wsc[warp][n];
         const float bias = 1152.0f * st.ones[j];  // int8 V offset (see softmax_pv)
+        if constexpr (DENSE) {
 #pragma unroll
-        for (int mt = 0; mt < 8; ++mt) {
-          atomicAdd(&sm.O[n][16 * mt + gq], (st.acc[mt][j] - bias) * sc);
-          atomicAdd(&sm.O[n][16 * mt + gq + 8], (st.acc[mt][2 + j] - bias) * sc);
+          for (int mt = 0; mt < 8; ++mt) {
+            atomicAdd(&sm.O[n][16 * mt + gq], (st.acc[mt][j] - bias) * sc);
+            atomicAdd(&sm.O[n][16 * mt + gq + 8], (st.acc[mt][2 + j] - bias) * sc);
+          }
+        } else {
+          float* stash = lut1p + (warp * G + n) * kHeadDim;
+#pragma unroll
+          for (int mt = 0; mt < 8; ++mt) {
+            stash[16 * mt + gq] = (st.acc[mt][j] - bias) * sc;
+            stash[16 * mt + gq + 8] = (st.acc[mt][2 + j] - bias) * sc;
+          }
         }
       }
     }
     named_bar_sync(1, nct);
-    // this CTA's (M, L) per head
-    float Mh[4], Lh[4];
+    if constexpr (!DENSE) {
+      for (int i = tid; i < G * kHeadDim; i += nct) {
+        const int n = i / kHeadDim, d = i % kHeadDim;
+        float o = 0.0f;
 #pragma unroll
-    for (int n = 0; n < 4; ++n) {
-      Mh[n] = -INFINITY;
-      Lh[n] = 0.0f;
-      if (n < G) {
-        for (int w = 0; w < kNCW; ++w) Mh[n] = fmaxf(Mh[n], sm.ml[w][n][0]);
-        if (Mh[n] != -INFINITY)
-          for (int w = 0; w < kNCW; ++w) {
-            const float mw = sm.ml[w][n][0];
-            if (mw != -INFINITY) Lh[n] += sm.ml[w][n][1] * exp2f(mw - Mh[n]);
-          }
+        for (int w = 0; w < kNCW; ++w) o += lut1p[(w * G + n) * kHeadDim + d];
+        sm.O[n][d] = o;
       }
+      named_bar_sync(1, nct);
     }
     // runs of the page list that touch unit u: run c holds page g when
     // floor(C(g) S / total) == c; the first and the last page of u give the
@@ -1172,10 +1201,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     if (nruns == 1) {
       for (int i = tid; i < G * kHeadDim; i += nct) {
         const int n = i / kHeadDim, d = i % kHeadDim;
-        const float L = Lh[n];
+        const float L = sm.LH[n];
         p.out[(obase + n) * kHeadDim + d] = L > 0.0f ? sm.O[n][d] / L : 0.0f;
         if (d == 0 && p.lse)
-          p.lse[obase + n] = L > 0.0f ? (Mh[n] + log2f(L)) * 0.69314718055994530942f : -INFINITY;
+          p.lse[obase + n] = L > 0.0f ? (sm.MH[n] + log2f(L)) * 0.69314718055994530942f : -INFINITY;
       }
     } else {
       float* part = p.part + (long long)(c + u) * G * kPartStride;
@@ -1183,8 +1212,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         const int n = i / kHeadDim, d = i % kHeadDim;
         __stcg(part + n * kPartStride + 4 + d, sm.O[n][d]);
         if (d == 0) {
-          __stcg(part + n * kPartStride + 0, Mh[n]);
-          __stcg(part + n * kPartStride + 1, Lh[n]);
+          __stcg(part + n * kPartStride + 0, sm.MH[n]);
+          __stcg(part + n * kPartStride + 1, sm.LH[n]);
         }
       }
       __threadfence();
