@@ -26,13 +26,16 @@
 // threads and several issuers run at once; one shared ring keeps several
 // of even the largest (dense 64-token) items in flight.
 //
-// Consumer lane map: lane = 4 t + g, t = token of an 8-row group, g = pair
-// group; each lane carries rows t and t + 8.  Logits: lane (t, g) sums 16
-// pairs (T1/T2: gathers from an fp32 shared-memory LUT holding all G query
-// heads of the group) or 32 dims (T0), a 4-lane reduce-scatter leaves head
-// g's logit in lane (t, g).  P.V: mma.sync m16n8k16, A = V^T fragments read
-// straight from the page (pages store V in fragment order), B = P of the 16
-// rows x 8 heads (zero-padded beyond G), fp32 accumulation.
+// Consumer lane map: lane = 4 t + g, t = token of an 8-row group, g = dim
+// group; each lane carries rows t and t + 8.  Logits of 16 rows: mma.sync
+// m16n8k16 with A = the rows' keys and B = the G query heads (fp32
+// accumulation): T0 / dense rows enter as they are stored (fp16 / bf16);
+// T1 / T2 rows are rebuilt from their codes by gathers from a constant
+// shared table of (share + 1) (cos, sin) per code, split into fp16 high and
+// low halves (two MMAs, fp32-level accuracy).  Lane (t, g) ends with the
+// logits of head g of rows t and t + 8.  P.V: mma.sync m16n8k16, A = V^T
+// fragments read straight from the page (pages store V in fragment order),
+// B = P of the 16 rows x 8 heads (zero-padded beyond G), fp32 accumulation.
 #include <algorithm>
 #include <cstddef>
 
@@ -72,19 +75,16 @@ static_assert(kPasses >= 1 && kGW * kRowsPerWarp == kItemRows, "warp row split")
 constexpr int kMetaTierShift = 4;
 constexpr int kMetaBadShift = 12;
 
-// Shared-memory plan: [ring][LUT1][LUT2][fixed block] (ADA) or
-// [ring][fixed block] (dense).  LUT1 / LUT2 start at shared addresses
-// aligned to their own size, so that a gather address is (code bits) |
-// (pair offset) | (table base) -- one shift and one LOP3; LUT1 is put as
-// high as the fixed block allows, which leaves the ring one contiguous run.
-template <int G>
-struct LutGeom {
-  static constexpr uint32_t kEnt = 4 * G;                // bytes per entry (G fp32)
-  static constexpr uint32_t kCode = kPairs * kEnt;       // bytes per code row
-  static constexpr uint32_t kLut1 = 64 * kCode;          // 6-bit codes
-  static constexpr uint32_t kLut2 = 16 * kCode;          // 4-bit codes
-  static constexpr int kCodeShift = (G == 4) ? 10 : (G == 2 ? 9 : 8);  // log2(kCode)
-};
+// Shared-memory plan: [ring][TBL1][TBL2][fixed block] (ADA) or
+// [ring][fixed block] (dense).  TBL1 / TBL2 are the reconstruction tables
+// of the T1 / T2 codes (see build_tables): entry e at table + 128 e holds
+// 16 copies of its 8 bytes, copy L % 16 read by lane L, so that a warp's
+// gathers of any entries are free of bank conflicts.  TBL2 starts on an
+// 8 KB boundary (its gather address is a LOP3 of the code bits and the
+// lane's base); TBL1 sits right below it and the ring below TBL1.
+constexpr uint32_t kTblEnt = 128;          // bytes per entry: 16 copies x 8 B
+constexpr uint32_t kTbl1 = 256 * kTblEnt;   // T1: entry = code byte (angle6 << 2) | share2
+constexpr uint32_t kTbl2 = 64 * kTblEnt;    // T2: entry = angle4 | share2 << 4
 
 struct PageCopy {  // one page of a ready item, for its issuer
   uint32_t src_lo, src_hi, bytes, dst;
@@ -121,29 +121,25 @@ using DecodeSmemG4 = DecodeSmem<4, false>;
 static_assert(offsetof(DecodeSmemG4, q32) % 16 == 0, "q32 must be 16-byte aligned");
 static_assert(offsetof(DecodeSmemG4, desc) % 16 == 0, "desc must be 16-byte aligned");
 
-// Shared addresses of the ring, LUT1 (LUT2 follows it) and the fixed block
+// Shared addresses of the ring, TBL1 (TBL2 follows it) and the fixed block
 // for a dynamic shared window [base, limit).  False when the ring would be
 // smaller than min_ring bytes.
 template <int G, bool DENSE>
 __host__ __device__ __forceinline__ bool smem_layout(uint32_t base, uint32_t limit,
                                                      uint32_t fixed_bytes, uint32_t min_ring,
                                                      uint32_t& ring_lo, uint32_t& ring_sz,
-                                                     uint32_t& lut1, uint32_t& fixed_at) {
-  using L = LutGeom<G>;
+                                                     uint32_t& tbl1, uint32_t& fixed_at) {
   ring_lo = (base + 127) / 128 * 128;
-  lut1 = 0;
-  uint32_t ring_hi;
-  if constexpr (DENSE) {
-    if (limit < ring_lo + fixed_bytes + 128) return false;
-    fixed_at = (limit - fixed_bytes) / 128 * 128;
-    ring_hi = fixed_at;
-  } else {
-    const uint32_t tot = L::kLut1 + L::kLut2;
-    if (limit < ring_lo + fixed_bytes + tot) return false;
-    lut1 = (limit - fixed_bytes - tot) / L::kLut1 * L::kLut1;
-    if (lut1 <= ring_lo) return false;
-    fixed_at = lut1 + tot;  // 128-aligned: tot is a multiple of 128
-    ring_hi = lut1;
+  tbl1 = 0;
+  if (limit < ring_lo + fixed_bytes + 128) return false;
+  fixed_at = (limit - fixed_bytes) / 128 * 128;
+  uint32_t ring_hi = fixed_at;
+  if constexpr (!DENSE) {
+    if (fixed_at < ring_lo + kTbl1 + kTbl2) return false;
+    const uint32_t tbl2 = (fixed_at - kTbl2) / kTbl2 * kTbl2;
+    if (tbl2 < ring_lo + kTbl1) return false;
+    tbl1 = tbl2 - kTbl1;
+    ring_hi = tbl1;
   }
   ring_sz = (ring_hi - ring_lo) / 128 * 128;
   return ring_sz >= min_ring;
@@ -283,220 +279,191 @@ __device__ __forceinline__ uint32_t lds16(uint32_t a) {
   return v;
 }
 
-// Logit accumulators of one row: G fp32 sums, as packed pairs for G >= 2
-// (fma.rn.f32x2: one issue slot for two heads).
-template <int G>
-struct RowAcc {
-  static constexpr int kN = G >= 2 ? G / 2 : 1;
-  float2 v[kN];
-  __device__ __forceinline__ void zero() {
-#pragma unroll
-    for (int i = 0; i < kN; ++i) v[i] = make_float2(0.0f, 0.0f);
-  }
-  __device__ __forceinline__ void to(float (&s)[G]) const {
-    if constexpr (G >= 2) {
-#pragma unroll
-      for (int i = 0; i < kN; ++i) {
-        s[2 * i] = v[i].x;
-        s[2 * i + 1] = v[i].y;
-      }
-    } else {
-      s[0] = v[0].x;
-    }
-  }
+// ------------------------------------------------------ logits (mma.sync) --
+// Logits of 16 rows are one m16n8k16 MMA chain: A = the rows' keys (16 rows
+// x 16 dims per k-step), B = the query heads (16 dims x 8 columns), fp32
+// accumulation.  Column n holds head (n / 2) % G for even n and zeros for
+// odd n, so that C element c0 (row t, column 2 g) of lane (t, g) is the
+// logit of head g % G and row t, c2 that of row t + 8: the layout the
+// online softmax takes, with no reduction across lanes.
+//
+// The k index is a permutation of the dims fixed by what a lane reads of a
+// row: lane (t, g) reads dims 32 i + 8 g + 0..7 (i = 0..3) of a T0 or dense
+// row (chunk 4 i + g) and the codes of the same dims' pairs 16 i + 4 g + 0..3
+// of a T1 / T2 row.  K-step 2 i + h takes, for lane (t, g), the dims
+// 32 i + 8 g + 4 h + {0, 1} as k = 2 g, 2 g + 1 and + {2, 3} as k = 2 g + 8,
+// 2 g + 9; B follows the same map.
+struct QFrag {
+  uint32_t b[16];   // B fragments, k-step s in b[2 s], b[2 s + 1]
+  uint32_t lo[16];  // dense kernel with fp16 q: the low bf16 halves of q
+  bool two;         // dense kernel: lo is in use
+  float c0;         // logit scale (log2 domain) of fp16 / bf16 keys, this lane's head
+  float c1;         // the same for codes (shares entered as code + 1 = 16 rho^)
 };
 
-// s += w * (G fp32 LUT entries at shared address a), where x holds the
-// 2-bit share b as the float 2^23 + b and w = b + 1 (no conversion
-// instruction: the share bits are placed into the mantissa of 2^23).
-template <int G>
-__device__ __forceinline__ void lut_fma(uint32_t a, float x, RowAcc<G>& s) {
-  if constexpr (G == 4) {
-    const uint4 e = lds128(a);
-    const float2 w = __fadd2_rn(make_float2(x, x), make_float2(-8388607.0f, -8388607.0f));
-    s.v[0] = __ffma2_rn(w, make_float2(__uint_as_float(e.x), __uint_as_float(e.y)), s.v[0]);
-    s.v[1] = __ffma2_rn(w, make_float2(__uint_as_float(e.z), __uint_as_float(e.w)), s.v[1]);
-  } else if constexpr (G == 2) {
-    const uint2 e = lds64(a);
-    const float2 w = __fadd2_rn(make_float2(x, x), make_float2(-8388607.0f, -8388607.0f));
-    s.v[0] = __ffma2_rn(w, make_float2(__uint_as_float(e.x), __uint_as_float(e.y)), s.v[0]);
-  } else {
-    s.v[0].x = fmaf(x - 8388607.0f, __uint_as_float(lds32(a)), s.v[0].x);
+__device__ __forceinline__ float pow2f(int e) { return __uint_as_float((uint32_t)(e + 127) << 23); }
+
+// B fragments of this lane's column from the fp32 query rows q32[head][dim].
+// ADA: keys are fp16, so q enters as fp16 scaled by a power of two per head
+// (its largest element to [2^14, 2^15): bf16 and fp16 queries convert
+// exactly), the scale being taken off in c0 / c1.  Dense: keys are bf16; a
+// bf16 q enters as it is, an fp16 q as the sum of two bf16 halves (exact).
+template <int G, bool DENSE>
+__device__ __forceinline__ void make_qfrag(const float (*q32)[kHeadDim], float qk_scale_log2,
+                                           bool q_bf16, int lane, QFrag& f) {
+  const int gq = lane >> 2, t4 = lane & 3;
+  const bool live = (gq & 1) == 0;
+  const int hn = (gq >> 1) % G;
+  float mx = 0.0f;
+#pragma unroll
+  for (int s = 0; s < 8; ++s) {
+    const float4 x = *reinterpret_cast<const float4*>(&q32[hn][32 * (s >> 1) + 8 * t4 + 4 * (s & 1)]);
+    mx = fmaxf(mx, fmaxf(fmaxf(fabsf(x.x), fabsf(x.y)), fmaxf(fabsf(x.z), fabsf(x.w))));
   }
-}
-
-// byte k of a word whose bytes each hold a 2-bit share, as the float 2^23 + share
-template <int K>
-__device__ __forceinline__ float share_byte(uint32_t spread) {
-  return __uint_as_float(__byte_perm(spread, 0x4B000000u, 0x7440u | K));
-}
-
-// A lane's LUT columns: table base | ((jj ^ (row & 3)) * 4 + g) * entry
-// bytes for jj = 0..3 (rows rA and rA + 8 of a 16-row step share row & 3,
-// which is t & 3 for every step).
-template <int G>
-__device__ __forceinline__ void lut_columns(uint32_t lut, int t, int g, uint32_t (&xo)[4]) {
-  const uint32_t x3 = (uint32_t)t & 3u;
+  mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 1));
+  mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 2));
+  int e = 0;
+  if (!DENSE && mx > 0.0f) e = min(126, 141 - (int)((__float_as_uint(mx) >> 23) & 0xFFu));
+  const float sc = pow2f(e);
+  f.two = DENSE && !q_bf16;
 #pragma unroll
-  for (int jj = 0; jj < 4; ++jj) xo[jj] = lut | ((((uint32_t)jj ^ x3) * 4 + g) * LutGeom<G>::kEnt);
-}
-
-// Partial logits (times 16: shares enter as code + 1) of rows rA, rA + 8 of
-// the T1 page at shared address pg.  Code byte 16g + j of a row holds pair
-// 4 (j ^ (row & 3)) + g as (angle6 << 2) | share2.
-template <int G>
-__device__ __forceinline__ void logits_t1(uint32_t pg, int P, int rA, int g,
-                                          const uint32_t (&xo)[4], RowAcc<G>& sA, RowAcc<G>& sB) {
-  const uint32_t cd = pg + kHdrBytes + 2 * P;
-  const uint4 ca = lds128(cd + rA * 64 + 16 * g);
-  const uint4 cb = lds128(cd + (rA + 8) * 64 + 16 * g);
-  const uint32_t wa[4] = {ca.x, ca.y, ca.z, ca.w};
-  const uint32_t wb[4] = {cb.x, cb.y, cb.z, cb.w};
-  uint32_t qa[4], qb[4];  // shares, one per byte
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    qa[k] = wa[k] & 0x03030303u;
-    qb[k] = wb[k] & 0x03030303u;
-  }
-  using L = LutGeom<G>;
-  // the table base is aligned to the table size: base | pair offset | code
-  // bits (xo: base | the lane's pair offset, see lut_columns); the part of
-  // the pair offset that depends on j alone is added (an immediate of the
-  // shared load)
-  constexpr uint32_t kMask = 0xFCu << (L::kCodeShift - 2);  // angle bits of a byte, scaled
-#pragma unroll
-  for (int j = 0; j < 16; ++j) {
-    const int sh = 8 * (j & 3) - (L::kCodeShift - 2);   // byte j sits at bit 8 (j & 3)
-    const uint32_t xa = sh >= 0 ? (wa[j >> 2] >> sh) : (wa[j >> 2] << -sh);
-    const uint32_t xb = sh >= 0 ? (wb[j >> 2] >> sh) : (wb[j >> 2] << -sh);
-    const uint32_t hi = (j & ~3) * 4 * L::kEnt;
-    float fa, fb;
-    switch (j & 3) {
-      case 0: fa = share_byte<0>(qa[j >> 2]); fb = share_byte<0>(qb[j >> 2]); break;
-      case 1: fa = share_byte<1>(qa[j >> 2]); fb = share_byte<1>(qb[j >> 2]); break;
-      case 2: fa = share_byte<2>(qa[j >> 2]); fb = share_byte<2>(qb[j >> 2]); break;
-      default: fa = share_byte<3>(qa[j >> 2]); fb = share_byte<3>(qb[j >> 2]); break;
+  for (int s = 0; s < 8; ++s) {
+    float4 x = *reinterpret_cast<const float4*>(&q32[hn][32 * (s >> 1) + 8 * t4 + 4 * (s & 1)]);
+    if (!live) x = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    if constexpr (DENSE) {
+      f.b[2 * s] = pack_bf16x2(x.x, x.y);
+      f.b[2 * s + 1] = pack_bf16x2(x.z, x.w);
+      const float hx = __uint_as_float(f.b[2 * s] << 16), hy = __uint_as_float(f.b[2 * s] & 0xFFFF0000u);
+      const float hz = __uint_as_float(f.b[2 * s + 1] << 16),
+                  hw = __uint_as_float(f.b[2 * s + 1] & 0xFFFF0000u);
+      f.lo[2 * s] = pack_bf16x2(x.x - hx, x.y - hy);
+      f.lo[2 * s + 1] = pack_bf16x2(x.z - hz, x.w - hw);
+    } else {
+      f.b[2 * s] = pack_f16x2(x.x * sc, x.y * sc);
+      f.b[2 * s + 1] = pack_f16x2(x.z * sc, x.w * sc);
     }
-    lut_fma<G>(((xa & kMask) | xo[j & 3]) + hi, fa, sA);
-    lut_fma<G>(((xb & kMask) | xo[j & 3]) + hi, fb, sB);
   }
+  // the lane's own head (column 2 t4) is the column of lane 8 t4
+  const float inv = __shfl_sync(0xFFFFFFFFu, pow2f(-e), 8 * t4);
+  f.c0 = qk_scale_log2 * inv;
+  f.c1 = qk_scale_log2 * 0.0625f * inv;
 }
 
-// T2: nibble j of bytes [8g, 8g+8) holds the 4-bit angle of pair
-// 4 (j ^ (row & 3)) + g, crumb j of bytes [32+4g, 36+4g) its share.
-template <int G>
-__device__ __forceinline__ void logits_t2(uint32_t pg, int P, int rA, int g,
-                                          const uint32_t (&xo)[4], RowAcc<G>& sA, RowAcc<G>& sB) {
-  const uint32_t cd = pg + kHdrBytes + 2 * P;
-  const uint2 na = lds64(cd + rA * 48 + 8 * g);
-  const uint2 nb = lds64(cd + (rA + 8) * 48 + 8 * g);
-  const uint32_t ra = lds32(cd + rA * 48 + 32 + 4 * g);
-  const uint32_t rb = lds32(cd + (rA + 8) * 48 + 32 + 4 * g);
-  // crumb j -> byte j >> 2 of word j & 3
-  uint32_t qa[4], qb[4];
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    qa[k] = (ra >> (2 * k)) & 0x03030303u;
-    qb[k] = (rb >> (2 * k)) & 0x03030303u;
-  }
-  using L = LutGeom<G>;
-  constexpr uint32_t kMask = 0xFu << L::kCodeShift;
-#pragma unroll
-  for (int j = 0; j < 16; ++j) {
-    const int sh = 4 * (j & 7) - L::kCodeShift;   // nibble j sits at bit 4 (j & 7)
-    const uint32_t wa = (j < 8) ? na.x : na.y, wb = (j < 8) ? nb.x : nb.y;
-    const uint32_t xa = sh >= 0 ? (wa >> sh) : (wa << -sh);
-    const uint32_t xb = sh >= 0 ? (wb >> sh) : (wb << -sh);
-    const uint32_t hi = (j & ~3) * 4 * L::kEnt;
-    float fa, fb;
-    switch (j >> 2) {
-      case 0: fa = share_byte<0>(qa[j & 3]); fb = share_byte<0>(qb[j & 3]); break;
-      case 1: fa = share_byte<1>(qa[j & 3]); fb = share_byte<1>(qb[j & 3]); break;
-      case 2: fa = share_byte<2>(qa[j & 3]); fb = share_byte<2>(qb[j & 3]); break;
-      default: fa = share_byte<3>(qa[j & 3]); fb = share_byte<3>(qb[j & 3]); break;
+// Reconstruction tables: T1 entry e = (a << 2) | s and T2 entry 256 + (a | s << 4)
+// hold the pair (x, y) = (s + 1) (cos, sin)(2 pi a / 2^b) (16 times the
+// key pair of unit radius: shares enter as code + 1) as fp16 hi and lo
+// halves, x = hi + lo to about 2^-22 relative: {hi(x), hi(y)}, {lo(x), lo(y)}.
+// The T2 entries follow T1's (TBL2 = TBL1 + 32 KB).
+__device__ __forceinline__ void build_tables(const DecodeParams& p, uint8_t* tbl1p, int n_entries,
+                                             int tid, int nthreads) {
+  for (int e = tid; e < n_entries; e += nthreads) {
+    float cs, sn, w;
+    if (e < 256) {
+      cs = p.cos6[e >> 2];
+      sn = p.sin6[e >> 2];
+      w = (float)((e & 3) + 1);
+    } else {
+      cs = p.cos4[(e - 256) & 15];
+      sn = p.sin4[(e - 256) & 15];
+      w = (float)(((e - 256) >> 4) + 1);
     }
-    lut_fma<G>(((xa & kMask) | xo[j & 3]) + hi, fa, sA);
-    lut_fma<G>(((xb & kMask) | xo[j & 3]) + hi, fb, sB);
+    const float x = w * cs, y = w * sn;
+    const __half hx = __float2half_rn(x), hy = __float2half_rn(y);
+    const __half lx = __float2half_rn(x - __half2float(hx)), ly = __float2half_rn(y - __half2float(hy));
+    const uint32_t hi = (uint32_t)__half_as_ushort(hx) | ((uint32_t)__half_as_ushort(hy) << 16);
+    const uint32_t lo = (uint32_t)__half_as_ushort(lx) | ((uint32_t)__half_as_ushort(ly) << 16);
+    uint4* dst = reinterpret_cast<uint4*>(tbl1p + (size_t)e * kTblEnt);
+#pragma unroll
+    for (int r = 0; r < 8; ++r) dst[r] = make_uint4(hi, lo, hi, lo);
   }
 }
 
-// fp16 pair (one 32-bit word) -> two fp32 values scaled by 2^-112, exactly
-// (normal and subnormal halves): the half's exponent and mantissa bits are
-// moved into an fp32 at bit 13; the 2^112 goes into the logit scale.
-__device__ __forceinline__ void half2_bits_to_f32_scaled(uint32_t w, float& lo, float& hi) {
-  lo = __int_as_float(((int32_t)(w << 16) >> 3) & (int32_t)0x8FFFE000);
-  hi = __int_as_float(((int32_t)w >> 3) & (int32_t)0x8FFFE000);
-}
-__device__ __forceinline__ void bf162_bits_to_f32(uint32_t w, float& lo, float& hi) {
-  lo = __int_as_float(w << 16);
-  hi = __int_as_float(w & 0xFFFF0000u);
+template <bool BF16>
+__device__ __forceinline__ void mma_k16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                        uint32_t a3, uint32_t b0, uint32_t b1) {
+  if constexpr (BF16)
+    mma_16816k16_bf16(d, a0, a1, a2, a3, b0, b1);
+  else
+    mma_16816k16_f16(d, a0, a1, a2, a3, b0, b1);
 }
 
-// T0 (fp16 K) or dense (bf16 K): lane (t, g) covers dims 8c..8c+7 for the
-// chunks c = 4i + g, stored at chunk position c ^ 4 (row & 1).
-template <int G, bool BF16>
-__device__ __forceinline__ void logits_dense(uint32_t pg, int rA, int g, uint32_t q32,
-                                             float (&sA)[G], float (&sB)[G]) {
+// T0 (fp16 K) or dense (bf16 K) rows rA, rA + 8: lane (t, g) reads chunks
+// c = 4 i + g (dims 8 c .. 8 c + 7), stored at chunk position c ^ 4 (row & 1).
+// Two accumulators (even / odd k-steps) halve the MMA dependency chain.
+template <bool BF16, bool TWO>
+__device__ __forceinline__ void logits_k16(uint32_t pg, int rA, int g, const QFrag& f,
+                                           float (&c)[4], float (&d)[4]) {
   const uint32_t ka = pg + kHdrBytes + rA * 256;
   const uint32_t kb = ka + 8 * 256;
   const uint32_t sw = 4u * (rA & 1);
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const uint32_t c = 4 * i + g;
-    const uint4 xa = lds128(ka + (c ^ sw) * 16);
-    const uint4 xb = lds128(kb + (c ^ sw) * 16);
-    const uint32_t wa[4] = {xa.x, xa.y, xa.z, xa.w};
-    const uint32_t wb[4] = {xb.x, xb.y, xb.z, xb.w};
-    float fa[8], fb[8];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      if constexpr (BF16) {
-        bf162_bits_to_f32(wa[e], fa[2 * e], fa[2 * e + 1]);
-        bf162_bits_to_f32(wb[e], fb[2 * e], fb[2 * e + 1]);
-      } else {
-        half2_bits_to_f32_scaled(wa[e], fa[2 * e], fa[2 * e + 1]);
-        half2_bits_to_f32_scaled(wb[e], fb[2 * e], fb[2 * e + 1]);
-      }
-    }
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-      const uint4 q0 = lds128(q32 + (h * kHeadDim + 8 * c) * 4);
-      const uint4 q1 = lds128(q32 + (h * kHeadDim + 8 * c + 4) * 4);
-      const float qv[8] = {__uint_as_float(q0.x), __uint_as_float(q0.y), __uint_as_float(q0.z),
-                           __uint_as_float(q0.w), __uint_as_float(q1.x), __uint_as_float(q1.y),
-                           __uint_as_float(q1.z), __uint_as_float(q1.w)};
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        sA[h] = fmaf(fa[e], qv[e], sA[h]);
-        sB[h] = fmaf(fb[e], qv[e], sB[h]);
-      }
+    const uint32_t pos = (((uint32_t)(4 * i + g)) ^ sw) * 16;
+    const uint4 xa = lds128(ka + pos), xb = lds128(kb + pos);
+    mma_k16<BF16>(c, xa.x, xb.x, xa.y, xb.y, f.b[4 * i], f.b[4 * i + 1]);
+    mma_k16<BF16>(d, xa.z, xb.z, xa.w, xb.w, f.b[4 * i + 2], f.b[4 * i + 3]);
+    if constexpr (TWO) {
+      mma_k16<BF16>(c, xa.x, xb.x, xa.y, xb.y, f.lo[4 * i], f.lo[4 * i + 1]);
+      mma_k16<BF16>(d, xa.z, xb.z, xa.w, xb.w, f.lo[4 * i + 2], f.lo[4 * i + 3]);
     }
   }
 }
 
-// 4-lane reduce-scatter: afterwards lane g holds the full sum of head g % G.
-template <int G>
-__device__ __forceinline__ float reduce_scatter(float (&s)[G], int g) {
-  if constexpr (G == 4) {
-    const bool up = (g & 2) != 0;
-    const float x0 = __shfl_xor_sync(0xFFFFFFFFu, up ? s[0] : s[2], 2);
-    const float x1 = __shfl_xor_sync(0xFFFFFFFFu, up ? s[1] : s[3], 2);
-    const float a0 = (up ? s[2] : s[0]) + x0;
-    const float a1 = (up ? s[3] : s[1]) + x1;
-    const bool odd = (g & 1) != 0;
-    const float y = __shfl_xor_sync(0xFFFFFFFFu, odd ? a0 : a1, 1);
-    return (odd ? a1 : a0) + y;
-  } else if constexpr (G == 2) {
-    const float a0 = s[0] + __shfl_xor_sync(0xFFFFFFFFu, s[0], 2);
-    const float a1 = s[1] + __shfl_xor_sync(0xFFFFFFFFu, s[1], 2);
-    const bool odd = (g & 1) != 0;
-    const float y = __shfl_xor_sync(0xFFFFFFFFu, odd ? a0 : a1, 1);
-    return (odd ? a1 : a0) + y;
-  } else {
-    float a = s[0];
-    a += __shfl_xor_sync(0xFFFFFFFFu, a, 2);
-    a += __shfl_xor_sync(0xFFFFFFFFu, a, 1);
-    return a;
+// table address of code byte k of w (T1: entry = the byte)
+__device__ __forceinline__ uint32_t t1_addr(uint32_t w, int k, uint32_t tb) {
+  return tb + (__byte_perm(w, 0u, 0x4440u | (uint32_t)k) << 7);
+}
+
+// T1 rows rA, rA + 8: lane (t, g) reads code bytes [16 g, 16 g + 16) of
+// each row; byte j holds pair 16 (j >> 2) + 4 g + (j & 3), so k-step s uses
+// bytes 2 s (k = 2 g, 2 g + 1) and 2 s + 1 (k = 2 g + 8, 2 g + 9).  hi and lo
+// table halves go to separate accumulators.
+__device__ __forceinline__ void logits_t1(uint32_t pg, int P, int rA, int g, uint32_t tb,
+                                          const QFrag& f, float (&c)[4], float (&d)[4]) {
+  const uint32_t cd = pg + kHdrBytes + 2 * P;
+  const uint4 ca = lds128(cd + rA * 64 + 16 * g);
+  const uint4 cb = lds128(cd + (rA + 8) * 64 + 16 * g);
+  const uint32_t wa[4] = {ca.x, ca.y, ca.z, ca.w};
+  const uint32_t wb[4] = {cb.x, cb.y, cb.z, cb.w};
+#pragma unroll
+  for (int s = 0; s < 8; ++s) {
+    const int i = s >> 1, k0 = 2 * (s & 1);
+    const uint2 ea0 = lds64(t1_addr(wa[i], k0, tb)), ea1 = lds64(t1_addr(wa[i], k0 + 1, tb));
+    const uint2 eb0 = lds64(t1_addr(wb[i], k0, tb)), eb1 = lds64(t1_addr(wb[i], k0 + 1, tb));
+    mma_k16<false>(c, ea0.x, eb0.x, ea1.x, eb1.x, f.b[2 * s], f.b[2 * s + 1]);
+    mma_k16<false>(d, ea0.y, eb0.y, ea1.y, eb1.y, f.b[2 * s], f.b[2 * s + 1]);
+  }
+}
+
+// table address of T2 pair j: nibble j of the 64-bit nibble word (n0, n1),
+// crumb j of the share word cw; entry angle | share << 4 (TBL2 is 8 KB
+// aligned: the address is tb | entry << 7; j is a constant once unrolled)
+__device__ __forceinline__ uint32_t t2_addr(uint32_t n0, uint32_t n1, uint32_t cw, int j,
+                                            uint32_t tb) {
+  const int sn = 4 * (j & 7) - 7, sc = 2 * j - 11;
+  const uint32_t nw = j < 8 ? n0 : n1;
+  const uint32_t xn = sn >= 0 ? (nw >> sn) : (nw << -sn);
+  const uint32_t xc = sc >= 0 ? (cw >> sc) : (cw << -sc);
+  return (xn & 0x780u) | (xc & 0x1800u) | tb;
+}
+
+// T2 rows rA, rA + 8: nibble j of bytes [8 g, 8 g + 8) holds the angle of
+// pair 16 (j >> 2) + 4 g + (j & 3), crumb j of bytes [32 + 4 g, 36 + 4 g) its share.
+__device__ __forceinline__ void logits_t2(uint32_t pg, int P, int rA, int g, uint32_t tb,
+                                          const QFrag& f, float (&c)[4], float (&d)[4]) {
+  const uint32_t cd = pg + kHdrBytes + 2 * P;
+  const uint2 na = lds64(cd + rA * 48 + 8 * g);
+  const uint2 nb = lds64(cd + (rA + 8) * 48 + 8 * g);
+  const uint32_t ra = lds32(cd + rA * 48 + 32 + 4 * g);
+  const uint32_t rb = lds32(cd + (rA + 8) * 48 + 32 + 4 * g);
+#pragma unroll
+  for (int s = 0; s < 8; ++s) {
+    const uint2 ea0 = lds64(t2_addr(na.x, na.y, ra, 2 * s, tb));
+    const uint2 ea1 = lds64(t2_addr(na.x, na.y, ra, 2 * s + 1, tb));
+    const uint2 eb0 = lds64(t2_addr(nb.x, nb.y, rb, 2 * s, tb));
+    const uint2 eb1 = lds64(t2_addr(nb.x, nb.y, rb, 2 * s + 1, tb));
+    mma_k16<false>(c, ea0.x, eb0.x, ea1.x, eb1.x, f.b[2 * s], f.b[2 * s + 1]);
+    mma_k16<false>(d, ea0.y, eb0.y, ea1.y, eb1.y, f.b[2 * s], f.b[2 * s + 1]);
   }
 }
 
@@ -602,12 +569,12 @@ __device__ __forceinline__ void softmax_pv(float lA, float lB, float vsA, float 
   }
 }
 
-// 16 rows [row0, row0 + 16) of one page at shared address pg.
+// 16 rows [row0, row0 + 16) of one page at shared address pg; tb1 / tb2:
+// this lane's copy in TBL1 / TBL2.
 template <int G, bool DENSE>
 __device__ __forceinline__ void process_rows(const DecodeParams& p, uint32_t pg, uint32_t tier,
-                                             int row0, const uint32_t (&xo1)[4],
-                                             const uint32_t (&xo2)[4], uint32_t q32,
-                                             WarpState& st, int lane) {
+                                             int row0, const QFrag& qf, uint32_t tb1,
+                                             uint32_t tb2, WarpState& st, int lane) {
   const int t = lane >> 2, g = lane & 3;
   const int P = p.P;
   // header {u16 count, u8 tier, u8 magic}
@@ -620,52 +587,37 @@ __device__ __forceinline__ void process_rows(const DecodeParams& p, uint32_t pg,
   if ((uint32_t)row0 >= cnt) return;
   const int rA = row0 + t, rB = rA + 8;
   const bool vA = (uint32_t)rA < cnt, vB = (uint32_t)rB < cnt;
-  float sA[G], sB[G];
+  float c[4] = {0.0f, 0.0f, 0.0f, 0.0f}, d[4] = {0.0f, 0.0f, 0.0f, 0.0f};
   const uint32_t vsec_dense = pg + kHdrBytes + 256 * P + (row0 >> 3) * 2048;
   if constexpr (DENSE) {
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-      sA[h] = 0.0f;
-      sB[h] = 0.0f;
-    }
-    logits_dense<G, true>(pg, rA, g, q32, sA, sB);
-    const float a = reduce_scatter<G>(sA, g), b = reduce_scatter<G>(sB, g);
-    const float c = p.qk_scale_log2;
-    softmax_pv<G, 2>(vA ? a * c : -INFINITY, vB ? b * c : -INFINITY, 1.0f, 1.0f, vsec_dense,
-                     vsec_dense + 2048, st, lane);
+    if (qf.two)
+      logits_k16<true, true>(pg, rA, g, qf, c, d);
+    else
+      logits_k16<true, false>(pg, rA, g, qf, c, d);
+    const float a = c[0] + d[0], b = c[2] + d[2];
+    softmax_pv<G, 2>(vA ? a * qf.c0 : -INFINITY, vB ? b * qf.c0 : -INFINITY, 1.0f, 1.0f,
+                     vsec_dense, vsec_dense + 2048, st, lane);
   } else {
     if (tier == SKV_TIER_T0) {
-#pragma unroll
-      for (int h = 0; h < G; ++h) {
-        sA[h] = 0.0f;
-        sB[h] = 0.0f;
-      }
-      logits_dense<G, false>(pg, rA, g, q32, sA, sB);
-      const float a = reduce_scatter<G>(sA, g), b = reduce_scatter<G>(sB, g);
-      const float c = p.qk_scale_log2 * 5.192296858534828e+33f;  // 2^112
-      softmax_pv<G, 1>(vA ? a * c : -INFINITY, vB ? b * c : -INFINITY, 1.0f, 1.0f, vsec_dense,
-                       vsec_dense + 2048, st, lane);
+      logits_k16<false, false>(pg, rA, g, qf, c, d);
+      const float a = c[0] + d[0], b = c[2] + d[2];
+      softmax_pv<G, 1>(vA ? a * qf.c0 : -INFINITY, vB ? b * qf.c0 : -INFINITY, 1.0f, 1.0f,
+                       vsec_dense, vsec_dense + 2048, st, lane);
     } else {
       const bool t1 = tier == SKV_TIER_T1;
-      RowAcc<G> rA2, rB2;
-      rA2.zero();
-      rB2.zero();
       if (t1)
-        logits_t1<G>(pg, P, rA, g, xo1, rA2, rB2);
+        logits_t1(pg, P, rA, g, tb1, qf, c, d);
       else
-        logits_t2<G>(pg, P, rA, g, xo2, rA2, rB2);
-      rA2.to(sA);
-      rB2.to(sB);
-      const float a = reduce_scatter<G>(sA, g), b = reduce_scatter<G>(sB, g);
+        logits_t2(pg, P, rA, g, tb2, qf, c, d);
+      const float a = c[0] + d[0], b = c[2] + d[2];
       const int cb = t1 ? 64 : 48;
       const uint32_t rs = pg + kHdrBytes, ss = pg + kHdrBytes + (2 + cb) * P;
       const float rtA = __half2float(__ushort_as_half((unsigned short)lds16(rs + 2 * rA)));
       const float rtB = __half2float(__ushort_as_half((unsigned short)lds16(rs + 2 * rB)));
       const float vsA = __half2float(__ushort_as_half((unsigned short)lds16(ss + 2 * rA)));
       const float vsB = __half2float(__ushort_as_half((unsigned short)lds16(ss + 2 * rB)));
-      const float c = p.qk_scale_log2 * 0.0625f;  // shares entered as code + 1 = 16 rho^
       const uint32_t vsec = pg + kHdrBytes + (2 + cb + 2) * P + (row0 >> 3) * 1024;
-      softmax_pv<G, 0>(vA ? a * (rtA * c) : -INFINITY, vB ? b * (rtB * c) : -INFINITY,
+      softmax_pv<G, 0>(vA ? a * (rtA * qf.c1) : -INFINITY, vB ? b * (rtB * qf.c1) : -INFINITY,
                        vA ? vsA : 0.0f, vB ? vsB : 0.0f, vsec, vsec + 1024, st, lane);
     }
   }
@@ -676,7 +628,6 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     decode_kernel(const __grid_constant__ DecodeParams p) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
   using Smem = DecodeSmem<G, DENSE>;
-  using LG = LutGeom<G>;
   const uint32_t base = smem_u32(smem_raw);
   const uint32_t limit = base + (uint32_t)p.smem_bytes;
   const int tid = threadIdx.x;
@@ -697,10 +648,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   // the largest item: ipp pages of the largest payload
   int maxpay = p.payload[0];
   if (!DENSE) maxpay = max(maxpay, max(p.payload[1], p.payload[2]));
-  uint32_t ring_lo, R, lut1, fixed_at;
+  uint32_t ring_lo, R, tbl1, fixed_at;
   const bool plan_ok = smem_layout<G, DENSE>(base, limit, (uint32_t)sizeof(Smem),
-                                             (uint32_t)(ipp * maxpay), ring_lo, R, lut1, fixed_at);
-  const uint32_t lut2 = lut1 + LG::kLut1;
+                                             (uint32_t)(ipp * maxpay), ring_lo, R, tbl1, fixed_at);
   Smem& sm = *reinterpret_cast<Smem*>(smem_raw + (plan_ok ? fixed_at - base : 0u));
 
   if (tid == 0) {
@@ -970,12 +920,13 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   const int nct = kNCW * 32;
   const int t4 = lane & 3, gq = lane >> 2;
   const int grp = warp / kGW, wi = warp % kGW;  // consumer group, warp within it
-  uint32_t xo1[4], xo2[4];  // this lane's LUT columns (see lut_columns)
-  lut_columns<G>(lut1, lane >> 2, lane & 3, xo1);
-  lut_columns<G>(lut2, lane >> 2, lane & 3, xo2);
-  const uint32_t q32 = smem_u32(sm.q32);
-  float* lut1p = reinterpret_cast<float*>(smem_raw + (lut1 - base));
-  float* lut2p = reinterpret_cast<float*>(smem_raw + (lut2 - base));
+  // this lane's copy in the reconstruction tables; TBL1's space doubles as
+  // the stash of the combine (then rebuilt before the next unit)
+  const uint32_t tb1 = tbl1 + (uint32_t)(lane & 15) * 8u, tb2 = tb1 + kTbl1;
+  uint8_t* const tbl1p = smem_raw + (tbl1 - base);
+  float* const stashp = reinterpret_cast<float*>(tbl1p);
+  static_assert(DENSE || kNCW * 4 * kHeadDim * 4 <= (int)kTbl1, "combine stash fits TBL1");
+  int tbl_entries = DENSE ? 0 : 256 + 64;  // table entries still to build
   int it = 0;  // item index within the run
   bool ok = true;
   for (int u = u0; u < U; ++u) {
@@ -993,53 +944,13 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
                               : __half2float(__ushort_as_half(raw));
       sm.O[h][d] = 0.0f;
     }
-    named_bar_sync(1, nct);
     if constexpr (!DENSE) {
-      // the tables this CTA's pages of the unit read (both when the page
-      // table gives no per-tier offsets)
-      bool need1 = true, need2 = true;
-      if (p.tier_indptr) {
-        const long long s1 = si.seg_start(3 * u + 1), s2 = si.seg_start(3 * u + 2),
-                        s3 = si.seg_start(3 * u + 3);
-        need1 = max(a, s1) < min(b, s2);
-        need2 = max(a, s2) < min(b, s3);
-      }
-#pragma unroll 2
-      for (int i = tid; need1 && i < 64 * kPairs; i += nct) {
-        const int cc = i >> 6, pr = i & 63;
-        const float cs = p.cos6[cc], sn = p.sin6[cc];
-        float v[G];
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-          const float2 qp = *reinterpret_cast<const float2*>(&sm.q32[h][2 * pr]);
-          v[h] = fmaf(qp.x, cs, qp.y * sn);
-        }
-        if constexpr (G == 4) {
-          *reinterpret_cast<float4*>(&lut1p[i * 4]) = make_float4(v[0], v[1], v[2], v[3]);
-        } else {
-#pragma unroll
-          for (int h = 0; h < G; ++h) lut1p[i * G + h] = v[h];
-        }
-      }
-#pragma unroll 2
-      for (int i = tid; need2 && i < 16 * kPairs; i += nct) {
-        const int cc = i >> 6, pr = i & 63;
-        const float cs = p.cos4[cc], sn = p.sin4[cc];
-        float v[G];
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-          const float2 qp = *reinterpret_cast<const float2*>(&sm.q32[h][2 * pr]);
-          v[h] = fmaf(qp.x, cs, qp.y * sn);
-        }
-        if constexpr (G == 4) {
-          *reinterpret_cast<float4*>(&lut2p[i * 4]) = make_float4(v[0], v[1], v[2], v[3]);
-        } else {
-#pragma unroll
-          for (int h = 0; h < G; ++h) lut2p[i * G + h] = v[h];
-        }
-      }
-      named_bar_sync(1, nct);
+      if (tbl_entries) build_tables(p, tbl1p, tbl_entries, tid, nct);
+      tbl_entries = 0;
     }
+    named_bar_sync(1, nct);
+    QFrag qf;
+    make_qfrag<G, DENSE>(sm.q32, p.qk_scale_log2, p.q_bf16 != 0, lane, qf);
     WarpState st;
     st.m = kNoMax;
     st.l = 0.0f;
@@ -1075,7 +986,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
                                          : (kp == 1 ? (d.z & 0xFFFFu)
                                                     : (kp == 2 ? (d.z >> 16) : d.w));
             process_rows<G, DENSE>(p, d.x + rel, (d.y >> (kMetaTierShift + 2 * kp)) & 3u, row0,
-                                   xo1, xo2, q32, st, lane);
+                                   qf, tb1, tb2, st, lane);
           }
         }
       }
@@ -1086,8 +997,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
 
     // ---- combine the warps' states into this CTA's partial for unit u:
     // one thread per head forms M, L and every warp's scale; each warp then
-    // writes its scaled accumulators to a stash (the idle LUT1 space; the
-    // dense kernel, which has none, adds them into O with shared atomics)
+    // writes its scaled accumulators to a stash (TBL1's space, rebuilt before
+    // the next unit; the dense kernel, which has no tables, adds them into O
+    // with shared atomics)
     // and every output element is summed over the warps
     float l = st.l;
     l += __shfl_xor_sync(0xFFFFFFFFu, l, 4);
@@ -1126,7 +1038,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
             atomicAdd(&sm.O[n][16 * mt + gq + 8], (st.acc[mt][2 + j] - bias) * sc);
           }
         } else {
-          float* stash = lut1p + (warp * G + n) * kHeadDim;
+          float* stash = stashp + (warp * G + n) * kHeadDim;
 #pragma unroll
           for (int mt = 0; mt < 8; ++mt) {
             stash[16 * mt + gq] = (st.acc[mt][j] - bias) * sc;
@@ -1141,9 +1053,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         const int n = i / kHeadDim, d = i % kHeadDim;
         float o = 0.0f;
 #pragma unroll
-        for (int w = 0; w < kNCW; ++w) o += lut1p[(w * G + n) * kHeadDim + d];
+        for (int w = 0; w < kNCW; ++w) o += stashp[(w * G + n) * kHeadDim + d];
         sm.O[n][d] = o;
       }
+      tbl_entries = 256;  // TBL1 holds the stash now
       named_bar_sync(1, nct);
     }
     // runs of the page list that touch unit u: run c holds page g when
@@ -1352,9 +1265,9 @@ template <int G, bool DENSE>
 bool decode_plan_ok(int smem_bytes, int max_item) {
   // the dynamic shared window starts at offset 0 or after a 1 KB reserve
   for (uint32_t b = 0; b <= 1024; b += 1024) {
-    uint32_t rlo, rsz, lut1, fixed_at;
+    uint32_t rlo, rsz, tbl1, fixed_at;
     if (!smem_layout<G, DENSE>(b, b + (uint32_t)smem_bytes, (uint32_t)sizeof(DecodeSmem<G, DENSE>),
-                               (uint32_t)max_item, rlo, rsz, lut1, fixed_at))
+                               (uint32_t)max_item, rlo, rsz, tbl1, fixed_at))
       return false;
   }
   return true;

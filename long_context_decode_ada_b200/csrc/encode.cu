@@ -222,7 +222,6 @@ __global__ void __launch_bounds__(256) encode_kernel(const __grid_constant__ Enc
     *reinterpret_cast<uint16_t*>(rsec + 2 * row) = rt;
     *reinterpret_cast<uint16_t*>(ssec + 2 * row) = __half_as_ushort(sh);
   }
-  const uint32_t x3 = row & 3;
   uint8_t* crow = csec + row * cb;
   if (t1) {
     // word wd (bytes 4wd..4wd+3): group g = wd / 4, j = 4 (wd % 4) + e
@@ -231,7 +230,7 @@ __global__ void __launch_bounds__(256) encode_kernel(const __grid_constant__ Enc
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const int g = wd >> 2, j = 4 * (wd & 3) + e;
-      const int pr = 4 * (j ^ (int)x3) + g;
+      const int pr = 16 * (j >> 2) + 4 * g + (j & 3);
       const uint32_t src = __shfl_sync(0xFFFFFFFFu, packed, pr >> 1);
       const uint32_t th = (src >> (8 * (pr & 1))) & 0xFFu;
       const uint32_t rh = (src >> (16 + 8 * (pr & 1))) & 0xFFu;
@@ -248,7 +247,7 @@ __global__ void __launch_bounds__(256) encode_kernel(const __grid_constant__ Enc
     for (int e = 0; e < 16; ++e) {
       const int g = crumbs ? wd - 8 : (wd >> 1);
       const int j = crumbs ? e : 8 * (wd & 1) + (e & 7);
-      const int pr = 4 * (j ^ (int)x3) + g;
+      const int pr = 16 * (j >> 2) + 4 * g + (j & 3);
       const uint32_t src = __shfl_sync(0xFFFFFFFFu, packed, pr >> 1);
       if (crumbs) {
         const uint32_t rh = (src >> (16 + 8 * (pr & 1))) & 3u;

@@ -552,10 +552,11 @@ int orc_allocate(int B, int Hkv, int Tmax, int d, int P, const int32_t* seq_lens
  * Within-row orders (the decode kernel reads with lane = 4*t + g, t the token
  * in an 8-row group and g one of four pair groups):
  *   T0 K row r: 16 chunks of 8 dims; chunk c at chunk position c ^ (4*(r&1)).
- *   T1 code row r: byte 16*g + j holds pair 4*(j ^ (r&3)) + g, as
- *       (angle6 << 2) | share2.
+ *   T1 code row r: byte 16*g + j holds pair 16*(j/4) + 4*g + j%4, as
+ *       (angle6 << 2) | share2 (lane g then holds the pairs of the dims
+ *       that it reads of a T0 row: chunks 4i + g).
  *   T2 code row r: nibble j of bytes [8g, 8g+8) (low nibble first) holds the
- *       4-bit angle of pair 4*(j ^ (r&3)) + g; crumb j of bytes
+ *       4-bit angle of pair 16*(j/4) + 4*g + j%4; crumb j of bytes
  *       [32+4g, 36+4g) (bits 2j..2j+1 of that little-endian word) its share.
  *   V (all tiers), per 8-row group k, m-tile mt (dims 16mt..16mt+15), lane
  *       L = 4*g + t4 (g = 0..7, t4 = 0..3): the four values
@@ -621,7 +622,7 @@ static void write_row(uint8_t* page, int tier, int P, int d, int r,
     put16(ss + 2 * r, sc);
     uint8_t* row = cs + (int64_t)r * codes_bytes;
     for (int p = 0; p < d / 2; p++) {
-        int g = p % 4, m = p / 4, j = m ^ (r & 3);
+        int g = (p / 4) % 4, j = 4 * (p / 16) + p % 4;
         int rho = orc_rho_code(k[2 * p], k[2 * p + 1], R2, d);
         if (tier == TIER_T1) {
             int th = orc_angle_code(k[2 * p], k[2 * p + 1], BITS_T1);

@@ -209,8 +209,8 @@ def read_row(page, tier, P, r):
     th = np.zeros(64, np.int64)
     rho = np.zeros(64, np.int64)
     for p in range(64):
-        g, m = p % 4, p // 4
-        j = m ^ (r & 3)
+        g = (p // 4) % 4
+        j = 4 * (p // 16) + p % 4
         if tier == 1:
             byte = int(row[16 * g + j])
             th[p], rho[p] = byte >> 2, byte & 3
