@@ -694,8 +694,19 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     // parallel as releases arrive.  kIss end-of-run markers follow the last
     // item, one per issuer.
     int u = u0;
+    long long pg = g0;  // first page of the next batch
+    // the ids of a batch's pages are loaded one batch ahead (read up to the
+    // end of the run, not of the unit: a batch starts where the previous one
+    // ended, or at the first page of the next unit, which follows it)
+    uint32_t idn[kMaxIPP];
+#pragma unroll
+    for (int q = 0; q < kMaxIPP; ++q) {
+      const long long pq = pg + (long long)lane * ipp + q;
+      idn[q] = (q < ipp && pq < g1) ? __ldg(p.ids + pq) : 0u;
+    }
     long long ub = min(g1, (long long)p.indptr[u0 + 1]);  // end of the current unit's run
-    long long pg = g0;                                     // first page of the next batch
+    // the end of the next unit, loaded one unit ahead
+    long long ub_next = u0 + 2 <= U ? (long long)p.indptr[u0 + 2] : g1;
     int it = 0;                 // next item
     int tail = 0;               // oldest item not known to be released
     uint32_t wr = 0;            // ring write offset
@@ -712,19 +723,26 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     while (ok && pg < g1) {
       while (pg >= ub) {  // next unit with pages in this run
         ++u;
-        ub = min(g1, (long long)p.indptr[u + 1]);
+        ub = min(g1, ub_next);
+        ub_next = u + 2 <= U ? (long long)p.indptr[u + 2] : g1;
       }
       const int nb = (int)min(32LL, (ub - pg + ipp - 1) / ipp);  // items in this batch
       // ---- lane-parallel decode of item it + lane
       uint32_t plo[kMaxIPP], phi[kMaxIPP], psz[kMaxIPP];
       uint32_t total = 0, imeta = 0, relz = 0, relw = 0;
+      uint32_t id[kMaxIPP];
+#pragma unroll
+      for (int q = 0; q < kMaxIPP; ++q) id[q] = idn[q];
+      {
+        const long long pn = min(ub, pg + (long long)nb * ipp);  // the next batch's first page
+#pragma unroll
+        for (int q = 0; q < kMaxIPP; ++q) {
+          const long long pq = pn + (long long)lane * ipp + q;
+          idn[q] = (q < ipp && pq < g1) ? __ldg(p.ids + pq) : 0u;
+        }
+      }
       if (lane < nb) {
         const long long ps = pg + (long long)lane * ipp;
-        // the ids are read up to the end of the run, not of the unit: the
-        // loads do not wait for the unit bound
-        uint32_t id[kMaxIPP];
-#pragma unroll
-        for (int q = 0; q < kMaxIPP; ++q) id[q] = (q < ipp && ps + q < g1) ? __ldg(p.ids + ps + q) : 0u;
         const int n = (int)min((long long)ipp, ub - ps);
         imeta = (uint32_t)n;
 #pragma unroll
