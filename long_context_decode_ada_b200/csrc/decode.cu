@@ -62,10 +62,12 @@ constexpr int kPasses = kRowsPerWarp / 16;
 constexpr int kNSlot = 16;                    // items in flight, at most
 constexpr int kMaxIPP = kItemRows / 16;       // pages per item (P >= 16)
 constexpr int kMergeRuns = 128;               // runs per unit merged through shared memory
+constexpr int kMergeBatch = 20;               // merge: runs whose loads are issued together
 constexpr int kTouchedUnits = 16;             // units whose segment costs a CTA keeps
 static_assert(kCG >= 1 && kCG <= 4, "consumer groups: 1..4");
 static_assert(kIss >= 1 && kIss <= 4, "issuers: 1..4");
 static_assert(kPasses >= 1 && kGW * kRowsPerWarp == kItemRows, "warp row split");
+static_assert(kMergeRuns <= kHeadDim, "merge: the runs' l values are kept in a row of O");
 
 // Item descriptor (16 B, written by the producer before it arms the slot's
 // full barrier): x = shared address of the item, y = meta, z/w = byte
@@ -188,6 +190,18 @@ __device__ __forceinline__ long long run_begin_in_unit(const SplitInfo& si,
   return seg[3];
 }
 
+// Unit-aligned split (used when there are at most as many units as runs):
+// unit u gets the runs [B(u), B(u + 1)), B(u) = u + round(P(u) (S - U) / C)
+// with P(u) the cost before unit u and C the total -- at least one run per
+// unit, the other S - U in proportion to cost -- and cuts them by cost
+// within the unit.  No run crosses a unit, so no CTA pays a second unit's
+// set-up, combine and merge for a sliver of pages.
+__device__ __forceinline__ int unit_first_run(int u, unsigned long long Pu, unsigned long long C,
+                                              int S, int U) {
+  if (C == 0) return u;
+  return u + (int)((2ull * Pu * (unsigned long long)(S - U) + C) / (2ull * C));
+}
+
 // This CTA's run [sm.run[0], sm.run[1]) (block-wide; contains barriers),
 // its first and last unit, the total cost, and the cost before every
 // segment of the units it touches (when they are at most kTouchedUnits).
@@ -222,24 +236,37 @@ __device__ __noinline__ void find_run(const SplitInfo& si, int c, int S, Smem& s
     tot += sm.scan[i];
   }
   const unsigned long long Su = (unsigned long long)S;
-  const unsigned long long T0 = (unsigned long long)c * tot, T1 = (unsigned long long)(c + 1) * tot;
+  const bool aligned = si.U <= S;
   unsigned long long cc = before;
-  for (int k = k0; k < k1; ++k) {
-    const long long a = si.seg_start(k), b = si.seg_start(k + 1);
-    const unsigned long long ws = si.weight(k) * Su;
-    const unsigned long long lo = cc * Su, hi = lo + (unsigned long long)(b - a) * ws;
-    if (lo < T0 && T0 <= hi) sm.run[0] = a + (long long)((T0 - lo + ws - 1) / ws);
-    if (lo < T1 && T1 <= hi) sm.run[1] = a + (long long)((T1 - lo + ws - 1) / ws);
-    cc += (unsigned long long)(b - a) * si.weight(k);
+  if (aligned) {
+    // this CTA's unit: the last u with B(u) <= c
+    for (int k = k0; k < k1; ++k) {
+      if (k % 3 == 0 && unit_first_run(k / 3, cc, tot, S, si.U) <= c) atomicMax(&sm.unit0, k / 3);
+      cc += (unsigned long long)(si.seg_start(k + 1) - si.seg_start(k)) * si.weight(k);
+    }
+  } else {
+    const unsigned long long T0 = (unsigned long long)c * tot, T1 = (unsigned long long)(c + 1) * tot;
+    for (int k = k0; k < k1; ++k) {
+      const long long a = si.seg_start(k), b = si.seg_start(k + 1);
+      const unsigned long long ws = si.weight(k) * Su;
+      const unsigned long long lo = cc * Su, hi = lo + (unsigned long long)(b - a) * ws;
+      if (lo < T0 && T0 <= hi) sm.run[0] = a + (long long)((T0 - lo + ws - 1) / ws);
+      if (lo < T1 && T1 <= hi) sm.run[1] = a + (long long)((T1 - lo + ws - 1) / ws);
+      cc += (unsigned long long)(b - a) * si.weight(k);
+    }
   }
   if (tid == 0) sm.ctot = tot;
   __syncthreads();
-  // the units of the run's first and last page (their segments hold them)
-  const long long g0 = sm.run[0], g1 = sm.run[1];
-  for (int k = k0; k < k1; ++k) {
-    const long long a = si.seg_start(k), b = si.seg_start(k + 1);
-    if (a <= g0 && g0 < b) sm.unit0 = k / 3;
-    if (a < g1 && g1 <= b) sm.unit1 = k / 3;
+  if (aligned) {
+    if (tid == 0) sm.unit1 = sm.unit0;
+  } else {
+    // the units of the run's first and last page (their segments hold them)
+    const long long g0 = sm.run[0], g1 = sm.run[1];
+    for (int k = k0; k < k1; ++k) {
+      const long long a = si.seg_start(k), b = si.seg_start(k + 1);
+      if (a <= g0 && g0 < b) sm.unit0 = k / 3;
+      if (a < g1 && g1 <= b) sm.unit1 = k / 3;
+    }
   }
   __syncthreads();
   const int ua = sm.unit0, ub = sm.unit1;
@@ -253,6 +280,23 @@ __device__ __noinline__ void find_run(const SplitInfo& si, int c, int S, Smem& s
     if (k1 == nseg && k0 < k1 && nseg <= 3 * ub + 3) sm.ucost[nseg - 3 * ua] = cc;
   }
   __syncthreads();
+  if (aligned && tid == 0) {
+    // run j of the n runs of unit u: its share of the unit's cost
+    const int u = sm.unit0;
+    const unsigned long long Pu = sm.ucost[0], cu = sm.ucost[3] - Pu;
+    const int B0 = unit_first_run(u, Pu, tot, S, si.U);
+    const int n = unit_first_run(u + 1, sm.ucost[3], tot, S, si.U) - B0, j = c - B0;
+    long long seg[4];
+    unsigned long long cr[4];
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      seg[t] = si.seg_start(3 * u + t);
+      cr[t] = sm.ucost[t] - Pu;
+    }
+    sm.run[0] = run_begin_in_unit(si, seg, cr, (unsigned long long)j * cu, (unsigned long long)n);
+    sm.run[1] = run_begin_in_unit(si, seg, cr, (unsigned long long)(j + 1) * cu, (unsigned long long)n);
+  }
+  if (aligned) __syncthreads();
 }
 
 // ------------------------------------------------------ shared loads (PTX) --
@@ -1106,28 +1150,46 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       }
     }
     named_bar_sync(1, nct);
-    const unsigned long long Su = (unsigned long long)p.S, ctot = sm.ctot;
-    int c0 = c, c1 = c;
-    if (ctot > 0) {
+    const unsigned long long ctot = sm.ctot;
+    const bool aligned = U <= p.S;
+    // run cc starts at the first page of u whose cost offset reaches
+    // (cc - cb) ct, in cost units scaled by Sr (global split: cb = 0,
+    // ct = total, Sr = S; unit-aligned split: cb = B(u), ct = the unit's
+    // cost, Sr = its run count, and costs relative to the unit)
+    unsigned long long cseg[4], Sr = (unsigned long long)p.S, ct = ctot;
+    int c0 = c, c1 = c, cb = 0;
+#pragma unroll
+    for (int t = 0; t < 4; ++t) cseg[t] = sm.cunit[t];
+    if (aligned) {
+      c0 = cb = unit_first_run(u, sm.cunit[0], ctot, p.S, U);
+      c1 = unit_first_run(u + 1, sm.cunit[3], ctot, p.S, U) - 1;
+      Sr = (unsigned long long)(c1 - c0 + 1);
+      ct = sm.cunit[3] - sm.cunit[0];
+#pragma unroll
+      for (int t = 0; t < 4; ++t) cseg[t] = sm.cunit[t] - sm.cunit[0];
+    } else if (ctot > 0) {
       int tl = 2;  // tier of the unit's last page
       while (tl > 0 && sm.useg[tl] == iu1) --tl;
-      c0 = (int)(sm.cunit[0] * Su / ctot);
-      c1 = (int)((sm.cunit[3] - si.weight(tl)) * Su / ctot);
+      c0 = (int)(sm.cunit[0] * Sr / ctot);
+      c1 = (int)((sm.cunit[3] - si.weight(tl)) * Sr / ctot);
     }
     // when no page costs more than a run (the usual case) every run from c0
     // to c1 holds pages of u; otherwise a run inside may be empty
     const unsigned long long wmax = (unsigned long long)max(si.w[0], max(si.w[1], si.w[2]));
-    const bool dense_runs = wmax * Su <= ctot;
+    const bool dense_runs = wmax * Sr <= ct;
     auto run_has_u = [&](int cc) -> bool {
-      if (dense_runs || cc == c0 || cc == c1) return true;
-      const long long ra = run_begin_in_unit(si, sm.useg, sm.cunit, (unsigned long long)cc * ctot, Su);
+      if (dense_runs || (!aligned && (cc == c0 || cc == c1))) return true;
+      const long long ra =
+          run_begin_in_unit(si, sm.useg, cseg, (unsigned long long)(cc - cb) * ct, Sr);
       const long long rb =
-          run_begin_in_unit(si, sm.useg, sm.cunit, (unsigned long long)(cc + 1) * ctot, Su);
+          run_begin_in_unit(si, sm.useg, cseg, (unsigned long long)(cc + 1 - cb) * ct, Sr);
       return rb > ra;
     };
+    // (global split: the runs of the unit's first and last page hold pages
+    // of u; unit-aligned split: the last runs of a unit may be empty)
     int nruns = c1 - c0 + 1;
     if (!dense_runs)
-      for (int cc = c0 + 1; cc < c1; ++cc) nruns -= run_has_u(cc) ? 0 : 1;
+      for (int cc = c0 + 1; cc < (aligned ? c1 + 1 : c1); ++cc) nruns -= run_has_u(cc) ? 0 : 1;
     const long long obase = (long long)bb * p.Hq + (long long)hkv * G;
     if (nruns == 1) {
       for (int i = tid; i < G * kHeadDim; i += nct) {
@@ -1160,57 +1222,71 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       }
       named_bar_sync(1, nct);
       if (sm.last_flag) {
-        // merge the runs' partials of unit u (this CTA's included): run
-        // weights 2^(m_run - M) / L per head first, then one weighted sum per
-        // output element with the run loads issued back to back
+        // merge the runs' partials of unit u (this CTA's included): the
+        // runs' (m, l), then per head (a warp each) M, the run weights
+        // 2^(m - M) and L, then per output pair the weighted sum over the
+        // runs with all of a batch's loads in flight at once
         const int nr = c1 - c0 + 1;
         if (nr <= kMergeRuns) {
           for (int i = tid; i < G * nr; i += nct) {
             const int n = i / nr, r = i % nr;
             const int cc = c0 + r;
-            float m = -INFINITY;  // an empty run contributes nothing
+            float2 ml = make_float2(-INFINITY, 0.0f);  // an empty run contributes nothing
             if (run_has_u(cc))
-              m = __ldcg(p.part + (long long)(cc + u) * G * kPartStride + n * kPartStride);
-            sm.mw[n][r] = m;
+              ml = __ldcg(reinterpret_cast<const float2*>(
+                  p.part + (long long)(cc + u) * G * kPartStride + n * kPartStride));
+            sm.mw[n][r] = ml.x;
+            sm.O[n][r] = ml.y;  // O is free: this CTA's partial has been written out
           }
           named_bar_sync(1, nct);
-          for (int i = tid; i < G * kHeadDim; i += nct) {
-            const int n = i / kHeadDim, d = i % kHeadDim;
+          if (warp < G) {
+            const int n = warp;
             float M = -INFINITY;
-            for (int r = 0; r < nr; ++r) M = fmaxf(M, sm.mw[n][r]);
-            float L = 0.0f, O = 0.0f;
-            if (M != -INFINITY) {
-              int r = 0;
-              for (; r + 4 <= nr; r += 4) {
-                float lv[4], ov[4], wv[4];
+            for (int r = lane; r < nr; r += 32) M = fmaxf(M, sm.mw[n][r]);
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                  const float* pp =
-                      p.part + (long long)(c0 + r + k + u) * G * kPartStride + n * kPartStride;
-                  const float m = sm.mw[n][r + k];
-                  wv[k] = (m == -INFINITY) ? 0.0f : exp2f(m - M);
-                  lv[k] = (m == -INFINITY) ? 0.0f : __ldcg(pp + 1);
-                  ov[k] = (m == -INFINITY) ? 0.0f : __ldcg(pp + 4 + d);
-                }
+            for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xFFFFFFFFu, M, o));
+            float L = 0.0f;
+            for (int r = lane; r < nr; r += 32) {
+              const float m = sm.mw[n][r];
+              const float wgt = (m == -INFINITY) ? 0.0f : exp2f(m - M);
+              sm.mw[n][r] = wgt;
+              L += wgt * sm.O[n][r];
+            }
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                  L += lv[k] * wv[k];
-                  O += ov[k] * wv[k];
-                }
+            for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xFFFFFFFFu, L, o);
+            if (lane == 0) {
+              sm.MH[n] = M;
+              sm.LH[n] = L;
+            }
+          }
+          named_bar_sync(1, nct);
+          for (int i = tid; i < G * kHeadDim / 2; i += nct) {
+            const int n = i / (kHeadDim / 2), j = i % (kHeadDim / 2);
+            const float* pn = p.part + (long long)(c0 + u) * G * kPartStride + n * kPartStride + 4 + 2 * j;
+            float ox = 0.0f, oy = 0.0f;
+            for (int r0 = 0; r0 < nr; r0 += kMergeBatch) {
+              float2 v[kMergeBatch];
+              float wv[kMergeBatch];
+#pragma unroll
+              for (int k = 0; k < kMergeBatch; ++k) {
+                const int r = r0 + k;
+                wv[k] = r < nr ? sm.mw[n][r] : 0.0f;
+                v[k] = wv[k] != 0.0f
+                           ? __ldcg(reinterpret_cast<const float2*>(pn + (long long)r * G * kPartStride))
+                           : make_float2(0.0f, 0.0f);
               }
-              for (; r < nr; ++r) {
-                const float m = sm.mw[n][r];
-                if (m == -INFINITY) continue;
-                const float* pp =
-                    p.part + (long long)(c0 + r + u) * G * kPartStride + n * kPartStride;
-                const float wgt = exp2f(m - M);
-                L += __ldcg(pp + 1) * wgt;
-                O += __ldcg(pp + 4 + d) * wgt;
+#pragma unroll
+              for (int k = 0; k < kMergeBatch; ++k) {
+                ox = fmaf(wv[k], v[k].x, ox);
+                oy = fmaf(wv[k], v[k].y, oy);
               }
             }
-            p.out[(obase + n) * kHeadDim + d] = L > 0.0f ? O / L : 0.0f;
-            if (d == 0 && p.lse)
-              p.lse[obase + n] = L > 0.0f ? (M + log2f(L)) * 0.69314718055994530942f : -INFINITY;
+            const float L = sm.LH[n];
+            float* o = p.out + (obase + n) * kHeadDim + 2 * j;
+            o[0] = L > 0.0f ? ox / L : 0.0f;
+            o[1] = L > 0.0f ? oy / L : 0.0f;
+            if (j == 0 && p.lse)
+              p.lse[obase + n] = L > 0.0f ? (sm.MH[n] + log2f(L)) * 0.69314718055994530942f : -INFINITY;
           }
         } else {
           for (int i = tid; i < G * kHeadDim; i += nct) {
