@@ -998,6 +998,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     if (a >= b) continue;
     const int bb = u / p.Hkv, hkv = u % p.Hkv;
     named_bar_sync(1, nct);
+    if (tid < 4) sm.useg[tid] = si.seg_start(3 * u + tid);  // for the merge, after the items
     for (int i = tid; i < G * kHeadDim; i += nct) {
       const int h = i / kHeadDim, d = i % kHeadDim;
       const long long qi = ((long long)bb * p.Hq + (long long)hkv * G + h) * kHeadDim + d;
@@ -1123,11 +1124,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     }
     // runs of the page list that touch unit u: run c holds page g when
     // floor(C(g) S / total) == c; the first and the last page of u give the
-    // range, a run strictly inside it may be empty (a page costlier than a run)
-    if (tid == 0) {
-#pragma unroll
-      for (int t = 0; t < 4; ++t) sm.useg[t] = si.seg_start(3 * u + t);
-    }
+    // range, a run strictly inside it may be empty (a page costlier than a
+    // run); sm.useg holds u's tier segment starts (loaded at the unit's start)
     if (sm.unit1 - sm.unit0 < kTouchedUnits) {
       if (tid < 4) sm.cunit[tid] = sm.ucost[3 * (u - sm.unit0) + tid];
     } else {
@@ -1209,9 +1207,11 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
           __stcg(part + n * kPartStride + 1, sm.LH[n]);
         }
       }
-      __threadfence();
+      // the CTA's stores, ordered by the barrier, are made visible by one
+      // cumulative fence of the thread that takes the ticket
       named_bar_sync(1, nct);
       if (tid == 0) {
+        __threadfence();
         const int ticket = atomicAdd(&counters[u], 1);
         const int last = ticket == nruns - 1;
         if (last) {
@@ -1222,71 +1222,50 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       }
       named_bar_sync(1, nct);
       if (sm.last_flag) {
-        // merge the runs' partials of unit u (this CTA's included): the
-        // runs' (m, l), then per head (a warp each) M, the run weights
-        // 2^(m - M) and L, then per output pair the weighted sum over the
-        // runs with all of a batch's loads in flight at once
+        // merge the runs' partials of unit u (this CTA's included): which
+        // runs hold pages of u, then per output pair an online log-sum-exp
+        // over the runs, every load of a batch of runs in flight at once
         const int nr = c1 - c0 + 1;
         if (nr <= kMergeRuns) {
-          for (int i = tid; i < G * nr; i += nct) {
-            const int n = i / nr, r = i % nr;
-            const int cc = c0 + r;
-            float2 ml = make_float2(-INFINITY, 0.0f);  // an empty run contributes nothing
-            if (run_has_u(cc))
-              ml = __ldcg(reinterpret_cast<const float2*>(
-                  p.part + (long long)(cc + u) * G * kPartStride + n * kPartStride));
-            sm.mw[n][r] = ml.x;
-            sm.O[n][r] = ml.y;  // O is free: this CTA's partial has been written out
-          }
-          named_bar_sync(1, nct);
-          if (warp < G) {
-            const int n = warp;
-            float M = -INFINITY;
-            for (int r = lane; r < nr; r += 32) M = fmaxf(M, sm.mw[n][r]);
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xFFFFFFFFu, M, o));
-            float L = 0.0f;
-            for (int r = lane; r < nr; r += 32) {
-              const float m = sm.mw[n][r];
-              const float wgt = (m == -INFINITY) ? 0.0f : exp2f(m - M);
-              sm.mw[n][r] = wgt;
-              L += wgt * sm.O[n][r];
-            }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xFFFFFFFFu, L, o);
-            if (lane == 0) {
-              sm.MH[n] = M;
-              sm.LH[n] = L;
-            }
-          }
+          for (int r = tid; r < nr; r += nct) sm.mw[0][r] = run_has_u(c0 + r) ? 1.0f : 0.0f;
           named_bar_sync(1, nct);
           for (int i = tid; i < G * kHeadDim / 2; i += nct) {
             const int n = i / (kHeadDim / 2), j = i % (kHeadDim / 2);
-            const float* pn = p.part + (long long)(c0 + u) * G * kPartStride + n * kPartStride + 4 + 2 * j;
-            float ox = 0.0f, oy = 0.0f;
+            const float* pn = p.part + (long long)(c0 + u) * G * kPartStride + n * kPartStride;
+            float M = -INFINITY, L = 0.0f, ox = 0.0f, oy = 0.0f;
             for (int r0 = 0; r0 < nr; r0 += kMergeBatch) {
-              float2 v[kMergeBatch];
-              float wv[kMergeBatch];
+              float2 ml[kMergeBatch], v[kMergeBatch];
 #pragma unroll
               for (int k = 0; k < kMergeBatch; ++k) {
                 const int r = r0 + k;
-                wv[k] = r < nr ? sm.mw[n][r] : 0.0f;
-                v[k] = wv[k] != 0.0f
-                           ? __ldcg(reinterpret_cast<const float2*>(pn + (long long)r * G * kPartStride))
-                           : make_float2(0.0f, 0.0f);
+                const bool live = r < nr && sm.mw[0][r] != 0.0f;
+                const float* pr = pn + (long long)r * G * kPartStride;
+                ml[k] = live ? __ldcg(reinterpret_cast<const float2*>(pr)) : make_float2(-INFINITY, 0.0f);
+                v[k] = live ? __ldcg(reinterpret_cast<const float2*>(pr + 4 + 2 * j))
+                            : make_float2(0.0f, 0.0f);
               }
+              float Mb = M;
+#pragma unroll
+              for (int k = 0; k < kMergeBatch; ++k) Mb = fmaxf(Mb, ml[k].x);
+              if (Mb == -INFINITY) continue;  // nothing yet
+              const float sc = (M == -INFINITY) ? 0.0f : exp2f(M - Mb);
+              L *= sc;
+              ox *= sc;
+              oy *= sc;
 #pragma unroll
               for (int k = 0; k < kMergeBatch; ++k) {
-                ox = fmaf(wv[k], v[k].x, ox);
-                oy = fmaf(wv[k], v[k].y, oy);
+                const float wgt = (ml[k].x == -INFINITY) ? 0.0f : exp2f(ml[k].x - Mb);
+                L = fmaf(wgt, ml[k].y, L);
+                ox = fmaf(wgt, v[k].x, ox);
+                oy = fmaf(wgt, v[k].y, oy);
               }
+              M = Mb;
             }
-            const float L = sm.LH[n];
             float* o = p.out + (obase + n) * kHeadDim + 2 * j;
             o[0] = L > 0.0f ? ox / L : 0.0f;
             o[1] = L > 0.0f ? oy / L : 0.0f;
             if (j == 0 && p.lse)
-              p.lse[obase + n] = L > 0.0f ? (sm.MH[n] + log2f(L)) * 0.69314718055994530942f : -INFINITY;
+              p.lse[obase + n] = L > 0.0f ? (M + log2f(L)) * 0.69314718055994530942f : -INFINITY;
           }
         } else {
           for (int i = tid; i < G * kHeadDim; i += nct) {
