@@ -991,21 +991,34 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   int tbl_entries = DENSE ? 0 : 256 + 64;  // table entries still to build
   int it = 0;  // item index within the run
   bool ok = true;
+  constexpr int kQPer = (4 * kHeadDim + kNCW * 32 - 1) / (kNCW * 32);  // q elements per thread
   for (int u = u0; u < U; ++u) {
+    const int bb = u / p.Hkv, hkv = u % p.Hkv;
+    // the unit's page range and its query elements, loaded together
     const long long iu0 = p.indptr[u], iu1 = p.indptr[u + 1];
+    uint16_t qraw[kQPer];
+#pragma unroll
+    for (int k = 0; k < kQPer; ++k) {
+      const int i = tid + k * nct;
+      qraw[k] = i < G * kHeadDim
+                    ? reinterpret_cast<const uint16_t*>(p.q)[((long long)bb * p.Hq + (long long)hkv * G) *
+                                                                 kHeadDim + i]
+                    : (uint16_t)0;
+    }
     if (iu0 >= g1) break;
     const long long a = max(g0, iu0), b = min(g1, iu1);
     if (a >= b) continue;
-    const int bb = u / p.Hkv, hkv = u % p.Hkv;
     named_bar_sync(1, nct);
     if (tid < 4) sm.useg[tid] = si.seg_start(3 * u + tid);  // for the merge, after the items
-    for (int i = tid; i < G * kHeadDim; i += nct) {
-      const int h = i / kHeadDim, d = i % kHeadDim;
-      const long long qi = ((long long)bb * p.Hq + (long long)hkv * G + h) * kHeadDim + d;
-      const uint16_t raw = reinterpret_cast<const uint16_t*>(p.q)[qi];
-      sm.q32[h][d] = p.q_bf16 ? __bfloat162float(__ushort_as_bfloat16(raw))
-                              : __half2float(__ushort_as_half(raw));
-      sm.O[h][d] = 0.0f;
+#pragma unroll
+    for (int k = 0; k < kQPer; ++k) {
+      const int i = tid + k * nct;
+      if (i < G * kHeadDim) {
+        const int h = i / kHeadDim, d = i % kHeadDim;
+        sm.q32[h][d] = p.q_bf16 ? __bfloat162float(__ushort_as_bfloat16(qraw[k]))
+                                : __half2float(__ushort_as_half(qraw[k]));
+        sm.O[h][d] = 0.0f;
+      }
     }
     if constexpr (!DENSE) {
       if (tbl_entries) build_tables(p, tbl1p, tbl_entries, tid, nct);
@@ -1294,6 +1307,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         }
       }
     }
+    if (b == g1) break;  // the run ends in this unit: no further page-table reads
   }
 }
 
