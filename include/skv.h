@@ -195,8 +195,10 @@ int skv_encode(skv_ctx* ctx, const uint16_t* K, const uint16_t* V, int B, int Hk
      page_indptr / page_ids / pools: the paged store (any slots, any order of
               pages within a unit; pages are streamed whole)
      page_tier_indptr  NULL, or skv_allocate's per-(unit, tier) offsets: the
-              pages of all units are then cut into runs of equal payload
-              bytes instead of equal page counts (same results either way)
+              runs are then cut by payload bytes instead of page counts
+              (same results either way).  When B*Hkv <= num_splits every
+              unit gets its own runs, in proportion to its cost; otherwise
+              the page list of all units is cut into runs of equal cost.
      out      fp32 [B][Hq][128] device; lse fp32 [B][Hq] device or NULL
               (a unit without resident tokens gives out 0, lse -inf)
      num_splits  number of page runs = CTAs (0 = default: the SM count)
