@@ -61,13 +61,11 @@ constexpr int kRowsPerWarp = kItemRows / kGW;  // rows of an item per consumer w
 constexpr int kPasses = kRowsPerWarp / 16;
 constexpr int kNSlot = 16;                    // items in flight, at most
 constexpr int kMaxIPP = kItemRows / 16;       // pages per item (P >= 16)
-constexpr int kMergeRuns = 128;               // runs per unit merged through shared memory
 constexpr int kMergeBatch = 20;               // merge: runs whose loads are issued together
 constexpr int kTouchedUnits = 16;             // units whose segment costs a CTA keeps
 static_assert(kCG >= 1 && kCG <= 4, "consumer groups: 1..4");
 static_assert(kIss >= 1 && kIss <= 4, "issuers: 1..4");
 static_assert(kPasses >= 1 && kGW * kRowsPerWarp == kItemRows, "warp row split");
-static_assert(kMergeRuns <= kHeadDim, "merge: the runs' l values are kept in a row of O");
 
 // Item descriptor (16 B, written by the producer before it arms the slot's
 // full barrier): x = shared address of the item, y = meta, z/w = byte
@@ -109,14 +107,12 @@ struct __align__(16) DecodeSmem {
   long long run[2];                    // this CTA's pages [run[0], run[1])
   int unit0, unit1;                    // the units of pages run[0] and run[1] - 1
   int abort_flag;
-  int last_flag;
   int pad_[2];
   __align__(16) float ml[kNCW][4][2];
   float wsc[kNCW][4];                   // combine: each warp's scale per head
   float MH[4], LH[4];                   // combine: this CTA's (M, L) per head
   __align__(16) float O[4][kHeadDim];
   __align__(16) float q32[4][kHeadDim];   // read with 16-byte shared loads
-  __align__(16) float mw[4][kMergeRuns];  // merge: per-run weights
 };
 constexpr uint32_t kEndOfRun = 0xFFFFFFFFu;
 using DecodeSmemG4 = DecodeSmem<4, false>;
@@ -710,19 +706,35 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       report(p.err, SKV_ERR_ARG);
     }
   }
-  // units without any resident page: out = 0, lse = -inf (written by CTA 0)
+  // the merge kernel may be launched now: it waits for this grid's end
+  asm volatile("griddepcontrol.launch_dependents;");
+  // units without any resident page: out = 0, lse = -inf, nothing to merge
+  // (written by CTA 0)
   if (c == 0) {
     for (int u = warp; u < U; u += kDecodeThreads / 32) {
       if (p.indptr[u + 1] > p.indptr[u]) continue;
       const long long o = (long long)(u / p.Hkv) * p.Hq + (long long)(u % p.Hkv) * G;
       for (int i = lane; i < G * kHeadDim; i += 32) p.out[o * kHeadDim + i] = 0.0f;
       if (p.lse && lane < G) p.lse[o + lane] = -INFINITY;
+      if (lane == 0) reinterpret_cast<int2*>(counters)[u] = make_int2(0, 0);
     }
   }
   if (!plan_ok) return;  // uniform: every thread computed the same layout
   find_run(si, c, p.S, sm, tid);
   const long long g0 = sm.run[0], g1 = sm.run[1];
-  if (g0 >= g1) return;
+  if (g0 >= g1) {
+    // an empty run inside a unit's runs (unit-aligned: a trailing run of a
+    // small unit; global: a run between two pages of one unit, when a page
+    // costs more than a run) leaves an empty partial in its slot
+    const int u = sm.unit0;
+    const bool inside = U <= p.S ? true : (g0 < (long long)p.indptr[U] && g0 > (long long)p.indptr[u]);
+    if (inside && tid < G) {
+      float* part = p.part + (long long)(c + u) * G * kPartStride + tid * kPartStride;
+      part[0] = -INFINITY;
+      part[1] = 0.0f;
+    }
+    return;
+  }
 
   const int u0 = sm.unit0;  // the unit holding page g0
 
@@ -1135,10 +1147,14 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       tbl_entries = 256;  // TBL1 holds the stash now
       named_bar_sync(1, nct);
     }
-    // runs of the page list that touch unit u: run c holds page g when
-    // floor(C(g) S / total) == c; the first and the last page of u give the
-    // range, a run strictly inside it may be empty (a page costlier than a
-    // run); sm.useg holds u's tier segment starts (loaded at the unit's start)
+    // ---- this CTA's result for unit u.  A unit inside one run is finished
+    // here; otherwise every run from c0 to c1 writes its partial to slot
+    // c + u (an empty run an empty one, at the kernel's start) and
+    // decode_merge_kernel combines them once this grid has completed.  The
+    // CTA of run c0 records (c0, c1) for it.  Runs: unit-aligned split,
+    // [B(u), B(u + 1)); global split, run c holds page g when
+    // floor(C(g) S / total) == c, so the runs of u's first and last page.
+    // sm.useg holds u's tier segment starts (loaded at the unit's start).
     if (sm.unit1 - sm.unit0 < kTouchedUnits) {
       if (tid < 4) sm.cunit[tid] = sm.ucost[3 * (u - sm.unit0) + tid];
     } else {
@@ -1161,48 +1177,19 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       }
     }
     named_bar_sync(1, nct);
-    const unsigned long long ctot = sm.ctot;
-    const bool aligned = U <= p.S;
-    // run cc starts at the first page of u whose cost offset reaches
-    // (cc - cb) ct, in cost units scaled by Sr (global split: cb = 0,
-    // ct = total, Sr = S; unit-aligned split: cb = B(u), ct = the unit's
-    // cost, Sr = its run count, and costs relative to the unit)
-    unsigned long long cseg[4], Sr = (unsigned long long)p.S, ct = ctot;
-    int c0 = c, c1 = c, cb = 0;
-#pragma unroll
-    for (int t = 0; t < 4; ++t) cseg[t] = sm.cunit[t];
-    if (aligned) {
-      c0 = cb = unit_first_run(u, sm.cunit[0], ctot, p.S, U);
+    const unsigned long long ctot = sm.ctot, Su = (unsigned long long)p.S;
+    int c0 = c, c1 = c;
+    if (U <= p.S) {
+      c0 = unit_first_run(u, sm.cunit[0], ctot, p.S, U);
       c1 = unit_first_run(u + 1, sm.cunit[3], ctot, p.S, U) - 1;
-      Sr = (unsigned long long)(c1 - c0 + 1);
-      ct = sm.cunit[3] - sm.cunit[0];
-#pragma unroll
-      for (int t = 0; t < 4; ++t) cseg[t] = sm.cunit[t] - sm.cunit[0];
     } else if (ctot > 0) {
       int tl = 2;  // tier of the unit's last page
       while (tl > 0 && sm.useg[tl] == iu1) --tl;
-      c0 = (int)(sm.cunit[0] * Sr / ctot);
-      c1 = (int)((sm.cunit[3] - si.weight(tl)) * Sr / ctot);
+      c0 = (int)(sm.cunit[0] * Su / ctot);
+      c1 = (int)((sm.cunit[3] - si.weight(tl)) * Su / ctot);
     }
-    // when no page costs more than a run (the usual case) every run from c0
-    // to c1 holds pages of u; otherwise a run inside may be empty
-    const unsigned long long wmax = (unsigned long long)max(si.w[0], max(si.w[1], si.w[2]));
-    const bool dense_runs = wmax * Sr <= ct;
-    auto run_has_u = [&](int cc) -> bool {
-      if (dense_runs || (!aligned && (cc == c0 || cc == c1))) return true;
-      const long long ra =
-          run_begin_in_unit(si, sm.useg, cseg, (unsigned long long)(cc - cb) * ct, Sr);
-      const long long rb =
-          run_begin_in_unit(si, sm.useg, cseg, (unsigned long long)(cc + 1 - cb) * ct, Sr);
-      return rb > ra;
-    };
-    // (global split: the runs of the unit's first and last page hold pages
-    // of u; unit-aligned split: the last runs of a unit may be empty)
-    int nruns = c1 - c0 + 1;
-    if (!dense_runs)
-      for (int cc = c0 + 1; cc < (aligned ? c1 + 1 : c1); ++cc) nruns -= run_has_u(cc) ? 0 : 1;
     const long long obase = (long long)bb * p.Hq + (long long)hkv * G;
-    if (nruns == 1) {
+    if (c0 == c1) {
       for (int i = tid; i < G * kHeadDim; i += nct) {
         const int n = i / kHeadDim, d = i % kHeadDim;
         const float L = sm.LH[n];
@@ -1214,101 +1201,72 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       float* part = p.part + (long long)(c + u) * G * kPartStride;
       for (int i = tid; i < G * kHeadDim; i += nct) {
         const int n = i / kHeadDim, d = i % kHeadDim;
-        __stcg(part + n * kPartStride + 4 + d, sm.O[n][d]);
+        part[n * kPartStride + 4 + d] = sm.O[n][d];
         if (d == 0) {
-          __stcg(part + n * kPartStride + 0, sm.MH[n]);
-          __stcg(part + n * kPartStride + 1, sm.LH[n]);
-        }
-      }
-      // the CTA's stores, ordered by the barrier, are made visible by one
-      // cumulative fence of the thread that takes the ticket
-      named_bar_sync(1, nct);
-      if (tid == 0) {
-        __threadfence();
-        const int ticket = atomicAdd(&counters[u], 1);
-        const int last = ticket == nruns - 1;
-        if (last) {
-          __threadfence();
-          counters[u] = 0;
-        }
-        sm.last_flag = last;
-      }
-      named_bar_sync(1, nct);
-      if (sm.last_flag) {
-        // merge the runs' partials of unit u (this CTA's included): which
-        // runs hold pages of u, then per output pair an online log-sum-exp
-        // over the runs, every load of a batch of runs in flight at once
-        const int nr = c1 - c0 + 1;
-        if (nr <= kMergeRuns) {
-          for (int r = tid; r < nr; r += nct) sm.mw[0][r] = run_has_u(c0 + r) ? 1.0f : 0.0f;
-          named_bar_sync(1, nct);
-          for (int i = tid; i < G * kHeadDim / 2; i += nct) {
-            const int n = i / (kHeadDim / 2), j = i % (kHeadDim / 2);
-            const float* pn = p.part + (long long)(c0 + u) * G * kPartStride + n * kPartStride;
-            float M = -INFINITY, L = 0.0f, ox = 0.0f, oy = 0.0f;
-            for (int r0 = 0; r0 < nr; r0 += kMergeBatch) {
-              float2 ml[kMergeBatch], v[kMergeBatch];
-#pragma unroll
-              for (int k = 0; k < kMergeBatch; ++k) {
-                const int r = r0 + k;
-                const bool live = r < nr && sm.mw[0][r] != 0.0f;
-                const float* pr = pn + (long long)r * G * kPartStride;
-                ml[k] = live ? __ldcg(reinterpret_cast<const float2*>(pr)) : make_float2(-INFINITY, 0.0f);
-                v[k] = live ? __ldcg(reinterpret_cast<const float2*>(pr + 4 + 2 * j))
-                            : make_float2(0.0f, 0.0f);
-              }
-              float Mb = M;
-#pragma unroll
-              for (int k = 0; k < kMergeBatch; ++k) Mb = fmaxf(Mb, ml[k].x);
-              if (Mb == -INFINITY) continue;  // nothing yet
-              const float sc = (M == -INFINITY) ? 0.0f : exp2f(M - Mb);
-              L *= sc;
-              ox *= sc;
-              oy *= sc;
-#pragma unroll
-              for (int k = 0; k < kMergeBatch; ++k) {
-                const float wgt = (ml[k].x == -INFINITY) ? 0.0f : exp2f(ml[k].x - Mb);
-                L = fmaf(wgt, ml[k].y, L);
-                ox = fmaf(wgt, v[k].x, ox);
-                oy = fmaf(wgt, v[k].y, oy);
-              }
-              M = Mb;
-            }
-            float* o = p.out + (obase + n) * kHeadDim + 2 * j;
-            o[0] = L > 0.0f ? ox / L : 0.0f;
-            o[1] = L > 0.0f ? oy / L : 0.0f;
-            if (j == 0 && p.lse)
-              p.lse[obase + n] = L > 0.0f ? (M + log2f(L)) * 0.69314718055994530942f : -INFINITY;
-          }
-        } else {
-          for (int i = tid; i < G * kHeadDim; i += nct) {
-            const int n = i / kHeadDim, d = i % kHeadDim;
-            float M = -INFINITY, L = 0.0f, O = 0.0f;
-            for (int cc = c0; cc <= c1; ++cc) {
-              if (!run_has_u(cc)) continue;
-              const float* pp = p.part + (long long)(cc + u) * G * kPartStride + n * kPartStride;
-              const float m = __ldcg(pp), lc = __ldcg(pp + 1), oc = __ldcg(pp + 4 + d);
-              if (m == -INFINITY) continue;
-              if (m > M) {
-                const float r = (M == -INFINITY) ? 0.0f : exp2f(M - m);
-                L = L * r + lc;
-                O = O * r + oc;
-                M = m;
-              } else {
-                const float r = exp2f(m - M);
-                L += lc * r;
-                O += oc * r;
-              }
-            }
-            p.out[(obase + n) * kHeadDim + d] = L > 0.0f ? O / L : 0.0f;
-            if (d == 0 && p.lse)
-              p.lse[obase + n] = L > 0.0f ? (M + log2f(L)) * 0.69314718055994530942f : -INFINITY;
-          }
+          part[n * kPartStride + 0] = sm.MH[n];
+          part[n * kPartStride + 1] = sm.LH[n];
         }
       }
     }
+    if (tid == 0 && c == c0) reinterpret_cast<int2*>(counters)[u] = make_int2(c0, c1);
     if (b == g1) break;  // the run ends in this unit: no further page-table reads
   }
+}
+
+// Cross-CTA merge (log-sum-exp) of the units that span several runs: one
+// CTA per unit, one thread per (head, output pair), launched behind the
+// decode grid as a programmatic dependent (its wait returns once the decode
+// grid has completed and its writes are visible).  A unit's record (c0, c1)
+// names its runs; every run in that range wrote slot c + u.  The loads of a
+// batch of runs are all in flight at once, with an online maximum across
+// batches.
+template <int G>
+__global__ void __launch_bounds__(G * kHeadDim / 2)
+    decode_merge_kernel(const __grid_constant__ DecodeParams p) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int u = blockIdx.x;
+  const int U = p.B * p.Hkv;
+  const DecodeWs wsl = decode_ws(p.S, U, G);
+  const int2 rr = reinterpret_cast<const int2*>(reinterpret_cast<const uint8_t*>(p.part) + wsl.ctr)[u];
+  const int c0 = rr.x, nr = rr.y - rr.x + 1;
+  if (nr <= 1) return;
+  const int n = threadIdx.x / (kHeadDim / 2), j = threadIdx.x % (kHeadDim / 2);
+  const float* pn = p.part + (long long)(c0 + u) * G * kPartStride + n * kPartStride;
+  float M = -INFINITY, L = 0.0f, ox = 0.0f, oy = 0.0f;
+  for (int r0 = 0; r0 < nr; r0 += kMergeBatch) {
+    float2 ml[kMergeBatch], v[kMergeBatch];
+#pragma unroll
+    for (int k = 0; k < kMergeBatch; ++k) {
+      const bool live = r0 + k < nr;
+      const float* pr = pn + (long long)(r0 + k) * G * kPartStride;
+      ml[k] = live ? __ldcg(reinterpret_cast<const float2*>(pr)) : make_float2(-INFINITY, 0.0f);
+      v[k] = live ? __ldcg(reinterpret_cast<const float2*>(pr + 4 + 2 * j)) : make_float2(0.0f, 0.0f);
+    }
+    float Mb = M;
+#pragma unroll
+    for (int k = 0; k < kMergeBatch; ++k) Mb = fmaxf(Mb, ml[k].x);
+    if (Mb == -INFINITY) continue;  // nothing yet
+    const float sc = (M == -INFINITY) ? 0.0f : exp2f(M - Mb);
+    L *= sc;
+    ox *= sc;
+    oy *= sc;
+#pragma unroll
+    for (int k = 0; k < kMergeBatch; ++k) {
+      // an empty partial (m = -inf) carries no l or o worth reading
+      if (ml[k].x == -INFINITY) continue;
+      const float wgt = exp2f(ml[k].x - Mb);
+      L = fmaf(wgt, ml[k].y, L);
+      ox = fmaf(wgt, v[k].x, ox);
+      oy = fmaf(wgt, v[k].y, oy);
+    }
+    M = Mb;
+  }
+  const long long obase = (long long)(u / p.Hkv) * p.Hq + (long long)(u % p.Hkv) * G;
+  float* o = p.out + (obase + n) * kHeadDim + 2 * j;
+  o[0] = L > 0.0f ? ox / L : 0.0f;
+  o[1] = L > 0.0f ? oy / L : 0.0f;
+  if (j == 0 && p.lse)
+    p.lse[obase + n] = L > 0.0f ? (M + log2f(L)) * 0.69314718055994530942f : -INFINITY;
 }
 
 template <int G, bool DENSE>
@@ -1332,13 +1290,22 @@ cudaError_t launch_decode_g(const DecodeParams& p, cudaStream_t stream, cudaEven
     if (dev >= 0 && dev < 64) configured[dev] = smem;
   }
   const int U = p.B * p.Hkv;
-  // the ticket counters start at zero
-  const DecodeWs wsl = decode_ws(p.S, U, G);
-  e = cudaMemsetAsync(reinterpret_cast<uint8_t*>(p.part) + wsl.ctr, 0, sizeof(int) * (size_t)U,
-                      stream);
-  if (e != cudaSuccess) return e;
   decode_kernel<G, DENSE><<<p.S, kDecodeThreads, p.smem_bytes, stream>>>(p);
   e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  // the merge: a programmatic dependent of the decode grid (it may be
+  // scheduled early and waits in-kernel for the grid's completion)
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)U);
+  cfg.blockDim = dim3(G * kHeadDim / 2);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, decode_merge_kernel<G>, p);
   if (e != cudaSuccess) return e;
   if (between) {
     // an external record node when the stream is being captured into a graph

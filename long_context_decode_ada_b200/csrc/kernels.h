@@ -88,15 +88,16 @@ struct AllocParams {
   int dense;                  // dense-bf16 baseline packing (every token kept, tier 0)
 };
 
-// Decode workspace: partials [(S + U) G][kPartStride] fp32, then U ticket
-// counters (int32, zeroed by every call).
+// Decode workspace: partials [(S + U) G][kPartStride] fp32, then per unit the
+// range (c0, c1) of runs that hold its partials (int32 pairs, written by every
+// call before they are read).
 struct DecodeWs {
   size_t ctr, bytes;
 };
 __host__ __device__ inline DecodeWs decode_ws(long long S, long long U, int G) {
   DecodeWs w;
   w.ctr = (size_t)(S + U) * G * kPartStride * 4;
-  w.bytes = w.ctr + 4 * (size_t)U;
+  w.bytes = w.ctr + 8 * (size_t)U;
   return w;
 }
 
