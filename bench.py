@@ -411,7 +411,7 @@ def run_skv(args, rank, world, local_rank):
                          "algorithmic_bytes": algo_bytes, "payload_bytes_streamed": payload_bytes},
             "cpu_baseline": cpu,
             "e2e": e2e,
-            "gpu_launches": args.steps,  # one decode_kernel per step (plus a driver memset)
+            "gpu_launches": 2 * args.steps,  # decode_kernel + decode_merge_kernel per step
             "clocks": clocks,
             "dense_bf16_baseline": dense,
             "ingest": {"allocate_ms": alloc_ms, "encode_ms": enc_ms, "gen_s": t_gen},

@@ -214,7 +214,7 @@ int skv_decode_attention(skv_ctx* ctx, const void* q, int q_dtype, int B, int Hq
    workspace (the paper has no counterpart: this is an interface convenience
    of this library).  Same arguments, results and device errors as
    skv_decode_attention (ADA decode only; page_tier_indptr may be NULL), but
-   the split partials and ticket counters live in a fixed 4 MiB device
+   the split partials and run ranges live in a fixed 4 MiB device
    array inside libskv, so the call allocates nothing.
      - A call that would need more than 4 MiB of scratch (the size
        skv_workspace_size(SKV_WS_DECODE) reports) is refused with

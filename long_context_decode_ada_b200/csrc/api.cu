@@ -75,9 +75,9 @@ bool valid_pools(const skv_pools* pools, int ntiers) {
 }  // namespace
 
 // ---------------------------------------------------------------------------
-// Fixed decode scratch for skv_decode_attention_static: the partials, ticket
-// counters, split flag and cost prefix live in this array instead of a
-// caller workspace.  Its device address is looked up once per device.
+// Fixed decode scratch for skv_decode_attention_static: the split partials
+// and the units' run ranges live in this array instead of a caller
+// workspace.  Its device address is looked up once per device.
 // ---------------------------------------------------------------------------
 constexpr size_t kStaticScratchBytes = size_t(4) << 20;  // 4 MiB
 static __device__ __align__(256) unsigned char g_decode_scratch[kStaticScratchBytes];
@@ -219,7 +219,7 @@ int skv_workspace_size(const skv_ctx* ctx, int which, int B, int Hkv, int Hq, in
     if (Hq <= 0 || Hq % Hkv != 0) return fail(SKV_ERR_ARG, "Hq must be a multiple of Hkv");
     const int G = Hq / Hkv;
     const long long S = decode_splits(ctx, num_splits);
-    // split partials, ticket counters, the split's published cost prefix
+    // split partials, then each unit's range of runs
     *bytes = skv::decode_ws(S, (long long)B * Hkv, G).bytes;
     return ok();
   }

@@ -3,13 +3,15 @@
 // materialised; 2.2: tier-homogeneous pages read in one header-guided pass)
 // and the dense bf16 paged-decode baseline built on the same skeleton.
 //
-// Work split ("split-K over pages"): the CSR page list of all units
-// (unit = (seq, kv head)) is one array of N pages, cut into S runs of about
-// equal streamed bytes (T0 pages cost 2.6x a T1 page); CTA c streams run c
-// and produces one partial (m, l, o) per unit it touches.  A unit covered
-// by a single run is finished in place; otherwise the partial goes to slot
-// c + u of the workspace and the CTA that brings the unit's ticket counter
-// to its run count merges them (log-sum-exp); no CTA waits for another.
+// Work split ("split-K over pages"): unit = (seq, kv head).  With at most
+// as many units as runs each unit gets its own runs, in proportion to its
+// streamed bytes, cut by bytes inside the unit; otherwise the CSR page list
+// of all units (N pages) is cut into S runs of about equal streamed bytes
+// (T0 pages cost 2.6x a T1 page).  CTA c streams run c and produces one
+// partial (m, l, o) per unit it touches.  A unit covered by a single run
+// is finished in place; otherwise the partial goes to slot c + u of the
+// workspace and decode_merge_kernel, launched as a programmatic dependent
+// of this grid, merges them (log-sum-exp); no CTA waits for another.
 //
 // CTA = kCG groups of 4 consumer warps + 1 planner warp + kIss issuer
 // warps around one byte ring in shared memory.  The CTA's run is cut into
