@@ -140,19 +140,30 @@ def measured_peaks():
 
 
 def written_partials(indptr: np.ndarray, ids: np.ndarray, payload, S: int) -> int:
-    """(run, unit) partials the decode kernel writes: the page list is cut
-    into S runs of equal payload bytes (page g is in run floor(C(g) S / C),
-    C(g) the bytes before it); a unit spread over several runs gets one
-    partial per run, a unit inside one run none."""
+    """(run, unit) partials the decode kernel writes (and the merge kernel
+    reads back).  Pages cost their tier's payload bytes.  With at most S
+    units, unit u gets runs [B(u), B(u+1)), B(u) = u + round(P(u)(S-U)/C)
+    (P(u) the bytes before u, C the total); otherwise page g is in run
+    floor(C(g) S / C), C(g) the bytes before it.  A unit spread over several
+    runs gets one partial per run, a unit inside one run none."""
     N = int(indptr[-1])
+    U = len(indptr) - 1
     if N == 0:
         return 0
     cost = np.asarray(payload, np.int64)[np.asarray(ids[:N], np.uint32) >> 30]
     before = np.concatenate([[0], np.cumsum(cost)[:-1]])
     total = int(cost.sum())
-    run = np.array([(int(x) * S) // total for x in before], np.int64)
     n = 0
-    for u in range(len(indptr) - 1):
+    if U <= S:
+        ucost = [int(cost[int(indptr[u]):int(indptr[u + 1])].sum()) for u in range(U)]
+        P = np.concatenate([[0], np.cumsum(ucost)])
+        first = [u + (2 * int(P[u]) * (S - U) + total) // (2 * total) for u in range(U + 1)]
+        for u in range(U):
+            k = first[u + 1] - first[u]
+            n += k if (k > 1 and ucost[u] > 0) else 0
+        return n
+    run = np.array([(int(x) * S) // total for x in before], np.int64)
+    for u in range(U):
         a, b = int(indptr[u]), int(indptr[u + 1])
         k = len(np.unique(run[a:b])) if b > a else 0
         n += k if k > 1 else 0
