@@ -204,7 +204,8 @@ __device__ __forceinline__ int unit_first_run(int u, unsigned long long Pu, unsi
 // its first and last unit, the total cost, and the cost before every
 // segment of the units it touches (when they are at most kTouchedUnits).
 template <class Smem>
-__device__ __noinline__ void find_run(const SplitInfo& si, int c, int S, Smem& sm, int tid) {
+__device__ __noinline__ void find_run(const SplitInfo& si, int c, int S, Smem& sm, int tid,
+                                      const uint32_t* ids) {
   constexpr int nt = kDecodeThreads;
   const int nseg = 3 * si.U;
   const int per = (nseg + nt - 1) / nt;
@@ -212,6 +213,14 @@ __device__ __noinline__ void find_run(const SplitInfo& si, int c, int S, Smem& s
   unsigned long long loc = 0;
   for (int k = k0; k < k1; ++k)
     loc += (unsigned long long)(si.seg_start(k + 1) - si.seg_start(k)) * si.weight(k);
+  if (k1 == nseg && k0 < k1) {
+    // the page count is known: CTA c brings slice c of the page-id array into
+    // L2, so that every planner's first id loads (after the split) hit L2
+    const long long lines = (si.seg_start(nseg) * 4 + 127) / 128;
+    const long long l0 = lines * c / S, l1 = lines * (c + 1) / S;
+    for (long long l = l0; l < l1; ++l)
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<const uint8_t*>(ids) + 128 * l));
+  }
   const int lane = tid & 31, w = tid >> 5;
   unsigned long long x = loc;
 #pragma unroll
@@ -237,11 +246,36 @@ __device__ __noinline__ void find_run(const SplitInfo& si, int c, int S, Smem& s
   const bool aligned = si.U <= S;
   unsigned long long cc = before;
   if (aligned) {
-    // this CTA's unit: the last u with B(u) <= c
+    // the thread holding the first segment of unit u knows P(u) and the
+    // unit's segments: if c is among u's runs [B(u), B(u + 1)) it writes the
+    // whole split of this CTA (run j of n: its share of the unit's cost)
     for (int k = k0; k < k1; ++k) {
-      if (k % 3 == 0 && unit_first_run(k / 3, cc, tot, S, si.U) <= c) atomicMax(&sm.unit0, k / 3);
+      if (k % 3 == 0) {
+        const int u = k / 3;
+        long long seg[4];
+        unsigned long long cr[4];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) seg[t] = si.seg_start(k + t);
+        cr[0] = 0;
+#pragma unroll
+        for (int t = 0; t < 3; ++t) cr[t + 1] = cr[t] + (unsigned long long)(seg[t + 1] - seg[t]) * si.weight(t);
+        const int B0 = unit_first_run(u, cc, tot, S, si.U);
+        const int B1 = unit_first_run(u + 1, cc + cr[3], tot, S, si.U);
+        if (B0 <= c && c < B1) {
+          const int n = B1 - B0, j = c - B0;
+          sm.unit0 = u;
+          sm.unit1 = u;
+#pragma unroll
+          for (int t = 0; t < 4; ++t) sm.ucost[t] = cc + cr[t];
+          sm.run[0] = run_begin_in_unit(si, seg, cr, (unsigned long long)j * cr[3], (unsigned long long)n);
+          sm.run[1] = run_begin_in_unit(si, seg, cr, (unsigned long long)(j + 1) * cr[3], (unsigned long long)n);
+        }
+      }
       cc += (unsigned long long)(si.seg_start(k + 1) - si.seg_start(k)) * si.weight(k);
     }
+    if (tid == 0) sm.ctot = tot;
+    __syncthreads();
+    return;
   } else {
     const unsigned long long T0 = (unsigned long long)c * tot, T1 = (unsigned long long)(c + 1) * tot;
     for (int k = k0; k < k1; ++k) {
@@ -255,9 +289,7 @@ __device__ __noinline__ void find_run(const SplitInfo& si, int c, int S, Smem& s
   }
   if (tid == 0) sm.ctot = tot;
   __syncthreads();
-  if (aligned) {
-    if (tid == 0) sm.unit1 = sm.unit0;
-  } else {
+  {
     // the units of the run's first and last page (their segments hold them)
     const long long g0 = sm.run[0], g1 = sm.run[1];
     for (int k = k0; k < k1; ++k) {
@@ -278,23 +310,6 @@ __device__ __noinline__ void find_run(const SplitInfo& si, int c, int S, Smem& s
     if (k1 == nseg && k0 < k1 && nseg <= 3 * ub + 3) sm.ucost[nseg - 3 * ua] = cc;
   }
   __syncthreads();
-  if (aligned && tid == 0) {
-    // run j of the n runs of unit u: its share of the unit's cost
-    const int u = sm.unit0;
-    const unsigned long long Pu = sm.ucost[0], cu = sm.ucost[3] - Pu;
-    const int B0 = unit_first_run(u, Pu, tot, S, si.U);
-    const int n = unit_first_run(u + 1, sm.ucost[3], tot, S, si.U) - B0, j = c - B0;
-    long long seg[4];
-    unsigned long long cr[4];
-#pragma unroll
-    for (int t = 0; t < 4; ++t) {
-      seg[t] = si.seg_start(3 * u + t);
-      cr[t] = sm.ucost[t] - Pu;
-    }
-    sm.run[0] = run_begin_in_unit(si, seg, cr, (unsigned long long)j * cu, (unsigned long long)n);
-    sm.run[1] = run_begin_in_unit(si, seg, cr, (unsigned long long)(j + 1) * cu, (unsigned long long)n);
-  }
-  if (aligned) __syncthreads();
 }
 
 // ------------------------------------------------------ shared loads (PTX) --
@@ -710,6 +725,13 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   }
   // the merge kernel may be launched now: it waits for this grid's end
   asm volatile("griddepcontrol.launch_dependents;");
+  if (tid == kDecodeThreads - 1) {
+    // CTA c brings slice c of the queries into L2 (the consumers load their
+    // unit's heads once the split is known)
+    const long long lines = ((long long)p.B * p.Hq * kHeadDim * 2 + 127) / 128;
+    for (long long l = lines * c / p.S; l < lines * (c + 1) / p.S; ++l)
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<const uint8_t*>(p.q) + 128 * l));
+  }
   // units without any resident page: out = 0, lse = -inf, nothing to merge
   // (written by CTA 0)
   if (c == 0) {
@@ -722,7 +744,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     }
   }
   if (!plan_ok) return;  // uniform: every thread computed the same layout
-  find_run(si, c, p.S, sm, tid);
+  find_run(si, c, p.S, sm, tid, p.ids);
   const long long g0 = sm.run[0], g1 = sm.run[1];
   if (g0 >= g1) {
     // an empty run inside a unit's runs (unit-aligned: a trailing run of a
@@ -1085,12 +1107,13 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     }
     it += nitems;
 
-    // ---- combine the warps' states into this CTA's partial for unit u:
-    // one thread per head forms M, L and every warp's scale; each warp then
-    // writes its scaled accumulators to a stash (TBL1's space, rebuilt before
-    // the next unit; the dense kernel, which has no tables, adds them into O
-    // with shared atomics)
-    // and every output element is summed over the warps
+    // ---- combine the warps' states into this CTA's partial for unit u.
+    // ADA: every warp writes its (m, l) per head and, once all warps are done
+    // with the tables, its unscaled accumulators to a stash (TBL1's space,
+    // rebuilt before the next unit); then each output element takes the
+    // warps' maximum, their weights 2^(m_w - M) and the weighted sum.  Dense (no
+    // tables): one thread per head forms M, L and the warps' scales, and the
+    // warps add their scaled accumulators into O with shared atomics.
     float l = st.l;
     l += __shfl_xor_sync(0xFFFFFFFFu, l, 4);
     l += __shfl_xor_sync(0xFFFFFFFFu, l, 8);
@@ -1099,52 +1122,70 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       sm.ml[warp][lane][0] = st.m <= kNoMax ? -INFINITY : st.m;  // no row seen: -inf
       sm.ml[warp][lane][1] = l;
     }
-    named_bar_sync(1, nct);
-    if (tid < G) {
-      const int n = tid;
-      float M = -INFINITY;
-      for (int w = 0; w < kNCW; ++w) M = fmaxf(M, sm.ml[w][n][0]);
-      float L = 0.0f;
-      for (int w = 0; w < kNCW; ++w) {
-        const float mw = sm.ml[w][n][0];
-        const float sc = (mw == -INFINITY) ? 0.0f : exp2f(mw - M);
-        sm.wsc[w][n] = sc;
-        L += sm.ml[w][n][1] * sc;
+    if constexpr (DENSE) {
+      named_bar_sync(1, nct);
+      if (tid < G) {
+        const int n = tid;
+        float M = -INFINITY;
+        for (int w = 0; w < kNCW; ++w) M = fmaxf(M, sm.ml[w][n][0]);
+        float L = 0.0f;
+        for (int w = 0; w < kNCW; ++w) {
+          const float mw = sm.ml[w][n][0];
+          const float sc = (mw == -INFINITY) ? 0.0f : exp2f(mw - M);
+          sm.wsc[w][n] = sc;
+          L += sm.ml[w][n][1] * sc;
+        }
+        sm.MH[n] = M;
+        sm.LH[n] = M == -INFINITY ? 0.0f : L;
       }
-      sm.MH[n] = M;
-      sm.LH[n] = M == -INFINITY ? 0.0f : L;
-    }
-    named_bar_sync(1, nct);
+      named_bar_sync(1, nct);
 #pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      const int n = 2 * t4 + j;
-      if (n < G) {
-        const float sc = sm.wsc[warp][n];
-        const float bias = 1152.0f * st.ones[j];  // int8 V offset (see softmax_pv)
-        if constexpr (DENSE) {
+      for (int j = 0; j < 2; ++j) {
+        const int n = 2 * t4 + j;
+        if (n < G) {
+          const float sc = sm.wsc[warp][n];
 #pragma unroll
           for (int mt = 0; mt < 8; ++mt) {
-            atomicAdd(&sm.O[n][16 * mt + gq], (st.acc[mt][j] - bias) * sc);
-            atomicAdd(&sm.O[n][16 * mt + gq + 8], (st.acc[mt][2 + j] - bias) * sc);
-          }
-        } else {
-          float* stash = stashp + (warp * G + n) * kHeadDim;
-#pragma unroll
-          for (int mt = 0; mt < 8; ++mt) {
-            stash[16 * mt + gq] = (st.acc[mt][j] - bias) * sc;
-            stash[16 * mt + gq + 8] = (st.acc[mt][2 + j] - bias) * sc;
+            atomicAdd(&sm.O[n][16 * mt + gq], st.acc[mt][j] * sc);
+            atomicAdd(&sm.O[n][16 * mt + gq + 8], st.acc[mt][2 + j] * sc);
           }
         }
       }
-    }
-    named_bar_sync(1, nct);
-    if constexpr (!DENSE) {
+      named_bar_sync(1, nct);
+    } else {
+      named_bar_sync(1, nct);  // every warp is done with the tables
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const int n = 2 * t4 + j;
+        if (n < G) {
+          const float bias = 1152.0f * st.ones[j];  // int8 V offset (see softmax_pv)
+          float* stash = stashp + (warp * G + n) * kHeadDim;
+#pragma unroll
+          for (int mt = 0; mt < 8; ++mt) {
+            stash[16 * mt + gq] = st.acc[mt][j] - bias;
+            stash[16 * mt + gq + 8] = st.acc[mt][2 + j] - bias;
+          }
+        }
+      }
+      named_bar_sync(1, nct);
       for (int i = tid; i < G * kHeadDim; i += nct) {
         const int n = i / kHeadDim, d = i % kHeadDim;
-        float o = 0.0f;
+        float M = -INFINITY;
 #pragma unroll
-        for (int w = 0; w < kNCW; ++w) o += stashp[(w * G + n) * kHeadDim + d];
+        for (int w = 0; w < kNCW; ++w) M = fmaxf(M, sm.ml[w][n][0]);
+        float o = 0.0f, L = 0.0f;
+#pragma unroll
+        for (int w = 0; w < kNCW; ++w) {
+          const float mw = sm.ml[w][n][0];
+          const float sc = (mw == -INFINITY) ? 0.0f : exp2f(mw - M);
+          o = fmaf(stashp[(w * G + n) * kHeadDim + d], sc, o);
+          L = fmaf(sm.ml[w][n][1], sc, L);
+        }
         sm.O[n][d] = o;
+        if (d == 0) {
+          sm.MH[n] = M;
+          sm.LH[n] = M == -INFINITY ? 0.0f : L;
+        }
       }
       tbl_entries = 256;  // TBL1 holds the stash now
       named_bar_sync(1, nct);
