@@ -1336,6 +1336,12 @@ cudaError_t launch_decode_g(const DecodeParams& p, cudaStream_t stream, cudaEven
   decode_kernel<G, DENSE><<<p.S, kDecodeThreads, p.smem_bytes, stream>>>(p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  if (between) {
+    // a profile point right after the decode grid (an external record node
+    // when the stream is being captured; the merge then follows it in order)
+    e = cudaEventRecordWithFlags(between, stream, cudaEventRecordExternal);
+    if (e != cudaSuccess) return e;
+  }
   // the merge: a programmatic dependent of the decode grid (it may be
   // scheduled early and waits in-kernel for the grid's completion)
   cudaLaunchConfig_t cfg = {};
@@ -1350,11 +1356,6 @@ cudaError_t launch_decode_g(const DecodeParams& p, cudaStream_t stream, cudaEven
   cfg.numAttrs = 1;
   e = cudaLaunchKernelEx(&cfg, decode_merge_kernel<G>, p);
   if (e != cudaSuccess) return e;
-  if (between) {
-    // an external record node when the stream is being captured into a graph
-    e = cudaEventRecordWithFlags(between, stream, cudaEventRecordExternal);
-    if (e != cudaSuccess) return e;
-  }
   return cudaSuccess;
 }
 
