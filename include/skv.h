@@ -61,6 +61,7 @@ extern "C" {
 #define SKV_WS_ALLOCATE 0
 #define SKV_WS_DECODE 1
 #define SKV_WS_DENSE_DECODE 2
+#define SKV_WS_APPEND 3
 
 /* host tables exported for tests (skv_tables) */
 #define SKV_TABLE_BOUNDARY6_X 0  /* 64 fp32: cos((j+1/2) 2pi/64)                */
@@ -121,6 +122,8 @@ int skv_device_info(const skv_ctx* ctx, int* sm_count, int* default_splits);
 
 /* Bytes of device workspace that a call needs.
    SKV_WS_ALLOCATE: skv_allocate on B sequences x Hkv heads x Tmax tokens.
+   SKV_WS_APPEND: skv_append on B x Hkv units; Tmax carries the page-id
+   capacity (page_cap) instead.
    SKV_WS_DECODE / SKV_WS_DENSE_DECODE: the decode with num_splits chunks
    (0 = default) over B x Hkv units with Hq query heads.  The workspace is
    scratch that the call may overwrite; it must stay allocated until the
@@ -181,6 +184,38 @@ int skv_encode(skv_ctx* ctx, const uint16_t* K, const uint16_t* V, int B, int Hk
                const int32_t* seq_lens, const uint8_t* tier, const int32_t* row_of,
                const int32_t* page_indptr, const uint32_t* page_ids, const skv_pools* pools,
                int32_t* err_word, void* stream);
+
+/* skv_append -- decode-time ingest of the newest token (technical summary
+   2.2: protected tokens keep the top tier; 2.3 / abstract: the paged store
+   of the serving loop).  The paper states no per-step update of the store;
+   this is the plainest one: the token at position t = seq_lens[b] of every
+   kv head h becomes resident as T0 (the newest token lies in the protected
+   recent window).  It takes the next row of its unit's last T0 page, or,
+   when that page is full or the unit has no T0 page, a new T0 page whose
+   slot is free0[*free0_cursor + k] (k counts the units that need one, in
+   unit order) inserted at the end of the unit's T0 segment; later page ids
+   move up and the unit's T1/T2 rows move one page down in row_of.  The
+   store then equals what skv_allocate + skv_encode give for the same tiers
+   (page slots aside).  Re-running skv_allocate later demotes ageing tokens.
+     K_new, V_new  fp16 [B][Hkv][128] device: the new token's key and value
+     Tmax          capacity of tier/row_of; seq_lens[b] < Tmax is required
+     seq_lens      int32 [B] device, incremented by one
+     tier, row_of, page_indptr, page_tier_indptr (required), page_ids: the
+                   store's arrays as skv_allocate wrote them, updated
+     page_cap      capacity of page_ids
+     pools         the pools (only the T0 pool is written)
+     free0, free0_len  T0 free slots (device); *free0_cursor (device int32)
+                   is the first unused entry and is advanced
+     workspace     skv_workspace_size(SKV_WS_APPEND, B, Hkv, 0, page_cap) bytes
+   Device errors: SKV_ERR_ARG (seq_lens[b] >= Tmax), SKV_ERR_POOL (free list
+   or page capacity exhausted), SKV_ERR_CORRUPT (bad last T0 page id); the
+   store is then left unchanged. */
+int skv_append(skv_ctx* ctx, const uint16_t* K_new, const uint16_t* V_new, int B, int Hkv,
+               int64_t Tmax, int32_t* seq_lens, uint8_t* tier, int32_t* row_of,
+               int32_t* page_indptr, int32_t* page_tier_indptr, uint32_t* page_ids,
+               int64_t page_cap, const skv_pools* pools, const uint32_t* free0,
+               int64_t free0_len, int32_t* free0_cursor, int32_t* err_word, void* workspace,
+               size_t ws_bytes, void* stream);
 
 /* skv_decode_attention -- the ADA decode step (technical summary 2.1: logits
    computed directly from the radius and angle codes, no dense key

@@ -223,6 +223,11 @@ int skv_workspace_size(const skv_ctx* ctx, int which, int B, int Hkv, int Hq, in
     *bytes = skv::decode_ws(S, (long long)B * Hkv, G).bytes;
     return ok();
   }
+  if (which == SKV_WS_APPEND) {
+    // Tmax carries the page-id capacity here
+    *bytes = 4 * skv::append_ws((long long)B * Hkv, Tmax).words;
+    return ok();
+  }
   return fail(SKV_ERR_ARG, "skv_workspace_size: unknown kind %d", which);
 }
 
@@ -330,6 +335,51 @@ int skv_encode(skv_ctx* ctx, const uint16_t* K, const uint16_t* V, int B, int Hk
   std::memcpy(p.by4, ctx->by4, sizeof(p.by4));
   cudaError_t e = skv::launch_encode(p, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "skv_encode launch");
+  return ok();
+}
+
+int skv_append(skv_ctx* ctx, const uint16_t* K_new, const uint16_t* V_new, int B, int Hkv,
+               int64_t Tmax, int32_t* seq_lens, uint8_t* tier, int32_t* row_of,
+               int32_t* page_indptr, int32_t* page_tier_indptr, uint32_t* page_ids,
+               int64_t page_cap, const skv_pools* pools, const uint32_t* free0,
+               int64_t free0_len, int32_t* free0_cursor, int32_t* err_word, void* workspace,
+               size_t ws_bytes, void* stream) {
+  if (!ctx) return fail(SKV_ERR_ARG, "skv_append: null ctx");
+  if (B < 0 || Hkv <= 0 || Tmax <= 0 || page_cap < 0 || free0_len < 0)
+    return fail(SKV_ERR_ARG, "skv_append: bad sizes");
+  if (!K_new || !V_new || !seq_lens || !tier || !row_of || !page_indptr || !page_tier_indptr ||
+      !page_ids || !free0_cursor || !err_word || (free0_len > 0 && !free0))
+    return fail(SKV_ERR_ARG, "skv_append: null argument");
+  if (!pools || !pools->base[0] || pools->slots[0] < 0) return fail(SKV_ERR_ARG, "skv_append: bad T0 pool");
+  if ((long long)B * Hkv > (1LL << 24)) return fail(SKV_ERR_ARG, "skv_append: too many units");
+  const size_t need = 4 * skv::append_ws((long long)B * Hkv, page_cap).words;
+  if (!workspace || ws_bytes < need)
+    return fail(SKV_ERR_ARG, "skv_append: workspace of %zu bytes, %zu needed", ws_bytes, need);
+  skv::AppendParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.K = K_new;
+  p.V = V_new;
+  p.B = B;
+  p.Hkv = Hkv;
+  p.Tmax = Tmax;
+  p.P = ctx->P;
+  p.seq_lens = seq_lens;
+  p.tier = tier;
+  p.row_of = row_of;
+  p.indptr = page_indptr;
+  p.tier_indptr = page_tier_indptr;
+  p.ids = page_ids;
+  p.page_cap = page_cap;
+  p.pool0 = static_cast<uint8_t*>(pools->base[0]);
+  p.slots0 = pools->slots[0];
+  p.stride0 = ctx->stride[0];
+  p.free0 = free0;
+  p.free0_len = free0_len;
+  p.free0_cursor = free0_cursor;
+  p.err = err_word;
+  p.ws = static_cast<int32_t*>(workspace);
+  cudaError_t e = skv::launch_append(p, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "skv_append launch");
   return ok();
 }
 

@@ -263,6 +263,201 @@ __global__ void __launch_bounds__(256) encode_kernel(const __grid_constant__ Enc
   for (int i = 0; i < 4; ++i) vsec[v_frag_offset(row, 4 * lane + i, 1)] = (uint8_t)v8[i];
 }
 
+// ------------------------------------------------------------------ append
+// Decode-time ingest (the step before the decode in a serving loop): the
+// token at position t = seq_lens[b] of every kv head h becomes resident as
+// T0, the newest token being in the protected recent window.  It goes into
+// the next row of its unit's last T0 page, or, when that page is full or
+// the unit has none, into a new T0 page (a slot from the T0 free list)
+// inserted at the end of the unit's T0 segment; the later page ids move up
+// and the T1/T2 rows of that unit move one page down (row_of += P).  The
+// result is the layout a fresh pack of the same tiers gives (page slots
+// aside).  Three kernels: plan (one block: per-unit decisions, a scan of the
+// new pages, the new CSR offsets), move (page ids to their new positions
+// and the new ids), write (the token's row, headers, tier and row_of).
+
+__global__ void __launch_bounds__(1024) append_plan_kernel(const __grid_constant__ AppendParams p) {
+  __shared__ int scan[1024];
+  __shared__ int bad;
+  const int U = p.B * p.Hkv;
+  const AppendWs wl = append_ws(U, p.page_cap);
+  int32_t* const ws = p.ws;
+  const int tid = threadIdx.x, nt = blockDim.x;
+  if (tid == 0) bad = 0;
+  __syncthreads();
+  // per unit: the token's position and whether a new T0 page is needed
+  const int per = (U + nt - 1) / nt;
+  const int ua = min(U, tid * per), ub = min(U, ua + per);
+  int cnt = 0;
+  for (int u = ua; u < ub; ++u) {
+    const int t = p.seq_lens[u / p.Hkv];
+    const int A0 = p.tier_indptr[3 * u], A1 = p.tier_indptr[3 * u + 1];
+    int need = 1;
+    if (t < 0 || (long long)t >= p.Tmax) atomicExch(&bad, SKV_ERR_ARG);
+    if (A1 > A0) {
+      const uint32_t id = p.ids[A1 - 1];
+      const uint32_t slot = id & 0x3FFFFFFFu;
+      if ((id >> 30) != 0u || (long long)slot >= p.slots0) {
+        atomicExch(&bad, SKV_ERR_CORRUPT);
+      } else {
+        const uint32_t cnt_rows = *reinterpret_cast<const uint16_t*>(p.pool0 + (long long)slot * p.stride0);
+        need = cnt_rows >= (uint32_t)p.P;
+      }
+    }
+    ws[wl.t + u] = t;
+    ws[wl.need + u] = need;
+    ws[wl.a1 + u] = A1;
+    cnt += need;
+  }
+  // exclusive scan of the new pages over the units
+  scan[tid] = cnt;
+  __syncthreads();
+  for (int o = 1; o < nt; o <<= 1) {
+    const int v = tid >= o ? scan[tid - o] : 0;
+    __syncthreads();
+    scan[tid] += v;
+    __syncthreads();
+  }
+  const int total = scan[nt - 1];
+  int before = scan[tid] - cnt;
+  for (int u = ua; u < ub; ++u) {
+    ws[wl.nb + u] = before;
+    before += ws[wl.need + u];
+  }
+  const int n_raw = p.indptr[U];
+  const int n_old = max(0, (int)min((long long)n_raw, p.page_cap));
+  const int cur = *p.free0_cursor;
+  if (tid == 0) {
+    if (n_raw < 0 || (long long)n_raw > p.page_cap || cur < 0) atomicExch(&bad, SKV_ERR_CORRUPT);
+    else if ((long long)n_old + total > p.page_cap || (long long)cur + total > p.free0_len)
+      atomicExch(&bad, SKV_ERR_POOL);
+  }
+  for (int g = tid; g < n_old; g += nt) ws[wl.oids + g] = (int32_t)p.ids[g];
+  for (int u = tid; u <= U; u += nt) ws[wl.oindptr + u] = p.indptr[u];
+  __syncthreads();
+  if (bad) {
+    if (tid == 0) {
+      report(p.err, bad);
+      ws[wl.flag] = 1;
+    }
+    return;
+  }
+  // the new offsets (every read of the old ones is above the barrier)
+  for (int u = ua; u < ub; ++u) {
+    const int nb = ws[wl.nb + u], need = ws[wl.need + u];
+    p.indptr[u] += nb;
+    p.tier_indptr[3 * u] += nb;
+    p.tier_indptr[3 * u + 1] += nb + need;
+    p.tier_indptr[3 * u + 2] += nb + need;
+  }
+  for (int b = tid; b < p.B; b += nt) p.seq_lens[b] += 1;
+  if (tid == 0) {
+    p.indptr[U] += total;
+    p.tier_indptr[3 * U] += total;
+    ws[wl.flag] = 0;
+    ws[wl.cur] = cur;
+    *p.free0_cursor = cur + total;
+  }
+}
+
+// a warp per unit: its old page ids to their new positions, and its new id
+__global__ void __launch_bounds__(256) append_move_kernel(const __grid_constant__ AppendParams p) {
+  const int U = p.B * p.Hkv;
+  const AppendWs wl = append_ws(U, p.page_cap);
+  const int32_t* const ws = p.ws;
+  const int u = (int)(((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5);
+  const int lane = threadIdx.x & 31;
+  if (u >= U || ws[wl.flag]) return;
+  const int oi0 = ws[wl.oindptr + u], oi1 = ws[wl.oindptr + u + 1];
+  const int nb = ws[wl.nb + u], need = ws[wl.need + u], a1 = ws[wl.a1 + u];
+  for (int g = oi0 + lane; g < oi1; g += 32)
+    p.ids[g + nb + (g >= a1 ? need : 0)] = (uint32_t)ws[wl.oids + g];
+  if (need && lane == 0) {
+    const uint32_t slot = p.free0[ws[wl.cur] + nb];
+    if ((long long)slot >= p.slots0) report(p.err, SKV_ERR_POOL);
+    p.ids[a1 + nb] = slot & 0x3FFFFFFFu;  // tier 0
+  }
+}
+
+// a warp per unit: the new page (zeroed, header) or the next row of the last
+// T0 page, the token's fp16 K and V in the T0 row order, tier and row_of
+__global__ void __launch_bounds__(256) append_write_kernel(const __grid_constant__ AppendParams p) {
+  const int U = p.B * p.Hkv;
+  const AppendWs wl = append_ws(U, p.page_cap);
+  const int32_t* const ws = p.ws;
+  const int u = (int)(((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5);
+  const int lane = threadIdx.x & 31;
+  if (u >= U || ws[wl.flag]) return;
+  const int b = u / p.Hkv, h = u % p.Hkv, P = p.P;
+  const int t = ws[wl.t + u], need = ws[wl.need + u];
+  const int first = p.tier_indptr[3 * u], t0end = p.tier_indptr[3 * u + 1];
+  const uint32_t id = p.ids[t0end - 1];
+  const uint32_t slot = id & 0x3FFFFFFFu;
+  if ((id >> 30) != 0u || (long long)slot >= p.slots0) {
+    if (lane == 0) report(p.err, SKV_ERR_CORRUPT);
+    return;
+  }
+  uint8_t* page = p.pool0 + (long long)slot * p.stride0;
+  int row;
+  if (need) {
+    const int payload = kHdrBytes + P * 512;
+    for (int o = 16 * lane; o < payload; o += 512) *reinterpret_cast<uint4*>(page + o) = make_uint4(0, 0, 0, 0);
+    __syncwarp();
+    if (lane == 0)
+      *reinterpret_cast<uint4*>(page) =
+          make_uint4(1u | ((uint32_t)SKV_TIER_T0 << 16) | ((uint32_t)kPageMagic << 24), (uint32_t)b,
+                     (uint32_t)h, (uint32_t)(t0end - 1 - first));
+    row = 0;
+  } else {
+    uint32_t c = 0;
+    if (lane == 0) {
+      c = *reinterpret_cast<const uint16_t*>(page);
+      *reinterpret_cast<uint16_t*>(page) = (uint16_t)(c + 1);
+    }
+    row = (int)__shfl_sync(0xFFFFFFFFu, c, 0);
+  }
+  __syncwarp();
+  // the row, as the pack lays out T0 rows (see encode_kernel)
+  const long long w = (long long)u * kHeadDim;
+  const uint2 kv = *reinterpret_cast<const uint2*>(p.K + w + 4 * lane);
+  const uint2 vv = *reinterpret_cast<const uint2*>(p.V + w + 4 * lane);
+  const int c = lane >> 1, e0 = (lane & 1) * 4;
+  const int pos = c ^ (4 * (row & 1));
+  *reinterpret_cast<uint2*>(page + kHdrBytes + row * 256 + pos * 16 + e0 * 2) = kv;
+  uint8_t* vsec = page + kHdrBytes + 256 * P;
+  const uint16_t v4[4] = {(uint16_t)(vv.x & 0xFFFF), (uint16_t)(vv.x >> 16),
+                          (uint16_t)(vv.y & 0xFFFF), (uint16_t)(vv.y >> 16)};
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    *reinterpret_cast<uint16_t*>(vsec + v_frag_offset(row, 4 * lane + i, 2)) = v4[i];
+  // tier and row map: the token; with a new page, the unit's T1/T2 rows
+  // follow it one page further down the list
+  const long long base = (long long)u * p.Tmax;
+  if (lane == 0) {
+    p.tier[base + t] = SKV_TIER_T0;
+    p.row_of[base + t] = (t0end - 1 - first) * P + row;
+  }
+  if (need)
+    for (int k = lane; k < t; k += 32) {
+      const uint8_t tr = p.tier[base + k];
+      if (tr == SKV_TIER_T1 || tr == SKV_TIER_T2) p.row_of[base + k] += P;
+    }
+}
+
+cudaError_t launch_append(const AppendParams& p, cudaStream_t stream) {
+  const int U = p.B * p.Hkv;
+  if (U == 0) return cudaSuccess;
+  append_plan_kernel<<<1, 1024, 0, stream>>>(p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const unsigned blocks = (unsigned)((U + 7) / 8);
+  append_move_kernel<<<blocks, 256, 0, stream>>>(p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  append_write_kernel<<<blocks, 256, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_encode(const EncodeParams& p, cudaStream_t stream) {
   const long long warps = (long long)p.B * p.Hkv * p.Tmax;
   if (warps == 0) return cudaSuccess;

@@ -52,6 +52,49 @@ struct EncodeParams {
   float bx6[64], by6[64], bx4[16], by4[16];
 };
 
+// Decode-time append of one token per sequence (every kv head) as T0.
+struct AppendParams {
+  const uint16_t* K;  // fp16 [B][Hkv][128]: the new token's keys
+  const uint16_t* V;  // fp16 [B][Hkv][128]
+  int B, Hkv;
+  long long Tmax;
+  int P;
+  int32_t* seq_lens;        // [B], incremented
+  uint8_t* tier;            // [B][Hkv][Tmax]
+  int32_t* row_of;          // [B][Hkv][Tmax]
+  int32_t* indptr;          // [U + 1], updated
+  int32_t* tier_indptr;     // [3U + 1], updated
+  uint32_t* ids;            // [page_cap], updated
+  long long page_cap;
+  uint8_t* pool0;           // the T0 pool
+  long long slots0, stride0;
+  const uint32_t* free0;    // T0 free slots, taken from *free0_cursor on
+  long long free0_len;
+  int32_t* free0_cursor;
+  int32_t* err;
+  int32_t* ws;              // append_ws() int32 words
+};
+
+// Append workspace (int32 words): per unit t, need, new-before, old T0 end;
+// the old indptr [U + 1]; a flag word (1: the call changes nothing); the
+// free-list cursor before the call; the old page ids [page_cap].
+struct AppendWs {
+  size_t t, need, nb, a1, oindptr, flag, cur, oids, words;
+};
+__host__ __device__ inline AppendWs append_ws(long long U, long long page_cap) {
+  AppendWs w;
+  w.t = 0;
+  w.need = w.t + (size_t)U;
+  w.nb = w.need + (size_t)U;
+  w.a1 = w.nb + (size_t)U;
+  w.oindptr = w.a1 + (size_t)U;
+  w.flag = w.oindptr + (size_t)U + 1;
+  w.cur = w.flag + 1;
+  w.oids = w.cur + 1;
+  w.words = w.oids + (size_t)page_cap;
+  return w;
+}
+
 struct AllocParams {
   const uint16_t* K;
   int B, Hkv;
@@ -109,6 +152,7 @@ constexpr int kDecodeItemRows = 64;  // tokens per decode item
 cudaError_t launch_decode(const DecodeParams& p, int G, bool dense, cudaStream_t stream,
                           cudaEvent_t between);
 cudaError_t launch_encode(const EncodeParams& p, cudaStream_t stream);
+cudaError_t launch_append(const AppendParams& p, cudaStream_t stream);
 size_t alloc_workspace_bytes(int B, int Hkv, long long Tmax);
 void alloc_carve(AllocParams& p, void* ws);
 cudaError_t launch_allocate(AllocParams& p, cudaStream_t stream);

@@ -25,13 +25,13 @@ SKV_OK, SKV_ERR_ARG, SKV_ERR_BUDGET, SKV_ERR_POOL, SKV_ERR_CORRUPT, SKV_ERR_CUDA
 TIER_T0, TIER_T1, TIER_T2, TIER_DROP = range(4)
 MODE_QUOTA, MODE_BUDGET = 0, 1
 Q_FP16, Q_BF16 = 0, 1
-WS_ALLOCATE, WS_DECODE, WS_DENSE_DECODE = 0, 1, 2
+WS_ALLOCATE, WS_DECODE, WS_DENSE_DECODE, WS_APPEND = 0, 1, 2, 3
 TABLE_BOUNDARY6_X, TABLE_BOUNDARY6_Y, TABLE_BOUNDARY4_X, TABLE_BOUNDARY4_Y, TABLE_KAPPA, \
     TABLE_RHO_LEVELS = range(6)
 
 EXPORTS = [
     "skv_create", "skv_destroy", "skv_last_error", "skv_page_bytes", "skv_tables",
-    "skv_device_info", "skv_workspace_size", "skv_allocate", "skv_encode",
+    "skv_device_info", "skv_workspace_size", "skv_allocate", "skv_encode", "skv_append",
     "skv_decode_attention", "skv_decode_attention_static", "skv_dense_pack_bf16",
     "skv_dense_decode_bf16",
     "skv_set_profile_event", "skv_check",
@@ -63,6 +63,8 @@ _SIGS = {
                           C.POINTER(SkvPools), _p, _p, _p, _p, _p, _i64, _p, _p, _sz, _p]),
     "skv_encode": (_i, [_p, _p, _p, _i, _i, _i64, _p, _p, _p, _p, _p, C.POINTER(SkvPools), _p,
                         _p]),
+    "skv_append": (_i, [_p, _p, _p, _i, _i, _i64, _p, _p, _p, _p, _p, _p, _i64, C.POINTER(SkvPools),
+                        _p, _i64, _p, _p, _p, _sz, _p]),
     "skv_decode_attention": (_i, [_p, _p, _i, _i, _i, _i, _p, _p, _p, C.POINTER(SkvPools), _p, _p,
                                   _p, _p, _sz, _i, _p]),
     "skv_decode_attention_static": (_i, [_p, _p, _i, _i, _i, _i, _p, _p, _p,
@@ -208,6 +210,7 @@ class PagedCache:
 
     def allocate(self, K, seq_lens, utility, protect, mode, budget, quota, free_lists,
                  stream=None):
+        self._free0_cursor = None  # append() restarts after the slots this call takes
         fl = SkvFreeLists()
         self._free = [f.to(self.device, dtype=torch.int32) if isinstance(f, torch.Tensor) else
                       torch.from_numpy(np.asarray(f, np.uint32).view(np.int32)).to(self.device)
@@ -222,6 +225,26 @@ class PagedCache:
             _ptr(self.page_tier_indptr), _ptr(self.page_ids),
             self.page_cap, _ptr(self.err), _ptr(self._ws_alloc), self._ws_alloc.numel(),
             _stream(stream)))
+
+    def append(self, K_new, V_new, seq_lens, stream=None):
+        """Make the token at position seq_lens[b] of every kv head resident as
+        T0 (skv_append) and advance seq_lens.  K_new, V_new: fp16
+        [B][Hkv][128].  The T0 free list is the one given to allocate();
+        its cursor starts after the slots allocate took."""
+        if getattr(self, "_free0_cursor", None) is None:
+            tip = self.page_tier_indptr
+            U = self.B * self.Hkv
+            n0 = (tip[1:3 * U:3] - tip[0:3 * U:3]).sum().to(torch.int32).reshape(1)
+            self._free0_cursor = n0.clone()
+            n = self.ctx.workspace_size(WS_APPEND, self.B, self.Hkv, 0, self.page_cap)
+            self._ws_append = torch.empty(max(n, 1), dtype=torch.uint8, device=self.device)
+        free0 = self._free[0]
+        _check(lib().skv_append(
+            self.ctx.handle, _ptr(K_new), _ptr(V_new), self.B, self.Hkv, self.Tmax, _ptr(seq_lens),
+            _ptr(self.tier), _ptr(self.row_of), _ptr(self.page_indptr), _ptr(self.page_tier_indptr),
+            _ptr(self.page_ids), self.page_cap, C.byref(self._pools_c),
+            _ptr(free0) if free0.numel() else None, free0.numel(), _ptr(self._free0_cursor),
+            _ptr(self.err), _ptr(self._ws_append), self._ws_append.numel(), _stream(stream)))
 
     def encode(self, K, V, seq_lens, stream=None):
         _check(lib().skv_encode(
