@@ -51,6 +51,7 @@ def parse_args():
     ap.add_argument("--num-splits", type=int, default=0)
     ap.add_argument("--no-dense", action="store_true", help="skip the dense bf16 baseline")
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle cpu_baseline leg")
+    ap.add_argument("--no-append", action="store_true", help="skip the skv_append timing")
     ap.add_argument("--graph-steps", type=int, default=100)
     ap.add_argument("--seed", type=int, default=0)
     return ap.parse_args()
@@ -410,6 +411,38 @@ def run_skv(args, rank, world, local_rank):
                  "ada_speedup_step": dms / ms_per_step}
         del dcs, dws
 
+    # ---- decode-time append (skv_append) on the same recipe: a store built
+    # n_app tokens short, then n_app appends timed one after another
+    append = None
+    if not args.no_append:
+        import dataclasses
+        n_app = 64
+        wa = dataclasses.replace(w, seq_lens=(w.seq_lens - n_app).astype(np.int32))
+        slots = list(w.pool_slots)
+        slots[0] += w.B * w.Hkv * (n_app // w.P + 2)
+        wa = dataclasses.replace(wa, pool_slots=slots,
+                                 free_lists=[np.arange(x, dtype=np.uint32) for x in slots])
+        da = skv.workload_to_device(wa, dev)
+        ca = skv.build_cache(ctx, wa, da)
+        ca.check()
+        seq_a = da["seq_lens"].clone()
+        kv = [(d["K"][:, :, T - n_app + i].contiguous(), d["V"][:, :, T - n_app + i].contiguous())
+              for i in range(n_app)]
+        ca.append(*kv[0], seq_a)      # allocates the append workspace
+        torch.cuda.synchronize()
+        ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ea.record()
+        for i in range(1, n_app):
+            ca.append(*kv[i], seq_a)
+        eb.record()
+        torch.cuda.synchronize()
+        ca.check()
+        append = {"us_per_step": ea.elapsed_time(eb) * 1e3 / (n_app - 1), "steps": n_app - 1,
+                  "how": "skv_append of one token per sequence and kv head, eager launches "
+                         "(4 kernels each; pages are added every P steps), CUDA events "
+                         "around the steps"}
+        del ca, da
+
     cpu = None
     if rank == 0 and not args.no_cpu:
         cpu = cpu_baseline(T_sample=args.seq_len)
@@ -440,6 +473,7 @@ def run_skv(args, rank, world, local_rank):
             "clocks": clocks,
             "dense_bf16_baseline": dense,
             "ingest": {"allocate_ms": alloc_ms, "encode_ms": enc_ms, "gen_s": t_gen},
+            "append": append,
             "step_ms_graph_events": float(np.mean(step_ms)),
         }
         print(json.dumps(line), flush=True)

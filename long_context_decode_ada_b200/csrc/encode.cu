@@ -272,9 +272,11 @@ __global__ void __launch_bounds__(256) encode_kernel(const __grid_constant__ Enc
 // inserted at the end of the unit's T0 segment; the later page ids move up
 // and the T1/T2 rows of that unit move one page down (row_of += P).  The
 // result is the layout a fresh pack of the same tiers gives (page slots
-// aside).  Three kernels: plan (one block: per-unit decisions, a scan of the
+// aside).  Four kernels: plan (one block: per-unit decisions, a scan of the
 // new pages, the new CSR offsets), move (page ids to their new positions
-// and the new ids), write (the token's row, headers, tier and row_of).
+// and the new ids) and rowmap (the T1/T2 rows of a unit that gained a page),
+// both idle unless a page is added, and write (the token's row, headers,
+// tier and row_of).
 
 __global__ void __launch_bounds__(1024) append_plan_kernel(const __grid_constant__ AppendParams p) {
   __shared__ int scan[1024];
@@ -332,8 +334,10 @@ __global__ void __launch_bounds__(1024) append_plan_kernel(const __grid_constant
     else if ((long long)n_old + total > p.page_cap || (long long)cur + total > p.free0_len)
       atomicExch(&bad, SKV_ERR_POOL);
   }
-  for (int g = tid; g < n_old; g += nt) ws[wl.oids + g] = (int32_t)p.ids[g];
-  for (int u = tid; u <= U; u += nt) ws[wl.oindptr + u] = p.indptr[u];
+  if (total > 0) {  // the page ids move only when pages are added
+    for (int g = tid; g < n_old; g += nt) ws[wl.oids + g] = (int32_t)p.ids[g];
+    for (int u = tid; u <= U; u += nt) ws[wl.oindptr + u] = p.indptr[u];
+  }
   __syncthreads();
   if (bad) {
     if (tid == 0) {
@@ -356,26 +360,53 @@ __global__ void __launch_bounds__(1024) append_plan_kernel(const __grid_constant
     p.tier_indptr[3 * U] += total;
     ws[wl.flag] = 0;
     ws[wl.cur] = cur;
+    ws[wl.total] = total;
     *p.free0_cursor = cur + total;
   }
 }
 
-// a warp per unit: its old page ids to their new positions, and its new id
+// old page g to its new position (its unit found by binary search over the
+// old offsets), and each unit's new id; nothing to do when no page is added
 __global__ void __launch_bounds__(256) append_move_kernel(const __grid_constant__ AppendParams p) {
   const int U = p.B * p.Hkv;
   const AppendWs wl = append_ws(U, p.page_cap);
   const int32_t* const ws = p.ws;
-  const int u = (int)(((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5);
-  const int lane = threadIdx.x & 31;
-  if (u >= U || ws[wl.flag]) return;
-  const int oi0 = ws[wl.oindptr + u], oi1 = ws[wl.oindptr + u + 1];
-  const int nb = ws[wl.nb + u], need = ws[wl.need + u], a1 = ws[wl.a1 + u];
-  for (int g = oi0 + lane; g < oi1; g += 32)
-    p.ids[g + nb + (g >= a1 ? need : 0)] = (uint32_t)ws[wl.oids + g];
-  if (need && lane == 0) {
+  if (ws[wl.flag] || ws[wl.total] == 0) return;
+  const long long nthr = (long long)gridDim.x * blockDim.x;
+  const long long i0 = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const int n_old = ws[wl.oindptr + U];
+  for (long long g = i0; g < n_old; g += nthr) {
+    int lo = 0, hi = U - 1;  // the unit u with oindptr[u] <= g < oindptr[u + 1]
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (ws[wl.oindptr + mid] <= g) lo = mid; else hi = mid - 1;
+    }
+    const int u = lo;
+    const long long shift = ws[wl.nb + u] + (g >= ws[wl.a1 + u] ? ws[wl.need + u] : 0);
+    p.ids[g + shift] = (uint32_t)ws[wl.oids + g];
+  }
+  for (long long u = i0; u < U; u += nthr) {
+    if (!ws[wl.need + u]) continue;
+    const int nb = ws[wl.nb + u];
     const uint32_t slot = p.free0[ws[wl.cur] + nb];
     if ((long long)slot >= p.slots0) report(p.err, SKV_ERR_POOL);
-    p.ids[a1 + nb] = slot & 0x3FFFFFFFu;  // tier 0
+    p.ids[ws[wl.a1 + u] + nb] = slot & 0x3FFFFFFFu;  // tier 0
+  }
+}
+
+// a unit that gained a T0 page: its T1/T2 rows move one page down the list
+__global__ void __launch_bounds__(256) append_rowmap_kernel(const __grid_constant__ AppendParams p) {
+  const int U = p.B * p.Hkv;
+  const AppendWs wl = append_ws(U, p.page_cap);
+  const int32_t* const ws = p.ws;
+  if (ws[wl.flag] || ws[wl.total] == 0) return;
+  const long long n = (long long)U * p.Tmax;
+  const long long nthr = (long long)gridDim.x * blockDim.x;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += nthr) {
+    const long long u = i / p.Tmax, k = i - u * p.Tmax;
+    if (!ws[wl.need + u] || k >= ws[wl.t + u]) continue;
+    const uint8_t tr = p.tier[i];
+    if (tr == SKV_TIER_T1 || tr == SKV_TIER_T2) p.row_of[i] += p.P;
   }
 }
 
@@ -437,11 +468,6 @@ __global__ void __launch_bounds__(256) append_write_kernel(const __grid_constant
     p.tier[base + t] = SKV_TIER_T0;
     p.row_of[base + t] = (t0end - 1 - first) * P + row;
   }
-  if (need)
-    for (int k = lane; k < t; k += 32) {
-      const uint8_t tr = p.tier[base + k];
-      if (tr == SKV_TIER_T1 || tr == SKV_TIER_T2) p.row_of[base + k] += P;
-    }
 }
 
 cudaError_t launch_append(const AppendParams& p, cudaStream_t stream) {
@@ -450,11 +476,14 @@ cudaError_t launch_append(const AppendParams& p, cudaStream_t stream) {
   append_plan_kernel<<<1, 1024, 0, stream>>>(p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const unsigned blocks = (unsigned)((U + 7) / 8);
-  append_move_kernel<<<blocks, 256, 0, stream>>>(p);
+  // grid-stride kernels that leave at once when no page is added
+  append_move_kernel<<<1184, 256, 0, stream>>>(p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  append_write_kernel<<<blocks, 256, 0, stream>>>(p);
+  append_rowmap_kernel<<<1184, 256, 0, stream>>>(p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  append_write_kernel<<<(unsigned)((U + 7) / 8), 256, 0, stream>>>(p);
   return cudaGetLastError();
 }
 

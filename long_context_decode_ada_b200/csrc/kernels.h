@@ -77,9 +77,10 @@ struct AppendParams {
 
 // Append workspace (int32 words): per unit t, need, new-before, old T0 end;
 // the old indptr [U + 1]; a flag word (1: the call changes nothing); the
-// free-list cursor before the call; the old page ids [page_cap].
+// free-list cursor before the call; the number of new pages; the old page
+// ids [page_cap] (copied only when pages are added).
 struct AppendWs {
-  size_t t, need, nb, a1, oindptr, flag, cur, oids, words;
+  size_t t, need, nb, a1, oindptr, flag, cur, total, oids, words;
 };
 __host__ __device__ inline AppendWs append_ws(long long U, long long page_cap) {
   AppendWs w;
@@ -90,7 +91,8 @@ __host__ __device__ inline AppendWs append_ws(long long U, long long page_cap) {
   w.oindptr = w.a1 + (size_t)U;
   w.flag = w.oindptr + (size_t)U + 1;
   w.cur = w.flag + 1;
-  w.oids = w.cur + 1;
+  w.total = w.cur + 1;
+  w.oids = w.total + 1;
   w.words = w.oids + (size_t)page_cap;
   return w;
 }
