@@ -144,7 +144,7 @@ def written_partials(indptr: np.ndarray, ids: np.ndarray, payload, S: int) -> in
     """(run, unit) partials the decode kernel writes (and the merge kernel
     reads back).  Pages cost their tier's payload bytes.  With at most S
     units, unit u gets runs [B(u), B(u+1)), B(u) = u + round(P(u)(S-U)/C)
-    (P(u) the bytes before u, C the total); otherwise page g is in run
+    (P(u) the bytes before u, C the total) when S >= 8 U; otherwise page g is in run
     floor(C(g) S / C), C(g) the bytes before it.  A unit spread over several
     runs gets one partial per run, a unit inside one run none."""
     N = int(indptr[-1])
@@ -155,7 +155,7 @@ def written_partials(indptr: np.ndarray, ids: np.ndarray, payload, S: int) -> in
     before = np.concatenate([[0], np.cumsum(cost)[:-1]])
     total = int(cost.sum())
     n = 0
-    if U <= S:
+    if 8 * U <= S:  # unit-aligned split: at least 8 runs per unit
         ucost = [int(cost[int(indptr[u]):int(indptr[u + 1])].sum()) for u in range(U)]
         P = np.concatenate([[0], np.cumsum(ucost)])
         first = [u + (2 * int(P[u]) * (S - U) + total) // (2 * total) for u in range(U + 1)]

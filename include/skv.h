@@ -231,9 +231,10 @@ int skv_append(skv_ctx* ctx, const uint16_t* K_new, const uint16_t* V_new, int B
               pages within a unit; pages are streamed whole)
      page_tier_indptr  NULL, or skv_allocate's per-(unit, tier) offsets: the
               runs are then cut by payload bytes instead of page counts
-              (same results either way).  When B*Hkv <= num_splits every
-              unit gets its own runs, in proportion to its cost; otherwise
-              the page list of all units is cut into runs of equal cost.
+              (same results either way).  When num_splits >= 8*B*Hkv
+              every unit gets its own runs, in proportion to its cost;
+              otherwise the page list of all units is cut into runs of
+              equal cost.
      out      fp32 [B][Hq][128] device; lse fp32 [B][Hq] device or NULL
               (a unit without resident tokens gives out 0, lse -inf)
      num_splits  number of page runs = CTAs (0 = default: the SM count)
