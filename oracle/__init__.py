@@ -71,6 +71,7 @@ _SIGS = {
                       _p, _p, _p, _i64,                       # row_of indptr ids cap
                       _p, _p, _p, _p]),                       # pool0..2 pool_slots
     "orc_decode": (_i, [_i, _i, _i, _i, _i, _p, _p, _p, _p, _p, _i, _p, _p, _p, _i]),
+    "orc_attention_mass": (_i, [_i, _i, _i, _i, _i, _p, _p, _p, _p, _i, _p]),
     "orc_d2h": (_u16, [_d]),
     "orc_h2d": (_d, [_u16]),
     "orc_bf2d": (_d, [_u16]),
@@ -295,6 +296,37 @@ def decode(B, Hq, Hkv, Tmax, d, seq_lens, K, V, tier, q, q_dtype: str,
     if rc != OK:
         raise OracleError(rc, "decode")
     return out, lse
+
+
+def attention_mass(B, Hq, Hkv, Tmax, d, seq_lens, K, tier, q, q_dtype: str) -> np.ndarray:
+    """fp64 softmax weight of every resident token, summed over the query
+    heads of its kv group: [B][Hkv][Tmax] (0 where not resident)."""
+    seq = np.ascontiguousarray(seq_lens, np.int32)
+    k = _u16(K)
+    tr = np.ascontiguousarray(tier, np.uint8)
+    qq = _u16(q)
+    mass = np.zeros((B, Hkv, Tmax), np.float64)
+    rc = lib().orc_attention_mass(B, Hq, Hkv, Tmax, d, _ptr(seq), _ptr(k), _ptr(tr), _ptr(qq),
+                                  1 if q_dtype == "bf16" else 0, _ptr(mass))
+    if rc != OK:
+        raise OracleError(rc, "attention_mass")
+    return mass
+
+
+def accumulate_utility(utility, mass, seq_lens, gamma: float) -> np.ndarray:
+    """The utility update of one decode step, in fp64: u <- gamma u + mass at
+    every position t < seq_lens[b] (mass is 0 for dropped tokens), positions
+    at or past seq_lens[b] unchanged.  READING: the pages only name an
+    "estimated future utility"; accumulated attention mass with a geometric
+    decay gamma (gamma = 1: the plain running sum) is the plainest estimator
+    that the decode itself supplies."""
+    u = np.array(utility, np.float64, copy=True)
+    m = np.asarray(mass, np.float64)
+    seq = np.asarray(seq_lens)
+    for b in range(u.shape[0]):
+        T = int(seq[b])
+        u[b, :, :T] = gamma * u[b, :, :T] + m[b, :, :T]
+    return u
 
 
 def run_workload(w, units=None, do_decode=True):

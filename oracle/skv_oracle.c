@@ -783,6 +783,66 @@ int orc_decode(int B, int Hq, int Hkv, int Tmax, int d, const int32_t* seq_lens,
     return bad ? ORC_ERR_ARG : ORC_OK;
 }
 
+/* Attention mass per resident token, the decode-side utility signal.
+   READING: [ABS] drives retention by an "estimated future utility" without
+   saying how it is estimated; the plainest estimator the decode supplies is
+   the softmax weight a token receives, summed over the query heads of its
+   kv group.  mass[b][h][t] = sum_{g<G} softmax_t(l_{hq})[t], hq = h G + g,
+   with l_t = q . k^_t / sqrt(d) exactly as in orc_decode; 0 for dropped
+   tokens and positions >= seq_lens[b].  Every unit with a resident token
+   has sum_t mass = G. */
+int orc_attention_mass(int B, int Hq, int Hkv, int Tmax, int d, const int32_t* seq_lens,
+                       const uint16_t* K, const uint8_t* tier, const uint16_t* q, int q_kind,
+                       double* mass) {
+    if (Hkv <= 0 || Hq % Hkv != 0 || d <= 0) return ORC_ERR_ARG;
+    init_once();
+    int G = Hq / Hkv;
+    for (int64_t i = 0; i < (int64_t)B * Hkv * Tmax; i++) mass[i] = 0.0;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int w = 0; w < B * Hq; w++) {
+        int b = w / Hq, hq = w % Hq, h = hq / G;
+        int T = seq_lens[b];
+        double* qd = (double*)malloc(sizeof(double) * d);
+        for (int c = 0; c < d; c++) {
+            uint16_t x = q[((int64_t)b * Hq + hq) * d + c];
+            qd[c] = q_kind ? bf2d(x) : h2d(x);
+        }
+        double* logit = (double*)malloc(sizeof(double) * (T > 0 ? T : 1));
+        double* kh = (double*)malloc(sizeof(double) * d);
+        double mx = -INFINITY;
+        for (int t = 0; t < T; t++) {
+            int64_t idx = ((int64_t)b * Hkv + h) * Tmax + t;
+            int tr = tier[idx];
+            if (tr == TIER_DROP) { logit[t] = -INFINITY; continue; }
+            const uint16_t* k = K + idx * d;
+            if (tr == TIER_T0)
+                for (int c = 0; c < d; c++) kh[c] = h2d(k[c]);
+            else
+                orc_reconstruct(k, d, tr == TIER_T1 ? BITS_T1 : BITS_T2, kh);
+            double s = 0.0;
+            for (int c = 0; c < d; c++) s += qd[c] * kh[c];
+            logit[t] = s / sqrt((double)d);
+            if (logit[t] > mx) mx = logit[t];
+        }
+        if (mx != -INFINITY) {
+            double l = 0.0;
+            for (int t = 0; t < T; t++)
+                if (logit[t] != -INFINITY) l += exp(logit[t] - mx);
+            for (int t = 0; t < T; t++) {
+                if (logit[t] == -INFINITY) continue;
+                int64_t idx = ((int64_t)b * Hkv + h) * Tmax + t;
+                double p = exp(logit[t] - mx) / l;
+#pragma omp atomic
+                mass[idx] += p;
+            }
+        }
+        free(qd);
+        free(logit);
+        free(kh);
+    }
+    return ORC_OK;
+}
+
 /* helpers exposed for pins: fp16 rounding, exact norm as double */
 uint16_t orc_d2h(double x) { return d2h(x); }
 double orc_h2d(uint16_t h) { return h2d(h); }
