@@ -52,6 +52,8 @@ def parse_args():
     ap.add_argument("--no-dense", action="store_true", help="skip the dense bf16 baseline")
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle cpu_baseline leg")
     ap.add_argument("--no-append", action="store_true", help="skip the skv_append timing")
+    ap.add_argument("--no-utility", action="store_true",
+                    help="skip the skv_decode_utility timing")
     ap.add_argument("--graph-steps", type=int, default=100)
     ap.add_argument("--seed", type=int, default=0)
     return ap.parse_args()
@@ -411,6 +413,51 @@ def run_skv(args, rank, world, local_rank):
                  "ada_speedup_step": dms / ms_per_step}
         del dcs, dws
 
+    # ---- the decode with the utility update (skv_decode_utility) on the same
+    # two stores, timed as the main step (graph replays, CUDA events)
+    utility = None
+    if not args.no_utility:
+        uts = [torch.zeros((w.B, w.Hkv, w.Tmax), dtype=torch.float32, device=dev)
+               for _ in range(2)]
+        uws = [c.utility_workspace(w.Hq, S) for c in caches]
+
+        def make_ustep(k):
+            def step(mid_event):
+                ctx.set_profile_event(mid_event)
+                caches[k].decode_utility(d["q"], d["q_dtype"], w.Hq, d["seq_lens"], uts[k], 0.9,
+                                         out=out, lse=lse, workspace=uws[k], num_splits=S)
+            return step
+
+        u_steps = 1000
+        gu, gu_tail, gu_prof, evu, reps_u = timed_graph_steps(
+            [make_ustep(0), make_ustep(1)], u_steps, 5, args.graph_steps, stream)
+        ctx.set_profile_event(None)
+        ua, ub = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ua.record()
+        for _ in range(reps_u):
+            gu.replay()
+        if gu_tail is not None:
+            gu_tail.replay()
+        ub.record()
+        torch.cuda.synchronize()
+        caches[0].check()
+        gu_prof.replay()
+        torch.cuda.synchronize()
+        u_kern = float(np.mean([a.elapsed_time(b) for a, b, c in evu]))
+        u_rest = float(np.mean([b.elapsed_time(c) for a, b, c in evu]))
+        G = w.Hq // w.Hkv
+        logit_bytes = resident * G * 4
+        utility = {"us_per_step": ua.elapsed_time(ub) * 1e3 / u_steps, "steps": u_steps,
+                   "decode_kernel_us": u_kern * 1e3, "merge_and_update_us": u_rest * 1e3,
+                   "plain_step_us": ms_per_step * 1e3,
+                   "logit_bytes_written": logit_bytes,
+                   "update_bytes": logit_bytes + w.B * w.Hkv * w.Tmax * (1 + 4 + 4 + 4),
+                   "how": "skv_decode_utility (decode with per-row logit capture, merge, "
+                          "utility update u <- 0.9 u + mass) in graphs of "
+                          f"{min(args.graph_steps, u_steps)} steps over the two stores; the "
+                          "profile graph's events split the decode kernel from the rest"}
+        del uts, uws, gu, gu_tail, gu_prof
+
     # ---- decode-time append (skv_append) on the same recipe: a store built
     # n_app tokens short, then n_app appends timed one after another
     append = None
@@ -474,6 +521,7 @@ def run_skv(args, rank, world, local_rank):
             "dense_bf16_baseline": dense,
             "ingest": {"allocate_ms": alloc_ms, "encode_ms": enc_ms, "gen_s": t_gen},
             "append": append,
+            "utility": utility,
             "step_ms_graph_events": float(np.mean(step_ms)),
         }
         print(json.dumps(line), flush=True)

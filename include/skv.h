@@ -62,6 +62,7 @@ extern "C" {
 #define SKV_WS_DECODE 1
 #define SKV_WS_DENSE_DECODE 2
 #define SKV_WS_APPEND 3
+#define SKV_WS_DECODE_UTILITY 4
 
 /* host tables exported for tests (skv_tables) */
 #define SKV_TABLE_BOUNDARY6_X 0  /* 64 fp32: cos((j+1/2) 2pi/64)                */
@@ -125,7 +126,10 @@ int skv_device_info(const skv_ctx* ctx, int* sm_count, int* default_splits);
    SKV_WS_APPEND: skv_append on B x Hkv units; Tmax carries the page-id
    capacity (page_cap) instead.
    SKV_WS_DECODE / SKV_WS_DENSE_DECODE: the decode with num_splits chunks
-   (0 = default) over B x Hkv units with Hq query heads.  The workspace is
+   (0 = default) over B x Hkv units with Hq query heads.
+   SKV_WS_DECODE_UTILITY: skv_decode_utility; Tmax carries the page-id
+   capacity (page_cap): the decode's scratch plus page_cap * P * (Hq/Hkv)
+   fp32 captured logits.  The workspace is
    scratch that the call may overwrite; it must stay allocated until the
    stream has run the call. */
 int skv_workspace_size(const skv_ctx* ctx, int which, int B, int Hkv, int Hq, int64_t Tmax,
@@ -245,6 +249,36 @@ int skv_decode_attention(skv_ctx* ctx, const void* q, int q_dtype, int B, int Hq
                          const int32_t* page_indptr, const int32_t* page_tier_indptr,
                          const uint32_t* page_ids, const skv_pools* pools, float* out, float* lse, int32_t* err_word,
                          void* workspace, size_t ws_bytes, int num_splits, void* stream);
+
+/* skv_decode_utility -- the decode of skv_decode_attention plus the
+   utility update that closes the retention loop.  The abstract's retention
+   decides by "estimated future utility" without saying how it is estimated;
+   this library's reading is the attention mass the decode itself computes:
+     mass[b][h][t] = sum_{g < G} softmax_t(l_{hG+g})[t]   (0 if dropped)
+     utility[b][h][t] <- gamma * utility[b][h][t] + mass[b][h][t]
+   for every t < seq_lens[b] (positions past it are left unchanged), so that
+   gamma = 1 keeps the running sum and gamma < 1 a geometric decay.  The
+   decode stores each resident row's logit (fp32, log2 domain) in the
+   workspace as it streams the pages; a second kernel forms the mass from
+   those logits and the merged lse.  The result feeds skv_allocate's utility.
+     q ... num_splits   as for skv_decode_attention (lse is required)
+     page_cap      capacity of page_ids (rows of the logit scratch / P)
+     Tmax, seq_lens, tier, row_of   skv_allocate's / skv_append's outputs
+                   for the same store (device; row_of locates a token's row)
+     gamma         decay of the previous utility (host float)
+     utility       fp32 [B][Hkv][Tmax] device, updated in place
+     workspace     skv_workspace_size(SKV_WS_DECODE_UTILITY, B, Hkv, Hq,
+                   page_cap, num_splits) bytes
+   Device errors: as skv_decode_attention, plus SKV_ERR_CORRUPT when a
+   resident token's row lies outside its unit's pages (its utility is then
+   left unchanged) and SKV_ERR_ARG when page_cap is below the page count. */
+int skv_decode_utility(skv_ctx* ctx, const void* q, int q_dtype, int B, int Hq, int Hkv,
+                       const int32_t* page_indptr, const int32_t* page_tier_indptr,
+                       const uint32_t* page_ids, int64_t page_cap, const skv_pools* pools,
+                       int64_t Tmax, const int32_t* seq_lens, const uint8_t* tier,
+                       const int32_t* row_of, float gamma, float* utility, float* out, float* lse,
+                       int32_t* err_word, void* workspace, size_t ws_bytes, int num_splits,
+                       void* stream);
 
 /* skv_decode_attention_static -- skv_decode_attention without a caller
    workspace (the paper has no counterpart: this is an interface convenience

@@ -207,6 +207,11 @@ static int decode_splits(const skv_ctx* ctx, int num_splits) {
   return num_splits > 0 ? num_splits : ctx->sm_count;
 }
 
+// offset of the logit rows in a SKV_WS_DECODE_UTILITY workspace (256-byte aligned)
+static size_t decode_utility_logits_at(long long S, long long U, int G) {
+  return (skv::decode_ws(S, U, G).bytes + 255) / 256 * 256;
+}
+
 int skv_workspace_size(const skv_ctx* ctx, int which, int B, int Hkv, int Hq, int64_t Tmax,
                        int num_splits, size_t* bytes) {
   if (!ctx || !bytes) return fail(SKV_ERR_ARG, "skv_workspace_size: null argument");
@@ -221,6 +226,16 @@ int skv_workspace_size(const skv_ctx* ctx, int which, int B, int Hkv, int Hq, in
     const long long S = decode_splits(ctx, num_splits);
     // split partials, then each unit's range of runs
     *bytes = skv::decode_ws(S, (long long)B * Hkv, G).bytes;
+    return ok();
+  }
+  if (which == SKV_WS_DECODE_UTILITY) {
+    // Tmax carries the page-id capacity here: the decode's scratch, then the
+    // captured logits of page_cap * P rows x G heads
+    if (Hq <= 0 || Hq % Hkv != 0) return fail(SKV_ERR_ARG, "Hq must be a multiple of Hkv");
+    const int G = Hq / Hkv;
+    const long long S = decode_splits(ctx, num_splits);
+    *bytes = decode_utility_logits_at(S, (long long)B * Hkv, G) +
+             (size_t)Tmax * (size_t)ctx->P * (size_t)G * 4;
     return ok();
   }
   if (which == SKV_WS_APPEND) {
@@ -388,7 +403,8 @@ static int decode_common(skv_ctx* ctx, const void* q, int q_dtype, int B, int Hq
                          const uint32_t* page_ids, const void* pool[3],
                          const long long slots[3], bool dense, float* out, float* lse,
                          int32_t* err_word, void* workspace, size_t ws_bytes, int num_splits,
-                         void* stream, const char* name) {
+                         void* stream, const char* name, float* logits = nullptr,
+                         long long logit_rows = 0) {
   if (!ctx) return fail(SKV_ERR_ARG, "%s: null ctx", name);
   if (B < 0 || Hkv <= 0 || Hq <= 0 || Hq % Hkv != 0)
     return fail(SKV_ERR_ARG, "%s: need B >= 0 and Hq a multiple of Hkv", name);
@@ -426,6 +442,8 @@ static int decode_common(skv_ctx* ctx, const void* q, int q_dtype, int B, int Hq
   p.lse = lse;
   p.err = err_word;
   p.part = static_cast<float*>(workspace);
+  p.logits = logits;
+  p.logit_rows = logit_rows;
   p.S = decode_splits(ctx, num_splits);
   p.P = ctx->P;
   p.log2P = ctx->log2P;
@@ -458,6 +476,58 @@ int skv_decode_attention(skv_ctx* ctx, const void* q, int q_dtype, int B, int Hq
                        slots, false, out,
                        lse, err_word, workspace, ws_bytes, num_splits, stream,
                        "skv_decode_attention");
+}
+
+int skv_decode_utility(skv_ctx* ctx, const void* q, int q_dtype, int B, int Hq, int Hkv,
+                       const int32_t* page_indptr, const int32_t* page_tier_indptr,
+                       const uint32_t* page_ids, int64_t page_cap, const skv_pools* pools,
+                       int64_t Tmax, const int32_t* seq_lens, const uint8_t* tier,
+                       const int32_t* row_of, float gamma, float* utility, float* out, float* lse,
+                       int32_t* err_word, void* workspace, size_t ws_bytes, int num_splits,
+                       void* stream) {
+  static const char* name = "skv_decode_utility";
+  if (!ctx) return fail(SKV_ERR_ARG, "%s: null ctx", name);
+  if (B < 0 || Hkv <= 0 || Hq <= 0 || Hq % Hkv != 0 || Tmax < 0 || page_cap < 0 ||
+      num_splits < 0)
+    return fail(SKV_ERR_ARG, "%s: bad sizes", name);
+  if (B == 0) return ok();
+  if (!seq_lens || !tier || !row_of || !utility || !lse)
+    return fail(SKV_ERR_ARG, "%s: null argument", name);
+  if (!valid_pools(pools, 3)) return fail(SKV_ERR_ARG, "%s: bad pools", name);
+  size_t need = 0;
+  int rc = skv_workspace_size(ctx, SKV_WS_DECODE_UTILITY, B, Hkv, Hq, page_cap, num_splits, &need);
+  if (rc != SKV_OK) return rc;
+  if (!workspace || ws_bytes < need)
+    return fail(SKV_ERR_ARG, "%s: workspace of %zu bytes needed", name, need);
+  const int G = Hq / Hkv;
+  const size_t at = decode_utility_logits_at(decode_splits(ctx, num_splits), (long long)B * Hkv, G);
+  float* logits = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + at);
+  const long long rows = (long long)page_cap * ctx->P;
+  const void* pool[3] = {pools->base[0], pools->base[1], pools->base[2]};
+  const long long slots[3] = {pools->slots[0], pools->slots[1], pools->slots[2]};
+  rc = decode_common(ctx, q, q_dtype, B, Hq, Hkv, page_indptr, page_tier_indptr, page_ids, pool,
+                     slots, false, out, lse, err_word, workspace, at, num_splits, stream, name,
+                     logits, rows);
+  if (rc != SKV_OK) return rc;
+  skv::UtilityParams u;
+  u.logits = logits;
+  u.logit_rows = rows;
+  u.lse = lse;
+  u.seq_lens = seq_lens;
+  u.tier = tier;
+  u.row_of = row_of;
+  u.indptr = page_indptr;
+  u.B = B;
+  u.Hkv = Hkv;
+  u.G = G;
+  u.P = ctx->P;
+  u.Tmax = Tmax;
+  u.gamma = gamma;
+  u.utility = utility;
+  u.err = err_word;
+  cudaError_t e = skv::launch_utility(u, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "skv_decode_utility: utility update");
+  return ok();
 }
 
 int skv_dense_decode_bf16(skv_ctx* ctx, const void* q, int q_dtype, int B, int Hq, int Hkv,

@@ -100,6 +100,7 @@ struct __align__(16) DecodeSmem {
   uint4 desc[kNSlot];                  // consumers' view of an item
   PageCopy copy[kNSlot][kMaxIPP];      // issuers' view of an item
   uint32_t copy_bytes[kNSlot];         // bytes of the item (0xFFFFFFFF: no more items)
+  uint32_t dpage[kNSlot];              // the item's first page (index into the page list)
   unsigned long long vstart[64];       // planner: virtual ring start of item j at j % 64
   unsigned long long scan[kDecodeThreads / 32];
   unsigned long long ucost[3 * kTouchedUnits + 1];  // cost before segments 3 unit0 ..
@@ -639,12 +640,25 @@ __device__ __forceinline__ void softmax_pv(float lA, float lB, float vsA, float 
   }
 }
 
+// Lane (t, g) holds the log2-domain logits of head g for rows rA and rB;
+// with capture on, heads g < G store them at lg[row * G + g] (the 8 rows of
+// a half-step and their G heads are contiguous: one 32 G-byte segment).
+template <int G>
+__device__ __forceinline__ void capture_logits(float* lg, int rA, int rB, bool vA, bool vB,
+                                               float lA, float lB, int g) {
+  if (lg != nullptr && g < G) {
+    if (vA) lg[rA * G + g] = lA;
+    if (vB) lg[rB * G + g] = lB;
+  }
+}
+
 // 16 rows [row0, row0 + 16) of one page at shared address pg; tb1 / tb2:
-// this lane's copy in TBL1 / TBL2.
-template <int G, bool DENSE>
+// this lane's copy in TBL1 / TBL2; lg: the page's logit rows, or NULL
+// (CAP: the kernel variant that captures logits).
+template <int G, bool DENSE, bool CAP>
 __device__ __forceinline__ void process_rows(const DecodeParams& p, uint32_t pg, uint32_t tier,
                                              int row0, const QFrag& qf, uint32_t tb1,
-                                             uint32_t tb2, WarpState& st, int lane) {
+                                             uint32_t tb2, WarpState& st, int lane, float* lg) {
   const int t = lane >> 2, g = lane & 3;
   const int P = p.P;
   // header {u16 count, u8 tier, u8 magic}
@@ -670,9 +684,10 @@ __device__ __forceinline__ void process_rows(const DecodeParams& p, uint32_t pg,
   } else {
     if (tier == SKV_TIER_T0) {
       logits_k16<false, false>(pg, rA, g, qf, c, d);
-      const float a = c[0] + d[0], b = c[2] + d[2];
-      softmax_pv<G, 1>(vA ? a * qf.c0 : -INFINITY, vB ? b * qf.c0 : -INFINITY, 1.0f, 1.0f,
-                       vsec_dense, vsec_dense + 2048, st, lane);
+      const float lA = vA ? (c[0] + d[0]) * qf.c0 : -INFINITY;
+      const float lB = vB ? (c[2] + d[2]) * qf.c0 : -INFINITY;
+      if constexpr (CAP) capture_logits<G>(lg, rA, rB, vA, vB, lA, lB, g);
+      softmax_pv<G, 1>(lA, lB, 1.0f, 1.0f, vsec_dense, vsec_dense + 2048, st, lane);
     } else {
       const bool t1 = tier == SKV_TIER_T1;
       if (t1)
@@ -687,13 +702,15 @@ __device__ __forceinline__ void process_rows(const DecodeParams& p, uint32_t pg,
       const float vsA = __half2float(__ushort_as_half((unsigned short)lds16(ss + 2 * rA)));
       const float vsB = __half2float(__ushort_as_half((unsigned short)lds16(ss + 2 * rB)));
       const uint32_t vsec = pg + kHdrBytes + (2 + cb + 2) * P + (row0 >> 3) * 1024;
-      softmax_pv<G, 0>(vA ? a * (rtA * qf.c1) : -INFINITY, vB ? b * (rtB * qf.c1) : -INFINITY,
-                       vA ? vsA : 0.0f, vB ? vsB : 0.0f, vsec, vsec + 1024, st, lane);
+      const float lA = vA ? a * (rtA * qf.c1) : -INFINITY;
+      const float lB = vB ? b * (rtB * qf.c1) : -INFINITY;
+      if constexpr (CAP) capture_logits<G>(lg, rA, rB, vA, vB, lA, lB, g);
+      softmax_pv<G, 0>(lA, lB, vA ? vsA : 0.0f, vB ? vsB : 0.0f, vsec, vsec + 1024, st, lane);
     }
   }
 }
 
-template <int G, bool DENSE>
+template <int G, bool DENSE, bool CAP>
 __global__ void __launch_bounds__(kDecodeThreads, 1)
     decode_kernel(const __grid_constant__ DecodeParams p) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
@@ -821,6 +838,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         ub_next = u + 2 <= U ? (long long)p.indptr[u + 2] : g1;
       }
       const int nb = (int)min(32LL, (ub - pg + ipp - 1) / ipp);  // items in this batch
+      const uint32_t my_pg = CAP ? (uint32_t)(pg + (long long)lane * ipp) : 0u;
       // ---- lane-parallel decode of item it + lane
       uint32_t plo[kMaxIPP], phi[kMaxIPP], psz[kMaxIPP];
       uint32_t total = 0, imeta = 0, relz = 0, relw = 0;
@@ -941,6 +959,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         if (now) {
           const int s = (it + lane) % kNSlot;
           sm.desc[s] = make_uint4(ring_lo + my_off, imeta, relz, relw);
+          if (CAP) sm.dpage[s] = my_pg;
           const uint32_t rel[kMaxIPP] = {0u, relz & 0xFFFFu, relz >> 16, relw};
 #pragma unroll
           for (int q = 0; q < kMaxIPP; ++q)
@@ -1102,6 +1121,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       if (ok) {
         const uint4 d = lds128(smem_u32(&sm.desc[s]));
         const uint32_t np = d.y & 7u;
+        const long long dpg = CAP ? (long long)sm.dpage[s] : -1;
 #pragma unroll
         for (int ps = 0; ps < kPasses; ++ps) {
           const int r = kRowsPerWarp * wi + 16 * ps;  // row within the item
@@ -1111,8 +1131,16 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
             const uint32_t rel = kp == 0 ? 0u
                                          : (kp == 1 ? (d.z & 0xFFFFu)
                                                     : (kp == 2 ? (d.z >> 16) : d.w));
-            process_rows<G, DENSE>(p, d.x + rel, (d.y >> (kMetaTierShift + 2 * kp)) & 3u, row0,
-                                   qf, tb1, tb2, st, lane);
+            float* lg = nullptr;
+            if (CAP && dpg >= 0) {
+              const long long r0 = (dpg + kp) * p.P;  // the page's first logit row
+              if (r0 + p.P <= p.logit_rows)
+                lg = p.logits + r0 * G;
+              else if (lane == 0)
+                report(p.err, SKV_ERR_ARG);
+            }
+            process_rows<G, DENSE, CAP>(p, d.x + rel, (d.y >> (kMetaTierShift + 2 * kp)) & 3u, row0,
+                                   qf, tb1, tb2, st, lane, lg);
           }
         }
       }
@@ -1280,6 +1308,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
 template <int G>
 __global__ void __launch_bounds__(G * kHeadDim / 2)
     decode_merge_kernel(const __grid_constant__ DecodeParams p) {
+  // a programmatic dependent of the merge (the utility update) may start
+  // its own prologue now; it waits for this grid before reading results
+  asm volatile("griddepcontrol.launch_dependents;");
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const int u = blockIdx.x;
   const int U = p.B * p.Hkv;
@@ -1326,6 +1357,106 @@ __global__ void __launch_bounds__(G * kHeadDim / 2)
     p.lse[obase + n] = L > 0.0f ? (M + log2f(L)) * 0.69314718055994530942f : -INFINITY;
 }
 
+// Utility update: every position t < seq_lens[b] of every unit takes
+// u <- gamma u + mass, where the mass of a resident token is its softmax
+// weight summed over the G query heads of its kv head, 2^(l_g - lse_g log2 e)
+// from the logit the decode captured for its row (page index in the unit's
+// list * P + row, from row_of); dropped tokens have mass 0.  Grid: x over
+// positions, y over units; one position per thread per pass, so the tier,
+// row map and utility streams are read in position order (a tier segment's
+// logit rows are in the same order).  Launched as a programmatic dependent
+// of the merge: the loads that do not depend on the decode (tier, row map,
+// old utility of the first position) are issued before the wait for the
+// decode's results.  The unit's lse goes through shared memory: one load
+// per block, not one per thread (the same 16 bytes requested by every
+// thread would queue at a single L2 slice).
+template <int G>
+__global__ void __launch_bounds__(256) utility_kernel(const UtilityParams p) {
+  constexpr float kLog2e = 1.4426950408889634f;
+  __shared__ float ls_s[G];
+  const int U = p.B * p.Hkv;
+  const int T = (int)p.Tmax;
+  bool waited = false;
+  for (int u = blockIdx.y; u < U; u += gridDim.y) {
+    const int len = min(T, p.seq_lens[u / p.Hkv]);
+    const long long base = (long long)u * T;
+    const int t0 = blockIdx.x * blockDim.x + threadIdx.x;
+    uint32_t tr = SKV_TIER_DROP;
+    int loc = -1;
+    float u_old = 0.0f;
+    if (t0 < len) {
+      tr = p.tier[base + t0];
+      loc = p.row_of[base + t0];
+      u_old = p.utility[base + t0];
+    }
+    if (!waited) {  // uniform: every thread of the block takes it on the first unit
+      asm volatile("griddepcontrol.wait;" ::: "memory");
+      waited = true;
+    }
+    __syncthreads();  // the previous unit's lse has been read
+    if (threadIdx.x < G) ls_s[threadIdx.x] = __ldcg(p.lse + (long long)u * G + threadIdx.x) * kLog2e;
+    __syncthreads();
+    float ls2[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) ls2[g] = ls_s[g];
+    const long long r0 = (long long)p.indptr[u] * p.P, r1 = (long long)p.indptr[u + 1] * p.P;
+    for (int t = t0; t < len; t += gridDim.x * blockDim.x) {
+      if (t != t0) {
+        tr = p.tier[base + t];
+        loc = p.row_of[base + t];
+        u_old = p.utility[base + t];
+      }
+      float mass = 0.0f;
+      if (tr != SKV_TIER_DROP) {
+        const long long gr = r0 + loc;
+        if (tr > SKV_TIER_DROP || loc < 0 || gr >= r1 || gr >= p.logit_rows) {
+          report(p.err, SKV_ERR_CORRUPT);
+          continue;
+        }
+        const float* l = p.logits + gr * G;
+        float lv[G];
+        if constexpr (G == 4) {
+          const float4 x = __ldcg(reinterpret_cast<const float4*>(l));
+          lv[0] = x.x; lv[1] = x.y; lv[2] = x.z; lv[3] = x.w;
+        } else if constexpr (G == 2) {
+          const float2 x = __ldcg(reinterpret_cast<const float2*>(l));
+          lv[0] = x.x; lv[1] = x.y;
+        } else {
+          lv[0] = __ldcg(l);
+        }
+#pragma unroll
+        for (int g = 0; g < G; ++g) mass += exp2f(lv[g] - ls2[g]);
+      }
+      p.utility[base + t] = p.gamma * u_old + mass;
+    }
+  }
+}
+
+cudaError_t launch_utility(const UtilityParams& p, cudaStream_t stream) {
+  const long long U = (long long)p.B * p.Hkv;
+  if (U == 0 || p.Tmax == 0) return cudaSuccess;
+  if (p.Tmax > (1LL << 30)) return cudaErrorInvalidValue;
+  // about 2 waves of 256-thread blocks over all units, at least one block per unit
+  const long long per_unit = std::max<long long>(1, (148LL * 8 * 2 + U - 1) / U);
+  const long long bx = std::min<long long>((p.Tmax + 255) / 256, per_unit);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)bx, (unsigned)std::min<long long>(U, 65535));
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  switch (p.G) {
+    case 1: return cudaLaunchKernelEx(&cfg, utility_kernel<1>, p);
+    case 2: return cudaLaunchKernelEx(&cfg, utility_kernel<2>, p);
+    case 4: return cudaLaunchKernelEx(&cfg, utility_kernel<4>, p);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
 template <int G, bool DENSE>
 size_t decode_smem_fixed() {
   return ((sizeof(DecodeSmem<G, DENSE>) + 127) / 128) * 128;
@@ -1334,20 +1465,22 @@ size_t decode_smem_fixed() {
 template <int G, bool DENSE>
 cudaError_t launch_decode_g(const DecodeParams& p, cudaStream_t stream, cudaEvent_t between) {
   const size_t smem = (size_t)p.smem_bytes;
-  // The shared-memory opt-in is set once per device and size (outside any
-  // stream capture: the first call on a device is expected to be eager).
-  static size_t configured[64] = {};
+  // the logit-capturing variant when a logits buffer is given (ADA only)
+  const bool cap = !DENSE && p.logits != nullptr;
+  auto kern = cap ? decode_kernel<G, DENSE, !DENSE> : decode_kernel<G, DENSE, false>;
+  // The shared-memory opt-in is set once per device, variant and size
+  // (outside any stream capture: the first call is expected to be eager).
+  static size_t configured[2][64] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= 64 || configured[dev] < smem) {
-    e = cudaFuncSetAttribute(decode_kernel<G, DENSE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem);
+  if (dev < 0 || dev >= 64 || configured[cap][dev] < smem) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    if (dev >= 0 && dev < 64) configured[dev] = smem;
+    if (dev >= 0 && dev < 64) configured[cap][dev] = smem;
   }
   const int U = p.B * p.Hkv;
-  decode_kernel<G, DENSE><<<p.S, kDecodeThreads, p.smem_bytes, stream>>>(p);
+  kern<<<p.S, kDecodeThreads, p.smem_bytes, stream>>>(p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (between) {

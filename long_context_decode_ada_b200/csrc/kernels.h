@@ -24,6 +24,8 @@ struct DecodeParams {
   float* lse;
   int32_t* err;
   float* part;
+  float* logits;         // per-row log2-domain logits [rows][G], or NULL (no capture)
+  long long logit_rows;  // rows the logits buffer holds (page_cap * P)
   int S;
   int P;
   int log2P;
@@ -153,6 +155,23 @@ bool decode_smem_ok(int G, bool dense, int smem_bytes, int max_item);
 constexpr int kDecodeItemRows = 64;  // tokens per decode item
 cudaError_t launch_decode(const DecodeParams& p, int G, bool dense, cudaStream_t stream,
                           cudaEvent_t between);
+
+// Utility update from the captured logits and the merged lse of one decode.
+struct UtilityParams {
+  const float* logits;   // [rows][G] log2-domain logits written by the decode
+  long long logit_rows;
+  const float* lse;      // [B][Hq] natural-log lse of the decode
+  const int32_t* seq_lens;
+  const uint8_t* tier;   // [B][Hkv][Tmax]
+  const int32_t* row_of; // [B][Hkv][Tmax]
+  const int32_t* indptr; // [B*Hkv + 1]
+  int B, Hkv, G, P;
+  long long Tmax;
+  float gamma;
+  float* utility;        // [B][Hkv][Tmax] fp32, updated in place
+  int32_t* err;
+};
+cudaError_t launch_utility(const UtilityParams& p, cudaStream_t stream);
 cudaError_t launch_encode(const EncodeParams& p, cudaStream_t stream);
 cudaError_t launch_append(const AppendParams& p, cudaStream_t stream);
 size_t alloc_workspace_bytes(int B, int Hkv, long long Tmax);

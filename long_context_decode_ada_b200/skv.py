@@ -25,14 +25,15 @@ SKV_OK, SKV_ERR_ARG, SKV_ERR_BUDGET, SKV_ERR_POOL, SKV_ERR_CORRUPT, SKV_ERR_CUDA
 TIER_T0, TIER_T1, TIER_T2, TIER_DROP = range(4)
 MODE_QUOTA, MODE_BUDGET = 0, 1
 Q_FP16, Q_BF16 = 0, 1
-WS_ALLOCATE, WS_DECODE, WS_DENSE_DECODE, WS_APPEND = 0, 1, 2, 3
+WS_ALLOCATE, WS_DECODE, WS_DENSE_DECODE, WS_APPEND, WS_DECODE_UTILITY = 0, 1, 2, 3, 4
 TABLE_BOUNDARY6_X, TABLE_BOUNDARY6_Y, TABLE_BOUNDARY4_X, TABLE_BOUNDARY4_Y, TABLE_KAPPA, \
     TABLE_RHO_LEVELS = range(6)
 
 EXPORTS = [
     "skv_create", "skv_destroy", "skv_last_error", "skv_page_bytes", "skv_tables",
     "skv_device_info", "skv_workspace_size", "skv_allocate", "skv_encode", "skv_append",
-    "skv_decode_attention", "skv_decode_attention_static", "skv_dense_pack_bf16",
+    "skv_decode_attention", "skv_decode_attention_static", "skv_decode_utility",
+    "skv_dense_pack_bf16",
     "skv_dense_decode_bf16",
     "skv_set_profile_event", "skv_check",
 ]
@@ -65,6 +66,8 @@ _SIGS = {
                         _p]),
     "skv_append": (_i, [_p, _p, _p, _i, _i, _i64, _p, _p, _p, _p, _p, _p, _i64, C.POINTER(SkvPools),
                         _p, _i64, _p, _p, _p, _sz, _p]),
+    "skv_decode_utility": (_i, [_p, _p, _i, _i, _i, _i, _p, _p, _p, _i64, C.POINTER(SkvPools),
+                                _i64, _p, _p, _p, C.c_float, _p, _p, _p, _p, _p, _sz, _i, _p]),
     "skv_decode_attention": (_i, [_p, _p, _i, _i, _i, _i, _p, _p, _p, C.POINTER(SkvPools), _p, _p,
                                   _p, _p, _sz, _i, _p]),
     "skv_decode_attention_static": (_i, [_p, _p, _i, _i, _i, _i, _p, _p, _p,
@@ -269,6 +272,34 @@ class PagedCache:
             _ptr(self.page_tier_indptr) if self.split_by_bytes else None,
             _ptr(self.page_ids), C.byref(self._pools_c), _ptr(out), _ptr(lse), _ptr(self.err),
             _ptr(workspace), workspace.numel(), num_splits, _stream(stream)))
+        return out, lse
+
+    def utility_workspace(self, Hq: int, num_splits: int = 0) -> torch.Tensor:
+        n = self.ctx.workspace_size(WS_DECODE_UTILITY, self.B, self.Hkv, Hq, self.page_cap,
+                                    num_splits)
+        return torch.empty(max(n, 1), dtype=torch.uint8, device=self.device)
+
+    def decode_utility(self, q: torch.Tensor, q_dtype: int, Hq: int, seq_lens: torch.Tensor,
+                       utility: torch.Tensor, gamma: float = 1.0, out=None, lse=None,
+                       workspace=None, num_splits: int = 0, stream=None):
+        """decode() plus the utility update u <- gamma u + attention mass
+        (skv_decode_utility); utility is fp32 [B][Hkv][Tmax] on the device."""
+        if utility.dtype != torch.float32 or tuple(utility.shape) != (self.B, self.Hkv, self.Tmax) \
+                or not utility.is_contiguous():
+            raise SkvError(SKV_ERR_ARG, "utility must be contiguous fp32 [B][Hkv][Tmax]")
+        if out is None:
+            out = torch.empty((self.B, Hq, self.ctx.d), dtype=torch.float32, device=self.device)
+        if lse is None:
+            lse = torch.empty((self.B, Hq), dtype=torch.float32, device=self.device)
+        if workspace is None:
+            workspace = self.utility_workspace(Hq, num_splits)
+        _check(lib().skv_decode_utility(
+            self.ctx.handle, _ptr(q), q_dtype, self.B, Hq, self.Hkv, _ptr(self.page_indptr),
+            _ptr(self.page_tier_indptr) if self.split_by_bytes else None,
+            _ptr(self.page_ids), self.page_cap, C.byref(self._pools_c), self.Tmax,
+            _ptr(seq_lens), _ptr(self.tier), _ptr(self.row_of), float(gamma), _ptr(utility),
+            _ptr(out), _ptr(lse), _ptr(self.err), _ptr(workspace), workspace.numel(), num_splits,
+            _stream(stream)))
         return out, lse
 
     def decode_static(self, q: torch.Tensor, q_dtype: int, Hq: int, out=None, lse=None,

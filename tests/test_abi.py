@@ -92,3 +92,26 @@ def test_workspace_sizes():
     assert ctx.workspace_size(skv.WS_DECODE, 1, 8, 32, 0, 10) == expect(10, 8, 4)
     assert ctx.workspace_size(skv.WS_DECODE, 3, 3, 6, 0, 10) == expect(10, 9, 2)
     assert ctx.workspace_size(skv.WS_ALLOCATE, 2, 8, 0, 1000) > 2 * 8 * 1000 * 4
+    # the utility decode: the decode's scratch rounded up to 256 bytes, then
+    # page_cap * P rows x G fp32 logits
+    for B, Hkv, Hq, cap in [(1, 8, 32, 1000), (3, 3, 6, 7), (2, 4, 4, 0)]:
+        base = ctx.workspace_size(skv.WS_DECODE, B, Hkv, Hq, 0, 10)
+        n = ctx.workspace_size(skv.WS_DECODE_UTILITY, B, Hkv, Hq, cap, 10)
+        assert n == (base + 255) // 256 * 256 + cap * 64 * (Hq // Hkv) * 4
+
+
+def test_decode_utility_argument_errors_without_gpu():
+    ctx = skv.Context(16)
+    pools = skv.SkvPools()
+    L = skv.lib()
+    # Hq not a multiple of Hkv; then a null utility (refused before any launch)
+    rc = L.skv_decode_utility(ctx.handle, None, 0, 1, 6, 4, None, None, None, 10, C.byref(pools),
+                              8, None, None, None, 1.0, None, None, None, None, None, 0, 0, None)
+    assert rc == skv.SKV_ERR_ARG
+    rc = L.skv_decode_utility(ctx.handle, None, 0, 1, 8, 4, None, None, None, 10, C.byref(pools),
+                              8, None, None, None, 1.0, None, None, None, None, None, 0, 0, None)
+    assert rc == skv.SKV_ERR_ARG
+    # B = 0 is a no-op
+    rc = L.skv_decode_utility(ctx.handle, None, 0, 0, 8, 4, None, None, None, 10, C.byref(pools),
+                              8, None, None, None, 1.0, None, None, None, None, None, 0, 0, None)
+    assert rc == skv.SKV_OK
