@@ -428,7 +428,7 @@ def run_skv(args, rank, world, local_rank):
                                          out=out, lse=lse, workspace=uws[k], num_splits=S)
             return step
 
-        u_steps = 1000
+        u_steps = max(2, min(1000, args.steps))
         gu, gu_tail, gu_prof, evu, reps_u = timed_graph_steps(
             [make_ustep(0), make_ustep(1)], u_steps, 5, args.graph_steps, stream)
         ctx.set_profile_event(None)
