@@ -342,31 +342,24 @@ def run_skv(args, rank, world, local_rank):
         q_host = d["q"].cpu().pin_memory()
         out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
         lse_host = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
-        q_dev = torch.empty_like(d["q"])
+        scratch = (torch.empty_like(d["q"]), out, lse)
         e2e_steps = max(10, min(args.steps, 2000))
         for i in range(5):
-            q_dev.copy_(q_host, non_blocking=True)
-            caches[i % 2].decode(q_dev, d["q_dtype"], w.Hq, out=out, lse=lse, workspace=ws[i % 2],
-                                 num_splits=S)
-            out_host.copy_(out, non_blocking=True)
-            lse_host.copy_(lse, non_blocking=True)
-            stream.synchronize()
+            caches[i % 2].decode_host(q_host, d["q_dtype"], w.Hq, out_host, lse_host, scratch,
+                                      workspace=ws[i % 2], num_splits=S, stream=stream)
         ta = time.perf_counter()
         for i in range(e2e_steps):
-            q_dev.copy_(q_host, non_blocking=True)
-            caches[i % 2].decode(q_dev, d["q_dtype"], w.Hq, out=out, lse=lse, workspace=ws[i % 2],
-                                 num_splits=S)
-            out_host.copy_(out, non_blocking=True)
-            lse_host.copy_(lse, non_blocking=True)
-            stream.synchronize()
+            caches[i % 2].decode_host(q_host, d["q_dtype"], w.Hq, out_host, lse_host, scratch,
+                                      workspace=ws[i % 2], num_splits=S, stream=stream)
         e2e_ms = (time.perf_counter() - ta) * 1e3 / e2e_steps
         caches[0].check()
         e2e = {"value": world * resident / (e2e_ms * 1e-3), "unit": UNIT,
                "h2d_bytes_per_step": int(q_host.numel() * q_host.element_size()),
-               "d2h_bytes_per_step": int(out_host.numel() * 4 + lse_host.numel() * 4),
+               "d2h_bytes_per_step": int(out_host.numel() * 4 + lse_host.numel() * 4 + 4),
                "ms_per_step": e2e_ms, "steps": e2e_steps,
-               "how": "pinned host q -> device, skv_decode_attention, out+lse -> pinned host, "
-                      "stream sync every step; host wall clock"}
+               "how": "skv_decode_attention_host every step: pinned host q -> device, the "
+                      "decode, out + lse + error word -> pinned host, stream sync, in one C-ABI "
+                      "call; host wall clock"}
 
     # ---- dense bf16 paged-decode baseline on the same K/V
     dense = None

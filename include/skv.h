@@ -250,6 +250,28 @@ int skv_decode_attention(skv_ctx* ctx, const void* q, int q_dtype, int B, int Hq
                          const uint32_t* page_ids, const skv_pools* pools, float* out, float* lse, int32_t* err_word,
                          void* workspace, size_t ws_bytes, int num_splits, void* stream);
 
+/* skv_decode_attention_host -- one decode step from and to host memory
+   (an interface convenience of this library; the operation is that of
+   skv_decode_attention): copies q_host to q_dev, runs the decode, copies
+   out and lse back to out_host / lse_host, synchronises the stream and
+   returns the device error word's verdict as skv_check does (and resets
+   it).  Every copy is a single cudaMemcpyAsync on `stream`; use pinned
+   host buffers so that they are asynchronous DMA transfers.
+     q_host    [B][Hq][128] 16-bit host buffer (q_dtype as for the decode)
+     q_dev     device buffer of the same size (caller-owned scratch)
+     out_dev / lse_dev   device fp32 [B][Hq][128] / [B][Hq] scratch
+     out_host / lse_host host fp32 [B][Hq][128] / [B][Hq] results
+     other arguments as for skv_decode_attention (lse is required here)
+   Returns SKV_OK, an argument / CUDA error, or the device error the step
+   reported (SKV_ERR_CORRUPT, SKV_ERR_TIMEOUT).  Blocks the calling thread
+   until the step is done. */
+int skv_decode_attention_host(skv_ctx* ctx, const void* q_host, int q_dtype, int B, int Hq,
+                              int Hkv, const int32_t* page_indptr,
+                              const int32_t* page_tier_indptr, const uint32_t* page_ids,
+                              const skv_pools* pools, void* q_dev, float* out_dev, float* lse_dev,
+                              float* out_host, float* lse_host, int32_t* err_word,
+                              void* workspace, size_t ws_bytes, int num_splits, void* stream);
+
 /* skv_decode_utility -- the decode of skv_decode_attention plus the
    utility update that closes the retention loop.  The abstract's retention
    decides by "estimated future utility" without saying how it is estimated;

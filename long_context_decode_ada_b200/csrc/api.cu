@@ -29,6 +29,7 @@ struct skv_ctx {
   long long payload[4];
   long long stride[4];
   cudaEvent_t profile_event;
+  int32_t* err_host = nullptr;  // pinned word for skv_decode_attention_host (lazily allocated)
 };
 
 namespace {
@@ -165,6 +166,7 @@ int skv_create(const skv_config* cfg, skv_ctx** out) {
 }
 
 int skv_destroy(skv_ctx* ctx) {
+  if (ctx && ctx->err_host) cudaFreeHost(ctx->err_host);
   delete ctx;
   return ok();
 }
@@ -476,6 +478,50 @@ int skv_decode_attention(skv_ctx* ctx, const void* q, int q_dtype, int B, int Hq
                        slots, false, out,
                        lse, err_word, workspace, ws_bytes, num_splits, stream,
                        "skv_decode_attention");
+}
+
+int skv_decode_attention_host(skv_ctx* ctx, const void* q_host, int q_dtype, int B, int Hq,
+                              int Hkv, const int32_t* page_indptr,
+                              const int32_t* page_tier_indptr, const uint32_t* page_ids,
+                              const skv_pools* pools, void* q_dev, float* out_dev, float* lse_dev,
+                              float* out_host, float* lse_host, int32_t* err_word,
+                              void* workspace, size_t ws_bytes, int num_splits, void* stream) {
+  static const char* name = "skv_decode_attention_host";
+  if (!ctx) return fail(SKV_ERR_ARG, "%s: null ctx", name);
+  if (B < 0 || Hkv <= 0 || Hq <= 0 || Hq % Hkv != 0)
+    return fail(SKV_ERR_ARG, "%s: need B >= 0 and Hq a multiple of Hkv", name);
+  if (B == 0) return ok();
+  if (!q_host || !q_dev || !out_dev || !lse_dev || !out_host || !lse_host || !err_word)
+    return fail(SKV_ERR_ARG, "%s: null argument", name);
+  if (!valid_pools(pools, 3)) return fail(SKV_ERR_ARG, "%s: bad pools", name);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaSuccess;
+  if (!ctx->err_host) {
+    e = cudaMallocHost(&ctx->err_host, sizeof(int32_t));
+    if (e != cudaSuccess) return cuda_fail(e, "skv_decode_attention_host: pinned error word");
+    *ctx->err_host = 0;
+  }
+  const size_t qn = (size_t)B * Hq * 128 * 2, on = (size_t)B * Hq * 128 * 4, ln = (size_t)B * Hq * 4;
+  e = cudaMemcpyAsync(q_dev, q_host, qn, cudaMemcpyHostToDevice, s);
+  if (e != cudaSuccess) return cuda_fail(e, "skv_decode_attention_host: copy of q");
+  const void* pool[3] = {pools->base[0], pools->base[1], pools->base[2]};
+  const long long slots[3] = {pools->slots[0], pools->slots[1], pools->slots[2]};
+  int rc = decode_common(ctx, q_dev, q_dtype, B, Hq, Hkv, page_indptr, page_tier_indptr, page_ids,
+                         pool, slots, false, out_dev, lse_dev, err_word, workspace, ws_bytes,
+                         num_splits, stream, name);
+  if (rc != SKV_OK) return rc;
+  e = cudaMemcpyAsync(out_host, out_dev, on, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(lse_host, lse_dev, ln, cudaMemcpyDeviceToHost, s);
+  // the error word rides along with the results, and is reset on the stream
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(ctx->err_host, err_word, sizeof(int32_t), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(err_word, 0, sizeof(int32_t), s);
+  if (e != cudaSuccess) return cuda_fail(e, "skv_decode_attention_host: copy of the results");
+  e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "skv_decode_attention_host: stream synchronize");
+  const int32_t v = *ctx->err_host;
+  if (v != 0) return fail(v, "%s: device reported error %d", name, v);
+  return ok();
 }
 
 int skv_decode_utility(skv_ctx* ctx, const void* q, int q_dtype, int B, int Hq, int Hkv,

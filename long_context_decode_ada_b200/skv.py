@@ -32,7 +32,8 @@ TABLE_BOUNDARY6_X, TABLE_BOUNDARY6_Y, TABLE_BOUNDARY4_X, TABLE_BOUNDARY4_Y, TABL
 EXPORTS = [
     "skv_create", "skv_destroy", "skv_last_error", "skv_page_bytes", "skv_tables",
     "skv_device_info", "skv_workspace_size", "skv_allocate", "skv_encode", "skv_append",
-    "skv_decode_attention", "skv_decode_attention_static", "skv_decode_utility",
+    "skv_decode_attention", "skv_decode_attention_static", "skv_decode_attention_host",
+    "skv_decode_utility",
     "skv_dense_pack_bf16",
     "skv_dense_decode_bf16",
     "skv_set_profile_event", "skv_check",
@@ -66,6 +67,8 @@ _SIGS = {
                         _p]),
     "skv_append": (_i, [_p, _p, _p, _i, _i, _i64, _p, _p, _p, _p, _p, _p, _i64, C.POINTER(SkvPools),
                         _p, _i64, _p, _p, _p, _sz, _p]),
+    "skv_decode_attention_host": (_i, [_p, _p, _i, _i, _i, _i, _p, _p, _p, C.POINTER(SkvPools),
+                                       _p, _p, _p, _p, _p, _p, _p, _sz, _i, _p]),
     "skv_decode_utility": (_i, [_p, _p, _i, _i, _i, _i, _p, _p, _p, _i64, C.POINTER(SkvPools),
                                 _i64, _p, _p, _p, C.c_float, _p, _p, _p, _p, _p, _sz, _i, _p]),
     "skv_decode_attention": (_i, [_p, _p, _i, _i, _i, _i, _p, _p, _p, C.POINTER(SkvPools), _p, _p,
@@ -301,6 +304,29 @@ class PagedCache:
             _ptr(out), _ptr(lse), _ptr(self.err), _ptr(workspace), workspace.numel(), num_splits,
             _stream(stream)))
         return out, lse
+
+    def decode_host(self, q_host: torch.Tensor, q_dtype: int, Hq: int, out_host: torch.Tensor,
+                    lse_host: torch.Tensor, scratch, workspace=None, num_splits: int = 0,
+                    stream=None):
+        """One decode step from host q to host out / lse (skv_decode_attention_host):
+        the copies, the decode and the stream synchronisation in one call.
+        scratch = (q_dev, out_dev, lse_dev) device tensors; host tensors
+        should be pinned."""
+        q_dev, out_dev, lse_dev = scratch
+        for t, dev_side in ((q_host, False), (out_host, False), (lse_host, False),
+                            (q_dev, True), (out_dev, True), (lse_dev, True)):
+            if t.is_cuda != dev_side or not t.is_contiguous():
+                raise SkvError(SKV_ERR_ARG, "decode_host: host tensors on the host, scratch on "
+                                            "the device, all contiguous")
+        if workspace is None:
+            workspace = self.workspace(Hq, num_splits)
+        _check(lib().skv_decode_attention_host(
+            self.ctx.handle, _ptr(q_host), q_dtype, self.B, Hq, self.Hkv, _ptr(self.page_indptr),
+            _ptr(self.page_tier_indptr) if self.split_by_bytes else None,
+            _ptr(self.page_ids), C.byref(self._pools_c), _ptr(q_dev), _ptr(out_dev),
+            _ptr(lse_dev), _ptr(out_host), _ptr(lse_host), _ptr(self.err), _ptr(workspace),
+            workspace.numel(), num_splits, _stream(stream)))
+        return out_host, lse_host
 
     def decode_static(self, q: torch.Tensor, q_dtype: int, Hq: int, out=None, lse=None,
                       num_splits: int = 0, stream=None):
