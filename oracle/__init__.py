@@ -329,6 +329,31 @@ def accumulate_utility(utility, mass, seq_lens, gamma: float) -> np.ndarray:
     return u
 
 
+def merge_partials(out_parts, lse_parts):
+    """Log-sum-exp merge of R attention partials over disjoint token sets, in
+    fp64: out_parts [R][...][d], lse_parts [R][...] -> (out [...][d], lse
+    [...]).  With M = max_r lse_r and w_r = exp(lse_r - M):
+        out = sum_r w_r out_r / sum_r w_r,   lse = M + log sum_r w_r.
+    Softmax over the union of the token sets factors this way because each
+    partial's out is its own normalised weighted sum and exp(lse_r) its
+    denominator.  Partials with lse = -inf (no resident token) carry no
+    weight; when every partial is empty the result is out 0, lse -inf, as the
+    decode gives for an empty unit."""
+    o = np.asarray(out_parts, np.float64)
+    l = np.asarray(lse_parts, np.float64)
+    M = l.max(axis=0)
+    live = np.isfinite(M)
+    Ms = np.where(live, M, 0.0)
+    w = np.where(np.isfinite(l), np.exp(l - Ms[None]), 0.0)
+    den = w.sum(axis=0)
+    out = np.zeros(o.shape[1:], np.float64)
+    num = (w[..., None] * np.where(np.isfinite(l)[..., None], o, 0.0)).sum(axis=0)
+    out[live] = num[live] / den[live][..., None]
+    lse = np.full(l.shape[1:], -np.inf)
+    lse[live] = Ms[live] + np.log(den[live])
+    return out, lse
+
+
 def run_workload(w, units=None, do_decode=True):
     """allocate -> pack -> decode on a workloads.Workload; returns a dict."""
     tier = allocate(w.B, w.Hkv, w.Tmax, w.d, w.P, w.seq_lens, w.K, w.utility, w.protect,
