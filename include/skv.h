@@ -272,6 +272,29 @@ int skv_decode_attention_host(skv_ctx* ctx, const void* q_host, int q_dtype, int
                               float* out_host, float* lse_host, int32_t* err_word,
                               void* workspace, size_t ws_bytes, int num_splits, void* stream);
 
+/* skv_merge_partials -- the exchange step of a context-parallel decode.
+   Each of R ranks attends (skv_decode_attention) over its own slice of every
+   sequence's tokens; softmax over the union of disjoint slices factors into
+   the slices' normalised outputs weighted by their denominators:
+     M = max_r lse_r,  w_r = exp(lse_r - M),
+     out = sum_r w_r out_r / sum_r w_r,   lse = M + log sum_r w_r
+   (partials with lse = -inf carry no weight; all empty gives out 0 and lse
+   -inf, as the decode gives for an empty unit).  The pages fix attention over
+   all resident tokens (technical summary 2.1); splitting it by slices is
+   this library's multi-GPU layout, not the paper's.
+     n            rows (B * Hq)
+     out_parts    fp32 device, rank r's out [n][128] at out_parts + r*rank_stride
+     lse_parts    fp32 device, rank r's lse [n] at lse_parts + r*rank_stride
+     rank_stride  floats between ranks (both arrays); e.g. a packed all-gather
+                  buffer of R blocks {out [n][128], lse [n], one pad float when
+                  n is odd} has out_parts = buf, lse_parts = buf + 128 n,
+                  rank_stride = 129 n + (n & 1)
+     out, lse     fp32 device [n][128] and [n] (lse may be NULL)
+   out_parts, out and rank_stride must be 8-byte aligned (float2 loads). */
+int skv_merge_partials(skv_ctx* ctx, int R, int64_t n, const float* out_parts,
+                       const float* lse_parts, int64_t rank_stride, float* out, float* lse,
+                       void* stream);
+
 /* skv_decode_utility -- the decode of skv_decode_attention plus the
    utility update that closes the retention loop.  The abstract's retention
    decides by "estimated future utility" without saying how it is estimated;

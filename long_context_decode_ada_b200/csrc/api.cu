@@ -524,6 +524,25 @@ int skv_decode_attention_host(skv_ctx* ctx, const void* q_host, int q_dtype, int
   return ok();
 }
 
+int skv_merge_partials(skv_ctx* ctx, int R, int64_t n, const float* out_parts,
+                       const float* lse_parts, int64_t rank_stride, float* out, float* lse,
+                       void* stream) {
+  static const char* name = "skv_merge_partials";
+  if (!ctx) return fail(SKV_ERR_ARG, "%s: null ctx", name);
+  if (R <= 0 || n < 0 || n > 0x7FFFFFFFLL)
+    return fail(SKV_ERR_ARG, "%s: need R > 0 and 0 <= n < 2^31", name);
+  if (n == 0) return ok();
+  if (!out_parts || !lse_parts || !out) return fail(SKV_ERR_ARG, "%s: null argument", name);
+  if (R > 1 && rank_stride < n) return fail(SKV_ERR_ARG, "%s: rank_stride < n", name);
+  if ((reinterpret_cast<uintptr_t>(out_parts) & 7) || (reinterpret_cast<uintptr_t>(out) & 7) ||
+      (rank_stride & 1))
+    return fail(SKV_ERR_ARG, "%s: out_parts, out and rank_stride must be 8-byte aligned", name);
+  cudaError_t e = skv::launch_merge_partials(R, n, out_parts, lse_parts, rank_stride, out, lse,
+                                             static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, name);
+  return ok();
+}
+
 int skv_decode_utility(skv_ctx* ctx, const void* q, int q_dtype, int B, int Hq, int Hkv,
                        const int32_t* page_indptr, const int32_t* page_tier_indptr,
                        const uint32_t* page_ids, int64_t page_cap, const skv_pools* pools,

@@ -1457,6 +1457,50 @@ cudaError_t launch_utility(const UtilityParams& p, cudaStream_t stream) {
   }
 }
 
+// Context-parallel combine: rank r attended over its own slice of every
+// sequence's tokens and produced (out_r, lse_r) per (sequence, query head);
+// the softmax over the union of the slices is out = sum_r w_r out_r /
+// sum_r w_r, lse = M + log sum_r w_r with w_r = exp(lse_r - M), M the largest
+// lse_r.  Empty partials (lse -inf) carry no weight; all empty: out 0,
+// lse -inf.  One block of 64 threads per row, a float2 of out per thread.
+__global__ void __launch_bounds__(64) merge_partials_kernel(int R, long long n,
+                                                            const float* __restrict__ out_parts,
+                                                            const float* __restrict__ lse_parts,
+                                                            long long rank_stride,
+                                                            float* __restrict__ out,
+                                                            float* __restrict__ lse) {
+  const long long row = blockIdx.x;
+  const int j = threadIdx.x;
+  float M = -INFINITY;
+  for (int r = 0; r < R; ++r) M = fmaxf(M, __ldg(lse_parts + r * rank_stride + row));
+  float L = 0.0f, ox = 0.0f, oy = 0.0f;
+  if (M != -INFINITY) {
+    for (int r = 0; r < R; ++r) {
+      const float lr = __ldg(lse_parts + r * rank_stride + row);
+      if (lr == -INFINITY) continue;  // an empty partial's out is never read
+      const float w = expf(lr - M);
+      const float2 o = __ldg(reinterpret_cast<const float2*>(out_parts + r * rank_stride +
+                                                             row * kHeadDim) + j);
+      L += w;
+      ox = fmaf(w, o.x, ox);
+      oy = fmaf(w, o.y, oy);
+    }
+  }
+  float2* dst = reinterpret_cast<float2*>(out + row * kHeadDim) + j;
+  *dst = L > 0.0f ? make_float2(ox / L, oy / L) : make_float2(0.0f, 0.0f);
+  if (j == 0 && lse) lse[row] = L > 0.0f ? M + logf(L) : -INFINITY;
+}
+
+cudaError_t launch_merge_partials(int R, long long n, const float* out_parts,
+                                  const float* lse_parts, long long rank_stride, float* out,
+                                  float* lse, cudaStream_t stream) {
+  if (n <= 0) return cudaSuccess;
+  if (R <= 0 || n > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
+  merge_partials_kernel<<<(unsigned)n, kHeadDim / 2, 0, stream>>>(R, n, out_parts, lse_parts,
+                                                                  rank_stride, out, lse);
+  return cudaGetLastError();
+}
+
 template <int G, bool DENSE>
 size_t decode_smem_fixed() {
   return ((sizeof(DecodeSmem<G, DENSE>) + 127) / 128) * 128;

@@ -172,6 +172,11 @@ struct UtilityParams {
   int32_t* err;
 };
 cudaError_t launch_utility(const UtilityParams& p, cudaStream_t stream);
+
+// Log-sum-exp merge of R attention partials per (sequence, query head).
+cudaError_t launch_merge_partials(int R, long long n, const float* out_parts,
+                                  const float* lse_parts, long long rank_stride, float* out,
+                                  float* lse, cudaStream_t stream);
 cudaError_t launch_encode(const EncodeParams& p, cudaStream_t stream);
 cudaError_t launch_append(const AppendParams& p, cudaStream_t stream);
 size_t alloc_workspace_bytes(int B, int Hkv, long long Tmax);

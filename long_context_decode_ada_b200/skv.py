@@ -33,7 +33,7 @@ EXPORTS = [
     "skv_create", "skv_destroy", "skv_last_error", "skv_page_bytes", "skv_tables",
     "skv_device_info", "skv_workspace_size", "skv_allocate", "skv_encode", "skv_append",
     "skv_decode_attention", "skv_decode_attention_static", "skv_decode_attention_host",
-    "skv_decode_utility",
+    "skv_decode_utility", "skv_merge_partials",
     "skv_dense_pack_bf16",
     "skv_dense_decode_bf16",
     "skv_set_profile_event", "skv_check",
@@ -69,6 +69,7 @@ _SIGS = {
                         _p, _i64, _p, _p, _p, _sz, _p]),
     "skv_decode_attention_host": (_i, [_p, _p, _i, _i, _i, _i, _p, _p, _p, C.POINTER(SkvPools),
                                        _p, _p, _p, _p, _p, _p, _p, _sz, _i, _p]),
+    "skv_merge_partials": (_i, [_p, _i, _i64, _p, _p, _i64, _p, _p, _p]),
     "skv_decode_utility": (_i, [_p, _p, _i, _i, _i, _i, _p, _p, _p, _i64, C.POINTER(SkvPools),
                                 _i64, _p, _p, _p, C.c_float, _p, _p, _p, _p, _p, _sz, _i, _p]),
     "skv_decode_attention": (_i, [_p, _p, _i, _i, _i, _i, _p, _p, _p, C.POINTER(SkvPools), _p, _p,
