@@ -54,6 +54,9 @@ def parse_args():
     ap.add_argument("--no-append", action="store_true", help="skip the skv_append timing")
     ap.add_argument("--no-utility", action="store_true",
                     help="skip the skv_decode_utility timing")
+    ap.add_argument("--cp", action="store_true",
+                    help="context-parallel decode: the ranks share one sequence, each "
+                         "holding a slice of its positions (strong scaling)")
     ap.add_argument("--graph-steps", type=int, default=100)
     ap.add_argument("--seed", type=int, default=0)
     return ap.parse_args()
@@ -622,6 +625,94 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def run_cp(args, rank, world, local_rank):
+    """Context-parallel decode of one 128K sequence over the ranks: rank r
+    holds slice r of its positions (its own allocate + encode), a step is
+    the local decode, the all-gather of the packed partials and the merge.
+    Enough copies of each slice's store rotate that the inputs of
+    consecutive steps exceed L2."""
+    from long_context_decode_ada_b200 import cp, skv
+    from long_context_decode_ada_b200 import workloads as wl
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    T = args.seq_len
+    w = wl.long_context(seed=args.seed, T=T)          # the same sequence on every rank
+    ws = cp.slice_workload(w, world, rank)
+    ctx = skv.Context(w.P)
+    d = skv.workload_to_device(ws, dev)
+    first = skv.build_cache(ctx, ws, d)
+    first.check()
+    store_bytes = sum(int(p.numel()) for p in first.pools)
+    n_copies = max(2, -(-300_000_000 // max(store_bytes, 1)) + 1)
+    caches = [first] + [clone_cache(first) for _ in range(n_copies - 1)]
+    del d["K"], d["V"]
+    torch.cuda.empty_cache()
+    S = args.num_splits
+    decs = [cp.ContextParallelDecoder(c, w.Hq, num_splits=S) for c in caches]
+    resident = int((first.tier != 3).sum().item())
+    total = torch.tensor([resident], dtype=torch.int64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(total)
+    total = int(total.item())
+    stream = torch.cuda.current_stream()
+
+    def make_step(k):
+        def step(mid_event):
+            ctx.set_profile_event(mid_event)
+            decs[k].step(d["q"], d["q_dtype"])   # on the current (capturing) stream
+        return step
+
+    g, g_tail, g_prof, ev, reps = timed_graph_steps(
+        [make_step(k) for k in range(n_copies)], args.steps, args.warmup,
+        min(args.graph_steps, 10 * n_copies), stream)
+    ctx.set_profile_event(None)
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    time.sleep(0.3)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(reps):
+        g.replay()
+    if g_tail is not None:
+        g_tail.replay()
+    t1.record()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = sampler.stop()
+    ms_per_step = max_over_ranks(t0.elapsed_time(t1), dev) / args.steps
+    g_prof.replay()
+    torch.cuda.synchronize()
+    first.check()
+    kern = float(np.mean([a.elapsed_time(b) for a, b, c in ev]))
+    rest = float(np.mean([b.elapsed_time(c) for a, b, c in ev]))
+    del g, g_tail, g_prof      # graphs holding NCCL calls go before the process group
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": total / (ms_per_step * 1e-3),
+            "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "strong",
+            "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+            "config": {"workload": workload_desc(T) + f", context-parallel over {world} ranks "
+                                                       f"(slices of {ws.Tmax} positions)",
+                       "parallelism": f"cp{world}", "num_splits": S or "default",
+                       "l2": f"{n_copies} rotating copies of each rank's "
+                             f"{store_bytes / 1e6:.0f} MB store",
+                       "resident_tokens_heads": total},
+            "cp": {"local_decode_kernel_us": kern * 1e3,
+                   "exchange_and_merge_us": rest * 1e3,
+                   "how": "graph replays of decode + all-gather + merge steps; the profile "
+                          "graph's events split rank 0's local decode kernel from the rest"},
+            "gpu_launches": 3 * args.steps,   # decode, its merge, the partials' merge
+            "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -635,7 +726,10 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                              device_id=torch.device("cuda", local_rank))
     try:
-        run_skv(args, rank, world, local_rank)
+        if args.cp:
+            run_cp(args, rank, world, local_rank)
+        else:
+            run_skv(args, rank, world, local_rank)
     finally:
         if world > 1:
             torch.distributed.destroy_process_group()

@@ -95,7 +95,10 @@ def slice_workload(w: wl.Workload, R: int, r: int, align: Optional[int] = None) 
 
 
 def gather_partials(part: torch.Tensor, group=None) -> torch.Tensor:
-    """All-gather of every rank's packed partial buffer: [R][len]."""
+    """All-gather of every rank's packed partial buffer: [R][len].  Without a
+    process group (or with one rank) there is nothing to exchange."""
+    if not dist.is_initialized() or dist.get_world_size(group) == 1:
+        return part.view(1, -1)
     R = dist.get_world_size(group)
     out = torch.empty((R, part.numel()), dtype=part.dtype, device=part.device)
     if dist.get_backend(group) == "nccl":
