@@ -72,6 +72,8 @@ _SIGS = {
                       _p, _p, _p, _p]),                       # pool0..2 pool_slots
     "orc_decode": (_i, [_i, _i, _i, _i, _i, _p, _p, _p, _p, _p, _i, _p, _p, _p, _i]),
     "orc_attention_mass": (_i, [_i, _i, _i, _i, _i, _p, _p, _p, _p, _i, _p]),
+    "orc_outlier": (_i, [_p, _i]),
+    "orc_outlier_flags": (_i, [_i, _i, _i, _i, _p, _p, _p]),
     "orc_d2h": (_u16, [_d]),
     "orc_h2d": (_d, [_u16]),
     "orc_bf2d": (_d, [_u16]),
@@ -311,6 +313,24 @@ def attention_mass(B, Hq, Hkv, Tmax, d, seq_lens, K, tier, q, q_dtype: str) -> n
     if rc != OK:
         raise OracleError(rc, "attention_mass")
     return mass
+
+
+def outlier(k16) -> bool:
+    """Whether one pair of the key holds a share beyond twice the share
+    grid's top level (u_i = (rho_i / r) sqrt(d/2) > 4)."""
+    k = _u16(k16)
+    return bool(lib().orc_outlier(_ptr(k), k.size))
+
+
+def outlier_flags(B, Hkv, Tmax, d, seq_lens, K) -> np.ndarray:
+    """uint8 [B][Hkv][Tmax]: outlier() of every resident position, else 0."""
+    seq = np.ascontiguousarray(seq_lens, np.int32)
+    k = _u16(K)
+    flags = np.zeros((B, Hkv, Tmax), np.uint8)
+    rc = lib().orc_outlier_flags(B, Hkv, Tmax, d, _ptr(seq), _ptr(k), _ptr(flags))
+    if rc != OK:
+        raise OracleError(rc, "outlier_flags")
+    return flags
 
 
 def accumulate_utility(utility, mass, seq_lens, gamma: float) -> np.ndarray:

@@ -783,6 +783,40 @@ int orc_decode(int B, int Hq, int Hkv, int Tmax, int d, const int32_t* seq_lens,
     return bad ? ORC_ERR_ARG : ORC_OK;
 }
 
+/* Outlier flag of a key, for the protection constraint [TS 2.2] (outliers
+   are among the states kept at the top tier).  READING: a key is an
+   outlier when one of its pairs holds a share far beyond the 2-bit share
+   grid: u_i = (rho_i / r) sqrt(d/2) > 4, twice the top level u = 2, where
+   the decoded share is under half of the pair's true one.  For Gaussian
+   keys u^2 is about Exp(1), so this flags about one key in 10^5 at d = 128;
+   a channel scaled up twentyfold flags every key.  Exact integer test:
+   (d/2) rho_i^2 > 16 R2; a tie is not an outlier. */
+int orc_outlier(const uint16_t* k, int d) {
+    uint64_t R2[2];
+    orc_norm2(k, d, R2);
+    u128 R = ((u128)R2[1] << 64) | R2[0];
+    for (int i = 0; i < d / 2; i++) {
+        int64_t mx = h2m(k[2 * i]), my = h2m(k[2 * i + 1]);
+        u128 ax = (u128)(mx < 0 ? -mx : mx), ay = (u128)(my < 0 ? -my : my);
+        u128 rho2 = ax * ax + ay * ay;
+        if (rho2 * (u128)(d / 2) > (u128)16 * R) return 1;
+    }
+    return 0;
+}
+
+/* flags[b][h][t] = orc_outlier(K[b][h][t]) for t < seq_lens[b], else 0 */
+int orc_outlier_flags(int B, int Hkv, int Tmax, int d, const int32_t* seq_lens,
+                      const uint16_t* K, uint8_t* flags) {
+    if (B < 0 || Hkv <= 0 || Tmax < 0 || d <= 0 || (d & 1)) return ORC_ERR_ARG;
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < (int64_t)B * Hkv * Tmax; i++) {
+        int b = (int)(i / ((int64_t)Hkv * Tmax));
+        int64_t t = i % Tmax;
+        flags[i] = t < seq_lens[b] ? (uint8_t)orc_outlier(K + i * d, d) : 0;
+    }
+    return ORC_OK;
+}
+
 /* Attention mass per resident token, the decode-side utility signal.
    READING: [ABS] drives retention by an "estimated future utility" without
    saying how it is estimated; the plainest estimator the decode supplies is
