@@ -75,7 +75,12 @@ extern "C" {
 typedef struct skv_config {
   int32_t head_dim;    /* d: 128 */
   int32_t page_size;   /* P: 16, 32 or 64 */
-  int32_t reserved[6]; /* zero */
+  int32_t outlier_protect; /* nonzero: skv_allocate also protects (keeps at T0)
+                          every key with a pair whose share lies beyond twice
+                          the share grid's top level, u = (rho/r) sqrt(d/2) > 4
+                          (technical summary 2.2: outliers are among the
+                          protected states) */
+  int32_t reserved[5]; /* zero */
 } skv_config;
 
 /* Device pools of page slots, one per tier.  Slot s of tier t starts at

@@ -35,6 +35,7 @@ size_t alloc_workspace_bytes(int B, int Hkv, long long Tmax) {
   n += al256(4 * U * 3);
   n += al256(4 * U * 3);
   n += al256(8 * (size_t)B);
+  n += al256(U * (size_t)Tmax);
   return n;
 }
 
@@ -53,9 +54,50 @@ void alloc_carve(AllocParams& p, void* ws) {
   p.tbase = reinterpret_cast<int32_t*>(w);
   w += al256(4 * U * 3);
   p.nprot = reinterpret_cast<long long*>(w);
+  w += al256(8 * (size_t)p.B);
+  p.eff_protect = w;
 }
 
 // ---------------------------------------------------------------- keys --
+
+// Outlier-aware protection: one warp per token; lane l holds dims 4l .. 4l+3
+// (pairs 2l, 2l+1).  A key is an outlier when some pair has
+// u = (rho / r) sqrt(d/2) > 4, twice the share grid's top level, tested
+// exactly on the fp16 integers: (d/2) rho^2 > 16 R2.  The flag joins the
+// caller's protection mask in eff_protect, which the key kernels then read.
+__global__ void __launch_bounds__(256) outlier_protect_kernel(const __grid_constant__ AllocParams p) {
+  const long long w = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (w >= (long long)p.B * p.Hkv * p.Tmax) return;
+  const long long t = w % p.Tmax;
+  const int b = (int)(w / p.Tmax / p.Hkv);
+  bool flag = false;
+  if (t < p.seq_lens[b]) {  // uniform across the warp
+    const uint2 kv = *reinterpret_cast<const uint2*>(p.K + w * kHeadDim + 4 * lane);
+    const uint16_t k4[4] = {(uint16_t)(kv.x & 0xFFFF), (uint16_t)(kv.x >> 16),
+                            (uint16_t)(kv.y & 0xFFFF), (uint16_t)(kv.y >> 16)};
+    u128 a[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const long long m = half_bits_to_m(k4[i]);
+      a[i] = (u128)(m < 0 ? -m : m);
+    }
+    const u128 pr0 = a[0] * a[0] + a[1] * a[1], pr1 = a[2] * a[2] + a[3] * a[3];
+    u128 sq = pr0 + pr1;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const unsigned long long lo = (unsigned long long)sq, hi = (unsigned long long)(sq >> 64);
+      const unsigned long long olo = __shfl_xor_sync(0xFFFFFFFFu, lo, o);
+      const unsigned long long ohi = __shfl_xor_sync(0xFFFFFFFFu, hi, o);
+      sq += ((u128)ohi << 64) | olo;
+    }
+    const u128 lim = (u128)16 * sq;
+    constexpr unsigned kHalfD = kHeadDim / 2;
+    flag = __any_sync(0xFFFFFFFFu, pr0 * kHalfD > lim || pr1 * kHalfD > lim);
+  }
+  if (lane == 0)
+    p.eff_protect[w] = (uint8_t)(((p.protect != nullptr && p.protect[w] != 0) || flag) ? 1 : 0);
+}
 
 __device__ __forceinline__ float valid_utility(const AllocParams& p, long long i) {
   if (!p.utility) return 0.0f;
@@ -462,6 +504,11 @@ cudaError_t launch_allocate(AllocParams& p, cudaStream_t stream) {
   if ((e = cudaMemsetAsync(p.nprot, 0, 8 * (size_t)p.B, stream)) != cudaSuccess) return e;
   if ((e = cudaMemsetAsync(p.hist, 0, 8 * (size_t)p.nseg * 3 * 256, stream)) != cudaSuccess)
     return e;
+  if (p.outlier && ntok > 0) {
+    outlier_protect_kernel<<<grid_for(ntok * 32, 256), 256, 0, stream>>>(p);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    p.protect = p.eff_protect;  // the key kernels read the joined mask
+  }
   if (ntok > 0) {
     if (p.mode == SKV_MODE_BUDGET)
       keys_budget_kernel<<<grid_for(ntok * 32, 256), 256, 0, stream>>>(p);

@@ -30,6 +30,7 @@ struct skv_ctx {
   long long stride[4];
   cudaEvent_t profile_event;
   int32_t* err_host = nullptr;  // pinned word for skv_decode_attention_host (lazily allocated)
+  int outlier_protect = 0;      // skv_config.outlier_protect
 };
 
 namespace {
@@ -118,6 +119,7 @@ int skv_create(const skv_config* cfg, skv_ctx** out) {
   if (!c) return fail(SKV_ERR_ARG, "out of host memory");
   c->d = 128;
   c->P = P;
+  c->outlier_protect = cfg->outlier_protect != 0;
   c->log2P = P == 16 ? 4 : (P == 32 ? 5 : 6);
   c->device = 0;
   c->profile_event = nullptr;
@@ -255,6 +257,7 @@ static int fill_alloc_common(skv::AllocParams& p, const skv_ctx* ctx, int B, int
   p.Hkv = Hkv;
   p.Tmax = Tmax;
   p.P = ctx->P;
+  p.outlier = ctx->outlier_protect;
   for (int k = 0; k < 3; ++k) p.kappa[k] = ctx->kappa[k];
   return SKV_OK;
 }

@@ -133,6 +133,8 @@ struct AllocParams {
   long long* nprot;           // [B]
   int nseg;
   int dense;                  // dense-bf16 baseline packing (every token kept, tier 0)
+  int outlier;                // outlier-aware protection on
+  uint8_t* eff_protect;       // [B*Hkv*Tmax]: protect | outlier flag (workspace)
 };
 
 // Decode workspace: partials [(S + U) G][kPartStride] fp32, then per unit the

@@ -41,7 +41,8 @@ EXPORTS = [
 
 
 class SkvConfig(C.Structure):
-    _fields_ = [("head_dim", C.c_int32), ("page_size", C.c_int32), ("reserved", C.c_int32 * 6)]
+    _fields_ = [("head_dim", C.c_int32), ("page_size", C.c_int32),
+                ("outlier_protect", C.c_int32), ("reserved", C.c_int32 * 5)]
 
 
 class SkvPools(C.Structure):
@@ -134,13 +135,15 @@ def _stream(stream=None):
 class Context:
     """An skv_ctx: head_dim 128, page size P; bound to the current device."""
 
-    def __init__(self, page_size: int, head_dim: int = 128):
-        cfg = SkvConfig(head_dim=head_dim, page_size=page_size)
+    def __init__(self, page_size: int, head_dim: int = 128, outlier_protect: bool = False):
+        cfg = SkvConfig(head_dim=head_dim, page_size=page_size,
+                        outlier_protect=1 if outlier_protect else 0)
         h = C.c_void_p()
         _check(lib().skv_create(C.byref(cfg), C.byref(h)))
         self._h = h
         self.P = page_size
         self.d = head_dim
+        self.outlier_protect = bool(outlier_protect)
 
     def __del__(self):
         h = getattr(self, "_h", None)
