@@ -73,6 +73,7 @@ _SIGS = {
     "orc_decode": (_i, [_i, _i, _i, _i, _i, _p, _p, _p, _p, _p, _i, _p, _p, _p, _i]),
     "orc_attention_mass": (_i, [_i, _i, _i, _i, _i, _p, _p, _p, _p, _i, _p]),
     "orc_outlier": (_i, [_p, _i]),
+    "orc_logit_grid": (_d, [_p, _p, _i, _i, _i, _p, _p]),
     "orc_outlier_flags": (_i, [_i, _i, _i, _i, _p, _p, _p]),
     "orc_d2h": (_u16, [_d]),
     "orc_h2d": (_d, [_u16]),
@@ -313,6 +314,20 @@ def attention_mass(B, Hq, Hkv, Tmax, d, seq_lens, K, tier, q, q_dtype: str) -> n
     if rc != OK:
         raise OracleError(rc, "attention_mass")
     return mass
+
+
+def logit_grid(q: np.ndarray, k16, b: int, levels_u=None, thresh_u=None) -> float:
+    """Logit of a tier variant: b-bit angles, shares quantised to the levels
+    (u = (rho/r) sqrt(d/2) domain) by the ascending thresholds; exact shares
+    when levels_u is None."""
+    k = _u16(k16)
+    q = np.ascontiguousarray(q, np.float64)
+    if levels_u is None:
+        return lib().orc_logit_grid(_ptr(q), _ptr(k), k.size, b, 0, None, None)
+    lv = np.ascontiguousarray(levels_u, np.float64)
+    th = np.ascontiguousarray(thresh_u if len(lv) > 1 else [0.0], np.float64)
+    assert th.size >= lv.size - 1
+    return lib().orc_logit_grid(_ptr(q), _ptr(k), k.size, b, lv.size, _ptr(lv), _ptr(th))
 
 
 def outlier(k16) -> bool:

@@ -392,6 +392,37 @@ double orc_logit_variant(const double* q, const uint16_t* k, int d, int b, int s
     return rt / sqrt((double)d) * s;
 }
 
+/* Tier/grid variant for the bytes-versus-logit-error study: b-bit angle
+   codes (the same coder), and the share u = (rho_i / r) sqrt(d/2) quantised
+   to L levels: code = the number of thresholds thresh_u[0..L-2] (ascending)
+   that u exceeds, decoded share levels_u[code] / sqrt(d/2); L = 0 keeps the
+   exact share.  The radius is r~ as in the tiers.  Returns the logit
+   (r~ / sqrt d) sum_i rho^_i (q_{2i} cos + q_{2i+1} sin)(2 pi c_i / 2^b). */
+double orc_logit_grid(const double* q, const uint16_t* k, int d, int b, int L,
+                      const double* levels_u, const double* thresh_u) {
+    uint64_t R2[2];
+    orc_norm2(k, d, R2);
+    double rt = h2d(orc_rtilde_from_r2(R2));
+    double r = sqrt(r2_double(R2)) * ldexp(1.0, -24);
+    double sq = sqrt(d / 2.0);
+    double s = 0.0;
+    for (int i = 0; i < d / 2; i++) {
+        double x = h2d(k[2 * i]), y = h2d(k[2 * i + 1]);
+        double share = (r > 0) ? sqrt(x * x + y * y) / r : 0.0;
+        if (L > 0) {
+            double u = share * sq;
+            int code = 0;
+            for (int j = 0; j < L - 1; j++)
+                if (u > thresh_u[j]) code++;
+            share = levels_u[code] / sq;
+        }
+        int c = orc_angle_code(k[2 * i], k[2 * i + 1], b);
+        double ang = 2.0 * M_PI * c / (double)(1 << b);
+        s += share * (q[2 * i] * cos(ang) + q[2 * i + 1] * sin(ang));
+    }
+    return rt / sqrt((double)d) * s;
+}
+
 /* ------------------------------------------------------------------ */
 /* RDR allocation [TS 2.2], [ABS]                                      */
 /* ------------------------------------------------------------------ */
