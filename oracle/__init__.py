@@ -73,6 +73,11 @@ _SIGS = {
     "orc_decode": (_i, [_i, _i, _i, _i, _i, _p, _p, _p, _p, _p, _i, _p, _p, _p, _i]),
     "orc_attention_mass": (_i, [_i, _i, _i, _i, _i, _p, _p, _p, _p, _i, _p]),
     "orc_outlier": (_i, [_p, _i]),
+    "orc_set_t1_scheme": (None, [_i]),
+    "orc_t1_scheme": (_i, []),
+    "orc_rho_code3": (_i, [_u16, _u16, _p, _i]),
+    "orc_rho_level3": (_d, [_i, _i]),
+    "orc_reconstruct_tier": (None, [_p, _i, _i, _p]),
     "orc_logit_grid": (_d, [_p, _p, _i, _i, _i, _p, _p]),
     "orc_outlier_flags": (_i, [_i, _i, _i, _i, _p, _p, _p]),
     "orc_d2h": (_u16, [_d]),
@@ -328,6 +333,40 @@ def logit_grid(q: np.ndarray, k16, b: int, levels_u=None, thresh_u=None) -> floa
     th = np.ascontiguousarray(thresh_u if len(lv) > 1 else [0.0], np.float64)
     assert th.size >= lv.size - 1
     return lib().orc_logit_grid(_ptr(q), _ptr(k), k.size, b, lv.size, _ptr(lv), _ptr(th))
+
+
+class t1_scheme:
+    """Context manager: the oracle's T1 code scheme inside the block (0: 6-bit
+    angle + 2-bit share, the pinned scheme; 1: 5-bit angle + 3-bit share)."""
+
+    def __init__(self, scheme: int):
+        self.scheme = scheme
+
+    def __enter__(self):
+        self.prev = lib().orc_t1_scheme()
+        lib().orc_set_t1_scheme(self.scheme)
+        return self
+
+    def __exit__(self, *exc):
+        lib().orc_set_t1_scheme(self.prev)
+        return False
+
+
+def rho_code3(x16: int, y16: int, R2: int, d: int) -> int:
+    a = np.array([R2 & (2**64 - 1), R2 >> 64], np.uint64)
+    return lib().orc_rho_code3(int(x16), int(y16), _ptr(a), d)
+
+
+def rho_level3(code: int, d: int = 128) -> float:
+    return lib().orc_rho_level3(code, d)
+
+
+def reconstruct_tier(k16, tier: int) -> np.ndarray:
+    """k^ of a key stored in tier 1 or 2 under the current T1 scheme."""
+    k = _u16(k16)
+    out = np.empty(k.size, np.float64)
+    lib().orc_reconstruct_tier(_ptr(k), k.size, tier, _ptr(out))
+    return out
 
 
 def outlier(k16) -> bool:

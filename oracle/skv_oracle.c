@@ -353,6 +353,54 @@ double orc_logit_codes(const double* q, const uint16_t* k, int d, int b) {
     return rt / sqrt((double)d) * s;
 }
 
+/* T1 code scheme.  0, the pinned scheme: 6-bit angle and a 2-bit share on
+   the uniform 4-level grid, code byte (angle << 2) | share.  1, the variant
+   the bytes-versus-logit-error study favours at the same 196 bytes: 5-bit
+   angle and a 3-bit share on the uniform 8-level grid u in {0.25, 0.5, ..,
+   2.0} (thresholds at the midpoints), code byte (angle << 3) | share.  The
+   scheme is process state set by orc_set_t1_scheme (tests only); T2 and the
+   allocation do not depend on it. */
+static int g_t1_scheme = 0;
+
+void orc_set_t1_scheme(int scheme) { g_t1_scheme = scheme ? 1 : 0; }
+int orc_t1_scheme(void) { return g_t1_scheme; }
+
+/* 3-bit share code: how many of the thresholds u > (2j + 3) / 8, j < 7,
+   hold; exact integer test 64 (d/2) rho^2 > (2j + 3)^2 R2, ties to the
+   lower code. */
+int orc_rho_code3(uint16_t xh, uint16_t yh, const uint64_t R2[2], int d) {
+    int64_t mx = h2m(xh), my = h2m(yh);
+    u128 ax = (u128)(mx < 0 ? -mx : mx), ay = (u128)(my < 0 ? -my : my);
+    u128 lhs = (ax * ax + ay * ay) * (u128)(64 * (d / 2));
+    u128 R = ((u128)R2[1] << 64) | R2[0];
+    int code = 0;
+    for (int j = 0; j < 7; j++) {
+        unsigned t = 2 * j + 3;
+        if (lhs > (u128)(t * t) * R) code++;
+    }
+    return code;
+}
+
+double orc_rho_level3(int code, int d) { return 0.25 * ((code & 7) + 1) / sqrt(d / 2.0); }
+
+/* k^ of a token stored in tier T1 or T2, under the current T1 scheme */
+void orc_reconstruct_tier(const uint16_t* k, int d, int tier, double* khat) {
+    if (tier != TIER_T1 || g_t1_scheme == 0) {
+        orc_reconstruct(k, d, tier == TIER_T1 ? BITS_T1 : BITS_T2, khat);
+        return;
+    }
+    uint64_t R2[2];
+    orc_norm2(k, d, R2);
+    double rt = h2d(orc_rtilde_from_r2(R2));
+    for (int i = 0; i < d / 2; i++) {
+        int c = orc_angle_code(k[2 * i], k[2 * i + 1], 5);
+        double rho = orc_rho_level3(orc_rho_code3(k[2 * i], k[2 * i + 1], R2, d), d);
+        double ang = 2.0 * M_PI * c / 32.0;
+        khat[2 * i] = rt * rho * cos(ang);
+        khat[2 * i + 1] = rt * rho * sin(ang);
+    }
+}
+
 /* q . k^ / sqrt(d) with k^ reconstructed (the decompress-then-dot form) */
 double orc_logit_recon(const double* q, const uint16_t* k, int d, int b) {
     double* kh = (double*)malloc(sizeof(double) * d);
@@ -655,7 +703,10 @@ static void write_row(uint8_t* page, int tier, int P, int d, int r,
     for (int p = 0; p < d / 2; p++) {
         int g = (p / 4) % 4, j = 4 * (p / 16) + p % 4;
         int rho = orc_rho_code(k[2 * p], k[2 * p + 1], R2, d);
-        if (tier == TIER_T1) {
+        if (tier == TIER_T1 && g_t1_scheme) {
+            int th = orc_angle_code(k[2 * p], k[2 * p + 1], 5);
+            row[16 * g + j] = (uint8_t)((th << 3) | orc_rho_code3(k[2 * p], k[2 * p + 1], R2, d));
+        } else if (tier == TIER_T1) {
             int th = orc_angle_code(k[2 * p], k[2 * p + 1], BITS_T1);
             row[16 * g + j] = (uint8_t)((th << 2) | rho);
         } else {
@@ -776,7 +827,7 @@ int orc_decode(int B, int Hq, int Hkv, int Tmax, int d, const int32_t* seq_lens,
             if (tr == TIER_T0)
                 for (int c = 0; c < d; c++) kh[c] = h2d(k[c]);
             else
-                orc_reconstruct(k, d, tr == TIER_T1 ? BITS_T1 : BITS_T2, kh);
+                orc_reconstruct_tier(k, d, tr, kh);
             double s = 0.0;
             for (int c = 0; c < d; c++) s += qd[c] * kh[c];
             logit[t] = s / sqrt((double)d);
@@ -883,7 +934,7 @@ int orc_attention_mass(int B, int Hq, int Hkv, int Tmax, int d, const int32_t* s
             if (tr == TIER_T0)
                 for (int c = 0; c < d; c++) kh[c] = h2d(k[c]);
             else
-                orc_reconstruct(k, d, tr == TIER_T1 ? BITS_T1 : BITS_T2, kh);
+                orc_reconstruct_tier(k, d, tr, kh);
             double s = 0.0;
             for (int c = 0; c < d; c++) s += qd[c] * kh[c];
             logit[t] = s / sqrt((double)d);
