@@ -71,6 +71,8 @@ extern "C" {
 #define SKV_TABLE_BOUNDARY4_Y 3  /* 16 fp32                                      */
 #define SKV_TABLE_KAPPA 4        /* 3 fp32: RDR slope per byte of each step      */
 #define SKV_TABLE_RHO_LEVELS 5   /* 4 fp32: decoded share of each 2-bit code     */
+#define SKV_TABLE_BOUNDARY5_X 6  /* 32 fp32: cos((j+1/2) 2pi/32)                */
+#define SKV_TABLE_BOUNDARY5_Y 7  /* 32 fp32: sin((j+1/2) 2pi/32)                */
 
 typedef struct skv_config {
   int32_t head_dim;    /* d: 128 */
@@ -80,7 +82,12 @@ typedef struct skv_config {
                           the share grid's top level, u = (rho/r) sqrt(d/2) > 4
                           (technical summary 2.2: outliers are among the
                           protected states) */
-  int32_t reserved[5]; /* zero */
+  int32_t t1_angle_bits; /* 0 or 6: T1 codes a pair as a 6-bit angle and a
+                          2-bit share (levels u = 0.5, 1.0, 1.5, 2.0); 5: a 5-bit
+                          angle and a 3-bit share (levels u = 0.25 .. 2.0 in
+                          steps of 0.25), the same byte per pair.  The second
+                          has about 40% lower logit error at the same 196 B */
+  int32_t reserved[4]; /* zero */
 } skv_config;
 
 /* Device pools of page slots, one per tier.  Slot s of tier t starts at

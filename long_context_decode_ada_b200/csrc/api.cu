@@ -22,8 +22,9 @@ struct skv_ctx {
   int device;
   int sm_count;
   size_t smem_optin;
-  float bx6[64], by6[64], bx4[16], by4[16];
-  float cos6[64], sin6[64], cos4[16], sin4[16];
+  float bx6[64], by6[64], bx4[16], by4[16], bx5[32], by5[32];
+  float cos6[64], sin6[64], cos4[16], sin4[16], cos5[32], sin5[32];
+  int t1_scheme = 0;            // 0: 6-bit angle + 2-bit share; 1: 5-bit + 3-bit
   float kappa[3];
   float rho_levels[4];
   long long payload[4];
@@ -120,6 +121,11 @@ int skv_create(const skv_config* cfg, skv_ctx** out) {
   c->d = 128;
   c->P = P;
   c->outlier_protect = cfg->outlier_protect != 0;
+  if (cfg->t1_angle_bits != 0 && cfg->t1_angle_bits != 5 && cfg->t1_angle_bits != 6) {
+    delete c;
+    return fail(SKV_ERR_ARG, "t1_angle_bits must be 0, 5 or 6 (got %d)", cfg->t1_angle_bits);
+  }
+  c->t1_scheme = cfg->t1_angle_bits == 5;
   c->log2P = P == 16 ? 4 : (P == 32 ? 5 : 6);
   c->device = 0;
   c->profile_event = nullptr;
@@ -144,6 +150,14 @@ int skv_create(const skv_config* cfg, skv_ctx** out) {
     const double a = 2.0 * M_PI * j / 64.0;
     c->cos6[j] = (float)std::cos(a);
     c->sin6[j] = (float)std::sin(a);
+  }
+  for (int j = 0; j < 32; ++j) {
+    const double beta = (j + 0.5) * (2.0 * M_PI / 32.0);
+    c->bx5[j] = (float)std::cos(beta);
+    c->by5[j] = (float)std::sin(beta);
+    const double a = 2.0 * M_PI * j / 32.0;
+    c->cos5[j] = (float)std::cos(a);
+    c->sin5[j] = (float)std::sin(a);
   }
   for (int j = 0; j < 16; ++j) {
     const double beta = (j + 0.5) * (2.0 * M_PI / 16.0);
@@ -193,6 +207,8 @@ int skv_tables(const skv_ctx* ctx, int which, float* out, int64_t n) {
     case SKV_TABLE_BOUNDARY4_Y: src = ctx->by4; len = 16; break;
     case SKV_TABLE_KAPPA: src = ctx->kappa; len = 3; break;
     case SKV_TABLE_RHO_LEVELS: src = ctx->rho_levels; len = 4; break;
+    case SKV_TABLE_BOUNDARY5_X: src = ctx->bx5; len = 32; break;
+    case SKV_TABLE_BOUNDARY5_Y: src = ctx->by5; len = 32; break;
     default: return fail(SKV_ERR_ARG, "skv_tables: unknown table %d", which);
   }
   if (n < len) return fail(SKV_ERR_ARG, "skv_tables: need %lld floats", (long long)len);
@@ -353,6 +369,9 @@ int skv_encode(skv_ctx* ctx, const uint16_t* K, const uint16_t* V, int B, int Hk
   std::memcpy(p.by6, ctx->by6, sizeof(p.by6));
   std::memcpy(p.bx4, ctx->bx4, sizeof(p.bx4));
   std::memcpy(p.by4, ctx->by4, sizeof(p.by4));
+  std::memcpy(p.bx5, ctx->bx5, sizeof(p.bx5));
+  std::memcpy(p.by5, ctx->by5, sizeof(p.by5));
+  p.t1_scheme = ctx->t1_scheme;
   cudaError_t e = skv::launch_encode(p, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "skv_encode launch");
   return ok();
@@ -463,6 +482,9 @@ static int decode_common(skv_ctx* ctx, const void* q, int q_dtype, int B, int Hq
   std::memcpy(p.sin6, ctx->sin6, sizeof(p.sin6));
   std::memcpy(p.cos4, ctx->cos4, sizeof(p.cos4));
   std::memcpy(p.sin4, ctx->sin4, sizeof(p.sin4));
+  std::memcpy(p.cos5, ctx->cos5, sizeof(p.cos5));
+  std::memcpy(p.sin5, ctx->sin5, sizeof(p.sin5));
+  p.t1_scheme = ctx->t1_scheme;
   cudaError_t e =
       skv::launch_decode(p, G, dense, static_cast<cudaStream_t>(stream), ctx->profile_event);
   if (e != cudaSuccess) return cuda_fail(e, name);

@@ -425,11 +425,17 @@ __device__ __forceinline__ void make_qfrag(const float (*q32)[kHeadDim], float q
 // key pair of unit radius: shares enter as code + 1) as fp16 hi and lo
 // halves, x = hi + lo to about 2^-22 relative: {hi(x), hi(y)}, {lo(x), lo(y)}.
 // The T2 entries follow T1's (TBL2 = TBL1 + 32 KB).
+// V53: the T1 variant, code byte (angle5 << 3) | share3 with weight (s + 1) / 2.
+template <bool V53>
 __device__ __forceinline__ void build_tables(const DecodeParams& p, uint8_t* tbl1p, int n_entries,
                                              int tid, int nthreads) {
   for (int e = tid; e < n_entries; e += nthreads) {
     float cs, sn, w;
-    if (e < 256) {
+    if (V53 && e < 256) {
+      cs = p.cos5[e >> 3];
+      sn = p.sin5[e >> 3];
+      w = 0.5f * (float)((e & 7) + 1);
+    } else if (e < 256) {
       cs = p.cos6[e >> 2];
       sn = p.sin6[e >> 2];
       w = (float)((e & 3) + 1);
@@ -710,7 +716,7 @@ __device__ __forceinline__ void process_rows(const DecodeParams& p, uint32_t pg,
   }
 }
 
-template <int G, bool DENSE, bool CAP>
+template <int G, bool DENSE, bool CAP, bool V53>
 __global__ void __launch_bounds__(kDecodeThreads, 1)
     decode_kernel(const __grid_constant__ DecodeParams p) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
@@ -1090,7 +1096,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       }
     }
     if constexpr (!DENSE) {
-      if (tbl_entries) build_tables(p, tbl1p, tbl_entries, tid, nct);
+      if (tbl_entries) build_tables<V53>(p, tbl1p, tbl_entries, tid, nct);
       tbl_entries = 0;
     }
     named_bar_sync(1, nct);
@@ -1511,17 +1517,23 @@ cudaError_t launch_decode_g(const DecodeParams& p, cudaStream_t stream, cudaEven
   const size_t smem = (size_t)p.smem_bytes;
   // the logit-capturing variant when a logits buffer is given (ADA only)
   const bool cap = !DENSE && p.logits != nullptr;
-  auto kern = cap ? decode_kernel<G, DENSE, !DENSE> : decode_kernel<G, DENSE, false>;
+  // the T1 variant's table (ADA only; the dense pages have no T1)
+  const bool v53 = !DENSE && p.t1_scheme != 0;
+  auto kern = cap ? (v53 ? decode_kernel<G, DENSE, !DENSE, !DENSE>
+                         : decode_kernel<G, DENSE, !DENSE, false>)
+                  : (v53 ? decode_kernel<G, DENSE, false, !DENSE>
+                         : decode_kernel<G, DENSE, false, false>);
+  const int vi = (cap ? 1 : 0) + (v53 ? 2 : 0);
   // The shared-memory opt-in is set once per device, variant and size
   // (outside any stream capture: the first call is expected to be eager).
-  static size_t configured[2][64] = {};
+  static size_t configured[4][64] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= 64 || configured[cap][dev] < smem) {
+  if (dev < 0 || dev >= 64 || configured[vi][dev] < smem) {
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    if (dev >= 0 && dev < 64) configured[cap][dev] = smem;
+    if (dev >= 0 && dev < 64) configured[vi][dev] = smem;
   }
   const int U = p.B * p.Hkv;
   kern<<<p.S, kDecodeThreads, p.smem_bytes, stream>>>(p);

@@ -65,6 +65,17 @@ __device__ __forceinline__ uint32_t angle_code(uint16_t xh, uint16_t yh, int b, 
   return (uint32_t)(base + lo) & (uint32_t)((1 << b) - 1);
 }
 
+// 3-bit share code of the T1 variant: thresholds u > (2j + 3) / 8, j < 7,
+// tested as 64 (d/2) rho^2 > (2j + 3)^2 R2; ties go to the lower code
+__device__ __forceinline__ uint32_t rho_code3(long long mx, long long my, u128 R2) {
+  const u128 ax = (u128)(mx < 0 ? -mx : mx), ay = (u128)(my < 0 ? -my : my);
+  const u128 lhs = (ax * ax + ay * ay) * (u128)(64 * (kHeadDim / 2));
+  uint32_t c = 0;
+#pragma unroll
+  for (int j = 0; j < 7; ++j) c += lhs > (u128)((2 * j + 3) * (2 * j + 3)) * R2;
+  return c;
+}
+
 __device__ __forceinline__ uint32_t rho_code(long long mx, long long my, u128 R2) {
   const u128 ax = (u128)(mx < 0 ? -mx : mx), ay = (u128)(my < 0 ? -my : my);
   const u128 lhs = (ax * ax + ay * ay) * (u128)(16 * (kHeadDim / 2));
@@ -85,10 +96,14 @@ __device__ __forceinline__ int v_frag_offset(int row, int dd, int elem_bytes) {
 }
 
 __global__ void __launch_bounds__(256) encode_kernel(const __grid_constant__ EncodeParams p) {
-  __shared__ float sbx6[64], sby6[64], sbx4[16], sby4[16];
+  __shared__ float sbx6[64], sby6[64], sbx4[16], sby4[16], sbx5[32], sby5[32];
   for (int i = threadIdx.x; i < 64; i += blockDim.x) {
     sbx6[i] = p.bx6[i];
     sby6[i] = p.by6[i];
+    if (i < 32) {
+      sbx5[i] = p.bx5[i];
+      sby5[i] = p.by5[i];
+    }
     if (i < 16) {
       sbx4[i] = p.bx4[i];
       sby4[i] = p.by4[i];
@@ -181,13 +196,14 @@ __global__ void __launch_bounds__(256) encode_kernel(const __grid_constant__ Enc
 
   // ---- codes of pairs 2 lane, 2 lane + 1
   const bool t1 = tr == SKV_TIER_T1;
-  const int bits = t1 ? 6 : 4;
-  const float* bx = t1 ? sbx6 : sbx4;
-  const float* by = t1 ? sby6 : sby4;
+  const bool v53 = t1 && p.t1_scheme;  // T1 variant: 5-bit angle + 3-bit share
+  const int bits = t1 ? (v53 ? 5 : 6) : 4;
+  const float* bx = t1 ? (v53 ? sbx5 : sbx6) : sbx4;
+  const float* by = t1 ? (v53 ? sby5 : sby6) : sby4;
   const uint32_t th0 = angle_code(k4[0], k4[1], bits, bx, by);
   const uint32_t th1 = angle_code(k4[2], k4[3], bits, bx, by);
-  const uint32_t rh0 = rho_code(m[0], m[1], R2);
-  const uint32_t rh1 = rho_code(m[2], m[3], R2);
+  const uint32_t rh0 = v53 ? rho_code3(m[0], m[1], R2) : rho_code(m[0], m[1], R2);
+  const uint32_t rh1 = v53 ? rho_code3(m[2], m[3], R2) : rho_code(m[2], m[3], R2);
   const uint32_t packed = th0 | (th1 << 8) | (rh0 << 16) | (rh1 << 24);
 
   // ---- V quantiser
@@ -234,7 +250,7 @@ __global__ void __launch_bounds__(256) encode_kernel(const __grid_constant__ Enc
       const uint32_t src = __shfl_sync(0xFFFFFFFFu, packed, pr >> 1);
       const uint32_t th = (src >> (8 * (pr & 1))) & 0xFFu;
       const uint32_t rh = (src >> (16 + 8 * (pr & 1))) & 0xFFu;
-      word |= ((th << 2) | rh) << (8 * e);
+      word |= ((th << (v53 ? 3 : 2)) | rh) << (8 * e);
     }
     if (lane < 16) *reinterpret_cast<uint32_t*>(crow + 4 * lane) = word;
   } else {

@@ -27,7 +27,7 @@ MODE_QUOTA, MODE_BUDGET = 0, 1
 Q_FP16, Q_BF16 = 0, 1
 WS_ALLOCATE, WS_DECODE, WS_DENSE_DECODE, WS_APPEND, WS_DECODE_UTILITY = 0, 1, 2, 3, 4
 TABLE_BOUNDARY6_X, TABLE_BOUNDARY6_Y, TABLE_BOUNDARY4_X, TABLE_BOUNDARY4_Y, TABLE_KAPPA, \
-    TABLE_RHO_LEVELS = range(6)
+    TABLE_RHO_LEVELS, TABLE_BOUNDARY5_X, TABLE_BOUNDARY5_Y = range(8)
 
 EXPORTS = [
     "skv_create", "skv_destroy", "skv_last_error", "skv_page_bytes", "skv_tables",
@@ -42,7 +42,8 @@ EXPORTS = [
 
 class SkvConfig(C.Structure):
     _fields_ = [("head_dim", C.c_int32), ("page_size", C.c_int32),
-                ("outlier_protect", C.c_int32), ("reserved", C.c_int32 * 5)]
+                ("outlier_protect", C.c_int32), ("t1_angle_bits", C.c_int32),
+                ("reserved", C.c_int32 * 4)]
 
 
 class SkvPools(C.Structure):
@@ -135,15 +136,17 @@ def _stream(stream=None):
 class Context:
     """An skv_ctx: head_dim 128, page size P; bound to the current device."""
 
-    def __init__(self, page_size: int, head_dim: int = 128, outlier_protect: bool = False):
+    def __init__(self, page_size: int, head_dim: int = 128, outlier_protect: bool = False,
+                 t1_angle_bits: int = 6):
         cfg = SkvConfig(head_dim=head_dim, page_size=page_size,
-                        outlier_protect=1 if outlier_protect else 0)
+                        outlier_protect=1 if outlier_protect else 0, t1_angle_bits=t1_angle_bits)
         h = C.c_void_p()
         _check(lib().skv_create(C.byref(cfg), C.byref(h)))
         self._h = h
         self.P = page_size
         self.d = head_dim
         self.outlier_protect = bool(outlier_protect)
+        self.t1_angle_bits = t1_angle_bits
 
     def __del__(self):
         h = getattr(self, "_h", None)

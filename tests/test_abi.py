@@ -46,6 +46,16 @@ def test_tables_match_oracle_bytes():
     assert ctx.table(skv.TABLE_KAPPA, 3).tobytes() == oracle.kappa(128).tobytes()
     lv = ctx.table(skv.TABLE_RHO_LEVELS, 4)
     assert list(lv) == [oracle.rho_level(c, 128) for c in range(4)]
+    bx5, by5 = oracle.boundaries(5)
+    assert ctx.table(skv.TABLE_BOUNDARY5_X, 32).tobytes() == bx5.tobytes()
+    assert ctx.table(skv.TABLE_BOUNDARY5_Y, 32).tobytes() == by5.tobytes()
+
+
+def test_t1_angle_bits_is_checked():
+    skv.Context(16, t1_angle_bits=5)
+    skv.Context(16, t1_angle_bits=6)
+    with pytest.raises(skv.SkvError):
+        skv.Context(16, t1_angle_bits=4)
 
 
 @pytest.mark.parametrize("P", [16, 32, 64])
