@@ -508,7 +508,7 @@ def run_skv(args, rank, world, local_rank):
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": profiled_traffic(),
                          "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)",
-                         "kernel": "decode_kernel<4,false>", "kernel_ms": kern_ms_avg,
+                         "kernel": "decode_kernel<4,false,false,false>", "kernel_ms": kern_ms_avg,
                          "algorithmic_bytes": algo_bytes, "payload_bytes_streamed": payload_bytes},
             "cpu_baseline": cpu,
             "e2e": e2e,
