@@ -769,8 +769,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<const uint8_t*>(p.q) + 128 * l));
   }
   // units without any resident page: out = 0, lse = -inf, nothing to merge
-  // (written by CTA 0)
+  // (written by CTA 0, once the grids this one depends on have completed)
   if (c == 0) {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     for (int u = warp; u < U; u += kDecodeThreads / 32) {
       if (p.indptr[u + 1] > p.indptr[u]) continue;
       const long long o = (long long)(u / p.Hkv) * p.Hq + (long long)(u % p.Hkv) * G;
@@ -790,6 +791,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     const bool inside = unit_aligned_split(U, p.S) ? true
                                                   : (g0 < (long long)p.indptr[U] && g0 > (long long)p.indptr[u]);
     if (inside && tid < G) {
+      asm volatile("griddepcontrol.wait;" ::: "memory");
       float* part = p.part + (long long)(c + u) * G * kPartStride + tid * kPartStride;
       part[0] = -INFINITY;
       part[1] = 0.0f;
@@ -1063,7 +1065,15 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   uint8_t* const tbl1p = smem_raw + (tbl1 - base);
   float* const stashp = reinterpret_cast<float*>(tbl1p);
   static_assert(DENSE || kNCW * 4 * kHeadDim * 4 <= (int)kTbl1, "combine stash fits TBL1");
-  int tbl_entries = DENSE ? 0 : 256 + 64;  // table entries still to build
+  // The decode may be a programmatic dependent of the previous step's grids
+  // (launched while they finish).  The planner and the issuers start on the
+  // page table and the pages at once: the store is never written by a grid
+  // that lets dependents start early.  The consumers build the code tables
+  // (parameters only), then wait for those grids before they read the
+  // queries or write any result or partial.
+  if constexpr (!DENSE) build_tables<V53>(p, tbl1p, 256 + 64, tid, nct);
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  int tbl_entries = 0;  // table entries still to build (after a combine's stash)
   int it = 0;  // item index within the run
   bool ok = true;
   constexpr int kQPer = (4 * kHeadDim + kNCW * 32 - 1) / (kNCW * 32);  // q elements per thread
@@ -1536,9 +1546,22 @@ cudaError_t launch_decode_g(const DecodeParams& p, cudaStream_t stream, cudaEven
     if (dev >= 0 && dev < 64) configured[vi][dev] = smem;
   }
   const int U = p.B * p.Hkv;
-  kern<<<p.S, kDecodeThreads, p.smem_bytes, stream>>>(p);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  {
+    // a programmatic dependent of the stream's previous kernel: its CTAs may
+    // start on the pages while that kernel finishes (see the kernel's waits)
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)p.S);
+    cfg.blockDim = dim3(kDecodeThreads);
+    cfg.dynamicSmemBytes = (size_t)p.smem_bytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, kern, p);
+    if (e != cudaSuccess) return e;
+  }
   if (between) {
     // a profile point right after the decode grid (an external record node
     // when the stream is being captured; the merge then follows it in order)
