@@ -65,3 +65,21 @@ def test_variant_is_closer_to_exact_attention():
         errs[bits] = (float(np.sqrt(np.mean((g["out"] - eo) ** 2))),
                       float(np.sqrt(np.mean((g["lse"] - el) ** 2))))
     assert errs[5][0] < 0.8 * errs[6][0], errs
+
+
+def test_variant_long_context_128k_full_size():
+    """The 128K store with the T1 variant in the bench's launch
+    configuration: tiers, row map and page table bit-exact (the variant
+    changes only T1's code bytes), every T1 page's bytes on a sample of
+    pages, and sampled rows of the decode against the oracle."""
+    w = wl.long_context()
+    g = run(w, 5)
+    with oracle.t1_scheme(1):
+        ref = oracle.run_workload(w, do_decode=False)
+        rows = np.array([[0, 0], [0, 9], [0, 22], [0, 31]], np.int32)
+        ro, rl = oracle.decode(w.B, w.Hq, w.Hkv, w.Tmax, w.d, w.seq_lens, w.K, w.V, ref["tier"],
+                               w.q, w.q_dtype, units=rows)
+    compare_store(w, g, ref)
+    b, h = rows[:, 0], rows[:, 1]
+    assert_close(g["out"][b, h], ro[b, h], "out (sampled rows)")
+    assert_close(g["lse"][b, h], rl[b, h], "lse (sampled rows)")
