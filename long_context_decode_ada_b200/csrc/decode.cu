@@ -1390,6 +1390,10 @@ template <int G>
 __global__ void __launch_bounds__(256) utility_kernel(const UtilityParams p) {
   constexpr float kLog2e = 1.4426950408889634f;
   __shared__ float ls_s[G];
+  // the next step's decode may start on the pages now (it waits for this
+  // grid before reading queries or writing results; the store is not
+  // written here)
+  asm volatile("griddepcontrol.launch_dependents;");
   const int U = p.B * p.Hkv;
   const int T = (int)p.Tmax;
   bool waited = false;

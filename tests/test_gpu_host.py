@@ -13,24 +13,26 @@ from _gpu import assert_close, run_gpu
 pytestmark = pytest.mark.gpu
 
 
-def host_buffers(w, dev):
-    q_host = dev["q"].cpu().pin_memory()
-    out_host = torch.empty((w.B, w.Hq, 128), dtype=torch.float32).pin_memory()
-    lse_host = torch.empty((w.B, w.Hq), dtype=torch.float32).pin_memory()
+def host_buffers(w, dev, pinned=True):
+    pin = (lambda t: t.pin_memory()) if pinned else (lambda t: t)
+    q_host = pin(dev["q"].cpu())
+    out_host = pin(torch.empty((w.B, w.Hq, 128), dtype=torch.float32))
+    lse_host = pin(torch.empty((w.B, w.Hq), dtype=torch.float32))
     scratch = (torch.empty_like(dev["q"]),
                torch.empty((w.B, w.Hq, 128), dtype=torch.float32, device=dev["q"].device),
                torch.empty((w.B, w.Hq), dtype=torch.float32, device=dev["q"].device))
     return q_host, out_host, lse_host, scratch
 
 
-@pytest.mark.parametrize("q_dtype", ["bf16", "fp16"])
-def test_host_step_equals_device_decode_and_oracle(q_dtype):
+@pytest.mark.parametrize("q_dtype,pinned", [("bf16", True), ("fp16", True), ("bf16", False)])
+def test_host_step_equals_device_decode_and_oracle(q_dtype, pinned):
+    # pageable host buffers work too (the copies are then synchronous)
     lens = [600, 77, 1]
     w = wl.custom(95, 3, 2, 4, 16, lens, wl.MODE_QUOTA,
                   quota=[[100, 300, 150], [10, 30, 20], [1, 0, 0]], q_dtype=q_dtype)
     g = run_gpu(w)
     cache, dev = g["cache"], g["dev"]
-    q_host, out_host, lse_host, scratch = host_buffers(w, dev)
+    q_host, out_host, lse_host, scratch = host_buffers(w, dev, pinned)
     cache.decode_host(q_host, dev["q_dtype"], w.Hq, out_host, lse_host, scratch)
     assert np.array_equal(out_host.numpy(), g["out"])
     assert np.array_equal(lse_host.numpy(), g["lse"])
