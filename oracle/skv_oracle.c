@@ -235,7 +235,7 @@ static double r2_double(const uint64_t R2[2]) {
 
 /* Quantised radius r~ = fp16(min(r, 65504)) with r = sqrt(R2) * 2^-24:
    one correctly rounded sqrt in double, one rounding to fp16.  READING: fp16
-   for r~ comes from the pinned scheme; saturation is this build's choice. */
+   for r~ comes from the pinned scheme; saturation is this implementation's choice. */
 uint16_t orc_rtilde_from_r2(const uint64_t R2[2]) {
     double r = sqrt(r2_double(R2)) * ldexp(1.0, -24);
     if (r > 65504.0) r = 65504.0;
