@@ -74,6 +74,8 @@ _SIGS = {
     "orc_attention_mass": (_i, [_i, _i, _i, _i, _i, _p, _p, _p, _p, _i, _p]),
     "orc_outlier": (_i, [_p, _i]),
     "orc_set_t1_scheme": (None, [_i]),
+    "orc_set_share_grid": (None, [_i]),
+    "orc_share_grid": (_i, []),
     "orc_t1_scheme": (_i, []),
     "orc_rho_code3": (_i, [_u16, _u16, _p, _i]),
     "orc_rho_level3": (_d, [_i, _i]),
@@ -349,6 +351,23 @@ class t1_scheme:
 
     def __exit__(self, *exc):
         lib().orc_set_t1_scheme(self.prev)
+        return False
+
+
+class share_grid:
+    """Context manager: the oracle's 2-bit share grid inside the block (0: the
+    uniform levels 0.5 .. 2.0; 1: the exact Lloyd-Max grid)."""
+
+    def __init__(self, grid: int):
+        self.grid = grid
+
+    def __enter__(self):
+        self.prev = lib().orc_share_grid()
+        lib().orc_set_share_grid(self.grid)
+        return self
+
+    def __exit__(self, *exc):
+        lib().orc_set_share_grid(self.prev)
         return False
 
 

@@ -151,10 +151,22 @@ void orc_boundaries(int b, float* bx, float* by) {
 /* Share grid.  READING (the pinned scheme says only "2-bit code on a fixed
    grid"): u = (rho_i / r) * sqrt(d/2) is quantised to the levels
    {0.5, 1.0, 1.5, 2.0} with thresholds {0.75, 1.25, 1.75}; the decoded share
-   is rho^_i = u_level / sqrt(d/2). */
+   is rho^_i = u_level / sqrt(d/2).
+   The non-uniform variant (share grid 1, set per process by
+   orc_set_share_grid; tests only) is the Lloyd-Max grid of the Rayleigh
+   density that u follows for Gaussian keys, made exact: levels
+   {383, 807, 1249, 1831} / 1024 and thresholds sqrt({22, 64, 145} / 64),
+   the nearest such values to the optimum (levels 0.3743, 0.7880, 1.2195,
+   1.7884; thresholds 0.5811, 1.0037, 1.5039). */
+static int g_share_grid = 0;
+
+void orc_set_share_grid(int grid) { g_share_grid = grid ? 1 : 0; }
+int orc_share_grid(void) { return g_share_grid; }
+
 double orc_rho_level(int code, int d) {
     static const double U[4] = {0.5, 1.0, 1.5, 2.0};
-    return U[code & 3] / sqrt(d / 2.0);
+    static const double LM[4] = {383.0 / 1024, 807.0 / 1024, 1249.0 / 1024, 1831.0 / 1024};
+    return (g_share_grid ? LM[code & 3] : U[code & 3]) / sqrt(d / 2.0);
 }
 
 /* Relative distortion of each tier, c(tier), for the RDR surrogate [TS 2.2]:
@@ -276,14 +288,15 @@ int orc_angle_code(uint16_t xh, uint16_t yh, int b) {
 /* 2-bit share code of the pair (x, y): how many of the thresholds
    u > {0.75, 1.25, 1.75} hold, u = (rho/r) sqrt(d/2).  Exact integer test:
    u > t  <=>  16 (d/2) rho^2 > (4t)^2 R2 with (4t)^2 = 9, 25, 49; a tie
-   goes to the lower code. */
+   goes to the lower code.  Share grid 1: 64 (d/2) rho^2 > {22, 64, 145} R2. */
 int orc_rho_code(uint16_t xh, uint16_t yh, const uint64_t R2[2], int d) {
-    static const unsigned U[3] = {9, 25, 49};
+    static const unsigned U16[3] = {9, 25, 49}, U64[3] = {22, 64, 145};
+    const unsigned* U = g_share_grid ? U64 : U16;
     int64_t mx = h2m(xh), my = h2m(yh);
     u128 ax = (u128)(mx < 0 ? -mx : mx), ay = (u128)(my < 0 ? -my : my);
     u128 rho2 = ax * ax + ay * ay;
     u128 R = ((u128)R2[1] << 64) | R2[0];
-    u128 lhs = rho2 * (u128)(16 * (d / 2));
+    u128 lhs = rho2 * (u128)((g_share_grid ? 64 : 16) * (d / 2));
     int code = 0;
     for (int j = 0; j < 3; j++)
         if (lhs > (u128)U[j] * R) code++;
