@@ -87,7 +87,13 @@ typedef struct skv_config {
                           angle and a 3-bit share (levels u = 0.25 .. 2.0 in
                           steps of 0.25), the same byte per pair.  The second
                           has about 40% lower logit error at the same 196 B */
-  int32_t reserved[4]; /* zero */
+  int32_t share_grid;  /* 0: the 2-bit share codes (T2, and T1 with 6 + 2 bits)
+                          on the uniform levels u = 0.5, 1.0, 1.5, 2.0; 1: on
+                          the exact Lloyd-Max grid of the Rayleigh density,
+                          levels {383, 807, 1249, 1831} / 1024, thresholds
+                          sqrt({22, 64, 145} / 64) (lower logit error at the
+                          same bytes) */
+  int32_t reserved[3]; /* zero */
 } skv_config;
 
 /* Device pools of page slots, one per tier.  Slot s of tier t starts at

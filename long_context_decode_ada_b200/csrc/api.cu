@@ -25,6 +25,7 @@ struct skv_ctx {
   float bx6[64], by6[64], bx4[16], by4[16], bx5[32], by5[32];
   float cos6[64], sin6[64], cos4[16], sin4[16], cos5[32], sin5[32];
   int t1_scheme = 0;            // 0: 6-bit angle + 2-bit share; 1: 5-bit + 3-bit
+  int share_grid = 0;           // 2-bit share grid: 0 uniform, 1 Lloyd-Max
   float kappa[3];
   float rho_levels[4];
   long long payload[4];
@@ -126,6 +127,11 @@ int skv_create(const skv_config* cfg, skv_ctx** out) {
     return fail(SKV_ERR_ARG, "t1_angle_bits must be 0, 5 or 6 (got %d)", cfg->t1_angle_bits);
   }
   c->t1_scheme = cfg->t1_angle_bits == 5;
+  if (cfg->share_grid != 0 && cfg->share_grid != 1) {
+    delete c;
+    return fail(SKV_ERR_ARG, "share_grid must be 0 or 1 (got %d)", cfg->share_grid);
+  }
+  c->share_grid = cfg->share_grid;
   c->log2P = P == 16 ? 4 : (P == 32 ? 5 : 6);
   c->device = 0;
   c->profile_event = nullptr;
@@ -372,6 +378,7 @@ int skv_encode(skv_ctx* ctx, const uint16_t* K, const uint16_t* V, int B, int Hk
   std::memcpy(p.bx5, ctx->bx5, sizeof(p.bx5));
   std::memcpy(p.by5, ctx->by5, sizeof(p.by5));
   p.t1_scheme = ctx->t1_scheme;
+  p.share_grid = ctx->share_grid;
   cudaError_t e = skv::launch_encode(p, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "skv_encode launch");
   return ok();
@@ -485,6 +492,7 @@ static int decode_common(skv_ctx* ctx, const void* q, int q_dtype, int B, int Hq
   std::memcpy(p.cos5, ctx->cos5, sizeof(p.cos5));
   std::memcpy(p.sin5, ctx->sin5, sizeof(p.sin5));
   p.t1_scheme = ctx->t1_scheme;
+  p.share_grid = ctx->share_grid;
   cudaError_t e =
       skv::launch_decode(p, G, dense, static_cast<cudaStream_t>(stream), ctx->profile_event);
   if (e != cudaSuccess) return cuda_fail(e, name);

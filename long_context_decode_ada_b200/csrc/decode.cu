@@ -425,24 +425,34 @@ __device__ __forceinline__ void make_qfrag(const float (*q32)[kHeadDim], float q
 // key pair of unit radius: shares enter as code + 1) as fp16 hi and lo
 // halves, x = hi + lo to about 2^-22 relative: {hi(x), hi(y)}, {lo(x), lo(y)}.
 // The T2 entries follow T1's (TBL2 = TBL1 + 32 KB).
-// V53: the T1 variant, code byte (angle5 << 3) | share3 with weight (s + 1) / 2.
-template <bool V53>
+// VAR bit 0: the T1 variant, code byte (angle5 << 3) | share3 with weight
+// (s + 1) / 2; bit 1: the 2-bit share codes on the Lloyd-Max grid, weights
+// 2 u_s = {766, 1614, 2498, 3662} / 1024 instead of s + 1 (share u_s / 8).
+template <int VAR>
+__device__ __forceinline__ float share2_weight(uint32_t s) {
+  if constexpr ((VAR & 2) != 0)
+    return s == 0 ? 766.0f / 1024 : (s == 1 ? 1614.0f / 1024 : (s == 2 ? 2498.0f / 1024 : 3662.0f / 1024));
+  else
+    return (float)(s + 1);
+}
+
+template <int VAR>
 __device__ __forceinline__ void build_tables(const DecodeParams& p, uint8_t* tbl1p, int n_entries,
                                              int tid, int nthreads) {
   for (int e = tid; e < n_entries; e += nthreads) {
     float cs, sn, w;
-    if (V53 && e < 256) {
+    if ((VAR & 1) && e < 256) {
       cs = p.cos5[e >> 3];
       sn = p.sin5[e >> 3];
       w = 0.5f * (float)((e & 7) + 1);
     } else if (e < 256) {
       cs = p.cos6[e >> 2];
       sn = p.sin6[e >> 2];
-      w = (float)((e & 3) + 1);
+      w = share2_weight<VAR>((uint32_t)e & 3u);
     } else {
       cs = p.cos4[(e - 256) & 15];
       sn = p.sin4[(e - 256) & 15];
-      w = (float)(((e - 256) >> 4) + 1);
+      w = share2_weight<VAR>((uint32_t)(e - 256) >> 4);
     }
     const float x = w * cs, y = w * sn;
     const __half hx = __float2half_rn(x), hy = __float2half_rn(y);
@@ -716,7 +726,7 @@ __device__ __forceinline__ void process_rows(const DecodeParams& p, uint32_t pg,
   }
 }
 
-template <int G, bool DENSE, bool CAP, bool V53>
+template <int G, bool DENSE, bool CAP, int VAR>
 __global__ void __launch_bounds__(kDecodeThreads, 1)
     decode_kernel(const __grid_constant__ DecodeParams p) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
@@ -1071,7 +1081,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   // that lets dependents start early.  The consumers build the code tables
   // (parameters only), then wait for those grids before they read the
   // queries or write any result or partial.
-  if constexpr (!DENSE) build_tables<V53>(p, tbl1p, 256 + 64, tid, nct);
+  if constexpr (!DENSE) build_tables<VAR>(p, tbl1p, 256 + 64, tid, nct);
   asm volatile("griddepcontrol.wait;" ::: "memory");
   int tbl_entries = 0;  // table entries still to build (after a combine's stash)
   int it = 0;  // item index within the run
@@ -1106,7 +1116,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       }
     }
     if constexpr (!DENSE) {
-      if (tbl_entries) build_tables<V53>(p, tbl1p, tbl_entries, tid, nct);
+      if (tbl_entries) build_tables<VAR>(p, tbl1p, tbl_entries, tid, nct);
       tbl_entries = 0;
     }
     named_bar_sync(1, nct);
@@ -1531,16 +1541,28 @@ cudaError_t launch_decode_g(const DecodeParams& p, cudaStream_t stream, cudaEven
   const size_t smem = (size_t)p.smem_bytes;
   // the logit-capturing variant when a logits buffer is given (ADA only)
   const bool cap = !DENSE && p.logits != nullptr;
-  // the T1 variant's table (ADA only; the dense pages have no T1)
-  const bool v53 = !DENSE && p.t1_scheme != 0;
-  auto kern = cap ? (v53 ? decode_kernel<G, DENSE, !DENSE, !DENSE>
-                         : decode_kernel<G, DENSE, !DENSE, false>)
-                  : (v53 ? decode_kernel<G, DENSE, false, !DENSE>
-                         : decode_kernel<G, DENSE, false, false>);
-  const int vi = (cap ? 1 : 0) + (v53 ? 2 : 0);
+  // the code-table variant (ADA only; the dense pages have no codes):
+  // bit 0 the T1 5 + 3 scheme, bit 1 the Lloyd-Max 2-bit share grid
+  const int var = DENSE ? 0 : ((p.t1_scheme ? 1 : 0) | (p.share_grid ? 2 : 0));
+  using K = void (*)(const DecodeParams);
+  K kern;
+  if (DENSE) {
+    kern = decode_kernel<G, DENSE, false, 0>;
+  } else if (cap) {
+    kern = var == 0 ? decode_kernel<G, DENSE, !DENSE, 0>
+         : var == 1 ? decode_kernel<G, DENSE, !DENSE, 1>
+         : var == 2 ? decode_kernel<G, DENSE, !DENSE, 2>
+                    : decode_kernel<G, DENSE, !DENSE, 3>;
+  } else {
+    kern = var == 0 ? decode_kernel<G, DENSE, false, 0>
+         : var == 1 ? decode_kernel<G, DENSE, false, 1>
+         : var == 2 ? decode_kernel<G, DENSE, false, 2>
+                    : decode_kernel<G, DENSE, false, 3>;
+  }
+  const int vi = (cap ? 1 : 0) + 2 * var;
   // The shared-memory opt-in is set once per device, variant and size
   // (outside any stream capture: the first call is expected to be eager).
-  static size_t configured[4][64] = {};
+  static size_t configured[8][64] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;

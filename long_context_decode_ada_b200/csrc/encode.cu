@@ -76,13 +76,16 @@ __device__ __forceinline__ uint32_t rho_code3(long long mx, long long my, u128 R
   return c;
 }
 
-__device__ __forceinline__ uint32_t rho_code(long long mx, long long my, u128 R2) {
+// 2-bit share code: how many thresholds u = (rho / r) sqrt(d/2) exceeds.
+// Uniform grid: u > {0.75, 1.25, 1.75}, i.e. 16 (d/2) rho^2 > {9, 25, 49} R2;
+// Lloyd-Max grid: u^2 > {22, 64, 145} / 64, i.e. 64 (d/2) rho^2 > {22, 64, 145} R2.
+__device__ __forceinline__ uint32_t rho_code(long long mx, long long my, u128 R2, int grid) {
   const u128 ax = (u128)(mx < 0 ? -mx : mx), ay = (u128)(my < 0 ? -my : my);
-  const u128 lhs = (ax * ax + ay * ay) * (u128)(16 * (kHeadDim / 2));
+  const u128 lhs = (ax * ax + ay * ay) * (u128)((grid ? 64 : 16) * (kHeadDim / 2));
   uint32_t c = 0;
-  c += lhs > (u128)9 * R2;
-  c += lhs > (u128)25 * R2;
-  c += lhs > (u128)49 * R2;
+  c += lhs > (u128)(grid ? 22 : 9) * R2;
+  c += lhs > (u128)(grid ? 64 : 25) * R2;
+  c += lhs > (u128)(grid ? 145 : 49) * R2;
   return c;
 }
 
@@ -202,8 +205,8 @@ __global__ void __launch_bounds__(256) encode_kernel(const __grid_constant__ Enc
   const float* by = t1 ? (v53 ? sby5 : sby6) : sby4;
   const uint32_t th0 = angle_code(k4[0], k4[1], bits, bx, by);
   const uint32_t th1 = angle_code(k4[2], k4[3], bits, bx, by);
-  const uint32_t rh0 = v53 ? rho_code3(m[0], m[1], R2) : rho_code(m[0], m[1], R2);
-  const uint32_t rh1 = v53 ? rho_code3(m[2], m[3], R2) : rho_code(m[2], m[3], R2);
+  const uint32_t rh0 = v53 ? rho_code3(m[0], m[1], R2) : rho_code(m[0], m[1], R2, p.share_grid);
+  const uint32_t rh1 = v53 ? rho_code3(m[2], m[3], R2) : rho_code(m[2], m[3], R2, p.share_grid);
   const uint32_t packed = th0 | (th1 << 8) | (rh0 << 16) | (rh1 << 24);
 
   // ---- V quantiser

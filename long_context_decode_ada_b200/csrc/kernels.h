@@ -34,6 +34,7 @@ struct DecodeParams {
   float cos6[64], sin6[64], cos4[16], sin4[16];
   float cos5[32], sin5[32];  // angles of the T1 variant (5-bit angle + 3-bit share)
   int t1_scheme;             // T1 code byte: 0 (angle6 << 2) | share2; 1 (angle5 << 3) | share3
+  int share_grid;            // 2-bit share grid: 0 uniform, 1 Lloyd-Max
 };
 
 struct EncodeParams {
@@ -56,6 +57,7 @@ struct EncodeParams {
   float bx6[64], by6[64], bx4[16], by4[16];
   float bx5[32], by5[32];
   int t1_scheme;        // 0: 6-bit angle + 2-bit share; 1: 5-bit angle + 3-bit share
+  int share_grid;       // 2-bit share grid: 0 uniform, 1 Lloyd-Max
 };
 
 // Decode-time append of one token per sequence (every kv head) as T0.

@@ -43,7 +43,7 @@ EXPORTS = [
 class SkvConfig(C.Structure):
     _fields_ = [("head_dim", C.c_int32), ("page_size", C.c_int32),
                 ("outlier_protect", C.c_int32), ("t1_angle_bits", C.c_int32),
-                ("reserved", C.c_int32 * 4)]
+                ("share_grid", C.c_int32), ("reserved", C.c_int32 * 3)]
 
 
 class SkvPools(C.Structure):
@@ -137,9 +137,10 @@ class Context:
     """An skv_ctx: head_dim 128, page size P; bound to the current device."""
 
     def __init__(self, page_size: int, head_dim: int = 128, outlier_protect: bool = False,
-                 t1_angle_bits: int = 6):
+                 t1_angle_bits: int = 6, share_grid: int = 0):
         cfg = SkvConfig(head_dim=head_dim, page_size=page_size,
-                        outlier_protect=1 if outlier_protect else 0, t1_angle_bits=t1_angle_bits)
+                        outlier_protect=1 if outlier_protect else 0, t1_angle_bits=t1_angle_bits,
+                        share_grid=share_grid)
         h = C.c_void_p()
         _check(lib().skv_create(C.byref(cfg), C.byref(h)))
         self._h = h
@@ -147,6 +148,7 @@ class Context:
         self.d = head_dim
         self.outlier_protect = bool(outlier_protect)
         self.t1_angle_bits = t1_angle_bits
+        self.share_grid = share_grid
 
     def __del__(self):
         h = getattr(self, "_h", None)

@@ -51,11 +51,14 @@ def test_tables_match_oracle_bytes():
     assert ctx.table(skv.TABLE_BOUNDARY5_Y, 32).tobytes() == by5.tobytes()
 
 
-def test_t1_angle_bits_is_checked():
+def test_t1_angle_bits_and_share_grid_are_checked():
     skv.Context(16, t1_angle_bits=5)
     skv.Context(16, t1_angle_bits=6)
+    skv.Context(16, share_grid=1)
     with pytest.raises(skv.SkvError):
         skv.Context(16, t1_angle_bits=4)
+    with pytest.raises(skv.SkvError):
+        skv.Context(16, share_grid=2)
 
 
 @pytest.mark.parametrize("P", [16, 32, 64])

@@ -1,7 +1,9 @@
-"""The T1 variant (skv_config.t1_angle_bits = 5: 5-bit angle + 3-bit share,
-the same code byte) against the oracle's variant scheme: the page bytes
-bit for bit, and the decode within tolerance; and, against exact fp16
-attention, a lower output error than the pinned 6 + 2 scheme."""
+"""The code variants against the oracle's matching schemes: the T1 variant
+(skv_config.t1_angle_bits = 5: 5-bit angle + 3-bit share, the same code
+byte) and the Lloyd-Max 2-bit share grid (skv_config.share_grid = 1), alone
+and together: the page bytes bit for bit, and the decode within tolerance;
+and, against exact fp16 attention, a lower output error than the pinned
+6 + 2 scheme."""
 import numpy as np
 import pytest
 import torch
@@ -14,8 +16,8 @@ from _gpu import assert_close, compare_store
 pytestmark = pytest.mark.gpu
 
 
-def run(w, bits, num_splits=0):
-    ctx = skv.Context(w.P, t1_angle_bits=bits)
+def run(w, bits, num_splits=0, grid=0):
+    ctx = skv.Context(w.P, t1_angle_bits=bits, share_grid=grid)
     dev = skv.workload_to_device(w)
     cache = skv.build_cache(ctx, w, dev)
     cache.check()
@@ -83,3 +85,29 @@ def test_variant_long_context_128k_full_size():
     b, h = rows[:, 0], rows[:, 1]
     assert_close(g["out"][b, h], ro[b, h], "out (sampled rows)")
     assert_close(g["lse"][b, h], rl[b, h], "lse (sampled rows)")
+
+
+@pytest.mark.parametrize("bits", [6, 5])
+def test_lloyd_max_share_grid_against_oracle(bits):
+    lens = [700, 260]
+    w = wl.custom(76, 2, 2, 4, 16, lens, wl.MODE_QUOTA,
+                  quota=[[T // 8, T // 3, T // 3] for T in lens])
+    g = run(w, bits, grid=1)
+    with oracle.t1_scheme(1 if bits == 5 else 0), oracle.share_grid(1):
+        ref = oracle.run_workload(w)
+    compare_store(w, g, ref)
+    assert_close(g["out"], ref["out"], "out")
+    assert_close(g["lse"], ref["lse"], "lse")
+
+
+def test_lloyd_max_grid_lowers_the_t2_error():
+    lens = [2048]
+    w = wl.custom(77, 1, 4, 4, 64, lens, wl.MODE_QUOTA, quota=[[0, 0, 2048]])
+    exact = np.zeros((1, w.Hkv, w.Tmax), np.uint8)
+    eo, el = oracle.decode(w.B, w.Hq, w.Hkv, w.Tmax, w.d, w.seq_lens, w.K, w.V, exact, w.q,
+                           w.q_dtype)
+    errs = {}
+    for grid in (0, 1):
+        g = run(w, 6, grid=grid)
+        errs[grid] = float(np.sqrt(np.mean((g["out"] - eo) ** 2)))
+    assert errs[1] < errs[0], errs
