@@ -261,6 +261,14 @@ int skv_append(skv_ctx* ctx, const uint16_t* K_new, const uint16_t* V_new, int B
               (a unit without resident tokens gives out 0, lse -inf)
      num_splits  number of page runs = CTAs (0 = default: the SM count)
      workspace   skv_workspace_size(SKV_WS_DECODE, ..., num_splits) bytes
+   Stream order: the decode is launched as a programmatic dependent of the
+   stream's previous kernel.  If that kernel lets its dependents start
+   early (griddepcontrol.launch_dependents, as this library's merge and
+   utility kernels do), the decode may read the page table and the pages
+   before that kernel has finished; it reads q and writes out, lse,
+   workspace and err_word only after it has.  So a kernel that writes the
+   store must not let its dependents start early (none in this library
+   does); q and the outputs follow ordinary stream order.
    Device errors: SKV_ERR_CORRUPT (bad page id / header: the page is
    skipped), SKV_ERR_TIMEOUT (a bounded wait ran out). */
 int skv_decode_attention(skv_ctx* ctx, const void* q, int q_dtype, int B, int Hq, int Hkv,
