@@ -265,8 +265,9 @@ int skv_append(skv_ctx* ctx, const uint16_t* K_new, const uint16_t* V_new, int B
    stream's previous kernel.  If that kernel lets its dependents start
    early (griddepcontrol.launch_dependents, as this library's merge and
    utility kernels do), the decode may read the page table and the pages
-   before that kernel has finished; it reads q and writes out, lse,
-   workspace and err_word only after it has.  So a kernel that writes the
+   before that kernel has finished; it reads q and writes out, lse and
+   the workspace only after it has (a corrupt page id may be reported into
+   err_word, atomically, before).  So a kernel that writes the
    store must not let its dependents start early (none in this library
    does); q and the outputs follow ordinary stream order.
    Device errors: SKV_ERR_CORRUPT (bad page id / header: the page is
