@@ -1396,7 +1396,32 @@ __global__ void __launch_bounds__(G * kHeadDim / 2)
 // decode's results.  The unit's lse goes through shared memory: one load
 // per block, not one per thread (the same 16 bytes requested by every
 // thread would queue at a single L2 slice).
-template <int G>
+// One chunk of V consecutive positions of unit u: tier, row map and old
+// utility (vector loads when V = 4: Tmax % 4 == 0 and the arrays aligned).
+template <int V>
+struct UtilChunk {
+  uint32_t tr[V];
+  int loc[V];
+  float u_old[V];
+};
+
+template <int V>
+__device__ __forceinline__ void load_chunk(const UtilityParams& p, long long at, UtilChunk<V>& c) {
+  if constexpr (V == 4) {
+    const uchar4 t = *reinterpret_cast<const uchar4*>(p.tier + at);
+    const int4 l = *reinterpret_cast<const int4*>(p.row_of + at);
+    const float4 u = *reinterpret_cast<const float4*>(p.utility + at);
+    c.tr[0] = t.x; c.tr[1] = t.y; c.tr[2] = t.z; c.tr[3] = t.w;
+    c.loc[0] = l.x; c.loc[1] = l.y; c.loc[2] = l.z; c.loc[3] = l.w;
+    c.u_old[0] = u.x; c.u_old[1] = u.y; c.u_old[2] = u.z; c.u_old[3] = u.w;
+  } else {
+    c.tr[0] = p.tier[at];
+    c.loc[0] = p.row_of[at];
+    c.u_old[0] = p.utility[at];
+  }
+}
+
+template <int G, int V>
 __global__ void __launch_bounds__(256) utility_kernel(const UtilityParams p) {
   constexpr float kLog2e = 1.4426950408889634f;
   __shared__ float ls_s[G];
@@ -1409,16 +1434,11 @@ __global__ void __launch_bounds__(256) utility_kernel(const UtilityParams p) {
   bool waited = false;
   for (int u = blockIdx.y; u < U; u += gridDim.y) {
     const int len = min(T, p.seq_lens[u / p.Hkv]);
+    const int nch = (len + V - 1) / V;  // chunks of V positions
     const long long base = (long long)u * T;
-    const int t0 = blockIdx.x * blockDim.x + threadIdx.x;
-    uint32_t tr = SKV_TIER_DROP;
-    int loc = -1;
-    float u_old = 0.0f;
-    if (t0 < len) {
-      tr = p.tier[base + t0];
-      loc = p.row_of[base + t0];
-      u_old = p.utility[base + t0];
-    }
+    const int c0 = blockIdx.x * blockDim.x + threadIdx.x;
+    UtilChunk<V> ch;
+    if (c0 < nch) load_chunk<V>(p, base + (long long)c0 * V, ch);
     if (!waited) {  // uniform: every thread of the block takes it on the first unit
       asm volatile("griddepcontrol.wait;" ::: "memory");
       waited = true;
@@ -1430,34 +1450,56 @@ __global__ void __launch_bounds__(256) utility_kernel(const UtilityParams p) {
 #pragma unroll
     for (int g = 0; g < G; ++g) ls2[g] = ls_s[g];
     const long long r0 = (long long)p.indptr[u] * p.P, r1 = (long long)p.indptr[u + 1] * p.P;
-    for (int t = t0; t < len; t += gridDim.x * blockDim.x) {
-      if (t != t0) {
-        tr = p.tier[base + t];
-        loc = p.row_of[base + t];
-        u_old = p.utility[base + t];
-      }
-      float mass = 0.0f;
-      if (tr != SKV_TIER_DROP) {
-        const long long gr = r0 + loc;
-        if (tr > SKV_TIER_DROP || loc < 0 || gr >= r1 || gr >= p.logit_rows) {
-          report(p.err, SKV_ERR_CORRUPT);
+    for (int ci = c0; ci < nch; ci += gridDim.x * blockDim.x) {
+      if (ci != c0) load_chunk<V>(p, base + (long long)ci * V, ch);
+      // every resident position's logits are loaded before any is used
+      float lv[V][G];
+      bool live[V];
+#pragma unroll
+      for (int v = 0; v < V; ++v) {
+        const int t = ci * V + v;
+        const uint32_t tr = ch.tr[v];
+        live[v] = t < len && tr != SKV_TIER_DROP;
+#pragma unroll
+        for (int g = 0; g < G; ++g) lv[v][g] = 0.0f;
+        if (!live[v]) continue;
+        const long long gr = r0 + ch.loc[v];
+        if (tr > SKV_TIER_DROP || ch.loc[v] < 0 || gr >= r1 || gr >= p.logit_rows) {
+          report(p.err, SKV_ERR_CORRUPT);  // the position keeps its old utility
+          live[v] = false;
           continue;
         }
         const float* l = p.logits + gr * G;
-        float lv[G];
         if constexpr (G == 4) {
           const float4 x = __ldcg(reinterpret_cast<const float4*>(l));
-          lv[0] = x.x; lv[1] = x.y; lv[2] = x.z; lv[3] = x.w;
+          lv[v][0] = x.x; lv[v][1] = x.y; lv[v][2] = x.z; lv[v][3] = x.w;
         } else if constexpr (G == 2) {
           const float2 x = __ldcg(reinterpret_cast<const float2*>(l));
-          lv[0] = x.x; lv[1] = x.y;
+          lv[v][0] = x.x; lv[v][1] = x.y;
         } else {
-          lv[0] = __ldcg(l);
+          lv[v][0] = __ldcg(l);
         }
-#pragma unroll
-        for (int g = 0; g < G; ++g) mass += exp2f(lv[g] - ls2[g]);
       }
-      p.utility[base + t] = p.gamma * u_old + mass;
+      float un[V];
+#pragma unroll
+      for (int v = 0; v < V; ++v) {
+        const int t = ci * V + v;
+        un[v] = ch.u_old[v];
+        if (t >= len) continue;  // past the sequence: unchanged
+        float mass = 0.0f;
+        if (live[v]) {
+#pragma unroll
+          for (int g = 0; g < G; ++g) mass += exp2f(lv[v][g] - ls2[g]);
+        } else if (ch.tr[v] != SKV_TIER_DROP) {
+          continue;  // a corrupt row: unchanged
+        }
+        un[v] = p.gamma * ch.u_old[v] + mass;
+      }
+      if constexpr (V == 4)
+        *reinterpret_cast<float4*>(p.utility + base + (long long)ci * 4) =
+            make_float4(un[0], un[1], un[2], un[3]);
+      else
+        p.utility[base + ci] = un[0];
     }
   }
 }
@@ -1466,9 +1508,14 @@ cudaError_t launch_utility(const UtilityParams& p, cudaStream_t stream) {
   const long long U = (long long)p.B * p.Hkv;
   if (U == 0 || p.Tmax == 0) return cudaSuccess;
   if (p.Tmax > (1LL << 30)) return cudaErrorInvalidValue;
+  // four positions per thread when the rows of four are aligned vectors
+  const bool vec = p.Tmax % 4 == 0 && (reinterpret_cast<uintptr_t>(p.tier) & 3) == 0 &&
+                   (reinterpret_cast<uintptr_t>(p.row_of) & 15) == 0 &&
+                   (reinterpret_cast<uintptr_t>(p.utility) & 15) == 0;
+  const long long V = vec ? 4 : 1;
   // about 2 waves of 256-thread blocks over all units, at least one block per unit
   const long long per_unit = std::max<long long>(1, (148LL * 8 * 2 + U - 1) / U);
-  const long long bx = std::min<long long>((p.Tmax + 255) / 256, per_unit);
+  const long long bx = std::min<long long>((p.Tmax + 256 * V - 1) / (256 * V), per_unit);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)bx, (unsigned)std::min<long long>(U, 65535));
   cfg.blockDim = dim3(256);
@@ -1479,10 +1526,18 @@ cudaError_t launch_utility(const UtilityParams& p, cudaStream_t stream) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  if (vec) {
+    switch (p.G) {
+      case 1: return cudaLaunchKernelEx(&cfg, utility_kernel<1, 4>, p);
+      case 2: return cudaLaunchKernelEx(&cfg, utility_kernel<2, 4>, p);
+      case 4: return cudaLaunchKernelEx(&cfg, utility_kernel<4, 4>, p);
+      default: return cudaErrorInvalidValue;
+    }
+  }
   switch (p.G) {
-    case 1: return cudaLaunchKernelEx(&cfg, utility_kernel<1>, p);
-    case 2: return cudaLaunchKernelEx(&cfg, utility_kernel<2>, p);
-    case 4: return cudaLaunchKernelEx(&cfg, utility_kernel<4>, p);
+    case 1: return cudaLaunchKernelEx(&cfg, utility_kernel<1, 1>, p);
+    case 2: return cudaLaunchKernelEx(&cfg, utility_kernel<2, 1>, p);
+    case 4: return cudaLaunchKernelEx(&cfg, utility_kernel<4, 1>, p);
     default: return cudaErrorInvalidValue;
   }
 }
