@@ -128,6 +128,36 @@ def _ptr(t: Optional[torch.Tensor]):
     return C.c_void_p(t.data_ptr())
 
 
+def _expect(t: torch.Tensor, name: str, numel: int, elem_size: int,
+            dtype: Optional[torch.dtype] = None, cuda: bool = True):
+    """Argument check before a pointer crosses the C-ABI (which cannot see
+    shapes): device, contiguity, element size or dtype, and element count."""
+    if not isinstance(t, torch.Tensor):
+        raise SkvError(SKV_ERR_ARG, f"{name}: a tensor is required")
+    if cuda and not t.is_cuda:
+        raise SkvError(SKV_ERR_ARG, f"{name}: must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise SkvError(SKV_ERR_ARG, f"{name}: must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise SkvError(SKV_ERR_ARG, f"{name}: dtype {t.dtype}, expected {dtype}")
+    if t.element_size() != elem_size:
+        raise SkvError(SKV_ERR_ARG, f"{name}: {t.element_size()}-byte elements, expected {elem_size}")
+    if t.numel() != numel:
+        raise SkvError(SKV_ERR_ARG, f"{name}: {t.numel()} elements, expected {numel}")
+
+
+def _decode_buffers(B: int, Hq: int, d: int, q, out, lse, device):
+    """The decode's q check and its out / lse, allocated or checked."""
+    _expect(q, "q", B * Hq * d, 2)
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=torch.float32, device=device)
+    if lse is None:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=device)
+    _expect(out, "out", B * Hq * d, 4, torch.float32)
+    _expect(lse, "lse", B * Hq, 4, torch.float32)
+    return out, lse
+
+
 def _stream(stream=None):
     s = stream if stream is not None else torch.cuda.current_stream()
     return C.c_void_p(s.cuda_stream)
@@ -273,10 +303,7 @@ class PagedCache:
 
     def decode(self, q: torch.Tensor, q_dtype: int, Hq: int, out=None, lse=None,
                workspace=None, num_splits: int = 0, stream=None):
-        if out is None:
-            out = torch.empty((self.B, Hq, self.ctx.d), dtype=torch.float32, device=self.device)
-        if lse is None:
-            lse = torch.empty((self.B, Hq), dtype=torch.float32, device=self.device)
+        out, lse = _decode_buffers(self.B, Hq, self.ctx.d, q, out, lse, self.device)
         if workspace is None:
             workspace = self.workspace(Hq, num_splits)
         _check(lib().skv_decode_attention(
@@ -299,10 +326,7 @@ class PagedCache:
         if utility.dtype != torch.float32 or tuple(utility.shape) != (self.B, self.Hkv, self.Tmax) \
                 or not utility.is_contiguous():
             raise SkvError(SKV_ERR_ARG, "utility must be contiguous fp32 [B][Hkv][Tmax]")
-        if out is None:
-            out = torch.empty((self.B, Hq, self.ctx.d), dtype=torch.float32, device=self.device)
-        if lse is None:
-            lse = torch.empty((self.B, Hq), dtype=torch.float32, device=self.device)
+        out, lse = _decode_buffers(self.B, Hq, self.ctx.d, q, out, lse, self.device)
         if workspace is None:
             workspace = self.utility_workspace(Hq, num_splits)
         _check(lib().skv_decode_utility(
@@ -327,6 +351,13 @@ class PagedCache:
             if t.is_cuda != dev_side or not t.is_contiguous():
                 raise SkvError(SKV_ERR_ARG, "decode_host: host tensors on the host, scratch on "
                                             "the device, all contiguous")
+        n = self.B * Hq * self.ctx.d
+        for t, name in ((q_host, "q_host"), (q_dev, "q_dev")):
+            _expect(t, name, n, 2, cuda=False)
+        for t, name in ((out_host, "out_host"), (out_dev, "out_dev")):
+            _expect(t, name, n, 4, torch.float32, cuda=False)
+        for t, name in ((lse_host, "lse_host"), (lse_dev, "lse_dev")):
+            _expect(t, name, self.B * Hq, 4, torch.float32, cuda=False)
         if workspace is None:
             workspace = self.workspace(Hq, num_splits)
         _check(lib().skv_decode_attention_host(
@@ -341,10 +372,7 @@ class PagedCache:
                       num_splits: int = 0, stream=None):
         """decode() with the library's fixed scratch instead of a workspace
         (skv_decode_attention_static: calls must not overlap in time)."""
-        if out is None:
-            out = torch.empty((self.B, Hq, self.ctx.d), dtype=torch.float32, device=self.device)
-        if lse is None:
-            lse = torch.empty((self.B, Hq), dtype=torch.float32, device=self.device)
+        out, lse = _decode_buffers(self.B, Hq, self.ctx.d, q, out, lse, self.device)
         _check(lib().skv_decode_attention_static(
             self.ctx.handle, _ptr(q), q_dtype, self.B, Hq, self.Hkv, _ptr(self.page_indptr),
             _ptr(self.page_tier_indptr) if self.split_by_bytes else None,
@@ -396,10 +424,7 @@ class DenseCache:
 
     def decode(self, q, q_dtype, Hq, out=None, lse=None, workspace=None, num_splits=0,
                stream=None):
-        if out is None:
-            out = torch.empty((self.B, Hq, self.ctx.d), dtype=torch.float32, device=self.device)
-        if lse is None:
-            lse = torch.empty((self.B, Hq), dtype=torch.float32, device=self.device)
+        out, lse = _decode_buffers(self.B, Hq, self.ctx.d, q, out, lse, self.device)
         if workspace is None:
             workspace = self.workspace(Hq, num_splits)
         _check(lib().skv_dense_decode_bf16(

@@ -8,6 +8,7 @@ import re
 
 import numpy as np
 import pytest
+import torch
 
 import oracle
 from long_context_decode_ada_b200 import skv
@@ -128,3 +129,19 @@ def test_decode_utility_argument_errors_without_gpu():
     rc = L.skv_decode_utility(ctx.handle, None, 0, 0, 8, 4, None, None, None, 10, C.byref(pools),
                               8, None, None, None, 1.0, None, None, None, None, None, 0, 0, None)
     assert rc == skv.SKV_OK
+
+
+def test_binding_checks_buffers_before_the_c_abi():
+    # the C-ABI takes plain pointers; the binding checks what it can see
+    q = torch.zeros((2, 8, 128), dtype=torch.float16)
+    skv._expect(q, "q", 2 * 8 * 128, 2, cuda=False)
+    with pytest.raises(skv.SkvError):
+        skv._expect(q, "q", 2 * 8 * 128 + 1, 2, cuda=False)          # wrong count
+    with pytest.raises(skv.SkvError):
+        skv._expect(q.float(), "q", 2 * 8 * 128, 2, cuda=False)      # wrong element size
+    with pytest.raises(skv.SkvError):
+        skv._expect(q[:, :, ::2], "q", 2 * 8 * 64, 2, cuda=False)    # not contiguous
+    with pytest.raises(skv.SkvError):
+        skv._expect(q, "q", 2 * 8 * 128, 2, cuda=True)               # not on the device
+    with pytest.raises(skv.SkvError):
+        skv._expect(torch.zeros(4, dtype=torch.int32), "lse", 4, 4, torch.float32, cuda=False)
