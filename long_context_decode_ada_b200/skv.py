@@ -158,6 +158,28 @@ def _decode_buffers(B: int, Hq: int, d: int, q, out, lse, device):
     return out, lse
 
 
+def _check_ingest(B: int, Hkv: int, Tmax: int, d: int, K=None, V=None, seq_lens=None,
+                  utility=None, protect=None, budget=None, quota=None, cuda: bool = True):
+    """The allocate / encode inputs that are given: K, V fp16 [B][Hkv][Tmax][d],
+    seq_lens int32 [B], utility fp32 and protect uint8 [B][Hkv][Tmax], budget
+    int64 [B], quota int32 [B][3]."""
+    n = B * Hkv * Tmax
+    if K is not None:
+        _expect(K, "K", n * d, 2, cuda=cuda)
+    if V is not None:
+        _expect(V, "V", n * d, 2, cuda=cuda)
+    if seq_lens is not None:
+        _expect(seq_lens, "seq_lens", B, 4, torch.int32, cuda=cuda)
+    if utility is not None:
+        _expect(utility, "utility", n, 4, torch.float32, cuda=cuda)
+    if protect is not None:
+        _expect(protect, "protect", n, 1, cuda=cuda)
+    if budget is not None:
+        _expect(budget, "budget", B, 8, torch.int64, cuda=cuda)
+    if quota is not None:
+        _expect(quota, "quota", 3 * B, 4, torch.int32, cuda=cuda)
+
+
 def _stream(stream=None):
     s = stream if stream is not None else torch.cuda.current_stream()
     return C.c_void_p(s.cuda_stream)
@@ -255,6 +277,8 @@ class PagedCache:
 
     def allocate(self, K, seq_lens, utility, protect, mode, budget, quota, free_lists,
                  stream=None):
+        _check_ingest(self.B, self.Hkv, self.Tmax, self.ctx.d, K=K, seq_lens=seq_lens,
+                      utility=utility, protect=protect, budget=budget, quota=quota)
         self._free0_cursor = None  # append() restarts after the slots this call takes
         fl = SkvFreeLists()
         self._free = [f.to(self.device, dtype=torch.int32) if isinstance(f, torch.Tensor) else
@@ -276,6 +300,9 @@ class PagedCache:
         T0 (skv_append) and advance seq_lens.  K_new, V_new: fp16
         [B][Hkv][128].  The T0 free list is the one given to allocate();
         its cursor starts after the slots allocate took."""
+        _expect(K_new, "K_new", self.B * self.Hkv * self.ctx.d, 2)
+        _expect(V_new, "V_new", self.B * self.Hkv * self.ctx.d, 2)
+        _expect(seq_lens, "seq_lens", self.B, 4, torch.int32)
         if getattr(self, "_free0_cursor", None) is None:
             tip = self.page_tier_indptr
             U = self.B * self.Hkv
@@ -292,6 +319,7 @@ class PagedCache:
             _ptr(self.err), _ptr(self._ws_append), self._ws_append.numel(), _stream(stream)))
 
     def encode(self, K, V, seq_lens, stream=None):
+        _check_ingest(self.B, self.Hkv, self.Tmax, self.ctx.d, K=K, V=V, seq_lens=seq_lens)
         _check(lib().skv_encode(
             self.ctx.handle, _ptr(K), _ptr(V), self.B, self.Hkv, self.Tmax, _ptr(seq_lens),
             _ptr(self.tier), _ptr(self.row_of), _ptr(self.page_indptr), _ptr(self.page_ids),

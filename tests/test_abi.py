@@ -145,3 +145,29 @@ def test_binding_checks_buffers_before_the_c_abi():
         skv._expect(q, "q", 2 * 8 * 128, 2, cuda=True)               # not on the device
     with pytest.raises(skv.SkvError):
         skv._expect(torch.zeros(4, dtype=torch.int32), "lse", 4, 4, torch.float32, cuda=False)
+
+
+def test_ingest_checks_accept_the_test_workloads():
+    # the inputs every GPU test builds (workload_to_device), here on the CPU
+    from long_context_decode_ada_b200 import workloads as wl
+    cases = [
+        wl.custom(81, 1, 2, 4, 16, [200], wl.MODE_BUDGET, protect_sink=150, zipf_alpha=1.1,
+                  budget=[150 * 2 * 512]),
+        wl.custom(82, 1, 1, 4, 16, [200], wl.MODE_QUOTA, quota=[[0, 200, 0]]),
+        wl.custom(93, 4, 2, 1, 16, [0, 40, 1, 77], wl.MODE_QUOTA,
+                  quota=[[0, 0, 0], [0, 1, 0], [0, 1, 0], [3, 30, 40]], q_dtype="fp16",
+                  utility=False),
+    ]
+    for w in cases:
+        d = skv.workload_to_device(w, "cpu")
+        skv._check_ingest(w.B, w.Hkv, w.Tmax, 128, K=d["K"], V=d["V"], seq_lens=d["seq_lens"],
+                          utility=d["utility"], protect=d["protect"], budget=d["budget"],
+                          quota=d["quota"], cuda=False)
+        skv._expect(d["q"], "q", w.B * w.Hq * 128, 2, cuda=False)
+        K_new = d["K"][:, :, 0].contiguous()
+        skv._expect(K_new, "K_new", w.B * w.Hkv * 128, 2, cuda=False)
+    with pytest.raises(skv.SkvError):
+        skv._check_ingest(1, 1, 4, 128, seq_lens=torch.zeros(1, dtype=torch.int64), cuda=False)
+    with pytest.raises(skv.SkvError):
+        skv._check_ingest(1, 1, 4, 128, K=torch.zeros((1, 1, 3, 128), dtype=torch.float16),
+                          cuda=False)
