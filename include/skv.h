@@ -291,7 +291,8 @@ int skv_decode_attention(skv_ctx* ctx, const void* q, int q_dtype, int B, int Hq
      other arguments as for skv_decode_attention (lse is required here)
    Returns SKV_OK, an argument / CUDA error, or the device error the step
    reported (SKV_ERR_CORRUPT, SKV_ERR_TIMEOUT).  Blocks the calling thread
-   until the step is done. */
+   until the step is done.  The context holds one pinned word for the error
+   copy: calls on one context from several host threads must not overlap. */
 int skv_decode_attention_host(skv_ctx* ctx, const void* q_host, int q_dtype, int B, int Hq,
                               int Hkv, const int32_t* page_indptr,
                               const int32_t* page_tier_indptr, const uint32_t* page_ids,

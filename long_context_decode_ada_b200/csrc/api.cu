@@ -529,10 +529,13 @@ int skv_decode_attention_host(skv_ctx* ctx, const void* q_host, int q_dtype, int
   if (!valid_pools(pools, 3)) return fail(SKV_ERR_ARG, "%s: bad pools", name);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e = cudaSuccess;
-  if (!ctx->err_host) {
-    e = cudaMallocHost(&ctx->err_host, sizeof(int32_t));
-    if (e != cudaSuccess) return cuda_fail(e, "skv_decode_attention_host: pinned error word");
-    *ctx->err_host = 0;
+  {
+    std::lock_guard<std::mutex> lock(g_scratch_mu);  // the first call allocates the word
+    if (!ctx->err_host) {
+      e = cudaMallocHost(&ctx->err_host, sizeof(int32_t));
+      if (e != cudaSuccess) return cuda_fail(e, "skv_decode_attention_host: pinned error word");
+      *ctx->err_host = 0;
+    }
   }
   const size_t qn = (size_t)B * Hq * 128 * 2, on = (size_t)B * Hq * 128 * 4, ln = (size_t)B * Hq * 4;
   e = cudaMemcpyAsync(q_dev, q_host, qn, cudaMemcpyHostToDevice, s);
