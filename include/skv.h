@@ -70,7 +70,7 @@ extern "C" {
 #define SKV_TABLE_BOUNDARY4_X 2  /* 16 fp32                                      */
 #define SKV_TABLE_BOUNDARY4_Y 3  /* 16 fp32                                      */
 #define SKV_TABLE_KAPPA 4        /* 3 fp32: RDR slope per byte of each step      */
-#define SKV_TABLE_RHO_LEVELS 5   /* 4 fp32: decoded share of each 2-bit code     */
+#define SKV_TABLE_RHO_LEVELS 5   /* 4 fp32: decoded share of each 2-bit code (the context's share grid) */
 #define SKV_TABLE_BOUNDARY5_X 6  /* 32 fp32: cos((j+1/2) 2pi/32)                */
 #define SKV_TABLE_BOUNDARY5_Y 7  /* 32 fp32: sin((j+1/2) 2pi/32)                */
 

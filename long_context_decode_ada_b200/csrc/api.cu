@@ -177,7 +177,10 @@ int skv_create(const skv_config* cfg, skv_ctx** out) {
   c->kappa[0] = (float)((1.0 - c4) / 180.0);
   c->kappa[1] = (float)((c4 - c6) / 16.0);
   c->kappa[2] = (float)(c6 / 316.0);
-  for (int k = 0; k < 4; ++k) c->rho_levels[k] = (float)((k + 1) / 16.0);
+  // decoded share of each 2-bit code: u_s / sqrt(d/2) on the context's grid
+  static const double kLevelsLM[4] = {383.0 / 1024, 807.0 / 1024, 1249.0 / 1024, 1831.0 / 1024};
+  for (int k = 0; k < 4; ++k)
+    c->rho_levels[k] = (float)(c->share_grid ? kLevelsLM[k] / 8.0 : (k + 1) / 16.0);
   const int rowb[4] = {512, 196, 180, 512};
   for (int t = 0; t < 4; ++t) {
     c->payload[t] = skv::kHdrBytes + (long long)P * rowb[t];

@@ -47,6 +47,9 @@ def test_tables_match_oracle_bytes():
     assert ctx.table(skv.TABLE_KAPPA, 3).tobytes() == oracle.kappa(128).tobytes()
     lv = ctx.table(skv.TABLE_RHO_LEVELS, 4)
     assert list(lv) == [oracle.rho_level(c, 128) for c in range(4)]
+    lm = skv.Context(64, share_grid=1).table(skv.TABLE_RHO_LEVELS, 4)
+    with oracle.share_grid(1):
+        np.testing.assert_allclose(lm, [oracle.rho_level(c, 128) for c in range(4)], rtol=1e-7)
     bx5, by5 = oracle.boundaries(5)
     assert ctx.table(skv.TABLE_BOUNDARY5_X, 32).tobytes() == bx5.tobytes()
     assert ctx.table(skv.TABLE_BOUNDARY5_Y, 32).tobytes() == by5.tobytes()
