@@ -14,7 +14,9 @@ does not enter the device timeline; two copies of the store alternate so the
 
 Under torchrun each rank (one GPU) decodes its own copy of the workload
 (independent sequences: weak scaling, no collective on the data path); the
-step time is the max over ranks.  --impl reference times the CPU oracle on a
+step time is the max over ranks.  `--gpus N` must match the launcher's
+WORLD_SIZE (a mismatch exits with status 2); without a launcher, N > 1
+re-runs the command under torch.distributed.run with N local processes.  --impl reference times the CPU oracle on a
 bounded sample of the same workload on the host cores (rank 0 only).
 """
 from __future__ import annotations
@@ -717,11 +719,41 @@ def run_cp(args, rank, world, local_rank):
         print(json.dumps(line), flush=True)
 
 
+def resolve_launch(gpus: int, env, argv):
+    """What `--gpus N` means for this process, from the launcher's environment.
+
+    - ("run", world, rank, local_rank): WORLD_SIZE is set and equals N (a
+      torchrun rank), or N = 1 without a launcher;
+    - ("spawn", cmd): N > 1 and no launcher: re-run this command under
+      torch.distributed.run with N processes on this node (127.0.0.1);
+    - ("error", message): WORLD_SIZE is set and differs from N, or N < 1.
+    The rank count and the reported n_gpus can therefore never disagree."""
+    if gpus < 1:
+        return ("error", f"--gpus must be >= 1 (got {gpus})")
+    if "WORLD_SIZE" in env:
+        world = int(env["WORLD_SIZE"])
+        if world != gpus:
+            return ("error", f"--gpus {gpus} but the launcher started {world} ranks "
+                             f"(WORLD_SIZE={world}); they must agree")
+        return ("run", world, int(env.get("RANK", "0")), int(env.get("LOCAL_RANK", "0")))
+    if gpus == 1:
+        return ("run", 1, 0, 0)
+    port = env.get("MASTER_PORT") or "29517"
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           f"--nproc-per-node={gpus}", "--master-addr=127.0.0.1", f"--master-port={port}",
+           os.path.abspath(__file__)] + list(argv)
+    return ("spawn", cmd)
+
+
 def main():
     args = parse_args()
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    how = resolve_launch(args.gpus, os.environ, sys.argv[1:])
+    if how[0] == "error":
+        print(f"bench.py: {how[1]}", file=sys.stderr)
+        sys.exit(2)
+    if how[0] == "spawn":
+        sys.exit(subprocess.call(how[1]))
+    _, world, rank, local_rank = how
     if args.impl == "reference":
         run_reference(args, rank, world)
         return

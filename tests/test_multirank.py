@@ -84,3 +84,36 @@ def test_reference_arm_prints_the_contract_line_on_rank_zero():
     assert line["impl"] == "reference" and line["value"] > 0
     assert line["metric"] == bench.METRIC and line["unit"] == bench.UNIT
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_gpus_flag_and_rank_count_cannot_disagree():
+    """--gpus N is honoured: a torchrun rank whose WORLD_SIZE differs from N
+    is an error, N > 1 without a launcher re-runs the command under
+    torch.distributed.run with N processes, N = 1 runs in place."""
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.resolve_launch(1, {}, []) == ("run", 1, 0, 0)
+    assert bench.resolve_launch(2, {"WORLD_SIZE": "2", "RANK": "1", "LOCAL_RANK": "1"},
+                                []) == ("run", 2, 1, 1)
+    how = bench.resolve_launch(8, {"WORLD_SIZE": "1"}, [])
+    assert how[0] == "error" and "WORLD_SIZE=1" in how[1]
+    how = bench.resolve_launch(1, {"WORLD_SIZE": "4", "RANK": "0"}, [])
+    assert how[0] == "error"
+    assert bench.resolve_launch(0, {}, [])[0] == "error"
+    how = bench.resolve_launch(4, {}, ["--gpus", "4", "--steps", "10"])
+    assert how[0] == "spawn"
+    cmd = how[1]
+    assert cmd[1:3] == ["-m", "torch.distributed.run"]
+    assert "--nproc-per-node=4" in cmd and "--master-addr=127.0.0.1" in cmd
+    assert cmd[-4:] == ["--gpus", "4", "--steps", "10"]
+
+
+def test_gpus_flag_mismatch_exits_nonzero_without_work():
+    """`bench.py --gpus 8` inside a one-rank launch refuses to run instead of
+    printing a line that says n_gpus 1."""
+    import subprocess
+    env = dict(os.environ, WORLD_SIZE="1", RANK="0", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "8"],
+                       env=env, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 2
+    assert r.stdout == "" and "--gpus 8" in r.stderr
