@@ -33,8 +33,8 @@
 // m16n8k16 with A = the rows' keys and B = the G query heads (fp32
 // accumulation): T0 / dense rows enter as they are stored (fp16 / bf16);
 // T1 / T2 rows are rebuilt from their codes by gathers from a constant
-// shared table of (share + 1) (cos, sin) per code, split into fp16 high and
-// low halves (two MMAs, fp32-level accuracy).  Lane (t, g) ends with the
+// shared table of (share + 1) (cos, sin) per code in fp16 (one 4-byte,
+// conflict-free gather per row and pair).  Lane (t, g) ends with the
 // logits of head g of rows t and t + 8.  P.V: mma.sync m16n8k16, A = V^T
 // fragments read straight from the page (pages store V in fragment order),
 // B = P of the 16 rows x 8 heads (zero-padded beyond G), fp32 accumulation.
@@ -80,11 +80,11 @@ constexpr int kMetaBadShift = 12;
 // Shared-memory plan: [ring][TBL1][TBL2][fixed block] (ADA) or
 // [ring][fixed block] (dense).  TBL1 / TBL2 are the reconstruction tables
 // of the T1 / T2 codes (see build_tables): entry e at table + 128 e holds
-// 16 copies of its 8 bytes, copy L % 16 read by lane L, so that a warp's
-// gathers of any entries are free of bank conflicts.  TBL2 starts on an
-// 8 KB boundary (its gather address is a LOP3 of the code bits and the
+// 32 copies of its 4 bytes, copy L read by lane L, so that a warp's
+// gathers of any entries are one conflict-free wavefront.  TBL2 starts on
+// an 8 KB boundary (its gather address is a LOP3 of the code bits and the
 // lane's base); TBL1 sits right below it and the ring below TBL1.
-constexpr uint32_t kTblEnt = 128;          // bytes per entry: 16 copies x 8 B
+constexpr uint32_t kTblEnt = 128;          // bytes per entry: 32 copies x 4 B
 constexpr uint32_t kTbl1 = 256 * kTblEnt;   // T1: entry = code byte (angle6 << 2) | share2
 constexpr uint32_t kTbl2 = 64 * kTblEnt;    // T2: entry = angle4 | share2 << 4
 
@@ -422,9 +422,11 @@ __device__ __forceinline__ void make_qfrag(const float (*q32)[kHeadDim], float q
 
 // Reconstruction tables: T1 entry e = (a << 2) | s and T2 entry 256 + (a | s << 4)
 // hold the pair (x, y) = (s + 1) (cos, sin)(2 pi a / 2^b) (16 times the
-// key pair of unit radius: shares enter as code + 1) as fp16 hi and lo
-// halves, x = hi + lo to about 2^-22 relative: {hi(x), hi(y)}, {lo(x), lo(y)}.
-// The T2 entries follow T1's (TBL2 = TBL1 + 32 KB).
+// key pair of unit radius: shares enter as code + 1) rounded to fp16
+// (relative error <= 2^-11 per component; the logit of a row is the
+// fp32-accumulated sum of exact fp16 x fp16 products).  The T2 entries
+// follow T1's (TBL2 = TBL1 + 32 KB).  Eight threads fill one entry's 128
+// bytes with 16-byte stores, so a warp writes 512 contiguous bytes.
 // VAR bit 0: the T1 variant, code byte (angle5 << 3) | share3 with weight
 // (s + 1) / 2; bit 1: the 2-bit share codes on the Lloyd-Max grid, weights
 // 2 u_s = {766, 1614, 2498, 3662} / 1024 instead of s + 1 (share u_s / 8).
@@ -439,7 +441,8 @@ __device__ __forceinline__ float share2_weight(uint32_t s) {
 template <int VAR>
 __device__ __forceinline__ void build_tables(const DecodeParams& p, uint8_t* tbl1p, int n_entries,
                                              int tid, int nthreads) {
-  for (int e = tid; e < n_entries; e += nthreads) {
+  for (int i = tid; i < 8 * n_entries; i += nthreads) {
+    const int e = i >> 3;
     float cs, sn, w;
     if ((VAR & 1) && e < 256) {
       cs = p.cos5[e >> 3];
@@ -455,13 +458,8 @@ __device__ __forceinline__ void build_tables(const DecodeParams& p, uint8_t* tbl
       w = share2_weight<VAR>((uint32_t)(e - 256) >> 4);
     }
     const float x = w * cs, y = w * sn;
-    const __half hx = __float2half_rn(x), hy = __float2half_rn(y);
-    const __half lx = __float2half_rn(x - __half2float(hx)), ly = __float2half_rn(y - __half2float(hy));
-    const uint32_t hi = (uint32_t)__half_as_ushort(hx) | ((uint32_t)__half_as_ushort(hy) << 16);
-    const uint32_t lo = (uint32_t)__half_as_ushort(lx) | ((uint32_t)__half_as_ushort(ly) << 16);
-    uint4* dst = reinterpret_cast<uint4*>(tbl1p + (size_t)e * kTblEnt);
-#pragma unroll
-    for (int r = 0; r < 8; ++r) dst[r] = make_uint4(hi, lo, hi, lo);
+    const uint32_t h = pack_f16x2(x, y);
+    reinterpret_cast<uint4*>(tbl1p)[i] = make_uint4(h, h, h, h);
   }
 }
 
@@ -503,8 +501,8 @@ __device__ __forceinline__ uint32_t t1_addr(uint32_t w, int k, uint32_t tb) {
 
 // T1 rows rA, rA + 8: lane (t, g) reads code bytes [16 g, 16 g + 16) of
 // each row; byte j holds pair 16 (j >> 2) + 4 g + (j & 3), so k-step s uses
-// bytes 2 s (k = 2 g, 2 g + 1) and 2 s + 1 (k = 2 g + 8, 2 g + 9).  hi and lo
-// table halves go to separate accumulators.
+// bytes 2 s (k = 2 g, 2 g + 1) and 2 s + 1 (k = 2 g + 8, 2 g + 9).  Even and
+// odd k-steps go to separate accumulators (two MMA chains of four).
 __device__ __forceinline__ void logits_t1(uint32_t pg, int P, int rA, int g, uint32_t tb,
                                           const QFrag& f, float (&c)[4], float (&d)[4]) {
   const uint32_t cd = pg + kHdrBytes + 2 * P;
@@ -515,10 +513,12 @@ __device__ __forceinline__ void logits_t1(uint32_t pg, int P, int rA, int g, uin
 #pragma unroll
   for (int s = 0; s < 8; ++s) {
     const int i = s >> 1, k0 = 2 * (s & 1);
-    const uint2 ea0 = lds64(t1_addr(wa[i], k0, tb)), ea1 = lds64(t1_addr(wa[i], k0 + 1, tb));
-    const uint2 eb0 = lds64(t1_addr(wb[i], k0, tb)), eb1 = lds64(t1_addr(wb[i], k0 + 1, tb));
-    mma_k16<false>(c, ea0.x, eb0.x, ea1.x, eb1.x, f.b[2 * s], f.b[2 * s + 1]);
-    mma_k16<false>(d, ea0.y, eb0.y, ea1.y, eb1.y, f.b[2 * s], f.b[2 * s + 1]);
+    const uint32_t ea0 = lds32(t1_addr(wa[i], k0, tb)), ea1 = lds32(t1_addr(wa[i], k0 + 1, tb));
+    const uint32_t eb0 = lds32(t1_addr(wb[i], k0, tb)), eb1 = lds32(t1_addr(wb[i], k0 + 1, tb));
+    if (s & 1)
+      mma_k16<false>(d, ea0, eb0, ea1, eb1, f.b[2 * s], f.b[2 * s + 1]);
+    else
+      mma_k16<false>(c, ea0, eb0, ea1, eb1, f.b[2 * s], f.b[2 * s + 1]);
   }
 }
 
@@ -545,12 +545,14 @@ __device__ __forceinline__ void logits_t2(uint32_t pg, int P, int rA, int g, uin
   const uint32_t rb = lds32(cd + (rA + 8) * 48 + 32 + 4 * g);
 #pragma unroll
   for (int s = 0; s < 8; ++s) {
-    const uint2 ea0 = lds64(t2_addr(na.x, na.y, ra, 2 * s, tb));
-    const uint2 ea1 = lds64(t2_addr(na.x, na.y, ra, 2 * s + 1, tb));
-    const uint2 eb0 = lds64(t2_addr(nb.x, nb.y, rb, 2 * s, tb));
-    const uint2 eb1 = lds64(t2_addr(nb.x, nb.y, rb, 2 * s + 1, tb));
-    mma_k16<false>(c, ea0.x, eb0.x, ea1.x, eb1.x, f.b[2 * s], f.b[2 * s + 1]);
-    mma_k16<false>(d, ea0.y, eb0.y, ea1.y, eb1.y, f.b[2 * s], f.b[2 * s + 1]);
+    const uint32_t ea0 = lds32(t2_addr(na.x, na.y, ra, 2 * s, tb));
+    const uint32_t ea1 = lds32(t2_addr(na.x, na.y, ra, 2 * s + 1, tb));
+    const uint32_t eb0 = lds32(t2_addr(nb.x, nb.y, rb, 2 * s, tb));
+    const uint32_t eb1 = lds32(t2_addr(nb.x, nb.y, rb, 2 * s + 1, tb));
+    if (s & 1)
+      mma_k16<false>(d, ea0, eb0, ea1, eb1, f.b[2 * s], f.b[2 * s + 1]);
+    else
+      mma_k16<false>(c, ea0, eb0, ea1, eb1, f.b[2 * s], f.b[2 * s + 1]);
   }
 }
 
@@ -1071,7 +1073,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   const int grp = warp / kGW, wi = warp % kGW;  // consumer group, warp within it
   // this lane's copy in the reconstruction tables; TBL1's space doubles as
   // the stash of the combine (then rebuilt before the next unit)
-  const uint32_t tb1 = tbl1 + (uint32_t)(lane & 15) * 8u, tb2 = tb1 + kTbl1;
+  const uint32_t tb1 = tbl1 + (uint32_t)lane * 4u, tb2 = tb1 + kTbl1;
   uint8_t* const tbl1p = smem_raw + (tbl1 - base);
   float* const stashp = reinterpret_cast<float*>(tbl1p);
   static_assert(DENSE || kNCW * 4 * kHeadDim * 4 <= (int)kTbl1, "combine stash fits TBL1");
