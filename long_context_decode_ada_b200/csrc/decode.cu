@@ -65,6 +65,7 @@ constexpr int kNSlot = 16;                    // items in flight, at most
 constexpr int kMaxIPP = kItemRows / 16;       // pages per item (P >= 16)
 constexpr int kMergeBatch = 20;               // merge: runs whose loads are issued together
 constexpr int kTouchedUnits = 16;             // units whose segment costs a CTA keeps
+constexpr int kStashRow = kHeadDim + 4;       // combine stash: floats per (warp, head) row
 static_assert(kCG >= 1 && kCG <= 4, "consumer groups: 1..4");
 static_assert(kIss >= 1 && kIss <= 4, "issuers: 1..4");
 static_assert(kPasses >= 1 && kGW * kRowsPerWarp == kItemRows, "warp row split");
@@ -114,6 +115,7 @@ struct __align__(16) DecodeSmem {
   __align__(16) float ml[kNCW][4][2];
   float wsc[kNCW][4];                   // combine: each warp's scale per head
   float MH[4], LH[4];                   // combine: this CTA's (M, L) per head
+  int c01[2];                           // the current unit's runs c0 .. c1
   __align__(16) float O[4][kHeadDim];
   __align__(16) float q32[4][kHeadDim];   // read with 16-byte shared loads
 };
@@ -170,6 +172,22 @@ struct SplitInfo {
   }
 };
 
+// floor(a / b) for b > 0.  Below 2^52 the quotient comes from one IEEE
+// double division (a and b convert exactly; the rounded quotient is off by
+// at most one) and is corrected with exact integer products, which keeps
+// the 64-bit integer division sequence off the start-up path.
+__device__ __forceinline__ unsigned long long udiv64(unsigned long long a, unsigned long long b) {
+  if (a < (1ull << 52) && b < (1ull << 52)) {
+    unsigned long long q = (unsigned long long)((double)a / (double)b);
+    if (q * b > a)
+      --q;
+    else if ((q + 1) * b <= a)
+      ++q;
+    return q;
+  }
+  return a / b;
+}
+
 // First page of the run that starts at cost target T (= run index x total)
 // among one unit's pages: seg[0..3] are the unit's tier segment starts,
 // cseg[0..3] the costs before them; clamped to [seg[0], seg[3]].
@@ -183,7 +201,7 @@ __device__ __forceinline__ long long run_begin_in_unit(const SplitInfo& si,
     if (T <= lo) return seg[t];
     if (T <= hi) {
       const unsigned long long ws = si.weight(t) * S;
-      return seg[t] + (long long)((T - lo + ws - 1) / ws);
+      return seg[t] + (long long)udiv64(T - lo + ws - 1, ws);
     }
   }
   return seg[3];
@@ -211,7 +229,7 @@ __host__ __device__ __forceinline__ bool unit_aligned_split(long long U, long lo
 __device__ __forceinline__ int unit_first_run(int u, unsigned long long Pu, unsigned long long C,
                                               int S, int U) {
   if (C == 0) return u;
-  return u + (int)((2ull * Pu * (unsigned long long)(S - U) + C) / (2ull * C));
+  return u + (int)udiv64(2ull * Pu * (unsigned long long)(S - U) + C, 2ull * C);
 }
 
 // This CTA's run [sm.run[0], sm.run[1]) (block-wide; contains barriers),
@@ -296,8 +314,8 @@ __device__ __noinline__ void find_run(const SplitInfo& si, int c, int S, Smem& s
       const long long a = si.seg_start(k), b = si.seg_start(k + 1);
       const unsigned long long ws = si.weight(k) * Su;
       const unsigned long long lo = cc * Su, hi = lo + (unsigned long long)(b - a) * ws;
-      if (lo < T0 && T0 <= hi) sm.run[0] = a + (long long)((T0 - lo + ws - 1) / ws);
-      if (lo < T1 && T1 <= hi) sm.run[1] = a + (long long)((T1 - lo + ws - 1) / ws);
+      if (lo < T0 && T0 <= hi) sm.run[0] = a + (long long)udiv64(T0 - lo + ws - 1, ws);
+      if (lo < T1 && T1 <= hi) sm.run[1] = a + (long long)udiv64(T1 - lo + ws - 1, ws);
       cc += (unsigned long long)(b - a) * si.weight(k);
     }
   }
@@ -835,9 +853,11 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       const long long pq = pg + (long long)lane * ipp + q;
       idn[q] = (q < ipp && pq < g1) ? __ldg(p.ids + pq) : 0u;
     }
-    long long ub = min(g1, (long long)p.indptr[u0 + 1]);  // end of the current unit's run
-    // the end of the next unit, loaded one unit ahead
-    long long ub_next = u0 + 2 <= U ? (long long)p.indptr[u0 + 2] : g1;
+    // end of the current unit's run and the end of the next unit, loaded
+    // one unit ahead (a unit-aligned run lies inside its unit: no loads)
+    const bool in_unit = unit_aligned_split(U, p.S);
+    long long ub = in_unit ? g1 : min(g1, (long long)p.indptr[u0 + 1]);
+    long long ub_next = (!in_unit && u0 + 2 <= U) ? (long long)p.indptr[u0 + 2] : g1;
     int it = 0;                 // next item
     int tail = 0;               // oldest item not known to be released
     uint32_t wr = 0;            // ring write offset
@@ -1076,7 +1096,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   const uint32_t tb1 = tbl1 + (uint32_t)lane * 4u, tb2 = tb1 + kTbl1;
   uint8_t* const tbl1p = smem_raw + (tbl1 - base);
   float* const stashp = reinterpret_cast<float*>(tbl1p);
-  static_assert(DENSE || kNCW * 4 * kHeadDim * 4 <= (int)kTbl1, "combine stash fits TBL1");
+  static_assert(DENSE || kNCW * 4 * kStashRow * 4 <= (int)kTbl1, "combine stash fits TBL1");
   // The decode may be a programmatic dependent of the previous step's grids
   // (launched while they finish).  The planner and the issuers start on the
   // page table and the pages at once: the store is never written by a grid
@@ -1106,7 +1126,17 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     const long long a = max(g0, iu0), b = min(g1, iu1);
     if (a >= b) continue;
     named_bar_sync(1, nct);
-    if (tid < 4) sm.useg[tid] = si.seg_start(3 * u + tid);  // for the merge, after the items
+    if (tid < 4) sm.useg[tid] = si.seg_start(3 * u + tid);
+    const bool many_units = sm.unit1 - sm.unit0 >= kTouchedUnits;
+    if (many_units) {
+      // many units in this run: the cost before unit u, summed afresh
+      unsigned long long part = 0;
+      for (int k = tid; k < 3 * u; k += nct)
+        part += (unsigned long long)(si.seg_start(k + 1) - si.seg_start(k)) * si.weight(k);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xFFFFFFFFu, part, o);
+      if (lane == 0) sm.scan[warp] = part;
+    }
 #pragma unroll
     for (int k = 0; k < kQPer; ++k) {
       const int i = tid + k * nct;
@@ -1114,7 +1144,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         const int h = i / kHeadDim, d = i % kHeadDim;
         sm.q32[h][d] = p.q_bf16 ? __bfloat162float(__ushort_as_bfloat16(qraw[k]))
                                 : __half2float(__ushort_as_half(qraw[k]));
-        sm.O[h][d] = 0.0f;
+        if constexpr (DENSE) sm.O[h][d] = 0.0f;
       }
     }
     if constexpr (!DENSE) {
@@ -1122,6 +1152,38 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       tbl_entries = 0;
     }
     named_bar_sync(1, nct);
+    if (tid == 0) {
+      // the runs that hold this unit's partials, c0 .. c1 (read by the
+      // combine, after its barriers): unit-aligned split, [B(u), B(u + 1));
+      // global split, the runs of u's first and last page, run c holding
+      // page g when floor(C(g) S / total) == c.  Computed now, while the
+      // first items are in flight, to keep the divisions off the tail.
+      unsigned long long cu[4];
+      if (!many_units) {
+#pragma unroll
+        for (int t = 0; t < 4; ++t) cu[t] = sm.ucost[3 * (u - sm.unit0) + t];
+      } else {
+        unsigned long long cb = 0;
+        for (int w2 = 0; w2 < kNCW; ++w2) cb += sm.scan[w2];
+        cu[0] = cb;
+#pragma unroll
+        for (int t = 0; t < 3; ++t)
+          cu[t + 1] = cu[t] + (unsigned long long)(sm.useg[t + 1] - sm.useg[t]) * si.weight(t);
+      }
+      const unsigned long long ctot = sm.ctot, Su = (unsigned long long)p.S;
+      int c0 = c, c1 = c;
+      if (unit_aligned_split(U, p.S)) {
+        c0 = unit_first_run(u, cu[0], ctot, p.S, U);
+        c1 = unit_first_run(u + 1, cu[3], ctot, p.S, U) - 1;
+      } else if (ctot > 0) {
+        int tl = 2;  // tier of the unit's last page
+        while (tl > 0 && sm.useg[tl] == iu1) --tl;
+        c0 = (int)udiv64(cu[0] * Su, ctot);
+        c1 = (int)udiv64((cu[3] - si.weight(tl)) * Su, ctot);
+      }
+      sm.c01[0] = c0;
+      sm.c01[1] = c1;
+    }
     QFrag qf;
     make_qfrag<G, DENSE>(sm.q32, p.qk_scale_log2, p.q_bf16 != 0, lane, qf);
     WarpState st;
@@ -1178,11 +1240,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     it += nitems;
 
     // ---- combine the warps' states into this CTA's partial for unit u.
-    // ADA: every warp writes its (m, l) per head and, once all warps are done
-    // with the tables, its unscaled accumulators to a stash (TBL1's space,
-    // rebuilt before the next unit); then each output element takes the
-    // warps' maximum, their weights 2^(m_w - M) and the weighted sum.  Dense (no
-    // tables): one thread per head forms M, L and the warps' scales, and the
+    // Every warp writes its (m, l) per head; one thread per head forms M,
+    // L and the warps' weights 2^(m_w - M).  ADA: the warps' unscaled
+    // accumulators go to a stash (TBL1's space, rebuilt before the next
+    // unit) and each output is their weighted sum.  Dense (no tables): the
     // warps add their scaled accumulators into O with shared atomics.
     float l = st.l;
     l += __shfl_xor_sync(0xFFFFFFFFu, l, 4);
@@ -1223,13 +1284,34 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       }
       named_bar_sync(1, nct);
     } else {
-      named_bar_sync(1, nct);  // every warp is done with the tables
+      // ADA: one thread per head forms M, L and the warps' scales while the
+      // warps stash their unscaled accumulators in TBL1's space (rows of
+      // kStashRow floats: the two heads a store instruction covers fall in
+      // different banks); then every output is a kNCW-term dot product of
+      // scales and stash, written straight to out or to the partial.
+      named_bar_sync(1, nct);  // every warp is done with the items and the tables
+      if (tid < G) {
+        const int n = tid;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kNCW; ++w) M = fmaxf(M, sm.ml[w][n][0]);
+        float L = 0.0f;
+#pragma unroll
+        for (int w = 0; w < kNCW; ++w) {
+          const float mw = sm.ml[w][n][0];
+          const float sc = (mw == -INFINITY) ? 0.0f : exp2f(mw - M);
+          sm.wsc[w][n] = sc;
+          L = fmaf(sm.ml[w][n][1], sc, L);
+        }
+        sm.MH[n] = M;
+        sm.LH[n] = M == -INFINITY ? 0.0f : L;
+      }
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
         const int n = 2 * t4 + j;
         if (n < G) {
           const float bias = 1152.0f * st.ones[j];  // int8 V offset (see softmax_pv)
-          float* stash = stashp + (warp * G + n) * kHeadDim;
+          float* stash = stashp + (warp * G + n) * kStashRow;
 #pragma unroll
           for (int mt = 0; mt < 8; ++mt) {
             stash[16 * mt + gq] = st.acc[mt][j] - bias;
@@ -1237,70 +1319,39 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
           }
         }
       }
-      named_bar_sync(1, nct);
-      for (int i = tid; i < G * kHeadDim; i += nct) {
-        const int n = i / kHeadDim, d = i % kHeadDim;
-        float M = -INFINITY;
-#pragma unroll
-        for (int w = 0; w < kNCW; ++w) M = fmaxf(M, sm.ml[w][n][0]);
-        float o = 0.0f, L = 0.0f;
-#pragma unroll
-        for (int w = 0; w < kNCW; ++w) {
-          const float mw = sm.ml[w][n][0];
-          const float sc = (mw == -INFINITY) ? 0.0f : exp2f(mw - M);
-          o = fmaf(stashp[(w * G + n) * kHeadDim + d], sc, o);
-          L = fmaf(sm.ml[w][n][1], sc, L);
-        }
-        sm.O[n][d] = o;
-        if (d == 0) {
-          sm.MH[n] = M;
-          sm.LH[n] = M == -INFINITY ? 0.0f : L;
-        }
-      }
       tbl_entries = 256;  // TBL1 holds the stash now
       named_bar_sync(1, nct);
-    }
-    // ---- this CTA's result for unit u.  A unit inside one run is finished
-    // here; otherwise every run from c0 to c1 writes its partial to slot
-    // c + u (an empty run an empty one, at the kernel's start) and
-    // decode_merge_kernel combines them once this grid has completed.  The
-    // CTA of run c0 records (c0, c1) for it.  Runs: unit-aligned split,
-    // [B(u), B(u + 1)); global split, run c holds page g when
-    // floor(C(g) S / total) == c, so the runs of u's first and last page.
-    // sm.useg holds u's tier segment starts (loaded at the unit's start).
-    if (sm.unit1 - sm.unit0 < kTouchedUnits) {
-      if (tid < 4) sm.cunit[tid] = sm.ucost[3 * (u - sm.unit0) + tid];
-    } else {
-      // many units in this run: the cost before unit u, summed afresh
-      unsigned long long part = 0;
-      for (int k = tid; k < 3 * u; k += nct)
-        part += (unsigned long long)(si.seg_start(k + 1) - si.seg_start(k)) * si.weight(k);
+      const int c0 = sm.c01[0], c1 = sm.c01[1];
+      const long long obase = (long long)bb * p.Hq + (long long)hkv * G;
+      float* part = p.part + (long long)(c + u) * G * kPartStride;
+      for (int i = tid; i < G * kHeadDim; i += nct) {
+        const int n = i / kHeadDim, d = i % kHeadDim;
+        float o = 0.0f;
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xFFFFFFFFu, part, o);
-      if (lane == 0) sm.scan[warp] = part;
-      named_bar_sync(1, nct);
-      if (tid == 0) {
-        unsigned long long cb = 0;
-        for (int w2 = 0; w2 < kNCW; ++w2) cb += sm.scan[w2];
-        sm.cunit[0] = cb;
-        for (int t = 0; t < 3; ++t)
-          sm.cunit[t + 1] = sm.cunit[t] + (unsigned long long)(si.seg_start(3 * u + t + 1) -
-                                                               si.seg_start(3 * u + t)) *
-                                              si.weight(t);
+        for (int w = 0; w < kNCW; ++w) o = fmaf(stashp[(w * G + n) * kStashRow + d], sm.wsc[w][n], o);
+        const float L = sm.LH[n];
+        if (c0 == c1) {
+          p.out[(obase + n) * kHeadDim + d] = L > 0.0f ? o / L : 0.0f;
+          if (d == 0 && p.lse)
+            p.lse[obase + n] = L > 0.0f ? (sm.MH[n] + log2f(L)) * 0.69314718055994530942f : -INFINITY;
+        } else {
+          part[n * kPartStride + 4 + d] = o;
+          if (d == 0) {
+            part[n * kPartStride + 0] = sm.MH[n];
+            part[n * kPartStride + 1] = L;
+          }
+        }
       }
+      if (tid == 0 && c == c0) reinterpret_cast<int2*>(counters)[u] = make_int2(c0, c1);
+      if (b == g1) break;  // the run ends in this unit: no further page-table reads
+      continue;
     }
-    named_bar_sync(1, nct);
-    const unsigned long long ctot = sm.ctot, Su = (unsigned long long)p.S;
-    int c0 = c, c1 = c;
-    if (unit_aligned_split(U, p.S)) {
-      c0 = unit_first_run(u, sm.cunit[0], ctot, p.S, U);
-      c1 = unit_first_run(u + 1, sm.cunit[3], ctot, p.S, U) - 1;
-    } else if (ctot > 0) {
-      int tl = 2;  // tier of the unit's last page
-      while (tl > 0 && sm.useg[tl] == iu1) --tl;
-      c0 = (int)(sm.cunit[0] * Su / ctot);
-      c1 = (int)((sm.cunit[3] - si.weight(tl)) * Su / ctot);
-    }
+    // ---- dense: this CTA's result for unit u (sm.O, sm.MH, sm.LH).  A unit
+    // inside one run is finished here; otherwise every run from c0 to c1
+    // writes its partial to slot c + u (an empty run an empty one, at the
+    // kernel's start) and decode_merge_kernel combines them once this grid
+    // has completed.  The CTA of run c0 records (c0, c1) for it.
+    const int c0 = sm.c01[0], c1 = sm.c01[1];
     const long long obase = (long long)bb * p.Hq + (long long)hkv * G;
     if (c0 == c1) {
       for (int i = tid; i < G * kHeadDim; i += nct) {
