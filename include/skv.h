@@ -93,7 +93,13 @@ typedef struct skv_config {
                           levels {383, 807, 1249, 1831} / 1024, thresholds
                           sqrt({22, 64, 145} / 64) (lower logit error at the
                           same bytes) */
-  int32_t reserved[3]; /* zero */
+  int32_t deterministic; /* nonzero: the decode never hands out pages at run
+                          time (no dynamic chunks; see skv_decode_attention), so
+                          repeated calls give bit-identical results; 0: the
+                          unit-aligned split balances its runs' tails at run
+                          time, and results may differ between calls in the
+                          last bits (about 1e-5 relative) */
+  int32_t reserved[2]; /* zero */
 } skv_config;
 
 /* Device pools of page slots, one per tier.  Slot s of tier t starts at
@@ -254,13 +260,19 @@ int skv_append(skv_ctx* ctx, const uint16_t* K_new, const uint16_t* V_new, int B
      page_tier_indptr  NULL, or skv_allocate's per-(unit, tier) offsets: the
               runs are then cut by payload bytes instead of page counts
               (same results either way).  When num_splits >= 8*B*Hkv
-              every unit gets its own runs, in proportion to its cost;
-              otherwise the page list of all units is cut into runs of
-              equal cost.
+              every unit gets its own runs, in proportion to its cost, and
+              about the last eighth of a unit's pages (whole chunks of 512
+              tokens) is handed out at run time, chunk by chunk, to the
+              unit's runs as they finish their static part (unless the
+              context is deterministic); otherwise the
+              page list of all units is cut into runs of equal cost.
      out      fp32 [B][Hq][128] device; lse fp32 [B][Hq] device or NULL
               (a unit without resident tokens gives out 0, lse -inf)
      num_splits  number of page runs = CTAs (0 = default: the SM count)
-     workspace   skv_workspace_size(SKV_WS_DECODE, ..., num_splits) bytes
+     workspace   skv_workspace_size(SKV_WS_DECODE, ..., num_splits) bytes;
+              its contents need no initialisation (the chunk counters carry
+              a per-launch tag and are reset by the launch that uses them),
+              but two decodes that overlap in time must not share one
    Stream order: the decode is launched as a programmatic dependent of the
    stream's previous kernel.  If that kernel lets its dependents start
    early (griddepcontrol.launch_dependents, as this library's merge and

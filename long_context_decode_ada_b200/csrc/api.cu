@@ -26,6 +26,7 @@ struct skv_ctx {
   float cos6[64], sin6[64], cos4[16], sin4[16], cos5[32], sin5[32];
   int t1_scheme = 0;            // 0: 6-bit angle + 2-bit share; 1: 5-bit + 3-bit
   int share_grid = 0;           // 2-bit share grid: 0 uniform, 1 Lloyd-Max
+  int deterministic = 0;        // the decode's split is static (no run-time chunks)
   float kappa[3];
   float rho_levels[4];
   long long payload[4];
@@ -132,6 +133,7 @@ int skv_create(const skv_config* cfg, skv_ctx** out) {
     return fail(SKV_ERR_ARG, "share_grid must be 0 or 1 (got %d)", cfg->share_grid);
   }
   c->share_grid = cfg->share_grid;
+  c->deterministic = cfg->deterministic != 0;
   c->log2P = P == 16 ? 4 : (P == 32 ? 5 : 6);
   c->device = 0;
   c->profile_event = nullptr;
@@ -230,6 +232,19 @@ int skv_device_info(const skv_ctx* ctx, int* sm_count, int* default_splits) {
   if (sm_count) *sm_count = ctx->sm_count;
   if (default_splits) *default_splits = ctx->sm_count;
   return ok();
+}
+
+// The decode's split weight of one page of tier ti (3: a dense bf16 page):
+// its payload bytes, a T2 page at least a T1 page's (their rows take about
+// the same consumer time), a T0 page SKV_T0_COST_PCT percent of its bytes.
+#ifndef SKV_T0_COST_PCT
+#define SKV_T0_COST_PCT 100
+#endif
+static long long split_cost(const skv_ctx* ctx, int ti) {
+  if (ti == 3) return ctx->payload[3];
+  if (ti == 0) return ctx->payload[0] * SKV_T0_COST_PCT / 100;
+  if (ti == 1) return ctx->payload[1];
+  return std::max(ctx->payload[2], ctx->payload[1]);
 }
 
 static int decode_splits(const skv_ctx* ctx, int num_splits) {
@@ -471,6 +486,7 @@ static int decode_common(skv_ctx* ctx, const void* q, int q_dtype, int B, int Hq
     const int ti = dense ? 3 : t;
     p.stride[t] = ctx->stride[ti];
     p.payload[t] = (int)ctx->payload[ti];
+    p.cost[t] = (int)split_cost(ctx, ti);
   }
   p.out = out;
   p.lse = lse;
@@ -496,6 +512,7 @@ static int decode_common(skv_ctx* ctx, const void* q, int q_dtype, int B, int Hq
   std::memcpy(p.sin5, ctx->sin5, sizeof(p.sin5));
   p.t1_scheme = ctx->t1_scheme;
   p.share_grid = ctx->share_grid;
+  p.dynamic = ctx->deterministic ? 0 : 1;
   cudaError_t e =
       skv::launch_decode(p, G, dense, static_cast<cudaStream_t>(stream), ctx->profile_event);
   if (e != cudaSuccess) return cuda_fail(e, name);

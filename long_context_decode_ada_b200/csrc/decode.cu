@@ -66,6 +66,18 @@ constexpr int kMaxIPP = kItemRows / 16;       // pages per item (P >= 16)
 constexpr int kMergeBatch = 20;               // merge: runs whose loads are issued together
 constexpr int kTouchedUnits = 16;             // units whose segment costs a CTA keeps
 constexpr int kStashRow = kHeadDim + 4;       // combine stash: floats per (warp, head) row
+// Unit-aligned split: the last ~1/kDynDen of a unit's pages (whole chunks of
+// kChunkItems items) are not cut into runs but handed out one chunk at a
+// time, through a per-unit counter, to the unit's runs as they finish their
+// static part; CTAs that stream faster take more of them.
+#ifndef SKV_DYN_DEN
+#define SKV_DYN_DEN 8
+#endif
+#ifndef SKV_CHUNK_ITEMS
+#define SKV_CHUNK_ITEMS 8
+#endif
+constexpr int kDynDen = SKV_DYN_DEN;
+constexpr int kChunkItems = SKV_CHUNK_ITEMS;
 static_assert(kCG >= 1 && kCG <= 4, "consumer groups: 1..4");
 static_assert(kIss >= 1 && kIss <= 4, "issuers: 1..4");
 static_assert(kPasses >= 1 && kGW * kRowsPerWarp == kItemRows, "warp row split");
@@ -77,6 +89,7 @@ static_assert(kPasses >= 1 && kGW * kRowsPerWarp == kItemRows, "warp row split")
 // unusable (bad id: nothing copied for it).
 constexpr int kMetaTierShift = 4;
 constexpr int kMetaBadShift = 12;
+constexpr uint32_t kMetaUnitEnd = 1u << 20;  // a unit-end marker (desc.z: the next unit's first item)
 
 // Shared-memory plan: [ring][TBL1][TBL2][fixed block] (ADA) or
 // [ring][fixed block] (dense).  TBL1 / TBL2 are the reconstruction tables
@@ -109,9 +122,13 @@ struct __align__(16) DecodeSmem {
   unsigned long long cunit[4];         // merge: cost before each segment of a unit, and its end
   long long useg[4];                   // merge: the unit's tier segment starts
   long long run[2];                    // this CTA's pages [run[0], run[1])
+  long long dyn_m;                     // unit-aligned: first page of the unit's dynamic part
+  int dyn_chunks, dyn_cp;              // its chunks and pages per chunk (0: no dynamic part)
+  int dyn_first;                       // this run is its unit's first (resets the counter)
   int unit0, unit1;                    // the units of pages run[0] and run[1] - 1
   int abort_flag;
-  int pad_[2];
+  int dyn_go;                          // consumers passed the wait for the previous grids
+  int pad_[1];
   __align__(16) float ml[kNCW][4][2];
   float wsc[kNCW][4];                   // combine: each warp's scale per head
   float MH[4], LH[4];                   // combine: this CTA's (M, L) per head
@@ -237,7 +254,7 @@ __device__ __forceinline__ int unit_first_run(int u, unsigned long long Pu, unsi
 // segment of the units it touches (when they are at most kTouchedUnits).
 template <class Smem>
 __device__ __noinline__ void find_run(const SplitInfo& si, int c, int S, Smem& sm, int tid,
-                                      const uint32_t* ids) {
+                                      const uint32_t* ids, int ipp, bool dynamic) {
   constexpr int nt = kDecodeThreads;
   const int nseg = 3 * si.U;
   const int per = (nseg + nt - 1) / nt;
@@ -266,6 +283,10 @@ __device__ __noinline__ void find_run(const SplitInfo& si, int c, int S, Smem& s
     sm.run[1] = 0;
     sm.unit0 = 0;
     sm.unit1 = -1;
+    sm.dyn_chunks = 0;
+    sm.dyn_cp = 0;
+    sm.dyn_m = 0;
+    sm.dyn_first = 0;
   }
   __syncthreads();
   unsigned long long before = x - loc, tot = 0;
@@ -299,8 +320,25 @@ __device__ __noinline__ void find_run(const SplitInfo& si, int c, int S, Smem& s
           sm.unit1 = u;
 #pragma unroll
           for (int t = 0; t < 4; ++t) sm.ucost[t] = cc + cr[t];
-          sm.run[0] = run_begin_in_unit(si, seg, cr, (unsigned long long)j * cr[3], (unsigned long long)n);
-          sm.run[1] = run_begin_in_unit(si, seg, cr, (unsigned long long)(j + 1) * cr[3], (unsigned long long)n);
+          // the dynamic part: whole chunks at the end of the unit, about
+          // 1/kDynDen of its pages (none for a unit with a single run); the
+          // static part [seg[0], M) is cut into the n runs by cost
+          const long long cp = (long long)kChunkItems * ipp;
+          const long long nch = (dynamic && n >= 2) ? (seg[3] - seg[0]) / (kDynDen * cp) : 0;
+          const long long M = seg[3] - nch * cp;
+          long long sg[4];
+          unsigned long long cs[4];
+#pragma unroll
+          for (int t = 0; t < 4; ++t) sg[t] = min(seg[t], M);
+          cs[0] = 0;
+#pragma unroll
+          for (int t = 0; t < 3; ++t) cs[t + 1] = cs[t] + (unsigned long long)(sg[t + 1] - sg[t]) * si.weight(t);
+          sm.run[0] = run_begin_in_unit(si, sg, cs, (unsigned long long)j * cs[3], (unsigned long long)n);
+          sm.run[1] = run_begin_in_unit(si, sg, cs, (unsigned long long)(j + 1) * cs[3], (unsigned long long)n);
+          sm.dyn_m = M;
+          sm.dyn_chunks = (int)nch;
+          sm.dyn_cp = (int)cp;
+          sm.dyn_first = j == 0;
         }
       }
       cc += (unsigned long long)(si.seg_start(k + 1) - si.seg_start(k)) * si.weight(k);
@@ -342,6 +380,18 @@ __device__ __noinline__ void find_run(const SplitInfo& si, int c, int S, Smem& s
     if (k1 == nseg && k0 < k1 && nseg <= 3 * ub + 3) sm.ucost[nseg - 3 * ua] = cc;
   }
   __syncthreads();
+}
+
+// A 32-bit tag of this grid launch (the low half of the temporal grid
+// identifier, which differs between launches in a context).
+__device__ __forceinline__ uint32_t launch_tag() {
+  unsigned long long g;
+  asm volatile("mov.u64 %0, %%gridid;" : "=l"(g));
+  return (uint32_t)g;
+}
+
+__device__ __forceinline__ int ld_volatile(const int* p) {
+  return *reinterpret_cast<const volatile int*>(p);
 }
 
 // ------------------------------------------------------ shared loads (PTX) --
@@ -761,9 +811,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   si.indptr = p.indptr;
   si.tier_indptr = p.tier_indptr;
   si.U = U;
-  si.w[0] = p.payload[0];
-  si.w[1] = DENSE ? p.payload[0] : p.payload[1];
-  si.w[2] = DENSE ? p.payload[0] : p.payload[2];
+  si.w[0] = p.cost[0];
+  si.w[1] = DENSE ? p.cost[0] : p.cost[1];
+  si.w[2] = DENSE ? p.cost[0] : p.cost[2];
   const DecodeWs wsl = decode_ws(p.S, U, G);
   uint8_t* const wsb = reinterpret_cast<uint8_t*>(p.part);
   int* const counters = reinterpret_cast<int*>(wsb + wsl.ctr);
@@ -784,6 +834,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         mbar_init(smem_u32(&sm.ready[i]), 1);
       }
       sm.abort_flag = 0;
+      sm.dyn_go = 0;
       fence_mbar_init();
     } else {
       report(p.err, SKV_ERR_ARG);
@@ -811,7 +862,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     }
   }
   if (!plan_ok) return;  // uniform: every thread computed the same layout
-  find_run(si, c, p.S, sm, tid, p.ids);
+  find_run(si, c, p.S, sm, tid, p.ids, ipp, p.dynamic != 0);
   const long long g0 = sm.run[0], g1 = sm.run[1];
   if (g0 >= g1) {
     // an empty run inside a unit's runs (unit-aligned: a trailing run of a
@@ -825,6 +876,11 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       float* part = p.part + (long long)(c + u) * G * kPartStride + tid * kPartStride;
       part[0] = -INFINITY;
       part[1] = 0.0f;
+      // (a unit's first run always holds pages; should it not, the counter
+      // of the unit's chunks is still reset here, after the wait)
+      if (tid == 0 && sm.dyn_chunks > 0 && sm.dyn_first)
+        atomicExch(reinterpret_cast<unsigned long long*>(wsb + wsl.dyn) + u,
+                   (unsigned long long)launch_tag() << 32);
     }
     return;
   }
@@ -833,31 +889,24 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
 
   if (warp == kPlannerWarp) {
     // ------------------------------------------------------------- planner
-    // Batches of up to 32 items of one unit: lane i decodes item it + i (its
-    // page ids -> sources, sizes, tiers) in parallel.  Placement is
-    // deterministic: an item goes at the write offset, or at 0 when it would
-    // cross the ring's end.  Before an item is published every older item
-    // whose bytes it may overwrite (virtual start < its virtual end - R) and
-    // the previous user of its slot must be released; each lane works out
-    // that count, and the lanes publish (descriptors + ready signal) in
-    // parallel as releases arrive.  kIss end-of-run markers follow the last
-    // item, one per issuer.
-    int u = u0;
-    long long pg = g0;  // first page of the next batch
-    // the ids of a batch's pages are loaded one batch ahead (read up to the
-    // end of the run, not of the unit: a batch starts where the previous one
-    // ended, or at the first page of the next unit, which follows it)
-    uint32_t idn[kMaxIPP];
-#pragma unroll
-    for (int q = 0; q < kMaxIPP; ++q) {
-      const long long pq = pg + (long long)lane * ipp + q;
-      idn[q] = (q < ipp && pq < g1) ? __ldg(p.ids + pq) : 0u;
-    }
-    // end of the current unit's run and the end of the next unit, loaded
-    // one unit ahead (a unit-aligned run lies inside its unit: no loads)
+    // The run is planned as page ranges inside one unit each: the run's part
+    // of every unit it touches (in order) and, under the unit-aligned split,
+    // the dynamic chunks this CTA takes from its unit's counter once its
+    // static part is planned.  A range is planned in batches of up to 32
+    // items: lane i decodes item it + i (its page ids -> sources, sizes,
+    // tiers) in parallel.  Placement is deterministic: an item goes at the
+    // write offset, or at 0 when it would cross the ring's end.  Before an
+    // item is published every older item whose bytes it may overwrite
+    // (virtual start < its virtual end - R) and the previous user of its
+    // slot must be released; each lane works out that count, and the lanes
+    // publish (descriptors + ready signal) in parallel as releases arrive.
+    // A unit's items are followed by kCG unit-end markers (one per consumer
+    // group, no bytes) that carry the index of the next unit's first item;
+    // the run ends with kIss end-of-run markers, one per issuer.
     const bool in_unit = unit_aligned_split(U, p.S);
-    long long ub = in_unit ? g1 : min(g1, (long long)p.indptr[u0 + 1]);
-    long long ub_next = (!in_unit && u0 + 2 <= U) ? (long long)p.indptr[u0 + 2] : g1;
+    const int dyn_chunks = in_unit ? sm.dyn_chunks : 0;
+    const long long dyn_m = sm.dyn_m;
+    const int dyn_cp = sm.dyn_cp;
     int it = 0;                 // next item
     int tail = 0;               // oldest item not known to be released
     uint32_t wr = 0;            // ring write offset
@@ -871,172 +920,240 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       ++tail;
       return true;
     };
+    // a marker item (no bytes, no copy) in the next slot
+    auto publish_marker = [&](uint32_t meta, uint32_t z, uint32_t bytes) -> bool {
+      while (it - tail >= kNSlot)
+        if (!release_tail()) return false;
+      const int s = it % kNSlot;
+      if (lane == 0) {
+        sm.vstart[it & 63] = V;
+        sm.desc[s] = make_uint4(0u, meta, z, 0u);
+        sm.copy_bytes[s] = bytes;
+        mbar_arrive(smem_u32(&sm.ready[s]));
+      }
+      __syncwarp();
+      ++it;
+      return true;
+    };
+    // the dynamic chunk counter of this run's unit: a grab returns {tag,
+    // index}; a tag other than this launch's means the counter was not
+    // reset yet (the grab is void)
+    unsigned long long* const dynctr = reinterpret_cast<unsigned long long*>(wsb + wsl.dyn) + u0;
+    const uint32_t tag = launch_tag();
+    unsigned long long fut = 0;  // lane 0: the result of the grab in flight
+    bool grabbed = false;
+    bool grab_ok = true;
+    auto issue_grab = [&]() {
+      if (!grabbed) {
+        // the first grab waits until the consumers have passed the wait for
+        // the previous grids (no earlier launch still takes chunks from this
+        // workspace) and, in the unit's first run, reset the counter
+        const long long t0 = clock64();
+        while (ld_volatile(&sm.dyn_go) == 0) {
+          if (ld_volatile(&sm.abort_flag) || clock64() - t0 > kWaitLimitCycles) {
+            grab_ok = false;  // no grab: fut stays 0, whose tag matches no launch
+            break;
+          }
+          __nanosleep(256);
+        }
+        grabbed = true;
+      }
+      if (grab_ok && lane == 0) fut = atomicAdd(dynctr, 1ull);
+    };
+    // the page ids of the unit's dynamic part, brought into L2 when the
+    // static part is planned (the chunks' first id loads then hit L2)
+    auto prefetch_dyn_ids = [&]() {
+      // the 128-byte lines that hold ids [dyn_m, dyn_m + chunks * cp)
+      const uintptr_t a = reinterpret_cast<uintptr_t>(p.ids + dyn_m);
+      const uintptr_t l0 = a / 128, l1 = (a + (uintptr_t)dyn_chunks * dyn_cp * 4 + 127) / 128;
+      for (uintptr_t l = l0 + lane; l < l1; l += 32)
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<const void*>(128 * l)));
+    };
+    // plan the items of pages [pg, pe) of one unit
+    auto plan_range = [&](long long pg, long long pe, bool grab_at_last) -> bool {
+      uint32_t idn[kMaxIPP];
+#pragma unroll
+      for (int q = 0; q < kMaxIPP; ++q) {
+        const long long pq = pg + (long long)lane * ipp + q;
+        idn[q] = (q < ipp && pq < pe) ? __ldg(p.ids + pq) : 0u;
+      }
+      while (pg < pe) {
+        const int nb = (int)min(32LL, (pe - pg + ipp - 1) / ipp);  // items in this batch
+        const long long pn = min(pe, pg + (long long)nb * ipp);    // the next batch's first page
+        if (grab_at_last && pn >= pe) {  // the range's last batch: the first chunk's grab
+          issue_grab();
+          prefetch_dyn_ids();
+        }
+        const uint32_t my_pg = CAP ? (uint32_t)(pg + (long long)lane * ipp) : 0u;
+        // ---- lane-parallel decode of item it + lane
+        uint32_t plo[kMaxIPP], phi[kMaxIPP], psz[kMaxIPP];
+        uint32_t total = 0, imeta = 0, relz = 0, relw = 0;
+        uint32_t id[kMaxIPP];
+#pragma unroll
+        for (int q = 0; q < kMaxIPP; ++q) id[q] = idn[q];
+#pragma unroll
+        for (int q = 0; q < kMaxIPP; ++q) {
+          const long long pq = pn + (long long)lane * ipp + q;
+          idn[q] = (q < ipp && pq < pe) ? __ldg(p.ids + pq) : 0u;
+        }
+        if (lane < nb) {
+          const long long ps = pg + (long long)lane * ipp;
+          const int n = (int)min((long long)ipp, pe - ps);
+          imeta = (uint32_t)n;
+#pragma unroll
+          for (int q = 0; q < kMaxIPP; ++q) {
+            plo[q] = 0;
+            phi[q] = 0;
+            psz[q] = 0;
+            if (q == 1) relz = total;
+            if (q == 2) relz |= total << 16;
+            if (q == 3) relw = total;
+            if (q < n) {
+              const uint32_t tr = id[q] >> 30, slot = id[q] & 0x3FFFFFFFu;
+              bool valid;
+              if (DENSE) {
+                valid = tr == 0 && slot < (unsigned long long)p.slots[0];
+              } else {
+                valid = (tr == 0 && slot < (unsigned long long)p.slots[0]) ||
+                        (tr == 1 && slot < (unsigned long long)p.slots[1]) ||
+                        (tr == 2 && slot < (unsigned long long)p.slots[2]);
+              }
+              if (valid) {
+                const uint8_t* src = tr == 0 ? p.pool[0] + (long long)slot * p.stride[0]
+                                             : (tr == 1 ? p.pool[1] + (long long)slot * p.stride[1]
+                                                        : p.pool[2] + (long long)slot * p.stride[2]);
+                plo[q] = (uint32_t)reinterpret_cast<uintptr_t>(src);
+                phi[q] = (uint32_t)(reinterpret_cast<uintptr_t>(src) >> 32);
+                psz[q] = (uint32_t)(tr == 0 ? p.payload[0] : (tr == 1 ? p.payload[1] : p.payload[2]));
+              } else {
+                report(p.err, SKV_ERR_CORRUPT);
+                imeta |= 1u << (kMetaBadShift + q);
+              }
+              imeta |= (tr & 3u) << (kMetaTierShift + 2 * q);
+              total += psz[q];
+            }
+          }
+        }
+        // ---- placement: a warp-parallel scan of the sizes, then each lane
+        // finds how many items must be released before its item may be
+        // written (need: all items before it), and the lanes publish in
+        // parallel, a prefix of the batch at a time, as releases come in
+        uint32_t my_off = 0;
+        unsigned long long my_v = 0;
+        {
+          // offsets = write offset + exclusive prefix of the sizes, restarted
+          // at 0 (after a pad to the next lap of the virtual position) at the
+          // first item of each stretch that would cross the ring's end
+          uint32_t incl = total;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+            if (lane >= o) incl += y;
+          }
+          const uint32_t excl = incl - total;
+          uint32_t base = wr;
+          unsigned long long vbase = V;
+          int from = 0;
+          while (true) {
+            const uint32_t ex0 = __shfl_sync(0xFFFFFFFFu, excl, from);
+            const uint32_t off = base + (excl - ex0);
+            const unsigned cross =
+                __ballot_sync(0xFFFFFFFFu, lane >= from && lane < nb && off + total > R);
+            const int j = cross ? __ffs(cross) - 1 : 32;
+            if (lane >= from && lane < j) {
+              my_off = off;
+              my_v = vbase + (excl - ex0);
+            }
+            if (!cross) break;
+            const uint32_t exj = __shfl_sync(0xFFFFFFFFu, excl, j);
+            vbase = vbase + (exj - ex0) + (R - (base + (exj - ex0)));
+            base = 0;
+            from = j;
+          }
+          const uint32_t lt = __shfl_sync(0xFFFFFFFFu, total, nb - 1);
+          wr = __shfl_sync(0xFFFFFFFFu, my_off, nb - 1) + lt;
+          V = __shfl_sync(0xFFFFFFFFu, my_v, nb - 1) + lt;
+        }
+        if (lane < nb) sm.vstart[(it + lane) & 63] = my_v;
+        __syncwarp();
+        int need = 0;
+        if (lane < nb) {
+          const int me = it + lane;
+          // slot reuse: item me - kNSlot must be released
+          need = max(0, me - kNSlot + 1);
+          // space: every item whose bytes start more than R before this
+          // item's end (V grows with the item index: a prefix of them)
+          const unsigned long long lim = my_v + total;
+          // binary search: the first j in [need, me) with vstart[j] + R >= lim
+          int lo = need, hi = me;
+          while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            if (sm.vstart[mid & 63] + R >= lim) hi = mid; else lo = mid + 1;
+          }
+          need = lo;
+        }
+        bool done = lane >= nb;
+        while (true) {
+          // released items, in order, without blocking
+          while (tail < it + nb &&
+                 mbar_test_wait(smem_u32(&sm.empty[tail % kNSlot]), (uint32_t)((tail / kNSlot) & 1)))
+            ++tail;
+          const bool now = !done && need <= tail;
+          if (now) {
+            const int s = (it + lane) % kNSlot;
+            sm.desc[s] = make_uint4(ring_lo + my_off, imeta, relz, relw);
+            if (CAP) sm.dpage[s] = my_pg;
+            const uint32_t rel[kMaxIPP] = {0u, relz & 0xFFFFu, relz >> 16, relw};
+#pragma unroll
+            for (int q = 0; q < kMaxIPP; ++q)
+              if (q < (int)(imeta & 7u))
+                sm.copy[s][q] = PageCopy{plo[q], phi[q], psz[q], ring_lo + my_off + rel[q]};
+            sm.copy_bytes[s] = total;
+            mbar_arrive(smem_u32(&sm.ready[s]));
+          }
+          done = done || now;
+          if (__all_sync(0xFFFFFFFFu, done)) break;
+          // the oldest unreleased item is published (its own need is met):
+          // sleep until it is released
+          if (!release_tail()) return false;
+        }
+        it += nb;
+        pg = pn;
+      }
+      return true;
+    };
+
+    int u = u0;
+    long long pg = g0;
+    // end of the current unit's part of the run and the end of the next
+    // unit, loaded one unit ahead (a unit-aligned run lies inside its unit)
+    long long ub = in_unit ? g1 : min(g1, (long long)p.indptr[u0 + 1]);
+    long long ub_next = (!in_unit && u0 + 2 <= U) ? (long long)p.indptr[u0 + 2] : g1;
     while (ok && pg < g1) {
       while (pg >= ub) {  // next unit with pages in this run
         ++u;
         ub = min(g1, ub_next);
         ub_next = u + 2 <= U ? (long long)p.indptr[u + 2] : g1;
       }
-      const int nb = (int)min(32LL, (ub - pg + ipp - 1) / ipp);  // items in this batch
-      const uint32_t my_pg = CAP ? (uint32_t)(pg + (long long)lane * ipp) : 0u;
-      // ---- lane-parallel decode of item it + lane
-      uint32_t plo[kMaxIPP], phi[kMaxIPP], psz[kMaxIPP];
-      uint32_t total = 0, imeta = 0, relz = 0, relw = 0;
-      uint32_t id[kMaxIPP];
-#pragma unroll
-      for (int q = 0; q < kMaxIPP; ++q) id[q] = idn[q];
-      {
-        const long long pn = min(ub, pg + (long long)nb * ipp);  // the next batch's first page
-#pragma unroll
-        for (int q = 0; q < kMaxIPP; ++q) {
-          const long long pq = pn + (long long)lane * ipp + q;
-          idn[q] = (q < ipp && pq < g1) ? __ldg(p.ids + pq) : 0u;
-        }
+      ok = plan_range(pg, ub, dyn_chunks > 0);
+      while (ok && dyn_chunks > 0) {
+        // dynamic chunks of the unit, one grab in flight ahead of the chunk
+        // being planned
+        const unsigned long long got = __shfl_sync(0xFFFFFFFFu, fut, 0);
+        const uint32_t k = (uint32_t)got;
+        if ((uint32_t)(got >> 32) != tag || k >= (uint32_t)dyn_chunks) break;
+        issue_grab();
+        const long long cs = dyn_m + (long long)k * dyn_cp;
+        ok = plan_range(cs, cs + dyn_cp, false);
       }
-      if (lane < nb) {
-        const long long ps = pg + (long long)lane * ipp;
-        const int n = (int)min((long long)ipp, ub - ps);
-        imeta = (uint32_t)n;
-#pragma unroll
-        for (int q = 0; q < kMaxIPP; ++q) {
-          plo[q] = 0;
-          phi[q] = 0;
-          psz[q] = 0;
-          if (q == 1) relz = total;
-          if (q == 2) relz |= total << 16;
-          if (q == 3) relw = total;
-          if (q < n) {
-            const uint32_t tr = id[q] >> 30, slot = id[q] & 0x3FFFFFFFu;
-            bool valid;
-            if (DENSE) {
-              valid = tr == 0 && slot < (unsigned long long)p.slots[0];
-            } else {
-              valid = (tr == 0 && slot < (unsigned long long)p.slots[0]) ||
-                      (tr == 1 && slot < (unsigned long long)p.slots[1]) ||
-                      (tr == 2 && slot < (unsigned long long)p.slots[2]);
-            }
-            if (valid) {
-              const uint8_t* src = tr == 0 ? p.pool[0] + (long long)slot * p.stride[0]
-                                           : (tr == 1 ? p.pool[1] + (long long)slot * p.stride[1]
-                                                      : p.pool[2] + (long long)slot * p.stride[2]);
-              plo[q] = (uint32_t)reinterpret_cast<uintptr_t>(src);
-              phi[q] = (uint32_t)(reinterpret_cast<uintptr_t>(src) >> 32);
-              psz[q] = (uint32_t)(tr == 0 ? p.payload[0] : (tr == 1 ? p.payload[1] : p.payload[2]));
-            } else {
-              report(p.err, SKV_ERR_CORRUPT);
-              imeta |= 1u << (kMetaBadShift + q);
-            }
-            imeta |= (tr & 3u) << (kMetaTierShift + 2 * q);
-            total += psz[q];
-          }
-        }
-      }
-      // ---- placement: a warp-parallel scan of the sizes, then each lane
-      // finds how many items must be released before its item may be
-      // written (need: all items before it), and the lanes publish in
-      // parallel, a prefix of the batch at a time, as releases come in
-      uint32_t my_off = 0;
-      unsigned long long my_v = 0;
-      {
-        // offsets = write offset + exclusive prefix of the sizes, restarted
-        // at 0 (after a pad to the next lap of the virtual position) at the
-        // first item of each stretch that would cross the ring's end
-        uint32_t incl = total;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-          if (lane >= o) incl += y;
-        }
-        const uint32_t excl = incl - total;
-        uint32_t base = wr;
-        unsigned long long vbase = V;
-        int from = 0;
-        while (true) {
-          const uint32_t ex0 = __shfl_sync(0xFFFFFFFFu, excl, from);
-          const uint32_t off = base + (excl - ex0);
-          const unsigned cross =
-              __ballot_sync(0xFFFFFFFFu, lane >= from && lane < nb && off + total > R);
-          const int j = cross ? __ffs(cross) - 1 : 32;
-          if (lane >= from && lane < j) {
-            my_off = off;
-            my_v = vbase + (excl - ex0);
-          }
-          if (!cross) break;
-          const uint32_t exj = __shfl_sync(0xFFFFFFFFu, excl, j);
-          vbase = vbase + (exj - ex0) + (R - (base + (exj - ex0)));
-          base = 0;
-          from = j;
-        }
-        const uint32_t lt = __shfl_sync(0xFFFFFFFFu, total, nb - 1);
-        wr = __shfl_sync(0xFFFFFFFFu, my_off, nb - 1) + lt;
-        V = __shfl_sync(0xFFFFFFFFu, my_v, nb - 1) + lt;
-      }
-      if (lane < nb) sm.vstart[(it + lane) & 63] = my_v;
-      __syncwarp();
-      int need = 0;
-      if (lane < nb) {
-        const int me = it + lane;
-        // slot reuse: item me - kNSlot must be released
-        need = max(0, me - kNSlot + 1);
-        // space: every item whose bytes start more than R before this
-        // item's end (V grows with the item index: a prefix of them)
-        const unsigned long long lim = my_v + total;
-        // binary search: the first j in [need, me) with vstart[j] + R >= lim
-        int lo = need, hi = me;
-        while (lo < hi) {
-          const int mid = (lo + hi) >> 1;
-          if (sm.vstart[mid & 63] + R >= lim) hi = mid; else lo = mid + 1;
-        }
-        need = lo;
-      }
-      bool done = lane >= nb;
-      while (true) {
-        // released items, in order, without blocking
-        while (tail < it + nb &&
-               mbar_test_wait(smem_u32(&sm.empty[tail % kNSlot]), (uint32_t)((tail / kNSlot) & 1)))
-          ++tail;
-        const bool now = !done && need <= tail;
-        if (now) {
-          const int s = (it + lane) % kNSlot;
-          sm.desc[s] = make_uint4(ring_lo + my_off, imeta, relz, relw);
-          if (CAP) sm.dpage[s] = my_pg;
-          const uint32_t rel[kMaxIPP] = {0u, relz & 0xFFFFu, relz >> 16, relw};
-#pragma unroll
-          for (int q = 0; q < kMaxIPP; ++q)
-            if (q < (int)(imeta & 7u))
-              sm.copy[s][q] = PageCopy{plo[q], phi[q], psz[q], ring_lo + my_off + rel[q]};
-          sm.copy_bytes[s] = total;
-          mbar_arrive(smem_u32(&sm.ready[s]));
-        }
-        done = done || now;
-        if (__all_sync(0xFFFFFFFFu, done)) break;
-        // the oldest unreleased item is published (its own need is met):
-        // sleep until it is released
-        if (!release_tail()) {
-          ok = false;
-          break;
-        }
-      }
-      if (!ok) break;
-      it += nb;
-      pg = min(ub, pg + (long long)nb * ipp);
+      // the unit's end: one marker per consumer group, carrying the index
+      // of the next unit's first item
+      const uint32_t next_first = (uint32_t)(it + kCG);
+      for (int e = 0; e < kCG && ok; ++e) ok = publish_marker(kMetaUnitEnd, next_first, 0u);
+      pg = ub;
     }
     // end-of-run markers: a slot each (its previous item released)
-    for (int e = 0; e < kIss && ok; ++e) {
-      while (it - tail >= kNSlot) {
-        if (!release_tail()) {
-          ok = false;
-          break;
-        }
-      }
-      if (!ok) break;
-      const int s = it % kNSlot;
-      if (lane == 0) {
-        sm.copy_bytes[s] = kEndOfRun;
-        mbar_arrive(smem_u32(&sm.ready[s]));
-      }
-      ++it;
-    }
+    for (int e = 0; e < kIss && ok; ++e) ok = publish_marker(0u, 0u, kEndOfRun);
     if (lane == 0 && !ok) {
       report(p.err, SKV_ERR_TIMEOUT);
       sm.abort_flag = 1;
@@ -1060,9 +1177,19 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       if (total == kEndOfRun) break;
       const uint32_t np = sm.desc[s].y & 7u;
       const uint32_t fullb = smem_u32(&sm.full[s]);
+      // the item's copy list is read before the arrive: once the phase can
+      // complete (no bytes to wait for), the slot may be released and
+      // rewritten for a later item
+      PageCopy cps[kMaxIPP];
+#pragma unroll
+      for (int q = 0; q < kMaxIPP; ++q) {
+        cps[q] = PageCopy{0u, 0u, 0u, 0u};
+        if ((uint32_t)q < np) cps[q] = sm.copy[s][q];
+      }
       mbar_arrive_expect_tx(fullb, total);
-      for (uint32_t q = 0; q < np; ++q) {
-        const PageCopy cp = sm.copy[s][q];
+#pragma unroll
+      for (int q = 0; q < kMaxIPP; ++q) {
+        const PageCopy& cp = cps[q];
         if (cp.bytes)
           bulk_g2s(cp.dst, reinterpret_cast<const void*>((uintptr_t)cp.src_lo |
                                                          ((uintptr_t)cp.src_hi << 32)),
@@ -1105,6 +1232,17 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   // queries or write any result or partial.
   if constexpr (!DENSE) build_tables<VAR>(p, tbl1p, 256 + 64, tid, nct);
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  if (tid == 0) {
+    // the previous grids have completed: no earlier launch takes chunks from
+    // this workspace any more.  The unit's first run resets its counter to
+    // this launch's tag; then the planner may grab.
+    if (sm.dyn_chunks > 0 && sm.dyn_first && unit_aligned_split(U, p.S)) {
+      unsigned long long* ctr = reinterpret_cast<unsigned long long*>(wsb + wsl.dyn) + u0;
+      atomicExch(ctr, (unsigned long long)launch_tag() << 32);
+      __threadfence();
+    }
+    *reinterpret_cast<volatile int*>(&sm.dyn_go) = 1;
+  }
   int tbl_entries = 0;  // table entries still to build (after a combine's stash)
   int it = 0;  // item index within the run
   bool ok = true;
@@ -1196,48 +1334,64 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
 #pragma unroll
     for (int e = 0; e < 4; ++e) st.ones[e] = 0.0f;
 
-    const int nitems = (int)((b - a + ipp - 1) / ipp);
-    // this group's items of the unit: it + i with (it + i) % kCG == grp
-    for (int i = ((grp - it % kCG) + kCG) % kCG; i < nitems; i += kCG) {
-      const int itm = it + i, s = itm % kNSlot;
-      const uint32_t fullb = smem_u32(&sm.full[s]), par = (uint32_t)((itm / kNSlot) & 1);
-      if (ok && !mbar_test_wait(fullb, par) && !mbar_wait_bounded(fullb, par, &sm.abort_flag)) {
+    // this group's items of the unit, it + i with (it + i) % kCG == grp, up
+    // to its unit-end marker (which gives the next unit's first item)
+    int next_it = it;
+    for (int itm = it + ((grp - it % kCG) + kCG) % kCG; ok; itm += kCG) {
+      const int s = itm % kNSlot;
+      const uint32_t par = (uint32_t)((itm / kNSlot) & 1);
+      // first the item's publication, then its data.  A phase-parity wait
+      // on `full` alone would alias: while the slot's previous item
+      // (itm - kNSlot, another group's) is still in flight, `full` is one
+      // phase behind and its parity test would already pass.  `ready` for
+      // item itm cannot be behind (the planner publishes in order and this
+      // group's previous item, itm - kCG, is published), and once itm is
+      // published the slot's previous item has been released, so `full`
+      // is then at itm's own phase.
+      const uint32_t readyb = smem_u32(&sm.ready[s]), fullb = smem_u32(&sm.full[s]);
+      if ((!mbar_test_wait(readyb, par) && !mbar_wait_bounded(readyb, par, &sm.abort_flag)) ||
+          (!mbar_test_wait(fullb, par) && !mbar_wait_bounded(fullb, par, &sm.abort_flag))) {
         ok = false;
         if (lane == 0) {
           report(p.err, SKV_ERR_TIMEOUT);
           sm.abort_flag = 1;
         }
+        break;
       }
-      if (ok) {
-        const uint4 d = lds128(smem_u32(&sm.desc[s]));
-        const uint32_t np = d.y & 7u;
-        const long long dpg = CAP ? (long long)sm.dpage[s] : -1;
+      const uint4 d = lds128(smem_u32(&sm.desc[s]));
+      if (d.y & kMetaUnitEnd) {
+        next_it = (int)d.z;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&sm.empty[s]));
+        break;
+      }
+      const uint32_t np = d.y & 7u;
+      const long long dpg = CAP ? (long long)sm.dpage[s] : -1;
 #pragma unroll
-        for (int ps = 0; ps < kPasses; ++ps) {
-          const int r = kRowsPerWarp * wi + 16 * ps;  // row within the item
-          const uint32_t kp = (uint32_t)(r >> p.log2P);
-          const int row0 = r & (p.P - 1);
-          if (kp < np && !((d.y >> (kMetaBadShift + kp)) & 1u)) {
-            const uint32_t rel = kp == 0 ? 0u
-                                         : (kp == 1 ? (d.z & 0xFFFFu)
-                                                    : (kp == 2 ? (d.z >> 16) : d.w));
-            float* lg = nullptr;
-            if (CAP && dpg >= 0) {
-              const long long r0 = (dpg + kp) * p.P;  // the page's first logit row
-              if (r0 + p.P <= p.logit_rows)
-                lg = p.logits + r0 * G;
-              else if (lane == 0)
-                report(p.err, SKV_ERR_ARG);
-            }
-            process_rows<G, DENSE, CAP>(p, d.x + rel, (d.y >> (kMetaTierShift + 2 * kp)) & 3u, row0,
-                                   qf, tb1, tb2, st, lane, lg);
+      for (int ps = 0; ps < kPasses; ++ps) {
+        const int r = kRowsPerWarp * wi + 16 * ps;  // row within the item
+        const uint32_t kp = (uint32_t)(r >> p.log2P);
+        const int row0 = r & (p.P - 1);
+        if (kp < np && !((d.y >> (kMetaBadShift + kp)) & 1u)) {
+          const uint32_t rel = kp == 0 ? 0u
+                                       : (kp == 1 ? (d.z & 0xFFFFu)
+                                                  : (kp == 2 ? (d.z >> 16) : d.w));
+          float* lg = nullptr;
+          if (CAP && dpg >= 0) {
+            const long long r0 = (dpg + kp) * p.P;  // the page's first logit row
+            if (r0 + p.P <= p.logit_rows)
+              lg = p.logits + r0 * G;
+            else if (lane == 0)
+              report(p.err, SKV_ERR_ARG);
           }
+          process_rows<G, DENSE, CAP>(p, d.x + rel, (d.y >> (kMetaTierShift + 2 * kp)) & 3u, row0,
+                                      qf, tb1, tb2, st, lane, lg);
         }
       }
       __syncwarp();
-      if (lane == 0 && ok) mbar_arrive(smem_u32(&sm.empty[s]));
+      if (lane == 0) mbar_arrive(smem_u32(&sm.empty[s]));
     }
-    it += nitems;
+    it = next_it;
 
     // ---- combine the warps' states into this CTA's partial for unit u.
     // Every warp writes its (m, l) per head; one thread per head forms M,

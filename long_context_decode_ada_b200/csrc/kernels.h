@@ -20,6 +20,7 @@ struct DecodeParams {
   long long slots[3];
   long long stride[3];
   int payload[3];
+  int cost[3];          // split weight of a page of each tier (split_cost)
   float* out;
   float* lse;
   int32_t* err;
@@ -35,6 +36,7 @@ struct DecodeParams {
   float cos5[32], sin5[32];  // angles of the T1 variant (5-bit angle + 3-bit share)
   int t1_scheme;             // T1 code byte: 0 (angle6 << 2) | share2; 1 (angle5 << 3) | share3
   int share_grid;            // 2-bit share grid: 0 uniform, 1 Lloyd-Max
+  int dynamic;               // unit-aligned split: hand out the units' last pages at run time
 };
 
 struct EncodeParams {
@@ -145,14 +147,17 @@ struct AllocParams {
 
 // Decode workspace: partials [(S + U) G][kPartStride] fp32, then per unit the
 // range (c0, c1) of runs that hold its partials (int32 pairs, written by every
-// call before they are read).
+// call before they are read), then per unit the 64-bit counter of the
+// unit's dynamic chunks: {launch tag (high 32 bits), chunks handed out}, reset
+// by the unit's first run of each launch (no state is kept between calls).
 struct DecodeWs {
-  size_t ctr, bytes;
+  size_t ctr, dyn, bytes;
 };
 __host__ __device__ inline DecodeWs decode_ws(long long S, long long U, int G) {
   DecodeWs w;
   w.ctr = (size_t)(S + U) * G * kPartStride * 4;
-  w.bytes = w.ctr + 8 * (size_t)U;
+  w.dyn = w.ctr + 8 * (size_t)U;
+  w.bytes = w.dyn + 8 * (size_t)U;
   return w;
 }
 

@@ -43,7 +43,8 @@ EXPORTS = [
 class SkvConfig(C.Structure):
     _fields_ = [("head_dim", C.c_int32), ("page_size", C.c_int32),
                 ("outlier_protect", C.c_int32), ("t1_angle_bits", C.c_int32),
-                ("share_grid", C.c_int32), ("reserved", C.c_int32 * 3)]
+                ("share_grid", C.c_int32), ("deterministic", C.c_int32),
+                ("reserved", C.c_int32 * 2)]
 
 
 class SkvPools(C.Structure):
@@ -189,10 +190,10 @@ class Context:
     """An skv_ctx: head_dim 128, page size P; bound to the current device."""
 
     def __init__(self, page_size: int, head_dim: int = 128, outlier_protect: bool = False,
-                 t1_angle_bits: int = 6, share_grid: int = 0):
+                 t1_angle_bits: int = 6, share_grid: int = 0, deterministic: bool = False):
         cfg = SkvConfig(head_dim=head_dim, page_size=page_size,
                         outlier_protect=1 if outlier_protect else 0, t1_angle_bits=t1_angle_bits,
-                        share_grid=share_grid)
+                        share_grid=share_grid, deterministic=1 if deterministic else 0)
         h = C.c_void_p()
         _check(lib().skv_create(C.byref(cfg), C.byref(h)))
         self._h = h
@@ -201,6 +202,7 @@ class Context:
         self.outlier_protect = bool(outlier_protect)
         self.t1_angle_bits = t1_angle_bits
         self.share_grid = share_grid
+        self.deterministic = bool(deterministic)
 
     def __del__(self):
         h = getattr(self, "_h", None)

@@ -102,8 +102,9 @@ def test_workspace_sizes():
     ctx = skv.Context(64)
     sm, splits = ctx.device_info()
     def expect(S, U, G):
-        # split partials, then each unit's range of runs (two int32)
-        return (S + U) * G * 132 * 4 + 8 * U
+        # split partials, then each unit's range of runs (two int32), then
+        # each unit's chunk counter (one 64-bit word)
+        return (S + U) * G * 132 * 4 + 8 * U + 8 * U
     n = ctx.workspace_size(skv.WS_DECODE, 1, 8, 32, 0, 0)
     assert n == expect(splits, 8, 4)
     assert ctx.workspace_size(skv.WS_DECODE, 1, 8, 32, 0, 10) == expect(10, 8, 4)

@@ -219,3 +219,72 @@ def test_gqa_group_equals_single_head_runs():
                         w.mode, w1.utility, None, w.budget, w.quota, 91, False)
         g1 = run_gpu(w1)
         np.testing.assert_allclose(g1["out"][0, 0], g["out"][0, hq], rtol=1e-5, atol=1e-6)
+
+
+@pytest.mark.parametrize("splits", [0, 16, 40])
+def test_dynamic_chunks_eager_and_graph_replays(splits):
+    """Unit-aligned split (num_splits >= 8 units): the last eighth of each
+    unit's pages is handed out at run time through a per-unit counter that
+    every launch tags and resets.  Eager calls and every replay of a
+    captured CUDA graph (several decodes per replay, one workspace) match
+    the oracle.  The chunk assignment may differ between launches, and with
+    it which rows share a warp's running maximum (the scale at which P is
+    rounded to fp16 for the P.V MMA): replays agree with each other to
+    1e-4, ten times inside the parity tolerance."""
+    lens = [9000, 6100]
+    quota = [[T // 10, 6 * T // 10, T // 5] for T in lens]
+    w = wl.custom(64, 2, 2, 4, 64, lens, wl.MODE_QUOTA, quota=quota, scatter=True)
+    ref = oracle.run_workload(w)
+    g = run_gpu(w, num_splits=splits)
+    assert_close(g["out"], ref["out"], "out (eager)")
+    assert_close(g["lse"], ref["lse"], "lse (eager)")
+    cache, dev = g["cache"], g["dev"]
+    ws = cache.workspace(w.Hq, splits)
+    out = torch.empty((w.B, w.Hq, 128), dtype=torch.float32, device="cuda")
+    lse = torch.empty((w.B, w.Hq), dtype=torch.float32, device="cuda")
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        for _ in range(3):
+            cache.decode(dev["q"], dev["q_dtype"], w.Hq, out=out, lse=lse, workspace=ws,
+                         num_splits=splits)
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr, stream=s):
+            for _ in range(3):
+                cache.decode(dev["q"], dev["q_dtype"], w.Hq, out=out, lse=lse, workspace=ws,
+                             num_splits=splits)
+    torch.cuda.synchronize()
+    first = None
+    for rep in range(5):
+        out.zero_()
+        gr.replay()
+        torch.cuda.synchronize()
+        cache.check()
+        o = out.cpu().numpy()
+        assert_close(o, ref["out"], f"out (replay {rep})")
+        assert_close(lse.cpu().numpy(), ref["lse"], f"lse (replay {rep})")
+        if first is None:
+            first = o
+        np.testing.assert_allclose(o, first, rtol=0, atol=1e-4)
+
+
+def test_deterministic_context_gives_bit_identical_calls():
+    """skv_config.deterministic: the unit-aligned split keeps every page in
+    a static run (no run-time chunks), so repeated calls and graph replays
+    return bit-identical results, which also match the oracle."""
+    lens = [9000, 6100]
+    quota = [[T // 10, 6 * T // 10, T // 5] for T in lens]
+    w = wl.custom(64, 2, 2, 4, 64, lens, wl.MODE_QUOTA, quota=quota, scatter=True)
+    ref = oracle.run_workload(w)
+    ctx = skv.Context(w.P, deterministic=True)
+    g = run_gpu(w, ctx=ctx)
+    assert_close(g["out"], ref["out"], "out")
+    cache, dev = g["cache"], g["dev"]
+    outs = []
+    for _ in range(4):
+        o, l = cache.decode(dev["q"], dev["q_dtype"], w.Hq)
+        cache.check()
+        outs.append((o.cpu().numpy(), l.cpu().numpy()))
+    for o, l in outs[1:]:
+        assert np.array_equal(o, outs[0][0]) and np.array_equal(l, outs[0][1])
+    assert np.array_equal(outs[0][0], g["out"])

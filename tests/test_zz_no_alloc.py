@@ -12,6 +12,7 @@ import torch
 
 from long_context_decode_ada_b200 import skv
 from long_context_decode_ada_b200 import workloads as wl
+from _gpu import ATOL, RTOL
 
 
 def test_static_scratch_rejects_calls_beyond_its_size():
@@ -34,9 +35,10 @@ def _close(a, b, what):
     assert np.array_equal(np.isfinite(a), np.isfinite(b)), what
     fin = np.isfinite(b)
     assert np.array_equal(a[~fin], b[~fin]), what
-    # the same kernel on the same store: only the order of the in-CTA fp32
-    # combine of warp partials may differ between launches
-    assert np.all(np.abs(a[fin] - b[fin]) <= 1e-6 + 1e-5 * np.abs(b[fin])), what
+    # the same kernel on the same store, within the parity tolerance of the
+    # GPU tests: the unit-aligned split hands out its last chunks at run
+    # time, so two launches may group rows differently (last-bit changes)
+    assert np.all(np.abs(a[fin] - b[fin]) <= ATOL + RTOL * np.abs(b[fin])), what
 
 
 @pytest.mark.gpu
