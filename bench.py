@@ -59,6 +59,9 @@ def parse_args():
     ap.add_argument("--cp", action="store_true",
                     help="context-parallel decode: the ranks share one sequence, each "
                          "holding a slice of its positions (strong scaling)")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the other workloads (Llama layer, ragged batch, 32-layer "
+                         "pipeline, tiny)")
     ap.add_argument("--graph-steps", type=int, default=100)
     ap.add_argument("--seed", type=int, default=0)
     return ap.parse_args()
@@ -147,9 +150,16 @@ def measured_peaks():
     return 6650.0, "fallback"
 
 
+def split_costs(payload):
+    """The decode's split weight per tier (the library's rule): a page's
+    payload bytes, a T2 page at least a T1 page's."""
+    p0, p1, p2 = (int(x) for x in payload)
+    return [p0, p1, max(p2, p1)]
+
+
 def written_partials(indptr: np.ndarray, ids: np.ndarray, payload, S: int) -> int:
     """(run, unit) partials the decode kernel writes (and the merge kernel
-    reads back).  Pages cost their tier's payload bytes.  With at most S
+    reads back).  Pages cost their tier's split weight (split_costs).  With at most S
     units, unit u gets runs [B(u), B(u+1)), B(u) = u + round(P(u)(S-U)/C)
     (P(u) the bytes before u, C the total) when S >= 8 U; otherwise page g is in run
     floor(C(g) S / C), C(g) the bytes before it.  A unit spread over several
@@ -158,7 +168,7 @@ def written_partials(indptr: np.ndarray, ids: np.ndarray, payload, S: int) -> in
     U = len(indptr) - 1
     if N == 0:
         return 0
-    cost = np.asarray(payload, np.int64)[np.asarray(ids[:N], np.uint32) >> 30]
+    cost = np.asarray(split_costs(payload), np.int64)[np.asarray(ids[:N], np.uint32) >> 30]
     before = np.concatenate([[0], np.cumsum(cost)[:-1]])
     total = int(cost.sum())
     n = 0
@@ -488,6 +498,12 @@ def run_skv(args, rank, world, local_rank):
                          "around the steps"}
         del ca, da
 
+    configs = None
+    if not args.no_configs:
+        del caches, ws
+        torch.cuda.empty_cache()
+        configs = run_configs(ctx, dev, peak, S_default=default_splits)
+
     cpu = None
     if rank == 0 and not args.no_cpu:
         cpu = cpu_baseline(T_sample=args.seq_len)
@@ -524,9 +540,143 @@ def run_skv(args, rank, world, local_rank):
             "ingest": {"allocate_ms": alloc_ms, "encode_ms": enc_ms, "gen_s": t_gen},
             "append": append,
             "utility": utility,
+            "configs": configs,
             "step_ms_graph_events": float(np.mean(step_ms)),
         }
         print(json.dumps(line), flush=True)
+
+
+def store_stats(cache):
+    """Tier counts, pages per tier and the decode's algorithmic bytes of one
+    store (tier bytes of the resident token-heads + 20 B per page)."""
+    tc = torch.bincount(cache.tier.flatten().to(torch.int64), minlength=4).cpu().numpy()
+    indptr = cache.page_indptr.cpu().numpy()
+    n = int(indptr[-1])
+    ids = cache.page_ids[:n].cpu().numpy().view(np.uint32)
+    ppt = np.bincount(ids >> 30, minlength=3)
+    byt = int(sum(int(tc[t]) * TIER_BYTES[t] for t in range(3))) + 20 * n + 4 * len(indptr)
+    return {"tier_tokens": {"T0": int(tc[0]), "T1": int(tc[1]), "T2": int(tc[2]),
+                            "dropped": int(tc[3])},
+            "pages": {"T0": int(ppt[0]), "T1": int(ppt[1]), "T2": int(ppt[2])},
+            "resident_tokens_heads": int(tc[:3].sum()), "bytes": byt}
+
+
+def graph_time_ms(fns, reps_per_graph, replays):
+    """Mean device time of one call of fns (cycled) in CUDA-graph replays:
+    3 eager warm-up calls, one graph of reps_per_graph calls, replays timed
+    with events on the current stream."""
+    for i in range(3):
+        fns[i % len(fns)]()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for i in range(reps_per_graph):
+            fns[i % len(fns)]()
+    g.replay()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(replays):
+        g.replay()
+    b.record()
+    torch.cuda.synchronize()
+    del g
+    return a.elapsed_time(b) / (replays * reps_per_graph)
+
+
+def run_configs(ctx, dev, peak, S_default):
+    """The other workloads of the decode path, drawn on the GPU with the same
+    recipes: the Llama-3-8B-shaped layer, the ragged batch of 64 (scattered
+    pages), the tiny all-T2 store and the 32-layer pipeline (allocate +
+    encode per layer, then a decode step over all 32 layers).  Stores larger
+    than L2 alternate between two copies; the tiny store (0.7 MB) is timed
+    warm in L2 and says so."""
+    from long_context_decode_ada_b200 import skv
+    from long_context_decode_ada_b200 import workloads as wl
+    res = {}
+
+    def one_layer(name, w, copies, note):
+        d = skv.workload_to_device(w, dev)
+        c0 = skv.build_cache(ctx, w, d)
+        c0.check()
+        caches = [c0] + [clone_cache(c0) for _ in range(copies - 1)]
+        del d["K"], d["V"]
+        wss = [c.workspace(w.Hq) for c in caches]
+        out = torch.empty((w.B, w.Hq, 128), dtype=torch.float32, device=dev)
+        lse = torch.empty((w.B, w.Hq), dtype=torch.float32, device=dev)
+        fns = [(lambda c=c, wsp=wsp: c.decode(d["q"], d["q_dtype"], w.Hq, out=out, lse=lse,
+                                              workspace=wsp)) for c, wsp in zip(caches, wss)]
+        ms = graph_time_ms(fns, 20 * copies if copies > 1 else 20, 10)
+        c0.check()
+        st = store_stats(c0)
+        gbs = st["bytes"] / (ms * 1e-3) / 1e9
+        res[name] = dict(st, us_per_decode=ms * 1e3, achieved_gbs=gbs, frac=gbs / peak,
+                         value=st["resident_tokens_heads"] / (ms * 1e-3), unit=UNIT,
+                         B=w.B, Hq=w.Hq, Hkv=w.Hkv, P=w.P, note=note)
+        del caches, wss, fns
+        torch.cuda.empty_cache()
+
+    one_layer("llama_layer", wl.llama_layer(device=dev), 2,
+              "B=8, T=32768, 32q/8kv, P=64, quota 10/50/25/15%; two alternating stores")
+    one_layer("ragged_batch", wl.ragged_batch(device=dev), 2,
+              "B=64, T~U[1024,8192], P=16, quota 20/40/40/0%, scattered pages; two "
+              "alternating stores")
+    one_layer("tiny_all_t2", wl.tiny(), 1,
+              "B=1, one head, T=4096, P=16, all T2: 0.74 MB, timed warm (in L2)")
+
+    # ---- 32-layer pipeline: allocate + encode per layer, one decode step over all layers
+    L = 32
+    caches, qs, wss = [], [], []
+    alloc_ms = enc_ms = 0.0
+    e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    for layer in range(L):
+        w = wl.pipeline_layer(layer, device=dev)
+        d = skv.workload_to_device(w, dev)
+        c = skv.PagedCache(ctx, w.B, w.Hkv, w.Tmax, w.pool_slots, device=dev)
+        e[0].record()
+        c.allocate(d["K"], d["seq_lens"], d["utility"], d["protect"], w.mode, d["budget"],
+                   d["quota"], d["free_lists"])
+        e[1].record()
+        c.encode(d["K"], d["V"], d["seq_lens"])
+        e[2].record()
+        c.check()
+        alloc_ms += e[0].elapsed_time(e[1])
+        enc_ms += e[1].elapsed_time(e[2])
+        caches.append(c)
+        qs.append(d["q"])
+        wss.append(c.workspace(w.Hq))
+        del d, w
+    Hq = 32
+    out = torch.empty((4, Hq, 128), dtype=torch.float32, device=dev)
+    lse = torch.empty((4, Hq), dtype=torch.float32, device=dev)
+
+    def step():
+        for layer in range(L):
+            caches[layer].decode(qs[layer], skv.Q_BF16, Hq, out=out, lse=lse,
+                                 workspace=wss[layer])
+    ms = graph_time_ms([step], 4, 10)
+    for c in caches:
+        c.check()
+    stats = [store_stats(c) for c in caches]
+    byt = sum(s_["bytes"] for s_ in stats)
+    tok = sum(s_["resident_tokens_heads"] for s_ in stats)
+    tiers = {k: sum(s_["tier_tokens"][k] for s_ in stats) for k in ("T0", "T1", "T2", "dropped")}
+    pages = {k: sum(s_["pages"][k] for s_ in stats) for k in ("T0", "T1", "T2")}
+    gbs = byt / (ms * 1e-3) / 1e9
+    res["pipeline_32_layers"] = {
+        "layers": L, "B": 4, "T": 65536, "Hq": 32, "Hkv": 8, "P": 64,
+        "allocate_ms_total": alloc_ms, "encode_ms_total": enc_ms,
+        "encode_gbs": L * 4 * 8 * 65536 * 512 / (enc_ms * 1e-3) / 1e9,
+        "decode_step_us": ms * 1e3, "decode_us_per_layer": ms * 1e3 / L,
+        "bytes": byt, "achieved_gbs": gbs, "frac": gbs / peak,
+        "value": tok / (ms * 1e-3), "unit": UNIT,
+        "tier_tokens": tiers, "pages": pages, "resident_tokens_heads": tok,
+        "note": "per layer: outlier channels x20, budget 30% of dense fp16 KV, Zipf(1.2) "
+                "utility; allocate and encode timed by events per layer (summed), the decode "
+                "step is one graph of 32 decodes (one per layer's store; 10 GB > L2)"}
+    del caches, qs, wss
+    torch.cuda.empty_cache()
+    return res
 
 
 def decode_source_digest() -> str:

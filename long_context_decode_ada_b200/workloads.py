@@ -8,7 +8,9 @@ Both the CUDA path and the CPU oracle take their inputs from here.
 
 Every draw uses a ``torch.Generator`` on the CPU seeded from ``(seed, stream)``
 so that each tensor is reproducible on its own, independent of draw order and
-of thread count.  bf16 queries are carried as ``uint16`` bit patterns
+of thread count.  The recipe functions also take ``device="cuda"``: the same
+distributions drawn by a CUDA generator on the GPU (a different random
+stream, for timing runs at full size; parity runs draw on the CPU).  bf16 queries are carried as ``uint16`` bit patterns
 (round-to-nearest-even from fp32), fp16 tensors as ``float16``.
 
 The workloads stand in for the pages' evaluation (PG-19, LongBench, AgentBench,
@@ -63,22 +65,24 @@ class Workload:
         return self.Hq // self.Hkv
 
 
-def _gen(seed: int, stream: int) -> torch.Generator:
-    g = torch.Generator()
+def _gen(seed: int, stream: int, device=None) -> torch.Generator:
+    g = torch.Generator(device=device or "cpu")
     g.manual_seed((seed * 1_000_003 + stream * 7_919 + 12_345) & 0x7FFF_FFFF_FFFF_FFFF)
     return g
 
 
-def _normal(shape, seed, stream) -> torch.Tensor:
-    return torch.randn(shape, generator=_gen(seed, stream), dtype=torch.float32)
+def _normal(shape, seed, stream, device=None) -> torch.Tensor:
+    return torch.randn(shape, generator=_gen(seed, stream, device), dtype=torch.float32,
+                       device=device or "cpu")
 
 
-def _uniform(shape, seed, stream) -> torch.Tensor:
-    return torch.rand(shape, generator=_gen(seed, stream), dtype=torch.float32)
+def _uniform(shape, seed, stream, device=None) -> torch.Tensor:
+    return torch.rand(shape, generator=_gen(seed, stream, device), dtype=torch.float32,
+                      device=device or "cpu")
 
 
-def _perm(n, seed, stream) -> torch.Tensor:
-    return torch.randperm(n, generator=_gen(seed, stream))
+def _perm(n, seed, stream, device=None) -> torch.Tensor:
+    return torch.randperm(n, generator=_gen(seed, stream, device), device=device or "cpu")
 
 
 def to_bf16_bits(x: torch.Tensor) -> torch.Tensor:
@@ -134,46 +138,46 @@ def tiny(seed: int = 0, T: int = 4096) -> Workload:
 
 
 def llama_layer(seed: int = 0, B: int = 8, T: int = 32768, Hkv: int = 8, G: int = 4,
-                P: int = 64) -> Workload:
+                P: int = 64, device=None) -> Workload:
     """Llama-3-8B-shaped decode layer: 32 query / 8 KV heads, d=128, batch 8,
     T=32768, P=64, bf16 q.  K has per-(head, channel) LogNormal(0, 0.5) scales
     times N(0,1); V ~ N(0,1).  Tier quotas 10% T0 / 50% T1 / 25% T2 / 15%
     dropped, ranked by U(0,1) utilities."""
     Hq = Hkv * G
-    scale = torch.exp(0.5 * _normal((1, Hkv, 1, D_HEAD), seed, 4))
-    K = (_normal((B, Hkv, T, D_HEAD), seed, 1) * scale).to(torch.float16)
-    V = _normal((B, Hkv, T, D_HEAD), seed, 2).to(torch.float16)
-    q = to_bf16_bits(_normal((B, Hq, D_HEAD), seed, 3))
-    u = _uniform((B, Hkv, T), seed, 5)
+    scale = torch.exp(0.5 * _normal((1, Hkv, 1, D_HEAD), seed, 4, device))
+    K = (_normal((B, Hkv, T, D_HEAD), seed, 1, device) * scale).to(torch.float16)
+    V = _normal((B, Hkv, T, D_HEAD), seed, 2, device).to(torch.float16)
+    q = to_bf16_bits(_normal((B, Hq, D_HEAD), seed, 3, device))
+    u = _uniform((B, Hkv, T), seed, 5, device)
     quota = [[int(0.10 * T), int(0.50 * T), int(0.25 * T)] for _ in range(B)]
     return _finish("llama3_8b_layer", B, Hq, Hkv, P, T, [T] * B, K, V, q, "bf16",
                    MODE_QUOTA, u, None, [0] * B, quota, seed, scatter=False)
 
 
-def zipf_utility(B, Hkv, T, alpha, seed, stream) -> torch.Tensor:
+def zipf_utility(B, Hkv, T, alpha, seed, stream, device=None) -> torch.Tensor:
     """u_t = (1 + pi(t))^-alpha with pi a seeded permutation per (seq, head):
     a Zipf law over positions whose ranks are scattered through the context."""
-    u = torch.empty((B, Hkv, T), dtype=torch.float32)
+    u = torch.empty((B, Hkv, T), dtype=torch.float32, device=device or "cpu")
     for b in range(B):
         for h in range(Hkv):
-            rank = _perm(T, seed, stream + 1000 * b + h).to(torch.float64)
+            rank = _perm(T, seed, stream + 1000 * b + h, device).to(torch.float64)
             u[b, h] = torch.pow(1.0 + rank, -alpha).to(torch.float32)
     return u
 
 
 def long_context(seed: int = 0, T: int = 131072, B: int = 1, Hkv: int = 8, G: int = 4,
                  P: int = 64, budget_frac: float = 0.40, sink: int = 64,
-                 recent: int = 1024) -> Workload:
+                 recent: int = 1024, device=None) -> Workload:
     """Long-context decode: B=1, 32 query / 8 KV heads, T=131072, P=64.  The
     first 64 and last 1024 tokens are protected (kept dense); the rest are
     allocated under a budget of 40% of the dense fp16 KV bytes, with Zipf(1.1)
     utilities over positions.  K, V, q ~ N(0,1); q in bf16."""
     Hq = Hkv * G
-    K = _normal((B, Hkv, T, D_HEAD), seed, 1).to(torch.float16)
-    V = _normal((B, Hkv, T, D_HEAD), seed, 2).to(torch.float16)
-    q = to_bf16_bits(_normal((B, Hq, D_HEAD), seed, 3))
-    u = zipf_utility(B, Hkv, T, 1.1, seed, 10)
-    prot = torch.zeros((B, Hkv, T), dtype=torch.uint8)
+    K = _normal((B, Hkv, T, D_HEAD), seed, 1, device).to(torch.float16)
+    V = _normal((B, Hkv, T, D_HEAD), seed, 2, device).to(torch.float16)
+    q = to_bf16_bits(_normal((B, Hq, D_HEAD), seed, 3, device))
+    u = zipf_utility(B, Hkv, T, 1.1, seed, 10, device)
+    prot = torch.zeros((B, Hkv, T), dtype=torch.uint8, device=device or "cpu")
     prot[:, :, :min(sink, T)] = 1
     prot[:, :, max(0, T - recent):] = 1
     budget = [int(math.floor(budget_frac * T * Hkv * 512))] * B
@@ -182,7 +186,7 @@ def long_context(seed: int = 0, T: int = 131072, B: int = 1, Hkv: int = 8, G: in
 
 
 def ragged_batch(seed: int = 0, B: int = 64, Tlo: int = 1024, Thi: int = 8192,
-                 Hkv: int = 8, G: int = 4, P: int = 16) -> Workload:
+                 Hkv: int = 8, G: int = 4, P: int = 16, device=None) -> Workload:
     """Ragged serving batch: 64 sequences with lengths uniform in [1024, 8192],
     32 query / 8 KV heads, P=16; every free list is a seeded permutation of a
     shared pool so pages are scattered; tiers 20% T0 / 40% T1 / 40% T2 (none
@@ -191,10 +195,10 @@ def ragged_batch(seed: int = 0, B: int = 64, Tlo: int = 1024, Thi: int = 8192,
     g = _gen(seed, 6)
     lens = torch.randint(Tlo, Thi + 1, (B,), generator=g).numpy().astype(np.int32)
     Tmax = int(lens.max())
-    K = _normal((B, Hkv, Tmax, D_HEAD), seed, 1).to(torch.float16)
-    V = _normal((B, Hkv, Tmax, D_HEAD), seed, 2).to(torch.float16)
-    q = to_bf16_bits(_normal((B, Hq, D_HEAD), seed, 3))
-    u = _uniform((B, Hkv, Tmax), seed, 5)
+    K = _normal((B, Hkv, Tmax, D_HEAD), seed, 1, device).to(torch.float16)
+    V = _normal((B, Hkv, Tmax, D_HEAD), seed, 2, device).to(torch.float16)
+    q = to_bf16_bits(_normal((B, Hq, D_HEAD), seed, 3, device))
+    u = _uniform((B, Hkv, Tmax), seed, 5, device)
     quota = []
     for b in range(B):
         T = int(lens[b])
@@ -206,7 +210,8 @@ def ragged_batch(seed: int = 0, B: int = 64, Tlo: int = 1024, Thi: int = 8192,
 
 def pipeline_layer(layer: int, seed: int = 0, B: int = 4, T: int = 65536, Hkv: int = 8,
                    G: int = 4, P: int = 64, budget_frac: float = 0.30,
-                   outlier_frac: float = 0.01, outlier_scale: float = 20.0) -> Workload:
+                   outlier_frac: float = 0.01, outlier_scale: float = 20.0,
+                   device=None) -> Workload:
     """One layer of the 32-layer pipeline: B=4, T=65536, 32 query / 8 KV heads.
     K ~ N(0,1) with round(1% of Hkv*d) outlier channels of this layer scaled
     x20 (chosen without replacement, seeded per layer); V ~ N(0,1); a budget
@@ -214,15 +219,15 @@ def pipeline_layer(layer: int, seed: int = 0, B: int = 4, T: int = 65536, Hkv: i
     an independent position permutation per (seq, head)."""
     Hq = Hkv * G
     s = seed * 97 + layer
-    K = _normal((B, Hkv, T, D_HEAD), s, 1)
+    K = _normal((B, Hkv, T, D_HEAD), s, 1, device)
     n_out = int(round(outlier_frac * Hkv * D_HEAD))
     chans = _perm(Hkv * D_HEAD, s, 7)[:n_out]
     for c in chans.tolist():
         K[:, c // D_HEAD, :, c % D_HEAD] *= outlier_scale
     K = K.to(torch.float16)
-    V = _normal((B, Hkv, T, D_HEAD), s, 2).to(torch.float16)
-    q = to_bf16_bits(_normal((B, Hq, D_HEAD), s, 3))
-    u = zipf_utility(B, Hkv, T, 1.2, s, 20)
+    V = _normal((B, Hkv, T, D_HEAD), s, 2, device).to(torch.float16)
+    q = to_bf16_bits(_normal((B, Hq, D_HEAD), s, 3, device))
+    u = zipf_utility(B, Hkv, T, 1.2, s, 20, device)
     budget = [int(math.floor(budget_frac * T * Hkv * 512))] * B
     return _finish(f"pipeline_layer{layer}", B, Hq, Hkv, P, T, [T] * B, K, V, q, "bf16",
                    MODE_BUDGET, u, None, budget, [[0, 0, 0]] * B, s, scatter=False)
