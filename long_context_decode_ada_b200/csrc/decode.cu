@@ -648,6 +648,66 @@ __device__ __forceinline__ float ex2_approx(float x) {
 // Online softmax of 16 rows and P.V into the accumulators.
 // lA / lB: log2-domain logits of rows t and t + 8 (head g % G) or -inf.
 // VK: 0 int8 V (1 KB per 8-row group), 1 fp16 V, 2 bf16 V (2 KB per group).
+// The online-softmax update of 16 rows: raises the running max when needed
+// (rescaling the accumulators), adds the rows' weights to l and returns the
+// P.V B fragments (k16 x n8: k = rows 2t4, 2t4+1 | 8+2t4, 9+2t4, n = head
+// gq) of the weights times the rows' V scales, as fp16 (F16) or bf16.
+template <int G, bool F16>
+__device__ __forceinline__ void softmax_weights(float lA, float lB, float vsA, float vsB,
+                                                WarpState& st, int lane, uint32_t& bf0,
+                                                uint32_t& bf1) {
+  const int gq = lane >> 2, t4 = lane & 3;
+  if (__any_sync(0xFFFFFFFFu, fmaxf(lA, lB) > st.m + kLazyMax)) {
+    float cm = fmaxf(lA, lB);
+    cm = fmaxf(cm, __shfl_xor_sync(0xFFFFFFFFu, cm, 4));
+    cm = fmaxf(cm, __shfl_xor_sync(0xFFFFFFFFu, cm, 8));
+    cm = fmaxf(cm, __shfl_xor_sync(0xFFFFFFFFu, cm, 16));
+    const float m_new = fmaxf(st.m, cm);
+    const float alpha = ex2_approx(st.m - m_new);  // 0 when st.m is kNoMax
+    st.l *= alpha;
+    st.m = m_new;
+    const int n0 = 2 * t4, n1 = 2 * t4 + 1;
+    const float a0 = __shfl_sync(0xFFFFFFFFu, alpha, n0 < G ? n0 : 0);
+    const float a1 = __shfl_sync(0xFFFFFFFFu, alpha, n1 < G ? n1 : 0);
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt) {
+      st.acc[mt][0] *= a0;
+      st.acc[mt][1] *= a1;
+      st.acc[mt][2] *= a0;
+      st.acc[mt][3] *= a1;
+    }
+    st.ones[0] *= a0;
+    st.ones[1] *= a1;
+    st.ones[2] *= a0;
+    st.ones[3] *= a1;
+  }
+  const float pA = ex2_approx(lA - st.m), pB = ex2_approx(lB - st.m);  // -inf -> 0
+  st.l += pA + pB;
+  const float ppA = pA * vsA, ppB = pB * vsB;
+  const int src = 8 * t4 + (gq < G ? gq : 0);
+  const float b0 = __shfl_sync(0xFFFFFFFFu, ppA, src);
+  const float b1 = __shfl_sync(0xFFFFFFFFu, ppA, src + 4);
+  const float b2 = __shfl_sync(0xFFFFFFFFu, ppB, src);
+  const float b3 = __shfl_sync(0xFFFFFFFFu, ppB, src + 4);
+  bf0 = F16 ? pack_f16x2(b0, b1) : pack_bf16x2(b0, b1);
+  bf1 = F16 ? pack_f16x2(b2, b3) : pack_bf16x2(b2, b3);
+}
+
+// P.V of 16 int8 V rows already in registers (fragment words of the two
+// 8-row blocks), v + 1152 as fp16, the bias taken off through the ones MMA.
+__device__ __forceinline__ void pv_int8_regs(const uint32_t (&wa)[8], const uint32_t (&wb)[8],
+                                             uint32_t bf0, uint32_t bf1, WarpState& st) {
+#pragma unroll
+  for (int mt = 0; mt < 8; ++mt) {
+    uint32_t a0, a1, a2, a3;
+    s8x4_to_f16x2x2_biased(wa[mt], a0, a1);
+    s8x4_to_f16x2x2_biased(wb[mt], a2, a3);
+    mma_16816k16_f16(st.acc[mt], a0, a1, a2, a3, bf0, bf1);
+  }
+  constexpr uint32_t kOnes = 0x3C003C00u;  // fp16 (1, 1)
+  mma_16816k16_f16(st.ones, kOnes, kOnes, kOnes, kOnes, bf0, bf1);
+}
+
 template <int G, int VK>
 __device__ __forceinline__ void softmax_pv(float lA, float lB, float vsA, float vsB, uint32_t va,
                                            uint32_t vb, WarpState& st, int lane) {
@@ -794,6 +854,114 @@ __device__ __forceinline__ void process_rows(const DecodeParams& p, uint32_t pg,
       softmax_pv<G, 0>(lA, lB, vA ? vsA : 0.0f, vB ? vsB : 0.0f, vsec, vsec + 1024, st, lane);
     }
   }
+}
+
+// The ring data a lane needs for 16 T1 / T2 rows of one page: the page's
+// header word, the lane's code words of rows rA and rA + 8, their radii and V
+// scales (fp16 bits, row A low), and its int8 V fragment words.  Loaded all
+// at once, so that the item's ring space can be released before the rows
+// are computed (the consumers then hold only registers, not ring bytes).
+struct CodeRows {
+  uint32_t hdr;
+  uint32_t ca[4], cb[4];  // T1: the 16 code bytes of each row; T2: nibbles (2) + crumbs (1)
+  uint32_t rs, vs;
+  uint32_t va[8], vb[8];
+};
+
+__device__ __forceinline__ void load_code_rows(uint32_t pg, int P, bool t1, int row0, int lane,
+                                               CodeRows& r) {
+  const int t = lane >> 2, g = lane & 3;
+  const int rA = row0 + t, rB = rA + 8;
+  r.hdr = lds32(pg);
+  const uint32_t cd = pg + kHdrBytes + 2 * P;
+  int cb;
+  if (t1) {
+    const uint4 a = lds128(cd + rA * 64 + 16 * g), b = lds128(cd + rB * 64 + 16 * g);
+    r.ca[0] = a.x; r.ca[1] = a.y; r.ca[2] = a.z; r.ca[3] = a.w;
+    r.cb[0] = b.x; r.cb[1] = b.y; r.cb[2] = b.z; r.cb[3] = b.w;
+    cb = 64;
+  } else {
+    const uint2 na = lds64(cd + rA * 48 + 8 * g), nb = lds64(cd + rB * 48 + 8 * g);
+    r.ca[0] = na.x; r.ca[1] = na.y; r.ca[2] = lds32(cd + rA * 48 + 32 + 4 * g); r.ca[3] = 0u;
+    r.cb[0] = nb.x; r.cb[1] = nb.y; r.cb[2] = lds32(cd + rB * 48 + 32 + 4 * g); r.cb[3] = 0u;
+    cb = 48;
+  }
+  const uint32_t rsec = pg + kHdrBytes, ssec = pg + kHdrBytes + (2 + cb) * P;
+  r.rs = lds16(rsec + 2 * rA) | (lds16(rsec + 2 * rB) << 16);
+  r.vs = lds16(ssec + 2 * rA) | (lds16(ssec + 2 * rB) << 16);
+  const uint32_t vsec = pg + kHdrBytes + (2 + cb + 2) * P + (row0 >> 3) * 1024;
+  const uint4 xa = lds128(vsec + lane * 16), ya = lds128(vsec + 512 + lane * 16);
+  const uint4 xb = lds128(vsec + 1024 + lane * 16), yb = lds128(vsec + 1536 + lane * 16);
+  r.va[0] = xa.x; r.va[1] = xa.y; r.va[2] = xa.z; r.va[3] = xa.w;
+  r.va[4] = ya.x; r.va[5] = ya.y; r.va[6] = ya.z; r.va[7] = ya.w;
+  r.vb[0] = xb.x; r.vb[1] = xb.y; r.vb[2] = xb.z; r.vb[3] = xb.w;
+  r.vb[4] = yb.x; r.vb[5] = yb.y; r.vb[6] = yb.z; r.vb[7] = yb.w;
+}
+
+// T1 logits from code words in registers (see logits_t1)
+__device__ __forceinline__ void logits_t1_regs(const uint32_t (&wa)[4], const uint32_t (&wb)[4],
+                                               uint32_t tb, const QFrag& f, float (&c)[4],
+                                               float (&d)[4]) {
+#pragma unroll
+  for (int s = 0; s < 8; ++s) {
+    const int i = s >> 1, k0 = 2 * (s & 1);
+    const uint32_t ea0 = lds32(t1_addr(wa[i], k0, tb)), ea1 = lds32(t1_addr(wa[i], k0 + 1, tb));
+    const uint32_t eb0 = lds32(t1_addr(wb[i], k0, tb)), eb1 = lds32(t1_addr(wb[i], k0 + 1, tb));
+    if (s & 1)
+      mma_k16<false>(d, ea0, eb0, ea1, eb1, f.b[2 * s], f.b[2 * s + 1]);
+    else
+      mma_k16<false>(c, ea0, eb0, ea1, eb1, f.b[2 * s], f.b[2 * s + 1]);
+  }
+}
+
+// T2 logits from code words in registers (see logits_t2)
+__device__ __forceinline__ void logits_t2_regs(const uint32_t (&wa)[4], const uint32_t (&wb)[4],
+                                               uint32_t tb, const QFrag& f, float (&c)[4],
+                                               float (&d)[4]) {
+#pragma unroll
+  for (int s = 0; s < 8; ++s) {
+    const uint32_t ea0 = lds32(t2_addr(wa[0], wa[1], wa[2], 2 * s, tb));
+    const uint32_t ea1 = lds32(t2_addr(wa[0], wa[1], wa[2], 2 * s + 1, tb));
+    const uint32_t eb0 = lds32(t2_addr(wb[0], wb[1], wb[2], 2 * s, tb));
+    const uint32_t eb1 = lds32(t2_addr(wb[0], wb[1], wb[2], 2 * s + 1, tb));
+    if (s & 1)
+      mma_k16<false>(d, ea0, eb0, ea1, eb1, f.b[2 * s], f.b[2 * s + 1]);
+    else
+      mma_k16<false>(c, ea0, eb0, ea1, eb1, f.b[2 * s], f.b[2 * s + 1]);
+  }
+}
+
+// 16 T1 / T2 rows [row0, row0 + 16) from their loaded ring data.
+template <int G, bool CAP>
+__device__ __forceinline__ void compute_code_rows(const DecodeParams& p, const CodeRows& r,
+                                                  uint32_t tier, int row0, const QFrag& qf,
+                                                  uint32_t tb1, uint32_t tb2, WarpState& st,
+                                                  int lane, float* lg) {
+  const int t = lane >> 2, g = lane & 3;
+  const uint32_t cnt = r.hdr & 0xFFFFu;
+  if ((r.hdr >> 16) != (tier | ((uint32_t)kPageMagic << 8)) || cnt > (uint32_t)p.P) {
+    if (lane == 0) report(p.err, SKV_ERR_CORRUPT);
+    return;
+  }
+  if ((uint32_t)row0 >= cnt) return;
+  const int rA = row0 + t, rB = rA + 8;
+  const bool vA = (uint32_t)rA < cnt, vB = (uint32_t)rB < cnt;
+  float c[4] = {0.0f, 0.0f, 0.0f, 0.0f}, d[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+  if (tier == SKV_TIER_T1)
+    logits_t1_regs(r.ca, r.cb, tb1, qf, c, d);
+  else
+    logits_t2_regs(r.ca, r.cb, tb2, qf, c, d);
+  const float a = c[0] + d[0], b = c[2] + d[2];
+  const float rtA = __half2float(__ushort_as_half((unsigned short)(r.rs & 0xFFFFu)));
+  const float rtB = __half2float(__ushort_as_half((unsigned short)(r.rs >> 16)));
+  const float vsA = __half2float(__ushort_as_half((unsigned short)(r.vs & 0xFFFFu)));
+  const float vsB = __half2float(__ushort_as_half((unsigned short)(r.vs >> 16)));
+  const float lA = vA ? a * (rtA * qf.c1) : -INFINITY;
+  const float lB = vB ? b * (rtB * qf.c1) : -INFINITY;
+  if constexpr (CAP) capture_logits<G>(lg, rA, rB, vA, vB, lA, lB, g);
+  uint32_t bf0, bf1;
+  softmax_weights<G, true>(lA, lB, vA ? vsA : 0.0f, vB ? vsB : 0.0f, st, lane, bf0, bf1);
+  pv_int8_regs(r.va, r.vb, bf0, bf1, st);
 }
 
 template <int G, bool DENSE, bool CAP, int VAR>
@@ -1367,9 +1535,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       }
       const uint32_t np = d.y & 7u;
       const long long dpg = CAP ? (long long)sm.dpage[s] : -1;
-#pragma unroll
-      for (int ps = 0; ps < kPasses; ++ps) {
-        const int r = kRowsPerWarp * wi + 16 * ps;  // row within the item
+      bool released = false;
+      static_assert(kPasses == 1, "one 16-row pass per warp and item");
+      {
+        const int r = kRowsPerWarp * wi;  // row within the item
         const uint32_t kp = (uint32_t)(r >> p.log2P);
         const int row0 = r & (p.P - 1);
         if (kp < np && !((d.y >> (kMetaBadShift + kp)) & 1u)) {
@@ -1384,12 +1553,23 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
             else if (lane == 0)
               report(p.err, SKV_ERR_ARG);
           }
-          process_rows<G, DENSE, CAP>(p, d.x + rel, (d.y >> (kMetaTierShift + 2 * kp)) & 3u, row0,
-                                      qf, tb1, tb2, st, lane, lg);
+          const uint32_t tier = (d.y >> (kMetaTierShift + 2 * kp)) & 3u;
+          if (!DENSE && (tier == SKV_TIER_T1 || tier == SKV_TIER_T2)) {
+            // code rows: everything this warp reads of the ring goes to
+            // registers first, then the warp releases its share of the item
+            CodeRows cr;
+            load_code_rows(d.x + rel, p.P, tier == SKV_TIER_T1, row0, lane, cr);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&sm.empty[s]));
+            released = true;
+            compute_code_rows<G, CAP>(p, cr, tier, row0, qf, tb1, tb2, st, lane, lg);
+          } else {
+            process_rows<G, DENSE, CAP>(p, d.x + rel, tier, row0, qf, tb1, tb2, st, lane, lg);
+          }
         }
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&sm.empty[s]));
+      if (lane == 0 && !released) mbar_arrive(smem_u32(&sm.empty[s]));
     }
     it = next_it;
 
