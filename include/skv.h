@@ -411,6 +411,15 @@ int skv_dense_decode_bf16(skv_ctx* ctx, const void* q, int q_dtype, int B, int H
    so that a caller can time the decode kernel alone with CUDA events. */
 int skv_set_profile_event(skv_ctx* ctx, void* event);
 
+/* The decode's bounded waits (the planner, issuers and consumers of a CTA
+   wait on shared-memory barriers for one another and for page copies): a
+   wait that runs longer than `cycles` SM clocks ends the CTA's work and
+   reports SKV_ERR_TIMEOUT in err_word; later calls work normally.  0 (the
+   default) means about one second.  A short limit exists to exercise that
+   error path: before the CTA leaves, every page copy it started is waited
+   for with the one-second limit, whatever `cycles` is. */
+int skv_set_wait_limit(skv_ctx* ctx, int64_t cycles);
+
 /* Synchronise `stream`, read the device error word, reset it to 0 and return
    SKV_OK or the recorded SKV_ERR_* code. */
 int skv_check(skv_ctx* ctx, int32_t* err_word, void* stream);

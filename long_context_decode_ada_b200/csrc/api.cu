@@ -27,6 +27,7 @@ struct skv_ctx {
   int t1_scheme = 0;            // 0: 6-bit angle + 2-bit share; 1: 5-bit + 3-bit
   int share_grid = 0;           // 2-bit share grid: 0 uniform, 1 Lloyd-Max
   int deterministic = 0;        // the decode's split is static (no run-time chunks)
+  long long wait_limit = 0;     // decode waits: SM clocks (0: the default, about 1 s)
   float kappa[3];
   float rho_levels[4];
   long long payload[4];
@@ -513,6 +514,7 @@ static int decode_common(skv_ctx* ctx, const void* q, int q_dtype, int B, int Hq
   p.t1_scheme = ctx->t1_scheme;
   p.share_grid = ctx->share_grid;
   p.dynamic = ctx->deterministic ? 0 : 1;
+  p.wait_limit = ctx->wait_limit > 0 ? ctx->wait_limit : 2000000000LL;
   cudaError_t e =
       skv::launch_decode(p, G, dense, static_cast<cudaStream_t>(stream), ctx->profile_event);
   if (e != cudaSuccess) return cuda_fail(e, name);
@@ -752,6 +754,12 @@ int skv_decode_attention_static(skv_ctx* ctx, const void* q, int q_dtype, int B,
 int skv_set_profile_event(skv_ctx* ctx, void* event) {
   if (!ctx) return fail(SKV_ERR_ARG, "skv_set_profile_event: null ctx");
   ctx->profile_event = static_cast<cudaEvent_t>(event);
+  return ok();
+}
+
+int skv_set_wait_limit(skv_ctx* ctx, int64_t cycles) {
+  if (!ctx || cycles < 0) return fail(SKV_ERR_ARG, "skv_set_wait_limit: null ctx or negative limit");
+  ctx->wait_limit = cycles;
   return ok();
 }
 

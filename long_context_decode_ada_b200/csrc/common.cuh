@@ -96,18 +96,28 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parit
   return ok != 0;
 }
 
-// A bounded wait: ~1 s of SM clocks at most.  Returns false when the limit
-// runs out or when another thread of the CTA has raised *abort.
+// A bounded wait: `limit` SM clocks at most (kWaitLimitCycles, ~1 s, by
+// default).  Returns false when the limit runs out or when another thread
+// of the CTA has raised *abort.
 constexpr long long kWaitLimitCycles = 2000000000LL;
 
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
-                                                  volatile int* abort_flag) {
+                                                  volatile int* abort_flag,
+                                                  long long limit = kWaitLimitCycles) {
+  if (limit < kWaitLimitCycles) {
+    // a short limit (set to exercise the timeout path): poll without
+    // suspending, so that the limit and not a sleep decides
+    const long long t0 = clock64();
+    while (!mbar_test_wait(bar, parity))
+      if (*abort_flag || clock64() - t0 > limit) return false;
+    return true;
+  }
   if (mbar_try_wait(bar, parity)) return true;
   long long t0 = clock64();
   while (true) {
     if (mbar_try_wait_sleep(bar, parity, 200000u)) return true;
     if (*abort_flag) return false;
-    if (clock64() - t0 > kWaitLimitCycles) return false;
+    if (clock64() - t0 > limit) return false;
   }
 }
 

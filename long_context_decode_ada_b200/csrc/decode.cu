@@ -259,9 +259,19 @@ __device__ __noinline__ void find_run(const SplitInfo& si, int c, int S, Smem& s
   const int nseg = 3 * si.U;
   const int per = (nseg + nt - 1) / nt;
   const int k0 = min(nseg, tid * per), k1 = min(nseg, k0 + per);
+  // the segment starts this thread needs in both passes (k0 .. k0 + 3, which
+  // covers a unit's four when k0 starts one), loaded together: one memory
+  // round trip on the start-up path
+  long long pre[4];
+#pragma unroll
+  for (int t = 0; t < 4; ++t) pre[t] = (k0 < k1 && k0 + t <= nseg) ? si.seg_start(k0 + t) : 0;
   unsigned long long loc = 0;
-  for (int k = k0; k < k1; ++k)
-    loc += (unsigned long long)(si.seg_start(k + 1) - si.seg_start(k)) * si.weight(k);
+  if (per == 1) {
+    if (k0 < k1) loc = (unsigned long long)(pre[1] - pre[0]) * si.weight(k0);
+  } else {
+    for (int k = k0; k < k1; ++k)
+      loc += (unsigned long long)(si.seg_start(k + 1) - si.seg_start(k)) * si.weight(k);
+  }
   if (k1 == nseg && k0 < k1) {
     // the page count is known: CTA c brings slice c of the page-id array into
     // L2, so that every planner's first id loads (after the split) hit L2
@@ -308,7 +318,7 @@ __device__ __noinline__ void find_run(const SplitInfo& si, int c, int S, Smem& s
         long long seg[4];
         unsigned long long cr[4];
 #pragma unroll
-        for (int t = 0; t < 4; ++t) seg[t] = si.seg_start(k + t);
+        for (int t = 0; t < 4; ++t) seg[t] = (k == k0) ? pre[t] : si.seg_start(k + t);
         cr[0] = 0;
 #pragma unroll
         for (int t = 0; t < 3; ++t) cr[t + 1] = cr[t] + (unsigned long long)(seg[t + 1] - seg[t]) * si.weight(t);
@@ -324,7 +334,8 @@ __device__ __noinline__ void find_run(const SplitInfo& si, int c, int S, Smem& s
           // 1/kDynDen of its pages (none for a unit with a single run); the
           // static part [seg[0], M) is cut into the n runs by cost
           const long long cp = (long long)kChunkItems * ipp;
-          const long long nch = (dynamic && n >= 2) ? (seg[3] - seg[0]) / (kDynDen * cp) : 0;
+          const long long nch =
+              (dynamic && n >= 2) ? (long long)udiv64((unsigned long long)(seg[3] - seg[0]), kDynDen * cp) : 0;
           const long long M = seg[3] - nch * cp;
           long long sg[4];
           unsigned long long cs[4];
@@ -1083,7 +1094,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     // wait until item `tail` is released, then advance tail
     auto release_tail = [&]() -> bool {
       if (!mbar_wait_bounded(smem_u32(&sm.empty[tail % kNSlot]), (uint32_t)((tail / kNSlot) & 1),
-                             &sm.abort_flag))
+                             &sm.abort_flag, p.wait_limit))
         return false;
       ++tail;
       return true;
@@ -1118,7 +1129,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         // workspace) and, in the unit's first run, reset the counter
         const long long t0 = clock64();
         while (ld_volatile(&sm.dyn_go) == 0) {
-          if (ld_volatile(&sm.abort_flag) || clock64() - t0 > kWaitLimitCycles) {
+          if (ld_volatile(&sm.abort_flag) || clock64() - t0 > p.wait_limit) {
             grab_ok = false;  // no grab: fut stays 0, whose tag matches no launch
             break;
           }
@@ -1337,7 +1348,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     while (true) {
       const int s = it % kNSlot;
       if (!mbar_wait_bounded(smem_u32(&sm.ready[s]), (uint32_t)((it / kNSlot) & 1),
-                             &sm.abort_flag)) {
+                             &sm.abort_flag, p.wait_limit)) {
         ok = false;
         break;
       }
@@ -1369,6 +1380,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       report(p.err, SKV_ERR_TIMEOUT);
       sm.abort_flag = 1;
       // let every copy this issuer started land before the CTA can exit
+      // (with the fixed ~1 s limit, whatever the run-time wait limit: no CTA
+      // may leave with a copy into its shared memory in flight)
       const long long t0 = clock64();
       for (int jj = it - kIss; jj >= 0 && jj >= it - kNSlot; jj -= kIss) {
         while (!mbar_try_wait(smem_u32(&sm.full[jj % kNSlot]), (uint32_t)((jj / kNSlot) & 1)) &&
@@ -1517,8 +1530,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       // published the slot's previous item has been released, so `full`
       // is then at itm's own phase.
       const uint32_t readyb = smem_u32(&sm.ready[s]), fullb = smem_u32(&sm.full[s]);
-      if ((!mbar_test_wait(readyb, par) && !mbar_wait_bounded(readyb, par, &sm.abort_flag)) ||
-          (!mbar_test_wait(fullb, par) && !mbar_wait_bounded(fullb, par, &sm.abort_flag))) {
+      if ((!mbar_test_wait(readyb, par) && !mbar_wait_bounded(readyb, par, &sm.abort_flag, p.wait_limit)) ||
+          (!mbar_test_wait(fullb, par) && !mbar_wait_bounded(fullb, par, &sm.abort_flag, p.wait_limit))) {
         ok = false;
         if (lane == 0) {
           report(p.err, SKV_ERR_TIMEOUT);

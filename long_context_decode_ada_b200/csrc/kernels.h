@@ -37,6 +37,7 @@ struct DecodeParams {
   int t1_scheme;             // T1 code byte: 0 (angle6 << 2) | share2; 1 (angle5 << 3) | share3
   int share_grid;            // 2-bit share grid: 0 uniform, 1 Lloyd-Max
   int dynamic;               // unit-aligned split: hand out the units' last pages at run time
+  long long wait_limit;      // SM clocks a planner / issuer / consumer wait may take
 };
 
 struct EncodeParams {

@@ -36,7 +36,7 @@ EXPORTS = [
     "skv_decode_utility", "skv_merge_partials",
     "skv_dense_pack_bf16",
     "skv_dense_decode_bf16",
-    "skv_set_profile_event", "skv_check",
+    "skv_set_profile_event", "skv_set_wait_limit", "skv_check",
 ]
 
 
@@ -84,6 +84,7 @@ _SIGS = {
     "skv_dense_decode_bf16": (_i, [_p, _p, _i, _i, _i, _i, _p, _p, _p, _i64, _p, _p, _p, _p, _sz,
                                    _i, _p]),
     "skv_set_profile_event": (_i, [_p, _p]),
+    "skv_set_wait_limit": (_i, [_p, _i64]),
     "skv_check": (_i, [_p, _p, _p]),
 }
 
@@ -236,6 +237,11 @@ class Context:
 
     def check(self, err: torch.Tensor, stream=None):
         _check(lib().skv_check(self._h, _ptr(err), _stream(stream)))
+
+    def set_wait_limit(self, cycles: int):
+        """SM clocks a decode wait may take before the call ends with
+        SKV_ERR_TIMEOUT (0: the default, about one second)."""
+        _check(lib().skv_set_wait_limit(self._h, int(cycles)))
 
     def set_profile_event(self, event: Optional[torch.cuda.Event]):
         """Record `event` between the decode and merge kernels of later calls."""

@@ -7,7 +7,7 @@ sampled (sequence, query head) rows, which the oracle computes one by one.
 Workloads: the Llama-3-8B-shaped layer (8 x 32768, P = 64, quota tiers),
 the 128K long-context store (budget mode, protected sink and recent
 window), the ragged batch of 64 sequences (P = 16, scattered pages) and
-two layers of the 32-layer pipeline (budget mode, outlier channels)."""
+eight layers of the 32-layer pipeline (budget mode, outlier channels)."""
 import numpy as np
 import pytest
 
@@ -64,7 +64,12 @@ def test_ragged_batch_full_size():
     full_size_check(w, nrows=32, seed=4)
 
 
-@pytest.mark.parametrize("layer", [0, 31])
+@pytest.mark.parametrize("layer", [0, 4, 9, 13, 18, 22, 27, 31])
 def test_pipeline_layer_full_size(layer):
+    """Eight layers spread over the 32 (each its own outlier channels and
+    utilities): store bit-exact, sampled rows within tolerance; the stores
+    hold T2 pages and dropped tokens."""
     w = wl.pipeline_layer(layer)
-    full_size_check(w, seed=5 + layer)
+    g, ref, npages = full_size_check(w, nrows=16 if layer not in (0, 31) else 24, seed=5 + layer)
+    counts = np.bincount(ref["tier"].ravel(), minlength=4)
+    assert counts[1] and counts[2] and counts[3]
