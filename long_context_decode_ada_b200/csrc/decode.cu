@@ -185,7 +185,8 @@ struct SplitInfo {
     return (k - 3 * u) == 0 ? indptr[u] : indptr[u + 1];
   }
   __device__ __forceinline__ unsigned long long weight(int k) const {
-    return (unsigned long long)w[k % 3];
+    const int t = k % 3;  // selects, not an indexed load: w stays in registers
+    return (unsigned long long)(t == 0 ? w[0] : (t == 1 ? w[1] : w[2]));
   }
 };
 
@@ -213,15 +214,23 @@ __device__ __forceinline__ long long run_begin_in_unit(const SplitInfo& si,
                                                        const unsigned long long* cseg,
                                                        unsigned long long T,
                                                        unsigned long long S) {
+  // unrolled with a result variable (constant indexes keep seg / cseg in
+  // registers)
+  long long res = seg[3];
+  bool found = false;
+#pragma unroll
   for (int t = 0; t < 3; ++t) {
     const unsigned long long lo = cseg[t] * S, hi = cseg[t + 1] * S;
-    if (T <= lo) return seg[t];
-    if (T <= hi) {
+    if (!found && T <= lo) {
+      res = seg[t];
+      found = true;
+    } else if (!found && T <= hi) {
       const unsigned long long ws = si.weight(t) * S;
-      return seg[t] + (long long)udiv64(T - lo + ws - 1, ws);
+      res = seg[t] + (long long)udiv64(T - lo + ws - 1, ws);
+      found = true;
     }
   }
-  return seg[3];
+  return res;
 }
 
 // Unit-aligned split (used when there are at most as many units as runs):
@@ -253,7 +262,7 @@ __device__ __forceinline__ int unit_first_run(int u, unsigned long long Pu, unsi
 // its first and last unit, the total cost, and the cost before every
 // segment of the units it touches (when they are at most kTouchedUnits).
 template <class Smem>
-__device__ __noinline__ void find_run(const SplitInfo& si, int c, int S, Smem& sm, int tid,
+__device__ __forceinline__ void find_run(const SplitInfo& si, int c, int S, Smem& sm, int tid,
                                       const uint32_t* ids, int ipp, bool dynamic) {
   constexpr int nt = kDecodeThreads;
   const int nseg = 3 * si.U;
@@ -1308,28 +1317,47 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     // unit, loaded one unit ahead (a unit-aligned run lies inside its unit)
     long long ub = in_unit ? g1 : min(g1, (long long)p.indptr[u0 + 1]);
     long long ub_next = (!in_unit && u0 + 2 <= U) ? (long long)p.indptr[u0 + 2] : g1;
-    while (ok && pg < g1) {
-      while (pg >= ub) {  // next unit with pages in this run
-        ++u;
-        ub = min(g1, ub_next);
-        ub_next = u + 2 <= U ? (long long)p.indptr[u + 2] : g1;
-      }
-      ok = plan_range(pg, ub, dyn_chunks > 0);
-      while (ok && dyn_chunks > 0) {
-        // dynamic chunks of the unit, one grab in flight ahead of the chunk
-        // being planned
+    // One loop, one call of plan_range (so that it is inlined and the
+    // planner's state stays in registers): each pass plans one range, the
+    // run's part of the next unit or, after a unit's static part, the next
+    // dynamic chunk grabbed (one grab in flight ahead of the chunk being
+    // planned).  A unit ends with one marker per consumer group, carrying
+    // the index of the next unit's first item.
+    bool chunks = false;  // the current unit's static part is planned: take chunks
+    while (ok) {
+      long long rs, re;
+      bool grab_last = false, unit_end = false;
+      if (chunks) {
         const unsigned long long got = __shfl_sync(0xFFFFFFFFu, fut, 0);
         const uint32_t k = (uint32_t)got;
-        if ((uint32_t)(got >> 32) != tag || k >= (uint32_t)dyn_chunks) break;
+        if ((uint32_t)(got >> 32) != tag || k >= (uint32_t)dyn_chunks) {
+          chunks = false;
+          const uint32_t next_first = (uint32_t)(it + kCG);
+          for (int e = 0; e < kCG && ok; ++e) ok = publish_marker(kMetaUnitEnd, next_first, 0u);
+          continue;
+        }
         issue_grab();
-        const long long cs = dyn_m + (long long)k * dyn_cp;
-        ok = plan_range(cs, cs + dyn_cp, false);
+        rs = dyn_m + (long long)k * dyn_cp;
+        re = rs + dyn_cp;
+      } else {
+        if (pg >= g1) break;
+        while (pg >= ub) {  // next unit with pages in this run
+          ++u;
+          ub = min(g1, ub_next);
+          ub_next = u + 2 <= U ? (long long)p.indptr[u + 2] : g1;
+        }
+        rs = pg;
+        re = ub;
+        pg = ub;
+        grab_last = dyn_chunks > 0;
+        chunks = dyn_chunks > 0;
+        unit_end = !chunks;
       }
-      // the unit's end: one marker per consumer group, carrying the index
-      // of the next unit's first item
-      const uint32_t next_first = (uint32_t)(it + kCG);
-      for (int e = 0; e < kCG && ok; ++e) ok = publish_marker(kMetaUnitEnd, next_first, 0u);
-      pg = ub;
+      ok = plan_range(rs, re, grab_last);
+      if (ok && unit_end) {
+        const uint32_t next_first = (uint32_t)(it + kCG);
+        for (int e = 0; e < kCG && ok; ++e) ok = publish_marker(kMetaUnitEnd, next_first, 0u);
+      }
     }
     // end-of-run markers: a slot each (its previous item released)
     for (int e = 0; e < kIss && ok; ++e) ok = publish_marker(0u, 0u, kEndOfRun);
