@@ -63,6 +63,7 @@ _SIGS = {
     "orc_logit_recon": (_d, [_p, _p, _i, _i]),
     "orc_logit_variant": (_d, [_p, _p, _i, _i, _i]),
     "orc_allocate": (_i, [_i, _i, _i, _i, _i, _p, _p, _p, _p, _i, _p, _p, _p]),
+    "orc_retier": (_i, [_i, _i, _i, _i, _i, _p, _p, _p, _p, _p, _p, _p]),
     "orc_page_payload": (_i64, [_i, _i, _i]),
     "orc_page_stride": (_i64, [_i, _i, _i]),
     "orc_pack": (_i, [_i, _i, _i, _i, _i,                     # B Hkv Tmax d P
@@ -257,6 +258,26 @@ def allocate(B, Hkv, Tmax, d, P, seq_lens, K, utility, protect, mode, budget, qu
                             _ptr(bud), _ptr(quo), _ptr(tier))
     if check and rc != OK:
         raise OracleError(rc, "allocate")
+    return (tier, rc) if not check else tier
+
+
+def retier(B, Hkv, Tmax, d, P, seq_lens, K, utility, tier_in, demote, budget,
+           check: bool = True):
+    """New tiers of a store whose rows flagged in `demote` (all T0) are
+    re-decided under the budget, the other resident tokens keeping their
+    tiers: uint8 [B][Hkv][Tmax] (3 = dropped); with check=False also the
+    status (ERR_BUDGET: the kept tokens alone exceed the budget)."""
+    seq = np.ascontiguousarray(seq_lens, np.int32)
+    k = _u16(K)
+    u = np.ascontiguousarray(utility.numpy() if hasattr(utility, "numpy") else utility, np.float32)
+    tin = np.ascontiguousarray(tier_in, np.uint8)
+    dm = np.ascontiguousarray(demote.numpy() if hasattr(demote, "numpy") else demote, np.uint8)
+    bud = np.ascontiguousarray(budget, np.int64)
+    tier = np.empty((B, Hkv, Tmax), np.uint8)
+    rc = lib().orc_retier(B, Hkv, Tmax, d, P, _ptr(seq), _ptr(k), _ptr(u), _ptr(tin), _ptr(dm),
+                          _ptr(bud), _ptr(tier))
+    if check and rc != OK:
+        raise OracleError(rc, "retier")
     return (tier, rc) if not check else tier
 
 

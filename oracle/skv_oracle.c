@@ -628,6 +628,84 @@ int orc_allocate(int B, int Hkv, int Tmax, int d, int P, const int32_t* seq_lens
     return err;
 }
 
+/* Re-tiering of a store's rows under its budget ([TS 2.2] keep/drop and
+   tier per token and head under a fixed budget; [TS 2.3] the retention
+   filter between the codes and the store, applied again as tokens age out
+   of the protected recent window).  Every resident token keeps its tier
+   except those marked in `demote`, which must be T0 (rows leaving the
+   recent window, whose exact fp16 keys the store still holds): they take
+   the greedy walk of orc_allocate's budget mode among themselves, with the
+   budget left after the kept tokens' bytes and the partial-page reserve,
+   budget - sum(tier bytes of kept tokens) - Hkv*(P-1)*(512+196+180).
+   Their steps, keys, ordering and prefix rule are orc_allocate's.  When the
+   kept tokens alone exceed that budget the demoted tokens are dropped and
+   ORC_ERR_BUDGET is returned (the store is over budget).  A demote flag on
+   a token that is not T0, or on a position past the sequence, is
+   ORC_ERR_ARG.  Positions at or beyond seq_lens[b] are dropped. */
+int orc_retier(int B, int Hkv, int Tmax, int d, int P, const int32_t* seq_lens,
+               const uint16_t* K, const float* utility, const uint8_t* tier_in,
+               const uint8_t* demote, const int64_t* budget, uint8_t* tier_out) {
+    if (B < 0 || Hkv <= 0 || Tmax < 0 || d <= 0 || P <= 0 || !utility) return ORC_ERR_ARG;
+    float kappa[3];
+    orc_kappa(d, kappa);
+    const int64_t step_bytes[3] = {
+        orc_tier_bytes(TIER_T2, d),
+        orc_tier_bytes(TIER_T1, d) - orc_tier_bytes(TIER_T2, d),
+        orc_tier_bytes(TIER_T0, d) - orc_tier_bytes(TIER_T1, d)};
+    int err = ORC_OK;
+    for (int b = 0; b < B; b++) {
+        int T = seq_lens[b];
+        if (T < 0 || T > Tmax) return ORC_ERR_ARG;
+        int64_t kept = 0, nsteps = 0;
+        for (int h = 0; h < Hkv; h++)
+            for (int t = 0; t < Tmax; t++) {
+                int64_t idx = ((int64_t)b * Hkv + h) * Tmax + t;
+                uint8_t tr = t < T ? tier_in[idx] : TIER_DROP;
+                if (demote && demote[idx]) {
+                    if (t >= T || tr != TIER_T0) return ORC_ERR_ARG;
+                    tier_out[idx] = TIER_DROP;
+                    nsteps += 3;
+                    continue;
+                }
+                if (tr > TIER_DROP) return ORC_ERR_ARG;
+                tier_out[idx] = tr;
+                if (tr != TIER_DROP) kept += orc_tier_bytes(tr, d);
+            }
+        int64_t left = budget[b] - kept -
+                       (int64_t)Hkv * (P - 1) *
+                           (orc_tier_bytes(TIER_T0, d) + orc_tier_bytes(TIER_T1, d) +
+                            orc_tier_bytes(TIER_T2, d));
+        if (left < 0) { err = ORC_ERR_BUDGET; continue; }
+        step_t* st = (step_t*)malloc(sizeof(step_t) * (nsteps > 0 ? nsteps : 1));
+        int64_t n = 0;
+        for (int h = 0; h < Hkv; h++)
+            for (int t = 0; t < T; t++) {
+                int64_t idx = ((int64_t)b * Hkv + h) * Tmax + t;
+                if (!(demote && demote[idx])) continue;
+                uint64_t R2[2];
+                orc_norm2(K + idx * d, d, R2);
+                float w = utility[idx] * r2_float(R2);
+                for (int k = 0; k < 3; k++) {
+                    st[n].key = w * kappa[k];
+                    st[n].k = k;
+                    st[n].h = h;
+                    st[n].t = t;
+                    n++;
+                }
+            }
+        qsort(st, n, sizeof(step_t), step_cmp);
+        int64_t used = 0;
+        for (int64_t i = 0; i < n; i++) {
+            if (used + step_bytes[st[i].k] > left) break;
+            used += step_bytes[st[i].k];
+            int64_t idx = ((int64_t)b * Hkv + st[i].h) * Tmax + st[i].t;
+            tier_out[idx] = (uint8_t)(st[i].k == 0 ? TIER_T2 : (st[i].k == 1 ? TIER_T1 : TIER_T0));
+        }
+        free(st);
+    }
+    return err;
+}
+
 /* ------------------------------------------------------------------ */
 /* Paged store [TS 2.2 tier-homogeneous pages], [TS 2.3], [ABS]        */
 /* ------------------------------------------------------------------ */
