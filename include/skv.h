@@ -224,7 +224,8 @@ int skv_encode(skv_ctx* ctx, const uint16_t* K, const uint16_t* V, int B, int Hk
    unit order) inserted at the end of the unit's T0 segment; later page ids
    move up and the unit's T1/T2 rows move one page down in row_of.  The
    store then equals what skv_allocate + skv_encode give for the same tiers
-   (page slots aside).  Re-running skv_allocate later demotes ageing tokens.
+   (page slots aside).  skv_retier later demotes the rows that leave the
+   protected window.
      K_new, V_new  fp16 [B][Hkv][128] device: the new token's key and value
      Tmax          capacity of tier/row_of; seq_lens[b] < Tmax is required
      seq_lens      int32 [B] device, incremented by one
@@ -243,6 +244,56 @@ int skv_append(skv_ctx* ctx, const uint16_t* K_new, const uint16_t* V_new, int B
                int32_t* page_indptr, int32_t* page_tier_indptr, uint32_t* page_ids,
                int64_t page_cap, const skv_pools* pools, const uint32_t* free0,
                int64_t free0_len, int32_t* free0_cursor, int32_t* err_word, void* workspace,
+               size_t ws_bytes, void* stream);
+
+/* skv_retier -- re-tiering of rows leaving the protected recent window, on
+   the store itself (technical summary 2.2, Rate-Distortion Retention: keep
+   or drop and the tier are per-token, per-head decisions under a fixed
+   budget; 2.3, System Integration: the retention filter sits between the
+   codes and the paged store).  The demoted rows are T0 rows; their exact
+   fp16 K and V are read back from their T0 pages, so no dense K/V is
+   needed.  Every other resident token keeps its tier.  The demoted rows are
+   re-decided by the budget walk of skv_allocate: with
+     left = budget[b] - (bytes of the kept tokens) - Hkv (P-1) (512+196+180)
+   their upgrade steps (drop->T2, T2->T1, T1->T0; keys u fp32(r^2) kappa,
+   ties by step, head, position) are taken in order while they fit, so a
+   demoted row ends T0, T1, T2 or dropped.  The store is then what
+   skv_allocate's layout + skv_encode give for the new tiers (page slots
+   aside), updated in place: in each (unit, tier) page segment the pages
+   wholly before the first changed row keep their slots; the later pages
+   are rewritten into slots free->ids[t][free_cursor[t] + k] and the old ones
+   are listed in `released`.
+     seq_lens      int32 [B] device (unchanged)
+     utility       fp32 [B][Hkv][Tmax] device: utilities of the demoted rows
+     demote        uint8 [B][Hkv][Tmax] device: 1 = re-decide this row (it must
+                   be resident T0; SKV_ERR_ARG otherwise, the row then kept)
+     budget        int64 [B] device: bytes per sequence
+     free, free_cursor  device free lists per tier and int32 [3] device
+                   cursors (first unused entry), advanced by the slots taken
+     pools         the pools of the store (128-byte aligned)
+     tier, row_of, page_indptr, page_tier_indptr (required), page_ids: the
+                   store's arrays, rewritten
+     page_cap      capacity of page_ids
+     released      uint32 [page_cap] device: ids (tier << 30 | slot) of the old
+                   pages that the store no longer references; n_released
+                   (int32 device) their count.  They may go back to the
+                   caller's free lists once the call has completed.
+     workspace     skv_retier_workspace_size() bytes of device scratch
+   Device errors: SKV_ERR_BUDGET when the kept tokens and the reserve
+   exceed a sequence's budget (its demoted rows are then dropped; the store
+   stays consistent); SKV_ERR_POOL (free list or page capacity exhausted)
+   and SKV_ERR_CORRUPT (a bad page id or row) leave the store invalid: it
+   must be rebuilt with skv_allocate + skv_encode.  Budget mode only; no
+   outlier protection is applied to the demoted rows (leave such rows out of
+   `demote`). */
+int skv_retier_workspace_size(const skv_ctx* ctx, int B, int Hkv, int64_t Tmax,
+                              int64_t page_cap, size_t* bytes);
+int skv_retier(skv_ctx* ctx, int B, int Hkv, int64_t Tmax, const int32_t* seq_lens,
+               const float* utility, const uint8_t* demote, const int64_t* budget,
+               const skv_free_lists* free, int32_t* free_cursor, const skv_pools* pools,
+               uint8_t* tier, int32_t* row_of, int32_t* page_indptr,
+               int32_t* page_tier_indptr, uint32_t* page_ids, int64_t page_cap,
+               uint32_t* released, int32_t* n_released, int32_t* err_word, void* workspace,
                size_t ws_bytes, void* stream);
 
 /* skv_decode_attention -- the ADA decode step (technical summary 2.1: logits

@@ -53,7 +53,7 @@ void alloc_carve(AllocParams& p, void* ws) {
   w += al256(4 * U * 3);
   p.tbase = reinterpret_cast<int32_t*>(w);
   w += al256(4 * U * 3);
-  p.nprot = reinterpret_cast<long long*>(w);
+  p.pinned = reinterpret_cast<long long*>(w);
   w += al256(8 * (size_t)p.B);
   p.eff_protect = w;
 }
@@ -109,22 +109,10 @@ __device__ __forceinline__ float valid_utility(const AllocParams& p, long long i
   return u;
 }
 
-// budget mode: one warp per token; keyw = u * fp32(r^2), -1 when protected
-__global__ void __launch_bounds__(256) keys_budget_kernel(const __grid_constant__ AllocParams p) {
-  const long long w = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (w >= (long long)p.B * p.Hkv * p.Tmax) return;
-  const long long t = w % p.Tmax;
-  const int b = (int)(w / p.Tmax / p.Hkv);
-  if (t >= p.seq_lens[b]) return;
-  if (p.protect && p.protect[w]) {
-    if (lane == 0) {
-      p.keyw[w] = -1.0f;
-      atomicAdd(reinterpret_cast<unsigned long long*>(&p.nprot[b]), 1ull);
-    }
-    return;
-  }
-  const uint2 kv = *reinterpret_cast<const uint2*>(p.K + w * kHeadDim + 4 * lane);
+// fp32(r^2) of a key from the warp's 32 lanes, each holding four of its fp16
+// components (any assignment of components to lanes: the sum of squares is
+// exact in 128-bit integers), rounded once to fp64 and once to fp32.
+__device__ __forceinline__ float warp_r2f(uint2 kv) {
   const uint16_t k4[4] = {(uint16_t)(kv.x & 0xFFFF), (uint16_t)(kv.x >> 16),
                           (uint16_t)(kv.y & 0xFFFF), (uint16_t)(kv.y >> 16)};
   u128 sq = 0;
@@ -141,11 +129,76 @@ __global__ void __launch_bounds__(256) keys_budget_kernel(const __grid_constant_
     unsigned long long ohi = __shfl_xor_sync(0xFFFFFFFFu, hi, o);
     sq += ((u128)ohi << 64) | olo;
   }
-  if (lane == 0) {
-    const double r2 = u128_to_double_rn((unsigned long long)(sq >> 64), (unsigned long long)sq);
-    const float r2f = __double2float_rn(__dmul_rn(r2, 3.552713678800501e-15));  // 2^-48
-    p.keyw[w] = __fmul_rn(valid_utility(p, w), r2f);
+  const double r2 = u128_to_double_rn((unsigned long long)(sq >> 64), (unsigned long long)sq);
+  return __double2float_rn(__dmul_rn(r2, 3.552713678800501e-15));  // 2^-48
+}
+
+// A token whose tier is fixed: keyw = -1 - tier (no upgrade steps), and its
+// bytes count against the sequence's budget before the walk.
+__device__ __forceinline__ void pin_token(const AllocParams& p, long long w, int b, int tier) {
+  p.keyw[w] = -1.0f - (float)tier;
+  if (tier < SKV_TIER_DROP)
+    atomicAdd(reinterpret_cast<unsigned long long*>(&p.pinned[b]),
+              (unsigned long long)tier_row_bytes(tier));
+}
+
+// budget mode: one warp per token; keyw = u * fp32(r^2), -1 when protected
+__global__ void __launch_bounds__(256) keys_budget_kernel(const __grid_constant__ AllocParams p) {
+  const long long w = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (w >= (long long)p.B * p.Hkv * p.Tmax) return;
+  const long long t = w % p.Tmax;
+  const int b = (int)(w / p.Tmax / p.Hkv);
+  if (t >= p.seq_lens[b]) return;
+  if (p.protect && p.protect[w]) {
+    if (lane == 0) pin_token(p, w, b, SKV_TIER_T0);
+    return;
   }
+  const float r2f = warp_r2f(*reinterpret_cast<const uint2*>(p.K + w * kHeadDim + 4 * lane));
+  if (lane == 0) p.keyw[w] = __fmul_rn(valid_utility(p, w), r2f);
+}
+
+// re-tiering: a demoted token (T0 in the old store) gets the budget key from
+// the fp16 key in its old T0 page (its row order does not matter for r^2);
+// every other resident token keeps its old tier.
+__global__ void __launch_bounds__(256) keys_retier_kernel(const __grid_constant__ AllocParams p) {
+  const long long w = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (w >= (long long)p.B * p.Hkv * p.Tmax) return;
+  const long long t = w % p.Tmax;
+  const long long u = w / p.Tmax;
+  const int b = (int)(u / p.Hkv);
+  if (t >= p.seq_lens[b]) return;
+  const int to = p.tier_old[w];
+  if (to > SKV_TIER_DROP) {
+    if (lane == 0) {
+      report(p.err, SKV_ERR_CORRUPT);
+      pin_token(p, w, b, SKV_TIER_DROP);
+    }
+    return;
+  }
+  if (!p.demote[w] || to != SKV_TIER_T0) {
+    if (lane == 0) {
+      if (p.demote[w]) report(p.err, SKV_ERR_ARG);  // only T0 rows can be demoted
+      pin_token(p, w, b, to);
+    }
+    return;
+  }
+  const int row = p.row_old[w];
+  const long long gi = (long long)p.indptr_old[u] + (row >= 0 ? row / p.P : 0);
+  const uint32_t id =
+      row >= 0 && gi < p.tindptr_old[3 * u + 1] && gi < p.page_cap ? p.ids_old[gi] : 0xFFFFFFFFu;
+  const uint32_t slot = id & 0x3FFFFFFFu;
+  if ((id >> 30) != 0u || (long long)slot >= p.slots[0]) {
+    if (lane == 0) {
+      report(p.err, SKV_ERR_CORRUPT);
+      pin_token(p, w, b, SKV_TIER_DROP);
+    }
+    return;
+  }
+  const uint8_t* krow = p.pool[0] + (long long)slot * p.stride[0] + kHdrBytes + 256 * (row % p.P);
+  const float r2f = warp_r2f(*reinterpret_cast<const uint2*>(krow + 8 * lane));
+  if (lane == 0) p.keyw[w] = __fmul_rn(valid_utility(p, w), r2f);
 }
 
 // quota mode: keyw = u (0 without utilities), -1 when protected
@@ -175,7 +228,7 @@ __global__ void sel_init_kernel(const __grid_constant__ AllocParams p) {
       return;
     }
     const long long reserve = (long long)p.Hkv * (p.P - 1) * (512 + 196 + 180);
-    const long long left = p.budget[seg] - 512LL * p.nprot[seg] - reserve;
+    const long long left = p.budget[seg] - p.pinned[seg] - reserve;
     if (left < 0) {
       report(p.err, SKV_ERR_BUDGET);
       st[2] = 1;  // prefix 0: nothing is selected
@@ -300,7 +353,7 @@ __global__ void tier_kernel(const __grid_constant__ AllocParams p) {
   if (t < p.seq_lens[b]) {
     const float w = p.keyw[i];
     if (w < 0.0f) {
-      tr = SKV_TIER_T0;
+      tr = (uint8_t)(-1 - (int)w);  // a fixed tier
     } else if (p.mode == SKV_MODE_BUDGET) {
       const unsigned long long cut = p.sel[(size_t)b * 3 * 3 + 0];
       int lvl = 0;
@@ -382,27 +435,72 @@ __device__ long long block_exclusive_scan(long long v, long long& total) {
   return before;
 }
 
+// re-tiering: the first row of each (unit, tier) segment at which the new
+// store differs from the old one -- a new row holding another token than
+// the old row of that index, or an old row whose token moved or left (rows
+// counted within the segment).  Rows of a segment are in position order in
+// both stores, so every page wholly before that row is byte-identical in
+// both (rows, count and header) and stays where it is.
+__global__ void diff_kernel(const __grid_constant__ AllocParams p) {
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= (long long)p.B * p.Hkv * p.Tmax) return;
+  const long long t = i % p.Tmax, u = i / p.Tmax;
+  if (t >= p.seq_lens[u / p.Hkv]) return;
+  const int tn = p.tier_out[i], to = p.tier_old[i];
+  // row within the tier's segment: row_of counts from the unit's first page,
+  // so the segment's page base (the pages of the tiers before it) comes off
+  const int P = p.P;
+  int rn = -1, ro = -1;
+  if (tn < SKV_TIER_DROP) {
+    const int c0 = p.counts[3 * u], c1 = p.counts[3 * u + 1];
+    const int pb = tn == 0 ? 0 : (c0 + P - 1) / P + (tn == 2 ? (c1 + P - 1) / P : 0);
+    rn = p.row_of[i] - pb * P;
+  }
+  if (to < SKV_TIER_DROP)
+    ro = p.row_old[i] - (p.tindptr_old[3 * u + to] - p.indptr_old[u]) * P;
+  if (tn == to && rn == ro) return;
+  if (tn < SKV_TIER_DROP) atomicMin(&p.diff[3 * u + tn], max(rn, 0));
+  if (to < SKV_TIER_DROP) atomicMin(&p.diff[3 * u + to], max(ro, 0));
+}
+
+// CSR offsets of the new page table and, per (unit, tier), the first index
+// into the tier's free list.  A re-tiering keeps each segment's leading
+// unchanged pages (keep), takes free slots only for the others (from the
+// list's cursor on) and lists the old pages it no longer references.
 __global__ void __launch_bounds__(1024) page_plan_kernel(const __grid_constant__ AllocParams p) {
   const int U = p.B * p.Hkv;
   const int per = (U + blockDim.x - 1) / blockDim.x;
   const int u0 = threadIdx.x * per, u1 = min(U, u0 + per);
-  long long s[4] = {0, 0, 0, 0};
+  const bool rt = p.keep != nullptr;
+  long long cur[3] = {0, 0, 0};
+  if (rt)
+    for (int t = 0; t < 3; ++t) cur[t] = p.cursor[t];
+  // s[0..2]: free slots taken per tier, s[3]: pages, s[4]: old pages released
+  long long s[5] = {0, 0, 0, 0, 0};
   for (int u = u0; u < u1; ++u) {
     for (int t = 0; t < 3; ++t) {
       const long long np = (p.counts[u * 3 + t] + p.P - 1) / p.P;
-      s[t] += np;
+      long long kp = 0;
+      if (rt) {
+        const long long npo = p.tindptr_old[3 * u + t + 1] - p.tindptr_old[3 * u + t];
+        kp = min(min((long long)p.diff[3 * u + t] / p.P, np), npo);
+        p.keep[3 * u + t] = (int32_t)kp;
+        s[4] += npo - kp;
+      }
+      s[t] += np - kp;
       s[3] += np;
     }
   }
-  long long base[4], tot[4];
-  for (int k = 0; k < 4; ++k) base[k] = block_exclusive_scan(s[k], tot[k]);
+  long long base[5], tot[5];
+  for (int k = 0; k < 5; ++k) base[k] = block_exclusive_scan(s[k], tot[k]);
   for (int u = u0; u < u1; ++u) {
     p.indptr[u] = (int32_t)base[3];
+    if (rt) p.rbase[u] = (int32_t)base[4];
     for (int t = 0; t < 3; ++t) {
       if (p.tier_indptr) p.tier_indptr[u * 3 + t] = (int32_t)base[3];
-      p.tbase[u * 3 + t] = (int32_t)base[t];
+      p.tbase[u * 3 + t] = (int32_t)(cur[t] + base[t]);
       const long long np = (p.counts[u * 3 + t] + p.P - 1) / p.P;
-      base[t] += np;
+      base[t] += np - (rt ? p.keep[3 * u + t] : 0);
       base[3] += np;
     }
   }
@@ -410,8 +508,12 @@ __global__ void __launch_bounds__(1024) page_plan_kernel(const __grid_constant__
     p.indptr[U] = (int32_t)tot[3];
     if (p.tier_indptr) p.tier_indptr[3 * U] = (int32_t)tot[3];
     bool bad = tot[3] > p.page_cap || tot[3] > 0x7FFFFFFFLL;
-    for (int t = 0; t < 3; ++t) bad |= tot[t] > p.free_len[t];
+    for (int t = 0; t < 3; ++t) bad |= cur[t] < 0 || cur[t] + tot[t] > p.free_len[t];
     if (bad) report(p.err, SKV_ERR_POOL);
+    if (rt) {
+      for (int t = 0; t < 3; ++t) p.cursor[t] = (int32_t)(cur[t] + tot[t]);
+      *p.n_released = (int32_t)tot[4];
+    }
   }
 }
 
@@ -462,7 +564,16 @@ __global__ void __launch_bounds__(256) page_write_kernel(const __grid_constant__
     if (local < np0) { t = 0; pg = local; n = n0; }
     else if (local < np0 + np1) { t = 1; pg = local - np0; n = n1; }
     else { t = 2; pg = local - np0 - np1; n = n2; }
-    const long long fi = p.tbase[u * 3 + t] + pg;
+    const long long kp = p.keep ? p.keep[u * 3 + t] : 0;
+    if (pg < kp) {  // an unchanged page of a re-tiered store: it stays
+      const long long go = p.tindptr_old[3 * u + t] + pg;
+      if (lane == 0) {
+        if (g < p.page_cap && go >= 0 && go < p.page_cap) p.page_ids[g] = p.ids_old[go];
+        else report(p.err, SKV_ERR_CORRUPT);
+      }
+      continue;
+    }
+    const long long fi = p.tbase[u * 3 + t] + pg - kp;
     if (g >= p.page_cap || fi >= p.free_len[t]) {
       if (lane == 0) report(p.err, SKV_ERR_POOL);
       continue;
@@ -490,6 +601,33 @@ __global__ void __launch_bounds__(256) page_write_kernel(const __grid_constant__
   }
 }
 
+// re-tiering: the ids of the old pages that the new store no longer holds,
+// per unit in (tier, page) order from rbase[u] on
+__global__ void release_kernel(const __grid_constant__ AllocParams p) {
+  const int U = p.B * p.Hkv;
+  const long long n_old = min((long long)p.indptr_old[U], p.page_cap);
+  const long long nthr = (long long)gridDim.x * blockDim.x;
+  for (long long g = (long long)blockIdx.x * blockDim.x + threadIdx.x; g < n_old; g += nthr) {
+    int lo = 0, hi = U - 1;  // the unit u with indptr_old[u] <= g < indptr_old[u + 1]
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (p.indptr_old[mid] <= g) lo = mid; else hi = mid - 1;
+    }
+    const int u = lo;
+    long long idx = p.rbase[u];
+    for (int t = 0; t < 3; ++t) {
+      const long long a = p.tindptr_old[3 * u + t], e = p.tindptr_old[3 * u + t + 1];
+      const long long kp = p.keep[3 * u + t];
+      if (g < e) {
+        const long long r = idx + (g - a - kp);
+        if (g - a >= kp && r >= 0 && r < p.page_cap) p.released[r] = p.ids_old[g];
+        break;
+      }
+      idx += (e - a) - kp;
+    }
+  }
+}
+
 static unsigned grid_for(long long n, int threads) {
   long long b = (n + threads - 1) / threads;
   return (unsigned)(b < 1 ? 1 : b);
@@ -501,7 +639,7 @@ cudaError_t launch_allocate(AllocParams& p, cudaStream_t stream) {
   p.dense = 0;
   p.nseg = p.mode == SKV_MODE_BUDGET ? p.B : U;
   cudaError_t e;
-  if ((e = cudaMemsetAsync(p.nprot, 0, 8 * (size_t)p.B, stream)) != cudaSuccess) return e;
+  if ((e = cudaMemsetAsync(p.pinned, 0, 8 * (size_t)p.B, stream)) != cudaSuccess) return e;
   if ((e = cudaMemsetAsync(p.hist, 0, 8 * (size_t)p.nseg * 3 * 256, stream)) != cudaSuccess)
     return e;
   if (p.outlier && ntok > 0) {
@@ -532,6 +670,77 @@ cudaError_t launch_allocate(AllocParams& p, cudaStream_t stream) {
   row_of_kernel<<<U, 1024, 0, stream>>>(p);
   page_write_kernel<<<grid_for(std::min<long long>(p.page_cap, 1LL << 22) * 32, 256), 256, 0,
                       stream>>>(p);
+  return cudaGetLastError();
+}
+
+size_t retier_workspace_bytes(int B, int Hkv, long long Tmax, long long page_cap) {
+  const size_t U = (size_t)B * Hkv;
+  return alloc_workspace_bytes(B, Hkv, Tmax) + al256(U * (size_t)Tmax) +
+         al256(4 * U * (size_t)Tmax) + al256(4 * (U + 1)) + al256(4 * (3 * U + 1)) +
+         al256(4 * (size_t)page_cap) + 2 * al256(4 * 3 * U) + al256(4 * U);
+}
+
+void retier_carve(AllocParams& p, void* ws) {
+  const size_t U = (size_t)p.B * p.Hkv;
+  alloc_carve(p, ws);
+  uint8_t* w = static_cast<uint8_t*>(ws) + alloc_workspace_bytes(p.B, p.Hkv, p.Tmax);
+  p.tier_old = w;
+  w += al256(U * (size_t)p.Tmax);
+  p.row_old = reinterpret_cast<int32_t*>(w);
+  w += al256(4 * U * (size_t)p.Tmax);
+  p.indptr_old = reinterpret_cast<int32_t*>(w);
+  w += al256(4 * (U + 1));
+  p.tindptr_old = reinterpret_cast<int32_t*>(w);
+  w += al256(4 * (3 * U + 1));
+  p.ids_old = reinterpret_cast<uint32_t*>(w);
+  w += al256(4 * (size_t)p.page_cap);
+  p.diff = reinterpret_cast<int32_t*>(w);
+  w += al256(4 * 3 * U);
+  p.keep = reinterpret_cast<int32_t*>(w);
+  w += al256(4 * 3 * U);
+  p.rbase = reinterpret_cast<int32_t*>(w);
+}
+
+cudaError_t launch_retier_plan(AllocParams& p, cudaStream_t stream) {
+  const long long ntok = (long long)p.B * p.Hkv * p.Tmax;
+  const int U = p.B * p.Hkv;
+  p.dense = 0;
+  p.mode = SKV_MODE_BUDGET;
+  p.nseg = p.B;
+  cudaError_t e;
+  // the store as it is: every later step reads the old layout from here
+  const size_t tok = (size_t)ntok;
+  if ((e = cudaMemcpyAsync(p.tier_old, p.tier_out, tok, cudaMemcpyDeviceToDevice, stream)) ||
+      (e = cudaMemcpyAsync(p.row_old, p.row_of, 4 * tok, cudaMemcpyDeviceToDevice, stream)) ||
+      (e = cudaMemcpyAsync(p.indptr_old, p.indptr, 4 * ((size_t)U + 1), cudaMemcpyDeviceToDevice,
+                           stream)) ||
+      (e = cudaMemcpyAsync(p.tindptr_old, p.tier_indptr, 4 * (3 * (size_t)U + 1),
+                           cudaMemcpyDeviceToDevice, stream)) ||
+      (e = cudaMemcpyAsync(p.ids_old, p.page_ids, 4 * (size_t)p.page_cap,
+                           cudaMemcpyDeviceToDevice, stream)))
+    return e;
+  if ((e = cudaMemsetAsync(p.pinned, 0, 8 * (size_t)p.B, stream)) != cudaSuccess) return e;
+  if ((e = cudaMemsetAsync(p.hist, 0, 8 * (size_t)p.nseg * 3 * 256, stream)) != cudaSuccess)
+    return e;
+  if ((e = cudaMemsetAsync(p.diff, 0x7F, 4 * 3 * (size_t)U, stream)) != cudaSuccess) return e;
+  if (ntok > 0) keys_retier_kernel<<<grid_for(ntok * 32, 256), 256, 0, stream>>>(p);
+  sel_init_kernel<<<grid_for(p.nseg * 3, 128), 128, 0, stream>>>(p);
+  const dim3 hgrid(grid_for((long long)p.Hkv * p.Tmax * 3, kHistItemsPerBlock), p.nseg);
+  for (int pass = 0; pass < 8; ++pass) {
+    const int shift = 56 - 8 * pass;
+    hist_kernel<<<hgrid, 256, 0, stream>>>(p, shift);
+    sel_step_kernel<<<grid_for(p.nseg * 3, 128), 128, 0, stream>>>(p, shift);
+  }
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (ntok > 0) tier_kernel<<<grid_for(ntok, 256), 256, 0, stream>>>(p);
+  unit_count_kernel<<<U, 256, 0, stream>>>(p);
+  row_of_kernel<<<U, 1024, 0, stream>>>(p);
+  if (ntok > 0) diff_kernel<<<grid_for(ntok, 256), 256, 0, stream>>>(p);
+  page_plan_kernel<<<1, 1024, 0, stream>>>(p);
+  page_write_kernel<<<grid_for(std::min<long long>(p.page_cap, 1LL << 22) * 32, 256), 256, 0,
+                      stream>>>(p);
+  release_kernel<<<grid_for(std::min<long long>(p.page_cap, 1LL << 20), 256), 256, 0, stream>>>(
+      p);
   return cudaGetLastError();
 }
 

@@ -448,6 +448,105 @@ int skv_append(skv_ctx* ctx, const uint16_t* K_new, const uint16_t* V_new, int B
   return ok();
 }
 
+int skv_retier_workspace_size(const skv_ctx* ctx, int B, int Hkv, int64_t Tmax,
+                              int64_t page_cap, size_t* bytes) {
+  if (!ctx || !bytes) return fail(SKV_ERR_ARG, "skv_retier_workspace_size: null argument");
+  if (B < 0 || Hkv <= 0 || Tmax < 0 || page_cap < 0)
+    return fail(SKV_ERR_ARG, "skv_retier_workspace_size: bad sizes");
+  *bytes = skv::retier_workspace_bytes(B, Hkv, Tmax, page_cap);
+  return ok();
+}
+
+int skv_retier(skv_ctx* ctx, int B, int Hkv, int64_t Tmax, const int32_t* seq_lens,
+               const float* utility, const uint8_t* demote, const int64_t* budget,
+               const skv_free_lists* free, int32_t* free_cursor, const skv_pools* pools,
+               uint8_t* tier, int32_t* row_of, int32_t* page_indptr,
+               int32_t* page_tier_indptr, uint32_t* page_ids, int64_t page_cap,
+               uint32_t* released, int32_t* n_released, int32_t* err_word, void* workspace,
+               size_t ws_bytes, void* stream) {
+  if (!ctx) return fail(SKV_ERR_ARG, "skv_retier: null ctx");
+  if (B < 0 || Hkv <= 0 || Hkv > 128 || Tmax < 0 || Tmax > (1LL << 23) || page_cap < 0 ||
+      page_cap > 0x7FFFFFFFLL)
+    return fail(SKV_ERR_ARG, "skv_retier: need B >= 0, 0 < Hkv <= 128, 0 <= Tmax <= 2^23");
+  if ((long long)B * Hkv > (1 << 24)) return fail(SKV_ERR_ARG, "skv_retier: too many units");
+  if (!seq_lens || !utility || !demote || !budget || !free || !free_cursor || !tier ||
+      !row_of || !page_indptr || !page_tier_indptr || !released || !n_released || !err_word)
+    return fail(SKV_ERR_ARG, "skv_retier: null argument");
+  if (page_cap > 0 && !page_ids) return fail(SKV_ERR_ARG, "skv_retier: null page_ids");
+  if (!valid_pools(pools, 3))
+    return fail(SKV_ERR_ARG, "skv_retier: pools need 128-byte aligned bases");
+  for (int t = 0; t < 3; ++t)
+    if (free->len[t] < 0 || (free->len[t] > 0 && !free->ids[t]))
+      return fail(SKV_ERR_ARG, "skv_retier: bad free list %d", t);
+  const size_t need = skv::retier_workspace_bytes(B, Hkv, Tmax, page_cap);
+  if (!workspace || ws_bytes < need)
+    return fail(SKV_ERR_ARG, "skv_retier: workspace of %zu bytes needed", need);
+  skv::AllocParams p;
+  fill_alloc_common(p, ctx, B, Hkv, Tmax);
+  p.seq_lens = seq_lens;
+  p.utility = utility;
+  p.demote = demote;
+  p.mode = SKV_MODE_BUDGET;
+  p.budget = budget;
+  for (int t = 0; t < 3; ++t) {
+    p.free_ids[t] = free->ids[t];
+    p.free_len[t] = free->len[t];
+    p.pool[t] = static_cast<uint8_t*>(pools->base[t]);
+    p.slots[t] = pools->slots[t];
+    p.stride[t] = ctx->stride[t];
+    p.payload[t] = (int)ctx->payload[t];
+  }
+  p.tier_out = tier;
+  p.row_of = row_of;
+  p.indptr = page_indptr;
+  p.tier_indptr = page_tier_indptr;
+  p.page_ids = page_ids;
+  p.page_cap = page_cap;
+  p.cursor = free_cursor;
+  p.released = released;
+  p.n_released = n_released;
+  p.err = err_word;
+  skv::retier_carve(p, workspace);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = skv::launch_retier_plan(p, st);
+  if (e != cudaSuccess) return cuda_fail(e, "skv_retier plan");
+  skv::TranscodeParams tp;
+  std::memset(&tp, 0, sizeof(tp));
+  tp.B = B;
+  tp.Hkv = Hkv;
+  tp.Tmax = Tmax;
+  tp.P = ctx->P;
+  tp.seq_lens = seq_lens;
+  tp.tier = tier;
+  tp.row_of = row_of;
+  tp.indptr = page_indptr;
+  tp.tier_indptr = page_tier_indptr;
+  tp.ids = page_ids;
+  tp.keep = p.keep;
+  tp.page_cap = page_cap;
+  tp.tier_old = p.tier_old;
+  tp.row_old = p.row_old;
+  tp.indptr_old = p.indptr_old;
+  tp.ids_old = p.ids_old;
+  for (int t = 0; t < 3; ++t) {
+    tp.pool[t] = p.pool[t];
+    tp.slots[t] = p.slots[t];
+    tp.stride[t] = p.stride[t];
+  }
+  tp.err = err_word;
+  std::memcpy(tp.bx6, ctx->bx6, sizeof(tp.bx6));
+  std::memcpy(tp.by6, ctx->by6, sizeof(tp.by6));
+  std::memcpy(tp.bx4, ctx->bx4, sizeof(tp.bx4));
+  std::memcpy(tp.by4, ctx->by4, sizeof(tp.by4));
+  std::memcpy(tp.bx5, ctx->bx5, sizeof(tp.bx5));
+  std::memcpy(tp.by5, ctx->by5, sizeof(tp.by5));
+  tp.t1_scheme = ctx->t1_scheme;
+  tp.share_grid = ctx->share_grid;
+  e = skv::launch_transcode(tp, st);
+  if (e != cudaSuccess) return cuda_fail(e, "skv_retier transcode");
+  return ok();
+}
+
 static int decode_common(skv_ctx* ctx, const void* q, int q_dtype, int B, int Hq, int Hkv,
                          const int32_t* page_indptr, const int32_t* page_tier_indptr,
                          const uint32_t* page_ids, const void* pool[3],

@@ -98,70 +98,39 @@ __device__ __forceinline__ int v_frag_offset(int row, int dd, int elem_bytes) {
   return k * 2048 + 512 * (mt >> 1) + 16 * L + 8 * (mt & 1) + 2 * e;
 }
 
-__global__ void __launch_bounds__(256) encode_kernel(const __grid_constant__ EncodeParams p) {
-  __shared__ float sbx6[64], sby6[64], sbx4[16], sby4[16], sbx5[32], sby5[32];
+// The boundary vectors of the three angle codes, in shared memory.
+struct Boundaries {
+  float bx6[64], by6[64], bx4[16], by4[16], bx5[32], by5[32];
+};
+
+template <class Prm>
+__device__ __forceinline__ void load_boundaries(const Prm& p, Boundaries& sb) {
   for (int i = threadIdx.x; i < 64; i += blockDim.x) {
-    sbx6[i] = p.bx6[i];
-    sby6[i] = p.by6[i];
+    sb.bx6[i] = p.bx6[i];
+    sb.by6[i] = p.by6[i];
     if (i < 32) {
-      sbx5[i] = p.bx5[i];
-      sby5[i] = p.by5[i];
+      sb.bx5[i] = p.bx5[i];
+      sb.by5[i] = p.by5[i];
     }
     if (i < 16) {
-      sbx4[i] = p.bx4[i];
-      sby4[i] = p.by4[i];
+      sb.bx4[i] = p.bx4[i];
+      sb.by4[i] = p.by4[i];
     }
   }
-  __syncthreads();
-  const long long w = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  const long long total = (long long)p.B * p.Hkv * p.Tmax;
-  if (w >= total) return;
-  const long long t = w % p.Tmax;
-  const long long bh = w / p.Tmax;
-  const int h = (int)(bh % p.Hkv), b = (int)(bh / p.Hkv);
-  if (t >= p.seq_lens[b]) return;
-  const int P = p.P;
-  int tr, pi, row;
-  if (p.dense_bf16) {
-    tr = 0;
-    pi = (int)(t / P);
-    row = (int)(t % P);
-  } else {
-    tr = p.tier[w];
-    if (tr == SKV_TIER_DROP) return;
-    const int loc = p.row_of[w];
-    if (tr > SKV_TIER_DROP || loc < 0) {
-      if (lane == 0) report(p.err, SKV_ERR_CORRUPT);
-      return;
-    }
-    pi = loc / P;
-    row = loc % P;
-  }
-  const long long gi = (long long)p.indptr[bh] + pi;
-  if (gi >= p.indptr[bh + 1]) {
-    if (lane == 0) report(p.err, SKV_ERR_CORRUPT);
-    return;
-  }
-  const uint32_t id = p.ids[gi];
-  const uint32_t slot = id & 0x3FFFFFFFu;
-  if ((int)(id >> 30) != tr || (long long)slot >= p.slots[tr]) {
-    if (lane == 0) report(p.err, SKV_ERR_CORRUPT);
-    return;
-  }
-  uint8_t* page = p.pool[tr] + (long long)slot * p.stride[tr];
-  const uint2 kv = *reinterpret_cast<const uint2*>(p.K + w * kHeadDim + 4 * lane);
-  const uint2 vv = *reinterpret_cast<const uint2*>(p.V + w * kHeadDim + 4 * lane);
-  const uint16_t k4[4] = {(uint16_t)(kv.x & 0xFFFF), (uint16_t)(kv.x >> 16),
-                          (uint16_t)(kv.y & 0xFFFF), (uint16_t)(kv.y >> 16)};
-  const uint16_t v4[4] = {(uint16_t)(vv.x & 0xFFFF), (uint16_t)(vv.x >> 16),
-                          (uint16_t)(vv.y & 0xFFFF), (uint16_t)(vv.y >> 16)};
+}
 
+// Write one token's row `row` into `page` (tier tr, P rows): the warp's lane
+// l holds the fp16 key and value components 4l..4l+3 in k4 / v4.  T0 keeps
+// them (as bf16 for the dense baseline), T1 / T2 encode them.
+__device__ __forceinline__ void write_row(uint8_t* page, int P, int tr, int row, int lane,
+                                          const uint16_t (&k4)[4], const uint16_t (&v4)[4],
+                                          bool dense_bf16, int t1_scheme, int share_grid,
+                                          const Boundaries& sb) {
   if (tr == SKV_TIER_T0) {
     uint16_t ko[4], vo[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      if (p.dense_bf16) {
+      if (dense_bf16) {
         ko[i] = __bfloat16_as_ushort(__float2bfloat16_rn(__half2float(__ushort_as_half(k4[i]))));
         vo[i] = __bfloat16_as_ushort(__float2bfloat16_rn(__half2float(__ushort_as_half(v4[i]))));
       } else {
@@ -199,16 +168,15 @@ __global__ void __launch_bounds__(256) encode_kernel(const __grid_constant__ Enc
 
   // ---- codes of pairs 2 lane, 2 lane + 1
   const bool t1 = tr == SKV_TIER_T1;
-  const bool v53 = t1 && p.t1_scheme;  // T1 variant: 5-bit angle + 3-bit share
+  const bool v53 = t1 && t1_scheme;  // T1 variant: 5-bit angle + 3-bit share
   const int bits = t1 ? (v53 ? 5 : 6) : 4;
-  const float* bx = t1 ? (v53 ? sbx5 : sbx6) : sbx4;
-  const float* by = t1 ? (v53 ? sby5 : sby6) : sby4;
+  const float* bx = t1 ? (v53 ? sb.bx5 : sb.bx6) : sb.bx4;
+  const float* by = t1 ? (v53 ? sb.by5 : sb.by6) : sb.by4;
   const uint32_t th0 = angle_code(k4[0], k4[1], bits, bx, by);
   const uint32_t th1 = angle_code(k4[2], k4[3], bits, bx, by);
-  const uint32_t rh0 = v53 ? rho_code3(m[0], m[1], R2) : rho_code(m[0], m[1], R2, p.share_grid);
-  const uint32_t rh1 = v53 ? rho_code3(m[2], m[3], R2) : rho_code(m[2], m[3], R2, p.share_grid);
+  const uint32_t rh0 = v53 ? rho_code3(m[0], m[1], R2) : rho_code(m[0], m[1], R2, share_grid);
+  const uint32_t rh1 = v53 ? rho_code3(m[2], m[3], R2) : rho_code(m[2], m[3], R2, share_grid);
   const uint32_t packed = th0 | (th1 << 8) | (rh0 << 16) | (rh1 << 24);
-
   // ---- V quantiser
   float vf[4], amax = 0.0f;
 #pragma unroll
@@ -280,6 +248,133 @@ __global__ void __launch_bounds__(256) encode_kernel(const __grid_constant__ Enc
   }
 #pragma unroll
   for (int i = 0; i < 4; ++i) vsec[v_frag_offset(row, 4 * lane + i, 1)] = (uint8_t)v8[i];
+}
+
+
+__global__ void __launch_bounds__(256) encode_kernel(const __grid_constant__ EncodeParams p) {
+  __shared__ Boundaries sb;
+  load_boundaries(p, sb);
+  __syncthreads();
+  const long long w = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const long long total = (long long)p.B * p.Hkv * p.Tmax;
+  if (w >= total) return;
+  const long long t = w % p.Tmax;
+  const long long bh = w / p.Tmax;
+  const int b = (int)(bh / p.Hkv);
+  if (t >= p.seq_lens[b]) return;
+  const int P = p.P;
+  int tr, pi, row;
+  if (p.dense_bf16) {
+    tr = 0;
+    pi = (int)(t / P);
+    row = (int)(t % P);
+  } else {
+    tr = p.tier[w];
+    if (tr == SKV_TIER_DROP) return;
+    const int loc = p.row_of[w];
+    if (tr > SKV_TIER_DROP || loc < 0) {
+      if (lane == 0) report(p.err, SKV_ERR_CORRUPT);
+      return;
+    }
+    pi = loc / P;
+    row = loc % P;
+  }
+  const long long gi = (long long)p.indptr[bh] + pi;
+  if (gi >= p.indptr[bh + 1]) {
+    if (lane == 0) report(p.err, SKV_ERR_CORRUPT);
+    return;
+  }
+  const uint32_t id = p.ids[gi];
+  const uint32_t slot = id & 0x3FFFFFFFu;
+  if ((int)(id >> 30) != tr || (long long)slot >= p.slots[tr]) {
+    if (lane == 0) report(p.err, SKV_ERR_CORRUPT);
+    return;
+  }
+  uint8_t* page = p.pool[tr] + (long long)slot * p.stride[tr];
+  const uint2 kv = *reinterpret_cast<const uint2*>(p.K + w * kHeadDim + 4 * lane);
+  const uint2 vv = *reinterpret_cast<const uint2*>(p.V + w * kHeadDim + 4 * lane);
+  const uint16_t k4[4] = {(uint16_t)(kv.x & 0xFFFF), (uint16_t)(kv.x >> 16),
+                          (uint16_t)(kv.y & 0xFFFF), (uint16_t)(kv.y >> 16)};
+  const uint16_t v4[4] = {(uint16_t)(vv.x & 0xFFFF), (uint16_t)(vv.x >> 16),
+                          (uint16_t)(vv.y & 0xFFFF), (uint16_t)(vv.y >> 16)};
+  write_row(page, P, tr, row, lane, k4, v4, p.dense_bf16 != 0, p.t1_scheme, p.share_grid, sb);
+}
+
+// ---------------------------------------------------------------- transcode
+// Re-tiering's data step, one warp per resident token of a rewritten page
+// (a page at or after its segment's first change).  Its old row is either
+// T0 -- the exact fp16 K and V, read back from the old page in the T0 row
+// order and written (T0) or encoded (T1 / T2) as the encode does from dense
+// inputs -- or T1 / T2 of the same tier, whose radius, code row, scale and
+// int8 V are copied (the V fragment order depends on the row index).
+
+// the page of row `loc` of unit u in a page table, or null when it is not
+// a page of tier tr in range
+__device__ __forceinline__ uint8_t* row_page(const TranscodeParams& p, const int32_t* indptr,
+                                             const uint32_t* ids, long long u, int tr, int loc) {
+  if (loc < 0) return nullptr;
+  const long long gi = (long long)indptr[u] + loc / p.P;
+  if (gi >= indptr[u + 1] || gi < 0 || gi >= p.page_cap) return nullptr;
+  const uint32_t id = ids[gi], slot = id & 0x3FFFFFFFu;
+  if ((int)(id >> 30) != tr || (long long)slot >= p.slots[tr]) return nullptr;
+  return p.pool[tr] + (long long)slot * p.stride[tr];
+}
+
+__global__ void __launch_bounds__(256) transcode_kernel(const __grid_constant__ TranscodeParams p) {
+  __shared__ Boundaries sb;
+  load_boundaries(p, sb);
+  __syncthreads();
+  const long long w = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (w >= (long long)p.B * p.Hkv * p.Tmax) return;
+  const long long t = w % p.Tmax, u = w / p.Tmax;
+  if (t >= p.seq_lens[u / p.Hkv]) return;
+  const int tn = p.tier[w];
+  if (tn >= SKV_TIER_DROP) return;
+  const int rn = p.row_of[w], P = p.P;
+  // rows of a kept page (before its segment's first change) are in place
+  if (rn >= 0 && rn / P - (p.tier_indptr[3 * u + tn] - p.indptr[u]) < p.keep[3 * u + tn]) return;
+  const int to = p.tier_old[w], ro = to < SKV_TIER_DROP ? p.row_old[w] : -1;
+  uint8_t* dst = row_page(p, p.indptr, p.ids, u, tn, rn);
+  const uint8_t* src = to < SKV_TIER_DROP ? row_page(p, p.indptr_old, p.ids_old, u, to, ro)
+                                          : nullptr;
+  if (!dst || !src || (to != SKV_TIER_T0 && to != tn)) {
+    if (lane == 0) report(p.err, SKV_ERR_CORRUPT);
+    return;
+  }
+  const int r_new = rn % P, r_old = ro % P;
+  if (to == SKV_TIER_T0) {
+    const int c = lane >> 1;
+    const uint2 kv = *reinterpret_cast<const uint2*>(src + kHdrBytes + r_old * 256 +
+                                                     (c ^ (4 * (r_old & 1))) * 16 + (lane & 1) * 8);
+    const uint8_t* vsec = src + kHdrBytes + 256 * P;
+    uint16_t k4[4] = {(uint16_t)(kv.x & 0xFFFF), (uint16_t)(kv.x >> 16),
+                      (uint16_t)(kv.y & 0xFFFF), (uint16_t)(kv.y >> 16)};
+    uint16_t v4[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      v4[i] = *reinterpret_cast<const uint16_t*>(vsec + v_frag_offset(r_old, 4 * lane + i, 2));
+    write_row(dst, P, tn, r_new, lane, k4, v4, false, p.t1_scheme, p.share_grid, sb);
+    return;
+  }
+  // T1 / T2 row: r~ (fp16 [P]), codes ([P][cb]), scale (fp16 [P]), int8 V
+  const int cb = tn == SKV_TIER_T1 ? 64 : 48;
+  const uint8_t* rs = src + kHdrBytes;
+  uint8_t* rd = dst + kHdrBytes;
+  if (lane == 0) {
+    *reinterpret_cast<uint16_t*>(rd + 2 * r_new) = *reinterpret_cast<const uint16_t*>(rs + 2 * r_old);
+    *reinterpret_cast<uint16_t*>(rd + (2 + cb) * P + 2 * r_new) =
+        *reinterpret_cast<const uint16_t*>(rs + (2 + cb) * P + 2 * r_old);
+  }
+  if (lane < cb / 4)
+    *reinterpret_cast<uint32_t*>(rd + 2 * P + cb * r_new + 4 * lane) =
+        *reinterpret_cast<const uint32_t*>(rs + 2 * P + cb * r_old + 4 * lane);
+  const uint8_t* vs = rs + (4 + cb) * P;
+  uint8_t* vd = rd + (4 + cb) * P;
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    vd[v_frag_offset(r_new, 4 * lane + i, 1)] = vs[v_frag_offset(r_old, 4 * lane + i, 1)];
 }
 
 // ------------------------------------------------------------------ append
@@ -503,6 +598,13 @@ cudaError_t launch_append(const AppendParams& p, cudaStream_t stream) {
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   append_write_kernel<<<(unsigned)((U + 7) / 8), 256, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_transcode(const TranscodeParams& p, cudaStream_t stream) {
+  const long long warps = (long long)p.B * p.Hkv * p.Tmax;
+  if (warps == 0) return cudaSuccess;
+  transcode_kernel<<<(unsigned)((warps * 32 + 255) / 256), 256, 0, stream>>>(p);
   return cudaGetLastError();
 }
 

@@ -139,11 +139,25 @@ struct AllocParams {
   unsigned long long* hist;   // [nseg*3*256]
   int32_t* counts;            // [U*3]
   int32_t* tbase;             // [U*3]
-  long long* nprot;           // [B]
+  long long* pinned;          // [B]: bytes of the tokens whose tier is fixed
   int nseg;
   int dense;                  // dense-bf16 baseline packing (every token kept, tier 0)
   int outlier;                // outlier-aware protection on
   uint8_t* eff_protect;       // [B*Hkv*Tmax]: protect | outlier flag (workspace)
+  // re-tiering (launch_retier_plan): the store as it was before the call,
+  // snapshotted into the workspace, and the page bookkeeping of the update
+  const uint8_t* demote;      // [B*Hkv*Tmax]: T0 rows to re-decide
+  uint8_t* tier_old;          // [B*Hkv*Tmax]
+  int32_t* row_old;           // [B*Hkv*Tmax]
+  int32_t* indptr_old;        // [U + 1]
+  int32_t* tindptr_old;       // [3U + 1]
+  uint32_t* ids_old;          // [page_cap]
+  int32_t* diff;              // [3U]: first row of each (unit, tier) segment that changes
+  int32_t* keep;              // [3U]: leading pages of each segment kept in place
+  int32_t* rbase;             // [U]: first released-list index of each unit
+  int32_t* cursor;            // [3]: free-list cursors, advanced by the pages taken
+  uint32_t* released;         // [page_cap]: ids of the old pages no longer referenced
+  int32_t* n_released;        // [1]
 };
 
 // Decode workspace: partials [(S + U) G][kPartStride] fp32, then per unit the
@@ -196,6 +210,41 @@ cudaError_t launch_append(const AppendParams& p, cudaStream_t stream);
 size_t alloc_workspace_bytes(int B, int Hkv, long long Tmax);
 void alloc_carve(AllocParams& p, void* ws);
 cudaError_t launch_allocate(AllocParams& p, cudaStream_t stream);
+size_t retier_workspace_bytes(int B, int Hkv, long long Tmax, long long page_cap);
+void retier_carve(AllocParams& p, void* ws);
+// The allocation half of a re-tiering: tiers, row map, page table, headers
+// of the rewritten pages and the released list (p.tier_out etc. are the
+// store's own arrays; their old contents are snapshotted first).
+cudaError_t launch_retier_plan(AllocParams& p, cudaStream_t stream);
+
+// The data half: every row of a rewritten page, copied from its old row or,
+// for a T0 row that becomes T1/T2, encoded from the fp16 K/V in its old page.
+struct TranscodeParams {
+  int B, Hkv;
+  long long Tmax;
+  int P;
+  const int32_t* seq_lens;
+  const uint8_t* tier;        // the new store
+  const int32_t* row_of;
+  const int32_t* indptr;
+  const int32_t* tier_indptr;
+  const uint32_t* ids;
+  const int32_t* keep;        // [3U]
+  long long page_cap;         // capacity of both page-id arrays
+  const uint8_t* tier_old;    // the old store
+  const int32_t* row_old;
+  const int32_t* indptr_old;
+  const uint32_t* ids_old;
+  uint8_t* pool[3];
+  long long slots[3];
+  long long stride[3];
+  int32_t* err;
+  float bx6[64], by6[64], bx4[16], by4[16];
+  float bx5[32], by5[32];
+  int t1_scheme;
+  int share_grid;
+};
+cudaError_t launch_transcode(const TranscodeParams& p, cudaStream_t stream);
 cudaError_t launch_dense_plan(AllocParams& p, cudaStream_t stream);
 
 }  // namespace skv

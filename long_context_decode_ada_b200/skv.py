@@ -32,6 +32,7 @@ TABLE_BOUNDARY6_X, TABLE_BOUNDARY6_Y, TABLE_BOUNDARY4_X, TABLE_BOUNDARY4_Y, TABL
 EXPORTS = [
     "skv_create", "skv_destroy", "skv_last_error", "skv_page_bytes", "skv_tables",
     "skv_device_info", "skv_workspace_size", "skv_allocate", "skv_encode", "skv_append",
+    "skv_retier", "skv_retier_workspace_size",
     "skv_decode_attention", "skv_decode_attention_static", "skv_decode_attention_host",
     "skv_decode_utility", "skv_merge_partials",
     "skv_dense_pack_bf16",
@@ -70,6 +71,9 @@ _SIGS = {
                         _p]),
     "skv_append": (_i, [_p, _p, _p, _i, _i, _i64, _p, _p, _p, _p, _p, _p, _i64, C.POINTER(SkvPools),
                         _p, _i64, _p, _p, _p, _sz, _p]),
+    "skv_retier_workspace_size": (_i, [_p, _i, _i, _i64, _i64, C.POINTER(_sz)]),
+    "skv_retier": (_i, [_p, _i, _i, _i64, _p, _p, _p, _p, C.POINTER(SkvFreeLists), _p,
+                        C.POINTER(SkvPools), _p, _p, _p, _p, _p, _i64, _p, _p, _p, _p, _sz, _p]),
     "skv_decode_attention_host": (_i, [_p, _p, _i, _i, _i, _i, _p, _p, _p, C.POINTER(SkvPools),
                                        _p, _p, _p, _p, _p, _p, _p, _sz, _i, _p]),
     "skv_merge_partials": (_i, [_p, _i, _i64, _p, _p, _i64, _p, _p, _p]),
@@ -287,7 +291,7 @@ class PagedCache:
                  stream=None):
         _check_ingest(self.B, self.Hkv, self.Tmax, self.ctx.d, K=K, seq_lens=seq_lens,
                       utility=utility, protect=protect, budget=budget, quota=quota)
-        self._free0_cursor = None  # append() restarts after the slots this call takes
+        self._cursor = None  # append() / retier() restart after the slots this call takes
         fl = SkvFreeLists()
         self._free = [f.to(self.device, dtype=torch.int32) if isinstance(f, torch.Tensor) else
                       torch.from_numpy(np.asarray(f, np.uint32).view(np.int32)).to(self.device)
@@ -295,6 +299,7 @@ class PagedCache:
         for t in range(3):
             fl.ids[t] = self._free[t].data_ptr() if self._free[t].numel() else None
             fl.len[t] = self._free[t].numel()
+        self._free_c = fl
         _check(lib().skv_allocate(
             self.ctx.handle, _ptr(K), self.B, self.Hkv, self.Tmax, _ptr(seq_lens), _ptr(utility),
             _ptr(protect), mode, _ptr(budget), _ptr(quota), C.byref(fl), C.byref(self._pools_c),
@@ -311,11 +316,8 @@ class PagedCache:
         _expect(K_new, "K_new", self.B * self.Hkv * self.ctx.d, 2)
         _expect(V_new, "V_new", self.B * self.Hkv * self.ctx.d, 2)
         _expect(seq_lens, "seq_lens", self.B, 4, torch.int32)
-        if getattr(self, "_free0_cursor", None) is None:
-            tip = self.page_tier_indptr
-            U = self.B * self.Hkv
-            n0 = (tip[1:3 * U:3] - tip[0:3 * U:3]).sum().to(torch.int32).reshape(1)
-            self._free0_cursor = n0.clone()
+        cursor = self.free_cursor()
+        if getattr(self, "_ws_append", None) is None:
             n = self.ctx.workspace_size(WS_APPEND, self.B, self.Hkv, 0, self.page_cap)
             self._ws_append = torch.empty(max(n, 1), dtype=torch.uint8, device=self.device)
         free0 = self._free[0]
@@ -323,8 +325,47 @@ class PagedCache:
             self.ctx.handle, _ptr(K_new), _ptr(V_new), self.B, self.Hkv, self.Tmax, _ptr(seq_lens),
             _ptr(self.tier), _ptr(self.row_of), _ptr(self.page_indptr), _ptr(self.page_tier_indptr),
             _ptr(self.page_ids), self.page_cap, C.byref(self._pools_c),
-            _ptr(free0) if free0.numel() else None, free0.numel(), _ptr(self._free0_cursor),
+            _ptr(free0) if free0.numel() else None, free0.numel(), _ptr(cursor),
             _ptr(self.err), _ptr(self._ws_append), self._ws_append.numel(), _stream(stream)))
+
+    def free_cursor(self) -> torch.Tensor:
+        """int32 [3] device: the first unused entry of each tier's free list
+        (after the pages allocate() took; advanced by append and retier)."""
+        if getattr(self, "_cursor", None) is None:
+            tip = self.page_tier_indptr
+            U = self.B * self.Hkv
+            self._cursor = torch.stack(
+                [(tip[t + 1:3 * U + 1:3] - tip[t:3 * U:3]).sum() for t in range(3)]
+            ).to(torch.int32)
+        return self._cursor
+
+    def retier(self, utility, demote, budget, seq_lens, stream=None):
+        """Re-decide the demoted T0 rows under the budget on the store itself
+        (skv_retier).  utility fp32 and demote uint8 [B][Hkv][Tmax], budget
+        int64 [B], all on the device.  New pages take slots from the free
+        lists given to allocate(); returns (released, n_released): the ids
+        of the old pages no longer referenced (device int32 [page_cap], the
+        first n_released valid) -- valid until the next retier call."""
+        _check_ingest(self.B, self.Hkv, self.Tmax, self.ctx.d, seq_lens=seq_lens,
+                      utility=utility, budget=budget)
+        _expect(demote, "demote", self.B * self.Hkv * self.Tmax, 1)
+        cursor = self.free_cursor()
+        if getattr(self, "_ws_retier", None) is None:
+            n = C.c_size_t()
+            _check(lib().skv_retier_workspace_size(self.ctx.handle, self.B, self.Hkv, self.Tmax,
+                                                   self.page_cap, C.byref(n)))
+            self._ws_retier = torch.empty(max(n.value, 1), dtype=torch.uint8, device=self.device)
+            self.released = torch.zeros(max(1, self.page_cap), dtype=torch.int32,
+                                         device=self.device)
+            self.n_released = torch.zeros(1, dtype=torch.int32, device=self.device)
+        _check(lib().skv_retier(
+            self.ctx.handle, self.B, self.Hkv, self.Tmax, _ptr(seq_lens), _ptr(utility),
+            _ptr(demote), _ptr(budget), C.byref(self._free_c), _ptr(cursor),
+            C.byref(self._pools_c), _ptr(self.tier), _ptr(self.row_of), _ptr(self.page_indptr),
+            _ptr(self.page_tier_indptr), _ptr(self.page_ids), self.page_cap, _ptr(self.released),
+            _ptr(self.n_released), _ptr(self.err), _ptr(self._ws_retier), self._ws_retier.numel(),
+            _stream(stream)))
+        return self.released, self.n_released
 
     def encode(self, K, V, seq_lens, stream=None):
         _check_ingest(self.B, self.Hkv, self.Tmax, self.ctx.d, K=K, V=V, seq_lens=seq_lens)
