@@ -685,14 +685,28 @@ def run_configs(ctx, dev, peak, S_default):
     return res
 
 
+def _decode_blocks(text: str) -> str:
+    """The decode kernel's part of kernels.h: its parameter block and the
+    layout of its workspace (the other kernels' blocks do not change it)."""
+    out = []
+    for head, tail in (("struct DecodeParams {", "\n};"), ("struct DecodeWs {", "return w;\n}")):
+        a = text.index(head)
+        out.append(text[a:text.index(tail, a) + len(tail)])
+    return "\n".join(out)
+
+
 def decode_source_digest() -> str:
     """sha256 of the decode kernel's sources (decides whether a profiled
-    DRAM traffic figure still describes the kernel that runs)."""
+    DRAM traffic figure still describes the kernel that runs): decode.cu,
+    common.cuh and the decode blocks of kernels.h."""
     import hashlib
     h = hashlib.sha256()
-    for f in ("decode.cu", "common.cuh", "kernels.h"):
-        with open(os.path.join(ROOT, "long_context_decode_ada_b200", "csrc", f), "rb") as fh:
+    csrc = os.path.join(ROOT, "long_context_decode_ada_b200", "csrc")
+    for f in ("decode.cu", "common.cuh"):
+        with open(os.path.join(csrc, f), "rb") as fh:
             h.update(fh.read())
+    with open(os.path.join(csrc, "kernels.h")) as fh:
+        h.update(_decode_blocks(fh.read()).encode())
     return h.hexdigest()
 
 
