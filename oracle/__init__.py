@@ -86,6 +86,9 @@ _SIGS = {
     "orc_d2h": (_u16, [_d]),
     "orc_h2d": (_d, [_u16]),
     "orc_bf2d": (_d, [_u16]),
+    "orc_h2bf": (_u16, [_u16]),
+    "orc_set_t0_bf16": (None, [_i]),
+    "orc_t0_bf16": (_i, []),
     "orc_threads": (_i, []),
 }
 
@@ -372,6 +375,24 @@ class t1_scheme:
 
     def __exit__(self, *exc):
         lib().orc_set_t1_scheme(self.prev)
+        return False
+
+
+class t0_bf16:
+    """Context manager: the oracle's T0 storage format inside the block
+    (False: fp16 K and V as given; True: rounded to bf16, the fused T0 /
+    bf16 decode path's pages)."""
+
+    def __init__(self, on: bool = True):
+        self.on = on
+
+    def __enter__(self):
+        self.prev = lib().orc_t0_bf16()
+        lib().orc_set_t0_bf16(1 if self.on else 0)
+        return self
+
+    def __exit__(self, *exc):
+        lib().orc_set_t0_bf16(self.prev)
         return False
 
 

@@ -88,6 +88,36 @@ static double bf2d(uint16_t h) {
     return (double)f;
 }
 
+/* fp16 bit pattern -> the bf16 bit pattern of its value rounded to 8
+   significant bits, ties to even.  Every finite fp16 value lies inside the
+   normal range of bf16 (2^-126 .. 2^128), so only the significand rounds:
+   x = m 2^e with m in [2^7, 2^8) after scaling, m rounded to an integer by
+   nearbyint (the default rounding mode is to nearest, ties to even), then
+   the fields of the result are formed from the rounded m and e. */
+static uint16_t h2bf(uint16_t h) {
+    double x = h2d(h);
+    uint16_t sign = (h & 0x8000) ? 0x8000 : 0;
+    if (x < 0) x = -x;
+    if (x == 0) return sign;
+    int ex;
+    frexp(x, &ex);                         /* x in [2^(ex-1), 2^ex) */
+    double m = nearbyint(ldexp(x, 8 - ex)); /* in [2^7, 2^8] */
+    if (m == 256.0) { m = 128.0; ex += 1; }
+    int E = ex - 1 + 127;                  /* biased exponent of 2^(ex-1) */
+    return sign | (uint16_t)(E << 7) | (uint16_t)((int)m - 128);
+}
+
+/* T0 storage format (process state, tests only: orc_set_t0_bf16): 0 keeps
+   the fp16 K and V of a T0 token as they are; 1 stores them as bf16 (each
+   component rounded by h2bf), the format of the fused T0 / bf16 decode
+   path, read back exactly as bf16. */
+static int g_t0_bf16 = 0;
+void orc_set_t0_bf16(int on) { g_t0_bf16 = on ? 1 : 0; }
+int orc_t0_bf16(void) { return g_t0_bf16; }
+
+/* value of a T0 component as the store holds it */
+static double t0_val(uint16_t h) { return g_t0_bf16 ? bf2d(h2bf(h)) : h2d(h); }
+
 /* fp16 value as an integer multiple of 2^-24: value = m * 2^-24, |m| < 2^41 */
 static int64_t h2m(uint16_t h) {
     int s = h >> 15, e = (h >> 10) & 31, f = h & 1023;
@@ -772,8 +802,8 @@ static void write_row(uint8_t* page, int tier, int P, int d, int r,
         for (int dd = 0; dd < d; dd++) {
             int c = dd / 8, e = dd % 8;
             int pos = c ^ (4 * (r & 1));
-            put16(ks + (int64_t)r * 256 + pos * 16 + e * 2, k[dd]);
-            put16(vs + v_frag_offset(r, dd, 2), v[dd]);
+            put16(ks + (int64_t)r * 256 + pos * 16 + e * 2, g_t0_bf16 ? h2bf(k[dd]) : k[dd]);
+            put16(vs + v_frag_offset(r, dd, 2), g_t0_bf16 ? h2bf(v[dd]) : v[dd]);
         }
         return;
     }
@@ -916,7 +946,7 @@ int orc_decode(int B, int Hq, int Hkv, int Tmax, int d, const int32_t* seq_lens,
             if (tr == TIER_DROP) { logit[t] = -INFINITY; continue; }
             const uint16_t* k = K + idx * d;
             if (tr == TIER_T0)
-                for (int c = 0; c < d; c++) kh[c] = h2d(k[c]);
+                for (int c = 0; c < d; c++) kh[c] = t0_val(k[c]);
             else
                 orc_reconstruct_tier(k, d, tr, kh);
             double s = 0.0;
@@ -939,7 +969,7 @@ int orc_decode(int B, int Hq, int Hkv, int Tmax, int d, const int32_t* seq_lens,
                 l += wgt;
                 const uint16_t* v = V + idx * d;
                 if (tier[idx] == TIER_T0) {
-                    for (int c = 0; c < d; c++) o[c] += wgt * h2d(v[c]);
+                    for (int c = 0; c < d; c++) o[c] += wgt * t0_val(v[c]);
                 } else {
                     orc_vquant(v, d, v8, &sc);
                     double s = h2d(sc);
@@ -1023,7 +1053,7 @@ int orc_attention_mass(int B, int Hq, int Hkv, int Tmax, int d, const int32_t* s
             if (tr == TIER_DROP) { logit[t] = -INFINITY; continue; }
             const uint16_t* k = K + idx * d;
             if (tr == TIER_T0)
-                for (int c = 0; c < d; c++) kh[c] = h2d(k[c]);
+                for (int c = 0; c < d; c++) kh[c] = t0_val(k[c]);
             else
                 orc_reconstruct_tier(k, d, tr, kh);
             double s = 0.0;
@@ -1054,6 +1084,7 @@ int orc_attention_mass(int B, int Hq, int Hkv, int Tmax, int d, const int32_t* s
 uint16_t orc_d2h(double x) { return d2h(x); }
 double orc_h2d(uint16_t h) { return h2d(h); }
 double orc_bf2d(uint16_t h) { return bf2d(h); }
+uint16_t orc_h2bf(uint16_t h) { return h2bf(h); }
 int orc_threads(void) {
 #ifdef _OPENMP
     return omp_get_max_threads();
