@@ -54,6 +54,8 @@ def parse_args():
     ap.add_argument("--no-dense", action="store_true", help="skip the dense bf16 baseline")
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle cpu_baseline leg")
     ap.add_argument("--no-append", action="store_true", help="skip the skv_append timing")
+    ap.add_argument("--no-t0-bf16", action="store_true",
+                    help="skip the fused T0 / bf16 variant's timing")
     ap.add_argument("--no-utility", action="store_true",
                     help="skip the skv_decode_utility timing")
     ap.add_argument("--cp", action="store_true",
@@ -421,6 +423,54 @@ def run_skv(args, rank, world, local_rank):
                  "ada_speedup_step": dms / ms_per_step}
         del dcs, dws
 
+    # ---- the fused T0 / bf16 variant: the same tiers with T0 pages in bf16,
+    # decoded on the bf16 path, timed as the main step
+    t0b = None
+    if not args.no_t0_bf16:
+        ctx_b = skv.Context(w.P, t0_bf16=True)
+        bcs = []
+        for k in range(2):
+            bc = skv.PagedCache(ctx_b, w.B, w.Hkv, w.Tmax, w.pool_slots, device=dev)
+            bc.allocate(d["K"], d["seq_lens"], d["utility"], d["protect"], w.mode, d["budget"],
+                        d["quota"], d["free_lists"])
+            bc.encode(d["K"], d["V"], d["seq_lens"])
+            bc.check()
+            bcs.append(bc)
+        bws = [bc.workspace(w.Hq, S) for bc in bcs]
+
+        def bstep(i):
+            def f(mid):
+                ctx_b.set_profile_event(mid)
+                bcs[i].decode(d["q"], d["q_dtype"], w.Hq, out=out, lse=lse, workspace=bws[i],
+                              num_splits=S)
+            return f
+        bsteps = max(10, min(args.steps, 2000))
+        gb, gb_tail, gb_prof, evb, repb = timed_graph_steps([bstep(0), bstep(1)], bsteps,
+                                                            min(args.warmup, 20), args.graph_steps,
+                                                            stream)
+        ctx_b.set_profile_event(None)
+        torch.cuda.synchronize()
+        ta, tb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ta.record()
+        for _ in range(repb):
+            gb.replay()
+        if gb_tail is not None:
+            gb_tail.replay()
+        tb.record()
+        torch.cuda.synchronize()
+        gb_prof.replay()
+        torch.cuda.synchronize()
+        bcs[0].check()
+        bms = ta.elapsed_time(tb) / bsteps
+        bk = float(np.mean([a.elapsed_time(b) for a, b, c in evb]))
+        t0b = {"ms_per_step": bms, "kernel_ms": bk, "steps": bsteps,
+               "step_ratio_vs_mixed": bms / ms_per_step,
+               "kernel_ratio_vs_mixed": bk / kern_ms_avg,
+               "how": "the same tiers and bytes, T0 pages in bf16 decoded on the dense "
+                      "kernel's bf16 logit and P.V steps (skv_config.t0_bf16); graph replays "
+                      "over two stores, CUDA events"}
+        del bcs, bws, gb, gb_tail, gb_prof
+
     # ---- the decode with the utility update (skv_decode_utility) on the same
     # two stores, timed as the main step (graph replays, CUDA events)
     utility = None
@@ -543,6 +593,7 @@ def run_skv(args, rank, world, local_rank):
             "gpu_launches": 2 * args.steps,  # decode_kernel + decode_merge_kernel per step
             "clocks": clocks,
             "dense_bf16_baseline": dense,
+            "t0_bf16_variant": t0b,
             "ingest": {"allocate_ms": alloc_ms, "encode_ms": enc_ms, "gen_s": t_gen},
             "append": append,
             "utility": utility,

@@ -99,7 +99,14 @@ typedef struct skv_config {
                           unit-aligned split balances its runs' tails at run
                           time, and results may differ between calls in the
                           last bits (about 1e-5 relative) */
-  int32_t reserved[2]; /* zero */
+  int32_t t0_bf16;     /* nonzero: the fused T0 / bf16 path.  T0 rows hold K and V
+                          as bf16 (each fp16 input rounded to nearest even, the
+                          dense baseline's element type) and the decode takes
+                          the dense kernel's bf16 logit and P.V path for T0
+                          pages; needs the default T1 scheme and share grid.
+                          skv_retier, which re-encodes T0 rows from their exact
+                          fp16 keys, refuses such a store (SKV_ERR_ARG) */
+  int32_t reserved[1]; /* zero */
 } skv_config;
 
 /* Device pools of page slots, one per tier.  Slot s of tier t starts at

@@ -27,6 +27,7 @@ struct skv_ctx {
   int t1_scheme = 0;            // 0: 6-bit angle + 2-bit share; 1: 5-bit + 3-bit
   int share_grid = 0;           // 2-bit share grid: 0 uniform, 1 Lloyd-Max
   int deterministic = 0;        // the decode's split is static (no run-time chunks)
+  int t0_bf16 = 0;              // T0 rows in bf16, decoded on the bf16 path
   long long wait_limit = 0;     // decode waits: SM clocks (0: the default, about 1 s)
   float kappa[3];
   float rho_levels[4];
@@ -135,6 +136,11 @@ int skv_create(const skv_config* cfg, skv_ctx** out) {
   }
   c->share_grid = cfg->share_grid;
   c->deterministic = cfg->deterministic != 0;
+  c->t0_bf16 = cfg->t0_bf16 != 0;
+  if (c->t0_bf16 && (c->t1_scheme || c->share_grid)) {
+    delete c;
+    return fail(SKV_ERR_ARG, "t0_bf16 needs the default T1 scheme and share grid");
+  }
   c->log2P = P == 16 ? 4 : (P == 32 ? 5 : 6);
   c->device = 0;
   c->profile_event = nullptr;
@@ -390,6 +396,7 @@ int skv_encode(skv_ctx* ctx, const uint16_t* K, const uint16_t* V, int B, int Hk
   }
   p.err = err_word;
   p.dense_bf16 = 0;
+  p.t0_bf16 = ctx->t0_bf16;
   std::memcpy(p.bx6, ctx->bx6, sizeof(p.bx6));
   std::memcpy(p.by6, ctx->by6, sizeof(p.by6));
   std::memcpy(p.bx4, ctx->bx4, sizeof(p.bx4));
@@ -443,6 +450,7 @@ int skv_append(skv_ctx* ctx, const uint16_t* K_new, const uint16_t* V_new, int B
   p.free0_cursor = free0_cursor;
   p.err = err_word;
   p.ws = static_cast<int32_t*>(workspace);
+  p.t0_bf16 = ctx->t0_bf16;
   cudaError_t e = skv::launch_append(p, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "skv_append launch");
   return ok();
@@ -465,6 +473,8 @@ int skv_retier(skv_ctx* ctx, int B, int Hkv, int64_t Tmax, const int32_t* seq_le
                uint32_t* released, int32_t* n_released, int32_t* err_word, void* workspace,
                size_t ws_bytes, void* stream) {
   if (!ctx) return fail(SKV_ERR_ARG, "skv_retier: null ctx");
+  if (ctx->t0_bf16)
+    return fail(SKV_ERR_ARG, "skv_retier: the demoted rows' exact fp16 keys are not in bf16 T0 pages");
   if (B < 0 || Hkv <= 0 || Hkv > 128 || Tmax < 0 || Tmax > (1LL << 23) || page_cap < 0 ||
       page_cap > 0x7FFFFFFFLL)
     return fail(SKV_ERR_ARG, "skv_retier: need B >= 0, 0 < Hkv <= 128, 0 <= Tmax <= 2^23");
@@ -612,6 +622,7 @@ static int decode_common(skv_ctx* ctx, const void* q, int q_dtype, int B, int Hq
   std::memcpy(p.sin5, ctx->sin5, sizeof(p.sin5));
   p.t1_scheme = ctx->t1_scheme;
   p.share_grid = ctx->share_grid;
+  p.t0_bf16 = dense ? 0 : ctx->t0_bf16;
   p.dynamic = ctx->deterministic ? 0 : 1;
   p.wait_limit = ctx->wait_limit > 0 ? ctx->wait_limit : 2000000000LL;
   cudaError_t e =

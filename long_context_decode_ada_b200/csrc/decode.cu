@@ -820,11 +820,14 @@ __device__ __forceinline__ void capture_logits(float* lg, int rA, int rB, bool v
 
 // 16 rows [row0, row0 + 16) of one page at shared address pg; tb1 / tb2:
 // this lane's copy in TBL1 / TBL2; lg: the page's logit rows, or NULL
-// (CAP: the kernel variant that captures logits).
-template <int G, bool DENSE, bool CAP>
+// (CAP: the kernel variant that captures logits).  T0B: the fused T0 / bf16
+// path, whose T0 pages hold bf16 K / V and take the dense kernel's logit and
+// P.V steps, with bf16 fragments of q formed from q32 for the page.
+template <int G, bool DENSE, bool CAP, bool T0B>
 __device__ __forceinline__ void process_rows(const DecodeParams& p, uint32_t pg, uint32_t tier,
                                              int row0, const QFrag& qf, uint32_t tb1,
-                                             uint32_t tb2, WarpState& st, int lane, float* lg) {
+                                             uint32_t tb2, WarpState& st, int lane, float* lg,
+                                             const float (*q32)[kHeadDim]) {
   const int t = lane >> 2, g = lane & 3;
   const int P = p.P;
   // header {u16 count, u8 tier, u8 magic}
@@ -848,7 +851,18 @@ __device__ __forceinline__ void process_rows(const DecodeParams& p, uint32_t pg,
     softmax_pv<G, 2>(vA ? a * qf.c0 : -INFINITY, vB ? b * qf.c0 : -INFINITY, 1.0f, 1.0f,
                      vsec_dense, vsec_dense + 2048, st, lane);
   } else {
-    if (tier == SKV_TIER_T0) {
+    if (T0B && tier == SKV_TIER_T0) {
+      QFrag qb;
+      make_qfrag<G, true>(q32, p.qk_scale_log2, p.q_bf16 != 0, lane, qb);
+      if (qb.two)
+        logits_k16<true, true>(pg, rA, g, qb, c, d);
+      else
+        logits_k16<true, false>(pg, rA, g, qb, c, d);
+      const float lA = vA ? (c[0] + d[0]) * qb.c0 : -INFINITY;
+      const float lB = vB ? (c[2] + d[2]) * qb.c0 : -INFINITY;
+      if constexpr (CAP) capture_logits<G>(lg, rA, rB, vA, vB, lA, lB, g);
+      softmax_pv<G, 2>(lA, lB, 1.0f, 1.0f, vsec_dense, vsec_dense + 2048, st, lane);
+    } else if (tier == SKV_TIER_T0) {
       logits_k16<false, false>(pg, rA, g, qf, c, d);
       const float lA = vA ? (c[0] + d[0]) * qf.c0 : -INFINITY;
       const float lB = vB ? (c[2] + d[2]) * qf.c0 : -INFINITY;
@@ -1605,7 +1619,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
             released = true;
             compute_code_rows<G, CAP>(p, cr, tier, row0, qf, tb1, tb2, st, lane, lg);
           } else {
-            process_rows<G, DENSE, CAP>(p, d.x + rel, tier, row0, qf, tb1, tb2, st, lane, lg);
+            process_rows<G, DENSE, CAP, (VAR & 4) != 0>(p, d.x + rel, tier, row0, qf, tb1, tb2,
+                                                        st, lane, lg, sm.q32);
           }
         }
       }
@@ -2025,8 +2040,10 @@ cudaError_t launch_decode_g(const DecodeParams& p, cudaStream_t stream, cudaEven
   // the logit-capturing variant when a logits buffer is given (ADA only)
   const bool cap = !DENSE && p.logits != nullptr;
   // the code-table variant (ADA only; the dense pages have no codes):
-  // bit 0 the T1 5 + 3 scheme, bit 1 the Lloyd-Max 2-bit share grid
-  const int var = DENSE ? 0 : ((p.t1_scheme ? 1 : 0) | (p.share_grid ? 2 : 0));
+  // bit 0 the T1 5 + 3 scheme, bit 1 the Lloyd-Max 2-bit share grid, bit 2
+  // the fused T0 / bf16 path (alone: the API refuses it with bits 0 / 1)
+  const int var = DENSE ? 0
+                        : (p.t0_bf16 ? 4 : ((p.t1_scheme ? 1 : 0) | (p.share_grid ? 2 : 0)));
   using K = void (*)(const DecodeParams);
   K kern;
   if (DENSE) {
@@ -2035,17 +2052,19 @@ cudaError_t launch_decode_g(const DecodeParams& p, cudaStream_t stream, cudaEven
     kern = var == 0 ? decode_kernel<G, DENSE, !DENSE, 0>
          : var == 1 ? decode_kernel<G, DENSE, !DENSE, 1>
          : var == 2 ? decode_kernel<G, DENSE, !DENSE, 2>
-                    : decode_kernel<G, DENSE, !DENSE, 3>;
+         : var == 3 ? decode_kernel<G, DENSE, !DENSE, 3>
+                    : decode_kernel<G, DENSE, !DENSE, 4>;
   } else {
     kern = var == 0 ? decode_kernel<G, DENSE, false, 0>
          : var == 1 ? decode_kernel<G, DENSE, false, 1>
          : var == 2 ? decode_kernel<G, DENSE, false, 2>
-                    : decode_kernel<G, DENSE, false, 3>;
+         : var == 3 ? decode_kernel<G, DENSE, false, 3>
+                    : decode_kernel<G, DENSE, false, 4>;
   }
   const int vi = (cap ? 1 : 0) + 2 * var;
   // The shared-memory opt-in is set once per device, variant and size
   // (outside any stream capture: the first call is expected to be eager).
-  static size_t configured[8][64] = {};
+  static size_t configured[10][64] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;

@@ -40,6 +40,14 @@ __device__ __forceinline__ u128 warp_sum_u128(u128 v) {
   return v;
 }
 
+// two fp16 (one 32-bit word) -> the two bf16 of their values, rounded to
+// nearest even
+__device__ __forceinline__ uint32_t half2_bits_to_bf16x2(uint32_t h) {
+  const __half2 x = *reinterpret_cast<const __half2*>(&h);
+  const float2 f = __half22float2(x);
+  return pack_bf16x2(f.x, f.y);
+}
+
 // b-bit angle sector of (x, y); bx/by: the 2^b boundary vectors.
 __device__ __forceinline__ uint32_t angle_code(uint16_t xh, uint16_t yh, int b, const float* bx,
                                                const float* by) {
@@ -121,7 +129,8 @@ __device__ __forceinline__ void load_boundaries(const Prm& p, Boundaries& sb) {
 
 // Write one token's row `row` into `page` (tier tr, P rows): the warp's lane
 // l holds the fp16 key and value components 4l..4l+3 in k4 / v4.  T0 keeps
-// them (as bf16 for the dense baseline), T1 / T2 encode them.
+// them (rounded to bf16 for the dense baseline and the fused T0 / bf16
+// path), T1 / T2 encode them.
 __device__ __forceinline__ void write_row(uint8_t* page, int P, int tr, int row, int lane,
                                           const uint16_t (&k4)[4], const uint16_t (&v4)[4],
                                           bool dense_bf16, int t1_scheme, int share_grid,
@@ -298,7 +307,8 @@ __global__ void __launch_bounds__(256) encode_kernel(const __grid_constant__ Enc
                           (uint16_t)(kv.y & 0xFFFF), (uint16_t)(kv.y >> 16)};
   const uint16_t v4[4] = {(uint16_t)(vv.x & 0xFFFF), (uint16_t)(vv.x >> 16),
                           (uint16_t)(vv.y & 0xFFFF), (uint16_t)(vv.y >> 16)};
-  write_row(page, P, tr, row, lane, k4, v4, p.dense_bf16 != 0, p.t1_scheme, p.share_grid, sb);
+  write_row(page, P, tr, row, lane, k4, v4, p.dense_bf16 != 0 || p.t0_bf16 != 0, p.t1_scheme,
+            p.share_grid, sb);
 }
 
 // ---------------------------------------------------------------- transcode
@@ -562,10 +572,15 @@ __global__ void __launch_bounds__(256) append_write_kernel(const __grid_constant
     row = (int)__shfl_sync(0xFFFFFFFFu, c, 0);
   }
   __syncwarp();
-  // the row, as the pack lays out T0 rows (see encode_kernel)
+  // the row, as the pack lays out T0 rows (see encode_kernel), in bf16 for
+  // the fused T0 / bf16 path
   const long long w = (long long)u * kHeadDim;
-  const uint2 kv = *reinterpret_cast<const uint2*>(p.K + w + 4 * lane);
-  const uint2 vv = *reinterpret_cast<const uint2*>(p.V + w + 4 * lane);
+  uint2 kv = *reinterpret_cast<const uint2*>(p.K + w + 4 * lane);
+  uint2 vv = *reinterpret_cast<const uint2*>(p.V + w + 4 * lane);
+  if (p.t0_bf16) {
+    kv = make_uint2(half2_bits_to_bf16x2(kv.x), half2_bits_to_bf16x2(kv.y));
+    vv = make_uint2(half2_bits_to_bf16x2(vv.x), half2_bits_to_bf16x2(vv.y));
+  }
   const int c = lane >> 1, e0 = (lane & 1) * 4;
   const int pos = c ^ (4 * (row & 1));
   *reinterpret_cast<uint2*>(page + kHdrBytes + row * 256 + pos * 16 + e0 * 2) = kv;

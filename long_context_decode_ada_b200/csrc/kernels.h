@@ -36,6 +36,7 @@ struct DecodeParams {
   float cos5[32], sin5[32];  // angles of the T1 variant (5-bit angle + 3-bit share)
   int t1_scheme;             // T1 code byte: 0 (angle6 << 2) | share2; 1 (angle5 << 3) | share3
   int share_grid;            // 2-bit share grid: 0 uniform, 1 Lloyd-Max
+  int t0_bf16;               // T0 pages hold bf16 K / V (the fused T0 / bf16 path)
   int dynamic;               // unit-aligned split: hand out the units' last pages at run time
   long long wait_limit;      // SM clocks a planner / issuer / consumer wait may take
 };
@@ -57,6 +58,7 @@ struct EncodeParams {
   long long stride[3];
   int32_t* err;
   int dense_bf16;
+  int t0_bf16;          // T0 rows as bf16 (the fused T0 / bf16 path)
   float bx6[64], by6[64], bx4[16], by4[16];
   float bx5[32], by5[32];
   int t1_scheme;        // 0: 6-bit angle + 2-bit share; 1: 5-bit angle + 3-bit share
@@ -84,6 +86,7 @@ struct AppendParams {
   int32_t* free0_cursor;
   int32_t* err;
   int32_t* ws;              // append_ws() int32 words
+  int t0_bf16;              // the T0 rows as bf16
 };
 
 // Append workspace (int32 words): per unit t, need, new-before, old T0 end;

@@ -45,7 +45,7 @@ class SkvConfig(C.Structure):
     _fields_ = [("head_dim", C.c_int32), ("page_size", C.c_int32),
                 ("outlier_protect", C.c_int32), ("t1_angle_bits", C.c_int32),
                 ("share_grid", C.c_int32), ("deterministic", C.c_int32),
-                ("reserved", C.c_int32 * 2)]
+                ("t0_bf16", C.c_int32), ("reserved", C.c_int32 * 1)]
 
 
 class SkvPools(C.Structure):
@@ -195,10 +195,12 @@ class Context:
     """An skv_ctx: head_dim 128, page size P; bound to the current device."""
 
     def __init__(self, page_size: int, head_dim: int = 128, outlier_protect: bool = False,
-                 t1_angle_bits: int = 6, share_grid: int = 0, deterministic: bool = False):
+                 t1_angle_bits: int = 6, share_grid: int = 0, deterministic: bool = False,
+                 t0_bf16: bool = False):
         cfg = SkvConfig(head_dim=head_dim, page_size=page_size,
                         outlier_protect=1 if outlier_protect else 0, t1_angle_bits=t1_angle_bits,
-                        share_grid=share_grid, deterministic=1 if deterministic else 0)
+                        share_grid=share_grid, deterministic=1 if deterministic else 0,
+                        t0_bf16=1 if t0_bf16 else 0)
         h = C.c_void_p()
         _check(lib().skv_create(C.byref(cfg), C.byref(h)))
         self._h = h
@@ -208,6 +210,7 @@ class Context:
         self.t1_angle_bits = t1_angle_bits
         self.share_grid = share_grid
         self.deterministic = bool(deterministic)
+        self.t0_bf16 = bool(t0_bf16)
 
     def __del__(self):
         h = getattr(self, "_h", None)
