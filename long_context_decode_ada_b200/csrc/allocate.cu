@@ -36,6 +36,7 @@ size_t alloc_workspace_bytes(int B, int Hkv, long long Tmax) {
   n += al256(4 * U * 3);
   n += al256(8 * (size_t)B);
   n += al256(U * (size_t)Tmax);
+  n += al256(12 * U * (size_t)((Tmax + kRowChunk - 1) / kRowChunk));
   return n;
 }
 
@@ -56,6 +57,8 @@ void alloc_carve(AllocParams& p, void* ws) {
   p.pinned = reinterpret_cast<long long*>(w);
   w += al256(8 * (size_t)p.B);
   p.eff_protect = w;
+  w += al256(U * (size_t)p.Tmax);
+  p.ccounts = reinterpret_cast<int32_t*>(w);
 }
 
 // ---------------------------------------------------------------- keys --
@@ -142,14 +145,17 @@ __device__ __forceinline__ void pin_token(const AllocParams& p, long long w, int
               (unsigned long long)tier_row_bytes(tier));
 }
 
-// budget mode: one warp per token; keyw = u * fp32(r^2), -1 when protected
-__global__ void __launch_bounds__(256) keys_budget_kernel(const __grid_constant__ AllocParams p) {
-  const long long w = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+// budget mode: one warp per token; keyw = u * fp32(r^2), -1 when protected.
+// Block x of a unit's nbx = ceil(Tmax / 8) blocks takes positions 8x .. 8x + 7
+// (one 32-bit division per block, none per token).
+__global__ void __launch_bounds__(256) keys_budget_kernel(const __grid_constant__ AllocParams p,
+                                                          unsigned nbx) {
   const int lane = threadIdx.x & 31;
-  if (w >= (long long)p.B * p.Hkv * p.Tmax) return;
-  const long long t = w % p.Tmax;
-  const int b = (int)(w / p.Tmax / p.Hkv);
-  if (t >= p.seq_lens[b]) return;
+  const unsigned u = blockIdx.x / nbx;
+  const long long t = (long long)(blockIdx.x - u * nbx) * 8 + (threadIdx.x >> 5);
+  const int b = (int)(u / (unsigned)p.Hkv);
+  if (t >= p.Tmax || t >= p.seq_lens[b]) return;
+  const long long w = (long long)u * p.Tmax + t;
   if (p.protect && p.protect[w]) {
     if (lane == 0) pin_token(p, w, b, SKV_TIER_T0);
     return;
@@ -247,40 +253,33 @@ __global__ void sel_init_kernel(const __grid_constant__ AllocParams p) {
   }
 }
 
-__device__ __forceinline__ bool item_composite(const AllocParams& p, int seg, long long i,
-                                               unsigned long long& comp, uint32_t& weight) {
-  if (p.mode == SKV_MODE_BUDGET) {
-    const int k = (int)(i % 3);
-    const long long ht = i / 3;
-    const int h = (int)(ht / p.Tmax);
-    const long long t = ht % p.Tmax;
-    if (t >= p.seq_lens[seg]) return false;
-    const float w = p.keyw[((long long)seg * p.Hkv + h) * p.Tmax + t];
-    if (w < 0.0f) return false;
-    const float key = __fmul_rn(w, p.kappa[k]);
-    comp = ((unsigned long long)(0xFFFFFFFFu - __float_as_uint(key)) << 32) |
-           ((unsigned long long)k << 30) | ((unsigned long long)h << 23) | (unsigned long long)t;
-    weight = (k == 0) ? 180u : (k == 1 ? 16u : 316u);
-    return true;
-  }
-  const int b = seg / p.Hkv;
-  if (i >= p.seq_lens[b]) return false;
-  const float w = p.keyw[(long long)seg * p.Tmax + i];
-  if (w < 0.0f) return false;
-  comp = ((unsigned long long)(0xFFFFFFFFu - __float_as_uint(w)) << 32) | (unsigned long long)i;
-  weight = 1;
-  return true;
+// 64-bit composite of budget step k of token (h, t) with weight w: the
+// priority fp32(w kappa_k) descending, then step, head, position ascending
+__device__ __forceinline__ unsigned long long budget_comp(const AllocParams& p, float w, int k,
+                                                         int h, long long t) {
+  const float key = __fmul_rn(w, p.kappa[k]);
+  return ((unsigned long long)(0xFFFFFFFFu - __float_as_uint(key)) << 32) |
+         ((unsigned long long)k << 30) | ((unsigned long long)h << 23) | (unsigned long long)t;
 }
 
-constexpr int kHistItemsPerBlock = 4096;
+constexpr int kHistItemsPerBlock = 4096;  // tokens (budget) or positions (quota) per block
 
+// Weighted histogram of one 8-bit digit of the composites that still match
+// each target's prefix.  Budget mode: a thread per token (h, t) of sequence
+// seg with its three steps (weights 180, 16, 316 bytes); quota mode: a thread
+// per position of unit seg (weight 1, three targets).  Every lane of a warp
+// runs the same number of rounds (the tail lanes with nothing), so the lanes
+// that add to the same bin are grouped: one shared atomic per group and
+// round instead of one per lane (the early passes put nearly every item into
+// a few bins).
 __global__ void __launch_bounds__(256) hist_kernel(const __grid_constant__ AllocParams p,
                                                    int shift) {
   __shared__ unsigned long long sh[3][256];
   __shared__ unsigned long long pre[3];
   __shared__ int dn[3];
   const int seg = blockIdx.y;
-  const int ntgt = p.mode == SKV_MODE_BUDGET ? 1 : 3;
+  const bool budget = p.mode == SKV_MODE_BUDGET;
+  const int ntgt = budget ? 1 : 3;
   if (threadIdx.x < 3) {
     const unsigned long long* st = p.sel + ((size_t)seg * 3 + threadIdx.x) * 3;
     pre[threadIdx.x] = st[0];
@@ -289,19 +288,47 @@ __global__ void __launch_bounds__(256) hist_kernel(const __grid_constant__ Alloc
   for (int i = threadIdx.x; i < 3 * 256; i += blockDim.x) (&sh[0][0])[i] = 0;
   __syncthreads();
   if (dn[0] && dn[1] && dn[2]) return;
-  const long long n_items =
-      p.mode == SKV_MODE_BUDGET ? (long long)p.Hkv * p.Tmax * 3 : (long long)p.Tmax;
+  const long long n = budget ? (long long)p.Hkv * p.Tmax : p.Tmax;
   const long long i0 = (long long)blockIdx.x * kHistItemsPerBlock;
-  const long long i1 = min(n_items, i0 + kHistItemsPerBlock);
-  for (long long i = i0 + threadIdx.x; i < i1; i += blockDim.x) {
-    unsigned long long comp;
-    uint32_t wgt;
-    if (!item_composite(p, seg, i, comp, wgt)) continue;
-    const int dig = (int)((comp >> shift) & 255u);
-    for (int j = 0; j < ntgt; ++j) {
-      if (dn[j]) continue;
-      if (shift < 56 && (comp >> (shift + 8)) != (pre[j] >> (shift + 8))) continue;
-      atomicAdd(&sh[j][dig], (unsigned long long)wgt);
+  const long long i1 = min(n, i0 + kHistItemsPerBlock);
+  const int lane = threadIdx.x & 31;
+  for (long long base = i0; base < i1; base += blockDim.x) {
+    const long long i = base + threadIdx.x;
+    if (budget) {
+      // token i = h Tmax + t of sequence seg (Hkv Tmax < 2^31: 32-bit division)
+      int h = 0;
+      long long t = 0;
+      float w = -1.0f;
+      if (i < i1) {
+        h = (int)((unsigned)i / (unsigned)p.Tmax);
+        t = i - (long long)h * p.Tmax;
+        if (t < p.seq_lens[seg]) w = p.keyw[(long long)seg * n + i];
+      }
+      const bool have = w >= 0.0f && !dn[0];
+#pragma unroll
+      for (int k = 0; k < 3; ++k) {
+        const unsigned long long comp = have ? budget_comp(p, w, k, h, t) : 0ull;
+        const int dig = (int)((comp >> shift) & 255u);
+        const bool in = have && (shift >= 56 || (comp >> (shift + 8)) == (pre[0] >> (shift + 8)));
+        const uint32_t peers = __match_any_sync(0xFFFFFFFFu, in ? (uint32_t)dig : ~0u);
+        if (in && lane == __ffs(peers) - 1)
+          atomicAdd(&sh[0][dig], (unsigned long long)(k == 0 ? 180u : (k == 1 ? 16u : 316u)) *
+                                     (unsigned long long)__popc(peers));
+      }
+    } else {
+      const int b = seg / p.Hkv;
+      float w = -1.0f;
+      if (i < i1 && i < p.seq_lens[b]) w = p.keyw[(long long)seg * p.Tmax + i];
+      const unsigned long long comp =
+          ((unsigned long long)(0xFFFFFFFFu - __float_as_uint(w)) << 32) | (unsigned long long)i;
+      const int dig = (int)((comp >> shift) & 255u);
+      for (int j = 0; j < 3; ++j) {
+        const bool in = w >= 0.0f && !dn[j] &&
+                        (shift >= 56 || (comp >> (shift + 8)) == (pre[j] >> (shift + 8)));
+        const uint32_t peers = __match_any_sync(0xFFFFFFFFu, in ? (uint32_t)dig : ~0u);
+        if (in && lane == __ffs(peers) - 1)
+          atomicAdd(&sh[j][dig], (unsigned long long)__popc(peers));
+      }
     }
   }
   __syncthreads();
@@ -311,31 +338,39 @@ __global__ void __launch_bounds__(256) hist_kernel(const __grid_constant__ Alloc
   }
 }
 
-__global__ void sel_step_kernel(const __grid_constant__ AllocParams p, int shift) {
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= p.nseg * 3) return;
+// One block of 256 threads per (segment, target): bin d of the histogram is
+// thread d's; a block-wide inclusive scan finds the one digit at which the
+// target's remaining weight falls (the cumulative weight before it at most
+// the remainder, with it above), and every bin is cleared for the next pass.
+__global__ void __launch_bounds__(256) sel_step_kernel(const __grid_constant__ AllocParams p,
+                                                       int shift) {
+  __shared__ unsigned long long wsum[8];
+  const int i = blockIdx.x;
+  if (i >= p.nseg * 3) return;  // uniform over the block
+  const int d = threadIdx.x, lane = d & 31, wid = d >> 5;
   unsigned long long* st = p.sel + (size_t)i * 3;
   unsigned long long* h = p.hist + (size_t)i * 256;
-  if (st[2]) {
-    for (int d = 0; d < 256; ++d) h[d] = 0;
-    return;
-  }
+  const unsigned long long v = h[d];
+  h[d] = 0;
+  const bool done = st[2] != 0;
   const unsigned long long rem = st[1];
-  unsigned long long cum = 0;
-  bool found = false;
-  for (int d = 0; d < 256; ++d) {
-    const unsigned long long v = h[d];
-    h[d] = 0;
-    if (found) continue;
-    if (cum + v > rem) {
-      st[0] |= (unsigned long long)d << shift;
-      st[1] = rem - cum;
-      found = true;
-    } else {
-      cum += v;
-    }
+  unsigned long long x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned long long y = __shfl_up_sync(0xFFFFFFFFu, x, o);
+    if (lane >= o) x += y;
   }
-  if (!found) {
+  if (lane == 31) wsum[wid] = x;
+  __syncthreads();  // every thread has read st before any writes it
+  unsigned long long before = 0;
+  for (int k = 0; k < wid; ++k) before += wsum[k];
+  const unsigned long long incl = before + x, excl = incl - v;
+  if (done) return;
+  if (excl <= rem && incl > rem) {  // at most one thread
+    st[0] |= (unsigned long long)d << shift;
+    st[1] = rem - excl;
+  }
+  if (d == 255 && incl <= rem) {
     st[2] = 1;
     st[0] = ~0ull;  // every item is below the cut
   }
@@ -358,13 +393,7 @@ __global__ void tier_kernel(const __grid_constant__ AllocParams p) {
       const unsigned long long cut = p.sel[(size_t)b * 3 * 3 + 0];
       int lvl = 0;
 #pragma unroll
-      for (int k = 0; k < 3; ++k) {
-        const float key = __fmul_rn(w, p.kappa[k]);
-        const unsigned long long comp =
-            ((unsigned long long)(0xFFFFFFFFu - __float_as_uint(key)) << 32) |
-            ((unsigned long long)k << 30) | ((unsigned long long)h << 23) | (unsigned long long)t;
-        lvl += comp < cut;
-      }
+      for (int k = 0; k < 3; ++k) lvl += budget_comp(p, w, k, h, t) < cut;
       tr = lvl == 3 ? SKV_TIER_T0 : (lvl == 2 ? SKV_TIER_T1 : (lvl == 1 ? SKV_TIER_T2 : SKV_TIER_DROP));
     } else {
       const unsigned long long comp =
@@ -381,29 +410,41 @@ __global__ void tier_kernel(const __grid_constant__ AllocParams p) {
 
 // -------------------------------------------------------- counts and plan --
 
-__global__ void unit_count_kernel(const __grid_constant__ AllocParams p) {
+// Tier counts per (unit, chunk of kRowChunk positions) into ccounts, and per
+// unit (counts, zeroed before) by atomics.  Grid: x the chunks, y a stride
+// over the units.
+__global__ void __launch_bounds__(256) unit_count_kernel(const __grid_constant__ AllocParams p) {
   __shared__ int c[3];
-  const int u = blockIdx.x;
-  const int b = u / p.Hkv;
-  if (threadIdx.x < 3) c[threadIdx.x] = 0;
-  __syncthreads();
-  const long long T = p.seq_lens[b];
-  int l0 = 0, l1 = 0, l2 = 0;
-  for (long long t = threadIdx.x; t < T; t += blockDim.x) {
-    if (p.dense) {
-      ++l0;
-      continue;
+  const int U = p.B * p.Hkv;
+  const int nch = (int)((p.Tmax + kRowChunk - 1) / kRowChunk);
+  const long long t0 = (long long)blockIdx.x * kRowChunk;
+  for (int u = blockIdx.y; u < U; u += gridDim.y) {
+    if (threadIdx.x < 3) c[threadIdx.x] = 0;
+    __syncthreads();
+    const long long T = p.seq_lens[u / p.Hkv];
+    const long long t1 = min(T, t0 + kRowChunk);
+    int l0 = 0, l1 = 0, l2 = 0;
+    for (long long t = t0 + threadIdx.x; t < t1; t += blockDim.x) {
+      if (p.dense) {
+        ++l0;
+        continue;
+      }
+      const uint8_t tr = p.tier_out[(long long)u * p.Tmax + t];
+      l0 += tr == 0;
+      l1 += tr == 1;
+      l2 += tr == 2;
     }
-    const uint8_t tr = p.tier_out[(long long)u * p.Tmax + t];
-    l0 += tr == 0;
-    l1 += tr == 1;
-    l2 += tr == 2;
+    if (l0) atomicAdd(&c[0], l0);
+    if (l1) atomicAdd(&c[1], l1);
+    if (l2) atomicAdd(&c[2], l2);
+    __syncthreads();
+    if (threadIdx.x < 3) {
+      const int v = c[threadIdx.x];
+      p.ccounts[((long long)u * nch + blockIdx.x) * 3 + threadIdx.x] = v;
+      if (v) atomicAdd(&p.counts[u * 3 + threadIdx.x], v);
+    }
+    __syncthreads();
   }
-  atomicAdd(&c[0], l0);
-  atomicAdd(&c[1], l1);
-  atomicAdd(&c[2], l2);
-  __syncthreads();
-  if (threadIdx.x < 3) p.counts[u * 3 + threadIdx.x] = c[threadIdx.x];
 }
 
 // block-wide exclusive scan of long long (blockDim.x = 1024)
@@ -517,16 +558,32 @@ __global__ void __launch_bounds__(1024) page_plan_kernel(const __grid_constant__
   }
 }
 
+// Row map, one block per (unit, chunk of kRowChunk positions): the chunk's
+// rank base per tier is the sum of the unit's earlier chunks' counts, and a
+// block scan ranks its positions (three 21-bit fields: a chunk holds at most
+// 1024 of each tier).
 __global__ void __launch_bounds__(1024) row_of_kernel(const __grid_constant__ AllocParams p) {
-  const int u = blockIdx.x;
-  const int b = u / p.Hkv;
-  const long long T = p.seq_lens[b];
+  const int U = p.B * p.Hkv;
+  const int nch = (int)((p.Tmax + kRowChunk - 1) / kRowChunk);
+  const int ch = blockIdx.x;
   const int P = p.P;
-  const long long c0 = p.counts[u * 3], c1 = p.counts[u * 3 + 1];
-  const long long pb[3] = {0, (c0 + P - 1) / P, (c0 + P - 1) / P + (c1 + P - 1) / P};
-  long long run[3] = {0, 0, 0};
-  for (long long base = 0; base < T; base += blockDim.x) {
-    const long long t = base + threadIdx.x;
+  for (int u = blockIdx.y; u < U; u += gridDim.y) {
+    const long long T = p.seq_lens[u / p.Hkv];
+    if ((long long)ch * kRowChunk >= T) continue;  // uniform over the block
+    long long s0 = 0, s1 = 0, s2 = 0;
+    for (int c = threadIdx.x; c < ch; c += blockDim.x) {
+      const int32_t* cc = p.ccounts + ((long long)u * nch + c) * 3;
+      s0 += cc[0];
+      s1 += cc[1];
+      s2 += cc[2];
+    }
+    long long base[3];
+    block_exclusive_scan(s0, base[0]);
+    block_exclusive_scan(s1, base[1]);
+    block_exclusive_scan(s2, base[2]);
+    const long long c0 = p.counts[u * 3], c1 = p.counts[u * 3 + 1];
+    const long long pb[3] = {0, (c0 + P - 1) / P, (c0 + P - 1) / P + (c1 + P - 1) / P};
+    const long long t = (long long)ch * kRowChunk + threadIdx.x;
     const long long i = (long long)u * p.Tmax + t;
     int tr = SKV_TIER_DROP;
     if (t < T) tr = p.tier_out[i];
@@ -534,10 +591,9 @@ __global__ void __launch_bounds__(1024) row_of_kernel(const __grid_constant__ Al
     long long tot;
     const long long ex = block_exclusive_scan(f, tot);
     if (t < T && tr < 3) {
-      const long long rank = run[tr] + ((ex >> (21 * tr)) & ((1LL << 21) - 1));
+      const long long rank = base[tr] + ((ex >> (21 * tr)) & ((1LL << 21) - 1));
       p.row_of[i] = (int32_t)((pb[tr] + rank / P) * P + rank % P);
     }
-    for (int k = 0; k < 3; ++k) run[k] += (tot >> (21 * k)) & ((1LL << 21) - 1);
   }
 }
 
@@ -633,6 +689,21 @@ static unsigned grid_for(long long n, int threads) {
   return (unsigned)(b < 1 ? 1 : b);
 }
 
+// chunks of positions (x) by a stride over the units (y)
+static dim3 row_grid(const AllocParams& p) {
+  const long long nch = (p.Tmax + kRowChunk - 1) / kRowChunk;
+  const long long U = (long long)p.B * p.Hkv;
+  return dim3((unsigned)(nch < 1 ? 1 : nch), (unsigned)std::max(1LL, std::min(U, 65535LL)));
+}
+
+static cudaError_t launch_counts(AllocParams& p, cudaStream_t stream) {
+  const size_t U = (size_t)p.B * p.Hkv;
+  cudaError_t e = cudaMemsetAsync(p.counts, 0, 4 * 3 * U, stream);
+  if (e != cudaSuccess) return e;
+  if (U > 0) unit_count_kernel<<<row_grid(p), 256, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_allocate(AllocParams& p, cudaStream_t stream) {
   const long long ntok = (long long)p.B * p.Hkv * p.Tmax;
   const int U = p.B * p.Hkv;
@@ -648,26 +719,28 @@ cudaError_t launch_allocate(AllocParams& p, cudaStream_t stream) {
     p.protect = p.eff_protect;  // the key kernels read the joined mask
   }
   if (ntok > 0) {
-    if (p.mode == SKV_MODE_BUDGET)
-      keys_budget_kernel<<<grid_for(ntok * 32, 256), 256, 0, stream>>>(p);
+    if (p.mode == SKV_MODE_BUDGET) {
+      const long long nbx = (p.Tmax + 7) / 8;
+      if ((long long)U * nbx > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
+      keys_budget_kernel<<<(unsigned)(U * nbx), 256, 0, stream>>>(p, (unsigned)nbx);
+    }
     else
       keys_quota_kernel<<<grid_for(ntok, 256), 256, 0, stream>>>(p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   sel_init_kernel<<<grid_for(p.nseg * 3, 128), 128, 0, stream>>>(p);
-  const long long n_items =
-      p.mode == SKV_MODE_BUDGET ? (long long)p.Hkv * p.Tmax * 3 : (long long)p.Tmax;
+  const long long n_items = p.mode == SKV_MODE_BUDGET ? (long long)p.Hkv * p.Tmax : p.Tmax;
   const dim3 hgrid(grid_for(n_items, kHistItemsPerBlock), p.nseg);
   for (int pass = 0; pass < 8; ++pass) {
     const int shift = 56 - 8 * pass;
     hist_kernel<<<hgrid, 256, 0, stream>>>(p, shift);
-    sel_step_kernel<<<grid_for(p.nseg * 3, 128), 128, 0, stream>>>(p, shift);
+    sel_step_kernel<<<std::max(1, p.nseg * 3), 256, 0, stream>>>(p, shift);
   }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (ntok > 0) tier_kernel<<<grid_for(ntok, 256), 256, 0, stream>>>(p);
-  unit_count_kernel<<<U, 256, 0, stream>>>(p);
+  if ((e = launch_counts(p, stream)) != cudaSuccess) return e;
   page_plan_kernel<<<1, 1024, 0, stream>>>(p);
-  row_of_kernel<<<U, 1024, 0, stream>>>(p);
+  row_of_kernel<<<row_grid(p), 1024, 0, stream>>>(p);
   page_write_kernel<<<grid_for(std::min<long long>(p.page_cap, 1LL << 22) * 32, 256), 256, 0,
                       stream>>>(p);
   return cudaGetLastError();
@@ -725,16 +798,16 @@ cudaError_t launch_retier_plan(AllocParams& p, cudaStream_t stream) {
   if ((e = cudaMemsetAsync(p.diff, 0x7F, 4 * 3 * (size_t)U, stream)) != cudaSuccess) return e;
   if (ntok > 0) keys_retier_kernel<<<grid_for(ntok * 32, 256), 256, 0, stream>>>(p);
   sel_init_kernel<<<grid_for(p.nseg * 3, 128), 128, 0, stream>>>(p);
-  const dim3 hgrid(grid_for((long long)p.Hkv * p.Tmax * 3, kHistItemsPerBlock), p.nseg);
+  const dim3 hgrid(grid_for((long long)p.Hkv * p.Tmax, kHistItemsPerBlock), p.nseg);
   for (int pass = 0; pass < 8; ++pass) {
     const int shift = 56 - 8 * pass;
     hist_kernel<<<hgrid, 256, 0, stream>>>(p, shift);
-    sel_step_kernel<<<grid_for(p.nseg * 3, 128), 128, 0, stream>>>(p, shift);
+    sel_step_kernel<<<std::max(1, p.nseg * 3), 256, 0, stream>>>(p, shift);
   }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (ntok > 0) tier_kernel<<<grid_for(ntok, 256), 256, 0, stream>>>(p);
-  unit_count_kernel<<<U, 256, 0, stream>>>(p);
-  row_of_kernel<<<U, 1024, 0, stream>>>(p);
+  if ((e = launch_counts(p, stream)) != cudaSuccess) return e;
+  row_of_kernel<<<row_grid(p), 1024, 0, stream>>>(p);
   if (ntok > 0) diff_kernel<<<grid_for(ntok, 256), 256, 0, stream>>>(p);
   page_plan_kernel<<<1, 1024, 0, stream>>>(p);
   page_write_kernel<<<grid_for(std::min<long long>(p.page_cap, 1LL << 22) * 32, 256), 256, 0,
@@ -745,9 +818,9 @@ cudaError_t launch_retier_plan(AllocParams& p, cudaStream_t stream) {
 }
 
 cudaError_t launch_dense_plan(AllocParams& p, cudaStream_t stream) {
-  const int U = p.B * p.Hkv;
   p.dense = 1;
-  unit_count_kernel<<<U, 256, 0, stream>>>(p);
+  cudaError_t e = launch_counts(p, stream);
+  if (e != cudaSuccess) return e;
   page_plan_kernel<<<1, 1024, 0, stream>>>(p);
   page_write_kernel<<<grid_for(std::min<long long>(p.page_cap, 1LL << 22) * 32, 256), 256, 0,
                       stream>>>(p);

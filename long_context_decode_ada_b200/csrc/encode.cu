@@ -15,6 +15,8 @@
 #include "common.cuh"
 #include "kernels.h"
 
+#include <algorithm>
+
 namespace skv {
 
 typedef unsigned __int128 u128;
@@ -23,10 +25,6 @@ __device__ __forceinline__ uint16_t double_to_half_rn(double x) {
   uint16_t r;
   asm("cvt.rn.f16.f64 %0, %1;" : "=h"(r) : "d"(x));
   return r;
-}
-
-__device__ __forceinline__ double half_to_double(uint16_t h) {
-  return (double)__half2float(__ushort_as_half(h));
 }
 
 __device__ __forceinline__ u128 warp_sum_u128(u128 v) {
@@ -48,10 +46,15 @@ __device__ __forceinline__ uint32_t half2_bits_to_bf16x2(uint32_t h) {
   return pack_bf16x2(f.x, f.y);
 }
 
-// b-bit angle sector of (x, y); bx/by: the 2^b boundary vectors.
-__device__ __forceinline__ uint32_t angle_code(uint16_t xh, uint16_t yh, int b, const float* bx,
-                                               const float* by) {
-  const double x = half_to_double(xh), y = half_to_double(yh);
+// b-bit angle sector of the pair (x, y) = (mx, my) 2^-24 (the fp16 values as
+// integers, half_bits_to_m); bx/by: the 2^b boundary vectors (fp32 values held
+// as doubles).  The sector depends only on the signs of the cross products
+// bx y - by x, unchanged by the positive scale 2^24; each product of a 24-bit
+// and an 11-bit significand is exact in fp64, and the difference is rounded
+// once, so its sign is exact.
+__device__ __forceinline__ uint32_t angle_code(long long mx, long long my, int b, const double* bx,
+                                               const double* by) {
+  const double x = (double)mx, y = (double)my;
   if (x == 0.0 && y == 0.0) return 0;
   int q;
   if (x > 0 && y >= 0) q = 0;
@@ -65,8 +68,7 @@ __device__ __forceinline__ uint32_t angle_code(uint16_t xh, uint16_t yh, int b, 
   int lo = 0, hi = per;
   while (lo < hi) {
     const int mid = (lo + hi) >> 1;
-    const double side = __dsub_rn(__dmul_rn((double)bx[base + mid], y),
-                                  __dmul_rn((double)by[base + mid], x));
+    const double side = __dsub_rn(__dmul_rn(bx[base + mid], y), __dmul_rn(by[base + mid], x));
     if (side >= 0.0) lo = mid + 1;
     else hi = mid;
   }
@@ -106,9 +108,10 @@ __device__ __forceinline__ int v_frag_offset(int row, int dd, int elem_bytes) {
   return k * 2048 + 512 * (mt >> 1) + 16 * L + 8 * (mt & 1) + 2 * e;
 }
 
-// The boundary vectors of the three angle codes, in shared memory.
+// The boundary vectors of the three angle codes (fp32 values), in shared
+// memory as doubles: the angle search then converts nothing.
 struct Boundaries {
-  float bx6[64], by6[64], bx4[16], by4[16], bx5[32], by5[32];
+  double bx6[64], by6[64], bx4[16], by4[16], bx5[32], by5[32];
 };
 
 template <class Prm>
@@ -179,10 +182,10 @@ __device__ __forceinline__ void write_row(uint8_t* page, int P, int tr, int row,
   const bool t1 = tr == SKV_TIER_T1;
   const bool v53 = t1 && t1_scheme;  // T1 variant: 5-bit angle + 3-bit share
   const int bits = t1 ? (v53 ? 5 : 6) : 4;
-  const float* bx = t1 ? (v53 ? sb.bx5 : sb.bx6) : sb.bx4;
-  const float* by = t1 ? (v53 ? sb.by5 : sb.by6) : sb.by4;
-  const uint32_t th0 = angle_code(k4[0], k4[1], bits, bx, by);
-  const uint32_t th1 = angle_code(k4[2], k4[3], bits, bx, by);
+  const double* bx = t1 ? (v53 ? sb.bx5 : sb.bx6) : sb.bx4;
+  const double* by = t1 ? (v53 ? sb.by5 : sb.by6) : sb.by4;
+  const uint32_t th0 = angle_code(m[0], m[1], bits, bx, by);
+  const uint32_t th1 = angle_code(m[2], m[3], bits, bx, by);
   const uint32_t rh0 = v53 ? rho_code3(m[0], m[1], R2) : rho_code(m[0], m[1], R2, share_grid);
   const uint32_t rh1 = v53 ? rho_code3(m[2], m[3], R2) : rho_code(m[2], m[3], R2, share_grid);
   const uint32_t packed = th0 | (th1 << 8) | (rh0 << 16) | (rh1 << 24);
@@ -260,24 +263,28 @@ __device__ __forceinline__ void write_row(uint8_t* page, int P, int tr, int row,
 }
 
 
-__global__ void __launch_bounds__(256) encode_kernel(const __grid_constant__ EncodeParams p) {
+// One warp per (unit, position): block x of a unit's nbx = ceil(Tmax / 8)
+// blocks takes positions 8x .. 8x + 7 (one 32-bit division per block, none
+// per token).
+#ifndef SKV_ENCODE_MIN_BLOCKS
+#define SKV_ENCODE_MIN_BLOCKS 5  // blocks per SM the register allocation must allow
+#endif
+__global__ void __launch_bounds__(256, SKV_ENCODE_MIN_BLOCKS)
+    encode_kernel(const __grid_constant__ EncodeParams p, unsigned nbx) {
   __shared__ Boundaries sb;
   load_boundaries(p, sb);
   __syncthreads();
-  const long long w = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
-  const long long total = (long long)p.B * p.Hkv * p.Tmax;
-  if (w >= total) return;
-  const long long t = w % p.Tmax;
-  const long long bh = w / p.Tmax;
-  const int b = (int)(bh / p.Hkv);
-  if (t >= p.seq_lens[b]) return;
-  const int P = p.P;
+  const unsigned bh = blockIdx.x / nbx;
+  const long long t = (long long)(blockIdx.x - bh * nbx) * 8 + (threadIdx.x >> 5);
+  const int P = p.P, lp = __ffs(P) - 1;  // P is a power of two
+  if (t >= p.Tmax || t >= p.seq_lens[bh / (unsigned)p.Hkv]) return;
+  const long long w = (long long)bh * p.Tmax + t;
   int tr, pi, row;
   if (p.dense_bf16) {
     tr = 0;
-    pi = (int)(t / P);
-    row = (int)(t % P);
+    pi = (int)(t >> lp);
+    row = (int)(t & (P - 1));
   } else {
     tr = p.tier[w];
     if (tr == SKV_TIER_DROP) return;
@@ -286,8 +293,8 @@ __global__ void __launch_bounds__(256) encode_kernel(const __grid_constant__ Enc
       if (lane == 0) report(p.err, SKV_ERR_CORRUPT);
       return;
     }
-    pi = loc / P;
-    row = loc % P;
+    pi = loc >> lp;
+    row = loc & (P - 1);
   }
   const long long gi = (long long)p.indptr[bh] + pi;
   if (gi >= p.indptr[bh + 1]) {
@@ -624,10 +631,11 @@ cudaError_t launch_transcode(const TranscodeParams& p, cudaStream_t stream) {
 }
 
 cudaError_t launch_encode(const EncodeParams& p, cudaStream_t stream) {
-  const long long warps = (long long)p.B * p.Hkv * p.Tmax;
-  if (warps == 0) return cudaSuccess;
-  const long long blocks = (warps * 32 + 255) / 256;
-  encode_kernel<<<(unsigned)blocks, 256, 0, stream>>>(p);
+  const long long U = (long long)p.B * p.Hkv;
+  if (U == 0 || p.Tmax == 0) return cudaSuccess;
+  const long long nbx = (p.Tmax + 7) / 8;
+  if (U * nbx > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
+  encode_kernel<<<(unsigned)(U * nbx), 256, 0, stream>>>(p, (unsigned)nbx);
   return cudaGetLastError();
 }
 

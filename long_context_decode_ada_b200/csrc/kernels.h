@@ -141,6 +141,7 @@ struct AllocParams {
   unsigned long long* sel;    // [nseg*3*3]: prefix, remaining (as u64), done
   unsigned long long* hist;   // [nseg*3*256]
   int32_t* counts;            // [U*3]
+  int32_t* ccounts;           // [U][chunks of kRowChunk positions][3]: tier counts per chunk
   int32_t* tbase;             // [U*3]
   long long* pinned;          // [B]: bytes of the tokens whose tier is fixed
   int nseg;
@@ -210,6 +211,7 @@ cudaError_t launch_merge_partials(int R, long long n, const float* out_parts,
                                   float* lse, cudaStream_t stream);
 cudaError_t launch_encode(const EncodeParams& p, cudaStream_t stream);
 cudaError_t launch_append(const AppendParams& p, cudaStream_t stream);
+constexpr int kRowChunk = 1024;  // positions per block of the count and row-map kernels
 size_t alloc_workspace_bytes(int B, int Hkv, long long Tmax);
 void alloc_carve(AllocParams& p, void* ws);
 cudaError_t launch_allocate(AllocParams& p, cudaStream_t stream);
