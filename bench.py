@@ -307,8 +307,11 @@ def run_skv(args, rank, world, local_rank):
 
     stream = torch.cuda.current_stream()
     ws = [c.workspace(w.Hq, S) for c in caches]
-    out = torch.empty((w.B, w.Hq, 128), dtype=torch.float32, device=dev)
-    lse = torch.empty((w.B, w.Hq), dtype=torch.float32, device=dev)
+    # out and lse in one buffer (lse right after out): the host step then
+    # returns both in one copy
+    nrow = w.B * w.Hq
+    res = torch.empty(nrow * 129, dtype=torch.float32, device=dev)
+    out, lse = res[:nrow * 128].view(w.B, w.Hq, 128), res[nrow * 128:].view(w.B, w.Hq)
 
     def make_step(c, wsp):
         def step(mid_event):
@@ -357,26 +360,29 @@ def run_skv(args, rank, world, local_rank):
     e2e = None
     if rank == 0 or world > 1:
         q_host = d["q"].cpu().pin_memory()
-        out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-        lse_host = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
-        scratch = (torch.empty_like(d["q"]), out, lse)
+        res_host = torch.empty(nrow * 129, dtype=torch.float32).pin_memory()
+        out_host = res_host[:nrow * 128].view(w.B, w.Hq, 128)
+        lse_host = res_host[nrow * 128:].view(w.B, w.Hq)
+        scratch = (torch.empty_like(d["q"]), res, None)   # packed: out then lse
         e2e_steps = max(10, min(args.steps, 2000))
         for i in range(5):
-            caches[i % 2].decode_host(q_host, d["q_dtype"], w.Hq, out_host, lse_host, scratch,
+            caches[i % 2].decode_host(q_host, d["q_dtype"], w.Hq, res_host, None, scratch,
                                       workspace=ws[i % 2], num_splits=S, stream=stream)
         ta = time.perf_counter()
         for i in range(e2e_steps):
-            caches[i % 2].decode_host(q_host, d["q_dtype"], w.Hq, out_host, lse_host, scratch,
+            caches[i % 2].decode_host(q_host, d["q_dtype"], w.Hq, res_host, None, scratch,
                                       workspace=ws[i % 2], num_splits=S, stream=stream)
         e2e_ms = (time.perf_counter() - ta) * 1e3 / e2e_steps
         caches[0].check()
+        breakdown = e2e_breakdown(caches, ws, d, w, q_host, res_host, res, out, lse, S, stream,
+                                  e2e_steps)
         e2e = {"value": world * resident / (e2e_ms * 1e-3), "unit": UNIT,
                "h2d_bytes_per_step": int(q_host.numel() * q_host.element_size()),
                "d2h_bytes_per_step": int(out_host.numel() * 4 + lse_host.numel() * 4 + 4),
-               "ms_per_step": e2e_ms, "steps": e2e_steps,
+               "ms_per_step": e2e_ms, "steps": e2e_steps, "breakdown": breakdown,
                "how": "skv_decode_attention_host every step: pinned host q -> device, the "
-                      "decode, out + lse + error word -> pinned host, stream sync, in one C-ABI "
-                      "call; host wall clock"}
+                      "decode, out + lse (packed, one copy) and the error word -> pinned host, "
+                      "stream sync, in one C-ABI call; host wall clock"}
 
     # ---- dense bf16 paged-decode baseline on the same K/V
     dense = None
@@ -601,6 +607,44 @@ def run_skv(args, rank, world, local_rank):
             "step_ms_graph_events": float(np.mean(step_ms)),
         }
         print(json.dumps(line), flush=True)
+
+
+def e2e_breakdown(caches, ws, d, w, q_host, res_host, res, out, lse, S, stream, steps):
+    """Where an end-to-end step's time goes.  Per round: an eager
+    device-buffer decode (decode + merge) between CUDA events; the result
+    copies alone (out + lse packed in one copy, the error word) between
+    events; and one skv_decode_attention_host call on the host wall clock.
+    The call's time beyond the two device parts is the q copy, host launch
+    and the stream-sync wake-up."""
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    scratch = (torch.empty_like(d["q"]), res, None)
+    err_host = torch.zeros(1, dtype=torch.int32).pin_memory()
+    dec = cop = wall = 0.0
+    n = max(10, min(steps, 500))
+    for i in range(n + 5):
+        c = caches[i % 2]
+        ev[0].record(stream)
+        c.decode(d["q"], d["q_dtype"], w.Hq, out=out, lse=lse, workspace=ws[i % 2], num_splits=S)
+        ev[1].record(stream)
+        res_host.copy_(res, non_blocking=True)
+        err_host.copy_(c.err, non_blocking=True)
+        ev[2].record(stream)
+        stream.synchronize()
+        ta = time.perf_counter()
+        c.decode_host(q_host, d["q_dtype"], w.Hq, res_host, None, scratch, workspace=ws[i % 2],
+                      num_splits=S, stream=stream)
+        tb = time.perf_counter()
+        if i >= 5:
+            wall += tb - ta
+            dec += ev[0].elapsed_time(ev[1])
+            cop += ev[1].elapsed_time(ev[2])
+    dec_us, cop_us, wall_us = dec / n * 1e3, cop / n * 1e3, wall / n * 1e6
+    return {"eager_decode_and_merge_us": dec_us, "result_copies_us": cop_us,
+            "call_wall_us": wall_us, "q_copy_launch_and_sync_us": wall_us - dec_us - cop_us,
+            "steps": n,
+            "how": "per round: an eager device-buffer decode between CUDA events, the result "
+                   "copies alone between events, and one skv_decode_attention_host call on the "
+                   "host wall clock; the rest = call - decode - copies"}
 
 
 def store_stats(cache):

@@ -353,7 +353,10 @@ int skv_decode_attention(skv_ctx* ctx, const void* q, int q_dtype, int B, int Hq
    out and lse back to out_host / lse_host, synchronises the stream and
    returns the device error word's verdict as skv_check does (and resets
    it).  Every copy is a single cudaMemcpyAsync on `stream`; use pinned
-   host buffers so that they are asynchronous DMA transfers.
+   host buffers so that they are asynchronous DMA transfers.  With lse_dev
+   and lse_host both NULL, lse lives right after out in the same buffers
+   (out_dev / out_host then hold B*Hq*129 floats: out, then lse) and one
+   copy returns both.
      q_host    [B][Hq][128] 16-bit host buffer (q_dtype as for the decode)
      q_dev     device buffer of the same size (caller-owned scratch)
      out_dev / lse_dev   device fp32 [B][Hq][128] / [B][Hq] scratch

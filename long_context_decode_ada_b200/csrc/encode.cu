@@ -47,13 +47,19 @@ __device__ __forceinline__ uint32_t half2_bits_to_bf16x2(uint32_t h) {
 }
 
 // b-bit angle sector of the pair (x, y) = (mx, my) 2^-24 (the fp16 values as
-// integers, half_bits_to_m); bx/by: the 2^b boundary vectors (fp32 values held
-// as doubles).  The sector depends only on the signs of the cross products
-// bx y - by x, unchanged by the positive scale 2^24; each product of a 24-bit
-// and an 11-bit significand is exact in fp64, and the difference is rounded
-// once, so its sign is exact.
-__device__ __forceinline__ uint32_t angle_code(long long mx, long long my, int b, const double* bx,
-                                               const double* by) {
+// integers, half_bits_to_m); bxy: the 2^b boundary vectors (fp32 values held
+// as doubles, (x, y) interleaved).  Within the point's quadrant q the code is
+// q 2^(b-2) + (the number of the quadrant's boundaries that the point is on
+// or counter-clockwise of): a prefix of them, since the side of boundary j,
+// sign(bx_j y - by_j x), falls from >= 0 to < 0 once.  Each product of a
+// 24-bit and an 11-bit significand is exact in fp64 and the difference is
+// rounded once, so every side is exact (and unchanged by the scale 2^24).
+// The count is first estimated from an fp32 arctangent of the point rotated
+// into quadrant 0 (error < 2e-3 rad, against sectors of at least pi/32 rad:
+// the estimate is off by at most one), then fixed by the exact sides of the
+// two boundaries around it.
+__device__ __forceinline__ uint32_t angle_code(long long mx, long long my, int b,
+                                               const double2* bxy) {
   const double x = (double)mx, y = (double)my;
   if (x == 0.0 && y == 0.0) return 0;
   int q;
@@ -63,15 +69,29 @@ __device__ __forceinline__ uint32_t angle_code(long long mx, long long my, int b
   else q = 3;
   const int per = 1 << (b - 2);
   const int base = q * per;
-  // count of boundaries j in [base, base + per) that the point is on or
-  // counter-clockwise of: a prefix of that range
-  int lo = 0, hi = per;
-  while (lo < hi) {
-    const int mid = (lo + hi) >> 1;
-    const double side = __dsub_rn(__dmul_rn(bx[base + mid], y), __dmul_rn(by[base + mid], x));
-    if (side >= 0.0) lo = mid + 1;
-    else hi = mid;
+  // (u, v): the point rotated by -q quarter turns, u > 0 and v >= 0
+  const float fx = (float)x, fy = (float)y;
+  const float u = q == 0 ? fx : (q == 1 ? fy : (q == 2 ? -fx : -fy));
+  const float v = q == 0 ? fy : (q == 1 ? -fx : (q == 2 ? -fy : fx));
+  const bool low = v <= u;
+  const float t = low ? __fdividef(v, u) : __fdividef(u, v);  // in [0, 1]
+  // atan(t) on [0, 1]: pi/4 t - t (t - 1)(0.2447 + 0.0663 t), |error| < 1.6e-3
+  const float at = t * (0.78539816f - (t - 1.0f) * (0.2447f + 0.0663f * t));
+  const float phi = low ? at : 1.57079633f - at;
+  int lo = (int)(phi * ((float)per * 0.63661977f) + 0.5f);  // boundaries at (j + 1/2) pi / (2 per)
+  lo = min(max(lo, 0), per);
+  // exact sides of the boundaries lo - 1 and lo: the true count is lo - 1,
+  // lo or lo + 1
+  bool below = false, above = false;
+  if (lo > 0) {
+    const double2 c = bxy[base + lo - 1];
+    below = __dsub_rn(__dmul_rn(c.x, y), __dmul_rn(c.y, x)) < 0.0;  // not yet past lo - 1
   }
+  if (lo < per) {
+    const double2 c = bxy[base + lo];
+    above = __dsub_rn(__dmul_rn(c.x, y), __dmul_rn(c.y, x)) >= 0.0;  // already past lo
+  }
+  lo += above ? 1 : (below ? -1 : 0);
   return (uint32_t)(base + lo) & (uint32_t)((1 << b) - 1);
 }
 
@@ -109,24 +129,17 @@ __device__ __forceinline__ int v_frag_offset(int row, int dd, int elem_bytes) {
 }
 
 // The boundary vectors of the three angle codes (fp32 values), in shared
-// memory as doubles: the angle search then converts nothing.
+// memory as doubles, (x, y) of a boundary in one 16-byte load.
 struct Boundaries {
-  double bx6[64], by6[64], bx4[16], by4[16], bx5[32], by5[32];
+  double2 b6[64], b4[16], b5[32];
 };
 
 template <class Prm>
 __device__ __forceinline__ void load_boundaries(const Prm& p, Boundaries& sb) {
   for (int i = threadIdx.x; i < 64; i += blockDim.x) {
-    sb.bx6[i] = p.bx6[i];
-    sb.by6[i] = p.by6[i];
-    if (i < 32) {
-      sb.bx5[i] = p.bx5[i];
-      sb.by5[i] = p.by5[i];
-    }
-    if (i < 16) {
-      sb.bx4[i] = p.bx4[i];
-      sb.by4[i] = p.by4[i];
-    }
+    sb.b6[i] = make_double2(p.bx6[i], p.by6[i]);
+    if (i < 32) sb.b5[i] = make_double2(p.bx5[i], p.by5[i]);
+    if (i < 16) sb.b4[i] = make_double2(p.bx4[i], p.by4[i]);
   }
 }
 
@@ -182,10 +195,9 @@ __device__ __forceinline__ void write_row(uint8_t* page, int P, int tr, int row,
   const bool t1 = tr == SKV_TIER_T1;
   const bool v53 = t1 && t1_scheme;  // T1 variant: 5-bit angle + 3-bit share
   const int bits = t1 ? (v53 ? 5 : 6) : 4;
-  const double* bx = t1 ? (v53 ? sb.bx5 : sb.bx6) : sb.bx4;
-  const double* by = t1 ? (v53 ? sb.by5 : sb.by6) : sb.by4;
-  const uint32_t th0 = angle_code(m[0], m[1], bits, bx, by);
-  const uint32_t th1 = angle_code(m[2], m[3], bits, bx, by);
+  const double2* bxy = t1 ? (v53 ? sb.b5 : sb.b6) : sb.b4;
+  const uint32_t th0 = angle_code(m[0], m[1], bits, bxy);
+  const uint32_t th1 = angle_code(m[2], m[3], bits, bxy);
   const uint32_t rh0 = v53 ? rho_code3(m[0], m[1], R2) : rho_code(m[0], m[1], R2, share_grid);
   const uint32_t rh1 = v53 ? rho_code3(m[2], m[3], R2) : rho_code(m[2], m[3], R2, share_grid);
   const uint32_t packed = th0 | (th1 << 8) | (rh0 << 16) | (rh1 << 24);

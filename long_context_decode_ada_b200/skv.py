@@ -424,20 +424,25 @@ class PagedCache:
         """One decode step from host q to host out / lse (skv_decode_attention_host):
         the copies, the decode and the stream synchronisation in one call.
         scratch = (q_dev, out_dev, lse_dev) device tensors; host tensors
-        should be pinned."""
+        should be pinned.  With lse_host and lse_dev None, out_host / out_dev
+        hold B*Hq*129 floats, out then lse, and one copy returns both."""
         q_dev, out_dev, lse_dev = scratch
+        packed = lse_host is None and lse_dev is None
         for t, dev_side in ((q_host, False), (out_host, False), (lse_host, False),
                             (q_dev, True), (out_dev, True), (lse_dev, True)):
-            if t.is_cuda != dev_side or not t.is_contiguous():
+            if t is None and packed:
+                continue
+            if t is None or t.is_cuda != dev_side or not t.is_contiguous():
                 raise SkvError(SKV_ERR_ARG, "decode_host: host tensors on the host, scratch on "
                                             "the device, all contiguous")
         n = self.B * Hq * self.ctx.d
         for t, name in ((q_host, "q_host"), (q_dev, "q_dev")):
             _expect(t, name, n, 2, cuda=False)
         for t, name in ((out_host, "out_host"), (out_dev, "out_dev")):
-            _expect(t, name, n, 4, torch.float32, cuda=False)
-        for t, name in ((lse_host, "lse_host"), (lse_dev, "lse_dev")):
-            _expect(t, name, self.B * Hq, 4, torch.float32, cuda=False)
+            _expect(t, name, n + (self.B * Hq if packed else 0), 4, torch.float32, cuda=False)
+        if not packed:
+            for t, name in ((lse_host, "lse_host"), (lse_dev, "lse_dev")):
+                _expect(t, name, self.B * Hq, 4, torch.float32, cuda=False)
         if workspace is None:
             workspace = self.workspace(Hq, num_splits)
         _check(lib().skv_decode_attention_host(
