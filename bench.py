@@ -56,6 +56,8 @@ def parse_args():
     ap.add_argument("--no-append", action="store_true", help="skip the skv_append timing")
     ap.add_argument("--no-t0-bf16", action="store_true",
                     help="skip the fused T0 / bf16 variant's timing")
+    ap.add_argument("--no-retier", action="store_true",
+                    help="skip the skv_retier timing (it follows the append leg)")
     ap.add_argument("--no-utility", action="store_true",
                     help="skip the skv_decode_utility timing")
     ap.add_argument("--cp", action="store_true",
@@ -276,9 +278,14 @@ def run_skv(args, rank, world, local_rank):
     ctx = skv.Context(w.P)
     d = skv.workload_to_device(w, dev)
 
-    # ---- ingest: allocate + encode (off the decode path; timed for context)
+    # ---- ingest: allocate + encode (off the decode path; timed for context,
+    # warm: the first pass loads the kernels' modules)
     e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
     cache = skv.PagedCache(ctx, w.B, w.Hkv, w.Tmax, w.pool_slots, device=dev)
+    cache.allocate(d["K"], d["seq_lens"], d["utility"], d["protect"], w.mode, d["budget"],
+                   d["quota"], d["free_lists"])
+    cache.encode(d["K"], d["V"], d["seq_lens"])
+    torch.cuda.synchronize()
     e0.record()
     cache.allocate(d["K"], d["seq_lens"], d["utility"], d["protect"], w.mode, d["budget"],
                    d["quota"], d["free_lists"])
@@ -525,12 +532,16 @@ def run_skv(args, rank, world, local_rank):
     # ---- decode-time append (skv_append) on the same recipe: a store built
     # n_app tokens short, then n_app appends timed one after another
     append = None
+    retier = None
     if not args.no_append:
         import dataclasses
         n_app = 64
         wa = dataclasses.replace(w, seq_lens=(w.seq_lens - n_app).astype(np.int32))
         slots = list(w.pool_slots)
         slots[0] += w.B * w.Hkv * (n_app // w.P + 2)
+        # room for the re-tiering's rewritten pages (the window's T0 pages from
+        # the first demoted row on, the last T1 / T2 pages and new ones)
+        slots = [x + w.B * w.Hkv * (1024 // w.P + 4) for x in slots]
         wa = dataclasses.replace(wa, pool_slots=slots,
                                  free_lists=[np.arange(x, dtype=np.uint32) for x in slots])
         da = skv.workload_to_device(wa, dev)
@@ -552,6 +563,39 @@ def run_skv(args, rank, world, local_rank):
                   "how": "skv_append of one token per sequence and kv head, eager launches "
                          "(4 kernels each; pages are added every P steps), CUDA events "
                          "around the steps"}
+        # ---- the window roll that follows: the oldest n_app - 1 rows of the
+        # protected recent window re-tiered under the budget grown with the
+        # appended tokens (skv_retier), on the store the appends left
+        if not args.no_retier:
+            lo = T - 1024
+            demote = torch.zeros((w.B, w.Hkv, w.Tmax), dtype=torch.uint8, device=dev)
+            demote[:, :, lo:lo + n_app - 1] = 1
+            budget = da["budget"] + int(0.4 * n_app * w.Hkv * 512)
+            # warm-up: a re-tiering with nothing demoted (and room in the
+            # budget) changes no byte, and loads the kernels' modules
+            ca.retier(da["utility"], torch.zeros_like(demote), 2 * budget, seq_a)
+            torch.cuda.synchronize()
+            ca.check()
+            before = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            n_pages0 = int(ca.page_indptr[-1])
+            cur0 = ca.free_cursor().clone()
+            before[0].record()
+            released, n_rel = ca.retier(da["utility"], demote, budget, seq_a)
+            before[1].record()
+            torch.cuda.synchronize()
+            ca.check()
+            new_t = ca.tier[:, :, lo:lo + n_app - 1].flatten().to(torch.int64)
+            retier = {"us": before[0].elapsed_time(before[1]) * 1e3,
+                      "rows_demoted": int(w.B * w.Hkv * (n_app - 1)),
+                      "demoted_to": {k: int((new_t == i).sum()) for i, k in
+                                     enumerate(("T0", "T1", "T2", "dropped"))},
+                      "pages_before": n_pages0, "pages_after": int(ca.page_indptr[-1]),
+                      "pages_rewritten": int((ca.free_cursor() - cur0).sum()),
+                      "pages_released": int(n_rel.item()),
+                      "how": "skv_retier of the window's oldest rows after the appends, one "
+                             "eager call (snapshot copies, key, select, tier, count, row-map, "
+                             "diff, plan, page-write, release and transcode kernels), CUDA "
+                             "events around it"}
         del ca, da
 
     configs = None
@@ -602,6 +646,7 @@ def run_skv(args, rank, world, local_rank):
             "t0_bf16_variant": t0b,
             "ingest": {"allocate_ms": alloc_ms, "encode_ms": enc_ms, "gen_s": t_gen},
             "append": append,
+            "retier": retier,
             "utility": utility,
             "configs": configs,
             "step_ms_graph_events": float(np.mean(step_ms)),

@@ -290,7 +290,8 @@ int skv_append(skv_ctx* ctx, const uint16_t* K_new, const uint16_t* V_new, int B
    exceed a sequence's budget (its demoted rows are then dropped; the store
    stays consistent); SKV_ERR_POOL (free list or page capacity exhausted)
    and SKV_ERR_CORRUPT (a bad page id or row) leave the store invalid: it
-   must be rebuilt with skv_allocate + skv_encode.  Budget mode only; no
+   must be rebuilt with skv_allocate + skv_encode.  B * Hkv * Tmax must be
+   below 2^32 (SKV_ERR_ARG otherwise).  Budget mode only; no
    outlier protection is applied to the demoted rows (leave such rows out of
    `demote`). */
 int skv_retier_workspace_size(const skv_ctx* ctx, int B, int Hkv, int64_t Tmax,

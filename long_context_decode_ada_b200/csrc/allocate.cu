@@ -164,47 +164,64 @@ __global__ void __launch_bounds__(256) keys_budget_kernel(const __grid_constant_
   if (lane == 0) p.keyw[w] = __fmul_rn(valid_utility(p, w), r2f);
 }
 
-// re-tiering: a demoted token (T0 in the old store) gets the budget key from
-// the fp16 key in its old T0 page (its row order does not matter for r^2);
-// every other resident token keeps its old tier.
-__global__ void __launch_bounds__(256) keys_retier_kernel(const __grid_constant__ AllocParams p) {
-  const long long w = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (w >= (long long)p.B * p.Hkv * p.Tmax) return;
-  const long long t = w % p.Tmax;
-  const long long u = w / p.Tmax;
-  const int b = (int)(u / p.Hkv);
-  if (t >= p.seq_lens[b]) return;
-  const int to = p.tier_old[w];
-  if (to > SKV_TIER_DROP) {
-    if (lane == 0) {
+// re-tiering, one thread per (unit, position): a demoted token (T0 in the
+// old store) gets the budget key from the fp16 key in its old T0 page (the
+// row's component order does not matter for r^2: the sum is exact); every
+// other resident token keeps its old tier (key -1 - tier) and its bytes are
+// summed per block, one atomic per block (a block holds positions of one
+// unit).  Demoted rows are few, so one thread computes a whole key's norm.
+__global__ void __launch_bounds__(256) keys_retier_kernel(const __grid_constant__ AllocParams p,
+                                                          unsigned nbx) {
+  __shared__ unsigned long long sum;
+  if (threadIdx.x == 0) sum = 0;
+  __syncthreads();
+  const unsigned u = blockIdx.x / nbx;
+  const long long t = (long long)(blockIdx.x - u * nbx) * blockDim.x + threadIdx.x;
+  const int b = (int)(u / (unsigned)p.Hkv);
+  unsigned long long bytes = 0;
+  if (t < p.Tmax && t < p.seq_lens[b]) {
+    const long long w = (long long)u * p.Tmax + t;
+    const int to = p.tier_old[w];
+    if (to > SKV_TIER_DROP) {
       report(p.err, SKV_ERR_CORRUPT);
-      pin_token(p, w, b, SKV_TIER_DROP);
-    }
-    return;
-  }
-  if (!p.demote[w] || to != SKV_TIER_T0) {
-    if (lane == 0) {
+      p.keyw[w] = -1.0f - (float)SKV_TIER_DROP;
+    } else if (!p.demote[w] || to != SKV_TIER_T0) {
       if (p.demote[w]) report(p.err, SKV_ERR_ARG);  // only T0 rows can be demoted
-      pin_token(p, w, b, to);
+      p.keyw[w] = -1.0f - (float)to;
+      bytes = to < SKV_TIER_DROP ? (unsigned long long)tier_row_bytes(to) : 0ull;
+    } else {
+      const int row = p.row_old[w];
+      const long long gi = (long long)p.indptr_old[u] + (row >= 0 ? row / p.P : 0);
+      const uint32_t id = row >= 0 && gi < p.tindptr_old[3 * u + 1] && gi < p.page_cap
+                              ? p.ids_old[gi] : 0xFFFFFFFFu;
+      const uint32_t slot = id & 0x3FFFFFFFu;
+      if ((id >> 30) != 0u || (long long)slot >= p.slots[0]) {
+        report(p.err, SKV_ERR_CORRUPT);
+        p.keyw[w] = -1.0f - (float)SKV_TIER_DROP;
+      } else {
+        const uint4* krow = reinterpret_cast<const uint4*>(
+            p.pool[0] + (long long)slot * p.stride[0] + kHdrBytes + 256 * (row % p.P));
+        u128 sq = 0;
+        for (int c = 0; c < 16; ++c) {
+          const uint4 v = krow[c];
+          const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const long long m = half_bits_to_m((wd[k >> 1] >> (16 * (k & 1))) & 0xFFFFu);
+            const u128 a = (u128)(m < 0 ? -m : m);
+            sq += a * a;
+          }
+        }
+        const double r2 = u128_to_double_rn((unsigned long long)(sq >> 64), (unsigned long long)sq);
+        const float r2f = __double2float_rn(__dmul_rn(r2, 3.552713678800501e-15));  // 2^-48
+        p.keyw[w] = __fmul_rn(valid_utility(p, w), r2f);
+      }
     }
-    return;
   }
-  const int row = p.row_old[w];
-  const long long gi = (long long)p.indptr_old[u] + (row >= 0 ? row / p.P : 0);
-  const uint32_t id =
-      row >= 0 && gi < p.tindptr_old[3 * u + 1] && gi < p.page_cap ? p.ids_old[gi] : 0xFFFFFFFFu;
-  const uint32_t slot = id & 0x3FFFFFFFu;
-  if ((id >> 30) != 0u || (long long)slot >= p.slots[0]) {
-    if (lane == 0) {
-      report(p.err, SKV_ERR_CORRUPT);
-      pin_token(p, w, b, SKV_TIER_DROP);
-    }
-    return;
-  }
-  const uint8_t* krow = p.pool[0] + (long long)slot * p.stride[0] + kHdrBytes + 256 * (row % p.P);
-  const float r2f = warp_r2f(*reinterpret_cast<const uint2*>(krow + 8 * lane));
-  if (lane == 0) p.keyw[w] = __fmul_rn(valid_utility(p, w), r2f);
+  if (bytes) atomicAdd(&sum, bytes);
+  __syncthreads();
+  if (threadIdx.x == 0 && sum)
+    atomicAdd(reinterpret_cast<unsigned long long*>(&p.pinned[b]), sum);
 }
 
 // quota mode: keyw = u (0 without utilities), -1 when protected
@@ -796,7 +813,11 @@ cudaError_t launch_retier_plan(AllocParams& p, cudaStream_t stream) {
   if ((e = cudaMemsetAsync(p.hist, 0, 8 * (size_t)p.nseg * 3 * 256, stream)) != cudaSuccess)
     return e;
   if ((e = cudaMemsetAsync(p.diff, 0x7F, 4 * 3 * (size_t)U, stream)) != cudaSuccess) return e;
-  if (ntok > 0) keys_retier_kernel<<<grid_for(ntok * 32, 256), 256, 0, stream>>>(p);
+  if (ntok > 0) {
+    const long long nbx = (p.Tmax + 255) / 256;
+    if ((long long)U * nbx > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
+    keys_retier_kernel<<<(unsigned)(U * nbx), 256, 0, stream>>>(p, (unsigned)nbx);
+  }
   sel_init_kernel<<<grid_for(p.nseg * 3, 128), 128, 0, stream>>>(p);
   const dim3 hgrid(grid_for((long long)p.Hkv * p.Tmax, kHistItemsPerBlock), p.nseg);
   for (int pass = 0; pass < 8; ++pass) {

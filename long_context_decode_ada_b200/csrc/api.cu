@@ -479,6 +479,8 @@ int skv_retier(skv_ctx* ctx, int B, int Hkv, int64_t Tmax, const int32_t* seq_le
       page_cap > 0x7FFFFFFFLL)
     return fail(SKV_ERR_ARG, "skv_retier: need B >= 0, 0 < Hkv <= 128, 0 <= Tmax <= 2^23");
   if ((long long)B * Hkv > (1 << 24)) return fail(SKV_ERR_ARG, "skv_retier: too many units");
+  if ((long long)B * Hkv * Tmax > 0xFFFFFFFFLL)  // rows to rewrite are listed by 32-bit index
+    return fail(SKV_ERR_ARG, "skv_retier: B * Hkv * Tmax must be below 2^32");
   if (!seq_lens || !utility || !demote || !budget || !free || !free_cursor || !tier ||
       !row_of || !page_indptr || !page_tier_indptr || !released || !n_released || !err_word)
     return fail(SKV_ERR_ARG, "skv_retier: null argument");
@@ -544,6 +546,9 @@ int skv_retier(skv_ctx* ctx, int B, int Hkv, int64_t Tmax, const int32_t* seq_le
     tp.stride[t] = p.stride[t];
   }
   tp.err = err_word;
+  // the key array and the histogram are free once the tiers are decided
+  tp.list = reinterpret_cast<uint32_t*>(p.keyw);
+  tp.count = p.hist;
   std::memcpy(tp.bx6, ctx->bx6, sizeof(tp.bx6));
   std::memcpy(tp.by6, ctx->by6, sizeof(tp.by6));
   std::memcpy(tp.bx4, ctx->bx4, sizeof(tp.bx4));

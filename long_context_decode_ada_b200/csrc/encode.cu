@@ -350,60 +350,93 @@ __device__ __forceinline__ uint8_t* row_page(const TranscodeParams& p, const int
   return p.pool[tr] + (long long)slot * p.stride[tr];
 }
 
+// First pass, one thread per (unit, position): the resident rows that lie in
+// rewritten pages (at or after their segment's first change) go to a list
+// (one atomic per warp).  Most rows are in kept pages, so the second pass
+// runs over few rows.
+__global__ void __launch_bounds__(256) transcode_list_kernel(const __grid_constant__ TranscodeParams p,
+                                                             unsigned nbx) {
+  const unsigned u = blockIdx.x / nbx;
+  const long long t = (long long)(blockIdx.x - u * nbx) * blockDim.x + threadIdx.x;
+  bool need = false;
+  long long w = 0;
+  if (t < p.Tmax && t < p.seq_lens[u / (unsigned)p.Hkv]) {
+    w = (long long)u * p.Tmax + t;
+    const int tn = p.tier[w];
+    if (tn < SKV_TIER_DROP) {
+      const int rn = p.row_of[w];
+      need = rn < 0 ||
+             rn / p.P - (p.tier_indptr[3 * u + tn] - p.indptr[u]) >= p.keep[3 * u + tn];
+    }
+  }
+  const unsigned mask = __ballot_sync(0xFFFFFFFFu, need);
+  if (!mask) return;
+  const int lane = threadIdx.x & 31, leader = __ffs(mask) - 1;
+  unsigned long long base = 0;
+  if (lane == leader) base = atomicAdd(p.count, (unsigned long long)__popc(mask));
+  base = __shfl_sync(0xFFFFFFFFu, base, leader);
+  if (need) p.list[base + __popc(mask & ((1u << lane) - 1))] = (uint32_t)w;
+}
+
+// Second pass, a warp per listed row (a grid-stride loop): its old row is
+// either T0 -- the exact fp16 K and V, read back from the old page in the T0
+// row order and written (T0) or encoded (T1 / T2) as the encode does from
+// dense inputs -- or T1 / T2 of the same tier, whose radius, code row, scale
+// and int8 V are copied (the V fragment order depends on the row index).
 __global__ void __launch_bounds__(256) transcode_kernel(const __grid_constant__ TranscodeParams p) {
   __shared__ Boundaries sb;
   load_boundaries(p, sb);
   __syncthreads();
-  const long long w = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
-  if (w >= (long long)p.B * p.Hkv * p.Tmax) return;
-  const long long t = w % p.Tmax, u = w / p.Tmax;
-  if (t >= p.seq_lens[u / p.Hkv]) return;
-  const int tn = p.tier[w];
-  if (tn >= SKV_TIER_DROP) return;
-  const int rn = p.row_of[w], P = p.P;
-  // rows of a kept page (before its segment's first change) are in place
-  if (rn >= 0 && rn / P - (p.tier_indptr[3 * u + tn] - p.indptr[u]) < p.keep[3 * u + tn]) return;
-  const int to = p.tier_old[w], ro = to < SKV_TIER_DROP ? p.row_old[w] : -1;
-  uint8_t* dst = row_page(p, p.indptr, p.ids, u, tn, rn);
-  const uint8_t* src = to < SKV_TIER_DROP ? row_page(p, p.indptr_old, p.ids_old, u, to, ro)
-                                          : nullptr;
-  if (!dst || !src || (to != SKV_TIER_T0 && to != tn)) {
-    if (lane == 0) report(p.err, SKV_ERR_CORRUPT);
-    return;
-  }
-  const int r_new = rn % P, r_old = ro % P;
-  if (to == SKV_TIER_T0) {
-    const int c = lane >> 1;
-    const uint2 kv = *reinterpret_cast<const uint2*>(src + kHdrBytes + r_old * 256 +
-                                                     (c ^ (4 * (r_old & 1))) * 16 + (lane & 1) * 8);
-    const uint8_t* vsec = src + kHdrBytes + 256 * P;
-    uint16_t k4[4] = {(uint16_t)(kv.x & 0xFFFF), (uint16_t)(kv.x >> 16),
-                      (uint16_t)(kv.y & 0xFFFF), (uint16_t)(kv.y >> 16)};
-    uint16_t v4[4];
+  const long long n = (long long)*p.count;
+  const long long nwarps = (long long)gridDim.x * (blockDim.x >> 5);
+  for (long long i = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5; i < n; i += nwarps) {
+    const long long w = p.list[i];
+    const long long u = w / p.Tmax;
+    const int tn = p.tier[w];
+    const int rn = p.row_of[w], P = p.P;
+    const int to = p.tier_old[w], ro = to < SKV_TIER_DROP ? p.row_old[w] : -1;
+    uint8_t* dst = row_page(p, p.indptr, p.ids, u, tn, rn);
+    const uint8_t* src = to < SKV_TIER_DROP ? row_page(p, p.indptr_old, p.ids_old, u, to, ro)
+                                            : nullptr;
+    if (!dst || !src || (to != SKV_TIER_T0 && to != tn)) {
+      if (lane == 0) report(p.err, SKV_ERR_CORRUPT);
+      continue;
+    }
+    const int r_new = rn % P, r_old = ro % P;
+    if (to == SKV_TIER_T0) {
+      const int c = lane >> 1;
+      const uint2 kv = *reinterpret_cast<const uint2*>(
+          src + kHdrBytes + r_old * 256 + (c ^ (4 * (r_old & 1))) * 16 + (lane & 1) * 8);
+      const uint8_t* vsec = src + kHdrBytes + 256 * P;
+      uint16_t k4[4] = {(uint16_t)(kv.x & 0xFFFF), (uint16_t)(kv.x >> 16),
+                        (uint16_t)(kv.y & 0xFFFF), (uint16_t)(kv.y >> 16)};
+      uint16_t v4[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-      v4[i] = *reinterpret_cast<const uint16_t*>(vsec + v_frag_offset(r_old, 4 * lane + i, 2));
-    write_row(dst, P, tn, r_new, lane, k4, v4, false, p.t1_scheme, p.share_grid, sb);
-    return;
-  }
-  // T1 / T2 row: r~ (fp16 [P]), codes ([P][cb]), scale (fp16 [P]), int8 V
-  const int cb = tn == SKV_TIER_T1 ? 64 : 48;
-  const uint8_t* rs = src + kHdrBytes;
-  uint8_t* rd = dst + kHdrBytes;
-  if (lane == 0) {
-    *reinterpret_cast<uint16_t*>(rd + 2 * r_new) = *reinterpret_cast<const uint16_t*>(rs + 2 * r_old);
-    *reinterpret_cast<uint16_t*>(rd + (2 + cb) * P + 2 * r_new) =
-        *reinterpret_cast<const uint16_t*>(rs + (2 + cb) * P + 2 * r_old);
-  }
-  if (lane < cb / 4)
-    *reinterpret_cast<uint32_t*>(rd + 2 * P + cb * r_new + 4 * lane) =
-        *reinterpret_cast<const uint32_t*>(rs + 2 * P + cb * r_old + 4 * lane);
-  const uint8_t* vs = rs + (4 + cb) * P;
-  uint8_t* vd = rd + (4 + cb) * P;
+      for (int k = 0; k < 4; ++k)
+        v4[k] = *reinterpret_cast<const uint16_t*>(vsec + v_frag_offset(r_old, 4 * lane + k, 2));
+      write_row(dst, P, tn, r_new, lane, k4, v4, false, p.t1_scheme, p.share_grid, sb);
+      continue;
+    }
+    // T1 / T2 row: r~ (fp16 [P]), codes ([P][cb]), scale (fp16 [P]), int8 V
+    const int cb = tn == SKV_TIER_T1 ? 64 : 48;
+    const uint8_t* rs = src + kHdrBytes;
+    uint8_t* rd = dst + kHdrBytes;
+    if (lane == 0) {
+      *reinterpret_cast<uint16_t*>(rd + 2 * r_new) =
+          *reinterpret_cast<const uint16_t*>(rs + 2 * r_old);
+      *reinterpret_cast<uint16_t*>(rd + (2 + cb) * P + 2 * r_new) =
+          *reinterpret_cast<const uint16_t*>(rs + (2 + cb) * P + 2 * r_old);
+    }
+    if (lane < cb / 4)
+      *reinterpret_cast<uint32_t*>(rd + 2 * P + cb * r_new + 4 * lane) =
+          *reinterpret_cast<const uint32_t*>(rs + 2 * P + cb * r_old + 4 * lane);
+    const uint8_t* vs = rs + (4 + cb) * P;
+    uint8_t* vd = rd + (4 + cb) * P;
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
-    vd[v_frag_offset(r_new, 4 * lane + i, 1)] = vs[v_frag_offset(r_old, 4 * lane + i, 1)];
+    for (int k = 0; k < 4; ++k)
+      vd[v_frag_offset(r_new, 4 * lane + k, 1)] = vs[v_frag_offset(r_old, 4 * lane + k, 1)];
+  }
 }
 
 // ------------------------------------------------------------------ append
@@ -636,9 +669,15 @@ cudaError_t launch_append(const AppendParams& p, cudaStream_t stream) {
 }
 
 cudaError_t launch_transcode(const TranscodeParams& p, cudaStream_t stream) {
-  const long long warps = (long long)p.B * p.Hkv * p.Tmax;
-  if (warps == 0) return cudaSuccess;
-  transcode_kernel<<<(unsigned)((warps * 32 + 255) / 256), 256, 0, stream>>>(p);
+  const long long U = (long long)p.B * p.Hkv;
+  if (U == 0 || p.Tmax == 0) return cudaSuccess;
+  const long long nbx = (p.Tmax + 255) / 256;
+  if (U * nbx > 0x7FFFFFFFLL || U * p.Tmax > 0xFFFFFFFFLL) return cudaErrorInvalidValue;
+  cudaError_t e = cudaMemsetAsync(p.count, 0, sizeof(unsigned long long), stream);
+  if (e != cudaSuccess) return e;
+  transcode_list_kernel<<<(unsigned)(U * nbx), 256, 0, stream>>>(p, (unsigned)nbx);
+  // a few resident blocks per SM loop over the listed rows
+  transcode_kernel<<<148 * 4, 256, 0, stream>>>(p);
   return cudaGetLastError();
 }
 

@@ -244,6 +244,8 @@ struct TranscodeParams {
   long long slots[3];
   long long stride[3];
   int32_t* err;
+  uint32_t* list;             // workspace: flat indices of the rows to write
+  unsigned long long* count;  // workspace: their number
   float bx6[64], by6[64], bx4[16], by4[16];
   float bx5[32], by5[32];
   int t1_scheme;

@@ -73,3 +73,65 @@ def test_pipeline_layer_full_size(layer):
     g, ref, npages = full_size_check(w, nrows=16 if layer not in (0, 31) else 24, seed=5 + layer)
     counts = np.bincount(ref["tier"].ravel(), minlength=4)
     assert counts[1] and counts[2] and counts[3]
+
+
+def test_long_context_window_roll_full_size():
+    """The 128K store built 64 tokens short, 64 decode-time appends, then
+    skv_retier of the protected window's oldest 63 rows under the budget
+    grown with the appended tokens (the bench's window roll): tiers and row
+    map bit-exact against the oracle's re-tiering, every unit's page bytes in
+    list order against the oracle's pack of those tiers, and sampled rows of
+    the decode against the oracle."""
+    import dataclasses
+
+    import torch
+
+    from long_context_decode_ada_b200 import skv
+    from test_gpu_append import page_bytes
+
+    w = wl.long_context()
+    T, n_app = int(w.seq_lens[0]), 64
+    slots = [x + w.B * w.Hkv * (1024 // w.P + 4) for x in w.pool_slots]
+    slots[0] += w.B * w.Hkv * (n_app // w.P + 2)
+    free = [np.arange(x, dtype=np.uint32) for x in slots]
+    wa = dataclasses.replace(w, seq_lens=(w.seq_lens - n_app).astype(np.int32), pool_slots=slots,
+                             free_lists=free)
+    ctx = skv.Context(w.P)
+    da = skv.workload_to_device(wa)
+    ca = skv.build_cache(ctx, wa, da)
+    ca.check()
+    seq = da["seq_lens"].clone()
+    for i in range(n_app):
+        ca.append(da["K"][:, :, T - n_app + i].contiguous(), da["V"][:, :, T - n_app + i].contiguous(),
+                  seq)
+    ca.check()
+    tier = oracle.allocate(w.B, w.Hkv, w.Tmax, w.d, w.P, wa.seq_lens, w.K, w.utility, w.protect,
+                           w.mode, w.budget, w.quota)
+    tier[:, :, T - n_app:T] = 0
+    assert np.array_equal(ca.tier.cpu().numpy(), tier), "tiers after the appends"
+    lo = T - 1024
+    demote = np.zeros_like(tier)
+    demote[:, :, lo:lo + n_app - 1] = 1
+    budget = (w.budget + int(0.4 * n_app * w.Hkv * 512)).astype(np.int64)
+    exp = oracle.retier(w.B, w.Hkv, w.Tmax, w.d, w.P, w.seq_lens, w.K, w.utility, tier, demote,
+                        budget)
+    ca.retier(da["utility"], torch.from_numpy(demote).cuda(), torch.from_numpy(budget).cuda(), seq)
+    ca.check()
+    assert np.array_equal(ca.tier.cpu().numpy(), exp), "tiers after the re-tiering"
+    assert np.any(exp[demote == 1] != 0), "some demoted rows leave T0"
+    ref = oracle.pack(w.B, w.Hkv, w.Tmax, w.d, w.P, w.seq_lens, w.K, w.V, exp, free, slots)
+    assert np.array_equal(ca.row_of.cpu().numpy(), ref["row_of"]), "row map"
+    ip = ca.page_indptr.cpu().numpy()
+    assert np.array_equal(ip, ref["page_indptr"]), "page_indptr"
+    ids = ca.page_ids[:ip[-1]].cpu().numpy().view(np.uint32)
+    got = page_bytes(ids, ip, [p.cpu().numpy() for p in ca.pools], w.P)
+    want = page_bytes(np.asarray(ref["page_ids"], np.uint32), ip, ref["pools"], w.P)
+    assert got == want, "page bytes"
+    out, lse = ca.decode(da["q"], da["q_dtype"], w.Hq)
+    ca.check()
+    rows = sample_rows(w, 16, 41)
+    ro, rl = oracle.decode(w.B, w.Hq, w.Hkv, w.Tmax, w.d, w.seq_lens, w.K, w.V, exp, w.q,
+                           w.q_dtype, units=rows)
+    b, h = rows[:, 0], rows[:, 1]
+    assert_close(out.cpu().numpy()[b, h], ro[b, h], "out (sampled rows)")
+    assert_close(lse.cpu().numpy()[b, h], rl[b, h], "lse (sampled rows)")
