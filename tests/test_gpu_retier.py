@@ -158,6 +158,7 @@ def check_pages_in_place(before, after, released, P):
     (41, 2, 2, 16, 600, 40, 64, 0.3),
     (42, 1, 4, 64, 2100, 70, 256, 0.25),
     (43, 3, 1, 16, 500, 33, 48, 0.9),   # a generous budget: demoted rows stay T0 too
+    (48, 2, 2, 32, 900, 50, 64, 0.2),  # P = 32 and a tight budget: T2 pages, dropped rows
 ])
 def test_retier_after_appends_matches_the_oracle(seed, B, Hkv, P, T, A, recent, frac):
     win = Window(seed, B, Hkv, P, T, A, recent, frac)
@@ -173,6 +174,8 @@ def test_retier_after_appends_matches_the_oracle(seed, B, Hkv, P, T, A, recent, 
     d = win.tier[:, :, t0 - recent:t0 - recent + A]
     if frac < 0.5:
         assert np.any(d == 3) and np.any((d == 1) | (d == 2)), "demoted rows coded and dropped"
+    if frac <= 0.2:
+        assert np.any(win.tier == 2), "the store holds T2 pages"
 
 
 def test_two_window_cycles():

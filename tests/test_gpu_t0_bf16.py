@@ -27,22 +27,23 @@ pytestmark = pytest.mark.gpu
 
 def t0_bound(w, tier, lse):
     """2^-9 sum_{t in T0} w_t |v_t| per (b, hq, dim), w_t = exp(l_t - lse)."""
-    Kb = w.K.to(torch.bfloat16).double().numpy()
-    Vb = w.V.to(torch.bfloat16).double().numpy()
     q = (w.q.view(torch.int16).view(torch.bfloat16).double() if w.q_dtype == "bf16"
          else w.q.view(torch.float16).double()).numpy()
     G = w.Hq // w.Hkv
     out = np.zeros((w.B, w.Hq, 128))
     for b in range(w.B):
         T = int(w.seq_lens[b])
-        for hq in range(w.Hq):
-            h = hq // G
-            sel = np.nonzero(tier[b, h, :T] == 0)[0]
-            if sel.size == 0 or not np.isfinite(lse[b, hq]):
+        for h in range(w.Hkv):
+            sel = torch.from_numpy(np.nonzero(tier[b, h, :T] == 0)[0])
+            if sel.numel() == 0:
                 continue
-            l = Kb[b, h, sel] @ q[b, hq] / np.sqrt(128)
-            wt = np.exp(l - lse[b, hq])
-            out[b, hq] = 2.0 ** -9 * (wt[:, None] * np.abs(Vb[b, h, sel])).sum(0)
+            Kb = w.K[b, h, sel].to(torch.bfloat16).double().numpy()
+            Vb = np.abs(w.V[b, h, sel].to(torch.bfloat16).double().numpy())
+            for hq in range(h * G, (h + 1) * G):
+                if not np.isfinite(lse[b, hq]):
+                    continue
+                wt = np.exp(Kb @ q[b, hq] / np.sqrt(128) - lse[b, hq])
+                out[b, hq] = 2.0 ** -9 * (wt[:, None] * Vb).sum(0)
     return out
 
 
@@ -162,3 +163,27 @@ def test_retier_and_variant_combinations_are_refused():
     with pytest.raises(skv.SkvError) as e:
         cache.retier(dev["utility"], demote, dev["budget"], dev["seq_lens"])
     assert e.value.code == skv.SKV_ERR_ARG
+
+
+def test_long_context_store_full_size():
+    """The 128K store with bf16 T0 pages (the bench's fused-path variant):
+    tiers, row map, page tables and every page's bytes bit-exact against the
+    oracle's bf16 T0 pack; sampled rows of the decode against the oracle
+    within the bound above."""
+    from test_gpu_fullsize import sample_rows
+    w = wl.long_context()
+    ctx = skv.Context(w.P, t0_bf16=True)
+    dev = skv.workload_to_device(w)
+    cache = skv.build_cache(ctx, w, dev)
+    cache.check()
+    with oracle.t0_bf16():
+        ref = oracle.run_workload(w, do_decode=False)
+        compare_store(w, dict(cache=cache), ref)
+        rows = sample_rows(w, 16, 77)
+        ro, rl = oracle.decode(w.B, w.Hq, w.Hkv, w.Tmax, w.d, w.seq_lens, w.K, w.V, ref["tier"],
+                               w.q, w.q_dtype, units=rows)
+    out, lse = cache.decode(dev["q"], dev["q_dtype"], w.Hq)
+    cache.check()
+    b, h = rows[:, 0], rows[:, 1]
+    bound = t0_bound(w, ref["tier"], rl)[b, h]
+    check_decode(out.cpu().numpy()[b, h], lse.cpu().numpy()[b, h], ro[b, h], rl[b, h], bound)
