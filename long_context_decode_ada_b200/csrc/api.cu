@@ -650,6 +650,42 @@ int skv_decode_attention(skv_ctx* ctx, const void* q, int q_dtype, int B, int Hq
                        "skv_decode_attention");
 }
 
+// The stream operations of one host step: q copy, decode (+ merge), the
+// result copies (one when packed), the error word's copy and its reset.
+static int host_step_ops(skv_ctx* ctx, const void* q_host, int q_dtype, int B, int Hq, int Hkv,
+                         const int32_t* page_indptr, const int32_t* page_tier_indptr,
+                         const uint32_t* page_ids, const skv_pools* pools, void* q_dev,
+                         float* out_dev, float* lse_dev, float* out_host, float* lse_host,
+                         bool packed, int32_t* err_word, void* workspace, size_t ws_bytes,
+                         int num_splits, void* stream, const char* name) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t qn = (size_t)B * Hq * 128 * 2, on = (size_t)B * Hq * 128 * 4, ln = (size_t)B * Hq * 4;
+  // a copy, not reads of mapped host memory by the decode: those made the
+  // step 8.5 us slower (99 against 90.5 us on the 128K store)
+  cudaError_t e = cudaMemcpyAsync(q_dev, q_host, qn, cudaMemcpyHostToDevice, s);
+  if (e != cudaSuccess) return cuda_fail(e, "skv_decode_attention_host: copy of q");
+  const void* pool[3] = {pools->base[0], pools->base[1], pools->base[2]};
+  const long long slots[3] = {pools->slots[0], pools->slots[1], pools->slots[2]};
+  int rc = decode_common(ctx, q_dev, q_dtype, B, Hq, Hkv, page_indptr, page_tier_indptr, page_ids,
+                         pool, slots, false, out_dev, lse_dev, err_word, workspace, ws_bytes,
+                         num_splits, stream, name);
+  if (rc != SKV_OK) return rc;
+  // copies, not kernel stores into mapped host memory: writing the results
+  // through the mapping made the step slower (103 against 98 us on the 128K store)
+  if (packed) {
+    e = cudaMemcpyAsync(out_host, out_dev, on + ln, cudaMemcpyDeviceToHost, s);
+  } else {
+    e = cudaMemcpyAsync(out_host, out_dev, on, cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(lse_host, lse_dev, ln, cudaMemcpyDeviceToHost, s);
+  }
+  // the error word rides along with the results, and is reset on the stream
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(ctx->err_host, err_word, sizeof(int32_t), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(err_word, 0, sizeof(int32_t), s);
+  if (e != cudaSuccess) return cuda_fail(e, "skv_decode_attention_host: copy of the results");
+  return SKV_OK;
+}
+
 int skv_decode_attention_host(skv_ctx* ctx, const void* q_host, int q_dtype, int B, int Hq,
                               int Hkv, const int32_t* page_indptr,
                               const int32_t* page_tier_indptr, const uint32_t* page_ids,
@@ -676,35 +712,17 @@ int skv_decode_attention_host(skv_ctx* ctx, const void* q_host, int q_dtype, int
       *ctx->err_host = 0;
     }
   }
-  const size_t qn = (size_t)B * Hq * 128 * 2, on = (size_t)B * Hq * 128 * 4, ln = (size_t)B * Hq * 4;
-  // a copy, not reads of mapped host memory by the decode: those made the
-  // step 8.5 us slower (99 against 90.5 us on the 128K store)
-  e = cudaMemcpyAsync(q_dev, q_host, qn, cudaMemcpyHostToDevice, s);
-  if (e != cudaSuccess) return cuda_fail(e, "skv_decode_attention_host: copy of q");
-  const size_t on_f = on / sizeof(float);
+  const size_t on_f = (size_t)B * Hq * 128;
   if (packed) {
     lse_dev = out_dev + on_f;
     lse_host = out_host + on_f;
   }
-  const void* pool[3] = {pools->base[0], pools->base[1], pools->base[2]};
-  const long long slots[3] = {pools->slots[0], pools->slots[1], pools->slots[2]};
-  int rc = decode_common(ctx, q_dev, q_dtype, B, Hq, Hkv, page_indptr, page_tier_indptr, page_ids,
-                         pool, slots, false, out_dev, lse_dev, err_word, workspace, ws_bytes,
-                         num_splits, stream, name);
+  // one eager step: a CUDA graph of the same operations, captured once and
+  // replayed, measured 5 us slower a step (91.7 against 86.7 us)
+  const int rc = host_step_ops(ctx, q_host, q_dtype, B, Hq, Hkv, page_indptr, page_tier_indptr,
+                               page_ids, pools, q_dev, out_dev, lse_dev, out_host, lse_host,
+                               packed, err_word, workspace, ws_bytes, num_splits, stream, name);
   if (rc != SKV_OK) return rc;
-  // copies, not kernel stores into mapped host memory: writing the results
-  // through the mapping made the step slower (103 against 98 us on the 128K store)
-  if (packed) {
-    e = cudaMemcpyAsync(out_host, out_dev, on + ln, cudaMemcpyDeviceToHost, s);
-  } else {
-    e = cudaMemcpyAsync(out_host, out_dev, on, cudaMemcpyDeviceToHost, s);
-    if (e == cudaSuccess) e = cudaMemcpyAsync(lse_host, lse_dev, ln, cudaMemcpyDeviceToHost, s);
-  }
-  // the error word rides along with the results, and is reset on the stream
-  if (e == cudaSuccess)
-    e = cudaMemcpyAsync(ctx->err_host, err_word, sizeof(int32_t), cudaMemcpyDeviceToHost, s);
-  if (e == cudaSuccess) e = cudaMemsetAsync(err_word, 0, sizeof(int32_t), s);
-  if (e != cudaSuccess) return cuda_fail(e, "skv_decode_attention_host: copy of the results");
   e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) return cuda_fail(e, "skv_decode_attention_host: stream synchronize");
   const int32_t v = *ctx->err_host;

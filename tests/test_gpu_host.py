@@ -79,3 +79,42 @@ def test_host_step_rejects_device_tensors_as_host_buffers():
     q_host, out_host, lse_host, scratch = host_buffers(w, dev)
     with pytest.raises(skv.SkvError):
         cache.decode_host(dev["q"], dev["q_dtype"], w.Hq, out_host, lse_host, scratch)
+
+
+def test_repeated_host_steps_on_a_side_stream_use_the_current_buffers():
+    """Repeated calls with the same buffers on a stream of their own: every
+    call decodes the q that is in the host buffer at that moment, and a
+    device error comes back as the call's status (then the next call is
+    clean again)."""
+    lens = [700, 333]
+    w = wl.custom(98, 2, 2, 4, 16, lens, wl.MODE_QUOTA,
+                  quota=[[100, 300, 150], [30, 100, 60]])
+    g = run_gpu(w)
+    cache, dev = g["cache"], g["dev"]
+    q_host, res_host, _, scratch = host_buffers(w, dev, True, adjacent=True)
+    n = w.B * w.Hq
+    qs = [dev["q"].cpu().clone(), (dev["q"].view(torch.bfloat16) * -0.5).view(torch.int16).cpu()]
+    refs = []
+    for q in qs:
+        wq = wl.custom(98, 2, 2, 4, 16, lens, wl.MODE_QUOTA,
+                       quota=[[100, 300, 150], [30, 100, 60]])
+        wq.q = q
+        refs.append(oracle.run_workload(wq))
+    side = torch.cuda.Stream()
+    for i in range(7):
+        q_host.copy_(qs[i % 2])
+        cache.decode_host(q_host, dev["q_dtype"], w.Hq, res_host, None, scratch, stream=side)
+        out = res_host[:n * 128].view(w.B, w.Hq, 128).numpy()
+        lse = res_host[n * 128:].view(w.B, w.Hq).numpy()
+        assert_close(out, refs[i % 2]["out"], f"out, call {i}")
+        assert_close(lse, refs[i % 2]["lse"], f"lse, call {i}")
+    good = int(cache.page_ids[2])
+    cache.page_ids[2] = (1 << 30) | (cache.pool_slots[1] + 5)   # slot out of range
+    torch.cuda.synchronize()
+    with pytest.raises(skv.SkvError) as e:
+        cache.decode_host(q_host, dev["q_dtype"], w.Hq, res_host, None, scratch, stream=side)
+    assert e.value.code == skv.SKV_ERR_CORRUPT
+    cache.page_ids[2] = good
+    torch.cuda.synchronize()
+    cache.decode_host(q_host, dev["q_dtype"], w.Hq, res_host, None, scratch, stream=side)
+    cache.check()
