@@ -375,6 +375,34 @@ int skv_decode_attention_host(skv_ctx* ctx, const void* q_host, int q_dtype, int
                               float* out_host, float* lse_host, int32_t* err_word,
                               void* workspace, size_t ws_bytes, int num_splits, void* stream);
 
+/* skv_decode_attention_host_pipelined -- the host step of
+   skv_decode_attention_host, pipelined across calls so that one step's
+   copies and the host's wait overlap the next step's decode.  Call k issues
+   step k: q_host -> slot k%2 of q_dev on a copy stream of the context, the
+   decode on `stream` once that copy is done, then out and lse packed into
+   res_host (B*Hq*128 floats of out, then B*Hq of lse) and the step's error
+   word on a second copy stream of the context once the decode is done.  It
+   returns once step k-1 is done: step k-1's results are then in the
+   res_host given to call k-1, and the return value is step k-1's status
+   (SKV_OK for the first call).  The caller therefore alternates two sets of
+   host buffers (q_host, res_host): the set of call k must not be touched
+   until call k+1 has returned.  skv_decode_attention_host_drain waits for
+   the last step issued and returns its status; call it before the buffers
+   are used otherwise, before the stream changes and before skv_destroy.
+     q_dev      device scratch of 2 x B*Hq*128 16-bit values (two slots)
+     res_dev    device scratch of 2 x B*Hq*129 floats (two slots)
+     other arguments as for skv_decode_attention_host (the error words are
+     the context's own)
+   Calls on one context must not overlap. */
+int skv_decode_attention_host_pipelined(skv_ctx* ctx, const void* q_host, int q_dtype, int B,
+                                        int Hq, int Hkv, const int32_t* page_indptr,
+                                        const int32_t* page_tier_indptr,
+                                        const uint32_t* page_ids, const skv_pools* pools,
+                                        void* q_dev, float* res_dev, float* res_host,
+                                        void* workspace, size_t ws_bytes, int num_splits,
+                                        void* stream);
+int skv_decode_attention_host_drain(skv_ctx* ctx);
+
 /* skv_merge_partials -- the exchange step of a context-parallel decode.
    Each of R ranks attends (skv_decode_attention) over its own slice of every
    sequence's tokens; softmax over the union of disjoint slices factors into

@@ -36,6 +36,18 @@ struct skv_ctx {
   cudaEvent_t profile_event;
   int32_t* err_host = nullptr;  // pinned word for skv_decode_attention_host (lazily allocated)
   int outlier_protect = 0;      // skv_config.outlier_protect
+  // skv_decode_attention_host_pipelined: per slot (two steps in flight) a
+  // device and a pinned error word and the events of the q copy, the decode
+  // and the result copies; the copy streams; the steps issued
+  int32_t* pipe_err = nullptr;       // pinned [2]
+  int32_t* pipe_err_dev = nullptr;   // device [2]
+  cudaEvent_t pipe_ev_q[2] = {nullptr, nullptr};
+  cudaEvent_t pipe_ev_d[2] = {nullptr, nullptr};
+  cudaEvent_t pipe_ev_r[2] = {nullptr, nullptr};
+  cudaStream_t pipe_in = nullptr, pipe_out = nullptr;
+  long long pipe_n = 0;
+  bool pipe_pending = false;
+  void* pipe_stream = nullptr;
 };
 
 namespace {
@@ -201,6 +213,15 @@ int skv_create(const skv_config* cfg, skv_ctx** out) {
 
 int skv_destroy(skv_ctx* ctx) {
   if (ctx && ctx->err_host) cudaFreeHost(ctx->err_host);
+  if (ctx && ctx->pipe_err) cudaFreeHost(ctx->pipe_err);
+  if (ctx && ctx->pipe_err_dev) cudaFree(ctx->pipe_err_dev);
+  for (int i = 0; ctx && i < 2; ++i) {
+    if (ctx->pipe_ev_q[i]) cudaEventDestroy(ctx->pipe_ev_q[i]);
+    if (ctx->pipe_ev_d[i]) cudaEventDestroy(ctx->pipe_ev_d[i]);
+    if (ctx->pipe_ev_r[i]) cudaEventDestroy(ctx->pipe_ev_r[i]);
+  }
+  if (ctx && ctx->pipe_in) cudaStreamDestroy(ctx->pipe_in);
+  if (ctx && ctx->pipe_out) cudaStreamDestroy(ctx->pipe_out);
   delete ctx;
   return ok();
 }
@@ -656,8 +677,8 @@ static int host_step_ops(skv_ctx* ctx, const void* q_host, int q_dtype, int B, i
                          const int32_t* page_indptr, const int32_t* page_tier_indptr,
                          const uint32_t* page_ids, const skv_pools* pools, void* q_dev,
                          float* out_dev, float* lse_dev, float* out_host, float* lse_host,
-                         bool packed, int32_t* err_word, void* workspace, size_t ws_bytes,
-                         int num_splits, void* stream, const char* name) {
+                         bool packed, int32_t* err_word, int32_t* err_dst, void* workspace,
+                         size_t ws_bytes, int num_splits, void* stream, const char* name) {
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const size_t qn = (size_t)B * Hq * 128 * 2, on = (size_t)B * Hq * 128 * 4, ln = (size_t)B * Hq * 4;
   // a copy, not reads of mapped host memory by the decode: those made the
@@ -680,7 +701,7 @@ static int host_step_ops(skv_ctx* ctx, const void* q_host, int q_dtype, int B, i
   }
   // the error word rides along with the results, and is reset on the stream
   if (e == cudaSuccess)
-    e = cudaMemcpyAsync(ctx->err_host, err_word, sizeof(int32_t), cudaMemcpyDeviceToHost, s);
+    e = cudaMemcpyAsync(err_dst, err_word, sizeof(int32_t), cudaMemcpyDeviceToHost, s);
   if (e == cudaSuccess) e = cudaMemsetAsync(err_word, 0, sizeof(int32_t), s);
   if (e != cudaSuccess) return cuda_fail(e, "skv_decode_attention_host: copy of the results");
   return SKV_OK;
@@ -721,12 +742,98 @@ int skv_decode_attention_host(skv_ctx* ctx, const void* q_host, int q_dtype, int
   // replayed, measured 5 us slower a step (91.7 against 86.7 us)
   const int rc = host_step_ops(ctx, q_host, q_dtype, B, Hq, Hkv, page_indptr, page_tier_indptr,
                                page_ids, pools, q_dev, out_dev, lse_dev, out_host, lse_host,
-                               packed, err_word, workspace, ws_bytes, num_splits, stream, name);
+                               packed, err_word, ctx->err_host, workspace, ws_bytes, num_splits,
+                               stream, name);
   if (rc != SKV_OK) return rc;
   e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) return cuda_fail(e, "skv_decode_attention_host: stream synchronize");
   const int32_t v = *ctx->err_host;
   if (v != 0) return fail(v, "%s: device reported error %d", name, v);
+  return ok();
+}
+
+int skv_decode_attention_host_pipelined(skv_ctx* ctx, const void* q_host, int q_dtype, int B,
+                                        int Hq, int Hkv, const int32_t* page_indptr,
+                                        const int32_t* page_tier_indptr,
+                                        const uint32_t* page_ids, const skv_pools* pools,
+                                        void* q_dev, float* res_dev, float* res_host,
+                                        void* workspace, size_t ws_bytes, int num_splits,
+                                        void* stream) {
+  static const char* name = "skv_decode_attention_host_pipelined";
+  if (!ctx) return fail(SKV_ERR_ARG, "%s: null ctx", name);
+  if (B <= 0 || Hkv <= 0 || Hq <= 0 || Hq % Hkv != 0)
+    return fail(SKV_ERR_ARG, "%s: need B > 0 and Hq a multiple of Hkv", name);
+  if (!q_host || !q_dev || !res_dev || !res_host)
+    return fail(SKV_ERR_ARG, "%s: null argument", name);
+  if (!valid_pools(pools, 3)) return fail(SKV_ERR_ARG, "%s: bad pools", name);
+  if (ctx->pipe_pending && ctx->pipe_stream != stream)
+    return fail(SKV_ERR_ARG, "%s: a step is pending on another stream (drain it first)", name);
+  cudaError_t e = cudaSuccess;
+  if (!ctx->pipe_err) {  // first use: the slots' words, events and copy streams
+    if ((e = cudaMallocHost(&ctx->pipe_err, 2 * sizeof(int32_t))) != cudaSuccess ||
+        (e = cudaMalloc(&ctx->pipe_err_dev, 2 * sizeof(int32_t))) != cudaSuccess ||
+        (e = cudaMemset(ctx->pipe_err_dev, 0, 2 * sizeof(int32_t))) != cudaSuccess ||
+        (e = cudaStreamCreateWithFlags(&ctx->pipe_in, cudaStreamNonBlocking)) != cudaSuccess ||
+        (e = cudaStreamCreateWithFlags(&ctx->pipe_out, cudaStreamNonBlocking)) != cudaSuccess)
+      return cuda_fail(e, "skv_decode_attention_host_pipelined: set-up");
+    ctx->pipe_err[0] = ctx->pipe_err[1] = 0;
+    for (int i = 0; i < 2; ++i)
+      if ((e = cudaEventCreateWithFlags(&ctx->pipe_ev_q[i], cudaEventDisableTiming)) !=
+              cudaSuccess ||
+          (e = cudaEventCreateWithFlags(&ctx->pipe_ev_d[i], cudaEventDisableTiming)) !=
+              cudaSuccess ||
+          (e = cudaEventCreateWithFlags(&ctx->pipe_ev_r[i], cudaEventDisableTiming)) != cudaSuccess)
+        return cuda_fail(e, "skv_decode_attention_host_pipelined: events");
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int slot = (int)(ctx->pipe_n & 1);
+  const size_t qn = (size_t)B * Hq * 128 * 2, rn = (size_t)B * Hq * 129;
+  uint8_t* qd = static_cast<uint8_t*>(q_dev) + slot * qn;
+  float* rd = res_dev + slot * rn;
+  int32_t* ed = ctx->pipe_err_dev + slot;
+  // q in on the copy-in stream (it may run while the previous decode does)
+  if ((e = cudaMemcpyAsync(qd, q_host, qn, cudaMemcpyHostToDevice, ctx->pipe_in)) != cudaSuccess ||
+      (e = cudaEventRecord(ctx->pipe_ev_q[slot], ctx->pipe_in)) != cudaSuccess ||
+      (e = cudaStreamWaitEvent(s, ctx->pipe_ev_q[slot], 0)) != cudaSuccess)
+    return cuda_fail(e, "skv_decode_attention_host_pipelined: q copy");
+  const void* pool[3] = {pools->base[0], pools->base[1], pools->base[2]};
+  const long long slots[3] = {pools->slots[0], pools->slots[1], pools->slots[2]};
+  int rc = decode_common(ctx, qd, q_dtype, B, Hq, Hkv, page_indptr, page_tier_indptr, page_ids,
+                         pool, slots, false, rd, rd + (size_t)B * Hq * 128, ed, workspace,
+                         ws_bytes, num_splits, stream, name);
+  if (rc != SKV_OK) return rc;
+  // out + lse and the error word out on the copy-out stream, behind the decode
+  if ((e = cudaEventRecord(ctx->pipe_ev_d[slot], s)) != cudaSuccess ||
+      (e = cudaStreamWaitEvent(ctx->pipe_out, ctx->pipe_ev_d[slot], 0)) != cudaSuccess ||
+      (e = cudaMemcpyAsync(res_host, rd, rn * sizeof(float), cudaMemcpyDeviceToHost,
+                           ctx->pipe_out)) != cudaSuccess ||
+      (e = cudaMemcpyAsync(&ctx->pipe_err[slot], ed, sizeof(int32_t), cudaMemcpyDeviceToHost,
+                           ctx->pipe_out)) != cudaSuccess ||
+      (e = cudaMemsetAsync(ed, 0, sizeof(int32_t), ctx->pipe_out)) != cudaSuccess ||
+      (e = cudaEventRecord(ctx->pipe_ev_r[slot], ctx->pipe_out)) != cudaSuccess)
+    return cuda_fail(e, "skv_decode_attention_host_pipelined: result copies");
+  const bool had_prev = ctx->pipe_pending;
+  ctx->pipe_n += 1;
+  ctx->pipe_pending = true;
+  ctx->pipe_stream = stream;
+  if (!had_prev) return ok();
+  // the previous step: its results are in the host buffer of the previous call
+  e = cudaEventSynchronize(ctx->pipe_ev_r[slot ^ 1]);
+  if (e != cudaSuccess) return cuda_fail(e, "skv_decode_attention_host_pipelined: event wait");
+  const int32_t v = ctx->pipe_err[slot ^ 1];
+  if (v != 0) return fail(v, "%s: the previous step reported error %d", name, v);
+  return ok();
+}
+
+int skv_decode_attention_host_drain(skv_ctx* ctx) {
+  if (!ctx) return fail(SKV_ERR_ARG, "skv_decode_attention_host_drain: null ctx");
+  if (!ctx->pipe_pending) return ok();
+  const int slot = (int)((ctx->pipe_n - 1) & 1);
+  ctx->pipe_pending = false;
+  cudaError_t e = cudaEventSynchronize(ctx->pipe_ev_r[slot]);
+  if (e != cudaSuccess) return cuda_fail(e, "skv_decode_attention_host_drain: event wait");
+  const int32_t v = ctx->pipe_err[slot];
+  if (v != 0) return fail(v, "skv_decode_attention_host_drain: the last step reported error %d", v);
   return ok();
 }
 

@@ -34,6 +34,7 @@ EXPORTS = [
     "skv_device_info", "skv_workspace_size", "skv_allocate", "skv_encode", "skv_append",
     "skv_retier", "skv_retier_workspace_size",
     "skv_decode_attention", "skv_decode_attention_static", "skv_decode_attention_host",
+    "skv_decode_attention_host_pipelined", "skv_decode_attention_host_drain",
     "skv_decode_utility", "skv_merge_partials",
     "skv_dense_pack_bf16",
     "skv_dense_decode_bf16",
@@ -76,6 +77,10 @@ _SIGS = {
                         C.POINTER(SkvPools), _p, _p, _p, _p, _p, _i64, _p, _p, _p, _p, _sz, _p]),
     "skv_decode_attention_host": (_i, [_p, _p, _i, _i, _i, _i, _p, _p, _p, C.POINTER(SkvPools),
                                        _p, _p, _p, _p, _p, _p, _p, _sz, _i, _p]),
+    "skv_decode_attention_host_pipelined": (_i, [_p, _p, _i, _i, _i, _i, _p, _p, _p,
+                                                 C.POINTER(SkvPools), _p, _p, _p, _p, _sz, _i,
+                                                 _p]),
+    "skv_decode_attention_host_drain": (_i, [_p]),
     "skv_merge_partials": (_i, [_p, _i, _i64, _p, _p, _i64, _p, _p, _p]),
     "skv_decode_utility": (_i, [_p, _p, _i, _i, _i, _i, _p, _p, _p, _i64, C.POINTER(SkvPools),
                                 _i64, _p, _p, _p, C.c_float, _p, _p, _p, _p, _p, _sz, _i, _p]),
@@ -244,6 +249,11 @@ class Context:
 
     def check(self, err: torch.Tensor, stream=None):
         _check(lib().skv_check(self._h, _ptr(err), _stream(stream)))
+
+    def drain_host_steps(self):
+        """Wait for the last pipelined host step and return its status as an
+        exception (skv_decode_attention_host_drain)."""
+        _check(lib().skv_decode_attention_host_drain(self._h))
 
     def set_wait_limit(self, cycles: int):
         """SM clocks a decode wait may take before the call ends with
@@ -452,6 +462,33 @@ class PagedCache:
             _ptr(lse_dev), _ptr(out_host), _ptr(lse_host), _ptr(self.err), _ptr(workspace),
             workspace.numel(), num_splits, _stream(stream)))
         return out_host, lse_host
+
+    def decode_host_pipelined(self, q_host: torch.Tensor, q_dtype: int, Hq: int,
+                              res_host: torch.Tensor, q_dev: torch.Tensor, res_dev: torch.Tensor,
+                              workspace=None, num_splits: int = 0, stream=None):
+        """Issue one host step (skv_decode_attention_host_pipelined) and wait
+        for the previous one: on return the previous call's res_host holds
+        that step's out (B*Hq*128 floats) then lse (B*Hq), and the previous
+        step's device error, if any, is raised.  Alternate two (q_host,
+        res_host) sets; ctx.drain_host_steps() waits for the last step.
+        q_dev holds 2 x B*Hq*128 16-bit values and res_dev 2 x B*Hq*129
+        floats (two slots)."""
+        n = self.B * Hq * self.ctx.d
+        for t, dev_side in ((q_host, False), (res_host, False), (q_dev, True), (res_dev, True)):
+            if t.is_cuda != dev_side or not t.is_contiguous():
+                raise SkvError(SKV_ERR_ARG, "decode_host_pipelined: host tensors on the host, "
+                                            "scratch on the device, all contiguous")
+        _expect(q_host, "q_host", n, 2, cuda=False)
+        _expect(q_dev, "q_dev", 2 * n, 2, cuda=False)
+        _expect(res_host, "res_host", n + self.B * Hq, 4, torch.float32, cuda=False)
+        _expect(res_dev, "res_dev", 2 * (n + self.B * Hq), 4, torch.float32, cuda=False)
+        if workspace is None:
+            workspace = self.workspace(Hq, num_splits)
+        _check(lib().skv_decode_attention_host_pipelined(
+            self.ctx.handle, _ptr(q_host), q_dtype, self.B, Hq, self.Hkv, _ptr(self.page_indptr),
+            _ptr(self.page_tier_indptr) if self.split_by_bytes else None, _ptr(self.page_ids),
+            C.byref(self._pools_c), _ptr(q_dev), _ptr(res_dev), _ptr(res_host),
+            _ptr(workspace), workspace.numel(), num_splits, _stream(stream)))
 
     def decode_static(self, q: torch.Tensor, q_dtype: int, Hq: int, out=None, lse=None,
                       num_splits: int = 0, stream=None):

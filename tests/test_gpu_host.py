@@ -118,3 +118,68 @@ def test_repeated_host_steps_on_a_side_stream_use_the_current_buffers():
     torch.cuda.synchronize()
     cache.decode_host(q_host, dev["q_dtype"], w.Hq, res_host, None, scratch, stream=side)
     cache.check()
+
+
+def test_pipelined_host_steps_return_each_previous_step():
+    """skv_decode_attention_host_pipelined: call k issues step k and returns
+    step k-1's results in the host buffers of call k-1 (two alternating
+    sets; the copies run on the context's own streams, two device slots);
+    the drain returns the last step.  A device error of one step is the
+    status of the next call; after the drain the next steps are clean."""
+    lens = [700, 333]
+    quota = [[100, 300, 150], [30, 100, 60]]
+    w = wl.custom(99, 2, 2, 4, 16, lens, wl.MODE_QUOTA, quota=quota)
+    g = run_gpu(w)
+    cache, dev, ctx = g["cache"], g["dev"], g["ctx"]
+    n = w.B * w.Hq
+    qs = [dev["q"].cpu().clone(), (dev["q"].view(torch.bfloat16) * -0.5).view(torch.int16).cpu()]
+    refs = []
+    for q in qs:
+        wq = wl.custom(99, 2, 2, 4, 16, lens, wl.MODE_QUOTA, quota=quota)
+        wq.q = q
+        refs.append(oracle.run_workload(wq))
+    sets = [(torch.empty_like(qs[0]).pin_memory(), torch.empty(n * 129).pin_memory())
+            for _ in range(2)]
+    q_dev = torch.empty(2 * n * 128, dtype=dev["q"].dtype, device=dev["q"].device)   # two slots
+    res_dev = torch.empty(2 * n * 129, dtype=torch.float32, device=q_dev.device)
+    side = torch.cuda.Stream()
+
+    def check(k):
+        res = sets[k % 2][1]
+        assert_close(res[:n * 128].view(w.B, w.Hq, 128).numpy(), refs[k % 2]["out"], f"out {k}")
+        assert_close(res[n * 128:].view(w.B, w.Hq).numpy(), refs[k % 2]["lse"], f"lse {k}")
+
+    for k in range(6):
+        qh, rh = sets[k % 2]
+        qh.copy_(qs[k % 2])
+        cache.decode_host_pipelined(qh, dev["q_dtype"], w.Hq, rh, q_dev, res_dev, stream=side)
+        if k > 0:
+            check(k - 1)
+    ctx.drain_host_steps()
+    check(5)
+    # a corrupt page id: the first call's step fails, which the second call
+    # reports; the drain reports the second step (it saw the same id)
+    good = int(cache.page_ids[2])
+    torch.cuda.synchronize()
+    cache.page_ids[2] = (1 << 30) | (cache.pool_slots[1] + 5)   # slot out of range
+    torch.cuda.synchronize()
+    for k in range(2):
+        qh, rh = sets[k % 2]
+        qh.copy_(qs[k % 2])
+        if k == 0:
+            cache.decode_host_pipelined(qh, dev["q_dtype"], w.Hq, rh, q_dev, res_dev, stream=side)
+        else:
+            with pytest.raises(skv.SkvError) as e:
+                cache.decode_host_pipelined(qh, dev["q_dtype"], w.Hq, rh, q_dev, res_dev,
+                                            stream=side)
+            assert e.value.code == skv.SKV_ERR_CORRUPT
+    with pytest.raises(skv.SkvError) as e:
+        ctx.drain_host_steps()
+    assert e.value.code == skv.SKV_ERR_CORRUPT
+    cache.page_ids[2] = good
+    torch.cuda.synchronize()
+    qh, rh = sets[0]
+    qh.copy_(qs[0])
+    cache.decode_host_pipelined(qh, dev["q_dtype"], w.Hq, rh, q_dev, res_dev, stream=side)
+    ctx.drain_host_steps()
+    check(0)
