@@ -588,7 +588,7 @@ def run_skv(args, rank, world, local_rank):
         ca.check()
         append = {"us_per_step": ea.elapsed_time(eb) * 1e3 / (n_app - 1), "steps": n_app - 1,
                   "how": "skv_append of one token per sequence and kv head, eager launches "
-                         "(4 kernels each; pages are added every P steps), CUDA events "
+                         "(3 kernels each; pages are added every P steps), CUDA events "
                          "around the steps"}
         # ---- the window roll that follows: the oldest n_app - 1 rows of the
         # protected recent window re-tiered under the budget grown with the

@@ -466,11 +466,10 @@ __global__ void __launch_bounds__(256) transcode_kernel(const __grid_constant__ 
 // inserted at the end of the unit's T0 segment; the later page ids move up
 // and the T1/T2 rows of that unit move one page down (row_of += P).  The
 // result is the layout a fresh pack of the same tiers gives (page slots
-// aside).  Four kernels: plan (one block: per-unit decisions, a scan of the
-// new pages, the new CSR offsets), move (page ids to their new positions
-// and the new ids) and rowmap (the T1/T2 rows of a unit that gained a page),
-// both idle unless a page is added, and write (the token's row, headers,
-// tier and row_of).
+// aside).  Three kernels: plan (one block: per-unit decisions, a scan of the
+// new pages, the new CSR offsets), move (page ids to their new positions,
+// the new ids and the row map of a unit that gained a page; idle unless a
+// page is added) and write (the token's row, headers, tier and row_of).
 
 __global__ void __launch_bounds__(1024) append_plan_kernel(const __grid_constant__ AppendParams p) {
   __shared__ int scan[1024];
@@ -559,8 +558,11 @@ __global__ void __launch_bounds__(1024) append_plan_kernel(const __grid_constant
   }
 }
 
-// old page g to its new position (its unit found by binary search over the
-// old offsets), and each unit's new id; nothing to do when no page is added
+// When pages are added: old page g to its new position (its unit found by
+// binary search over the old offsets), each unit's new id, and, for a unit
+// that gained a T0 page, its T1/T2 rows one page further down the list (the
+// three are independent).  One small grid-stride launch that leaves at once
+// on the steps that add no page.
 __global__ void __launch_bounds__(256) append_move_kernel(const __grid_constant__ AppendParams p) {
   const int U = p.B * p.Hkv;
   const AppendWs wl = append_ws(U, p.page_cap);
@@ -586,17 +588,8 @@ __global__ void __launch_bounds__(256) append_move_kernel(const __grid_constant_
     if ((long long)slot >= p.slots0) report(p.err, SKV_ERR_POOL);
     p.ids[ws[wl.a1 + u] + nb] = slot & 0x3FFFFFFFu;  // tier 0
   }
-}
-
-// a unit that gained a T0 page: its T1/T2 rows move one page down the list
-__global__ void __launch_bounds__(256) append_rowmap_kernel(const __grid_constant__ AppendParams p) {
-  const int U = p.B * p.Hkv;
-  const AppendWs wl = append_ws(U, p.page_cap);
-  const int32_t* const ws = p.ws;
-  if (ws[wl.flag] || ws[wl.total] == 0) return;
   const long long n = (long long)U * p.Tmax;
-  const long long nthr = (long long)gridDim.x * blockDim.x;
-  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += nthr) {
+  for (long long i = i0; i < n; i += nthr) {
     const long long u = i / p.Tmax, k = i - u * p.Tmax;
     if (!ws[wl.need + u] || k >= ws[wl.t + u]) continue;
     const uint8_t tr = p.tier[i];
@@ -675,11 +668,8 @@ cudaError_t launch_append(const AppendParams& p, cudaStream_t stream) {
   append_plan_kernel<<<1, 1024, 0, stream>>>(p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  // grid-stride kernels that leave at once when no page is added
-  append_move_kernel<<<1184, 256, 0, stream>>>(p);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  append_rowmap_kernel<<<1184, 256, 0, stream>>>(p);
+  // two blocks per SM, leaving at once when no page is added
+  append_move_kernel<<<296, 256, 0, stream>>>(p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   append_write_kernel<<<(unsigned)((U + 7) / 8), 256, 0, stream>>>(p);
