@@ -557,12 +557,14 @@ def run_skv(args, rank, world, local_rank):
         del uts, uws, gu, gu_tail, gu_prof
 
     # ---- decode-time append (skv_append) on the same recipe: a store built
-    # n_app tokens short, then n_app appends timed one after another
+    # n_app tokens short; the first n_eager appends timed one after another,
+    # then the serving step (append + decode, one CUDA graph) for the rest
     append = None
     retier = None
+    serving = None
     if not args.no_append:
         import dataclasses
-        n_app = 64
+        n_app, n_eager = 128, 64
         wa = dataclasses.replace(w, seq_lens=(w.seq_lens - n_app).astype(np.int32))
         slots = list(w.pool_slots)
         slots[0] += w.B * w.Hkv * (n_app // w.P + 2)
@@ -581,15 +583,44 @@ def run_skv(args, rank, world, local_rank):
         torch.cuda.synchronize()
         ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         ea.record()
-        for i in range(1, n_app):
+        for i in range(1, n_eager):
             ca.append(*kv[i], seq_a)
         eb.record()
         torch.cuda.synchronize()
         ca.check()
-        append = {"us_per_step": ea.elapsed_time(eb) * 1e3 / (n_app - 1), "steps": n_app - 1,
+        append = {"us_per_step": ea.elapsed_time(eb) * 1e3 / (n_eager - 1), "steps": n_eager - 1,
                   "how": "skv_append of one token per sequence and kv head, eager launches "
                          "(3 kernels each; pages are added every P steps), CUDA events "
                          "around the steps"}
+        # ---- the serving step: skv_append of the new token (its K / V in the
+        # step's input buffers, where the model would write them) and the
+        # decode over the store it grew, 8 steps to a CUDA graph
+        per_graph = 8
+        kvb = [(kv[n_eager + j][0].clone(), kv[n_eager + j][1].clone()) for j in range(per_graph)]
+        wsa = [ca.workspace(w.Hq, S) for _ in range(2)]
+        out_s = torch.empty_like(out)
+        lse_s = torch.empty_like(lse)
+        gs = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gs):
+            for j in range(per_graph):
+                ca.append(*kvb[j], seq_a)
+                ca.decode(d["q"], d["q_dtype"], w.Hq, out=out_s, lse=lse_s, workspace=wsa[j % 2],
+                          num_splits=S)
+        torch.cuda.synchronize()
+        n_srv = (n_app - n_eager) // per_graph * per_graph
+        ea.record()
+        for i in range(n_srv // per_graph):
+            gs.replay()
+        eb.record()
+        torch.cuda.synchronize()
+        ca.check()
+        assert int(seq_a[0]) == T - (n_app - n_eager - n_srv), "the serving steps appended"
+        serving = {"us_per_step": ea.elapsed_time(eb) * 1e3 / n_srv, "steps": n_srv,
+                   "how": "per token: skv_append (its K and V in the step's input buffers) and "
+                          "the decode over the store it grew, 8 steps to a CUDA graph (the "
+                          "buffers hold the same 8 tokens at each replay); 128K store, its last "
+                          "64 tokens; CUDA events around the replays"}
+        del gs
         # ---- the window roll that follows: the oldest n_app - 1 rows of the
         # protected recent window re-tiered under the budget grown with the
         # appended tokens (skv_retier), on the store the appends left
@@ -673,6 +704,7 @@ def run_skv(args, rank, world, local_rank):
             "t0_bf16_variant": t0b,
             "ingest": {"allocate_ms": alloc_ms, "encode_ms": enc_ms, "gen_s": t_gen},
             "append": append,
+            "serving_step": serving,
             "retier": retier,
             "utility": utility,
             "configs": configs,
