@@ -1,8 +1,8 @@
-"""The oracle against the hand-worked examples in tests/golden/ (see its
-README: the pages print no worked example, so each fixture is derived by
-hand from the passage it cites).  Each expected number is also recomputed
-here from the closed form the fixture states, so that a typo in a fixture
-fails as well."""
+"""The oracle against the hand-worked examples in tests/golden/.  The pages
+print no worked example, so each fixture is derived by hand from the
+passage it cites.  Each expected number is also recomputed here from the
+closed form the fixture states, so that a typo in a fixture fails as
+well."""
 import json
 import math
 import os
