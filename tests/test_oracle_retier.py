@@ -109,6 +109,36 @@ def test_demoted_assignment_is_optimal_at_every_breakpoint(seed):
     assert nbreak >= 3 * n
 
 
+@pytest.mark.parametrize("P", [16, 64])
+def test_reserve_comes_off_the_budget_before_the_walk(P):
+    """P > 1: the walk gets budget - kept bytes - Hkv (P - 1)(512 + 196 + 180).
+    With the budget raised by exactly that reserve, the demoted tokens get
+    the P = 1 assignment (no reserve) at every budget of a sweep; a budget
+    one byte below the kept bytes plus the reserve is reported, with the
+    demoted rows dropped and the kept rows unchanged."""
+    n, m = 4, 7
+    w = wl.custom(40 + P, 1, 1, 1, 1, [m], wl.MODE_BUDGET, budget=[0])
+    r = np.random.default_rng(P)
+    w.utility = torch.tensor(r.uniform(0.01, 1.0, (1, 1, m)), dtype=torch.float32)
+    tier_in = np.zeros((1, 1, m), np.uint8)
+    tier_in[0, 0, n:] = [1, 2, 3]
+    demote = np.zeros_like(tier_in)
+    demote[0, 0, :n] = 1
+    reserve = (P - 1) * (512 + 196 + 180)
+    kept = 196 + 180
+    for left in range(0, 512 * n + 8, 20):
+        ref = oracle.retier(1, 1, m, w.d, 1, w.seq_lens, w.K, w.utility, tier_in, demote,
+                            [kept + left])
+        got = oracle.retier(1, 1, m, w.d, P, w.seq_lens, w.K, w.utility, tier_in, demote,
+                            [kept + left + reserve])
+        assert np.array_equal(got, ref), left
+    # below the reserve: reported, demoted rows dropped, kept rows unchanged
+    out, rc = oracle.retier(1, 1, m, w.d, P, w.seq_lens, w.K, w.utility, tier_in, demote,
+                            [kept + reserve - 1], check=False)
+    assert rc == oracle.ERR_BUDGET
+    assert np.all(out[0, 0, :n] == 3) and np.array_equal(out[0, 0, n:], tier_in[0, 0, n:])
+
+
 def window_store(seed, T, A, recent, frac, B=2, Hkv=2):
     """A store allocated over the first T - A tokens (recent window of
     `recent` tokens protected, budget frac of dense at T - A) to which A
