@@ -175,3 +175,46 @@ def test_ingest_checks_accept_the_test_workloads():
     with pytest.raises(skv.SkvError):
         skv._check_ingest(1, 1, 4, 128, K=torch.zeros((1, 1, 3, 128), dtype=torch.float16),
                           cuda=False)
+
+
+def test_retier_and_pipelined_host_step_argument_errors_without_gpu():
+    ctx = skv.Context(16)
+    pools = skv.SkvPools()
+    free = skv.SkvFreeLists()
+    L = skv.lib()
+    # the re-tiering's workspace: the allocation's plus the old store's copies
+    # (tiers, row map, both CSR tables, page ids) and the per-segment words
+    n = C.c_size_t()
+    assert L.skv_retier_workspace_size(ctx.handle, 2, 4, 1000, 500, C.byref(n)) == skv.SKV_OK
+    assert n.value >= ctx.workspace_size(skv.WS_ALLOCATE, 2, 4, 0, 1000) + 8 * 1000 * 5 + 500 * 4
+    assert L.skv_retier_workspace_size(ctx.handle, 2, 0, 1000, 500, C.byref(n)) == skv.SKV_ERR_ARG
+    # null arguments are refused before any launch
+    rc = L.skv_retier(ctx.handle, 1, 1, 16, None, None, None, None, C.byref(free), None,
+                      C.byref(pools), None, None, None, None, None, 0, None, None, None, None, 0,
+                      None)
+    assert rc == skv.SKV_ERR_ARG
+    # too many positions for the 32-bit row list
+    rc = L.skv_retier(ctx.handle, 1024, 128, 1 << 23, None, None, None, None, C.byref(free), None,
+                      C.byref(pools), None, None, None, None, None, 0, None, None, None, None, 0,
+                      None)
+    assert rc == skv.SKV_ERR_ARG
+    # the pipelined host step: B = 0 and null buffers are refused; a drain
+    # with nothing in flight is a no-op
+    rc = L.skv_decode_attention_host_pipelined(ctx.handle, None, 0, 0, 8, 4, None, None, None,
+                                               C.byref(pools), None, None, None, None, 0, 0, None)
+    assert rc == skv.SKV_ERR_ARG
+    rc = L.skv_decode_attention_host_pipelined(ctx.handle, None, 0, 1, 8, 4, None, None, None,
+                                               C.byref(pools), None, None, None, None, 0, 0, None)
+    assert rc == skv.SKV_ERR_ARG
+    assert L.skv_decode_attention_host_drain(ctx.handle) == skv.SKV_OK
+    assert L.skv_decode_attention_host_drain(None) == skv.SKV_ERR_ARG
+
+
+def test_t0_bf16_refuses_the_code_variants_without_gpu():
+    with pytest.raises(skv.SkvError) as e:
+        skv.Context(16, t0_bf16=True, t1_angle_bits=5)
+    assert e.value.code == skv.SKV_ERR_ARG
+    with pytest.raises(skv.SkvError) as e:
+        skv.Context(16, t0_bf16=True, share_grid=1)
+    assert e.value.code == skv.SKV_ERR_ARG
+    assert skv.Context(16, t0_bf16=True).t0_bf16
